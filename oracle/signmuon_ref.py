@@ -1,0 +1,300 @@
+"""CPU oracle for the Sign-Muon optimizer step.  TEST INFRASTRUCTURE ONLY.
+
+Only the tests, the package's smoke check and the benchmark's CPU-baseline leg
+may import this module.  It is plain numpy in float64 (the update is rounded
+once to float32 at the end), slow, and shares no code with the CUDA path.
+
+Sources, by page title:
+
+* [paper]  "SignMuon: 通信高效的分布式Muon优化" -- a rendering of the arXiv paper
+  (Mishra, Trivedi & Kumar, arXiv 2605.16311).
+* [blog]   "SignMuon: Matrix Directions, Majority Votes, and the Actual Bytes
+  Sent" (the authors' methodology post).
+* [radio]  "SignMuon: Communication-Efficient Distributed Muon Optimization"
+  (AI Radio episode, a paraphrase of the paper).
+
+What one step computes, for M workers that share the weights W:
+
+1. coupled weight decay and momentum per worker       [paper] Algorithm 1, Algorithm 2
+2. a polar direction U_m = PolarNS(Mom_m) per matrix  [paper] §3 (Muon update rule), §4
+3. entrywise signs of U_m, one bit each               [paper] §3, Algorithm 2; [blog] bytes
+4. majority vote sign(sum of signs), ties to 0        [blog] "A tiny aggregation calculation"
+5. optional post-vote local polar step                [paper] §4 (where to orthogonalise)
+6. W <- W - eta * D                                    [paper] Algorithm 1, Algorithm 2
+
+Readings taken where the pages are silent or disagree (each is listed with its
+reason in the design notes):
+
+R1  Non-square NS: iterate on the orientation X (m x n, m <= n) whose Gram
+    X X^T is the small one; transpose back at the end.
+R2  Power iteration: start u0 = ones(m)/sqrt(m) on the small side (m = min dim
+    of the wide orientation), each iteration u <- X(X^T u)/||X(X^T u)||, and
+    sigma = ||X^T u|| after P iterations.  A zero iterate stays zero.
+R3  Scale: X0 = Mom / (s + eps).
+R4  Quintic NS: X <- X (15/8 I - 10/8 X^T X + 3/8 (X^T X)^2), the second-order
+    expansion of (X^T X)^(-1/2); cubic is X <- X (3/2 I - 1/2 X^T X).
+R5  One-bit sign: bit = (U >= 0), so 0 and -0 send +1.  The ternary sign keeps
+    sign(0) = 0 as in [paper] §3.
+R6  Packing: one flat bit stream over all matrices (shapes order, row-major),
+    bit j of byte b is element 8b+j; ceil(d/8) bytes; pad bits 0.
+R7  Ties map to 0 ([blog]); the +1 policy of [paper] Algorithm 2 is not used.
+R8  Post-vote polar: D = PolarNS(majority as floats) with the same K, eps,
+    scale and P; no second sign, no rescale.
+R9  Update: W_new = float32 nearest to (W - eta*D), one rounding.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+# Newton-Schulz polynomials: X <- X * p(X^T X)
+CUBIC = (1.5, -0.5)                 # [paper] §4: X(3/2 I - 1/2 X^T X)
+QUINTIC = (15.0 / 8.0, -10.0 / 8.0, 3.0 / 8.0)  # reading R4
+
+
+# ---------------------------------------------------------------------------
+# 1. weight decay + momentum
+# ---------------------------------------------------------------------------
+
+def momentum_update(mom, g, w, beta, lam):
+    """Coupled weight decay then an exponential moving average.
+
+    [paper] Algorithm 1 and Algorithm 2: the decayed gradient is
+    G~ = G + lambda*W, and the new momentum is beta*Mom + (1-beta)*G~
+    (momentum starts at zero).
+    """
+    g_tilde = np.asarray(g, np.float64) + float(lam) * np.asarray(w, np.float64)
+    return float(beta) * np.asarray(mom, np.float64) + (1.0 - float(beta)) * g_tilde
+
+
+# ---------------------------------------------------------------------------
+# 2. PolarNS
+# ---------------------------------------------------------------------------
+
+def frobenius_norm(x):
+    """||X||_F = sqrt(sum of squared entries) ([paper] §3 notation)."""
+    x = np.asarray(x, np.float64)
+    return math.sqrt(float(np.sum(x * x)))
+
+
+def power_sigma(x, P):
+    """Estimate of the largest singular value of a wide X (m <= n) by P power
+    iterations on X X^T (reading R2; [paper] Algorithm 1 input P, §4)."""
+    x = np.asarray(x, np.float64)
+    m = x.shape[0]
+    u = np.full(m, 1.0 / math.sqrt(m))
+    for _ in range(int(P)):
+        y = x @ (x.T @ u)
+        nrm = math.sqrt(float(y @ y))
+        u = y / nrm if nrm > 0.0 else np.zeros(m)
+    z = x.T @ u
+    return math.sqrt(float(z @ z))
+
+
+def ns_iterate(x0, K, order="cubic", coeffs=None):
+    """K Newton-Schulz steps on a wide X (m <= n).
+
+    With A = X X^T, the step X(aI + b X^T X) equals aX + b A X ([paper] §3,
+    two-coefficient form; §4, cubic a=3/2, b=-1/2).  The quintic step (reading
+    R4) is aX + (bA + cA^2) X.
+    """
+    x = np.asarray(x0, np.float64)
+    if order == "cubic":
+        a, b = coeffs if coeffs is not None else CUBIC
+        for _ in range(int(K)):
+            gram = x @ x.T
+            x = a * x + b * (gram @ x)
+    elif order == "quintic":
+        a, b, c = coeffs if coeffs is not None else QUINTIC
+        for _ in range(int(K)):
+            gram = x @ x.T
+            x = a * x + (b * gram + c * (gram @ gram)) @ x
+    else:
+        raise ValueError(order)
+    return x
+
+
+def polar_ns(mat, K, eps, scale, P=1, order="cubic", coeffs=None, return_scale=False):
+    """PolarNS(Mat; K, eps, scale, P) of one matrix ([paper] Algorithm 1, §4).
+
+    Works on the wide orientation (R1), divides by s + eps where s is the
+    Frobenius norm or the power-iteration estimate of the spectral norm
+    (R2, R3), runs K Newton-Schulz steps and returns the result in the
+    matrix's own orientation.
+    """
+    mat = np.asarray(mat, np.float64)
+    tall = mat.shape[0] > mat.shape[1]
+    x = mat.T if tall else mat
+    if scale == "fro":
+        s = frobenius_norm(x)
+    elif scale == "spectral":
+        s = power_sigma(x, P)
+    else:
+        raise ValueError(scale)
+    x = x / (s + float(eps))
+    x = ns_iterate(x, K, order, coeffs)
+    out = x.T if tall else x
+    return (out, s) if return_scale else out
+
+
+# ---------------------------------------------------------------------------
+# 3. signs and 1-bit packing
+# ---------------------------------------------------------------------------
+
+def sign_ternary(u):
+    """Entrywise sign with sign(0) = 0 ([paper] §3 notation; [blog] example)."""
+    u = np.asarray(u)
+    return (u > 0).astype(np.int32) - (u < 0).astype(np.int32)
+
+
+def sign_bits(u):
+    """One-bit sign: True means +1.  0 and -0 send +1 (reading R5)."""
+    return np.asarray(u) >= 0
+
+
+def packed_nbytes(d):
+    """Payload of d one-bit signs: ceil(d/8) bytes ([blog] "d/8 bytes")."""
+    return (int(d) + 7) // 8
+
+
+def pack_bits(bits):
+    """Flat bool vector -> uint8 bytes, bit j of byte b is element 8b+j (R6)."""
+    bits = np.asarray(bits, bool).ravel()
+    d = bits.size
+    padded = np.zeros(packed_nbytes(d) * 8, np.uint8)
+    padded[:d] = bits
+    out = np.zeros(packed_nbytes(d), np.uint8)
+    for j in range(8):
+        out |= (padded[j::8] << j).astype(np.uint8)
+    return out
+
+
+def unpack_bits(packed, d):
+    """Inverse of pack_bits: first d bits as a bool vector."""
+    packed = np.asarray(packed, np.uint8)
+    out = np.zeros(packed.size * 8, bool)
+    for j in range(8):
+        out[j::8] = (packed >> j) & 1
+    return out[: int(d)]
+
+
+# ---------------------------------------------------------------------------
+# 4. majority vote
+# ---------------------------------------------------------------------------
+
+class AccumulatorOverflow(ValueError):
+    """An int8 accumulator cannot hold sums in [-M, M] for M > 127."""
+
+
+def vote_sums_from_bits(packed_list, d, acc="int32"):
+    """sum_i = sum over workers of (+1 if bit else -1) ([paper] Algorithm 2:
+    an integer SUM of the workers' signs; [blog] on the [-P, P] range and
+    int8 overflow)."""
+    M = len(packed_list)
+    if acc == "int8" and M > 127:
+        raise AccumulatorOverflow(f"int8 sums overflow for M={M} > 127")
+    total = np.zeros(int(d), np.int64)
+    for p in packed_list:
+        b = unpack_bits(p, d).astype(np.int64)
+        total += 2 * b - 1
+    return total.astype(np.int8 if acc == "int8" else np.int32)
+
+
+def vote_sums_ternary(sign_list):
+    """Integer sum of ternary sign arrays (the [blog] worked example)."""
+    total = np.zeros(np.shape(sign_list[0]), np.int64)
+    for s in sign_list:
+        total += np.asarray(s, np.int64)
+    return total.astype(np.int32)
+
+
+def majority(sums):
+    """sign(sum) with a tie (sum 0) mapped to 0 (R7, [blog])."""
+    return sign_ternary(sums).astype(np.int8)
+
+
+# ---------------------------------------------------------------------------
+# 6. update
+# ---------------------------------------------------------------------------
+
+def _round_f32(s, err):
+    """float32 nearest to the exact value s + err (s float64, |err| at most half
+    an ulp of s, err the exact residual), ties to even.
+
+    float32(s) is already right unless s sits exactly on a float32 midpoint
+    and err != 0; then the exact value lies to err's side of the midpoint.
+    """
+    r = s.astype(np.float32)
+    toward = np.nextafter(r, np.where(s > r.astype(np.float64), np.float32(np.inf),
+                                      np.float32(-np.inf)).astype(np.float32))
+    mid = (r.astype(np.float64) + toward.astype(np.float64)) * 0.5
+    on_mid = (r.astype(np.float64) != s) & (mid == s) & (err != 0)
+    hi = np.maximum(r, toward)
+    lo = np.minimum(r, toward)
+    return np.where(on_mid, np.where(err > 0, hi, lo), r).astype(np.float32)
+
+
+def update(w, direction, eta):
+    """W_new = W - eta*D, rounded once to float32 ([paper] Algorithm 1, 2;
+    reading R9).  W, D and eta are float32 values; eta*D is exact in float64
+    and the subtraction's rounding error is recovered exactly (two-sum)."""
+    w64 = np.asarray(w, np.float32).astype(np.float64)
+    p = np.float64(np.float32(eta)) * np.asarray(direction, np.float32).astype(np.float64)
+    a, b = w64, -p
+    s = a + b
+    bb = s - a
+    err = (a - (s - bb)) + (b - bb)
+    return _round_f32(s, err)
+
+
+# ---------------------------------------------------------------------------
+# the whole step
+# ---------------------------------------------------------------------------
+
+def split(flat, shapes, offsets=None):
+    """Views of a flat vector as the matrices of ``shapes`` (row-major)."""
+    out, off = [], 0
+    for r, c in shapes:
+        out.append(np.asarray(flat)[off: off + r * c].reshape(r, c))
+        off += r * c
+    return out
+
+
+def step(W, G_list, mom_list, shapes, *, beta, lam, eta, K, eps, scale, P=1,
+         order="cubic", post_polar=False, acc="int32"):
+    """One distributed Sign-Muon step ([paper] Algorithm 2, with the vote of
+    [blog] and the optional post-vote polar step of [paper] §4).
+
+    Returns a dict with the new momentum (float64), the polar factors U_m,
+    the packed bits, the vote sums, the majority, the direction D and the new
+    W (float32).  Inputs are flat vectors; momentum is float64 or float32.
+    """
+    M = len(G_list)
+    d = int(np.asarray(W).size)
+    new_mom, U_list, packed = [], [], []
+    for m in range(M):
+        mom = momentum_update(mom_list[m], G_list[m], W, beta, lam)
+        new_mom.append(mom)
+        u = np.empty(d, np.float64)
+        off = 0
+        for (r, c), mat in zip(shapes, split(mom, shapes)):
+            u[off: off + r * c] = polar_ns(mat, K, eps, scale, P, order).ravel()
+            off += r * c
+        U_list.append(u)
+        packed.append(pack_bits(sign_bits(u)))
+    sums = vote_sums_from_bits(packed, d, acc)
+    maj = majority(sums)
+    if post_polar:
+        D = np.empty(d, np.float64)
+        off = 0
+        for (r, c), mat in zip(shapes, split(maj.astype(np.float64), shapes)):
+            D[off: off + r * c] = polar_ns(mat, K, eps, scale, P, order).ravel()
+            off += r * c
+        D32 = D.astype(np.float32)
+    else:
+        D = maj.astype(np.float64)
+        D32 = maj.astype(np.float32)
+    W_new = update(W, D32, eta)
+    return dict(mom=new_mom, U=U_list, packed=packed, sums=sums, majority=maj,
+                D=D, D32=D32, W=W_new)
