@@ -1,0 +1,372 @@
+"""Benchmark of the Sign-Muon optimizer step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = the whole hot path through the C ABI (signmuon_step): momentum
+pass, power iteration, 5 cubic Newton-Schulz iterations on the tensor cores
+for each of M=8 simulated workers, one-bit pack, majority vote, post-vote
+polar step and the update, on nanoGPT-124M-shaped weights (48 matrices,
+d = 84,934,656).  Inputs are seeded synthetic gradients resident in HBM (two
+alternating 2.7 GB sets, larger than L2).  With N > 1 (torchrun) every rank
+runs an independent replica of the same workload; the path has no data
+exchange between GPUs.
+
+Rank 0 prints one JSON line.  ``--impl reference`` times the CPU oracle on
+the host cores instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "Sign-Muon steps/s (nanoGPT-124M, M=8); NS TFLOP/s and vote GB/s % of peak"
+WL = synth.WORKLOADS["nanogpt"]
+HP = synth.HYPER
+SHAPES = WL["shapes"]
+M = WL["M"]
+K_NS = WL["K"]
+D = synth.numel(SHAPES)
+WORKLOAD_DESC = ("nanoGPT-124M weight shapes: 12 x {2304x768, 768x768, 3072x768, 768x3072} "
+                 f"(d={D:,}); M={M} simulated workers; G_m = S + 2.0 N_m; K={K_NS} cubic Newton-Schulz "
+                 "in bf16 on tcgen05 with fp32 accumulation; spectral scale with P=2 power iterations; "
+                 "post-vote polar step; beta=0.9 lambda=0.01 eta=0.02 eps=1e-7")
+
+# per-(GPU) fallback peaks, used only when MEASURED_PEAKS.json is absent
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return j, "measured"
+    return FALLBACK, "fallback"
+
+
+def ns_flops_per_step(shapes, M, K, post_polar):
+    """Algorithmic Newton-Schulz flops: per matrix and cubic iteration two
+    GEMMs, X X^T (2 m^2 n) and A X (2 m^2 n), m = min dim, n = max dim."""
+    per_worker = sum(4.0 * min(r, c) ** 2 * max(r, c) for r, c in shapes) * K
+    return per_worker * (M + (1 if post_polar else 0))
+
+
+def gram_bytes(shapes):
+    return sum(2.0 * min(r, c) ** 2 for r, c in shapes)
+
+
+def hbm_bytes_per_step(shapes, M, P, post_polar):
+    """Algorithmic HBM bytes of each streaming kernel per step."""
+    d = synth.numel(shapes)
+    b = {
+        "momentum": d * (14.0 * M + 4.0),          # G r, Mom r+w, X w (bf16) per worker; W r once
+        "pack": d * M * (4.0 + 1.0 / 8.0),          # U r (fp32), bits w
+        "power_iter": (P + 1) * M * gram_bytes(shapes),
+        "vote": M * d / 8.0 + (4.0 * d if post_polar else 8.0 * d),  # bits r; D w, or W r+w
+        "stage": 6.0 * d,                           # D r (fp32), X w (bf16)
+        "update": 12.0 * d,                         # W r+w, D r
+    }
+    if post_polar:
+        b["power_iter"] += (P + 1) * gram_bytes(shapes)
+    return b
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+REASON_FIELDS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+
+class ClockSampler:
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             + ",".join("clocks_event_reasons." + r for r in REASON_FIELDS))
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                                          "-lms", "50", "-i", str(self.gpu_id)],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, reasons = [], None, set()
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 5 + len(REASON_FIELDS):
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(REASON_FIELDS, parts[5:]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def gpu_smi_id(dev_index):
+    import torch
+    try:
+        u = torch.cuda.get_device_properties(dev_index).uuid
+        s = str(u)
+        return s if s.startswith("GPU-") else "GPU-" + s
+    except Exception:
+        return str(dev_index)
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (baseline leg and --impl reference)
+# ---------------------------------------------------------------------------
+def cpu_oracle_sample(step_idx=0):
+    """One oracle step on one transformer layer (4 of the 48 matrices, 1/12 of
+    the weights and of the work) for all 8 workers, including the post-vote
+    polar step; returns seconds."""
+    from oracle import signmuon_ref as ref
+    shapes = SHAPES[:4]
+    w = synth.weights0(shapes, 3)
+    G = synth.gradients(shapes, M, WL["sigma"], step=step_idx, config_id=3)
+    mom = synth.momentum0(shapes, M, 3, scale=0.5)
+    t0 = time.perf_counter()
+    ref.step(w, G, mom, shapes, beta=HP["beta"], lam=HP["lam"], eta=HP["eta"], K=K_NS, eps=HP["eps"],
+             scale=WL["scale"], P=WL["P"], post_polar=WL["post_polar"])
+    return time.perf_counter() - t0
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+CPU_SAMPLE = ("one of the 12 transformer layers (2304x768, 768x768, 3072x768, 768x3072; 7,077,888 weights) "
+              "x 8 workers, full oracle step incl. power iteration and post-vote polar, numpy float64; "
+              "steps/s scaled by 1/12 to the whole model")
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    for i in range(args.warmup):
+        cpu_oracle_sample(i)
+    times = [cpu_oracle_sample(args.warmup + i) for i in range(args.steps)]
+    per_step = 12.0 * sum(times) / len(times)
+    value = 1.0 / per_step
+    cores = cpu_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD_DESC, "sample": CPU_SAMPLE},
+        "cpu_baseline": {"value": value, "unit": "steps/s", "cores": cores, "kind": "oracle",
+                         "sample": CPU_SAMPLE},
+        "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+    import sign_muon_optimizer_b200 as smo
+
+    stream = torch.cuda.current_stream()
+    flags = smo.SIGNMUON_POST_POLAR if WL["post_polar"] else 0
+    opt = smo.SignMuon(SHAPES, M, beta=HP["beta"], lam=HP["lam"], K=K_NS, eps=HP["eps"], scale=WL["scale"],
+                       P=WL["P"], flags=flags, stream=stream.cuda_stream)
+    W = synth.device_weights0(SHAPES, config_id=3 + rank)
+    pool = [synth.device_gradients(SHAPES, M, WL["sigma"], step=s, config_id=3 + rank) for s in range(2)]
+    gptrs = [[pool[s][m] for m in range(M)] for s in range(2)]
+    torch.cuda.synchronize()
+
+    for i in range(args.warmup):
+        opt.step(W, gptrs[i % 2], HP["eta"])
+    opt.profile(True)
+    opt.profile_read()
+    launches0 = smo.signmuon_kernel_launches()
+    sampler = ClockSampler(gpu_smi_id(local))
+    sampler.start()
+    time.sleep(0.2)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for i in range(args.steps):
+        opt.step(W, gptrs[i % 2], HP["eta"])
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    launches = smo.signmuon_kernel_launches() - launches0
+    prof = opt.profile_read()
+    opt.profile(False)
+    ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_per_step = ms / args.steps
+    value = world * args.steps / (ms / 1e3)
+
+    pk, pk_kind = peaks()
+    steps = args.steps
+    flops = ns_flops_per_step(SHAPES, M, K_NS, WL["post_polar"])
+    gemm_ms = prof["ns_gemm"][0] + prof["post_ns_gemm"][0]
+    gemm_launches = prof["ns_gemm"][1] + prof["post_ns_gemm"][1]
+    tflops = flops * steps / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else None
+    peak_tc = pk["bf16_tflops_sustained"]
+    roofline = {"kernel": "k_gemm_tc (grouped Newton-Schulz GEMM, tcgen05)", "bound": "tensor",
+                "achieved": tflops, "peak": peak_tc, "unit": "TFLOP/s",
+                "frac": (tflops / peak_tc) if tflops else None, "traffic": None,
+                "peak_kind": f"bf16 sustained, {pk_kind}",
+                "flops_per_launch": flops / max(1, gemm_launches / steps),
+                "avg_launch_ms": gemm_ms / max(1, gemm_launches)}
+    hbm = hbm_bytes_per_step(SHAPES, M, WL["P"], WL["post_polar"])
+    kernels = {}
+    for kind, (kms, n) in prof.items():
+        if n == 0:
+            continue
+        e = {"ms_per_step": kms / steps, "launches_per_step": n / steps}
+        if kind in ("ns_gemm", "post_ns_gemm"):
+            f = ns_flops_per_step(SHAPES, M if kind == "ns_gemm" else 0, K_NS, kind == "post_ns_gemm")
+            e["TFLOP/s"] = f / (kms / steps / 1e3) / 1e12
+            e["frac_of_bf16_peak"] = e["TFLOP/s"] / peak_tc
+        elif kind in hbm:
+            e["GB/s"] = hbm[kind] / (kms / steps / 1e3) / 1e9
+            e["frac_of_hbm"] = e["GB/s"] / pk["hbm_gbs"]
+        kernels[kind] = e
+
+    # end to end through the public API with host buffers (pinned)
+    e2e = None
+    if args.e2e_steps > 0:
+        Wh = torch.empty(D, dtype=torch.float32, pin_memory=True)
+        Wh.copy_(W)
+        Gh = [torch.empty(D, dtype=torch.float32, pin_memory=True) for _ in range(M)]
+        for m in range(M):
+            Gh[m].copy_(pool[0][m])
+        Wn, Gn = Wh.numpy(), [g.numpy() for g in Gh]
+        opt.step_host(Wn, Gn, HP["eta"])
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        ev0.record(stream)
+        for i in range(args.e2e_steps):
+            opt.step_host(Wn, Gn, HP["eta"])
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        wall = time.perf_counter() - t0
+        ems = max(ev0.elapsed_time(ev1), wall * 1e3)
+        if world > 1:
+            t = torch.tensor([ems], device="cuda", dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        e2e = {"value": world * args.e2e_steps / (ems / 1e3), "unit": "steps/s",
+               "h2d_bytes_per_step": (M + 1) * D * 4, "d2h_bytes_per_step": D * 4,
+               "api": "signmuon_step_host (pinned host W and G)"}
+        del Gh, Wh
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        t = cpu_oracle_sample(0)
+        cpu = {"value": 1.0 / (12.0 * t), "unit": "steps/s", "cores": cpu_threads(), "kind": "oracle",
+               "sample": CPU_SAMPLE}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": WORKLOAD_DESC, "M": M, "d": D,
+                       "l2": "inputs larger than L2: 2.72 GB of gradients per step, two alternating sets",
+                       "parallelism": "replicas" if world > 1 else "single GPU"},
+            "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": launches, "clocks": clocks,
+            "ns_tflops_per_step": flops / 1e12,
+        }
+        print(json.dumps(line), flush=True)
+    opt.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,199 @@
+/*
+ * signmuon.h -- C ABI of libsignmuon.so, a B200 (sm_100a) implementation of
+ * one Sign-Muon optimizer step for M workers simulated on one GPU.
+ *
+ * Sources, by page title:
+ *   [paper] "SignMuon: 通信高效的分布式Muon优化" (a rendering of arXiv 2605.16311)
+ *   [blog]  "SignMuon: Matrix Directions, Majority Votes, and the Actual Bytes Sent"
+ *
+ * Conventions shared by every entry point
+ *   - Every call returns an int status (SIGNMUON_OK or an error below) and
+ *     never aborts the process.  signmuon_last_error() gives the text of the
+ *     handle's last error.
+ *   - "device" pointers are CUDA device allocations of the calling process on
+ *     the handle's device (for example torch tensors); "host" pointers are
+ *     ordinary (ideally pinned) host memory.  Pointers passed as float/uint8
+ *     arrays must be 16-byte aligned.
+ *   - The parameter vector is flat: the matrices of `shapes` concatenated in
+ *     order, each row-major, d = sum(rows*cols) elements.  Convolution weights
+ *     are flattened to out x (in*kh*kw) by the caller.
+ *   - Work is enqueued on the CUDA stream given at init.  Calls return without
+ *     waiting for the GPU, except where a call says otherwise.
+ *   - The caller owns W, G, signs, sums, majority and every buffer it passes;
+ *     the library owns the momentum, the Newton-Schulz workspace and the
+ *     packed sign buffers of the step.
+ */
+#ifndef SIGNMUON_H
+#define SIGNMUON_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct signmuon_ctx* signmuon_t;
+
+/* status codes */
+#define SIGNMUON_OK            0
+#define SIGNMUON_E_INVALID     1  /* bad argument: shape, M, K, beta, lambda, eps, P, null or misaligned pointer */
+#define SIGNMUON_E_OVERFLOW    2  /* int8 vote accumulator requested with M > 127 */
+#define SIGNMUON_E_NONFINITE   3  /* a momentum norm was NaN/Inf: W was not updated */
+#define SIGNMUON_E_CUDA        4  /* a CUDA runtime/driver call failed */
+#define SIGNMUON_E_NOMEM       5  /* device allocation failed */
+#define SIGNMUON_E_TIMEOUT     6  /* a kernel's bounded wait expired; results are invalid */
+#define SIGNMUON_E_UNSUPPORTED 7  /* call not available for this handle (e.g. step on a vote-only handle) */
+
+/* scale step of PolarNS ([paper] Algorithm 1 input "scale") */
+#define SIGNMUON_SCALE_FRO      0  /* X0 = Mom / (||Mom||_F + eps) */
+#define SIGNMUON_SCALE_SPECTRAL 1  /* X0 = Mom / (sigma + eps), sigma by P power iterations */
+
+/* flags for signmuon_init */
+#define SIGNMUON_NS_FP32     (1u << 0) /* fp32 Newton-Schulz (SIMT) instead of bf16 tcgen05 tensor cores */
+#define SIGNMUON_NS_QUINTIC  (1u << 1) /* quintic NS X(15/8 I - 10/8 X^T X + 3/8 (X^T X)^2) */
+#define SIGNMUON_POST_POLAR  (1u << 2) /* post-vote local polar step: D = PolarNS(majority) */
+#define SIGNMUON_ACC_INT8    (1u << 3) /* signmuon_vote writes int8 sums (requires M <= 127) */
+#define SIGNMUON_ASYNC       (1u << 4) /* signmuon_step does not wait; signmuon_sync reports status */
+#define SIGNMUON_VOTE_ONLY   (1u << 5) /* allocate no step workspace: vote/pack/update calls only */
+
+/* ------------------------------------------------------------------------
+ * signmuon_init -- plan the step and allocate its device state.
+ *
+ * Defines the problem of [paper] Algorithm 1 and Algorithm 2 (their input
+ * lists: beta, lambda, K, eps, scale, P, and M workers).
+ *   out     host out-pointer; receives the handle (NULL on error).
+ *   shapes  host array of n_mats (rows, cols) pairs, each >= 1.
+ *   M       number of workers, 1..256.
+ *   beta    momentum in [0, 1).      lambda  coupled weight decay >= 0.
+ *   K       Newton-Schulz iterations >= 0 (0: U = X0, the scaled momentum).
+ *   eps     stability constant > 0, added to the scale: X0 = Mom/(s+eps).
+ *   scale   SIGNMUON_SCALE_FRO or SIGNMUON_SCALE_SPECTRAL.
+ *   P       power iterations (>= 1 when scale is spectral; ignored for fro).
+ *   flags   SIGNMUON_* flags above.
+ *   stream  cudaStream_t to enqueue on (NULL = the legacy default stream).
+ * Momentum starts at zero ([paper] Algorithm 2 initialisation).  Errors:
+ * E_INVALID, E_OVERFLOW (ACC_INT8 with M > 127), E_NOMEM, E_CUDA.
+ * ---------------------------------------------------------------------- */
+int signmuon_init(signmuon_t* out, const int64_t* shapes, int n_mats, int M,
+                  float beta, float lambda, int K, float eps, int scale, int P,
+                  unsigned flags, void* stream);
+
+/* ------------------------------------------------------------------------
+ * signmuon_step -- one distributed Sign-Muon step ([paper] Algorithm 2 with
+ * the tie-to-zero vote of [blog] "A tiny aggregation calculation", and the
+ * optional post-vote polar step of [paper] §4).
+ *   W    device float[d], updated in place: W <- fl32(W - eta*D).
+ *   G    host array of M device pointers, each float[d]: worker gradients.
+ *   eta  step size.
+ * Per worker: Mom_m <- beta*Mom_m + (1-beta)(G_m + lambda*W); U_m =
+ * PolarNS(Mom_m) per matrix; bits_m = (U_m >= 0) packed LSB-first.  Then
+ * sums = sum_m (2 bits_m - 1), majority = sign(sums) (0 on a tie), D =
+ * majority or PolarNS(majority) per matrix.  Unless SIGNMUON_ASYNC, waits for
+ * the GPU and returns E_NONFINITE when a momentum norm is NaN/Inf; W is then
+ * left unchanged (the momentum keeps the non-finite values: restore it with
+ * signmuon_set_momentum).
+ * ---------------------------------------------------------------------- */
+int signmuon_step(signmuon_t h, float* W, const float* const* G, float eta);
+
+/* ------------------------------------------------------------------------
+ * signmuon_step_host -- signmuon_step on HOST buffers: copies W and the M
+ * gradients to library-owned device buffers (allocated on first use),
+ * runs the step and copies W back.  Always waits.  Pinned host memory gives
+ * full copy bandwidth.
+ * ---------------------------------------------------------------------- */
+int signmuon_step_host(signmuon_t h, float* W_host, const float* const* G_host, float eta);
+
+/* ------------------------------------------------------------------------
+ * signmuon_vote -- majority vote over M packed one-bit sign buffers
+ * ([paper] Algorithm 2: integer SUM of signs, then sign(); [blog]: ties map
+ * to 0, sums range over [-M, M]).
+ *   signs     host array of M device pointers, each ceil(d/8) bytes; bit j of
+ *             byte b is element 8b+j, a set bit means +1.
+ *   d         number of entries (>= 0).
+ *   sums      device int32[d] (int8[d] when SIGNMUON_ACC_INT8), may be NULL.
+ *   majority  device int8[d] in {-1, 0, +1}, may be NULL.
+ * Results are bit-exact integers.
+ * ---------------------------------------------------------------------- */
+int signmuon_vote(signmuon_t h, const uint8_t* const* signs, int64_t d, void* sums,
+                  int8_t* majority);
+
+/* ------------------------------------------------------------------------
+ * signmuon_pack -- entrywise one-bit sign of a flat float vector ([paper] §3
+ * entrywise sign; [blog] d/8-byte payload): bit = (U >= 0), so 0 and -0 send
+ * +1 and NaN sends 0.  U device float[d]; out device uint8[ceil(d/8)], pad
+ * bits 0.
+ * ---------------------------------------------------------------------- */
+int signmuon_pack(signmuon_t h, const float* U, int64_t d, uint8_t* out);
+
+/* ------------------------------------------------------------------------
+ * signmuon_apply_update -- W <- fl32(W - eta*D), one rounding (fused
+ * multiply-add), [paper] Algorithm 1/2 update.  W, D device float[d].
+ * ---------------------------------------------------------------------- */
+int signmuon_apply_update(signmuon_t h, float* W, const float* D, int64_t d, float eta);
+
+/* ------------------------------------------------------------------------
+ * signmuon_polar -- PolarNS of every matrix of the plan for M independent
+ * inputs ([paper] §3 Muon polar factor, §4 Newton-Schulz), with the handle's
+ * K, eps, scale, P and precision flags.
+ *   X  host array of M device pointers, each float[d] (flat matrices).
+ *   U  host array of M device pointers, each float[d] (output).
+ * ---------------------------------------------------------------------- */
+int signmuon_polar(signmuon_t h, const float* const* X, float* const* U);
+
+/* ------------------------------------------------------------------------
+ * State access (device float[d] / uint8[ceil(d/8)] buffers of the caller).
+ * get/set_momentum: worker m's momentum (checkpoint / resume).
+ * get_polar: worker m's U from the last step.  get_signs: worker m's packed
+ * bits from the last step.  get_direction: the last step's D.
+ * get_scales: host float[M*n_mats]: the last step's scale s per (worker,
+ * matrix), worker-major (waits for the GPU).
+ * ---------------------------------------------------------------------- */
+int signmuon_get_momentum(signmuon_t h, int m, float* dst);
+int signmuon_set_momentum(signmuon_t h, int m, const float* src);
+int signmuon_get_polar(signmuon_t h, int m, float* dst);
+int signmuon_get_signs(signmuon_t h, int m, uint8_t* dst);
+int signmuon_get_direction(signmuon_t h, float* dst);
+int signmuon_get_scales(signmuon_t h, float* dst_host);
+
+/* Newton-Schulz coefficients: n=2 (a, b) for X <- aX + b(XX^T)X ([paper] §3
+ * two-coefficient form), n=3 (a, b, c) for the quintic flag.  Defaults:
+ * (1.5, -0.5) and (15/8, -10/8, 3/8). */
+int signmuon_set_ns_coeffs(signmuon_t h, const float* coeffs, int n);
+
+/* Wait for the handle's stream; returns the first deferred error
+ * (E_NONFINITE, E_TIMEOUT, E_CUDA) since the last sync, and clears it. */
+int signmuon_sync(signmuon_t h);
+
+/* Sizes: out[0]=d, out[1]=packed bytes per worker, out[2]=device bytes owned
+ * by the handle, out[3]=number of shape groups, out[4]=M, out[5]=n_mats. */
+int signmuon_info(signmuon_t h, int64_t* out, int n);
+
+/* Host-only planning (no GPU needed): same outputs as signmuon_info for a
+ * would-be handle; validates like signmuon_init. */
+int signmuon_plan(const int64_t* shapes, int n_mats, int M, int K, int scale, int P,
+                  unsigned flags, int64_t* out, int n);
+
+/* Per-kernel timing.  signmuon_profile(h, 1) makes the following calls record
+ * a CUDA event pair around every kernel they launch on the handle's stream;
+ * signmuon_profile_read() waits for the stream, adds up the elapsed times per
+ * kind (ms[k], launches[k] for k < n) since the last read, and resets them.
+ * Kinds: 0 momentum pass, 1 norm finalisation, 2 Newton-Schulz GEMMs,
+ * 3 power iteration, 4 one-bit pack, 5 vote (fused with the update or writing
+ * D), 6 staging of the majority, 7 post-vote Newton-Schulz GEMMs, 8 update,
+ * 9 K=0 scaling. */
+#define SIGNMUON_PROF_KINDS 10
+int signmuon_profile(signmuon_t h, int enable);
+int signmuon_profile_read(signmuon_t h, double* ms, int64_t* launches, int n);
+
+/* Number of kernels this library has launched in this process (all handles). */
+int64_t signmuon_kernel_launches(void);
+
+const char* signmuon_last_error(signmuon_t h);
+const char* signmuon_status_string(int status);
+void signmuon_destroy(signmuon_t h);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SIGNMUON_H */

@@ -1,0 +1,325 @@
+"""Python binding of libsignmuon.so (the C ABI in include/signmuon.h).
+
+Argument marshalling only: every step of the optimizer runs in the library's
+CUDA kernels.  Device buffers are passed as torch CUDA tensors (or raw integer
+device addresses); host buffers as numpy arrays.  The functions keep the C
+names; each raises SignMuonError on a non-zero status.
+
+The library must be built first (``python -m sign_muon_optimizer_b200.build``);
+importing this package without it raises ImportError -- there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsignmuon.so")
+
+# status codes, scales and flags (include/signmuon.h)
+SIGNMUON_OK = 0
+SIGNMUON_E_INVALID = 1
+SIGNMUON_E_OVERFLOW = 2
+SIGNMUON_E_NONFINITE = 3
+SIGNMUON_E_CUDA = 4
+SIGNMUON_E_NOMEM = 5
+SIGNMUON_E_TIMEOUT = 6
+SIGNMUON_E_UNSUPPORTED = 7
+SIGNMUON_SCALE_FRO = 0
+SIGNMUON_SCALE_SPECTRAL = 1
+SIGNMUON_NS_FP32 = 1 << 0
+SIGNMUON_NS_QUINTIC = 1 << 1
+SIGNMUON_POST_POLAR = 1 << 2
+SIGNMUON_ACC_INT8 = 1 << 3
+SIGNMUON_ASYNC = 1 << 4
+SIGNMUON_VOTE_ONLY = 1 << 5
+
+EXPORTED = [
+    "signmuon_init", "signmuon_step", "signmuon_step_host", "signmuon_vote", "signmuon_pack",
+    "signmuon_apply_update", "signmuon_polar", "signmuon_get_momentum", "signmuon_set_momentum",
+    "signmuon_get_polar", "signmuon_get_signs", "signmuon_get_direction", "signmuon_get_scales",
+    "signmuon_set_ns_coeffs", "signmuon_sync", "signmuon_info", "signmuon_plan",
+    "signmuon_kernel_launches", "signmuon_last_error", "signmuon_status_string", "signmuon_destroy",
+    "signmuon_profile", "signmuon_profile_read",
+]
+PROF_KINDS = ["momentum", "norm_finalize", "ns_gemm", "power_iter", "pack", "vote", "stage",
+              "post_ns_gemm", "update", "k0_scale"]
+
+
+class SignMuonError(RuntimeError):
+    def __init__(self, status, msg):
+        super().__init__(f"signmuon status {status}: {msg}")
+        self.status = status
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is not built; run `python -m sign_muon_optimizer_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, I64, F, U = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_uint
+    PP = ctypes.POINTER(ctypes.c_void_p)
+    sig = {
+        "signmuon_init": (I, [ctypes.POINTER(P), ctypes.POINTER(I64), I, I, F, F, I, F, I, I, U, P]),
+        "signmuon_step": (I, [P, P, PP, F]),
+        "signmuon_step_host": (I, [P, P, PP, F]),
+        "signmuon_vote": (I, [P, PP, I64, P, P]),
+        "signmuon_pack": (I, [P, P, I64, P]),
+        "signmuon_apply_update": (I, [P, P, P, I64, F]),
+        "signmuon_polar": (I, [P, PP, PP]),
+        "signmuon_get_momentum": (I, [P, I, P]),
+        "signmuon_set_momentum": (I, [P, I, P]),
+        "signmuon_get_polar": (I, [P, I, P]),
+        "signmuon_get_signs": (I, [P, I, P]),
+        "signmuon_get_direction": (I, [P, P]),
+        "signmuon_get_scales": (I, [P, P]),
+        "signmuon_set_ns_coeffs": (I, [P, ctypes.POINTER(F), I]),
+        "signmuon_sync": (I, [P]),
+        "signmuon_info": (I, [P, ctypes.POINTER(I64), I]),
+        "signmuon_plan": (I, [ctypes.POINTER(I64), I, I, I, I, I, U, ctypes.POINTER(I64), I]),
+        "signmuon_kernel_launches": (I64, []),
+        "signmuon_last_error": (ctypes.c_char_p, [P]),
+        "signmuon_status_string": (ctypes.c_char_p, [I]),
+        "signmuon_destroy": (None, [P]),
+        "signmuon_profile": (I, [P, I]),
+        "signmuon_profile_read": (I, [P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(I64), I]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib = _load()
+
+
+def _ptr(x):
+    """Device/host address of a torch tensor, numpy array or int."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    if hasattr(x, "data_ptr"):
+        return x.data_ptr()
+    if isinstance(x, np.ndarray):
+        return x.ctypes.data
+    raise TypeError(f"cannot take the address of {type(x)}")
+
+
+def _ptr_array(xs):
+    arr = (ctypes.c_void_p * len(xs))()
+    for i, x in enumerate(xs):
+        arr[i] = _ptr(x)
+    return arr
+
+
+def _check(h, rc):
+    if rc != 0:
+        raise SignMuonError(rc, _lib.signmuon_last_error(h).decode(errors="replace"))
+
+
+def _shapes_arr(shapes):
+    flat = [int(v) for rc in shapes for v in rc]
+    return (ctypes.c_int64 * max(1, len(flat)))(*flat), len(shapes)
+
+
+def _default_stream():
+    try:
+        import torch
+        if torch.cuda.is_available():
+            return torch.cuda.current_stream().cuda_stream
+    except Exception:
+        pass
+    return None
+
+
+# ---- functions with the C names -------------------------------------------
+
+def signmuon_init(shapes, M, beta, lam, K, eps, scale, P=1, flags=0, stream=None):
+    if isinstance(scale, str):
+        scale = {"fro": SIGNMUON_SCALE_FRO, "spectral": SIGNMUON_SCALE_SPECTRAL}[scale]
+    arr, n = _shapes_arr(shapes)
+    h = ctypes.c_void_p()
+    if stream is None:
+        stream = _default_stream()
+    rc = _lib.signmuon_init(ctypes.byref(h), arr, n, int(M), float(beta), float(lam), int(K), float(eps),
+                            int(scale), int(P), int(flags), stream)
+    _check(None, rc)
+    return h
+
+
+def signmuon_step(h, W, G, eta):
+    _check(h, _lib.signmuon_step(h, _ptr(W), _ptr_array(G), float(eta)))
+
+
+def signmuon_step_host(h, W_host, G_host, eta):
+    _check(h, _lib.signmuon_step_host(h, _ptr(W_host), _ptr_array(G_host), float(eta)))
+
+
+def signmuon_vote(h, signs, d, sums=None, majority=None):
+    _check(h, _lib.signmuon_vote(h, _ptr_array(signs), int(d), _ptr(sums), _ptr(majority)))
+
+
+def signmuon_pack(h, U, d, out):
+    _check(h, _lib.signmuon_pack(h, _ptr(U), int(d), _ptr(out)))
+
+
+def signmuon_apply_update(h, W, D, d, eta):
+    _check(h, _lib.signmuon_apply_update(h, _ptr(W), _ptr(D), int(d), float(eta)))
+
+
+def signmuon_polar(h, X, U):
+    _check(h, _lib.signmuon_polar(h, _ptr_array(X), _ptr_array(U)))
+
+
+def signmuon_get_momentum(h, m, dst):
+    _check(h, _lib.signmuon_get_momentum(h, int(m), _ptr(dst)))
+
+
+def signmuon_set_momentum(h, m, src):
+    _check(h, _lib.signmuon_set_momentum(h, int(m), _ptr(src)))
+
+
+def signmuon_get_polar(h, m, dst):
+    _check(h, _lib.signmuon_get_polar(h, int(m), _ptr(dst)))
+
+
+def signmuon_get_signs(h, m, dst):
+    _check(h, _lib.signmuon_get_signs(h, int(m), _ptr(dst)))
+
+
+def signmuon_get_direction(h, dst):
+    _check(h, _lib.signmuon_get_direction(h, _ptr(dst)))
+
+
+def signmuon_get_scales(h, M, n_mats):
+    out = np.zeros(M * n_mats, np.float32)
+    _check(h, _lib.signmuon_get_scales(h, out.ctypes.data))
+    return out.reshape(M, n_mats)
+
+
+def signmuon_set_ns_coeffs(h, coeffs):
+    c = (ctypes.c_float * len(coeffs))(*[float(v) for v in coeffs])
+    _check(h, _lib.signmuon_set_ns_coeffs(h, c, len(coeffs)))
+
+
+def signmuon_sync(h):
+    _check(h, _lib.signmuon_sync(h))
+
+
+def signmuon_info(h):
+    out = (ctypes.c_int64 * 6)()
+    _check(h, _lib.signmuon_info(h, out, 6))
+    return dict(zip(["d", "packed_bytes", "device_bytes", "groups", "M", "n_mats"], list(out)))
+
+
+def signmuon_plan(shapes, M, K=5, scale=SIGNMUON_SCALE_FRO, P=1, flags=0):
+    if isinstance(scale, str):
+        scale = {"fro": SIGNMUON_SCALE_FRO, "spectral": SIGNMUON_SCALE_SPECTRAL}[scale]
+    arr, n = _shapes_arr(shapes)
+    out = (ctypes.c_int64 * 6)()
+    _check(None, _lib.signmuon_plan(arr, n, int(M), int(K), int(scale), int(P), int(flags), out, 6))
+    return dict(zip(["d", "packed_bytes", "device_bytes", "groups", "M", "n_mats"], list(out)))
+
+
+def signmuon_kernel_launches():
+    return int(_lib.signmuon_kernel_launches())
+
+
+def signmuon_last_error(h=None):
+    return _lib.signmuon_last_error(h).decode(errors="replace")
+
+
+def signmuon_status_string(status):
+    return _lib.signmuon_status_string(int(status)).decode()
+
+
+def signmuon_destroy(h):
+    _lib.signmuon_destroy(h)
+
+
+def signmuon_profile(h, enable):
+    _check(h, _lib.signmuon_profile(h, 1 if enable else 0))
+
+
+def signmuon_profile_read(h):
+    """{kind: (total ms, launches)} since the last read (waits for the stream)."""
+    n = len(PROF_KINDS)
+    ms = (ctypes.c_double * n)()
+    cnt = (ctypes.c_int64 * n)()
+    _check(h, _lib.signmuon_profile_read(h, ms, cnt, n))
+    return {k: (float(ms[i]), int(cnt[i])) for i, k in enumerate(PROF_KINDS)}
+
+
+class SignMuon:
+    """Owning wrapper of a handle: ``SignMuon(shapes, M, ...)`` then
+    ``.step(W, G, eta)``; the remaining methods mirror the C calls."""
+
+    def __init__(self, shapes, M, beta=0.9, lam=0.01, K=5, eps=1e-7, scale="fro", P=1, flags=0,
+                 stream=None):
+        self.shapes = [(int(r), int(c)) for r, c in shapes]
+        self.M = int(M)
+        self.h = signmuon_init(self.shapes, M, beta, lam, K, eps, scale, P, flags, stream)
+        self.info = signmuon_info(self.h)
+        self.d = self.info["d"]
+
+    def step(self, W, G, eta):
+        signmuon_step(self.h, W, G, eta)
+
+    def step_host(self, W, G, eta):
+        signmuon_step_host(self.h, W, G, eta)
+
+    def vote(self, signs, d, sums=None, majority=None):
+        signmuon_vote(self.h, signs, d, sums, majority)
+
+    def pack(self, U, d, out):
+        signmuon_pack(self.h, U, d, out)
+
+    def apply_update(self, W, D, d, eta):
+        signmuon_apply_update(self.h, W, D, d, eta)
+
+    def polar(self, X, U):
+        signmuon_polar(self.h, X, U)
+
+    def get_momentum(self, m, dst):
+        signmuon_get_momentum(self.h, m, dst)
+
+    def set_momentum(self, m, src):
+        signmuon_set_momentum(self.h, m, src)
+
+    def get_polar(self, m, dst):
+        signmuon_get_polar(self.h, m, dst)
+
+    def get_signs(self, m, dst):
+        signmuon_get_signs(self.h, m, dst)
+
+    def get_direction(self, dst):
+        signmuon_get_direction(self.h, dst)
+
+    def get_scales(self):
+        return signmuon_get_scales(self.h, self.M, len(self.shapes))
+
+    def set_ns_coeffs(self, coeffs):
+        signmuon_set_ns_coeffs(self.h, coeffs)
+
+    def sync(self):
+        signmuon_sync(self.h)
+
+    def profile(self, enable=True):
+        signmuon_profile(self.h, enable)
+
+    def profile_read(self):
+        return signmuon_profile_read(self.h)
+
+    def close(self):
+        if self.h is not None:
+            signmuon_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -1,0 +1,133 @@
+// common.cuh -- device-side plan records and launch wrappers shared by the
+// kernels of libsignmuon.so.
+//
+// Data layout in HBM (one handle):
+//   flat vectors      W, G_m, Mom_m, U_m, D: d floats, matrices in plan order,
+//                     each row-major (the caller's layout)
+//   grouped X / A / B matrices of equal shape share a "group"; problem b of a
+//                     group (b = worker*count + index-in-group) sits at
+//                     base + b*rows*ld (X) or base + b*g*gld (A, B); rows are
+//                     padded to ld = round_up(cols, 8) elements so that every
+//                     row starts on a 16-byte boundary (TMA stride rule)
+//   packed bits       one ceil(d/8)-byte stream per worker, padded to 16 bytes
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+namespace sm {
+
+constexpr int kMaxWorkers = 256;
+
+struct MatInfo {      // one parameter matrix
+  int64_t off;        // start in the flat vector
+  int rows, cols;
+  int group, q;       // shape group and index within it
+};
+
+struct GroupInfo {    // all matrices of one shape
+  int rows, cols, ld; // natural shape, padded row stride of X
+  int g, gld;         // g = min(rows, cols): Gram side; padded row stride of A/B
+  int wide;           // rows <= cols: Gram X X^T; else X^T X
+  int count;          // matrices of this shape
+  int first;          // index into the group->matrix list
+  int64_t x_base;     // element offset of the group in an X buffer
+  int64_t a_base;     // element offset of the group in the A/B buffers
+};
+
+struct Chunk {        // a piece of one matrix for the flat elementwise kernels
+  int mat;
+  int len;            // <= kChunk elements
+  int64_t start;      // element offset within the matrix
+};
+constexpr int kChunk = 4096;
+
+struct ProbRows {     // a block of Gram rows for the power-iteration matvec
+  int p;              // problem id (worker*n_mats + mat)
+  int row0;
+};
+constexpr int kPiRows = 32;
+
+struct WorkerPtrs {   // per-worker device pointers passed by value
+  const float* p[kMaxWorkers];
+};
+
+// One shape group's tiles inside one grouped GEMM launch.
+struct TileGroup {
+  int group;
+  int Mdim, Ndim, Kdim;
+  int BN;             // 64, 128 or 256
+  int tiles_m, tiles_n;
+  int batch;          // problems of this group in the launch
+  int tile_start;     // first global tile index of this group
+};
+
+enum GemmOp { OP_GRAM = 0, OP_SQUARE = 1, OP_APPLY = 2 };
+
+// Arguments of one grouped Newton-Schulz GEMM launch (both precisions).
+struct GemmArgs {
+  const TileGroup* tiles;
+  int n_tile_groups;
+  int total_tiles;
+  const GroupInfo* groups;
+  const int* group_mats;     // matrices of each group, in order
+  const int64_t* mat_off;    // flat offset of each matrix
+  int n_mats;
+  int op;
+  void* X_src;               // X buffer read (APPLY/GRAM operand and APPLY epilogue)
+  void* X_dst;               // X buffer written by a non-final APPLY
+  void* A;                   // Gram buffer
+  void* B;                   // quintic polynomial buffer
+  int p_from_b;              // APPLY multiplies by B (quintic) instead of A
+  int map_src, map_dst;      // tensor-map slots of X_src / X_dst (TMA path)
+  // epilogue coefficients: per-problem float2 when coef is non-null, else (c0, c1)
+  const float2* coef;
+  float c0, c1;
+  // final APPLY: fp32 flat output out + worker*out_stride + mat_off + r*cols + c
+  float* out;
+  int64_t out_stride;
+  int final_out;
+  int* err;
+};
+
+// ---- launch wrappers (host) ----------------------------------------------
+void count_launch();
+
+void launch_momentum(cudaStream_t s, const WorkerPtrs& G, const float* W, float* Mom, int64_t d,
+                     int M, float beta, float lambda, void* X, int x_bf16, const Chunk* chunks,
+                     int n_chunks, const MatInfo* mats, const GroupInfo* groups, float* partials);
+void launch_stage(cudaStream_t s, const WorkerPtrs& in, int M, void* X, int x_bf16,
+                  const Chunk* chunks, int n_chunks, const MatInfo* mats, const GroupInfo* groups,
+                  float* partials);
+void launch_fro_finalize(cudaStream_t s, int n_probs, int n_mats, int M, const float* partials,
+                         const int* mat_chunk0, const int* mat_nchunks, int use_for_scale,
+                         float eps, int quintic, float a, float b, float c, float* scale,
+                         float2* coef_apply, float2* coef_square, int* status);
+void launch_pi_init(cudaStream_t s, int n_probs, const int64_t* uoff, const int* prob_g, float* u);
+void launch_pi_matvec(cudaStream_t s, const ProbRows* rows, int n_rows, const void* A, int a_bf16,
+                      const int64_t* prob_a_off, const int* prob_g, const int* prob_gld,
+                      const int64_t* uoff, const float* u, float* y);
+void launch_pi_normalize(cudaStream_t s, int n_probs, const int64_t* uoff, const int* prob_g,
+                         const float* y, float* u);
+void launch_pi_finalize(cudaStream_t s, int n_probs, const int64_t* uoff, const int* prob_g,
+                        const float* u, const float* y, float eps, int quintic, float a, float b,
+                        float c, float* scale, float2* coef_apply, float2* coef_square, int* status);
+void launch_scale_flat(cudaStream_t s, const WorkerPtrs& in, int M, float* out, int64_t out_stride,
+                       const Chunk* chunks, int n_chunks, const MatInfo* mats, int n_mats,
+                       const float* scale, float eps);
+void launch_pack(cudaStream_t s, const float* U, int64_t u_stride, int64_t d, uint8_t* out,
+                 int64_t out_stride, int M);
+void launch_vote(cudaStream_t s, const WorkerPtrs& signs, int M, int64_t d, void* sums, int acc8,
+                 int8_t* majority);
+void launch_vote_update(cudaStream_t s, const uint8_t* bits, int64_t bits_stride, int M, int64_t d,
+                        float* W, float eta, const int* status);
+void launch_vote_major(cudaStream_t s, const uint8_t* bits, int64_t bits_stride, int M, int64_t d,
+                       float* D);
+void launch_update(cudaStream_t s, float* W, const float* D, int64_t d, float eta,
+                   const int* status);
+
+void launch_gemm_simt(cudaStream_t s, const GemmArgs& a, int x_f32);
+int gemm_tc_smem_bytes();
+void launch_gemm_tc(cudaStream_t s, const GemmArgs& a, const void* maps, int n_sm);
+
+}  // namespace sm

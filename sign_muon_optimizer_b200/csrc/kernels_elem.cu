@@ -1,0 +1,612 @@
+// kernels_elem.cu -- the HBM-bound kernels of the Sign-Muon step:
+//   momentum pass (weight decay + momentum + X staging + Frobenius partials),
+//   scale finalisation, power iteration on the Gram matrix, one-bit pack,
+//   majority vote (API form, fused with the update, or emitting D), update.
+//
+// Sources, by page title:
+//   [paper] "SignMuon: 通信高效的分布式Muon优化" (a rendering of arXiv 2605.16311)
+//   [blog]  "SignMuon: Matrix Directions, Majority Votes, and the Actual Bytes Sent"
+#include "common.cuh"
+
+#include <cmath>
+
+namespace sm {
+
+namespace {
+
+constexpr int kThreads = 256;
+
+__device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ void st4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
+
+__device__ __forceinline__ float warp_sum(float v) {
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ double warp_sum_d(double v) {
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Fixed-order block reduction (deterministic): warp sums, then warp 0.
+template <typename T>
+__device__ T block_sum(T v, T* red) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  v = (sizeof(T) == 8) ? (T)warp_sum_d((double)v) : (T)warp_sum((float)v);
+  __syncthreads();
+  if (lane == 0) red[wid] = v;
+  __syncthreads();
+  T t = 0;
+  if (wid == 0) {
+    t = (lane < (int)(blockDim.x >> 5)) ? red[lane] : (T)0;
+    t = (sizeof(T) == 8) ? (T)warp_sum_d((double)t) : (T)warp_sum((float)t);
+  }
+  return t;  // valid in thread 0
+}
+
+__device__ __forceinline__ void store_x(void* X, int64_t idx, float v, bool bf16) {
+  if (bf16) reinterpret_cast<__nv_bfloat16*>(X)[idx] = __float2bfloat16_rn(v);
+  else reinterpret_cast<float*>(X)[idx] = v;
+}
+__device__ __forceinline__ void store_x4(void* X, int64_t idx, float4 v, bool bf16) {
+  if (bf16) {
+    __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y);
+    __nv_bfloat162 hi = __floats2bfloat162_rn(v.z, v.w);
+    uint2 u;
+    u.x = *reinterpret_cast<uint32_t*>(&lo);
+    u.y = *reinterpret_cast<uint32_t*>(&hi);
+    *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(X) + idx) = u;
+  } else {
+    st4(reinterpret_cast<float*>(X) + idx, v);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Momentum pass ([paper] Algorithm 1 / Algorithm 2: G~ = G + lambda W, then
+// Mom <- beta Mom + (1-beta) G~).  One block owns one chunk of one matrix
+// and loops over the workers, so W is read once per element.  It writes the
+// new momentum, the Newton-Schulz input X (bf16 or fp32, grouped layout) and
+// the chunk's sum of squares per worker (for the Frobenius scale and the
+// non-finite check).  MOMENTUM=false stages a caller's vector unchanged.
+// ---------------------------------------------------------------------------
+template <bool MOMENTUM>
+__global__ void __launch_bounds__(kThreads)
+k_momentum(WorkerPtrs G, const float* __restrict__ W, float* __restrict__ Mom, int64_t d, int M,
+           float beta, float lambda, void* __restrict__ X, int x_bf16,
+           const Chunk* __restrict__ chunks, const MatInfo* __restrict__ mats,
+           const GroupInfo* __restrict__ groups, float* __restrict__ partials) {
+  __shared__ float red[32];
+  const Chunk ch = chunks[blockIdx.x];
+  const MatInfo mi = mats[ch.mat];
+  const GroupInfo gi = groups[mi.group];
+  const int64_t base = mi.off + ch.start;
+  const bool vec = ((base & 3) == 0) && ((ch.len & 3) == 0) && ((mi.cols & 3) == 0);
+  const float omb = 1.f - beta;
+  const bool bf = x_bf16 != 0;
+  constexpr int kV = kChunk / (kThreads * 4);  // float4 groups per thread
+  float4 wv[kV];
+  if (MOMENTUM && vec) {
+#pragma unroll
+    for (int j = 0; j < kV; ++j) {
+      const int e = (threadIdx.x + j * kThreads) * 4;
+      wv[j] = (e < ch.len) ? ld4(W + base + e) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
+  for (int m = 0; m < M; ++m) {
+    const float* g = G.p[m];
+    float* mom = MOMENTUM ? Mom + (int64_t)m * d : nullptr;
+    const int64_t xb = gi.x_base + (int64_t)(m * gi.count + mi.q) * gi.rows * gi.ld;
+    float ss = 0.f;
+    if (vec) {
+#pragma unroll
+      for (int j = 0; j < kV; ++j) {
+        const int e = (threadIdx.x + j * kThreads) * 4;
+        if (e < ch.len) {
+          const int64_t fe = base + e;
+          float4 v = ld4(g + fe);
+          if (MOMENTUM) {
+            const float4 mo = ld4(mom + fe);
+            v.x = fmaf(beta, mo.x, omb * fmaf(lambda, wv[j].x, v.x));
+            v.y = fmaf(beta, mo.y, omb * fmaf(lambda, wv[j].y, v.y));
+            v.z = fmaf(beta, mo.z, omb * fmaf(lambda, wv[j].z, v.z));
+            v.w = fmaf(beta, mo.w, omb * fmaf(lambda, wv[j].w, v.w));
+            st4(mom + fe, v);
+          }
+          ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+          const int le = (int)(ch.start + e);
+          const int r = le / mi.cols, c = le - r * mi.cols;
+          store_x4(X, xb + (int64_t)r * gi.ld + c, v, bf);
+        }
+      }
+    } else {
+      for (int e = threadIdx.x; e < ch.len; e += kThreads) {
+        const int64_t fe = base + e;
+        float v = g[fe];
+        if (MOMENTUM) {
+          v = fmaf(beta, mom[fe], omb * fmaf(lambda, W[fe], v));
+          mom[fe] = v;
+        }
+        ss += v * v;
+        const int le = (int)(ch.start + e);
+        const int r = le / mi.cols, c = le - r * mi.cols;
+        store_x(X, xb + (int64_t)r * gi.ld + c, v, bf);
+      }
+    }
+    const float t = block_sum<float>(ss, red);
+    if (threadIdx.x == 0) partials[(int64_t)blockIdx.x * M + m] = t;
+  }
+}
+
+__device__ __forceinline__ void set_coefs(int p, float cc, int quintic, float a, float b, float c,
+                                          float2* coef_apply, float2* coef_square) {
+  // Iteration 0 runs on the unscaled X~ and Gram A~ = X~ X~^T.  With X0 = cc X~:
+  //   cubic:   X1 = a cc X~ + b cc^3 A~ X~
+  //   quintic: B = b cc^2 A~ + c cc^4 A~^2;  X1 = cc (a X~ + B X~)
+  if (!quintic) {
+    coef_apply[p] = make_float2(a * cc, b * cc * cc * cc);
+  } else {
+    coef_square[p] = make_float2(b * cc * cc, c * cc * cc * cc * cc);
+    coef_apply[p] = make_float2(a * cc, cc);
+  }
+}
+
+// Sum the chunk partials of each (worker, matrix) in a fixed order.
+__global__ void __launch_bounds__(kThreads)
+k_fro_finalize(int n_mats, int M, const float* __restrict__ partials, const int* __restrict__ mat_chunk0,
+               const int* __restrict__ mat_nchunks, int use_for_scale, float eps, int quintic,
+               float a, float b, float c, float* __restrict__ scale, float2* coef_apply,
+               float2* coef_square, int* status) {
+  __shared__ double red[32];
+  const int p = blockIdx.x;
+  const int w = p / n_mats, i = p - w * n_mats;
+  const int c0 = mat_chunk0[i], nc = mat_nchunks[i];
+  double s = 0.0;
+  for (int j = threadIdx.x; j < nc; j += kThreads) s += (double)partials[(int64_t)(c0 + j) * M + w];
+  const double t = block_sum<double>(s, red);
+  if (threadIdx.x == 0) {
+    if (!isfinite(t)) atomicOr(status, 1);
+    if (use_for_scale) {
+      const float sc = (float)sqrt(t);
+      scale[p] = sc;
+      set_coefs(p, 1.f / (sc + eps), quintic, a, b, c, coef_apply, coef_square);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Power iteration on the Gram matrix A~ = X~ X~^T of the wide orientation
+// ([paper] Algorithm 1 inputs scale=spectral and P; §4 spectral
+// normalisation by power iteration): u0 = ones/sqrt(g); u <- A~u/||A~u|| P
+// times; sigma^2 = u^T A~ u (= ||X~^T u||^2).  The Gram is the first
+// Newton-Schulz GEMM's output, so no extra pass over X is needed.
+// ---------------------------------------------------------------------------
+__global__ void k_pi_init(const int64_t* __restrict__ uoff, const int* __restrict__ prob_g,
+                          float* __restrict__ u) {
+  const int p = blockIdx.x;
+  const int g = prob_g[p];
+  const float v = rsqrtf((float)g);
+  for (int k = threadIdx.x; k < g; k += blockDim.x) u[uoff[p] + k] = v;
+}
+
+template <bool BF16>
+__global__ void __launch_bounds__(kThreads)
+k_pi_matvec(const ProbRows* __restrict__ rows, const void* __restrict__ A,
+            const int64_t* __restrict__ prob_a_off, const int* __restrict__ prob_g,
+            const int* __restrict__ prob_gld, const int64_t* __restrict__ uoff,
+            const float* __restrict__ u, float* __restrict__ y) {
+  const ProbRows pr = rows[blockIdx.x];
+  const int p = pr.p;
+  const int g = prob_g[p], gld = prob_gld[p];
+  const float* up = u + uoff[p];
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  constexpr int kRowsPerWarp = kPiRows / (kThreads / 32);
+  for (int j = 0; j < kRowsPerWarp; ++j) {
+    const int r = pr.row0 + wid * kRowsPerWarp + j;
+    if (r >= g) break;
+    float acc = 0.f;
+    if (BF16) {
+      const __nv_bfloat16* a = reinterpret_cast<const __nv_bfloat16*>(A) + prob_a_off[p] + (int64_t)r * gld;
+      const int g8 = g & ~7;
+      for (int k = lane * 8; k < g8; k += 256) {
+        const uint4 raw = *reinterpret_cast<const uint4*>(a + k);
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const float2 f = __bfloat1622float2(h[t]);
+          acc = fmaf(f.x, up[k + 2 * t], acc);
+          acc = fmaf(f.y, up[k + 2 * t + 1], acc);
+        }
+      }
+      for (int k = g8 + lane; k < g; k += 32) acc = fmaf(__bfloat162float(a[k]), up[k], acc);
+    } else {
+      const float* a = reinterpret_cast<const float*>(A) + prob_a_off[p] + (int64_t)r * gld;
+      const int g4 = g & ~3;
+      for (int k = lane * 4; k < g4; k += 128) {
+        const float4 f = ld4(a + k);
+        acc = fmaf(f.x, up[k], acc);
+        acc = fmaf(f.y, up[k + 1], acc);
+        acc = fmaf(f.z, up[k + 2], acc);
+        acc = fmaf(f.w, up[k + 3], acc);
+      }
+      for (int k = g4 + lane; k < g; k += 32) acc = fmaf(a[k], up[k], acc);
+    }
+    acc = warp_sum(acc);
+    if (lane == 0) y[uoff[p] + r] = acc;
+  }
+}
+
+__global__ void __launch_bounds__(kThreads)
+k_pi_normalize(const int64_t* __restrict__ uoff, const int* __restrict__ prob_g,
+               const float* __restrict__ y, float* __restrict__ u) {
+  __shared__ double red[32];
+  __shared__ float inv;
+  const int p = blockIdx.x;
+  const int g = prob_g[p];
+  const float* yp = y + uoff[p];
+  double s = 0.0;
+  for (int k = threadIdx.x; k < g; k += kThreads) s += (double)yp[k] * (double)yp[k];
+  const double t = block_sum<double>(s, red);
+  if (threadIdx.x == 0) inv = (t > 0.0) ? (float)(1.0 / sqrt(t)) : 0.f;  // a zero iterate stays zero
+  __syncthreads();
+  for (int k = threadIdx.x; k < g; k += kThreads) u[uoff[p] + k] = yp[k] * inv;
+}
+
+__global__ void __launch_bounds__(kThreads)
+k_pi_finalize(const int64_t* __restrict__ uoff, const int* __restrict__ prob_g,
+              const float* __restrict__ u, const float* __restrict__ y, float eps, int quintic,
+              float a, float b, float c, float* __restrict__ scale, float2* coef_apply,
+              float2* coef_square, int* status) {
+  __shared__ double red[32];
+  const int p = blockIdx.x;
+  const int g = prob_g[p];
+  double s = 0.0;
+  for (int k = threadIdx.x; k < g; k += kThreads) s += (double)u[uoff[p] + k] * (double)y[uoff[p] + k];
+  const double t = block_sum<double>(s, red);
+  if (threadIdx.x == 0) {
+    const float sc = (float)sqrt(fmax(t, 0.0));
+    if (!isfinite(t)) atomicOr(status, 1);
+    scale[p] = sc;
+    set_coefs(p, 1.f / (sc + eps), quintic, a, b, c, coef_apply, coef_square);
+  }
+}
+
+// K = 0: U = X0 = in / (s + eps) straight from the fp32 input.
+__global__ void __launch_bounds__(kThreads)
+k_scale_flat(WorkerPtrs in, float* __restrict__ out, int64_t out_stride,
+             const Chunk* __restrict__ chunks, const MatInfo* __restrict__ mats, int n_mats,
+             const float* __restrict__ scale, float eps) {
+  const Chunk ch = chunks[blockIdx.x];
+  const int w = blockIdx.y;
+  const MatInfo mi = mats[ch.mat];
+  const float cc = 1.f / (scale[w * n_mats + ch.mat] + eps);
+  const float* src = in.p[w];
+  float* dst = out + (int64_t)w * out_stride;
+  const int64_t base = mi.off + ch.start;
+  for (int e = threadIdx.x; e < ch.len; e += kThreads) dst[base + e] = src[base + e] * cc;
+}
+
+// ---------------------------------------------------------------------------
+// One-bit pack ([paper] §3 entrywise sign; [blog] d/8-byte payload).
+// bit = (u >= 0): 0 and -0 send +1, NaN sends 0.  A warp takes 1024
+// consecutive entries as 8 rounds of 32 lanes x float4; four __ballot_sync
+// calls per round give the sign of entry 4*lane+j in bit lane of mask j, and
+// a bit interleave turns the four masks into the round's four LSB-first words.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t spread8(uint32_t x) {  // bit i -> bit 4i
+  x = (x | (x << 12)) & 0x000F000Fu;
+  x = (x | (x << 6)) & 0x03030303u;
+  x = (x | (x << 3)) & 0x11111111u;
+  return x;
+}
+
+__global__ void __launch_bounds__(kThreads)
+k_pack(const float* __restrict__ U, int64_t u_stride, int64_t d, uint8_t* __restrict__ out,
+       int64_t out_stride) {
+  const int w = blockIdx.y;
+  U += (int64_t)w * u_stride;
+  out += (int64_t)w * out_stride;
+  const int lane = threadIdx.x & 31;
+  const int64_t warp0 = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * kThreads) >> 5;
+  const int64_t nchunks = (d + 1023) >> 10;
+  const int64_t nb = (d + 7) >> 3;
+  const int k = lane & 3;
+  for (int64_t c = warp0; c < nchunks; c += nwarps) {
+    uint32_t mine = 0;
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+      const int64_t e = c * 1024 + it * 128 + lane * 4;
+      bool b0, b1, b2, b3;
+      if (e + 3 < d) {
+        const float4 v = ld4(U + e);
+        b0 = v.x >= 0.f; b1 = v.y >= 0.f; b2 = v.z >= 0.f; b3 = v.w >= 0.f;
+      } else {
+        b0 = (e < d) && (U[e] >= 0.f);
+        b1 = (e + 1 < d) && (U[e + 1] >= 0.f);
+        b2 = (e + 2 < d) && (U[e + 2] >= 0.f);
+        b3 = (e + 3 < d) && (U[e + 3] >= 0.f);
+      }
+      const uint32_t m0 = __ballot_sync(0xffffffffu, b0);
+      const uint32_t m1 = __ballot_sync(0xffffffffu, b1);
+      const uint32_t m2 = __ballot_sync(0xffffffffu, b2);
+      const uint32_t m3 = __ballot_sync(0xffffffffu, b3);
+      const int sh = 8 * k;
+      const uint32_t word = spread8((m0 >> sh) & 0xFFu) | (spread8((m1 >> sh) & 0xFFu) << 1) |
+                            (spread8((m2 >> sh) & 0xFFu) << 2) | (spread8((m3 >> sh) & 0xFFu) << 3);
+      if ((lane >> 2) == it) mine = word;
+    }
+    const int64_t byte0 = (c * 32 + lane) * 4;
+    if (byte0 + 4 <= nb) {
+      *reinterpret_cast<uint32_t*>(out + byte0) = mine;
+    } else {
+      for (int t = 0; t < 4; ++t)
+        if (byte0 + t < nb) out[byte0 + t] = (uint8_t)(mine >> (8 * t));
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Majority vote ([paper] Algorithm 2: integer SUM of the signs then sign();
+// [blog]: ties give 0, sums lie in [-M, M]).  A block takes 1024 entries:
+// it stages the M workers' 128-byte slices in shared memory with 16-byte
+// loads, then each thread counts the +1 votes of 4 consecutive entries with
+// byte-lane counters (nibble * 0x00204081 & 0x01010101 spreads 4 bits into
+// 4 bytes) and writes 4 sums and 4 majority signs with vector stores.
+// ---------------------------------------------------------------------------
+constexpr int kVoteTile = 1024;
+
+struct BitsSrc {
+  const uint8_t* base;  // worker m at base + m*stride when ptrs == nullptr
+  int64_t stride;
+  const WorkerPtrs* ptrs;
+};
+
+__device__ __forceinline__ void count4(const uint32_t* sw, int M, int wi, int shift, int& c0,
+                                       int& c1, int& c2, int& c3) {
+  c0 = c1 = c2 = c3 = 0;
+  int m = 0;
+  while (m < M) {
+    const int end = min(M, m + 255);
+    uint32_t acc = 0;
+    for (; m < end; ++m) {
+      const uint32_t nib = (sw[m * 32 + wi] >> shift) & 0xFu;
+      acc += (nib * 0x00204081u) & 0x01010101u;
+    }
+    c0 += acc & 0xFF; c1 += (acc >> 8) & 0xFF; c2 += (acc >> 16) & 0xFF; c3 += acc >> 24;
+  }
+}
+
+__device__ __forceinline__ int sgn(int s) { return (s > 0) - (s < 0); }
+
+// MODE 0: API vote (sums + majority); 1: fused update of W; 2: write D = majority.
+template <int MODE, bool ACC8>
+__global__ void __launch_bounds__(kThreads)
+k_vote(WorkerPtrs signs, const uint8_t* __restrict__ bits, int64_t bits_stride, int M, int64_t d,
+       void* __restrict__ sums, int8_t* __restrict__ maj, float* __restrict__ W, float eta,
+       float* __restrict__ D, const int* __restrict__ status) {
+  extern __shared__ uint32_t sw[];  // [M][32]
+  if (MODE == 1 && status != nullptr && (status[0] | status[1]) != 0) return;  // keep W on error
+  const int64_t n_full = d / kVoteTile;
+  for (int64_t t = blockIdx.x; t < n_full; t += gridDim.x) {
+    for (int idx = threadIdx.x; idx < M * 8; idx += kThreads) {
+      const int m = idx >> 3, v = idx & 7;
+      const uint8_t* src = (MODE == 0) ? reinterpret_cast<const uint8_t*>(signs.p[m]) : bits + (int64_t)m * bits_stride;
+      const uint4 x = reinterpret_cast<const uint4*>(src + t * 128)[v];
+      reinterpret_cast<uint4*>(sw + m * 32)[v] = x;
+    }
+    __syncthreads();
+    const int wi = threadIdx.x >> 3, shift = (threadIdx.x & 7) * 4;
+    int c0, c1, c2, c3;
+    count4(sw, M, wi, shift, c0, c1, c2, c3);
+    const int s0 = 2 * c0 - M, s1 = 2 * c1 - M, s2 = 2 * c2 - M, s3 = 2 * c3 - M;
+    const int64_t e = t * kVoteTile + threadIdx.x * 4;
+    if (MODE == 0) {
+      if (sums != nullptr) {
+        if (ACC8) {
+          char4 v = make_char4((signed char)s0, (signed char)s1, (signed char)s2, (signed char)s3);
+          *reinterpret_cast<char4*>(reinterpret_cast<int8_t*>(sums) + e) = v;
+        } else {
+          *reinterpret_cast<int4*>(reinterpret_cast<int32_t*>(sums) + e) = make_int4(s0, s1, s2, s3);
+        }
+      }
+      if (maj != nullptr)
+        *reinterpret_cast<char4*>(maj + e) =
+            make_char4((signed char)sgn(s0), (signed char)sgn(s1), (signed char)sgn(s2), (signed char)sgn(s3));
+    } else if (MODE == 1) {
+      float4 w = ld4(W + e);
+      w.x = fmaf(-eta, (float)sgn(s0), w.x);
+      w.y = fmaf(-eta, (float)sgn(s1), w.y);
+      w.z = fmaf(-eta, (float)sgn(s2), w.z);
+      w.w = fmaf(-eta, (float)sgn(s3), w.w);
+      st4(W + e, w);
+    } else {
+      st4(D + e, make_float4((float)sgn(s0), (float)sgn(s1), (float)sgn(s2), (float)sgn(s3)));
+    }
+    __syncthreads();
+  }
+  // ragged tail (< 1024 entries): byte loads, one entry per thread
+  if (blockIdx.x == gridDim.x - 1) {
+    for (int64_t e = n_full * kVoteTile + threadIdx.x; e < d; e += kThreads) {
+      int c = 0;
+      for (int m = 0; m < M; ++m) {
+        const uint8_t* src = (MODE == 0) ? reinterpret_cast<const uint8_t*>(signs.p[m]) : bits + (int64_t)m * bits_stride;
+        c += (src[e >> 3] >> (e & 7)) & 1;
+      }
+      const int s = 2 * c - M;
+      if (MODE == 0) {
+        if (sums != nullptr) {
+          if (ACC8) reinterpret_cast<int8_t*>(sums)[e] = (int8_t)s;
+          else reinterpret_cast<int32_t*>(sums)[e] = s;
+        }
+        if (maj != nullptr) maj[e] = (int8_t)sgn(s);
+      } else if (MODE == 1) {
+        W[e] = fmaf(-eta, (float)sgn(s), W[e]);
+      } else {
+        D[e] = (float)sgn(s);
+      }
+    }
+  }
+}
+
+// W <- fl32(W - eta D), one rounding ([paper] Algorithm 1/2 update).
+__global__ void __launch_bounds__(kThreads)
+k_update(float* __restrict__ W, const float* __restrict__ D, int64_t d, float eta,
+         const int* __restrict__ status) {
+  if (status != nullptr && (status[0] | status[1]) != 0) return;  // keep W on error
+  const int64_t n4 = d >> 2;
+  const int64_t stride = (int64_t)gridDim.x * kThreads;
+  for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < n4; i += stride) {
+    float4 w = ld4(W + 4 * i);
+    const float4 dd = ld4(D + 4 * i);
+    w.x = fmaf(-eta, dd.x, w.x);
+    w.y = fmaf(-eta, dd.y, w.y);
+    w.z = fmaf(-eta, dd.z, w.z);
+    w.w = fmaf(-eta, dd.w, w.w);
+    st4(W + 4 * i, w);
+  }
+  if (blockIdx.x == 0)
+    for (int64_t e = 4 * n4 + threadIdx.x; e < d; e += kThreads) W[e] = fmaf(-eta, D[e], W[e]);
+}
+
+int g_num_sms = 0;
+int num_sms() {
+  if (g_num_sms == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (g_num_sms <= 0) g_num_sms = 148;
+  }
+  return g_num_sms;
+}
+
+int stream_grid(int64_t work_items, int per_sm) {
+  const int64_t cap = (int64_t)num_sms() * per_sm;
+  if (work_items < 1) return 1;
+  return (int)(work_items < cap ? work_items : cap);
+}
+
+}  // namespace
+
+// ---- launch wrappers --------------------------------------------------------
+
+void launch_momentum(cudaStream_t s, const WorkerPtrs& G, const float* W, float* Mom, int64_t d,
+                     int M, float beta, float lambda, void* X, int x_bf16, const Chunk* chunks,
+                     int n_chunks, const MatInfo* mats, const GroupInfo* groups, float* partials) {
+  if (n_chunks <= 0) return;
+  count_launch();
+  k_momentum<true><<<n_chunks, kThreads, 0, s>>>(G, W, Mom, d, M, beta, lambda, X, x_bf16, chunks,
+                                                 mats, groups, partials);
+}
+
+void launch_stage(cudaStream_t s, const WorkerPtrs& in, int M, void* X, int x_bf16,
+                  const Chunk* chunks, int n_chunks, const MatInfo* mats, const GroupInfo* groups,
+                  float* partials) {
+  if (n_chunks <= 0) return;
+  count_launch();
+  k_momentum<false><<<n_chunks, kThreads, 0, s>>>(in, nullptr, nullptr, 0, M, 0.f, 0.f, X, x_bf16,
+                                                  chunks, mats, groups, partials);
+}
+
+void launch_fro_finalize(cudaStream_t s, int n_probs, int n_mats, int M, const float* partials,
+                         const int* mat_chunk0, const int* mat_nchunks, int use_for_scale,
+                         float eps, int quintic, float a, float b, float c, float* scale,
+                         float2* coef_apply, float2* coef_square, int* status) {
+  count_launch();
+  k_fro_finalize<<<n_probs, kThreads, 0, s>>>(n_mats, M, partials, mat_chunk0, mat_nchunks,
+                                              use_for_scale, eps, quintic, a, b, c, scale,
+                                              coef_apply, coef_square, status);
+}
+
+void launch_pi_init(cudaStream_t s, int n_probs, const int64_t* uoff, const int* prob_g, float* u) {
+  count_launch();
+  k_pi_init<<<n_probs, kThreads, 0, s>>>(uoff, prob_g, u);
+}
+
+void launch_pi_matvec(cudaStream_t s, const ProbRows* rows, int n_rows, const void* A, int a_bf16,
+                      const int64_t* prob_a_off, const int* prob_g, const int* prob_gld,
+                      const int64_t* uoff, const float* u, float* y) {
+  count_launch();
+  if (a_bf16)
+    k_pi_matvec<true><<<n_rows, kThreads, 0, s>>>(rows, A, prob_a_off, prob_g, prob_gld, uoff, u, y);
+  else
+    k_pi_matvec<false><<<n_rows, kThreads, 0, s>>>(rows, A, prob_a_off, prob_g, prob_gld, uoff, u, y);
+}
+
+void launch_pi_normalize(cudaStream_t s, int n_probs, const int64_t* uoff, const int* prob_g,
+                         const float* y, float* u) {
+  count_launch();
+  k_pi_normalize<<<n_probs, kThreads, 0, s>>>(uoff, prob_g, y, u);
+}
+
+void launch_pi_finalize(cudaStream_t s, int n_probs, const int64_t* uoff, const int* prob_g,
+                        const float* u, const float* y, float eps, int quintic, float a, float b,
+                        float c, float* scale, float2* coef_apply, float2* coef_square, int* status) {
+  count_launch();
+  k_pi_finalize<<<n_probs, kThreads, 0, s>>>(uoff, prob_g, u, y, eps, quintic, a, b, c, scale,
+                                             coef_apply, coef_square, status);
+}
+
+void launch_scale_flat(cudaStream_t s, const WorkerPtrs& in, int M, float* out, int64_t out_stride,
+                       const Chunk* chunks, int n_chunks, const MatInfo* mats, int n_mats,
+                       const float* scale, float eps) {
+  if (n_chunks <= 0) return;
+  count_launch();
+  dim3 grid(n_chunks, M);
+  k_scale_flat<<<grid, kThreads, 0, s>>>(in, out, out_stride, chunks, mats, n_mats, scale, eps);
+}
+
+void launch_pack(cudaStream_t s, const float* U, int64_t u_stride, int64_t d, uint8_t* out,
+                 int64_t out_stride, int M) {
+  if (d <= 0) return;
+  count_launch();
+  const int64_t warps = (d + 1023) / 1024;
+  const int blocks = stream_grid((warps + 7) / 8, 16);
+  dim3 grid(blocks, M);
+  k_pack<<<grid, kThreads, 0, s>>>(U, u_stride, d, out, out_stride);
+}
+
+void launch_vote(cudaStream_t s, const WorkerPtrs& signs, int M, int64_t d, void* sums, int acc8,
+                 int8_t* majority) {
+  if (d <= 0) return;
+  count_launch();
+  const int blocks = stream_grid(d / kVoteTile + 1, 8);
+  const size_t smem = (size_t)M * 32 * 4;
+  if (acc8)
+    k_vote<0, true><<<blocks, kThreads, smem, s>>>(signs, nullptr, 0, M, d, sums, majority, nullptr,
+                                                   0.f, nullptr, nullptr);
+  else
+    k_vote<0, false><<<blocks, kThreads, smem, s>>>(signs, nullptr, 0, M, d, sums, majority, nullptr,
+                                                    0.f, nullptr, nullptr);
+}
+
+void launch_vote_update(cudaStream_t s, const uint8_t* bits, int64_t bits_stride, int M, int64_t d,
+                        float* W, float eta, const int* status) {
+  if (d <= 0) return;
+  count_launch();
+  const int blocks = stream_grid(d / kVoteTile + 1, 8);
+  const size_t smem = (size_t)M * 32 * 4;
+  WorkerPtrs none{};
+  k_vote<1, false><<<blocks, kThreads, smem, s>>>(none, bits, bits_stride, M, d, nullptr, nullptr, W,
+                                                  eta, nullptr, status);
+}
+
+void launch_vote_major(cudaStream_t s, const uint8_t* bits, int64_t bits_stride, int M, int64_t d,
+                       float* D) {
+  if (d <= 0) return;
+  count_launch();
+  const int blocks = stream_grid(d / kVoteTile + 1, 8);
+  const size_t smem = (size_t)M * 32 * 4;
+  WorkerPtrs none{};
+  k_vote<2, false><<<blocks, kThreads, smem, s>>>(none, bits, bits_stride, M, d, nullptr, nullptr,
+                                                  nullptr, 0.f, D, nullptr);
+}
+
+void launch_update(cudaStream_t s, float* W, const float* D, int64_t d, float eta,
+                   const int* status) {
+  if (d <= 0) return;
+  count_launch();
+  const int blocks = stream_grid((d / 4 + kThreads - 1) / kThreads + 1, 8);
+  k_update<<<blocks, kThreads, 0, s>>>(W, D, d, eta, status);
+}
+
+}  // namespace sm

@@ -1,0 +1,197 @@
+// plan.cpp -- host planning for a Sign-Muon handle (see plan.h).
+#include "plan.h"
+
+#include <algorithm>
+#include <climits>
+#include <map>
+#include <utility>
+
+#include "../../include/signmuon.h"
+
+namespace sm {
+
+namespace {
+
+int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
+
+// Output tile width for the tensor-core kernel: wider tiles keep shared
+// memory below its bandwidth limit (N=256 reads 96 B/clk of operands, N=64
+// 192 B/clk), narrower ones waste less on ragged edges.
+int pick_bn(int n) {
+  const int cand[3] = {256, 128, 64};
+  const double speed[3] = {1.0, 0.9, 0.6};
+  int best = 256;
+  double best_eff = -1.0;
+  for (int i = 0; i < 3; ++i) {
+    const int64_t tiles = (n + cand[i] - 1) / cand[i];
+    const double eff = (double)n / (double)(tiles * cand[i]) * speed[i];
+    if (eff > best_eff + 1e-9) {
+      best_eff = eff;
+      best = cand[i];
+    }
+  }
+  return best;
+}
+
+void build_tiles(Plan& p, int op, int nw, TileTable* tt) {
+  std::vector<TileGroup> v;
+  for (int gidx = 0; gidx < (int)p.groups.size(); ++gidx) {
+    const GroupInfo& g = p.groups[gidx];
+    TileGroup t{};
+    t.group = gidx;
+    if (op == OP_GRAM) {
+      t.Mdim = t.Ndim = g.g;
+      t.Kdim = g.wide ? g.cols : g.rows;
+    } else if (op == OP_SQUARE) {
+      t.Mdim = t.Ndim = t.Kdim = g.g;
+    } else {
+      t.Mdim = g.rows;
+      t.Ndim = g.cols;
+      t.Kdim = g.g;
+    }
+    t.BN = p.fp32 ? 128 : pick_bn(t.Ndim);
+    t.tiles_m = (t.Mdim + 127) / 128;
+    t.tiles_n = (t.Ndim + t.BN - 1) / t.BN;
+    t.batch = nw * g.count;
+    v.push_back(t);
+  }
+  // longest tiles first: a better static round-robin balance
+  std::stable_sort(v.begin(), v.end(), [](const TileGroup& x, const TileGroup& y) { return x.Kdim > y.Kdim; });
+  int start = 0;
+  for (auto& t : v) {
+    t.tile_start = start;
+    start += t.tiles_m * t.tiles_n * t.batch;
+  }
+  tt->groups = v;
+  tt->total = start;
+}
+
+}  // namespace
+
+int make_plan(const int64_t* shapes, int n_mats, int M, int K, int scale, int P, unsigned flags,
+              Plan* plan, std::string* err) {
+  if (shapes == nullptr || n_mats < 1) { *err = "need at least one matrix shape"; return SIGNMUON_E_INVALID; }
+  if (M < 1 || M > kMaxWorkers) { *err = "M must be in [1, 256]"; return SIGNMUON_E_INVALID; }
+  if ((flags & SIGNMUON_ACC_INT8) && M > 127) { *err = "int8 vote sums overflow for M > 127"; return SIGNMUON_E_OVERFLOW; }
+  if (K < 0) { *err = "K must be >= 0"; return SIGNMUON_E_INVALID; }
+  if (scale != SIGNMUON_SCALE_FRO && scale != SIGNMUON_SCALE_SPECTRAL) { *err = "unknown scale"; return SIGNMUON_E_INVALID; }
+  if (scale == SIGNMUON_SCALE_SPECTRAL && P < 1) { *err = "spectral scaling needs P >= 1"; return SIGNMUON_E_INVALID; }
+  Plan& p = *plan;
+  p = Plan();
+  p.M = M;
+  p.n_mats = n_mats;
+  p.fp32 = (flags & SIGNMUON_NS_FP32) != 0;
+  p.quintic = (flags & SIGNMUON_NS_QUINTIC) != 0;
+  std::map<std::pair<int64_t, int64_t>, int> gid;
+  int64_t off = 0;
+  for (int i = 0; i < n_mats; ++i) {
+    const int64_t r = shapes[2 * i], c = shapes[2 * i + 1];
+    if (r < 1 || c < 1) { *err = "matrix " + std::to_string(i) + " has a non-positive dimension"; return SIGNMUON_E_INVALID; }
+    if (r * c > (int64_t)INT_MAX) { *err = "matrix " + std::to_string(i) + " has more than 2^31-1 entries"; return SIGNMUON_E_INVALID; }
+    auto key = std::make_pair(r, c);
+    auto it = gid.find(key);
+    int g;
+    if (it == gid.end()) {
+      g = (int)p.groups.size();
+      gid[key] = g;
+      GroupInfo gi{};
+      gi.rows = (int)r;
+      gi.cols = (int)c;
+      gi.ld = (int)round_up(c, 8);
+      gi.wide = r <= c ? 1 : 0;
+      gi.g = (int)std::min(r, c);
+      gi.gld = (int)round_up(gi.g, 8);
+      gi.count = 0;
+      p.groups.push_back(gi);
+    } else {
+      g = it->second;
+    }
+    MatInfo mi{};
+    mi.off = off;
+    mi.rows = (int)r;
+    mi.cols = (int)c;
+    mi.group = g;
+    mi.q = p.groups[g].count++;
+    p.mats.push_back(mi);
+    p.mat_off.push_back(off);
+    off += r * c;
+  }
+  p.d = off;
+  p.dpad = round_up(p.d, 64);
+  p.nb = (p.d + 7) / 8;
+  p.nb_pad = round_up(p.nb, 16);
+  // group -> matrices, group bases (every base a multiple of 8 elements)
+  int first = 0;
+  for (auto& g : p.groups) {
+    g.first = first;
+    first += g.count;
+  }
+  p.group_mats.assign(n_mats, 0);
+  for (int i = 0; i < n_mats; ++i) {
+    const MatInfo& mi = p.mats[i];
+    p.group_mats[p.groups[mi.group].first + mi.q] = i;
+  }
+  int64_t xb = 0, ab = 0;
+  for (auto& g : p.groups) {
+    g.x_base = xb;
+    g.a_base = ab;
+    xb += (int64_t)M * g.count * g.rows * g.ld;
+    ab += (int64_t)M * g.count * g.g * g.gld;
+  }
+  p.x_elems = xb;
+  p.a_elems = ab;
+  // elementwise chunks: pieces of <= kChunk elements, never crossing a matrix
+  p.mat_chunk0.resize(n_mats);
+  p.mat_nchunks.resize(n_mats);
+  for (int i = 0; i < n_mats; ++i) {
+    const int64_t n = (int64_t)p.mats[i].rows * p.mats[i].cols;
+    p.mat_chunk0[i] = (int)p.chunks.size();
+    for (int64_t s = 0; s < n; s += kChunk) {
+      Chunk c{};
+      c.mat = i;
+      c.start = s;
+      c.len = (int)std::min<int64_t>(kChunk, n - s);
+      p.chunks.push_back(c);
+    }
+    p.mat_nchunks[i] = (int)p.chunks.size() - p.mat_chunk0[i];
+  }
+  for (int op = 0; op < 3; ++op) {
+    build_tiles(p, op, M, &p.tiles[op][0]);
+    build_tiles(p, op, 1, &p.tiles[op][1]);
+  }
+  // power iteration tables (worker-major problems so worker 0 is a prefix)
+  int64_t u = 0;
+  for (int w = 0; w < M; ++w) {
+    for (int i = 0; i < n_mats; ++i) {
+      const MatInfo& mi = p.mats[i];
+      const GroupInfo& g = p.groups[mi.group];
+      const int pid = w * n_mats + i;
+      p.uoff.push_back(u);
+      p.prob_g.push_back(g.g);
+      p.prob_gld.push_back(g.gld);
+      p.prob_aoff.push_back(g.a_base + (int64_t)(w * g.count + mi.q) * g.g * g.gld);
+      u += g.g;
+      for (int r0 = 0; r0 < g.g; r0 += kPiRows) p.pi_rows.push_back(ProbRows{pid, r0});
+    }
+    if (w == 0) p.n_pi_rows_one = (int)p.pi_rows.size();
+  }
+  p.u_elems = u;
+  const int64_t esz = p.fp32 ? 4 : 2;
+  int64_t bytes = 0;
+  if (!(flags & SIGNMUON_VOTE_ONLY)) {
+    bytes += 2 * (int64_t)M * p.dpad * 4;                 // momentum, U
+    bytes += 2 * p.x_elems * esz;                         // X ping/pong
+    bytes += p.a_elems * esz * (p.quintic ? 2 : 1);       // A (and B)
+    bytes += (int64_t)M * p.nb_pad;                       // packed bits
+    bytes += p.dpad * 4;                                  // D
+    bytes += (int64_t)p.chunks.size() * M * 4;            // norm partials
+    bytes += (int64_t)M * n_mats * (4 + 8 + 8);           // scales, coefficients
+    bytes += 2 * p.u_elems * 4;                           // power-iteration vectors
+    bytes += (int64_t)p.groups.size() * 4 * 128;          // tensor maps
+  }
+  p.device_bytes = bytes;
+  (void)K;
+  return SIGNMUON_OK;
+}
+
+}  // namespace sm

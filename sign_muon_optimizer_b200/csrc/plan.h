@@ -1,0 +1,50 @@
+// plan.h -- host-side planning of one Sign-Muon handle: shape groups, chunk
+// lists, grouped GEMM tile lists, power-iteration row blocks and buffer
+// sizes.  Pure host code (no CUDA calls), so that it can be checked without a
+// GPU through signmuon_plan().
+#pragma once
+#include <cstdint>
+#include <string>
+#include <vector>
+
+#include "common.cuh"
+
+namespace sm {
+
+struct TileTable {
+  std::vector<TileGroup> groups;
+  int total = 0;
+};
+
+struct Plan {
+  int M = 0, n_mats = 0;
+  bool fp32 = false, quintic = false;
+  int64_t d = 0;        // parameters
+  int64_t dpad = 0;     // stride of the library's flat per-worker vectors
+  int64_t nb = 0;       // ceil(d/8) packed bytes per worker
+  int64_t nb_pad = 0;   // stride of the library's packed buffers (16-byte multiple)
+  std::vector<MatInfo> mats;
+  std::vector<GroupInfo> groups;
+  std::vector<int> group_mats;
+  std::vector<int64_t> mat_off;
+  std::vector<Chunk> chunks;
+  std::vector<int> mat_chunk0, mat_nchunks;
+  int64_t x_elems = 0;  // elements of one grouped X buffer (all workers)
+  int64_t a_elems = 0;  // elements of the grouped A (and B) buffer
+  // tile lists: [op][0 = all M workers, 1 = one worker]
+  TileTable tiles[3][2];
+  // power iteration: problems p = worker*n_mats + mat (worker-major)
+  std::vector<ProbRows> pi_rows;
+  int n_pi_rows_one = 0;  // rows blocks of worker 0 (prefix)
+  std::vector<int64_t> uoff;
+  std::vector<int> prob_g, prob_gld;
+  std::vector<int64_t> prob_aoff;
+  int64_t u_elems = 0;
+  int64_t device_bytes = 0;  // everything the handle allocates
+};
+
+// Validates and plans; returns a SIGNMUON_* status and fills *err on failure.
+int make_plan(const int64_t* shapes, int n_mats, int M, int K, int scale, int P, unsigned flags,
+              Plan* plan, std::string* err);
+
+}  // namespace sm

@@ -1,0 +1,723 @@
+// signmuon_api.cu -- the C ABI of libsignmuon.so (declared in
+// include/signmuon.h): handle life cycle, device buffers, TMA tensor maps and
+// the kernel sequence of one Sign-Muon step.
+//
+// Step sequence on the handle's stream ([paper] "SignMuon: 通信高效的分布式Muon优化"
+// Algorithm 2; the vote of [blog] "SignMuon: Matrix Directions, Majority
+// Votes, and the Actual Bytes Sent"):
+//   momentum pass -> Frobenius partials -> NS GEMMs (GRAM [-> power iteration]
+//   [-> SQUARE] -> APPLY) x K -> one-bit pack -> vote fused with the update,
+//   or vote -> stage -> NS x K -> update for the post-vote polar step.
+#include <cuda.h>
+
+#include <atomic>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <string>
+#include <vector>
+
+#include "../../include/signmuon.h"
+#include "common.cuh"
+#include "plan.h"
+
+namespace sm {
+static std::atomic<int64_t> g_launches{0};
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+}  // namespace sm
+
+using sm::Plan;
+
+struct signmuon_ctx {
+  Plan plan;
+  int M = 0, K = 0, scale = 0, P = 1;
+  float beta = 0.f, lambda = 0.f, eps = 0.f;
+  float ns_a = 1.5f, ns_b = -0.5f, ns_c = 0.f;
+  unsigned flags = 0;
+  cudaStream_t stream = nullptr;
+  int device = 0, n_sm = 148;
+  bool vote_only = false;
+  // device plan tables
+  sm::MatInfo* d_mats = nullptr;
+  sm::GroupInfo* d_groups = nullptr;
+  int* d_group_mats = nullptr;
+  int64_t* d_mat_off = nullptr;
+  sm::Chunk* d_chunks = nullptr;
+  int* d_mat_chunk0 = nullptr;
+  int* d_mat_nchunks = nullptr;
+  sm::TileGroup* d_tiles[3][2] = {{nullptr}};
+  sm::ProbRows* d_pi_rows = nullptr;
+  int64_t* d_uoff = nullptr;
+  int* d_prob_g = nullptr;
+  int* d_prob_gld = nullptr;
+  int64_t* d_prob_aoff = nullptr;
+  void* d_maps = nullptr;
+  // device state / workspace
+  float* Mom = nullptr;
+  void* X[2] = {nullptr, nullptr};
+  void* A = nullptr;
+  void* B = nullptr;
+  float* U = nullptr;
+  uint8_t* bits = nullptr;
+  float* D = nullptr;
+  float* partials = nullptr;
+  float* scale_v = nullptr;
+  float2* coef_apply = nullptr;
+  float2* coef_square = nullptr;
+  float* pi_u = nullptr;
+  float* pi_y = nullptr;
+  int* status = nullptr;        // [0] non-finite flag, [1] kernel error code
+  int* h_status = nullptr;      // pinned mirror
+  bool pending = false;         // an async step's status not yet read
+  // step_host staging
+  float* hw_W = nullptr;
+  float* hw_G = nullptr;
+  std::vector<void*> allocs;
+  int64_t bytes = 0;
+  std::string err;
+  // optional per-kernel timing: event pairs recorded around each launch
+  bool prof = false;
+  std::vector<cudaEvent_t> ev_pool;
+  size_t ev_used = 0;
+  std::vector<int> ev_kind;           // kind of each recorded pair
+  double prof_ms[SIGNMUON_PROF_KINDS] = {0};
+  int64_t prof_n[SIGNMUON_PROF_KINDS] = {0};
+};
+
+namespace {
+
+std::string g_noh_err;  // errors raised before a handle exists
+
+int fail(signmuon_t h, int code, const std::string& msg) {
+  if (h) h->err = msg;
+  else g_noh_err = msg;
+  return code;
+}
+
+#define CK(h, call)                                                                   \
+  do {                                                                                \
+    cudaError_t e_ = (call);                                                          \
+    if (e_ != cudaSuccess) {                                                          \
+      cudaGetLastError();                                                             \
+      return fail((h), e_ == cudaErrorMemoryAllocation ? SIGNMUON_E_NOMEM : SIGNMUON_E_CUDA, \
+                  std::string(#call) + ": " + cudaGetErrorString(e_));                \
+    }                                                                                 \
+  } while (0)
+
+template <typename T>
+int dalloc(signmuon_t h, T** p, int64_t count) {
+  *p = nullptr;
+  if (count <= 0) count = 1;
+  void* q = nullptr;
+  cudaError_t e = cudaMalloc(&q, (size_t)count * sizeof(T));
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(h, SIGNMUON_E_NOMEM, std::string("cudaMalloc: ") + cudaGetErrorString(e));
+  }
+  h->allocs.push_back(q);
+  h->bytes += count * (int64_t)sizeof(T);
+  *p = reinterpret_cast<T*>(q);
+  return SIGNMUON_OK;
+}
+
+template <typename T>
+int upload(signmuon_t h, T** dst, const std::vector<T>& src) {
+  int rc = dalloc(h, dst, (int64_t)src.size());
+  if (rc) return rc;
+  if (!src.empty()) CK(h, cudaMemcpy(*dst, src.data(), src.size() * sizeof(T), cudaMemcpyHostToDevice));
+  return SIGNMUON_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  }
+  return fn;
+}
+
+// 3-D bf16 tensor map over `batch` matrices of rows x cols (row stride ld),
+// 64x64 boxes with the 128-byte swizzle; out-of-range boxes read zeros.
+int encode_map(signmuon_t h, CUtensorMap* m, void* base, int cols, int rows, int ld, int batch) {
+  EncodeTiledFn fn = get_encode();
+  if (!fn) return fail(h, SIGNMUON_E_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)batch};
+  cuuint64_t strides[2] = {(cuuint64_t)ld * 2, (cuuint64_t)rows * ld * 2};
+  cuuint32_t box[3] = {64, 64, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(h, SIGNMUON_E_CUDA, "cuTensorMapEncodeTiled failed: " + std::to_string((int)r));
+  return SIGNMUON_OK;
+}
+
+sm::WorkerPtrs worker_ptrs(const float* const* p, int M) {
+  sm::WorkerPtrs w{};
+  for (int m = 0; m < M; ++m) w.p[m] = p[m];
+  return w;
+}
+
+sm::WorkerPtrs strided_ptrs(const float* base, int64_t stride, int M) {
+  sm::WorkerPtrs w{};
+  for (int m = 0; m < M; ++m) w.p[m] = base + (int64_t)m * stride;
+  return w;
+}
+
+// Record the event pair of one kernel launch of `kind` (no-op unless timing).
+struct ProfScope {
+  signmuon_t h;
+  int kind;
+  cudaEvent_t e1 = nullptr;
+  ProfScope(signmuon_t h_, int kind_) : h(h_), kind(kind_) {
+    if (!h->prof) return;
+    while (h->ev_pool.size() < h->ev_used + 2) {
+      cudaEvent_t e;
+      cudaEventCreate(&e);
+      h->ev_pool.push_back(e);
+    }
+    cudaEventRecord(h->ev_pool[h->ev_used], h->stream);
+    e1 = h->ev_pool[h->ev_used + 1];
+    h->ev_used += 2;
+    h->ev_kind.push_back(kind);
+  }
+  ~ProfScope() {
+    if (e1) cudaEventRecord(e1, h->stream);
+  }
+};
+
+void prof_collect(signmuon_t h) {
+  if (h->ev_used == 0) return;
+  cudaStreamSynchronize(h->stream);
+  for (size_t i = 0; i < h->ev_kind.size(); ++i) {
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, h->ev_pool[2 * i], h->ev_pool[2 * i + 1]) == cudaSuccess) {
+      h->prof_ms[h->ev_kind[i]] += ms;
+      h->prof_n[h->ev_kind[i]] += 1;
+    }
+  }
+  cudaGetLastError();
+  h->ev_used = 0;
+  h->ev_kind.clear();
+}
+
+// ---------------------------------------------------------------------------
+// PolarNS for nw workers whose X~ (unscaled) is staged in X[0]; the Frobenius
+// scale (if used) is already final.  Writes U (fp32, flat) to out +
+// worker*out_stride.  kzero_in is the fp32 input used when K == 0.
+// ---------------------------------------------------------------------------
+void gemm(signmuon_t h, int op, int slot, int src, int nw, const float2* coef, float c0, float c1,
+          bool final_out, float* out, int64_t out_stride) {
+  const Plan& p = h->plan;
+  sm::GemmArgs a{};
+  a.tiles = h->d_tiles[op][slot];
+  a.n_tile_groups = (int)p.tiles[op][slot].groups.size();
+  a.total_tiles = p.tiles[op][slot].total;
+  a.groups = h->d_groups;
+  a.group_mats = h->d_group_mats;
+  a.mat_off = h->d_mat_off;
+  a.n_mats = p.n_mats;
+  a.op = op;
+  a.X_src = h->X[src];
+  a.X_dst = h->X[src ^ 1];
+  a.A = h->A;
+  a.B = h->B;
+  a.p_from_b = (op == sm::OP_APPLY && p.quintic) ? 1 : 0;
+  a.map_src = src;
+  a.map_dst = src ^ 1;
+  a.coef = coef;
+  a.c0 = c0;
+  a.c1 = c1;
+  a.out = out;
+  a.out_stride = out_stride;
+  a.final_out = final_out ? 1 : 0;
+  a.err = h->status + 1;
+  (void)nw;
+  ProfScope ps(h, nw == 1 ? 7 : 2);
+  if (p.fp32) sm::launch_gemm_simt(h->stream, a, 1);
+  else sm::launch_gemm_tc(h->stream, a, h->d_maps, h->n_sm);
+}
+
+void power_iteration(signmuon_t h, int nw) {
+  const Plan& p = h->plan;
+  const int nprob = nw * p.n_mats;
+  const int nrows = nw == 1 ? p.n_pi_rows_one : (int)p.pi_rows.size();
+  ProfScope ps(h, 3);
+  sm::launch_pi_init(h->stream, nprob, h->d_uoff, h->d_prob_g, h->pi_u);
+  for (int it = 0; it < h->P; ++it) {
+    sm::launch_pi_matvec(h->stream, h->d_pi_rows, nrows, h->A, p.fp32 ? 0 : 1, h->d_prob_aoff, h->d_prob_g,
+                         h->d_prob_gld, h->d_uoff, h->pi_u, h->pi_y);
+    sm::launch_pi_normalize(h->stream, nprob, h->d_uoff, h->d_prob_g, h->pi_y, h->pi_u);
+  }
+  sm::launch_pi_matvec(h->stream, h->d_pi_rows, nrows, h->A, p.fp32 ? 0 : 1, h->d_prob_aoff, h->d_prob_g,
+                       h->d_prob_gld, h->d_uoff, h->pi_u, h->pi_y);
+  sm::launch_pi_finalize(h->stream, nprob, h->d_uoff, h->d_prob_g, h->pi_u, h->pi_y, h->eps, p.quintic ? 1 : 0,
+                         h->ns_a, h->ns_b, h->ns_c, h->scale_v, h->coef_apply, h->coef_square, h->status);
+}
+
+void run_ns(signmuon_t h, int nw, const sm::WorkerPtrs& kzero_in, float* out, int64_t out_stride) {
+  const Plan& p = h->plan;
+  const int slot = nw == 1 ? 1 : 0;
+  const bool spectral = h->scale == SIGNMUON_SCALE_SPECTRAL;
+  if (h->K == 0) {
+    if (spectral) {
+      gemm(h, sm::OP_GRAM, slot, 0, nw, nullptr, 0.f, 0.f, false, nullptr, 0);
+      power_iteration(h, nw);
+    }
+    ProfScope ps(h, 9);
+    sm::launch_scale_flat(h->stream, kzero_in, nw, out, out_stride, h->d_chunks, (int)p.chunks.size(), h->d_mats,
+                          p.n_mats, h->scale_v, h->eps);
+    return;
+  }
+  int cur = 0;
+  for (int k = 0; k < h->K; ++k) {
+    gemm(h, sm::OP_GRAM, slot, cur, nw, nullptr, 0.f, 0.f, false, nullptr, 0);
+    if (k == 0 && spectral) power_iteration(h, nw);
+    if (p.quintic)
+      gemm(h, sm::OP_SQUARE, slot, cur, nw, k == 0 ? h->coef_square : nullptr, h->ns_b, h->ns_c, false, nullptr, 0);
+    const bool last = (k == h->K - 1);
+    gemm(h, sm::OP_APPLY, slot, cur, nw, k == 0 ? h->coef_apply : nullptr, h->ns_a, p.quintic ? 1.f : h->ns_b, last,
+         out, out_stride);
+    cur ^= 1;
+  }
+}
+
+void fro_finalize(signmuon_t h, int nw) {
+  const Plan& p = h->plan;
+  ProfScope ps(h, 1);
+  sm::launch_fro_finalize(h->stream, nw * p.n_mats, p.n_mats, nw, h->partials, h->d_mat_chunk0, h->d_mat_nchunks,
+                          h->scale == SIGNMUON_SCALE_FRO ? 1 : 0, h->eps, p.quintic ? 1 : 0, h->ns_a, h->ns_b,
+                          h->ns_c, h->scale_v, h->coef_apply, h->coef_square, h->status);
+}
+
+int finish(signmuon_t h, bool wait) {
+  CK(h, cudaMemcpyAsync(h->h_status, h->status, 2 * sizeof(int), cudaMemcpyDeviceToHost, h->stream));
+  CK(h, cudaGetLastError());
+  if (!wait) {
+    h->pending = true;
+    return SIGNMUON_OK;
+  }
+  CK(h, cudaStreamSynchronize(h->stream));
+  h->pending = false;
+  if (h->h_status[1] != 0) return fail(h, SIGNMUON_E_TIMEOUT, "a kernel's bounded wait expired");
+  if (h->h_status[0] != 0) return fail(h, SIGNMUON_E_NONFINITE, "a momentum norm is NaN or Inf; W was not updated");
+  return SIGNMUON_OK;
+}
+
+int check_handle(signmuon_t h, bool need_step) {
+  if (h == nullptr) return fail(nullptr, SIGNMUON_E_INVALID, "null handle");
+  if (need_step && h->vote_only) return fail(h, SIGNMUON_E_UNSUPPORTED, "handle was created with SIGNMUON_VOTE_ONLY");
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev != h->device) cudaSetDevice(h->device);
+  return SIGNMUON_OK;
+}
+
+}  // namespace
+
+// ===========================================================================
+// C ABI
+// ===========================================================================
+extern "C" {
+
+const char* signmuon_status_string(int s) {
+  switch (s) {
+    case SIGNMUON_OK: return "ok";
+    case SIGNMUON_E_INVALID: return "invalid argument";
+    case SIGNMUON_E_OVERFLOW: return "int8 accumulator overflow (M > 127)";
+    case SIGNMUON_E_NONFINITE: return "non-finite momentum norm";
+    case SIGNMUON_E_CUDA: return "CUDA error";
+    case SIGNMUON_E_NOMEM: return "out of device memory";
+    case SIGNMUON_E_TIMEOUT: return "kernel wait timed out";
+    case SIGNMUON_E_UNSUPPORTED: return "unsupported for this handle";
+    default: return "unknown status";
+  }
+}
+
+const char* signmuon_last_error(signmuon_t h) { return h ? h->err.c_str() : g_noh_err.c_str(); }
+
+int64_t signmuon_kernel_launches(void) { return sm::g_launches.load(); }
+
+static void fill_info(const Plan& p, int64_t* out, int n) {
+  const int64_t v[6] = {p.d, p.nb, p.device_bytes, (int64_t)p.groups.size(), p.M, p.n_mats};
+  for (int i = 0; i < n && i < 6; ++i) out[i] = v[i];
+}
+
+int signmuon_plan(const int64_t* shapes, int n_mats, int M, int K, int scale, int P, unsigned flags,
+                  int64_t* out, int n) {
+  Plan p;
+  std::string err;
+  const int rc = sm::make_plan(shapes, n_mats, M, K, scale, P, flags, &p, &err);
+  if (rc) return fail(nullptr, rc, err);
+  if (out) fill_info(p, out, n);
+  return SIGNMUON_OK;
+}
+
+void signmuon_destroy(signmuon_t h) {
+  if (!h) return;
+  cudaStreamSynchronize(h->stream);
+  for (cudaEvent_t e : h->ev_pool) cudaEventDestroy(e);
+  for (void* q : h->allocs) cudaFree(q);
+  if (h->h_status) cudaFreeHost(h->h_status);
+  delete h;
+}
+
+int signmuon_init(signmuon_t* out, const int64_t* shapes, int n_mats, int M, float beta, float lambda, int K,
+                  float eps, int scale, int P, unsigned flags, void* stream) {
+  if (out == nullptr) return fail(nullptr, SIGNMUON_E_INVALID, "null out-pointer");
+  *out = nullptr;
+  if (!(beta >= 0.f && beta < 1.f)) return fail(nullptr, SIGNMUON_E_INVALID, "beta must be in [0, 1)");
+  if (!(lambda >= 0.f)) return fail(nullptr, SIGNMUON_E_INVALID, "lambda must be >= 0");
+  if (!(eps > 0.f)) return fail(nullptr, SIGNMUON_E_INVALID, "eps must be > 0");
+  signmuon_t h = new (std::nothrow) signmuon_ctx();
+  if (!h) return fail(nullptr, SIGNMUON_E_NOMEM, "host allocation failed");
+  std::string err;
+  int rc = sm::make_plan(shapes, n_mats, M, K, scale, P, flags, &h->plan, &err);
+  if (rc) {
+    delete h;
+    return fail(nullptr, rc, err);
+  }
+  h->M = M; h->K = K; h->scale = scale; h->P = P;
+  h->beta = beta; h->lambda = lambda; h->eps = eps; h->flags = flags;
+  h->stream = reinterpret_cast<cudaStream_t>(stream);
+  h->vote_only = (flags & SIGNMUON_VOTE_ONLY) != 0;
+  if (flags & SIGNMUON_NS_QUINTIC) { h->ns_a = 15.f / 8.f; h->ns_b = -10.f / 8.f; h->ns_c = 3.f / 8.f; }
+  cudaError_t e = cudaGetDevice(&h->device);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&h->n_sm, cudaDevAttrMultiProcessorCount, h->device);
+  if (e == cudaSuccess) e = cudaMallocHost(&h->h_status, 2 * sizeof(int));
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    delete h;
+    return fail(nullptr, SIGNMUON_E_CUDA, std::string("CUDA unavailable: ") + cudaGetErrorString(e));
+  }
+  h->h_status[0] = h->h_status[1] = 0;
+  auto bail = [&](int code) {
+    g_noh_err = h->err;
+    signmuon_destroy(h);
+    return code;
+  };
+  if ((rc = dalloc(h, &h->status, 2))) return bail(rc);
+  if (cudaMemset(h->status, 0, 2 * sizeof(int)) != cudaSuccess) return bail(fail(h, SIGNMUON_E_CUDA, "memset"));
+  if (h->vote_only) {
+    *out = h;
+    return SIGNMUON_OK;
+  }
+  const Plan& p = h->plan;
+  if ((rc = upload(h, &h->d_mats, p.mats))) return bail(rc);
+  if ((rc = upload(h, &h->d_groups, p.groups))) return bail(rc);
+  if ((rc = upload(h, &h->d_group_mats, p.group_mats))) return bail(rc);
+  if ((rc = upload(h, &h->d_mat_off, p.mat_off))) return bail(rc);
+  if ((rc = upload(h, &h->d_chunks, p.chunks))) return bail(rc);
+  if ((rc = upload(h, &h->d_mat_chunk0, p.mat_chunk0))) return bail(rc);
+  if ((rc = upload(h, &h->d_mat_nchunks, p.mat_nchunks))) return bail(rc);
+  for (int op = 0; op < 3; ++op)
+    for (int s = 0; s < 2; ++s)
+      if ((rc = upload(h, &h->d_tiles[op][s], p.tiles[op][s].groups))) return bail(rc);
+  if ((rc = upload(h, &h->d_pi_rows, p.pi_rows))) return bail(rc);
+  if ((rc = upload(h, &h->d_uoff, p.uoff))) return bail(rc);
+  if ((rc = upload(h, &h->d_prob_g, p.prob_g))) return bail(rc);
+  if ((rc = upload(h, &h->d_prob_gld, p.prob_gld))) return bail(rc);
+  if ((rc = upload(h, &h->d_prob_aoff, p.prob_aoff))) return bail(rc);
+  const int64_t esz = p.fp32 ? 4 : 2;
+  if ((rc = dalloc(h, &h->Mom, (int64_t)M * p.dpad))) return bail(rc);
+  if ((rc = dalloc(h, &h->U, (int64_t)M * p.dpad))) return bail(rc);
+  for (int i = 0; i < 2; ++i) {
+    uint8_t* x = nullptr;
+    if ((rc = dalloc(h, &x, p.x_elems * esz))) return bail(rc);
+    h->X[i] = x;
+  }
+  {
+    uint8_t* x = nullptr;
+    if ((rc = dalloc(h, &x, p.a_elems * esz))) return bail(rc);
+    h->A = x;
+    if (p.quintic) {
+      if ((rc = dalloc(h, &x, p.a_elems * esz))) return bail(rc);
+      h->B = x;
+    } else {
+      h->B = h->A;
+    }
+  }
+  if ((rc = dalloc(h, &h->bits, (int64_t)M * p.nb_pad))) return bail(rc);
+  if ((rc = dalloc(h, &h->D, p.dpad))) return bail(rc);
+  if ((rc = dalloc(h, &h->partials, (int64_t)p.chunks.size() * M))) return bail(rc);
+  if ((rc = dalloc(h, &h->scale_v, (int64_t)M * p.n_mats))) return bail(rc);
+  if ((rc = dalloc(h, &h->coef_apply, (int64_t)M * p.n_mats))) return bail(rc);
+  if ((rc = dalloc(h, &h->coef_square, (int64_t)M * p.n_mats))) return bail(rc);
+  if ((rc = dalloc(h, &h->pi_u, p.u_elems))) return bail(rc);
+  if ((rc = dalloc(h, &h->pi_y, p.u_elems))) return bail(rc);
+  if (cudaMemset(h->Mom, 0, (size_t)M * p.dpad * 4) != cudaSuccess ||
+      cudaMemset(h->bits, 0, (size_t)M * p.nb_pad) != cudaSuccess ||
+      cudaMemset(h->scale_v, 0, (size_t)M * p.n_mats * 4) != cudaSuccess)
+    return bail(fail(h, SIGNMUON_E_CUDA, "memset"));
+  if (!p.fp32) {
+    std::vector<CUtensorMap> maps(p.groups.size() * 4);
+    for (size_t g = 0; g < p.groups.size(); ++g) {
+      const sm::GroupInfo& gi = p.groups[g];
+      const int batch = M * gi.count;
+      for (int i = 0; i < 2; ++i) {
+        void* xb = reinterpret_cast<__nv_bfloat16*>(h->X[i]) + gi.x_base;
+        if ((rc = encode_map(h, &maps[g * 4 + i], xb, gi.cols, gi.rows, gi.ld, batch))) return bail(rc);
+      }
+      void* ab = reinterpret_cast<__nv_bfloat16*>(h->A) + gi.a_base;
+      void* bb = reinterpret_cast<__nv_bfloat16*>(h->B) + gi.a_base;
+      if ((rc = encode_map(h, &maps[g * 4 + 2], ab, gi.g, gi.g, gi.gld, batch))) return bail(rc);
+      if ((rc = encode_map(h, &maps[g * 4 + 3], bb, gi.g, gi.g, gi.gld, batch))) return bail(rc);
+    }
+    uint8_t* m = nullptr;
+    if ((rc = dalloc(h, &m, (int64_t)(maps.size() * sizeof(CUtensorMap) + 128)))) return bail(rc);
+    h->d_maps = reinterpret_cast<void*>((reinterpret_cast<uintptr_t>(m) + 127) & ~(uintptr_t)127);
+    if (cudaMemcpy(h->d_maps, maps.data(), maps.size() * sizeof(CUtensorMap), cudaMemcpyHostToDevice) != cudaSuccess)
+      return bail(fail(h, SIGNMUON_E_CUDA, "tensor map upload"));
+  }
+  if (cudaDeviceSynchronize() != cudaSuccess) return bail(fail(h, SIGNMUON_E_CUDA, "init sync"));
+  *out = h;
+  return SIGNMUON_OK;
+}
+
+int signmuon_set_ns_coeffs(signmuon_t h, const float* c, int n) {
+  int rc = check_handle(h, false);
+  if (rc) return rc;
+  if (c == nullptr) return fail(h, SIGNMUON_E_INVALID, "null coefficients");
+  if (h->plan.quintic) {
+    if (n != 3) return fail(h, SIGNMUON_E_INVALID, "quintic NS takes 3 coefficients");
+    h->ns_a = c[0]; h->ns_b = c[1]; h->ns_c = c[2];
+  } else {
+    if (n != 2) return fail(h, SIGNMUON_E_INVALID, "NS takes 2 coefficients (a, b)");
+    h->ns_a = c[0]; h->ns_b = c[1];
+  }
+  return SIGNMUON_OK;
+}
+
+int signmuon_step(signmuon_t h, float* W, const float* const* G, float eta) {
+  int rc = check_handle(h, true);
+  if (rc) return rc;
+  const Plan& p = h->plan;
+  if (W == nullptr || G == nullptr) return fail(h, SIGNMUON_E_INVALID, "null W or G");
+  if (!aligned16(W)) return fail(h, SIGNMUON_E_INVALID, "W must be 16-byte aligned");
+  for (int m = 0; m < h->M; ++m)
+    if (G[m] == nullptr || !aligned16(G[m])) return fail(h, SIGNMUON_E_INVALID, "G[m] null or not 16-byte aligned");
+  cudaStream_t s = h->stream;
+  CK(h, cudaMemsetAsync(h->status, 0, 2 * sizeof(int), s));
+  const sm::WorkerPtrs gp = worker_ptrs(G, h->M);
+  {
+    ProfScope ps(h, 0);
+    sm::launch_momentum(s, gp, W, h->Mom, p.dpad, h->M, h->beta, h->lambda, h->X[0], p.fp32 ? 0 : 1, h->d_chunks,
+                        (int)p.chunks.size(), h->d_mats, h->d_groups, h->partials);
+  }
+  fro_finalize(h, h->M);
+  run_ns(h, h->M, strided_ptrs(h->Mom, p.dpad, h->M), h->U, p.dpad);
+  {
+    ProfScope ps(h, 4);
+    sm::launch_pack(s, h->U, p.dpad, p.d, h->bits, p.nb_pad, h->M);
+  }
+  if (h->flags & SIGNMUON_POST_POLAR) {
+    {
+      ProfScope ps(h, 5);
+      sm::launch_vote_major(s, h->bits, p.nb_pad, h->M, p.d, h->D);
+    }
+    const sm::WorkerPtrs dp = strided_ptrs(h->D, 0, 1);
+    {
+      ProfScope ps(h, 6);
+      sm::launch_stage(s, dp, 1, h->X[0], p.fp32 ? 0 : 1, h->d_chunks, (int)p.chunks.size(), h->d_mats,
+                       h->d_groups, h->partials);
+    }
+    fro_finalize(h, 1);
+    run_ns(h, 1, dp, h->D, 0);
+    ProfScope ps(h, 8);
+    sm::launch_update(s, W, h->D, p.d, eta, h->status);
+  } else {
+    ProfScope ps(h, 5);
+    sm::launch_vote_update(s, h->bits, p.nb_pad, h->M, p.d, W, eta, h->status);
+  }
+  return finish(h, (h->flags & SIGNMUON_ASYNC) == 0);
+}
+
+int signmuon_step_host(signmuon_t h, float* W_host, const float* const* G_host, float eta) {
+  int rc = check_handle(h, true);
+  if (rc) return rc;
+  const Plan& p = h->plan;
+  if (W_host == nullptr || G_host == nullptr) return fail(h, SIGNMUON_E_INVALID, "null W or G");
+  if (!h->hw_W) {
+    if ((rc = dalloc(h, &h->hw_W, p.dpad))) return rc;
+    if ((rc = dalloc(h, &h->hw_G, (int64_t)h->M * p.dpad))) return rc;
+  }
+  cudaStream_t s = h->stream;
+  CK(h, cudaMemcpyAsync(h->hw_W, W_host, (size_t)p.d * 4, cudaMemcpyHostToDevice, s));
+  std::vector<const float*> gd(h->M);
+  for (int m = 0; m < h->M; ++m) {
+    if (G_host[m] == nullptr) return fail(h, SIGNMUON_E_INVALID, "null G[m]");
+    gd[m] = h->hw_G + (int64_t)m * p.dpad;
+    CK(h, cudaMemcpyAsync(const_cast<float*>(gd[m]), G_host[m], (size_t)p.d * 4, cudaMemcpyHostToDevice, s));
+  }
+  const unsigned saved = h->flags;
+  h->flags |= SIGNMUON_ASYNC;
+  rc = signmuon_step(h, h->hw_W, gd.data(), eta);
+  h->flags = saved;
+  if (rc) return rc;
+  CK(h, cudaMemcpyAsync(W_host, h->hw_W, (size_t)p.d * 4, cudaMemcpyDeviceToHost, s));
+  return signmuon_sync(h);
+}
+
+int signmuon_sync(signmuon_t h) {
+  if (h == nullptr) return fail(nullptr, SIGNMUON_E_INVALID, "null handle");
+  CK(h, cudaStreamSynchronize(h->stream));
+  if (!h->pending) return SIGNMUON_OK;
+  h->pending = false;
+  if (h->h_status[1] != 0) return fail(h, SIGNMUON_E_TIMEOUT, "a kernel's bounded wait expired");
+  if (h->h_status[0] != 0) return fail(h, SIGNMUON_E_NONFINITE, "a momentum norm is NaN or Inf; W was not updated");
+  return SIGNMUON_OK;
+}
+
+int signmuon_vote(signmuon_t h, const uint8_t* const* signs, int64_t d, void* sums, int8_t* majority) {
+  int rc = check_handle(h, false);
+  if (rc) return rc;
+  if (d < 0 || signs == nullptr) return fail(h, SIGNMUON_E_INVALID, "bad vote arguments");
+  for (int m = 0; m < h->M; ++m)
+    if (signs[m] == nullptr || !aligned16(signs[m])) return fail(h, SIGNMUON_E_INVALID, "signs[m] null or misaligned");
+  if ((sums && !aligned16(sums)) || (majority && !aligned16(majority)))
+    return fail(h, SIGNMUON_E_INVALID, "sums/majority must be 16-byte aligned");
+  sm::WorkerPtrs sp{};
+  for (int m = 0; m < h->M; ++m) sp.p[m] = reinterpret_cast<const float*>(signs[m]);
+  sm::launch_vote(h->stream, sp, h->M, d, sums, (h->flags & SIGNMUON_ACC_INT8) ? 1 : 0, majority);
+  CK(h, cudaGetLastError());
+  return SIGNMUON_OK;
+}
+
+int signmuon_pack(signmuon_t h, const float* U, int64_t d, uint8_t* out) {
+  int rc = check_handle(h, false);
+  if (rc) return rc;
+  if (d < 0 || (d > 0 && (U == nullptr || out == nullptr))) return fail(h, SIGNMUON_E_INVALID, "bad pack arguments");
+  if (!aligned16(U) || !aligned16(out)) return fail(h, SIGNMUON_E_INVALID, "U/out must be 16-byte aligned");
+  sm::launch_pack(h->stream, U, 0, d, out, 0, 1);
+  CK(h, cudaGetLastError());
+  return SIGNMUON_OK;
+}
+
+int signmuon_apply_update(signmuon_t h, float* W, const float* D, int64_t d, float eta) {
+  int rc = check_handle(h, false);
+  if (rc) return rc;
+  if (d < 0 || (d > 0 && (W == nullptr || D == nullptr))) return fail(h, SIGNMUON_E_INVALID, "bad update arguments");
+  if (!aligned16(W) || !aligned16(D)) return fail(h, SIGNMUON_E_INVALID, "W/D must be 16-byte aligned");
+  sm::launch_update(h->stream, W, D, d, eta, nullptr);
+  CK(h, cudaGetLastError());
+  return SIGNMUON_OK;
+}
+
+int signmuon_polar(signmuon_t h, const float* const* X, float* const* U) {
+  int rc = check_handle(h, true);
+  if (rc) return rc;
+  const Plan& p = h->plan;
+  if (X == nullptr || U == nullptr) return fail(h, SIGNMUON_E_INVALID, "null X or U");
+  for (int m = 0; m < h->M; ++m)
+    if (!X[m] || !U[m] || !aligned16(X[m]) || !aligned16(U[m]))
+      return fail(h, SIGNMUON_E_INVALID, "X[m]/U[m] null or misaligned");
+  cudaStream_t s = h->stream;
+  CK(h, cudaMemsetAsync(h->status, 0, 2 * sizeof(int), s));
+  const sm::WorkerPtrs xp = worker_ptrs(X, h->M);
+  sm::launch_stage(s, xp, h->M, h->X[0], p.fp32 ? 0 : 1, h->d_chunks, (int)p.chunks.size(), h->d_mats, h->d_groups,
+                   h->partials);
+  fro_finalize(h, h->M);
+  run_ns(h, h->M, xp, h->U, p.dpad);
+  for (int m = 0; m < h->M; ++m)
+    CK(h, cudaMemcpyAsync(U[m], h->U + (int64_t)m * p.dpad, (size_t)p.d * 4, cudaMemcpyDeviceToDevice, s));
+  return finish(h, (h->flags & SIGNMUON_ASYNC) == 0);
+}
+
+int signmuon_get_momentum(signmuon_t h, int m, float* dst) {
+  int rc = check_handle(h, true);
+  if (rc) return rc;
+  if (m < 0 || m >= h->M || !dst) return fail(h, SIGNMUON_E_INVALID, "bad worker index or null dst");
+  CK(h, cudaMemcpyAsync(dst, h->Mom + (int64_t)m * h->plan.dpad, (size_t)h->plan.d * 4, cudaMemcpyDeviceToDevice,
+                        h->stream));
+  return SIGNMUON_OK;
+}
+
+int signmuon_set_momentum(signmuon_t h, int m, const float* src) {
+  int rc = check_handle(h, true);
+  if (rc) return rc;
+  if (m < 0 || m >= h->M || !src) return fail(h, SIGNMUON_E_INVALID, "bad worker index or null src");
+  CK(h, cudaMemcpyAsync(h->Mom + (int64_t)m * h->plan.dpad, src, (size_t)h->plan.d * 4, cudaMemcpyDeviceToDevice,
+                        h->stream));
+  return SIGNMUON_OK;
+}
+
+int signmuon_get_polar(signmuon_t h, int m, float* dst) {
+  int rc = check_handle(h, true);
+  if (rc) return rc;
+  if (m < 0 || m >= h->M || !dst) return fail(h, SIGNMUON_E_INVALID, "bad worker index or null dst");
+  CK(h, cudaMemcpyAsync(dst, h->U + (int64_t)m * h->plan.dpad, (size_t)h->plan.d * 4, cudaMemcpyDeviceToDevice,
+                        h->stream));
+  return SIGNMUON_OK;
+}
+
+int signmuon_get_signs(signmuon_t h, int m, uint8_t* dst) {
+  int rc = check_handle(h, true);
+  if (rc) return rc;
+  if (m < 0 || m >= h->M || !dst) return fail(h, SIGNMUON_E_INVALID, "bad worker index or null dst");
+  CK(h, cudaMemcpyAsync(dst, h->bits + (int64_t)m * h->plan.nb_pad, (size_t)h->plan.nb, cudaMemcpyDeviceToDevice,
+                        h->stream));
+  return SIGNMUON_OK;
+}
+
+int signmuon_get_direction(signmuon_t h, float* dst) {
+  int rc = check_handle(h, true);
+  if (rc) return rc;
+  if (!dst || !aligned16(dst)) return fail(h, SIGNMUON_E_INVALID, "null or misaligned dst");
+  const Plan& p = h->plan;
+  if (h->flags & SIGNMUON_POST_POLAR) {
+    CK(h, cudaMemcpyAsync(dst, h->D, (size_t)p.d * 4, cudaMemcpyDeviceToDevice, h->stream));
+  } else {
+    // the step fuses the vote into the update; recompute the majority from
+    // the last step's packed signs
+    sm::launch_vote_major(h->stream, h->bits, p.nb_pad, h->M, p.d, dst);
+    CK(h, cudaGetLastError());
+  }
+  return SIGNMUON_OK;
+}
+
+int signmuon_get_scales(signmuon_t h, float* dst_host) {
+  int rc = check_handle(h, true);
+  if (rc) return rc;
+  if (!dst_host) return fail(h, SIGNMUON_E_INVALID, "null dst");
+  CK(h, cudaMemcpyAsync(dst_host, h->scale_v, (size_t)h->M * h->plan.n_mats * 4, cudaMemcpyDeviceToHost, h->stream));
+  CK(h, cudaStreamSynchronize(h->stream));
+  return SIGNMUON_OK;
+}
+
+int signmuon_profile(signmuon_t h, int enable) {
+  if (h == nullptr) return fail(nullptr, SIGNMUON_E_INVALID, "null handle");
+  prof_collect(h);
+  h->prof = enable != 0;
+  return SIGNMUON_OK;
+}
+
+int signmuon_profile_read(signmuon_t h, double* ms, int64_t* launches, int n) {
+  if (h == nullptr) return fail(nullptr, SIGNMUON_E_INVALID, "null handle");
+  prof_collect(h);
+  for (int k = 0; k < n && k < SIGNMUON_PROF_KINDS; ++k) {
+    if (ms) ms[k] = h->prof_ms[k];
+    if (launches) launches[k] = h->prof_n[k];
+    h->prof_ms[k] = 0.0;
+    h->prof_n[k] = 0;
+  }
+  return SIGNMUON_OK;
+}
+
+int signmuon_info(signmuon_t h, int64_t* out, int n) {
+  if (h == nullptr) return fail(nullptr, SIGNMUON_E_INVALID, "null handle");
+  if (!out) return fail(h, SIGNMUON_E_INVALID, "null out");
+  fill_info(h->plan, out, n);
+  if (n > 2) out[2] = h->bytes;
+  return SIGNMUON_OK;
+}
+
+}  // extern "C"

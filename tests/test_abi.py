@@ -1,0 +1,75 @@
+"""CPU-side checks of the C ABI: the library loads, exports every symbol the
+header declares, and the host-only planner validates and sizes plans like
+signmuon_init would (no GPU calls)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "signmuon.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"\b(signmuon_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    import sign_muon_optimizer_b200 as smo
+    lib = ctypes.CDLL(smo.LIB_PATH)
+    names = _declared()
+    assert len(names) >= 20
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in signmuon.h but not exported"
+    assert sorted(smo.EXPORTED) == names
+
+
+def test_plan_sizes_for_the_workloads():
+    import sign_muon_optimizer_b200 as smo
+    p = smo.signmuon_plan(synth.NANOGPT_SHAPES, 8, 5, "spectral", 2)
+    assert p["d"] == 84_934_656 and p["packed_bytes"] == 10_616_832 and p["groups"] == 4
+    p = smo.signmuon_plan(synth.RESNET50_SHAPES, 4, 5, "spectral", 2)
+    assert p["d"] == 25_502_912 and p["n_mats"] == 54
+    p = smo.signmuon_plan(synth.LLAMA_LAYER_SHAPES, 16, flags=smo.SIGNMUON_VOTE_ONLY)
+    assert p["d"] == 717_225_984 and p["packed_bytes"] == 89_653_248 and p["device_bytes"] == 0
+    p = smo.signmuon_plan([(3, 5)], 1)
+    assert p["packed_bytes"] == 2  # ceil(15/8)
+
+
+@pytest.mark.parametrize("shapes,M,K,scale,P,flags,status", [
+    ([(3, 0)], 2, 5, "fro", 1, 0, 1),
+    ([(3, 3)], 0, 5, "fro", 1, 0, 1),
+    ([(3, 3)], 257, 5, "fro", 1, 0, 1),
+    ([(3, 3)], 2, -1, "fro", 1, 0, 1),
+    ([(3, 3)], 2, 5, "spectral", 0, 0, 1),
+    ([(3, 3)], 128, 5, "fro", 1, 1 << 3, 2),
+    ([(70000, 70000)], 1, 5, "fro", 1, 0, 1),
+])
+def test_plan_rejects_invalid(shapes, M, K, scale, P, flags, status):
+    import sign_muon_optimizer_b200 as smo
+    with pytest.raises(smo.SignMuonError) as e:
+        smo.signmuon_plan(shapes, M, K, scale, P, flags)
+    assert e.value.status == status
+    assert smo.signmuon_last_error(None)
+
+
+def test_init_validation_without_gpu():
+    # argument checks run before any CUDA call
+    import sign_muon_optimizer_b200 as smo
+    for kw in (dict(beta=1.0), dict(beta=-0.1), dict(lam=-1.0), dict(eps=0.0)):
+        args = dict(beta=0.9, lam=0.0, K=5, eps=1e-7, scale="fro", P=1)
+        args.update(kw)
+        with pytest.raises(smo.SignMuonError) as e:
+            smo.signmuon_init([(4, 4)], 2, args["beta"], args["lam"], args["K"], args["eps"], args["scale"],
+                              args["P"])
+        assert e.value.status == smo.SIGNMUON_E_INVALID
+
+
+def test_status_strings():
+    import sign_muon_optimizer_b200 as smo
+    for s in range(8):
+        assert smo.signmuon_status_string(s)

@@ -1,0 +1,155 @@
+"""GPU parity of the individual stages, through the C ABI, against the oracle.
+
+Bit-exact: one-bit pack, vote sums / majority (int32 and int8), the update.
+Tolerance: the momentum pass (fp32 against float64) and PolarNS (2e-2 bf16,
+1e-4 fp32 max abs; <= 1e-3 sign disagreements above the 1e-3 mask).
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+
+import synth
+from oracle import signmuon_ref as ref
+
+from gpu_helpers import assert_polar_close, dev, host, oracle_polar_flat
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+import sign_muon_optimizer_b200 as smo  # noqa: E402
+
+
+def _vote_handle(M, acc8=False):
+    flags = smo.SIGNMUON_VOTE_ONLY | (smo.SIGNMUON_ACC_INT8 if acc8 else 0)
+    return smo.SignMuon([(1, 1)], M, flags=flags)
+
+
+@pytest.mark.parametrize("d", [1, 7, 31, 33, 1000, 1024, 1025, 5 * 1024 + 17, 100003])
+def test_pack_bit_exact(d):
+    u = synth.uniform_values(d, config_id=11, step=d)
+    if d > 40:
+        u[5] = np.nan
+        u[6] = np.float32(-0.0)
+        u[7] = np.float32(0.0)
+    h = _vote_handle(1)
+    U = dev(u)
+    out = torch.zeros((d + 7) // 8 + 16, dtype=torch.uint8, device="cuda")
+    h.pack(U, d, out)
+    got = host(out)
+    want = ref.pack_bits(ref.sign_bits(u))
+    assert np.array_equal(got[: want.size], want)
+    assert not got[want.size:].any()  # nothing written past ceil(d/8)
+
+
+def test_vote_blog_worked_example():
+    g = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "blog_worked_example.json")))
+    dirs = np.array(g["directions"], np.float32)
+    h = _vote_handle(3)
+    signs = [dev(ref.pack_bits(ref.sign_bits(x.ravel()))) for x in dirs]
+    signs = [torch.nn.functional.pad(s, (0, 15)) for s in signs]  # 16-byte aligned copies
+    sums = torch.zeros(4, dtype=torch.int32, device="cuda")
+    maj = torch.zeros(16, dtype=torch.int8, device="cuda")
+    h.vote(signs, 4, sums, maj)
+    assert host(sums).reshape(2, 2).tolist() == g["sums"]
+    assert host(maj)[:4].reshape(2, 2).tolist() == g["majority"]
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 16, 127, 200])
+@pytest.mark.parametrize("d", [1, 7, 1024, 5000, 40 * 1024 + 3])
+def test_vote_bit_exact(M, d):
+    bits = synth.bernoulli_bits(d, M, config_id=M * 1000 + d % 997)
+    packed = [ref.pack_bits(b) for b in bits]
+    want_sums = ref.vote_sums_from_bits(packed, d, "int32")
+    want_maj = ref.majority(want_sums)
+    nb = (d + 7) // 8
+    signs = [dev(np.concatenate([p, np.zeros(16, np.uint8)])) for p in packed]
+    h = _vote_handle(M)
+    sums = torch.zeros(d, dtype=torch.int32, device="cuda")
+    maj = torch.zeros(d, dtype=torch.int8, device="cuda")
+    h.vote(signs, d, sums, maj)
+    assert np.array_equal(host(sums), want_sums)
+    assert np.array_equal(host(maj), want_maj)
+    if M <= 127:
+        h8 = _vote_handle(M, acc8=True)
+        sums8 = torch.zeros(d, dtype=torch.int8, device="cuda")
+        h8.vote(signs, d, sums8, None)
+        assert np.array_equal(host(sums8), ref.vote_sums_from_bits(packed, d, "int8"))
+    assert nb == ref.packed_nbytes(d)
+
+
+def test_int8_guard_rejects_large_M():
+    with pytest.raises(smo.SignMuonError) as e:
+        _vote_handle(128, acc8=True)
+    assert e.value.status == smo.SIGNMUON_E_OVERFLOW
+
+
+@pytest.mark.parametrize("kind", ["ternary", "real"])
+@pytest.mark.parametrize("d", [1, 5, 4096, 100003])
+def test_update_bit_exact(kind, d):
+    w = synth.weights0([(1, d)], config_id=d)
+    if kind == "ternary":
+        D = synth.ternary_direction(d, config_id=d)
+    else:
+        D = synth.uniform_values(d, config_id=d, step=3)
+    eta = np.float32(0.02)
+    h = _vote_handle(1)
+    W = dev(w)
+    h.apply_update(W, dev(D), d, eta)
+    want = ref.update(w, D, eta)
+    assert np.array_equal(host(W).view(np.uint32), want.view(np.uint32))
+
+
+SHAPES_SMALL = [(3, 5), (5, 3), (130, 70), (64, 147), (200, 200), (96, 300)]
+
+
+def _polar_case(shapes, M, K, scale, P, precision, order, seed):
+    flags = (smo.SIGNMUON_NS_FP32 if precision == "fp32" else 0) | (smo.SIGNMUON_NS_QUINTIC if order == "quintic" else 0)
+    h = smo.SignMuon(shapes, M, beta=0.9, lam=0.0, K=K, eps=1e-7, scale=scale, P=P, flags=flags)
+    xs = synth.gaussian_matrices(shapes, M, config_id=seed)
+    X = [dev(x) for x in xs]
+    U = [torch.zeros_like(x) for x in X]
+    h.polar(X, U)
+    worst = 0.0
+    for m in range(M):
+        want = oracle_polar_flat(xs[m].astype(np.float64), shapes, K, 1e-7, scale, P, order)
+        err, _, _ = assert_polar_close(host(U[m]), want, precision, f"worker {m}")
+        worst = max(worst, err)
+    return worst
+
+
+@pytest.mark.parametrize("precision", ["fp32", "bf16"])
+@pytest.mark.parametrize("scale,P", [("fro", 1), ("spectral", 2)])
+@pytest.mark.parametrize("K", [0, 1, 5])
+def test_polar_cubic(precision, scale, P, K):
+    _polar_case(SHAPES_SMALL, 2, K, scale, P, precision, "cubic", seed=100 + K)
+
+
+@pytest.mark.parametrize("precision", ["fp32", "bf16"])
+def test_polar_quintic(precision):
+    _polar_case(SHAPES_SMALL, 2, 5, "spectral", 2, precision, "quintic", seed=7)
+
+
+@pytest.mark.parametrize("precision", ["fp32", "bf16"])
+def test_polar_large_tiles(precision):
+    # several 128x256 tiles per problem, ragged edges, both orientations
+    _polar_case([(768, 2304), (2304, 768), (520, 600)], 2, 5, "spectral", 2, precision, "cubic", seed=21)
+
+
+def test_momentum_pass():
+    shapes = [(256, 128), (3, 5), (64, 147)]
+    M = 3
+    h = smo.SignMuon(shapes, M, beta=0.9, lam=0.01, K=1, eps=1e-7, scale="fro", flags=smo.SIGNMUON_NS_FP32)
+    d = h.d
+    w = synth.weights0(shapes, 1)
+    mom0 = synth.momentum0(shapes, M, 1)
+    for m in range(M):
+        h.set_momentum(m, dev(mom0[m]))
+    G = synth.gradients(shapes, M, 0.5, step=1, config_id=1)
+    h.step(dev(w), [dev(g) for g in G], 0.02)
+    for m in range(M):
+        got = torch.zeros(d, device="cuda")
+        h.get_momentum(m, got)
+        want = ref.momentum_update(mom0[m], G[m], w, 0.9, 0.01)
+        assert np.max(np.abs(host(got) - want) / (np.abs(want) + 1e-3)) < 1e-5

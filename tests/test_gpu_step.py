@@ -1,0 +1,216 @@
+"""GPU parity of the whole Sign-Muon step (signmuon_step through the C ABI).
+
+The oracle runs the same step independently from the same seeded state (W0,
+momentum, gradients).  Momentum and U are compared with tolerances; the packed
+signs may differ only on entries whose |U| is within the precision's noise
+(counted by the 1e-3 sign-disagreement bar); wherever every worker's sign
+agrees the majority must be identical, and wherever D agrees W must be
+bit-exact.
+"""
+import numpy as np
+import pytest
+
+import synth
+from oracle import signmuon_ref as ref
+
+from gpu_helpers import assert_polar_close, dev, host
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+import sign_muon_optimizer_b200 as smo  # noqa: E402
+
+HP = dict(beta=0.9, lam=0.01, eta=0.02, eps=1e-7)
+
+
+def _flags(precision, post_polar=False, order="cubic"):
+    f = smo.SIGNMUON_NS_FP32 if precision == "fp32" else 0
+    if post_polar:
+        f |= smo.SIGNMUON_POST_POLAR
+    if order == "quintic":
+        f |= smo.SIGNMUON_NS_QUINTIC
+    return f
+
+
+def _run_one_step(shapes, M, sigma, K, scale, P, precision, post_polar, seed, order="cubic"):
+    h = smo.SignMuon(shapes, M, beta=HP["beta"], lam=HP["lam"], K=K, eps=HP["eps"], scale=scale, P=P,
+                     flags=_flags(precision, post_polar, order))
+    d = h.d
+    w0 = synth.weights0(shapes, seed)
+    mom0 = synth.momentum0(shapes, M, seed, scale=0.5)
+    G = synth.gradients(shapes, M, sigma, step=1, config_id=seed)
+    for m in range(M):
+        h.set_momentum(m, dev(mom0[m]))
+    W = dev(w0)
+    h.step(W, [dev(g) for g in G], HP["eta"])
+    gpu = dict(W=host(W), mom=[], U=[], bits=[])
+    for m in range(M):
+        t = torch.zeros(d, device="cuda")
+        h.get_momentum(m, t)
+        gpu["mom"].append(host(t))
+        t = torch.zeros(d, device="cuda")
+        h.get_polar(m, t)
+        gpu["U"].append(host(t))
+        b = torch.zeros(ref.packed_nbytes(d), dtype=torch.uint8, device="cuda")
+        h.get_signs(m, b)
+        gpu["bits"].append(host(b))
+    D = torch.zeros(d, device="cuda")
+    h.get_direction(D)
+    gpu["D"] = host(D)
+    gpu["scales"] = h.get_scales()
+    want = ref.step(w0, G, mom0, shapes, beta=HP["beta"], lam=HP["lam"], eta=HP["eta"], K=K, eps=HP["eps"],
+                    scale=scale, P=P, order=order, post_polar=post_polar)
+    return h, gpu, want
+
+
+def _np_bits(packed, d):
+    return np.unpackbits(np.asarray(packed, np.uint8), bitorder="little")[:d].astype(bool)
+
+
+def _np_majority(packed_list, d):
+    s = np.zeros(d, np.int64)
+    for p in packed_list:
+        s += 2 * _np_bits(p, d).astype(np.int64) - 1
+    return np.sign(s).astype(np.int8)
+
+
+def _compare_step(shapes, M, gpu, want, precision, post_polar):
+    d = synth.numel(shapes)
+    for m in range(M):
+        assert np.max(np.abs(gpu["mom"][m] - want["mom"][m]) / (np.abs(want["mom"][m]) + 1e-3)) < 1e-5
+        assert_polar_close(gpu["U"][m], want["U"][m], precision, f"U worker {m}")
+    # the GPU's packed signs are exactly the signs of its own U (numpy check)
+    for m in range(M):
+        assert np.array_equal(gpu["bits"][m], np.packbits(gpu["U"][m] >= 0, bitorder="little"))
+    # wherever every worker's sign agrees with the oracle's, the vote agrees exactly
+    agree = np.ones(d, bool)
+    for m in range(M):
+        agree &= _np_bits(gpu["bits"][m], d) == _np_bits(want["packed"][m], d)
+    gpu_maj = _np_majority(gpu["bits"], d)
+    assert np.array_equal(gpu_maj[agree], want["majority"][agree])
+    assert (~agree).mean() <= M * 1e-3
+    if not post_polar:
+        assert np.array_equal(gpu["D"], gpu_maj.astype(np.float32))
+        same = gpu["D"] == want["D32"]
+        assert np.array_equal(gpu["W"][same].view(np.uint32), want["W"][same].view(np.uint32))
+        assert (~same).mean() <= M * 1e-3
+    else:
+        off = 0
+        compared = 0
+        for r, c in shapes:
+            sl = slice(off, off + r * c)
+            if np.array_equal(gpu_maj[sl], want["majority"][sl]):
+                assert_polar_close(gpu["D"][sl], want["D"][sl], precision, f"post-polar D {r}x{c}")
+                tol = HP["eta"] * (2e-2 if precision == "bf16" else 1e-4) + 1e-6
+                assert np.max(np.abs(gpu["W"][sl] - want["W"][sl])) <= tol
+                compared += 1
+            off += r * c
+        assert compared >= 1
+
+
+@pytest.mark.parametrize("precision", ["fp32", "bf16"])
+def test_step_config1_single(precision):
+    shapes = synth.CONFIG1_SHAPES
+    h, gpu, want = _run_one_step(shapes, 3, 0.5, 5, "fro", 1, precision, False, seed=1)
+    _compare_step(shapes, 3, gpu, want, precision, False)
+
+
+@pytest.mark.parametrize("precision", ["fp32", "bf16"])
+@pytest.mark.parametrize("scale,P", [("fro", 1), ("spectral", 2)])
+def test_step_ragged_post_polar(precision, scale, P):
+    shapes = [(3, 5), (130, 70), (64, 147), (96, 300)]
+    M = 4  # even: ties occur and must map to zero
+    h, gpu, want = _run_one_step(shapes, M, 1.0, 5, scale, P, precision, True, seed=3)
+    _compare_step(shapes, M, gpu, want, precision, True)
+
+
+def test_step_quintic_fp32():
+    shapes = [(64, 96), (96, 64)]
+    h, gpu, want = _run_one_step(shapes, 2, 1.0, 3, "spectral", 2, "fp32", False, seed=5, order="quintic")
+    _compare_step(shapes, 2, gpu, want, "fp32", False)
+
+
+def test_step_config1_ten_steps_drift():
+    """Config 1 end to end: 10 steps on the GPU (fp32 NS) and in the oracle,
+    each from its own state; the trajectories may part only where a sign was
+    within rounding of zero."""
+    shapes = synth.CONFIG1_SHAPES
+    M = 3
+    h = smo.SignMuon(shapes, M, beta=HP["beta"], lam=HP["lam"], K=5, eps=HP["eps"], scale="fro",
+                     flags=smo.SIGNMUON_NS_FP32)
+    w0 = synth.weights0(shapes, 0)
+    W = dev(w0)
+    w_ref = w0.copy()
+    mom_ref = [np.zeros(h.d)] * M
+    for t in range(10):
+        G = synth.gradients(shapes, M, 0.5, step=t, config_id=0)
+        h.step(W, [dev(g) for g in G], HP["eta"])
+        out = ref.step(w_ref, G, mom_ref, shapes, beta=HP["beta"], lam=HP["lam"], eta=HP["eta"], K=5,
+                       eps=HP["eps"], scale="fro")
+        w_ref, mom_ref = out["W"], out["mom"]
+    w_gpu = host(W)
+    differ = w_gpu != w_ref
+    assert differ.mean() <= 1e-2, f"{differ.sum()} of {w_gpu.size} weights differ after 10 steps"
+    assert np.max(np.abs(w_gpu - w_ref)) <= 2 * HP["eta"] * 10 + 1e-6
+
+
+def test_nonfinite_gradient_keeps_w():
+    shapes = [(64, 96)]
+    h = smo.SignMuon(shapes, 2, K=2, scale="fro")
+    w0 = synth.weights0(shapes, 9)
+    G = synth.gradients(shapes, 2, 1.0, step=0, config_id=9)
+    G[1][17] = np.nan
+    W = dev(w0)
+    with pytest.raises(smo.SignMuonError) as e:
+        h.step(W, [dev(g) for g in G], 0.02)
+    assert e.value.status == smo.SIGNMUON_E_NONFINITE
+    assert np.array_equal(host(W).view(np.uint32), w0.view(np.uint32))
+
+
+@pytest.mark.parametrize("precision", ["fp32", "bf16"])
+def test_checkpoint_resume_bit_exact(precision):
+    shapes = [(128, 256), (300, 64)]
+    M = 3
+    kw = dict(beta=0.9, lam=0.01, K=5, eps=1e-7, scale="spectral", P=2, flags=_flags(precision))
+    w0 = synth.weights0(shapes, 4)
+    grads = [synth.gradients(shapes, M, 1.0, step=t, config_id=4) for t in range(10)]
+    a = smo.SignMuon(shapes, M, **kw)
+    Wa = dev(w0)
+    for t in range(10):
+        a.step(Wa, [dev(g) for g in grads[t]], 0.02)
+    b = smo.SignMuon(shapes, M, **kw)
+    Wb = dev(w0)
+    for t in range(5):
+        b.step(Wb, [dev(g) for g in grads[t]], 0.02)
+    saved = []
+    for m in range(M):
+        s = torch.zeros(b.d, device="cuda")
+        b.get_momentum(m, s)
+        saved.append(s)
+    b.close()
+    c = smo.SignMuon(shapes, M, **kw)
+    for m in range(M):
+        c.set_momentum(m, saved[m])
+    for t in range(5, 10):
+        c.step(Wb, [dev(g) for g in grads[t]], 0.02)
+    assert np.array_equal(host(Wa).view(np.uint32), host(Wb).view(np.uint32))
+    for m in range(M):
+        x = torch.zeros(a.d, device="cuda")
+        y = torch.zeros(a.d, device="cuda")
+        a.get_momentum(m, x)
+        c.get_momentum(m, y)
+        assert torch.equal(x, y)
+
+
+def test_step_host_matches_device_step():
+    shapes = [(128, 256)]
+    M = 2
+    w0 = synth.weights0(shapes, 6)
+    G = synth.gradients(shapes, M, 1.0, step=0, config_id=6)
+    a = smo.SignMuon(shapes, M, K=3, scale="fro")
+    W = dev(w0)
+    a.step(W, [dev(g) for g in G], 0.02)
+    b = smo.SignMuon(shapes, M, K=3, scale="fro")
+    wh = w0.copy()
+    b.step_host(wh, G, 0.02)
+    assert np.array_equal(wh.view(np.uint32), host(W).view(np.uint32))
