@@ -158,11 +158,13 @@ def gpu_smi_id(dev_index):
 # CPU oracle (baseline leg and --impl reference)
 # ---------------------------------------------------------------------------
 def cpu_oracle_sample(step_idx=0):
-    """One oracle step on one transformer layer (4 of the 48 matrices, 1/12 of
-    the weights and of the work) for all 8 workers, including the post-vote
-    polar step; returns seconds."""
+    """One oracle step on the 768x768 attention projection of one layer for
+    all 8 workers, including power iteration and the post-vote polar step;
+    returns seconds.  Every nanoGPT matrix has 768 as its small side, so both
+    the Newton-Schulz flops and the elementwise work of a matrix scale with
+    its element count: this sample is exactly 1/144 of one whole step."""
     from oracle import signmuon_ref as ref
-    shapes = SHAPES[:4]
+    shapes = [SHAPES[1]]
     w = synth.weights0(shapes, 3)
     G = synth.gradients(shapes, M, WL["sigma"], step=step_idx, config_id=3)
     mom = synth.momentum0(shapes, M, 3, scale=0.5)
@@ -170,6 +172,9 @@ def cpu_oracle_sample(step_idx=0):
     ref.step(w, G, mom, shapes, beta=HP["beta"], lam=HP["lam"], eta=HP["eta"], K=K_NS, eps=HP["eps"],
              scale=WL["scale"], P=WL["P"], post_polar=WL["post_polar"])
     return time.perf_counter() - t0
+
+
+CPU_SCALE = float(D) / (SHAPES[1][0] * SHAPES[1][1])  # 144
 
 
 def cpu_threads():
@@ -183,9 +188,9 @@ def cpu_threads():
     return os.cpu_count() or 1
 
 
-CPU_SAMPLE = ("one of the 12 transformer layers (2304x768, 768x768, 3072x768, 768x3072; 7,077,888 weights) "
-              "x 8 workers, full oracle step incl. power iteration and post-vote polar, numpy float64; "
-              "steps/s scaled by 1/12 to the whole model")
+CPU_SAMPLE = ("the 768x768 attention projection of one layer (589,824 weights, 1/144 of the model's "
+              "weights and Newton-Schulz flops) x 8 workers, full oracle step incl. power iteration and "
+              "post-vote polar, numpy float64; steps/s scaled by 1/144 to the whole model")
 
 
 def run_reference(args):
@@ -195,7 +200,7 @@ def run_reference(args):
     for i in range(args.warmup):
         cpu_oracle_sample(i)
     times = [cpu_oracle_sample(args.warmup + i) for i in range(args.steps)]
-    per_step = 12.0 * sum(times) / len(times)
+    per_step = CPU_SCALE * sum(times) / len(times)
     value = 1.0 / per_step
     cores = cpu_threads()
     line = {
@@ -271,8 +276,9 @@ def run_ours(args):
     pk, pk_kind = peaks()
     steps = args.steps
     flops = ns_flops_per_step(SHAPES, M, K_NS, WL["post_polar"])
-    gemm_ms = prof["ns_gemm"][0] + prof["post_ns_gemm"][0]
-    gemm_launches = prof["ns_gemm"][1] + prof["post_ns_gemm"][1]
+    gemm_kinds = ["ns_gram", "ns_square", "ns_apply", "post_gram", "post_square", "post_apply"]
+    gemm_ms = sum(prof[k][0] for k in gemm_kinds)
+    gemm_launches = sum(prof[k][1] for k in gemm_kinds)
     tflops = flops * steps / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else None
     peak_tc = pk["bf16_tflops_sustained"]
     roofline = {"kernel": "k_gemm_tc (grouped Newton-Schulz GEMM, tcgen05)", "bound": "tensor",
@@ -287,8 +293,10 @@ def run_ours(args):
         if n == 0:
             continue
         e = {"ms_per_step": kms / steps, "launches_per_step": n / steps}
-        if kind in ("ns_gemm", "post_ns_gemm"):
-            f = ns_flops_per_step(SHAPES, M if kind == "ns_gemm" else 0, K_NS, kind == "post_ns_gemm")
+        if kind in gemm_kinds:
+            # cubic: the Gram and the apply GEMM each do half of the 4 m^2 n flops
+            f = 0.5 * ns_flops_per_step(SHAPES, 0 if kind.startswith("post") else M, K_NS,
+                                        kind.startswith("post"))
             e["TFLOP/s"] = f / (kms / steps / 1e3) / 1e12
             e["frac_of_bf16_peak"] = e["TFLOP/s"] / peak_tc
         elif kind in hbm:
@@ -328,8 +336,8 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        t = cpu_oracle_sample(0)
-        cpu = {"value": 1.0 / (12.0 * t), "unit": "steps/s", "cores": cpu_threads(), "kind": "oracle",
+        t = 0.5 * (cpu_oracle_sample(0) + cpu_oracle_sample(1))
+        cpu = {"value": 1.0 / (CPU_SCALE * t), "unit": "steps/s", "cores": cpu_threads(), "kind": "oracle",
                "sample": CPU_SAMPLE}
 
     if rank == 0:
@@ -352,6 +360,25 @@ def run_ours(args):
     return 0
 
 
+def run_capture(args):
+    """Profiler-capture mode (prints no bench line): the same step on the first
+    L transformer layers of the nanoGPT shapes, M=8, a few steps."""
+    import torch
+    import sign_muon_optimizer_b200 as smo
+    shapes = SHAPES[: 4 * args.capture_layers]
+    flags = smo.SIGNMUON_POST_POLAR if WL["post_polar"] else 0
+    opt = smo.SignMuon(shapes, M, beta=HP["beta"], lam=HP["lam"], K=K_NS, eps=HP["eps"], scale=WL["scale"],
+                       P=WL["P"], flags=flags)
+    W = synth.device_weights0(shapes, config_id=3)
+    G = synth.device_gradients(shapes, M, WL["sigma"], step=0, config_id=3)
+    for _ in range(args.steps):
+        opt.step(W, [G[m] for m in range(M)], HP["eta"])
+    torch.cuda.synchronize()
+    print(f"capture run done: {len(shapes)} matrices, {args.steps} steps, "
+          f"{smo.signmuon_kernel_launches()} kernel launches")
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -360,7 +387,11 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--capture-layers", type=int, default=0,
+                    help="profiler capture mode on the first L layers; prints no bench line")
     args = ap.parse_args()
+    if args.capture_layers > 0:
+        return run_capture(args)
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":

@@ -155,6 +155,11 @@ int signmuon_get_polar(signmuon_t h, int m, float* dst);
 int signmuon_get_signs(signmuon_t h, int m, uint8_t* dst);
 int signmuon_get_direction(signmuon_t h, float* dst);
 int signmuon_get_scales(signmuon_t h, float* dst_host);
+/* get_gram: the Gram matrix (g x g, g = min(rows, cols), row-major floats on
+ * the host) that the last Newton-Schulz iteration of worker m used for
+ * matrix `mat`: X X^T of the wide orientation; after one iteration it is the
+ * unscaled Gram of the staged momentum (waits for the GPU). */
+int signmuon_get_gram(signmuon_t h, int m, int mat, float* dst_host);
 
 /* Newton-Schulz coefficients: n=2 (a, b) for X <- aX + b(XX^T)X ([paper] §3
  * two-coefficient form), n=3 (a, b, c) for the quintic flag.  Defaults:
@@ -178,11 +183,12 @@ int signmuon_plan(const int64_t* shapes, int n_mats, int M, int K, int scale, in
  * a CUDA event pair around every kernel they launch on the handle's stream;
  * signmuon_profile_read() waits for the stream, adds up the elapsed times per
  * kind (ms[k], launches[k] for k < n) since the last read, and resets them.
- * Kinds: 0 momentum pass, 1 norm finalisation, 2 Newton-Schulz GEMMs,
- * 3 power iteration, 4 one-bit pack, 5 vote (fused with the update or writing
- * D), 6 staging of the majority, 7 post-vote Newton-Schulz GEMMs, 8 update,
- * 9 K=0 scaling. */
-#define SIGNMUON_PROF_KINDS 10
+ * Kinds: 0 momentum pass, 1 norm finalisation, 2/3/4 Newton-Schulz GEMMs
+ * (Gram, quintic square, apply), 5 power iteration, 6 one-bit pack, 7 vote
+ * (fused with the update or writing D), 8 staging of the majority, 9/10/11
+ * post-vote Newton-Schulz GEMMs (Gram, square, apply), 12 update, 13 K=0
+ * scaling. */
+#define SIGNMUON_PROF_KINDS 14
 int signmuon_profile(signmuon_t h, int enable);
 int signmuon_profile_read(signmuon_t h, double* ms, int64_t* launches, int n);
 

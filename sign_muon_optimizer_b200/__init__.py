@@ -5,7 +5,7 @@ CUDA kernels.  Device buffers are passed as torch CUDA tensors (or raw integer
 device addresses); host buffers as numpy arrays.  The functions keep the C
 names; each raises SignMuonError on a non-zero status.
 
-The library must be built first (``python -m sign_muon_optimizer_b200.build``);
+The library must be built first (``python sign_muon_optimizer_b200/build.py``);
 importing this package without it raises ImportError -- there is no fallback.
 """
 from __future__ import annotations
@@ -42,10 +42,10 @@ EXPORTED = [
     "signmuon_get_polar", "signmuon_get_signs", "signmuon_get_direction", "signmuon_get_scales",
     "signmuon_set_ns_coeffs", "signmuon_sync", "signmuon_info", "signmuon_plan",
     "signmuon_kernel_launches", "signmuon_last_error", "signmuon_status_string", "signmuon_destroy",
-    "signmuon_profile", "signmuon_profile_read",
+    "signmuon_profile", "signmuon_profile_read", "signmuon_get_gram",
 ]
-PROF_KINDS = ["momentum", "norm_finalize", "ns_gemm", "power_iter", "pack", "vote", "stage",
-              "post_ns_gemm", "update", "k0_scale"]
+PROF_KINDS = ["momentum", "norm_finalize", "ns_gram", "ns_square", "ns_apply", "power_iter", "pack",
+              "vote", "stage", "post_gram", "post_square", "post_apply", "update", "k0_scale"]
 
 
 class SignMuonError(RuntimeError):
@@ -56,7 +56,7 @@ class SignMuonError(RuntimeError):
 
 def _load():
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is not built; run `python -m sign_muon_optimizer_b200.build`")
+        raise ImportError(f"{LIB_PATH} is not built; run `python sign_muon_optimizer_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
     P, I, I64, F, U = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_uint
     PP = ctypes.POINTER(ctypes.c_void_p)
@@ -83,6 +83,7 @@ def _load():
         "signmuon_status_string": (ctypes.c_char_p, [I]),
         "signmuon_destroy": (None, [P]),
         "signmuon_profile": (I, [P, I]),
+        "signmuon_get_gram": (I, [P, I, I, P]),
         "signmuon_profile_read": (I, [P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(I64), I]),
     }
     for name, (res, args) in sig.items():
@@ -200,6 +201,12 @@ def signmuon_get_scales(h, M, n_mats):
     return out.reshape(M, n_mats)
 
 
+def signmuon_get_gram(h, m, mat, g):
+    out = np.zeros((g, g), np.float32)
+    _check(h, _lib.signmuon_get_gram(h, int(m), int(mat), out.ctypes.data))
+    return out
+
+
 def signmuon_set_ns_coeffs(h, coeffs):
     c = (ctypes.c_float * len(coeffs))(*[float(v) for v in coeffs])
     _check(h, _lib.signmuon_set_ns_coeffs(h, c, len(coeffs)))
@@ -297,6 +304,10 @@ class SignMuon:
 
     def get_direction(self, dst):
         signmuon_get_direction(self.h, dst)
+
+    def get_gram(self, m, mat):
+        r, c = self.shapes[mat]
+        return signmuon_get_gram(self.h, m, mat, min(r, c))
 
     def get_scales(self):
         return signmuon_get_scales(self.h, self.M, len(self.shapes))

@@ -17,6 +17,14 @@
 
 namespace sm {
 
+// tensor-core GEMM pipeline depth and widest output tile (build-time knobs)
+#ifndef SM_TC_STAGES
+#define SM_TC_STAGES 4
+#endif
+#ifndef SM_TC_BN_MAX
+#define SM_TC_BN_MAX 256
+#endif
+
 constexpr int kMaxWorkers = 256;
 
 struct MatInfo {      // one parameter matrix
@@ -56,7 +64,8 @@ struct WorkerPtrs {   // per-worker device pointers passed by value
 struct TileGroup {
   int group;
   int Mdim, Ndim, Kdim;
-  int BN;             // 64, 128 or 256
+  int BM, BN;         // output tile (tensor cores: 256 x {128, 256}; fp32 SIMT: 128 x 128)
+  int sym;            // symmetric output: only tiles with tm <= tn (tiles_m == tiles_n)
   int tiles_m, tiles_n;
   int batch;          // problems of this group in the launch
   int tile_start;     // first global tile index of this group

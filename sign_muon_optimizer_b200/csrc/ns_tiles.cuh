@@ -32,15 +32,26 @@ __device__ __forceinline__ TileCoord decode_tile(const GemmArgs& a, int tile) {
   while (t + 1 < a.n_tile_groups && a.tiles[t + 1].tile_start <= tile) ++t;
   const TileGroup tg = a.tiles[t];
   const int local = tile - tg.tile_start;
-  const int per = tg.tiles_m * tg.tiles_n;
+  const int per = tg.sym ? tg.tiles_m * (tg.tiles_m + 1) / 2 : tg.tiles_m * tg.tiles_n;
   TileCoord c;
   c.tg = t;
   c.group = tg.group;
   c.b = local / per;
-  const int rem = local - c.b * per;
-  const int tm = rem / tg.tiles_n;
-  c.m0 = tm * 128;
-  c.n0 = (rem - tm * tg.tiles_n) * tg.BN;
+  int rem = local - c.b * per;
+  int tm, tn;
+  if (tg.sym) {  // row tm holds the tiles tn = tm .. tiles_m-1
+    tm = 0;
+    while (rem >= tg.tiles_m - tm) {
+      rem -= tg.tiles_m - tm;
+      ++tm;
+    }
+    tn = tm + rem;
+  } else {
+    tm = rem / tg.tiles_n;
+    tn = rem - tm * tg.tiles_n;
+  }
+  c.m0 = tm * tg.BM;
+  c.n0 = tn * tg.BN;
   c.Mdim = tg.Mdim;
   c.Ndim = tg.Ndim;
   c.Kdim = tg.Kdim;

@@ -14,15 +14,16 @@ namespace {
 
 int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
 
-// Output tile width for the tensor-core kernel: wider tiles keep shared
-// memory below its bandwidth limit (N=256 reads 96 B/clk of operands, N=64
-// 192 B/clk), narrower ones waste less on ragged edges.
+// Output tile width for the 2-SM tensor-core kernel (256 rows per CTA pair):
+// N=256 moves the fewest operand bytes per flop, N=128 wastes less on ragged
+// edges.
 int pick_bn(int n) {
-  const int cand[3] = {256, 128, 64};
-  const double speed[3] = {1.0, 0.9, 0.6};
-  int best = 256;
+  const int cand[2] = {256, 128};
+  const double speed[2] = {1.0, 0.85};
+  int best = 128;
   double best_eff = -1.0;
-  for (int i = 0; i < 3; ++i) {
+  for (int i = 0; i < 2; ++i) {
+    if (cand[i] > SM_TC_BN_MAX) continue;
     const int64_t tiles = (n + cand[i] - 1) / cand[i];
     const double eff = (double)n / (double)(tiles * cand[i]) * speed[i];
     if (eff > best_eff + 1e-9) {
@@ -49,9 +50,12 @@ void build_tiles(Plan& p, int op, int nw, TileTable* tt) {
       t.Ndim = g.cols;
       t.Kdim = g.g;
     }
+    t.BM = p.fp32 ? 128 : 256;
     t.BN = p.fp32 ? 128 : pick_bn(t.Ndim);
-    t.tiles_m = (t.Mdim + 127) / 128;
+    t.tiles_m = (t.Mdim + t.BM - 1) / t.BM;
     t.tiles_n = (t.Ndim + t.BN - 1) / t.BN;
+    // the Gram X X^T is symmetric: with square tiles only the upper ones run
+    t.sym = (op == OP_GRAM && !p.fp32 && t.BM == t.BN) ? 1 : 0;
     t.batch = nw * g.count;
     v.push_back(t);
   }
@@ -60,7 +64,8 @@ void build_tiles(Plan& p, int op, int nw, TileTable* tt) {
   int start = 0;
   for (auto& t : v) {
     t.tile_start = start;
-    start += t.tiles_m * t.tiles_n * t.batch;
+    const int per = t.sym ? t.tiles_m * (t.tiles_m + 1) / 2 : t.tiles_m * t.tiles_n;
+    start += per * t.batch;
   }
   tt->groups = v;
   tt->total = start;
@@ -187,7 +192,7 @@ int make_plan(const int64_t* shapes, int n_mats, int M, int K, int scale, int P,
     bytes += (int64_t)p.chunks.size() * M * 4;            // norm partials
     bytes += (int64_t)M * n_mats * (4 + 8 + 8);           // scales, coefficients
     bytes += 2 * p.u_elems * 4;                           // power-iteration vectors
-    bytes += (int64_t)p.groups.size() * 4 * 128;          // tensor maps
+    bytes += (int64_t)p.groups.size() * 8 * 128;          // tensor maps
   }
   p.device_bytes = bytes;
   (void)K;

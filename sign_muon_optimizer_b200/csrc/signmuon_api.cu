@@ -147,13 +147,14 @@ EncodeTiledFn get_encode() {
 }
 
 // 3-D bf16 tensor map over `batch` matrices of rows x cols (row stride ld),
-// 64x64 boxes with the 128-byte swizzle; out-of-range boxes read zeros.
-int encode_map(signmuon_t h, CUtensorMap* m, void* base, int cols, int rows, int ld, int batch) {
+// boxes of 64 columns x box_rows rows with the 128-byte swizzle;
+// out-of-range parts of a box read as zeros and are not written.
+int encode_map(signmuon_t h, CUtensorMap* m, void* base, int cols, int rows, int ld, int batch, int box_rows) {
   EncodeTiledFn fn = get_encode();
   if (!fn) return fail(h, SIGNMUON_E_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)batch};
   cuuint64_t strides[2] = {(cuuint64_t)ld * 2, (cuuint64_t)rows * ld * 2};
-  cuuint32_t box[3] = {64, 64, 1};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
   cuuint32_t es[3] = {1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, es,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -243,7 +244,7 @@ void gemm(signmuon_t h, int op, int slot, int src, int nw, const float2* coef, f
   a.final_out = final_out ? 1 : 0;
   a.err = h->status + 1;
   (void)nw;
-  ProfScope ps(h, nw == 1 ? 7 : 2);
+  ProfScope ps(h, (nw == 1 ? 9 : 2) + op);
   if (p.fp32) sm::launch_gemm_simt(h->stream, a, 1);
   else sm::launch_gemm_tc(h->stream, a, h->d_maps, h->n_sm);
 }
@@ -252,7 +253,7 @@ void power_iteration(signmuon_t h, int nw) {
   const Plan& p = h->plan;
   const int nprob = nw * p.n_mats;
   const int nrows = nw == 1 ? p.n_pi_rows_one : (int)p.pi_rows.size();
-  ProfScope ps(h, 3);
+  ProfScope ps(h, 5);
   sm::launch_pi_init(h->stream, nprob, h->d_uoff, h->d_prob_g, h->pi_u);
   for (int it = 0; it < h->P; ++it) {
     sm::launch_pi_matvec(h->stream, h->d_pi_rows, nrows, h->A, p.fp32 ? 0 : 1, h->d_prob_aoff, h->d_prob_g,
@@ -274,7 +275,7 @@ void run_ns(signmuon_t h, int nw, const sm::WorkerPtrs& kzero_in, float* out, in
       gemm(h, sm::OP_GRAM, slot, 0, nw, nullptr, 0.f, 0.f, false, nullptr, 0);
       power_iteration(h, nw);
     }
-    ProfScope ps(h, 9);
+    ProfScope ps(h, 13);
     sm::launch_scale_flat(h->stream, kzero_in, nw, out, out_stride, h->d_chunks, (int)p.chunks.size(), h->d_mats,
                           p.n_mats, h->scale_v, h->eps);
     return;
@@ -459,18 +460,24 @@ int signmuon_init(signmuon_t* out, const int64_t* shapes, int n_mats, int M, flo
       cudaMemset(h->scale_v, 0, (size_t)M * p.n_mats * 4) != cudaSuccess)
     return bail(fail(h, SIGNMUON_E_CUDA, "memset"));
   if (!p.fp32) {
-    std::vector<CUtensorMap> maps(p.groups.size() * 4);
+    // per group: slots 0..3 = X ping, X pong, A, B with 64-row boxes;
+    // slots 4..7 = the same tensors with 128-row boxes
+    std::vector<CUtensorMap> maps(p.groups.size() * 8);
     for (size_t g = 0; g < p.groups.size(); ++g) {
       const sm::GroupInfo& gi = p.groups[g];
       const int batch = M * gi.count;
-      for (int i = 0; i < 2; ++i) {
-        void* xb = reinterpret_cast<__nv_bfloat16*>(h->X[i]) + gi.x_base;
-        if ((rc = encode_map(h, &maps[g * 4 + i], xb, gi.cols, gi.rows, gi.ld, batch))) return bail(rc);
+      for (int box = 0; box < 2; ++box) {
+        const int br = box ? 128 : 64;
+        CUtensorMap* mm = &maps[g * 8 + 4 * box];
+        for (int i = 0; i < 2; ++i) {
+          void* xb = reinterpret_cast<__nv_bfloat16*>(h->X[i]) + gi.x_base;
+          if ((rc = encode_map(h, &mm[i], xb, gi.cols, gi.rows, gi.ld, batch, br))) return bail(rc);
+        }
+        void* ab = reinterpret_cast<__nv_bfloat16*>(h->A) + gi.a_base;
+        void* bb = reinterpret_cast<__nv_bfloat16*>(h->B) + gi.a_base;
+        if ((rc = encode_map(h, &mm[2], ab, gi.g, gi.g, gi.gld, batch, br))) return bail(rc);
+        if ((rc = encode_map(h, &mm[3], bb, gi.g, gi.g, gi.gld, batch, br))) return bail(rc);
       }
-      void* ab = reinterpret_cast<__nv_bfloat16*>(h->A) + gi.a_base;
-      void* bb = reinterpret_cast<__nv_bfloat16*>(h->B) + gi.a_base;
-      if ((rc = encode_map(h, &maps[g * 4 + 2], ab, gi.g, gi.g, gi.gld, batch))) return bail(rc);
-      if ((rc = encode_map(h, &maps[g * 4 + 3], bb, gi.g, gi.g, gi.gld, batch))) return bail(rc);
     }
     uint8_t* m = nullptr;
     if ((rc = dalloc(h, &m, (int64_t)(maps.size() * sizeof(CUtensorMap) + 128)))) return bail(rc);
@@ -516,26 +523,26 @@ int signmuon_step(signmuon_t h, float* W, const float* const* G, float eta) {
   fro_finalize(h, h->M);
   run_ns(h, h->M, strided_ptrs(h->Mom, p.dpad, h->M), h->U, p.dpad);
   {
-    ProfScope ps(h, 4);
+    ProfScope ps(h, 6);
     sm::launch_pack(s, h->U, p.dpad, p.d, h->bits, p.nb_pad, h->M);
   }
   if (h->flags & SIGNMUON_POST_POLAR) {
     {
-      ProfScope ps(h, 5);
+      ProfScope ps(h, 7);
       sm::launch_vote_major(s, h->bits, p.nb_pad, h->M, p.d, h->D);
     }
     const sm::WorkerPtrs dp = strided_ptrs(h->D, 0, 1);
     {
-      ProfScope ps(h, 6);
+      ProfScope ps(h, 8);
       sm::launch_stage(s, dp, 1, h->X[0], p.fp32 ? 0 : 1, h->d_chunks, (int)p.chunks.size(), h->d_mats,
                        h->d_groups, h->partials);
     }
     fro_finalize(h, 1);
     run_ns(h, 1, dp, h->D, 0);
-    ProfScope ps(h, 8);
+    ProfScope ps(h, 12);
     sm::launch_update(s, W, h->D, p.d, eta, h->status);
   } else {
-    ProfScope ps(h, 5);
+    ProfScope ps(h, 7);
     sm::launch_vote_update(s, h->bits, p.nb_pad, h->M, p.d, W, eta, h->status);
   }
   return finish(h, (h->flags & SIGNMUON_ASYNC) == 0);
@@ -709,6 +716,34 @@ int signmuon_profile_read(signmuon_t h, double* ms, int64_t* launches, int n) {
     h->prof_ms[k] = 0.0;
     h->prof_n[k] = 0;
   }
+  return SIGNMUON_OK;
+}
+
+int signmuon_get_gram(signmuon_t h, int m, int mat, float* dst_host) {
+  int rc = check_handle(h, true);
+  if (rc) return rc;
+  const Plan& p = h->plan;
+  if (m < 0 || m >= h->M || mat < 0 || mat >= p.n_mats || !dst_host)
+    return fail(h, SIGNMUON_E_INVALID, "bad worker/matrix index or null dst");
+  const sm::MatInfo& mi = p.mats[mat];
+  const sm::GroupInfo& g = p.groups[mi.group];
+  const int64_t off = g.a_base + (int64_t)(m * g.count + mi.q) * g.g * g.gld;
+  const size_t esz = p.fp32 ? 4 : 2;
+  std::vector<uint8_t> buf((size_t)g.g * g.gld * esz);
+  CK(h, cudaStreamSynchronize(h->stream));
+  CK(h, cudaMemcpy(buf.data(), reinterpret_cast<uint8_t*>(h->A) + off * esz, buf.size(), cudaMemcpyDeviceToHost));
+  for (int r = 0; r < g.g; ++r)
+    for (int c = 0; c < g.g; ++c) {
+      const size_t i = (size_t)r * g.gld + c;
+      if (p.fp32) {
+        dst_host[(size_t)r * g.g + c] = reinterpret_cast<const float*>(buf.data())[i];
+      } else {
+        const uint32_t bits = (uint32_t)reinterpret_cast<const uint16_t*>(buf.data())[i] << 16;
+        float f;
+        std::memcpy(&f, &bits, 4);
+        dst_host[(size_t)r * g.g + c] = f;
+      }
+    }
   return SIGNMUON_OK;
 }
 

@@ -47,3 +47,16 @@ def assert_polar_close(u_gpu, u_ref, precision, what=""):
     n_dis, n = sign_disagreement(u_gpu, u_ref)
     assert n_dis <= SIGN_FRAC * n, f"{what}: {n_dis} sign disagreements of {n} entries"
     return err, n_dis, n
+
+
+def assert_momentum_close(got, mom0, g, w, beta, lam):
+    """fp32 momentum against float64: at most a few fp32 roundings of the
+    terms beta*|Mom|, (1-beta)*|G|, (1-beta)*lambda*|W| (unit roundoff 2^-24)."""
+    mom0 = np.asarray(mom0, np.float64)
+    g = np.asarray(g, np.float64)
+    w = np.asarray(w, np.float64)
+    want = ref.momentum_update(mom0, g, w, beta, lam)
+    scale = beta * np.abs(mom0) + (1 - beta) * (np.abs(g) + lam * np.abs(w)) + np.abs(want)
+    err = np.abs(np.asarray(got, np.float64) - want)
+    bad = err > 4 * 2.0 ** -24 * scale + 1e-30
+    assert not bad.any(), f"{bad.sum()} momentum entries off; worst {err[bad].max():.3e}"

@@ -13,7 +13,7 @@ import pytest
 import synth
 from oracle import signmuon_ref as ref
 
-from gpu_helpers import assert_polar_close, dev, host, oracle_polar_flat
+from gpu_helpers import assert_momentum_close, assert_polar_close, dev, host, oracle_polar_flat
 
 pytestmark = pytest.mark.gpu
 
@@ -151,5 +151,34 @@ def test_momentum_pass():
     for m in range(M):
         got = torch.zeros(d, device="cuda")
         h.get_momentum(m, got)
-        want = ref.momentum_update(mom0[m], G[m], w, 0.9, 0.01)
-        assert np.max(np.abs(host(got) - want) / (np.abs(want) + 1e-3)) < 1e-5
+        assert_momentum_close(host(got), mom0[m], G[m], w, 0.9, 0.01)
+
+
+@pytest.mark.parametrize("precision", ["bf16", "fp32"])
+@pytest.mark.parametrize("shapes", [[(200, 200), (130, 70)], [(600, 900)], [(768, 2304), (300, 64)]])
+def test_gram_matches_bf16_product(precision, shapes):
+    """The first Newton-Schulz GEMM's output (the Gram of the staged input,
+    wide orientation) against numpy on the same staged values: bf16-rounded
+    inputs with exact products, fp32-accumulated, then rounded to bf16 (or
+    kept fp32).  Covers multi-tile Grams, the mirrored upper-triangle tiles
+    and ragged edges of every 64x64 block."""
+    flags = smo.SIGNMUON_NS_FP32 if precision == "fp32" else 0
+    M = 2
+    h = smo.SignMuon(shapes, M, beta=0.9, lam=0.0, K=1, eps=1e-7, scale="fro", flags=flags)
+    xs = synth.gaussian_matrices(shapes, M, config_id=77)
+    X = [dev(x) for x in xs]
+    U = [torch.zeros_like(x) for x in X]
+    h.polar(X, U)
+    for m in range(M):
+        off = 0
+        for i, (r, c) in enumerate(shapes):
+            mat = xs[m][off: off + r * c].reshape(r, c)
+            off += r * c
+            if precision == "bf16":
+                mat = torch.from_numpy(mat).bfloat16().double().numpy()
+            wide = mat.astype(np.float64) if r <= c else mat.astype(np.float64).T
+            want = wide @ wide.T
+            got = h.get_gram(m, i).astype(np.float64)
+            tol = (2.0 ** -7 if precision == "bf16" else 1e-5) * np.abs(want).max()
+            bad = np.abs(got - want) > tol
+            assert not bad.any(), f"{r}x{c} worker {m}: {bad.sum()} Gram entries off, rows {np.nonzero(bad)[0][:5]}"

@@ -13,7 +13,7 @@ import pytest
 import synth
 from oracle import signmuon_ref as ref
 
-from gpu_helpers import assert_polar_close, dev, host
+from gpu_helpers import assert_momentum_close, assert_polar_close, dev, host
 
 pytestmark = pytest.mark.gpu
 
@@ -60,6 +60,7 @@ def _run_one_step(shapes, M, sigma, K, scale, P, precision, post_polar, seed, or
     gpu["scales"] = h.get_scales()
     want = ref.step(w0, G, mom0, shapes, beta=HP["beta"], lam=HP["lam"], eta=HP["eta"], K=K, eps=HP["eps"],
                     scale=scale, P=P, order=order, post_polar=post_polar)
+    want.update(mom0=mom0, G=G, w0=w0)
     return h, gpu, want
 
 
@@ -77,7 +78,7 @@ def _np_majority(packed_list, d):
 def _compare_step(shapes, M, gpu, want, precision, post_polar):
     d = synth.numel(shapes)
     for m in range(M):
-        assert np.max(np.abs(gpu["mom"][m] - want["mom"][m]) / (np.abs(want["mom"][m]) + 1e-3)) < 1e-5
+        assert_momentum_close(gpu["mom"][m], want["mom0"][m], want["G"][m], want["w0"], HP["beta"], HP["lam"])
         assert_polar_close(gpu["U"][m], want["U"][m], precision, f"U worker {m}")
     # the GPU's packed signs are exactly the signs of its own U (numpy check)
     for m in range(M):
