@@ -192,6 +192,35 @@ int signmuon_plan(const int64_t* shapes, int n_mats, int M, int K, int scale, in
 int signmuon_profile(signmuon_t h, int enable);
 int signmuon_profile_read(signmuon_t h, double* ms, int64_t* launches, int n);
 
+/* ------------------------------------------------------------------------
+ * signmuon_spectral_norm_noalloc -- power-iteration estimate of the largest
+ * singular value of one matrix, for callers that cannot allocate device
+ * memory (code running under CUDA graph capture, frameworks that own all
+ * device memory through their own allocator, real-time paths that must not
+ * enter the driver's allocator).  It needs no handle and allocates nothing:
+ * its working vectors live in one static device array of 1,048,576 floats
+ * (4 MiB) that every GPU loading this library holds until the process exits.
+ * The paper has no counterpart to this call; it is the step's spectral scale
+ * made available on its own.
+ *   X       device float[rows*cols], row-major.
+ *   rows, cols >= 1 with max(rows,cols) + 2*min(rows,cols) <= 1048576;
+ *           larger sizes return SIGNMUON_E_INVALID (see signmuon_last_error(NULL)).
+ *   P       power iterations >= 1.
+ *   sigma   device float[1], receives the estimate.
+ *   stream  cudaStream_t (NULL = the legacy default stream).
+ * Same estimate as the step's spectral scale: on the orientation whose small
+ * side is m, u0 = ones/sqrt(m), u <- X(X^T u)/||X(X^T u)||, P times, then
+ * sigma = ||X^T u||; computed in fp32 from X directly.
+ * The first call on a device looks up the static array's device address
+ * (and may load the library's device code); make that first call before any
+ * stream capture.  All calls share the array and every call rewrites what it
+ * reads; calls that overlap on the same GPU (for example on different
+ * streams) race on it -- serialize them.  Enqueued on
+ * `stream`; returns without waiting.
+ * ---------------------------------------------------------------------- */
+int signmuon_spectral_norm_noalloc(const float* X, int64_t rows, int64_t cols, int P, float* sigma,
+                                   void* stream);
+
 /* Number of kernels this library has launched in this process (all handles). */
 int64_t signmuon_kernel_launches(void);
 

@@ -43,6 +43,7 @@ EXPORTED = [
     "signmuon_set_ns_coeffs", "signmuon_sync", "signmuon_info", "signmuon_plan",
     "signmuon_kernel_launches", "signmuon_last_error", "signmuon_status_string", "signmuon_destroy",
     "signmuon_profile", "signmuon_profile_read", "signmuon_get_gram",
+    "signmuon_spectral_norm_noalloc",
 ]
 PROF_KINDS = ["momentum", "norm_finalize", "ns_gram", "ns_square", "ns_apply", "power_iter", "pack",
               "vote", "stage", "post_gram", "post_square", "post_apply", "update", "k0_scale"]
@@ -84,6 +85,7 @@ def _load():
         "signmuon_destroy": (None, [P]),
         "signmuon_profile": (I, [P, I]),
         "signmuon_get_gram": (I, [P, I, I, P]),
+        "signmuon_spectral_norm_noalloc": (I, [P, I64, I64, I, P, P]),
         "signmuon_profile_read": (I, [P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(I64), I]),
     }
     for name, (res, args) in sig.items():
@@ -199,6 +201,14 @@ def signmuon_get_scales(h, M, n_mats):
     out = np.zeros(M * n_mats, np.float32)
     _check(h, _lib.signmuon_get_scales(h, out.ctypes.data))
     return out.reshape(M, n_mats)
+
+
+def signmuon_spectral_norm_noalloc(X, rows, cols, P, sigma, stream=None):
+    """Power-iteration sigma of one matrix without any device allocation
+    (see include/signmuon.h); X and sigma are device buffers."""
+    if stream is None:
+        stream = _default_stream()
+    _check(None, _lib.signmuon_spectral_norm_noalloc(_ptr(X), int(rows), int(cols), int(P), _ptr(sigma), stream))
 
 
 def signmuon_get_gram(h, m, mat, g):

@@ -101,6 +101,7 @@ struct GemmArgs {
 
 // ---- launch wrappers (host) ----------------------------------------------
 void count_launch();
+void set_global_error(const char* msg);  // text for signmuon_last_error(NULL)
 
 void launch_momentum(cudaStream_t s, const WorkerPtrs& G, const float* W, float* Mom, int64_t d,
                      int M, float beta, float lambda, void* X, int x_bf16, const Chunk* chunks,

@@ -88,6 +88,12 @@ namespace {
 
 std::string g_noh_err;  // errors raised before a handle exists
 
+}  // namespace
+
+void sm::set_global_error(const char* msg) { g_noh_err = msg; }
+
+namespace {
+
 int fail(signmuon_t h, int code, const std::string& msg) {
   if (h) h->err = msg;
   else g_noh_err = msg;
