@@ -73,6 +73,12 @@ struct TileGroup {
 
 enum GemmOp { OP_GRAM = 0, OP_SQUARE = 1, OP_APPLY = 2 };
 
+// Tile and group tables small enough to travel inside the kernel
+// parameters (read through the constant cache; a per-tile decode from global
+// memory is a chain of dependent loads).
+constexpr int kParamGroups = 24;
+constexpr int kParamMats = 64;
+
 // Arguments of one grouped Newton-Schulz GEMM launch (both precisions).
 struct GemmArgs {
   const TileGroup* tiles;
@@ -97,6 +103,10 @@ struct GemmArgs {
   int64_t out_stride;
   int final_out;
   int* err;
+  int param_tables;                        // 1: the p* copies below are valid
+  TileGroup ptiles[kParamGroups];
+  GroupInfo pgroups[kParamGroups];
+  int pgroup_mats[kParamMats];
 };
 
 // ---- launch wrappers (host) ----------------------------------------------

@@ -73,12 +73,12 @@ __device__ __forceinline__ void store_slab(const Operand& o, float (*s)[TM + 4],
 }
 
 __global__ void __launch_bounds__(NT)
-k_gemm_simt(const GemmArgs a) {
+k_gemm_simt(const __grid_constant__ GemmArgs a) {
   __shared__ __align__(16) float As[2][TK][TM + 4];
   __shared__ __align__(16) float Bs[2][TK][TN + 4];
 
   const TileCoord tc = decode_tile(a, blockIdx.x);
-  const GroupInfo gi = a.groups[tc.group];
+  const GroupInfo gi = group_info(a, tc.group);
   int mat = 0;
   const int p = problem_id(a, gi, tc.b, &mat);
   const int op = a.op;

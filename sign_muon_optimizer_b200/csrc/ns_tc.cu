@@ -11,8 +11,8 @@
 // 2*128*BN*64 flops (a one-SM 128 x BN tile needs 48 KB).  Per CTA, 192
 // threads:
 //   warp 0      TMA producer: bf16 boxes of 64 columns (128-byte swizzle)
-//               into a STAGES-deep ring; both CTAs' loads complete on the
-//               leader CTA's "full" barrier
+//               into a 5-deep (Gram) or 3-deep ring; both CTAs' loads
+//               complete on the leader CTA's "full" barrier
 //   warp 1      allocates 512 TMEM columns (cta_group::2); in the leader CTA
 //               one lane issues tcgen05.mma.cta_group::2 (M=256, N=BN, K=16)
 //               and tcgen05.commit multicast to both CTAs' barriers
@@ -31,16 +31,22 @@
 namespace sm {
 namespace {
 
-constexpr int BK = 64, STAGES = SM_TC_STAGES;
+constexpr int BK = 64;
 constexpr int BOX_BYTES = 64 * 64 * 2;                  // one 64x64 bf16 TMA box
 constexpr int A_BYTES = 128 * BK * 2;                   // 16 KB: this CTA's 128 rows of A
 constexpr int B_BYTES = 128 * BK * 2;                   // 16 KB: this CTA's BN/2 <= 128 rows of B
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int EPI_BYTES = 128 * 256 * 2;                // 64 KB: the affine operand tile
+constexpr int EPI_BYTES = 128 * 256 * 2;                // 64 KB: one staging tile
+// Shared memory is split per GEMM role: the Gram runs a 5-deep operand ring
+// and one staging tile; SQUARE/APPLY a 3-deep ring and two staging tiles so
+// that the next tile's affine operand loads while this tile is processed.
+constexpr int RING_GRAM = 5, RING_AFFINE = 3, RING_MAX = 5;
+constexpr int DATA_BYTES = RING_GRAM * STAGE_BYTES + EPI_BYTES;   // 224 KB either way
+static_assert(RING_AFFINE * STAGE_BYTES + 2 * EPI_BYTES == DATA_BYTES, "smem split");
 constexpr int TMEM_COLS = 512;
 constexpr int NTHREADS = 320;   // producer, MMA, 8 epilogue warps
 constexpr unsigned long long kTimeoutNs = 2000000000ull;  // 2 s
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+constexpr int SMEM_BYTES = DATA_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -214,29 +220,31 @@ __device__ __forceinline__ const CUtensorMap* map_at(const CUtensorMap* maps, in
 __device__ __forceinline__ const CUtensorMap* map128(const CUtensorMap* m) { return m + 4; }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
-k_gemm_tc(const GemmArgs a, const CUtensorMap* __restrict__ maps) {
+k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ maps) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* gbase = smem_raw + (base - raw);
-  const uint32_t epi = base + STAGES * STAGE_BYTES;     // affine operand tile
-  const uint8_t* epi_ptr = gbase + STAGES * STAGE_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(gbase + STAGES * STAGE_BYTES + EPI_BYTES);
-  // bars: full[STAGES], empty[STAGES], tmem_full[2], tmem_empty[2], epi_full
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+  const int op = a.op;
+  const int nst = (op == OP_GRAM) ? RING_GRAM : RING_AFFINE;   // operand ring depth
+  const uint32_t epi0 = base + nst * STAGE_BYTES;              // staging tile(s)
+  uint8_t* const epi_ptr0 = gbase + nst * STAGE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(gbase + DATA_BYTES);
+  // bars: full[RING_MAX], empty[RING_MAX], tmem_full[2], tmem_empty[2], epi_full[2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * RING_MAX + 6);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const uint32_t bar0 = smem_addr(bars);
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
-  auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
-  auto tfull_bar = [&](int s) { return bar0 + 8u * (2 * STAGES + s); };
-  auto tempty_bar = [&](int s) { return bar0 + 8u * (2 * STAGES + 2 + s); };
-  const uint32_t efull_bar = bar0 + 8u * (2 * STAGES + 4);
+  auto empty_bar = [&](int s) { return bar0 + 8u * (RING_MAX + s); };
+  auto tfull_bar = [&](int s) { return bar0 + 8u * (2 * RING_MAX + s); };
+  auto tempty_bar = [&](int s) { return bar0 + 8u * (2 * RING_MAX + 2 + s); };
+  auto efull_bar = [&](int b) { return bar0 + 8u * (2 * RING_MAX + 4 + b); };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();          // 0 = leader (issues the MMAs)
   const int cid = (int)cluster_id_x(), ncl = (int)n_clusters_x();
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < RING_MAX; ++s) {
       mbar_init(full_bar(s), 1);
       mbar_init(empty_bar(s), 1);
     }
@@ -244,7 +252,8 @@ k_gemm_tc(const GemmArgs a, const CUtensorMap* __restrict__ maps) {
       mbar_init(tfull_bar(s), 1);
       mbar_init(tempty_bar(s), 16);  // 8 epilogue warps in each CTA of the pair
     }
-    mbar_init(efull_bar, 1);
+    mbar_init(efull_bar(0), 1);
+    mbar_init(efull_bar(1), 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -259,7 +268,6 @@ k_gemm_tc(const GemmArgs a, const CUtensorMap* __restrict__ maps) {
   cluster_sync();   // the peer's barriers are initialised before any remote arrive
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int op = a.op;
 
   if (warp == 0) {
     // ---------------- TMA producer (both CTAs) ----------------
@@ -270,7 +278,7 @@ k_gemm_tc(const GemmArgs a, const CUtensorMap* __restrict__ maps) {
       bool ok = true;
       for (int tile = cid; tile < a.total_tiles && ok; tile += ncl) {
         const TileCoord tc = decode_tile(a, tile);
-        const GroupInfo gi = a.groups[tc.group];
+        const GroupInfo gi = group_info(a, tc.group);
         const int nk = (tc.Kdim + BK - 1) / BK;
         const int amn = a_is_mn(op, gi.wide), bmn = b_is_mn(op, gi.wide);
         const CUtensorMap* mA;
@@ -311,12 +319,12 @@ k_gemm_tc(const GemmArgs a, const CUtensorMap* __restrict__ maps) {
           }
           issued |= 1u << stage;
           last_par = (last_par & ~(1u << stage)) | (phase << stage);
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          if (++stage == nst) { stage = 0; phase ^= 1u; }
         }
       }
       if (!ok && rank == 0) {
         // drain: every issued stage's last loads must land before teardown
-        for (int s = 0; s < STAGES; ++s) {
+        for (int s = 0; s < nst; ++s) {
           if (!(issued & (1u << s))) continue;
           const uint32_t par = (last_par >> s) & 1u;
           const uint64_t t0 = globaltimer();
@@ -337,7 +345,7 @@ k_gemm_tc(const GemmArgs a, const CUtensorMap* __restrict__ maps) {
       bool ok = true;
       for (int tile = cid; tile < a.total_tiles && ok; tile += ncl) {
         const TileCoord tc = decode_tile(a, tile);
-        const GroupInfo gi = a.groups[tc.group];
+        const GroupInfo gi = group_info(a, tc.group);
         const int nk = (tc.Kdim + BK - 1) / BK;
         const int amn = a_is_mn(op, gi.wide), bmn = b_is_mn(op, gi.wide);
         const uint32_t idesc = instr_desc(amn, bmn, tc.BN);
@@ -356,7 +364,7 @@ k_gemm_tc(const GemmArgs a, const CUtensorMap* __restrict__ maps) {
             tc_mma(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
           }
           tc_commit_pair(empty_bar(stage));
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          if (++stage == nst) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
         tc_commit_pair(tfull_bar(acc));
@@ -373,22 +381,37 @@ k_gemm_tc(const GemmArgs a, const CUtensorMap* __restrict__ maps) {
   } else {
     // ---------------- epilogue (warps 2..9, both CTAs) ----------------
     // Two warps per TMEM lane quarter, each taking half of the tile's columns.
-    // The CTA's 128 x BN output tile is staged in shared memory in the same
-    // swizzled 64x64-box layout that TMA reads and writes: SQUARE/APPLY first
-    // load their affine operand there, each thread overwrites its operand
-    // chunk with the result, and one thread stores the tile with TMA.
+    // The CTA's 128 x BN output tile is staged in shared memory in the
+    // swizzled box layout that TMA reads and writes: SQUARE/APPLY load their
+    // affine operand there (one tile ahead, alternating two staging tiles),
+    // each thread overwrites its operand chunk with the result, and one
+    // thread stores the tile with TMA.
     const int q = warp & 3;                // TMEM lane quarter this warp may access
     const int half = (warp - 2) >> 2;      // column half of the tile
     const int rloc = q * 32 + lane;        // row within this CTA's 128 rows
     const bool leader_thr = (warp == 2 && lane == 0);
+    const bool affine = op != OP_GRAM;
+    const bool final_out = (op == OP_APPLY) && a.final_out;
     const uint32_t tempty_leader0 = leader_addr(tempty_bar(0));
     const uint32_t tempty_leader1 = leader_addr(tempty_bar(1));
+    // operand load of `tile` into staging tile `b` (leader thread)
+    auto load_operand = [&](int tile, int b) {
+      const TileCoord t2 = decode_tile(a, tile);
+      const CUtensorMap* mO = (op == OP_SQUARE) ? map_at(maps, t2.group, 2) : map_at(maps, t2.group, a.map_src);
+      const int rb = t2.m0 + 128 * (int)rank;
+      mbar_expect_tx(efull_bar(b), (uint32_t)(t2.BN / 64) * 2u * BOX_BYTES);
+      for (int j = 0; j < t2.BN / 64; ++j)
+        tma_load_local(epi0 + (uint32_t)b * EPI_BYTES + (uint32_t)j * 2u * BOX_BYTES, map128(mO), efull_bar(b),
+                       t2.n0 + 64 * j, rb, t2.b);
+    };
+    if (affine && leader_thr && cid < a.total_tiles) load_operand(cid, 0);
     int acc = 0;
     uint32_t acc_phase = 0;
-    uint32_t e_phase = 0;
-    for (int tile = cid; tile < a.total_tiles; tile += ncl) {
+    uint32_t e_phase = 0;       // bit b: phase of staging tile b's operand barrier
+    int li = 0;                 // tiles handled by this CTA
+    for (int tile = cid; tile < a.total_tiles; tile += ncl, ++li) {
       const TileCoord tc = decode_tile(a, tile);
-      const GroupInfo gi = a.groups[tc.group];
+      const GroupInfo gi = group_info(a, tc.group);
       int mat = 0;
       const int p = problem_id(a, gi, tc.b, &mat);
       float c0 = a.c0, c1 = a.c1;
@@ -397,31 +420,27 @@ k_gemm_tc(const GemmArgs a, const CUtensorMap* __restrict__ maps) {
         c0 = cf.x;
         c1 = cf.y;
       }
+      const int buf = affine ? (li & 1) : 0;
+      uint8_t* const epi_ptr = epi_ptr0 + buf * EPI_BYTES;
+      const uint32_t epi = epi0 + (uint32_t)buf * EPI_BYTES;
       const int rbase = tc.m0 + 128 * (int)rank;
       const int row = rbase + rloc;
       const bool row_ok = row < tc.Mdim;
       const int64_t aoff = gi.a_base + (int64_t)tc.b * gi.g * gi.gld;
       const int w = tc.b / gi.count;
       const int nch = tc.BN / 32;
-      const bool affine = op != OP_GRAM;
-      const bool final_out = (op == OP_APPLY) && a.final_out;
-      // the staging tile is free once the previous tile's TMA store has read it
-      if (leader_thr) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-      // ... and every epilogue warp is past it; stop together if a wait gave up
+      // Gram: the single staging tile is free once the previous tile's TMA
+      // store has read it (affine roles wait for this one tile later)
+      if (!affine && leader_thr) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+      // every epilogue warp is here; stop together if a wait gave up
       if (epi_bar_or(*abort_flag != 0)) break;
-      if (affine && leader_thr) {
-        const CUtensorMap* mO = (op == OP_SQUARE) ? map_at(maps, tc.group, 2) : map_at(maps, tc.group, a.map_src);
-        mbar_expect_tx(efull_bar, (uint32_t)(tc.BN / 64) * 2u * BOX_BYTES);
-        for (int j = 0; j < tc.BN / 64; ++j)
-          tma_load_local(epi + (uint32_t)j * 2u * BOX_BYTES, map128(mO), efull_bar, tc.n0 + 64 * j, rbase, tc.b);
-      }
       int okw = 1;
       if (lane == 0) {
         okw = mbar_wait(tfull_bar(acc), acc_phase, abort_flag, a.err) ? 1 : 0;
-        if (okw && affine) okw = mbar_wait(efull_bar, e_phase, abort_flag, a.err) ? 1 : 0;
+        if (okw && affine) okw = mbar_wait(efull_bar(buf), (e_phase >> buf) & 1u, abort_flag, a.err) ? 1 : 0;
       }
       okw = __shfl_sync(0xffffffffu, okw, 0);
-      if (affine) e_phase ^= 1u;
+      if (affine) e_phase ^= 1u << buf;
       // collective: if any warp's wait gave up, all skip to the next barrier,
       // which then stops them together
       if (epi_bar_or(!okw)) continue;
@@ -493,6 +512,7 @@ k_gemm_tc(const GemmArgs a, const CUtensorMap* __restrict__ maps) {
           // one 64-column x 128-row box per store, each in its own bulk
           // group (several vertically adjacent boxes in one group were seen
           // to lose all but the first on this hardware)
+          int groups = 0;
           if (rbase < tc.Mdim) {
             for (int j = 0; j < tc.BN / 64; ++j) {
               const int x = tc.n0 + 64 * j;
@@ -503,9 +523,26 @@ k_gemm_tc(const GemmArgs a, const CUtensorMap* __restrict__ maps) {
                   "r"(epi + (uint32_t)j * 2u * BOX_BYTES)
                   : "memory");
               asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+              ++groups;
             }
           }
+          if (affine) {
+            // the other staging tile is free once the previous tile's stores
+            // (all groups but this tile's) have read it; then prefetch the
+            // next tile's operand into it
+            switch (groups) {
+              case 0: asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); break;
+              case 1: asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); break;
+              case 2: asm volatile("cp.async.bulk.wait_group.read 2;" ::: "memory"); break;
+              case 3: asm volatile("cp.async.bulk.wait_group.read 3;" ::: "memory"); break;
+              default: asm volatile("cp.async.bulk.wait_group.read 4;" ::: "memory"); break;
+            }
+            if (tile + ncl < a.total_tiles) load_operand(tile + ncl, buf ^ 1);
+          }
         }
+      } else if (affine && leader_thr) {
+        // final APPLY (no stores): prefetch the next tile's operand
+        if (tile + ncl < a.total_tiles) load_operand(tile + ncl, buf ^ 1);
       }
     }
     if (leader_thr) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");

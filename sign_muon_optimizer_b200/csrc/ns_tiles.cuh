@@ -27,10 +27,18 @@ struct TileCoord {
   int Mdim, Ndim, Kdim, BN;
 };
 
+__device__ __forceinline__ const TileGroup* tile_table(const GemmArgs& a) {
+  return a.param_tables ? a.ptiles : a.tiles;
+}
+__device__ __forceinline__ const GroupInfo& group_info(const GemmArgs& a, int g) {
+  return a.param_tables ? a.pgroups[g] : a.groups[g];
+}
+
 __device__ __forceinline__ TileCoord decode_tile(const GemmArgs& a, int tile) {
+  const TileGroup* tiles = tile_table(a);
   int t = 0;
-  while (t + 1 < a.n_tile_groups && a.tiles[t + 1].tile_start <= tile) ++t;
-  const TileGroup tg = a.tiles[t];
+  while (t + 1 < a.n_tile_groups && tiles[t + 1].tile_start <= tile) ++t;
+  const TileGroup tg = tiles[t];
   const int local = tile - tg.tile_start;
   const int per = tg.sym ? tg.tiles_m * (tg.tiles_m + 1) / 2 : tg.tiles_m * tg.tiles_n;
   TileCoord c;
@@ -63,7 +71,7 @@ __device__ __forceinline__ TileCoord decode_tile(const GemmArgs& a, int tile) {
 __device__ __forceinline__ int problem_id(const GemmArgs& a, const GroupInfo& gi, int b, int* mat_out) {
   const int w = b / gi.count;
   const int q = b - w * gi.count;
-  const int mat = a.group_mats[gi.first + q];
+  const int mat = a.param_tables ? a.pgroup_mats[gi.first + q] : a.group_mats[gi.first + q];
   *mat_out = mat;
   return w * a.n_mats + mat;
 }

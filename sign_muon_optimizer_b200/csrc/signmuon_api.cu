@@ -250,6 +250,14 @@ void gemm(signmuon_t h, int op, int slot, int src, int nw, const float2* coef, f
   a.final_out = final_out ? 1 : 0;
   a.err = h->status + 1;
   (void)nw;
+  const auto& tg = p.tiles[op][slot].groups;
+  if ((int)tg.size() <= sm::kParamGroups && (int)p.groups.size() <= sm::kParamGroups &&
+      p.n_mats <= sm::kParamMats) {
+    a.param_tables = 1;
+    for (size_t i = 0; i < tg.size(); ++i) a.ptiles[i] = tg[i];
+    for (size_t i = 0; i < p.groups.size(); ++i) a.pgroups[i] = p.groups[i];
+    for (int i = 0; i < p.n_mats; ++i) a.pgroup_mats[i] = p.group_mats[i];
+  }
   ProfScope ps(h, (nw == 1 ? 9 : 2) + op);
   if (p.fp32) sm::launch_gemm_simt(h->stream, a, 1);
   else sm::launch_gemm_tc(h->stream, a, h->d_maps, h->n_sm);
