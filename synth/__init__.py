@@ -178,6 +178,14 @@ def device_gradients(shapes, M, sigma, step, config_id=0, device="cuda", out=Non
     return out
 
 
+def device_gaussian(d, M, seed=0, device="cuda"):
+    """(M, d) float32 i.i.d. N(0,1) on the device (NS sweep momentum)."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(int(np.random.SeedSequence([int(seed), 9]).generate_state(1)[0]))
+    return torch.randn((M, d), generator=g, device=device, dtype=torch.float32)
+
+
 def device_weights0(shapes, config_id=0, device="cuda"):
     import torch
     d = numel(shapes)
