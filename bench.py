@@ -57,6 +57,19 @@ def peaks():
     return FALLBACK, "fallback"
 
 
+def gemm_traffic_from_profile():
+    """DRAM bytes per Newton-Schulz GEMM launch from the committed ncu summary
+    (a 2-layer capture scaled to the full workload), or None."""
+    p = os.path.join(ROOT, "profiles", "k_gemm_tc_nanogpt_2layers.md")
+    try:
+        for line in open(p):
+            if line.startswith("traffic per full-size launch (bytes):"):
+                return float(line.split(":", 1)[1])
+    except OSError:
+        pass
+    return None
+
+
 def ns_flops_per_step(shapes, M, K, post_polar):
     """Algorithmic Newton-Schulz flops: per matrix and cubic iteration two
     GEMMs, X X^T (2 m^2 n) and A X (2 m^2 n), m = min dim, n = max dim."""
@@ -82,6 +95,23 @@ def hbm_bytes_per_step(shapes, M, P, post_polar):
     if post_polar:
         b["power_iter"] += (P + 1) * gram_bytes(shapes)
     return b
+
+
+def max_over_ranks(x, device="cpu"):
+    """The maximum of a per-rank float over all ranks of the process group
+    (the slowest rank's time); the value itself on a single process."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, steps, ms):
+    """Whole-job steps/s: every rank runs ``steps`` steps; ``ms`` is the max over ranks."""
+    return world * steps / (ms / 1e3)
 
 
 # ---------------------------------------------------------------------------
@@ -265,13 +295,9 @@ def run_ours(args):
     launches = smo.signmuon_kernel_launches() - launches0
     prof = opt.profile_read()
     opt.profile(False)
-    ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ev0.elapsed_time(ev1), "cuda")
     ms_per_step = ms / args.steps
-    value = world * args.steps / (ms / 1e3)
+    value = job_throughput(world, args.steps, ms)
 
     pk, pk_kind = peaks()
     steps = args.steps
@@ -283,7 +309,7 @@ def run_ours(args):
     peak_tc = pk["bf16_tflops_sustained"]
     roofline = {"kernel": "k_gemm_tc (grouped Newton-Schulz GEMM, tcgen05)", "bound": "tensor",
                 "achieved": tflops, "peak": peak_tc, "unit": "TFLOP/s",
-                "frac": (tflops / peak_tc) if tflops else None, "traffic": None,
+                "frac": (tflops / peak_tc) if tflops else None, "traffic": gemm_traffic_from_profile(),
                 "peak_kind": f"bf16 sustained, {pk_kind}",
                 "flops_per_launch": flops / max(1, gemm_launches / steps),
                 "avg_launch_ms": gemm_ms / max(1, gemm_launches)}
@@ -324,12 +350,8 @@ def run_ours(args):
         ev1.record(stream)
         torch.cuda.synchronize()
         wall = time.perf_counter() - t0
-        ems = max(ev0.elapsed_time(ev1), wall * 1e3)
-        if world > 1:
-            t = torch.tensor([ems], device="cuda", dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
-        e2e = {"value": world * args.e2e_steps / (ems / 1e3), "unit": "steps/s",
+        ems = max_over_ranks(max(ev0.elapsed_time(ev1), wall * 1e3), "cuda")
+        e2e = {"value": job_throughput(world, args.e2e_steps, ems), "unit": "steps/s",
                "h2d_bytes_per_step": (M + 1) * D * 4, "d2h_bytes_per_step": D * 4,
                "api": "signmuon_step_host (pinned host W and G)"}
         del Gh, Wh

@@ -1,0 +1,92 @@
+"""Host-side logic of bench.py: the multi-process timing reduction (world size
+2 over gloo on the CPU), the reference arm's rank handling and the
+algorithmic flop and byte counts the roofline divides by."""
+import os
+import socket
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+import synth  # noqa: E402
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, q):
+    import datetime
+
+    import torch.distributed as dist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        my_ms = [12.5, 30.25][rank]
+        ms = bench.max_over_ranks(my_ms, "cpu")
+        q.put((rank, ms, bench.job_throughput(world, 10, ms)))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_gloo_world2():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+    assert all(p.exitcode == 0 for p in procs)
+    got = sorted(q.get(timeout=5) for _ in range(2))
+    for rank, ms, value in got:
+        assert ms == 30.25                      # every rank sees the slowest rank's time
+        assert value == pytest.approx(2 * 10 / 0.03025)   # both ranks' steps over that time
+
+
+def test_max_over_ranks_single_process():
+    assert bench.max_over_ranks(7.0) == 7.0
+    assert bench.job_throughput(1, 50, 1000.0) == pytest.approx(50.0)
+
+
+def test_reference_arm_nonzero_rank_does_nothing(monkeypatch, capsys):
+    monkeypatch.setenv("RANK", "1")
+
+    class A:
+        steps, warmup, gpus = 2, 3, 2
+
+    def boom(*a, **k):
+        raise AssertionError("rank 1 must not run the oracle")
+    monkeypatch.setattr(bench, "cpu_oracle_sample", boom)
+    assert bench.run_reference(A()) == 0
+    assert capsys.readouterr().out == ""
+
+
+def test_nanogpt_flop_count():
+    # 12 layers x (768^2 x (2304 + 768 + 3072 + 3072)) x 4 flops per cubic
+    # iteration x 5 iterations x (8 workers + the post-vote problem)
+    assert bench.ns_flops_per_step(synth.NANOGPT_SHAPES, 8, 5, True) == 11_741_366_845_440
+    assert bench.ns_flops_per_step(synth.NANOGPT_SHAPES, 8, 5, False) == 8 * 1_304_596_316_160
+
+
+def test_hbm_bytes_counts():
+    d = synth.numel(synth.NANOGPT_SHAPES)
+    b = bench.hbm_bytes_per_step(synth.NANOGPT_SHAPES, 8, 2, True)
+    assert d == 84_934_656
+    assert b["momentum"] == d * 116          # W once + 8 x (G + Mom r/w + bf16 X)
+    assert b["pack"] == d * 8 * 4.125        # fp32 U read + one bit written per worker
+    assert b["vote"] == d + 4 * d            # 8 bits per entry read, fp32 D written
+    assert b["power_iter"] == 3 * 9 * 48 * 768 * 768 * 2
+
+
+def test_cpu_sample_is_one_144th():
+    assert bench.CPU_SCALE == 144.0
