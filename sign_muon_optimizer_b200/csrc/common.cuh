@@ -77,6 +77,9 @@ enum GemmOp { OP_GRAM = 0, OP_SQUARE = 1, OP_APPLY = 2 };
 // parameters (read through the constant cache; a per-tile decode from global
 // memory is a chain of dependent loads).
 constexpr int kParamGroups = 24;
+// TMA tensor maps per shape group (bf16 path): X ping/pong, A, B with 64-row,
+// 128-row and 32-row boxes.
+constexpr int kMapsPerGroup = 12;
 constexpr int kParamMats = 64;
 
 // Arguments of one grouped Newton-Schulz GEMM launch (both precisions).

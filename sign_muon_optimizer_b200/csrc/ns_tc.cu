@@ -8,18 +8,20 @@
 // all shape groups.  A cluster of two CTAs (one per SM) computes one 256 x BN
 // output tile: each CTA stages its 128 rows of the A operand and its BN/2
 // rows of the B operand, so an SM moves 32 KB per 64-deep k-block for
-// 2*128*BN*64 flops (a one-SM 128 x BN tile needs 48 KB).  Per CTA, 192
+// 2*128*BN*64 flops (a one-SM 128 x BN tile needs 48 KB).  Per CTA, 384
 // threads:
-//   warp 0      TMA producer: bf16 boxes of 64 columns (128-byte swizzle)
-//               into a 5-deep (Gram) or 3-deep ring; both CTAs' loads
-//               complete on the leader CTA's "full" barrier
-//   warp 1      allocates 512 TMEM columns (cta_group::2); in the leader CTA
+//   warps 0..2  TMA producers taking turns over the k-blocks: bf16 boxes of
+//               64 columns (128-byte swizzle) into a 5-deep ring, one box per
+//               lane; both CTAs' loads complete on the leader CTA's "full"
+//               barrier
+//   warp 3      allocates 512 TMEM columns (cta_group::2); in the leader CTA
 //               one lane issues tcgen05.mma.cta_group::2 (M=256, N=BN, K=16)
 //               and tcgen05.commit multicast to both CTAs' barriers
-//   warps 2..9  epilogue: the affine operand (X for APPLY, A for SQUARE) of
-//               the tile comes into shared memory by TMA while the MMAs run;
-//               tcgen05.ld 32x32b.x32 -> a*operand + b*acc -> bf16 results
-//               written over the operand in shared memory -> TMA store
+//   warps 4..11 epilogue, each on its own 32-row x BN/2 slice of the tile:
+//               the slice of the affine operand (X for APPLY, A for SQUARE)
+//               comes into shared memory by TMA; tcgen05.ld 32x32b.x32 ->
+//               a*operand + b*acc -> bf16 results written over the operand
+//               in shared memory -> TMA store of the slice
 // The Gram matrix is symmetric: only tiles on or above the diagonal are
 // computed, and the epilogue also writes each off-diagonal tile transposed.
 // Every mbarrier wait is bounded (2 s): on expiry the CTA records
@@ -37,14 +39,22 @@ constexpr int A_BYTES = 128 * BK * 2;                   // 16 KB: this CTA's 128
 constexpr int B_BYTES = 128 * BK * 2;                   // 16 KB: this CTA's BN/2 <= 128 rows of B
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int EPI_BYTES = 128 * 256 * 2;                // 64 KB: one staging tile
-// Shared memory is split per GEMM role: the Gram runs a 5-deep operand ring
-// and one staging tile; SQUARE/APPLY a 3-deep ring and two staging tiles so
-// that the next tile's affine operand loads while this tile is processed.
-constexpr int RING_GRAM = 5, RING_AFFINE = 3, RING_MAX = 5;
-constexpr int DATA_BYTES = RING_GRAM * STAGE_BYTES + EPI_BYTES;   // 224 KB either way
-static_assert(RING_AFFINE * STAGE_BYTES + 2 * EPI_BYTES == DATA_BYTES, "smem split");
+// Shared memory: a 5-deep operand ring and one staging tile (224 KB).
+constexpr int RING = 5, RING_MAX = RING;
+constexpr int DATA_BYTES = RING * STAGE_BYTES + EPI_BYTES;
 constexpr int TMEM_COLS = 512;
-constexpr int NTHREADS = 320;   // producer, MMA, 8 epilogue warps
+// Warp roles.  A warp completes only about one TMA load instruction every
+// 500-700 cycles however many it has in flight, while the lanes of one
+// instruction and separate warps overlap (measured on B200 with boxes of
+// 8-32 KB).  So all boxes of one k-block go out in a single instruction, one
+// box per lane, and three producer warps take turns over the k-blocks; each
+// epilogue warp loads and stores its own slice of the staging tile.  (Twelve
+// warps keep 168 registers per thread for the epilogue; from 13 warps on the
+// compiler caps them at 128.)
+constexpr int NPROD = 3;                    // producer warps 0..2
+constexpr int MMA_WARP = NPROD;             // TMEM allocation + MMA issue
+constexpr int EPI_WARP0 = NPROD + 1;        // 8 epilogue warps
+constexpr int NTHREADS = (NPROD + 1 + 8) * 32;
 constexpr unsigned long long kTimeoutNs = 2000000000ull;  // 2 s
 constexpr int SMEM_BYTES = DATA_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 
@@ -89,6 +99,25 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
 // arrive on a barrier given by its shared::cluster address (own or peer CTA)
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cl_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cl_addr) : "memory");
+}
+// Relaxed forms: no release fence in front of the arrival (a release at
+// cluster scope held the arriving warp for ~2,000 cycles).  Used where the
+// arrival orders nothing but tcgen05 reads already completed by
+// tcgen05.wait::ld, or precedes the transfer it announces.
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cl_addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cl_addr) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx_relaxed(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.relaxed.cta.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+// shared-memory 16-byte load / store by shared-window address
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
@@ -152,8 +181,8 @@ __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t
       ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum)
       : "memory");
 }
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-  uint32_t r[32];
+// tcgen05.ld without the wait; tmem_wait_ld() then reg_fence() before use
+__device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
       "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
@@ -163,24 +192,13 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
         "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
         "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// keeps the compiler from moving uses of r above the preceding wait
+__device__ __forceinline__ void reg_fence(uint32_t (&r)[32]) {
 #pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+  for (int i = 0; i < 32; ++i) asm volatile("" : "+r"(r[i]));
 }
-// Named barrier of the 8 epilogue warps, also OR-reducing a flag over them.
-__device__ __forceinline__ int epi_bar_or(int pred) {
-  int r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.b32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, 1, 256, p;\n\t"
-      "selp.b32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"(pred)
-      : "memory");
-  return r;
-}
-
 // Shared-memory matrix descriptors, 128-byte swizzle, sm_100 version bit.
 //   K-major tile:  rows of 64 bf16 (128 B), 8-row groups 1024 B apart (SBO)
 //   MN-major tile: 64-element MN blocks 8 KB apart (LBO, one TMA box each),
@@ -213,9 +231,10 @@ __device__ __forceinline__ void unpack_bf16x8(uint4 u, float* f) {
   }
 }
 // Tensor-map slots per group: 0/1 = X ping/pong, 2 = A, 3 = B, with 64-row
-// boxes; the same four with 128-row boxes at slot + 4.
+// boxes; the same four with 128-row boxes at slot + 4 and with 32-row boxes
+// (one epilogue warp's slice) at slot + 8.
 __device__ __forceinline__ const CUtensorMap* map_at(const CUtensorMap* maps, int group, int slot) {
-  return maps + group * 8 + slot;
+  return maps + group * kMapsPerGroup + slot;
 }
 __device__ __forceinline__ const CUtensorMap* map128(const CUtensorMap* m) { return m + 4; }
 
@@ -226,12 +245,12 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* gbase = smem_raw + (base - raw);
   const int op = a.op;
-  const int nst = (op == OP_GRAM) ? RING_GRAM : RING_AFFINE;   // operand ring depth
-  const uint32_t epi0 = base + nst * STAGE_BYTES;              // staging tile(s)
-  uint8_t* const epi_ptr0 = gbase + nst * STAGE_BYTES;
+  const int nst = RING;                                        // operand ring depth
+  const uint32_t epi0 = base + nst * STAGE_BYTES;              // staging tile
   uint64_t* bars = reinterpret_cast<uint64_t*>(gbase + DATA_BYTES);
-  // bars: full[RING_MAX], empty[RING_MAX], tmem_full[2], tmem_empty[2], epi_full[2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * RING_MAX + 6);
+  // bars: full[RING_MAX], empty[RING_MAX], tmem_full[2], tmem_empty[2],
+  // epi_full[8] (one per epilogue warp)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * RING_MAX + 12);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const uint32_t bar0 = smem_addr(bars);
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
@@ -252,13 +271,12 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
       mbar_init(tfull_bar(s), 1);
       mbar_init(tempty_bar(s), 16);  // 8 epilogue warps in each CTA of the pair
     }
-    mbar_init(efull_bar(0), 1);
-    mbar_init(efull_bar(1), 1);
+    for (int b = 0; b < 8; ++b) mbar_init(efull_bar(b), 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
-  if (warp == 1) {
+  if (warp == MMA_WARP) {
     asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(tmem_slot)),
                  "r"(TMEM_COLS));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
@@ -269,70 +287,91 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp == 0) {
-    // ---------------- TMA producer (both CTAs) ----------------
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      uint32_t issued = 0, last_par = 0;
-      bool ok = true;
-      for (int tile = cid; tile < a.total_tiles && ok; tile += ncl) {
-        const TileCoord tc = decode_tile(a, tile);
-        const GroupInfo gi = group_info(a, tc.group);
-        const int nk = (tc.Kdim + BK - 1) / BK;
-        const int amn = a_is_mn(op, gi.wide), bmn = b_is_mn(op, gi.wide);
-        const CUtensorMap* mA;
-        const CUtensorMap* mB;
-        if (op == OP_GRAM) {
-          mA = mB = map_at(maps, tc.group, a.map_src);
-        } else if (op == OP_SQUARE) {
-          mA = mB = map_at(maps, tc.group, 2);
-        } else {
-          const CUtensorMap* mP = map_at(maps, tc.group, a.p_from_b ? 3 : 2);
-          const CUtensorMap* mX = map_at(maps, tc.group, a.map_src);
-          mA = gi.wide ? mP : mX;
-          mB = gi.wide ? mX : mP;
-        }
-        const int a0 = tc.m0 + 128 * (int)rank;          // this CTA's A rows
-        const int hb = tc.BN / 2;                        // this CTA's B rows
-        const int b0 = tc.n0 + hb * (int)rank;
-        const uint32_t bytes = 2u * (uint32_t)(128 + hb) * BK * 2;   // both CTAs
-        for (int kb = 0; kb < nk; ++kb) {
-          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, a.err)) { ok = false; break; }
-          if (rank == 0) mbar_expect_tx(full_bar(stage), bytes);
-          const uint32_t fb = leader_addr(full_bar(stage));
-          const uint32_t sa = base + stage * STAGE_BYTES;
-          const uint32_t sb = sa + A_BYTES;
+  if (warp < NPROD) {
+    // ---------------- TMA producers (both CTAs) ----------------
+    // k-block j of this CTA's tile sequence goes to ring stage j mod nst and
+    // is loaded by producer warp j mod NPROD (NPROD <= nst, so a warp never
+    // waits on a stage barrier more than one phase ahead).  Lane 0 waits
+    // until the stage is free and posts the expected bytes; then lanes
+    // 0..n-1 issue the stage's n boxes (A first, then B) in one instruction.
+    int stage = 0, turn = 0;
+    uint32_t phase = 0;
+    uint32_t issued = 0, last_par = 0;   // lane 0: stages this warp loaded, their parity
+    bool ok = true;
+    for (int tile = cid; tile < a.total_tiles && ok; tile += ncl) {
+      const TileCoord tc = decode_tile(a, tile);
+      const GroupInfo gi = group_info(a, tc.group);
+      const int nk = (tc.Kdim + BK - 1) / BK;
+      const int amn = a_is_mn(op, gi.wide), bmn = b_is_mn(op, gi.wide);
+      const CUtensorMap* mA;
+      const CUtensorMap* mB;
+      if (op == OP_GRAM) {
+        mA = mB = map_at(maps, tc.group, a.map_src);
+      } else if (op == OP_SQUARE) {
+        mA = mB = map_at(maps, tc.group, 2);
+      } else {
+        const CUtensorMap* mP = map_at(maps, tc.group, a.p_from_b ? 3 : 2);
+        const CUtensorMap* mX = map_at(maps, tc.group, a.map_src);
+        mA = gi.wide ? mP : mX;
+        mB = gi.wide ? mX : mP;
+      }
+      const int a0 = tc.m0 + 128 * (int)rank;          // this CTA's A rows
+      const int hb = tc.BN / 2;                        // this CTA's B rows
+      const int b0 = tc.n0 + hb * (int)rank;
+      const uint32_t bytes = 2u * (uint32_t)(128 + hb) * BK * 2;   // both CTAs
+      // This lane's box, if any: K-major tiles come in one box of 128 (or
+      // hb) rows, MN-major tiles as one 64x64 box per 64 MN indices.
+      const int nA = amn ? 2 : 1;
+      const int nB = bmn ? hb / 64 : 1;
+      const bool box_a = lane < nA, box_b = !box_a && lane < nA + nB;
+      const CUtensorMap* lmap = nullptr;
+      uint32_t loff = 0;
+      int lx = 0, ly = 0;            // MN-major: (mn index, -); K-major: (-, row)
+      bool lmn = false;
+      if (box_a) {
+        lmn = amn;
+        lmap = amn ? mA : map128(mA);
+        loff = (uint32_t)lane * BOX_BYTES;
+        lx = a0 + 64 * lane;
+        ly = a0;
+      } else if (box_b) {
+        const int i = lane - nA;
+        lmn = bmn;
+        lmap = bmn ? mB : (hb == 128 ? map128(mB) : mB);
+        loff = A_BYTES + (uint32_t)i * BOX_BYTES;
+        lx = b0 + 64 * i;
+        ly = b0;
+      }
+      for (int kb = 0; kb < nk; ++kb) {
+        if (turn == warp) {
+          int w_ok = 1;
+          if (lane == 0) w_ok = mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, a.err) ? 1 : 0;
+          w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
+          if (!w_ok) { ok = false; break; }
+          if (lane == 0 && rank == 0) mbar_expect_tx(full_bar(stage), bytes);
+          __syncwarp();
           const int k0 = kb * BK;
-          // K-major tiles come in one box of 128 (or hb) rows; MN-major tiles
-          // as one 64x64 box per 64 MN indices
-          if (amn) {
-            tma_load_pair(sa, mA, fb, a0, k0, tc.b);
-            tma_load_pair(sa + BOX_BYTES, mA, fb, a0 + 64, k0, tc.b);
-          } else {
-            tma_load_pair(sa, map128(mA), fb, k0, a0, tc.b);
-          }
-          if (bmn) {
-            for (int j = 0; j < hb / 64; ++j) tma_load_pair(sb + j * BOX_BYTES, mB, fb, b0 + 64 * j, k0, tc.b);
-          } else {
-            tma_load_pair(sb, hb == 128 ? map128(mB) : mB, fb, k0, b0, tc.b);
-          }
+          if (box_a || box_b)
+            tma_load_pair(base + stage * STAGE_BYTES + loff, lmap, leader_addr(full_bar(stage)), lmn ? lx : k0,
+                          lmn ? k0 : ly, tc.b);
+          __syncwarp();
           issued |= 1u << stage;
           last_par = (last_par & ~(1u << stage)) | (phase << stage);
-          if (++stage == nst) { stage = 0; phase ^= 1u; }
         }
-      }
-      if (!ok && rank == 0) {
-        // drain: every issued stage's last loads must land before teardown
-        for (int s = 0; s < nst; ++s) {
-          if (!(issued & (1u << s))) continue;
-          const uint32_t par = (last_par >> s) & 1u;
-          const uint64_t t0 = globaltimer();
-          while (!mbar_try_wait(full_bar(s), par) && globaltimer() - t0 < kTimeoutNs) {}
-        }
+        if (++turn == NPROD) turn = 0;
+        if (++stage == nst) { stage = 0; phase ^= 1u; }
       }
     }
-  } else if (warp == 1) {
+    if (!ok && rank == 0 && lane == 0) {
+      // drain: the last loads this warp issued into each stage must land
+      for (int s = 0; s < nst; ++s) {
+        if (!(issued & (1u << s))) continue;
+        const uint32_t par = (last_par >> s) & 1u;
+        const uint64_t t0 = globaltimer();
+        while (!mbar_try_wait(full_bar(s), par) && globaltimer() - t0 < kTimeoutNs) {}
+      }
+    }
+  } else if (warp == MMA_WARP) {
     // ---------------- MMA issuer (leader CTA) ----------------
     if (lane == 0 && rank == 0) {
       int stage = 0;
@@ -379,38 +418,47 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
       }
     }
   } else {
-    // ---------------- epilogue (warps 2..9, both CTAs) ----------------
-    // Two warps per TMEM lane quarter, each taking half of the tile's columns.
-    // The CTA's 128 x BN output tile is staged in shared memory in the
-    // swizzled box layout that TMA reads and writes: SQUARE/APPLY load their
-    // affine operand there (one tile ahead, alternating two staging tiles),
-    // each thread overwrites its operand chunk with the result, and one
-    // thread stores the tile with TMA.
+    // ---------------- epilogue (warps 6..13, both CTAs) ----------------
+    // Warp e = warp - 6 owns rows 32*q .. 32*q+31 of the CTA's 128 (its TMEM
+    // lane quarter q = warp % 4) and the column half e / 4 of the tile, i.e.
+    // one 32-row slice of one or two 64-column atoms of the staging tile
+    // (swizzled box layout [atom][128 rows][128 B]).  Each warp runs on its
+    // own: it TMA-loads its slice of the affine operand (X for APPLY, A for
+    // SQUARE), drains its accumulator slice, writes bf16 results over the
+    // operand and TMA-stores the slice, with no barrier between warps.
+    const int e = warp - EPI_WARP0;
     const int q = warp & 3;                // TMEM lane quarter this warp may access
-    const int half = (warp - 2) >> 2;      // column half of the tile
+    const int half = e >> 2;               // column half of the tile
     const int rloc = q * 32 + lane;        // row within this CTA's 128 rows
-    const bool leader_thr = (warp == 2 && lane == 0);
     const bool affine = op != OP_GRAM;
     const bool final_out = (op == OP_APPLY) && a.final_out;
     const uint32_t tempty_leader0 = leader_addr(tempty_bar(0));
     const uint32_t tempty_leader1 = leader_addr(tempty_bar(1));
-    // operand load of `tile` into staging tile `b` (leader thread)
-    auto load_operand = [&](int tile, int b) {
-      const TileCoord t2 = decode_tile(a, tile);
-      const CUtensorMap* mO = (op == OP_SQUARE) ? map_at(maps, t2.group, 2) : map_at(maps, t2.group, a.map_src);
-      const int rb = t2.m0 + 128 * (int)rank;
-      mbar_expect_tx(efull_bar(b), (uint32_t)(t2.BN / 64) * 2u * BOX_BYTES);
-      for (int j = 0; j < t2.BN / 64; ++j)
-        tma_load_local(epi0 + (uint32_t)b * EPI_BYTES + (uint32_t)j * 2u * BOX_BYTES, map128(mO), efull_bar(b),
-                       t2.n0 + 64 * j, rb, t2.b);
+    const uint32_t my_efull = efull_bar(e);
+    // this warp's slice of atom j starts at epi0 + j * 16 KB + q * 4 KB
+    auto slice_addr = [&](int j) { return epi0 + (uint32_t)j * 2u * BOX_BYTES + (uint32_t)q * 4096u; };
+    // operand slice of `tile`: lane i < atoms loads atom (first + i), 32 x 64
+    auto load_operand = [&](const TileCoord& t2) {
+      const CUtensorMap* mO = map_at(maps, t2.group, (op == OP_SQUARE) ? 10 : 8 + a.map_src);
+      const int atoms = t2.BN / 128, j0 = half * atoms;
+      if (lane == 0) mbar_expect_tx_relaxed(my_efull, (uint32_t)atoms * 4096u);
+      __syncwarp();
+      if (lane < atoms)
+        tma_load_local(slice_addr(j0 + lane), mO, my_efull, t2.n0 + 64 * (j0 + lane), t2.m0 + 128 * (int)rank + 32 * q,
+                       t2.b);
     };
-    if (affine && leader_thr && cid < a.total_tiles) load_operand(cid, 0);
+    uint32_t e_par = 0;          // phase of my operand barrier
+    bool load_pending = false;   // an operand load is in flight
+    if (affine && cid < a.total_tiles) {
+      load_operand(decode_tile(a, cid));
+      load_pending = true;
+    }
     int acc = 0;
     uint32_t acc_phase = 0;
-    uint32_t e_phase = 0;       // bit b: phase of staging tile b's operand barrier
-    int li = 0;                 // tiles handled by this CTA
-    for (int tile = cid; tile < a.total_tiles; tile += ncl, ++li) {
+    for (int tile = cid; tile < a.total_tiles; tile += ncl) {
       const TileCoord tc = decode_tile(a, tile);
+      const bool more = tile + ncl < a.total_tiles;
+      const TileCoord tnext = decode_tile(a, more ? tile + ncl : tile);
       const GroupInfo gi = group_info(a, tc.group);
       int mat = 0;
       const int p = problem_id(a, gi, tc.b, &mat);
@@ -420,138 +468,145 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
         c0 = cf.x;
         c1 = cf.y;
       }
-      const int buf = affine ? (li & 1) : 0;
-      uint8_t* const epi_ptr = epi_ptr0 + buf * EPI_BYTES;
-      const uint32_t epi = epi0 + (uint32_t)buf * EPI_BYTES;
       const int rbase = tc.m0 + 128 * (int)rank;
       const int row = rbase + rloc;
       const bool row_ok = row < tc.Mdim;
       const int64_t aoff = gi.a_base + (int64_t)tc.b * gi.g * gi.gld;
       const int w = tc.b / gi.count;
-      const int nch = tc.BN / 32;
-      // Gram: the single staging tile is free once the previous tile's TMA
-      // store has read it (affine roles wait for this one tile later)
-      if (!affine && leader_thr) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-      // every epilogue warp is here; stop together if a wait gave up
-      if (epi_bar_or(*abort_flag != 0)) break;
+      const int atoms = tc.BN / 128;                 // atoms of this warp
+      const int ch0 = half * (tc.BN / 64), ch1 = ch0 + tc.BN / 64;   // 32-column chunks
+      // Gram: my slice is free once my previous stores have read it
+      if (!affine) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
       int okw = 1;
       if (lane == 0) {
         okw = mbar_wait(tfull_bar(acc), acc_phase, abort_flag, a.err) ? 1 : 0;
-        if (okw && affine) okw = mbar_wait(efull_bar(buf), (e_phase >> buf) & 1u, abort_flag, a.err) ? 1 : 0;
+        if (okw && affine) okw = mbar_wait(my_efull, e_par, abort_flag, a.err) ? 1 : 0;
       }
       okw = __shfl_sync(0xffffffffu, okw, 0);
-      if (affine) e_phase ^= 1u << buf;
-      // collective: if any warp's wait gave up, all skip to the next barrier,
-      // which then stops them together
-      if (epi_bar_or(!okw)) continue;
+      if (!okw) break;
+      if (affine) {
+        e_par ^= 1u;
+        load_pending = false;
+      }
       tc_fence_after();
       // symmetric Gram: an off-diagonal tile is also written transposed
       const bool mirror = (op == OP_GRAM) && (tc.n0 != tc.m0);
-      const int h = rloc >> 6, rr = rloc & 63;
-      const int ch0 = half * (nch / 2), ch1 = ch0 + nch / 2;
-#pragma unroll 1
-      for (int ch = ch0; ch < ch1; ++ch) {
+      const uint32_t tm_row = tmem_base + (uint32_t)(acc * 256) + ((uint32_t)(q * 32) << 16);
+      // drain the accumulator slice two 32-column chunks per TMEM round
+      // trip; the slice is released after its last TMEM load, before the
+      // last results are formed
+      auto form = [&](int ch, uint32_t (&rr)[32]) {
         float v[32];
-        tmem_ld32(tmem_base + (uint32_t)(acc * 256 + ch * 32) + ((uint32_t)(q * 32) << 16), v);
+#pragma unroll
+        for (int u = 0; u < 32; ++u) v[u] = __uint_as_float(rr[u]);
         const int col0 = tc.n0 + ch * 32;
         const bool live = row_ok && col0 < tc.Ndim;
         const int ncol = live ? min(32, tc.Ndim - col0) : 0;
-        // this thread's 64-byte slice of the staging tile: box (j, h), row rr
-        uint8_t* rowp = const_cast<uint8_t*>(epi_ptr) + ((ch >> 1) * 2 + h) * BOX_BYTES + rr * 128;
+        const uint32_t rowa = epi0 + (uint32_t)((ch >> 1) * 2 * BOX_BYTES + rloc * 128);
         if (affine) {
-          float xv[32];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            const int unit = ((ch & 1) * 4 + u) ^ (rr & 7);
-            unpack_bf16x8(*reinterpret_cast<const uint4*>(rowp + unit * 16), xv + 8 * u);
-          }
+            const uint4 xo = lds128(rowa + (uint32_t)((((ch & 1) * 4 + u) ^ (rloc & 7)) * 16));
+            float xv[8];
+            unpack_bf16x8(xo, xv);
 #pragma unroll
-          for (int u = 0; u < 32; ++u) v[u] = fmaf(c0, xv[u], c1 * v[u]);
+            for (int i = 0; i < 8; ++i) v[8 * u + i] = fmaf(c0, xv[i], c1 * v[8 * u + i]);
+          }
         }
         if (final_out) {
-          if (!live) continue;
+          if (!live) return;
           float* dst = a.out + (int64_t)w * a.out_stride + a.mat_off[mat] + (int64_t)row * gi.cols + col0;
           if (ncol == 32 && ((reinterpret_cast<uintptr_t>(dst) & 15u) == 0)) {
 #pragma unroll
             for (int u = 0; u < 8; ++u)
               reinterpret_cast<float4*>(dst)[u] = make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
           } else {
-            for (int u = 0; u < ncol; ++u) dst[u] = v[u];
+            // fully unrolled with a guard: a loop bounded by ncol would index
+            // v dynamically and move it to local memory
+#pragma unroll
+            for (int u = 0; u < 32; ++u)
+              if (u < ncol) dst[u] = v[u];
           }
-          continue;
+          return;
         }
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          const int unit = ((ch & 1) * 4 + u) ^ (rr & 7);
+          const int unit = ((ch & 1) * 4 + u) ^ (rloc & 7);
           uint4 o;
           o.x = pack_bf16x2(v[8 * u + 0], v[8 * u + 1]);
           o.y = pack_bf16x2(v[8 * u + 2], v[8 * u + 3]);
           o.z = pack_bf16x2(v[8 * u + 4], v[8 * u + 5]);
           o.w = pack_bf16x2(v[8 * u + 6], v[8 * u + 7]);
-          *reinterpret_cast<uint4*>(rowp + unit * 16) = o;
+          sts128(rowa + (uint32_t)(unit * 16), o);
         }
         if (mirror && live) {
           // lanes hold consecutive rows: each store below is 64 contiguous bytes
           __nv_bfloat16* A = reinterpret_cast<__nv_bfloat16*>(a.A) + aoff;
-#pragma unroll 8
-          for (int u = 0; u < ncol; ++u) A[(int64_t)(col0 + u) * gi.gld + row] = __float2bfloat16_rn(v[u]);
+#pragma unroll
+          for (int u = 0; u < 32; ++u)
+            if (u < ncol) A[(int64_t)(col0 + u) * gi.gld + row] = __float2bfloat16_rn(v[u]);
         }
+      };
+#pragma unroll 1
+      for (int cp = ch0; cp < ch1; cp += 2) {
+        uint32_t r[2][32];
+        tmem_ld32_async(tm_row + (uint32_t)(cp * 32), r[0]);
+        tmem_ld32_async(tm_row + (uint32_t)((cp + 1) * 32), r[1]);
+        tmem_wait_ld();
+        reg_fence(r[0]);
+        reg_fence(r[1]);
+        if (cp + 2 == ch1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster_relaxed(acc == 0 ? tempty_leader0 : tempty_leader1);
+        }
+        form(cp, r[0]);
+        form(cp + 1, r[1]);
       }
-      // make the staged results visible to the TMA (async proxy), release the
-      // accumulator, then one thread stores the tile
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(acc == 0 ? tempty_leader0 : tempty_leader1);
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      // make the staged results visible to the TMA (async proxy), then store
+      // my slice
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncwarp();
       if (!final_out) {
-        epi_bar_or(0);
-        if (leader_thr) {
-          const int slot = (op == OP_GRAM) ? 2 : (op == OP_SQUARE ? 3 : a.map_dst);
-          const CUtensorMap* mD = map_at(maps, tc.group, slot);
-          // one 64-column x 128-row box per store, each in its own bulk
-          // group (several vertically adjacent boxes in one group were seen
-          // to lose all but the first on this hardware)
-          int groups = 0;
-          if (rbase < tc.Mdim) {
-            for (int j = 0; j < tc.BN / 64; ++j) {
-              const int x = tc.n0 + 64 * j;
-              if (x >= tc.Ndim) break;
-              asm volatile(
-                  "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%1, %2, %3}], [%4];"
-                  ::"l"(reinterpret_cast<uint64_t>(map128(mD))), "r"(x), "r"(rbase), "r"(tc.b),
-                  "r"(epi + (uint32_t)j * 2u * BOX_BYTES)
-                  : "memory");
-              asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-              ++groups;
-            }
-          }
-          if (affine) {
-            // the other staging tile is free once the previous tile's stores
-            // (all groups but this tile's) have read it; then prefetch the
-            // next tile's operand into it
-            switch (groups) {
-              case 0: asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); break;
-              case 1: asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); break;
-              case 2: asm volatile("cp.async.bulk.wait_group.read 2;" ::: "memory"); break;
-              case 3: asm volatile("cp.async.bulk.wait_group.read 3;" ::: "memory"); break;
-              default: asm volatile("cp.async.bulk.wait_group.read 4;" ::: "memory"); break;
-            }
-            if (tile + ncl < a.total_tiles) load_operand(tile + ncl, buf ^ 1);
+        const int slot = (op == OP_GRAM) ? 10 : (op == OP_SQUARE ? 11 : 8 + a.map_dst);
+        const CUtensorMap* mD = map_at(maps, tc.group, slot);
+        const int j = half * atoms + lane;
+        const int x = tc.n0 + 64 * j, y = rbase + 32 * q;
+        // one 64 x 32 box per lane, each in a bulk group of its own
+        if (lane < atoms && y < tc.Mdim && x < tc.Ndim) {
+          asm volatile(
+              "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%1, %2, %3}], [%4];"
+              ::"l"(reinterpret_cast<uint64_t>(mD)), "r"(x), "r"(y), "r"(tc.b), "r"(slice_addr(j))
+              : "memory");
+          asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+        }
+        if (affine) {
+          // the slice takes the next operand once my stores have read it
+          asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+          __syncwarp();
+          if (more) {
+            load_operand(tnext);
+            load_pending = true;
           }
         }
-      } else if (affine && leader_thr) {
-        // final APPLY (no stores): prefetch the next tile's operand
-        if (tile + ncl < a.total_tiles) load_operand(tile + ncl, buf ^ 1);
+      } else if (affine && more) {
+        // final APPLY (no stores): this warp is done reading its slice
+        load_operand(tnext);
+        load_pending = true;
       }
     }
-    if (leader_thr) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+    if (load_pending && lane == 0) {
+      // a wait gave up with an operand load in flight: let it land
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try_wait(my_efull, e_par) && globaltimer() - t0 < kTimeoutNs) {}
+    }
   }
-
   tc_fence_before();
   __syncthreads();
   cluster_sync();   // both CTAs are done with the pair's TMEM and barriers
-  if (warp == 1) {
+  if (warp == MMA_WARP) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS));
   }

@@ -475,14 +475,16 @@ int signmuon_init(signmuon_t* out, const int64_t* shapes, int n_mats, int M, flo
     return bail(fail(h, SIGNMUON_E_CUDA, "memset"));
   if (!p.fp32) {
     // per group: slots 0..3 = X ping, X pong, A, B with 64-row boxes;
-    // slots 4..7 = the same tensors with 128-row boxes
-    std::vector<CUtensorMap> maps(p.groups.size() * 8);
+    // slots 4..7 = the same tensors with 128-row boxes; slots 8..11 with
+    // 32-row boxes
+    std::vector<CUtensorMap> maps(p.groups.size() * sm::kMapsPerGroup);
+    std::memset(maps.data(), 0, maps.size() * sizeof(CUtensorMap));
     for (size_t g = 0; g < p.groups.size(); ++g) {
       const sm::GroupInfo& gi = p.groups[g];
       const int batch = M * gi.count;
-      for (int box = 0; box < 2; ++box) {
-        const int br = box ? 128 : 64;
-        CUtensorMap* mm = &maps[g * 8 + 4 * box];
+      for (int box = 0; box < 3; ++box) {
+        const int br = box == 0 ? 64 : (box == 1 ? 128 : 32);
+        CUtensorMap* mm = &maps[g * sm::kMapsPerGroup + 4 * box];
         for (int i = 0; i < 2; ++i) {
           void* xb = reinterpret_cast<__nv_bfloat16*>(h->X[i]) + gi.x_base;
           if ((rc = encode_map(h, &mm[i], xb, gi.cols, gi.rows, gi.ld, batch, br))) return bail(rc);
