@@ -123,7 +123,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(bar), "r"(parity)
@@ -132,7 +132,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 // Bounded wait: false when the CTA is aborting or 2 s passed (then the error
 // word gets the timeout code and the abort flag is raised).
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* err) {
+__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* err) {
   uint64_t t0 = 0;
   for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -149,6 +149,10 @@ __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile i
     }
   }
 }
+// first attempt inline; the bounded loop only when the phase is not done yet
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* err) {
+  return mbar_try_wait(bar, parity) || mbar_wait_slow(bar, parity, abort_flag, err);
+}
 // 2-SM TMA load: the transaction bytes complete on `bar_cl`, a barrier of the
 // leader CTA given by its shared::cluster address.
 __device__ __forceinline__ void tma_load_pair(uint32_t dst, const void* map, uint32_t bar_cl, int x, int y, int z) {
@@ -156,6 +160,31 @@ __device__ __forceinline__ void tma_load_pair(uint32_t dst, const void* map, uin
       "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
       ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar_cl)
       : "memory");
+}
+// 2-SM TMA load of a 4-D box (the two-atom views of slots 20/21)
+__device__ __forceinline__ void tma_load_pair4(uint32_t dst, const void* map, uint32_t bar_cl, int x, int y, int z,
+                                               int w) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], [%6];"
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(bar_cl)
+      : "memory");
+}
+// one-CTA 4-D TMA load / store (the slice views of slots 12..19)
+__device__ __forceinline__ void tma_load_local4(uint32_t dst, const void* map, uint32_t bar, int x, int y, int z, int w) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], [%6];"
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void tma_store4(const void* map, uint32_t src, int x, int y, int z, int w) {
+  asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%1, %2, %3, %4}], [%5];"
+               ::"l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(src)
+               : "memory");
+}
+__device__ __forceinline__ void tma_store3(const void* map, uint32_t src, int x, int y, int z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%1, %2, %3}], [%4];"
+               ::"l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(src)
+               : "memory");
 }
 // plain one-CTA TMA load completing on this CTA's barrier
 __device__ __forceinline__ void tma_load_local(uint32_t dst, const void* map, uint32_t bar, int x, int y, int z) {
@@ -232,7 +261,12 @@ __device__ __forceinline__ void unpack_bf16x8(uint4 u, float* f) {
 }
 // Tensor-map slots per group: 0/1 = X ping/pong, 2 = A, 3 = B, with 64-row
 // boxes; the same four with 128-row boxes at slot + 4 and with 32-row boxes
-// (one epilogue warp's slice) at slot + 8.
+// at slot + 8.  When the tensor's column count is a multiple of 64 there are
+// also 4-D views (64-column atom, row, atom index, matrix): the same four
+// with a box of two atoms x 32 rows at slot + 12 and of one atom x 32 rows
+// at slot + 16 (one epilogue warp's slice in one request), and X ping/pong
+// with a box of two atoms x 64 rows at 20/21 (an MN-major operand half of a
+// k-block in one request).
 __device__ __forceinline__ const CUtensorMap* map_at(const CUtensorMap* maps, int group, int slot) {
   return maps + group * kMapsPerGroup + slot;
 }
@@ -320,24 +354,30 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
       const int b0 = tc.n0 + hb * (int)rank;
       const uint32_t bytes = 2u * (uint32_t)(128 + hb) * BK * 2;   // both CTAs
       // This lane's box, if any: K-major tiles come in one box of 128 (or
-      // hb) rows, MN-major tiles as one 64x64 box per 64 MN indices.
-      const int nA = amn ? 2 : 1;
-      const int nB = bmn ? hb / 64 : 1;
+      // hb) rows; MN-major tiles (always X) in one 4-D box of two 64x64
+      // atoms when X's column count is a multiple of 64, else as one 64x64
+      // box per 64 MN indices.
+      const bool x4 = (gi.cols % 64) == 0;
+      const CUtensorMap* mX4 = map_at(maps, tc.group, 20 + a.map_src);
+      const int nA = amn ? (x4 ? 1 : 2) : 1;
+      const int nB = bmn ? ((x4 && hb == 128) ? 1 : hb / 64) : 1;
       const bool box_a = lane < nA, box_b = !box_a && lane < nA + nB;
       const CUtensorMap* lmap = nullptr;
       uint32_t loff = 0;
       int lx = 0, ly = 0;            // MN-major: (mn index, -); K-major: (-, row)
-      bool lmn = false;
+      bool lmn = false, l4 = false;
       if (box_a) {
         lmn = amn;
-        lmap = amn ? mA : map128(mA);
+        l4 = amn && x4;
+        lmap = l4 ? mX4 : (amn ? mA : map128(mA));
         loff = (uint32_t)lane * BOX_BYTES;
         lx = a0 + 64 * lane;
         ly = a0;
       } else if (box_b) {
         const int i = lane - nA;
         lmn = bmn;
-        lmap = bmn ? mB : (hb == 128 ? map128(mB) : mB);
+        l4 = bmn && x4 && hb == 128;
+        lmap = l4 ? mX4 : (bmn ? mB : (hb == 128 ? map128(mB) : mB));
         loff = A_BYTES + (uint32_t)i * BOX_BYTES;
         lx = b0 + 64 * i;
         ly = b0;
@@ -348,10 +388,12 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
           if (lane == 0) w_ok = mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, a.err) ? 1 : 0;
           w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
           if (!w_ok) { ok = false; break; }
-          if (lane == 0 && rank == 0) mbar_expect_tx(full_bar(stage), bytes);
+          if (lane == 0 && rank == 0) mbar_expect_tx_relaxed(full_bar(stage), bytes);
           __syncwarp();
           const int k0 = kb * BK;
-          if (box_a || box_b)
+          if (l4)
+            tma_load_pair4(base + stage * STAGE_BYTES + loff, lmap, leader_addr(full_bar(stage)), 0, k0, lx >> 6, tc.b);
+          else if (box_a || box_b)
             tma_load_pair(base + stage * STAGE_BYTES + loff, lmap, leader_addr(full_bar(stage)), lmn ? lx : k0,
                           lmn ? k0 : ly, tc.b);
           __syncwarp();
@@ -382,8 +424,11 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
       int last_acc = 0;
       uint32_t last_acc_par = 0;
       bool ok = true;
+      // the next tile is decoded while the current one's first MMAs run, so
+      // that a tile boundary costs the MMA queue no decode time
+      TileCoord tn = decode_tile(a, cid < a.total_tiles ? cid : 0);
       for (int tile = cid; tile < a.total_tiles && ok; tile += ncl) {
-        const TileCoord tc = decode_tile(a, tile);
+        const TileCoord tc = tn;
         const GroupInfo gi = group_info(a, tc.group);
         const int nk = (tc.Kdim + BK - 1) / BK;
         const int amn = a_is_mn(op, gi.wide), bmn = b_is_mn(op, gi.wide);
@@ -404,6 +449,7 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
           }
           tc_commit_pair(empty_bar(stage));
           if (++stage == nst) { stage = 0; phase ^= 1u; }
+          if (kb == 0 && tile + ncl < a.total_tiles) tn = decode_tile(a, tile + ncl);
         }
         if (!ok) break;
         tc_commit_pair(tfull_bar(acc));
@@ -435,17 +481,29 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
     const uint32_t tempty_leader0 = leader_addr(tempty_bar(0));
     const uint32_t tempty_leader1 = leader_addr(tempty_bar(1));
     const uint32_t my_efull = efull_bar(e);
-    // this warp's slice of atom j starts at epi0 + j * 16 KB + q * 4 KB
-    auto slice_addr = [&](int j) { return epi0 + (uint32_t)j * 2u * BOX_BYTES + (uint32_t)q * 4096u; };
-    // operand slice of `tile`: lane i < atoms loads atom (first + i), 32 x 64
+    // This warp's slice occupies 8 KB of the staging tile: its i-th atom
+    // (32 rows x 64 columns, 128-byte rows, swizzled) at slice + i * 4 KB.
+    const uint32_t slice = epi0 + (uint32_t)e * 8192u;
+    // the operand and the stored tensor have columns in whole 64-column
+    // atoms (then one 4-D request per slice) or not (one request per atom)
+    const int opnd_slot = (op == OP_SQUARE) ? 2 : a.map_src;
+    const int dst_slot = (op == OP_GRAM) ? 2 : (op == OP_SQUARE ? 3 : a.map_dst);
+    auto whole_atoms = [&](const GroupInfo& g2, int slot) { return ((slot >= 2 ? g2.g : g2.cols) % 64) == 0; };
+    // operand slice of a tile
     auto load_operand = [&](const TileCoord& t2) {
-      const CUtensorMap* mO = map_at(maps, t2.group, (op == OP_SQUARE) ? 10 : 8 + a.map_src);
+      const GroupInfo g2 = group_info(a, t2.group);
       const int atoms = t2.BN / 128, j0 = half * atoms;
+      const int y = t2.m0 + 128 * (int)rank + 32 * q;
       if (lane == 0) mbar_expect_tx_relaxed(my_efull, (uint32_t)atoms * 4096u);
       __syncwarp();
-      if (lane < atoms)
-        tma_load_local(slice_addr(j0 + lane), mO, my_efull, t2.n0 + 64 * (j0 + lane), t2.m0 + 128 * (int)rank + 32 * q,
-                       t2.b);
+      if (whole_atoms(g2, opnd_slot)) {
+        if (lane == 0)
+          tma_load_local4(slice, map_at(maps, t2.group, (atoms == 2 ? 12 : 16) + opnd_slot), my_efull, 0, y,
+                          (t2.n0 >> 6) + j0, t2.b);
+      } else if (lane < atoms) {
+        tma_load_local(slice + (uint32_t)lane * 4096u, map_at(maps, t2.group, 8 + opnd_slot), my_efull,
+                       t2.n0 + 64 * (j0 + lane), y, t2.b);
+      }
     };
     uint32_t e_par = 0;          // phase of my operand barrier
     bool load_pending = false;   // an operand load is in flight
@@ -502,11 +560,11 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
         const int col0 = tc.n0 + ch * 32;
         const bool live = row_ok && col0 < tc.Ndim;
         const int ncol = live ? min(32, tc.Ndim - col0) : 0;
-        const uint32_t rowa = epi0 + (uint32_t)((ch >> 1) * 2 * BOX_BYTES + rloc * 128);
+        const uint32_t rowa = slice + (uint32_t)(((ch - ch0) >> 1) * 4096 + lane * 128);
         if (affine) {
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            const uint4 xo = lds128(rowa + (uint32_t)((((ch & 1) * 4 + u) ^ (rloc & 7)) * 16));
+            const uint4 xo = lds128(rowa + (uint32_t)((((ch & 1) * 4 + u) ^ (lane & 7)) * 16));
             float xv[8];
             unpack_bf16x8(xo, xv);
 #pragma unroll
@@ -531,7 +589,7 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
         }
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          const int unit = ((ch & 1) * 4 + u) ^ (rloc & 7);
+          const int unit = ((ch & 1) * 4 + u) ^ (lane & 7);
           uint4 o;
           o.x = pack_bf16x2(v[8 * u + 0], v[8 * u + 1]);
           o.y = pack_bf16x2(v[8 * u + 2], v[8 * u + 3]);
@@ -569,17 +627,21 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       __syncwarp();
       if (!final_out) {
-        const int slot = (op == OP_GRAM) ? 10 : (op == OP_SQUARE ? 11 : 8 + a.map_dst);
-        const CUtensorMap* mD = map_at(maps, tc.group, slot);
-        const int j = half * atoms + lane;
-        const int x = tc.n0 + 64 * j, y = rbase + 32 * q;
-        // one 64 x 32 box per lane, each in a bulk group of its own
-        if (lane < atoms && y < tc.Mdim && x < tc.Ndim) {
-          asm volatile(
-              "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%1, %2, %3}], [%4];"
-              ::"l"(reinterpret_cast<uint64_t>(mD)), "r"(x), "r"(y), "r"(tc.b), "r"(slice_addr(j))
-              : "memory");
-          asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+        // the slice in one 4-D store, or one 64 x 32 box per lane, each
+        // request in a bulk group of its own
+        const int y = rbase + 32 * q;
+        const int j0 = half * atoms;
+        if (whole_atoms(gi, dst_slot)) {
+          if (lane == 0 && y < tc.Mdim && tc.n0 + 64 * j0 < tc.Ndim) {
+            tma_store4(map_at(maps, tc.group, (atoms == 2 ? 12 : 16) + dst_slot), slice, 0, y, (tc.n0 >> 6) + j0, tc.b);
+            asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+          }
+        } else {
+          const int x = tc.n0 + 64 * (j0 + lane);
+          if (lane < atoms && y < tc.Mdim && x < tc.Ndim) {
+            tma_store3(map_at(maps, tc.group, 8 + dst_slot), slice + (uint32_t)lane * 4096u, x, y, tc.b);
+            asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+          }
         }
         if (affine) {
           // the slice takes the next operand once my stores have read it

@@ -169,6 +169,25 @@ int encode_map(signmuon_t h, CUtensorMap* m, void* base, int cols, int rows, int
   return SIGNMUON_OK;
 }
 
+// 4-D view of the same matrices: (64-column atom, row, atom index, matrix),
+// strides (row, 128 B, matrix); a box of `atoms` atoms x box_rows rows lands
+// in shared memory atom after atom.  Requires cols % 64 == 0, so that no
+// atom reaches past the end of a row and stores clip at the last column.
+int encode_map_atoms(signmuon_t h, CUtensorMap* m, void* base, int cols, int rows, int ld, int batch, int box_rows,
+                     int atoms) {
+  EncodeTiledFn fn = get_encode();
+  if (!fn) return fail(h, SIGNMUON_E_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t dims[4] = {64, (cuuint64_t)rows, (cuuint64_t)(cols / 64), (cuuint64_t)batch};
+  cuuint64_t strides[3] = {(cuuint64_t)ld * 2, 128, (cuuint64_t)rows * ld * 2};
+  cuuint32_t box[4] = {64, (cuuint32_t)box_rows, (cuuint32_t)atoms, 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base, dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(h, SIGNMUON_E_CUDA, "cuTensorMapEncodeTiled (4-D) failed: " + std::to_string((int)r));
+  return SIGNMUON_OK;
+}
+
 sm::WorkerPtrs worker_ptrs(const float* const* p, int M) {
   sm::WorkerPtrs w{};
   for (int m = 0; m < M; ++m) w.p[m] = p[m];
@@ -476,7 +495,9 @@ int signmuon_init(signmuon_t* out, const int64_t* shapes, int n_mats, int M, flo
   if (!p.fp32) {
     // per group: slots 0..3 = X ping, X pong, A, B with 64-row boxes;
     // slots 4..7 = the same tensors with 128-row boxes; slots 8..11 with
-    // 32-row boxes
+    // 32-row boxes; when the column count is a multiple of 64, 4-D atom
+    // views with 2-atom x 32-row boxes at 12..15, 1-atom x 32-row boxes at
+    // 16..19, and X ping/pong with 2-atom x 64-row boxes at 20/21
     std::vector<CUtensorMap> maps(p.groups.size() * sm::kMapsPerGroup);
     std::memset(maps.data(), 0, maps.size() * sizeof(CUtensorMap));
     for (size_t g = 0; g < p.groups.size(); ++g) {
@@ -493,6 +514,16 @@ int signmuon_init(signmuon_t* out, const int64_t* shapes, int n_mats, int M, flo
         void* bb = reinterpret_cast<__nv_bfloat16*>(h->B) + gi.a_base;
         if ((rc = encode_map(h, &mm[2], ab, gi.g, gi.g, gi.gld, batch, br))) return bail(rc);
         if ((rc = encode_map(h, &mm[3], bb, gi.g, gi.g, gi.gld, batch, br))) return bail(rc);
+      }
+      CUtensorMap* mg = &maps[g * sm::kMapsPerGroup];
+      for (int i = 0; i < 4; ++i) {
+        void* tb = i < 2 ? reinterpret_cast<void*>(reinterpret_cast<__nv_bfloat16*>(h->X[i]) + gi.x_base)
+                         : reinterpret_cast<void*>(reinterpret_cast<__nv_bfloat16*>(i == 2 ? h->A : h->B) + gi.a_base);
+        const int cols = i < 2 ? gi.cols : gi.g, rows = i < 2 ? gi.rows : gi.g, ld = i < 2 ? gi.ld : gi.gld;
+        if (cols % 64 != 0) continue;
+        if ((rc = encode_map_atoms(h, &mg[12 + i], tb, cols, rows, ld, batch, 32, 2))) return bail(rc);
+        if ((rc = encode_map_atoms(h, &mg[16 + i], tb, cols, rows, ld, batch, 32, 1))) return bail(rc);
+        if (i < 2 && (rc = encode_map_atoms(h, &mg[20 + i], tb, cols, rows, ld, batch, 64, 2))) return bail(rc);
       }
     }
     uint8_t* m = nullptr;
