@@ -78,10 +78,9 @@ enum GemmOp { OP_GRAM = 0, OP_SQUARE = 1, OP_APPLY = 2 };
 // memory is a chain of dependent loads).
 constexpr int kParamGroups = 24;
 // TMA tensor maps per shape group (bf16 path): X ping/pong, A, B with 64-row,
-// 128-row and 32-row boxes; 4-D atom views of the four with slice boxes of
-// two and of one atom; X ping/pong as 4-D atom views with two-atom operand
-// boxes.
-constexpr int kMapsPerGroup = 22;
+// 128-row and 32-row boxes, and X ping/pong as 4-D atom views with two-atom
+// operand boxes.
+constexpr int kMapsPerGroup = 14;
 constexpr int kParamMats = 64;
 
 // Arguments of one grouped Newton-Schulz GEMM launch (both precisions).

@@ -38,9 +38,12 @@ constexpr int BOX_BYTES = 64 * 64 * 2;                  // one 64x64 bf16 TMA bo
 constexpr int A_BYTES = 128 * BK * 2;                   // 16 KB: this CTA's 128 rows of A
 constexpr int B_BYTES = 128 * BK * 2;                   // 16 KB: this CTA's BN/2 <= 128 rows of B
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int EPI_BYTES = 128 * 256 * 2;                // 64 KB: one staging tile
-// Shared memory: a 5-deep operand ring and one staging tile (224 KB).
-constexpr int RING = 5, RING_MAX = RING;
+constexpr int EPI_BYTES = 8 * 32 * 64 * 2;              // 32 KB: one 32x64 atom per epilogue warp
+// Shared memory: a 6-deep operand ring and the epilogue's staging atoms
+// (224 KB).  The ring depth is what hides the operand latency: a freed stage
+// is refilled ~2,500 cycles later under load, against ~650 cycles of MMA work
+// per stage.
+constexpr int RING = 6, RING_MAX = RING;
 constexpr int DATA_BYTES = RING * STAGE_BYTES + EPI_BYTES;
 constexpr int TMEM_COLS = 512;
 // Warp roles.  A warp completes only about one TMA load instruction every
@@ -92,13 +95,6 @@ __device__ __forceinline__ void cluster_sync() {
 }
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-// arrive on a barrier given by its shared::cluster address (own or peer CTA)
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cl_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cl_addr) : "memory");
 }
 // Relaxed forms: no release fence in front of the arrival (a release at
 // cluster scope held the arriving warp for ~2,000 cycles).  Used where the
@@ -161,25 +157,13 @@ __device__ __forceinline__ void tma_load_pair(uint32_t dst, const void* map, uin
       ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar_cl)
       : "memory");
 }
-// 2-SM TMA load of a 4-D box (the two-atom views of slots 20/21)
+// 2-SM TMA load of a 4-D box (the two-atom views of slots 12/13)
 __device__ __forceinline__ void tma_load_pair4(uint32_t dst, const void* map, uint32_t bar_cl, int x, int y, int z,
                                                int w) {
   asm volatile(
       "cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], [%6];"
       ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(bar_cl)
       : "memory");
-}
-// one-CTA 4-D TMA load / store (the slice views of slots 12..19)
-__device__ __forceinline__ void tma_load_local4(uint32_t dst, const void* map, uint32_t bar, int x, int y, int z, int w) {
-  asm volatile(
-      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], [%6];"
-      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(bar)
-      : "memory");
-}
-__device__ __forceinline__ void tma_store4(const void* map, uint32_t src, int x, int y, int z, int w) {
-  asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%1, %2, %3, %4}], [%5];"
-               ::"l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(src)
-               : "memory");
 }
 __device__ __forceinline__ void tma_store3(const void* map, uint32_t src, int x, int y, int z) {
   asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%1, %2, %3}], [%4];"
@@ -261,12 +245,10 @@ __device__ __forceinline__ void unpack_bf16x8(uint4 u, float* f) {
 }
 // Tensor-map slots per group: 0/1 = X ping/pong, 2 = A, 3 = B, with 64-row
 // boxes; the same four with 128-row boxes at slot + 4 and with 32-row boxes
-// at slot + 8.  When the tensor's column count is a multiple of 64 there are
-// also 4-D views (64-column atom, row, atom index, matrix): the same four
-// with a box of two atoms x 32 rows at slot + 12 and of one atom x 32 rows
-// at slot + 16 (one epilogue warp's slice in one request), and X ping/pong
-// with a box of two atoms x 64 rows at 20/21 (an MN-major operand half of a
-// k-block in one request).
+// (an epilogue warp's atom) at slot + 8.  When X's column count is a
+// multiple of 64, slots 12/13 hold X ping/pong as 4-D views (64-column atom,
+// row, atom index, matrix) with a box of two atoms x 64 rows: an MN-major
+// operand half of a k-block in one request.
 __device__ __forceinline__ const CUtensorMap* map_at(const CUtensorMap* maps, int group, int slot) {
   return maps + group * kMapsPerGroup + slot;
 }
@@ -358,7 +340,7 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
       // atoms when X's column count is a multiple of 64, else as one 64x64
       // box per 64 MN indices.
       const bool x4 = (gi.cols % 64) == 0;
-      const CUtensorMap* mX4 = map_at(maps, tc.group, 20 + a.map_src);
+      const CUtensorMap* mX4 = map_at(maps, tc.group, 12 + a.map_src);
       const int nA = amn ? (x4 ? 1 : 2) : 1;
       const int nB = bmn ? ((x4 && hb == 128) ? 1 : hb / 64) : 1;
       const bool box_a = lane < nA, box_b = !box_a && lane < nA + nB;
@@ -481,39 +463,42 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
     const uint32_t tempty_leader0 = leader_addr(tempty_bar(0));
     const uint32_t tempty_leader1 = leader_addr(tempty_bar(1));
     const uint32_t my_efull = efull_bar(e);
-    // This warp's slice occupies 8 KB of the staging tile: its i-th atom
-    // (32 rows x 64 columns, 128-byte rows, swizzled) at slice + i * 4 KB.
-    const uint32_t slice = epi0 + (uint32_t)e * 8192u;
-    // the operand and the stored tensor have columns in whole 64-column
-    // atoms (then one 4-D request per slice) or not (one request per atom)
+    // This warp's staging slice is one atom, 32 rows x 64 columns (4 KB,
+    // 128-byte rows, swizzled); the warp's 64- or 128-column part of a tile
+    // passes through it one atom at a time.
+    const uint32_t slice = epi0 + (uint32_t)e * 4096u;
     const int opnd_slot = (op == OP_SQUARE) ? 2 : a.map_src;
     const int dst_slot = (op == OP_GRAM) ? 2 : (op == OP_SQUARE ? 3 : a.map_dst);
-    auto whole_atoms = [&](const GroupInfo& g2, int slot) { return ((slot >= 2 ? g2.g : g2.cols) % 64) == 0; };
-    // operand slice of a tile
-    auto load_operand = [&](const TileCoord& t2) {
-      const GroupInfo g2 = group_info(a, t2.group);
-      const int atoms = t2.BN / 128, j0 = half * atoms;
-      const int y = t2.m0 + 128 * (int)rank + 32 * q;
-      if (lane == 0) mbar_expect_tx_relaxed(my_efull, (uint32_t)atoms * 4096u);
-      __syncwarp();
-      if (whole_atoms(g2, opnd_slot)) {
-        if (lane == 0)
-          tma_load_local4(slice, map_at(maps, t2.group, (atoms == 2 ? 12 : 16) + opnd_slot), my_efull, 0, y,
-                          (t2.n0 >> 6) + j0, t2.b);
-      } else if (lane < atoms) {
-        tma_load_local(slice + (uint32_t)lane * 4096u, map_at(maps, t2.group, 8 + opnd_slot), my_efull,
-                       t2.n0 + 64 * (j0 + lane), y, t2.b);
+    // atom i (of this warp's part) of a tile's affine operand, 64 x 32 box
+    auto load_operand = [&](const TileCoord& t2, int i) {
+      const int j = half * (t2.BN / 128) + i;
+      if (lane == 0) {
+        mbar_expect_tx_relaxed(my_efull, 4096u);
+        tma_load_local(slice, map_at(maps, t2.group, 8 + opnd_slot), my_efull, t2.n0 + 64 * j,
+                       t2.m0 + 128 * (int)rank + 32 * q, t2.b);
       }
     };
     uint32_t e_par = 0;          // phase of my operand barrier
     bool load_pending = false;   // an operand load is in flight
     if (affine && cid < a.total_tiles) {
-      load_operand(decode_tile(a, cid));
+      load_operand(decode_tile(a, cid), 0);
       load_pending = true;
     }
+    // lane 0 waits for my operand barrier; false if the wait gave up
+    auto wait_operand = [&]() {
+      int okw = 1;
+      if (lane == 0) okw = mbar_wait(my_efull, e_par, abort_flag, a.err) ? 1 : 0;
+      okw = __shfl_sync(0xffffffffu, okw, 0);
+      if (okw) {
+        e_par ^= 1u;
+        load_pending = false;
+      }
+      return okw != 0;
+    };
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int tile = cid; tile < a.total_tiles; tile += ncl) {
+    bool alive = true;
+    for (int tile = cid; tile < a.total_tiles && alive; tile += ncl) {
       const TileCoord tc = decode_tile(a, tile);
       const bool more = tile + ncl < a.total_tiles;
       const TileCoord tnext = decode_tile(a, more ? tile + ncl : tile);
@@ -532,27 +517,16 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
       const int64_t aoff = gi.a_base + (int64_t)tc.b * gi.g * gi.gld;
       const int w = tc.b / gi.count;
       const int atoms = tc.BN / 128;                 // atoms of this warp
-      const int ch0 = half * (tc.BN / 64), ch1 = ch0 + tc.BN / 64;   // 32-column chunks
-      // Gram: my slice is free once my previous stores have read it
-      if (!affine) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+      const int ch0 = half * (tc.BN / 64);           // first 32-column chunk
       int okw = 1;
-      if (lane == 0) {
-        okw = mbar_wait(tfull_bar(acc), acc_phase, abort_flag, a.err) ? 1 : 0;
-        if (okw && affine) okw = mbar_wait(my_efull, e_par, abort_flag, a.err) ? 1 : 0;
-      }
+      if (lane == 0) okw = mbar_wait(tfull_bar(acc), acc_phase, abort_flag, a.err) ? 1 : 0;
       okw = __shfl_sync(0xffffffffu, okw, 0);
       if (!okw) break;
-      if (affine) {
-        e_par ^= 1u;
-        load_pending = false;
-      }
       tc_fence_after();
       // symmetric Gram: an off-diagonal tile is also written transposed
       const bool mirror = (op == OP_GRAM) && (tc.n0 != tc.m0);
       const uint32_t tm_row = tmem_base + (uint32_t)(acc * 256) + ((uint32_t)(q * 32) << 16);
-      // drain the accumulator slice two 32-column chunks per TMEM round
-      // trip; the slice is released after its last TMEM load, before the
-      // last results are formed
+      // results of one 32-column chunk from its accumulator registers
       auto form = [&](int ch, uint32_t (&rr)[32]) {
         float v[32];
 #pragma unroll
@@ -560,7 +534,7 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
         const int col0 = tc.n0 + ch * 32;
         const bool live = row_ok && col0 < tc.Ndim;
         const int ncol = live ? min(32, tc.Ndim - col0) : 0;
-        const uint32_t rowa = slice + (uint32_t)(((ch - ch0) >> 1) * 4096 + lane * 128);
+        const uint32_t rowa = slice + (uint32_t)(lane * 128);
         if (affine) {
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
@@ -606,57 +580,56 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
         }
       };
 #pragma unroll 1
-      for (int cp = ch0; cp < ch1; cp += 2) {
+      for (int i = 0; i < atoms; ++i) {
+        const int ch = ch0 + 2 * i;
+        // the atom's operand has landed (affine); the slice is free of my
+        // previous store (Gram)
+        if (affine) {
+          if (!wait_operand()) { alive = false; break; }
+        } else {
+          asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+          __syncwarp();
+        }
+        // two 32-column chunks per TMEM round trip; the accumulator slice is
+        // released after its last TMEM load
         uint32_t r[2][32];
-        tmem_ld32_async(tm_row + (uint32_t)(cp * 32), r[0]);
-        tmem_ld32_async(tm_row + (uint32_t)((cp + 1) * 32), r[1]);
+        tmem_ld32_async(tm_row + (uint32_t)(ch * 32), r[0]);
+        tmem_ld32_async(tm_row + (uint32_t)((ch + 1) * 32), r[1]);
         tmem_wait_ld();
         reg_fence(r[0]);
         reg_fence(r[1]);
-        if (cp + 2 == ch1) {
+        if (i + 1 == atoms) {
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive_cluster_relaxed(acc == 0 ? tempty_leader0 : tempty_leader1);
         }
-        form(cp, r[0]);
-        form(cp + 1, r[1]);
-      }
-      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
-      // make the staged results visible to the TMA (async proxy), then store
-      // my slice
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      __syncwarp();
-      if (!final_out) {
-        // the slice in one 4-D store, or one 64 x 32 box per lane, each
-        // request in a bulk group of its own
-        const int y = rbase + 32 * q;
-        const int j0 = half * atoms;
-        if (whole_atoms(gi, dst_slot)) {
-          if (lane == 0 && y < tc.Mdim && tc.n0 + 64 * j0 < tc.Ndim) {
-            tma_store4(map_at(maps, tc.group, (atoms == 2 ? 12 : 16) + dst_slot), slice, 0, y, (tc.n0 >> 6) + j0, tc.b);
-            asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-          }
-        } else {
-          const int x = tc.n0 + 64 * (j0 + lane);
-          if (lane < atoms && y < tc.Mdim && x < tc.Ndim) {
-            tma_store3(map_at(maps, tc.group, 8 + dst_slot), slice + (uint32_t)lane * 4096u, x, y, tc.b);
+        form(ch, r[0]);
+        form(ch + 1, r[1]);
+        // make the staged results visible to the TMA (async proxy), store
+        // the atom (one 64 x 32 box in a bulk group of its own)
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (!final_out && lane == 0) {
+          const int x = tc.n0 + 64 * (half * atoms + i), y = rbase + 32 * q;
+          if (y < tc.Mdim && x < tc.Ndim) {
+            tma_store3(map_at(maps, tc.group, 8 + dst_slot), slice, x, y, tc.b);
             asm volatile("cp.async.bulk.commit_group;" ::: "memory");
           }
         }
         if (affine) {
-          // the slice takes the next operand once my stores have read it
-          asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+          // the slice takes the next operand atom once my store has read it
+          if (!final_out) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
           __syncwarp();
-          if (more) {
-            load_operand(tnext);
+          if (i + 1 < atoms) {
+            load_operand(tc, i + 1);
+            load_pending = true;
+          } else if (more) {
+            load_operand(tnext, 0);
             load_pending = true;
           }
         }
-      } else if (affine && more) {
-        // final APPLY (no stores): this warp is done reading its slice
-        load_operand(tnext);
-        load_pending = true;
       }
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
     asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
     if (load_pending && lane == 0) {

@@ -495,9 +495,8 @@ int signmuon_init(signmuon_t* out, const int64_t* shapes, int n_mats, int M, flo
   if (!p.fp32) {
     // per group: slots 0..3 = X ping, X pong, A, B with 64-row boxes;
     // slots 4..7 = the same tensors with 128-row boxes; slots 8..11 with
-    // 32-row boxes; when the column count is a multiple of 64, 4-D atom
-    // views with 2-atom x 32-row boxes at 12..15, 1-atom x 32-row boxes at
-    // 16..19, and X ping/pong with 2-atom x 64-row boxes at 20/21
+    // 32-row boxes; when X's column count is a multiple of 64, X ping/pong
+    // as 4-D atom views with 2-atom x 64-row boxes at 12/13
     std::vector<CUtensorMap> maps(p.groups.size() * sm::kMapsPerGroup);
     std::memset(maps.data(), 0, maps.size() * sizeof(CUtensorMap));
     for (size_t g = 0; g < p.groups.size(); ++g) {
@@ -515,15 +514,13 @@ int signmuon_init(signmuon_t* out, const int64_t* shapes, int n_mats, int M, flo
         if ((rc = encode_map(h, &mm[2], ab, gi.g, gi.g, gi.gld, batch, br))) return bail(rc);
         if ((rc = encode_map(h, &mm[3], bb, gi.g, gi.g, gi.gld, batch, br))) return bail(rc);
       }
-      CUtensorMap* mg = &maps[g * sm::kMapsPerGroup];
-      for (int i = 0; i < 4; ++i) {
-        void* tb = i < 2 ? reinterpret_cast<void*>(reinterpret_cast<__nv_bfloat16*>(h->X[i]) + gi.x_base)
-                         : reinterpret_cast<void*>(reinterpret_cast<__nv_bfloat16*>(i == 2 ? h->A : h->B) + gi.a_base);
-        const int cols = i < 2 ? gi.cols : gi.g, rows = i < 2 ? gi.rows : gi.g, ld = i < 2 ? gi.ld : gi.gld;
-        if (cols % 64 != 0) continue;
-        if ((rc = encode_map_atoms(h, &mg[12 + i], tb, cols, rows, ld, batch, 32, 2))) return bail(rc);
-        if ((rc = encode_map_atoms(h, &mg[16 + i], tb, cols, rows, ld, batch, 32, 1))) return bail(rc);
-        if (i < 2 && (rc = encode_map_atoms(h, &mg[20 + i], tb, cols, rows, ld, batch, 64, 2))) return bail(rc);
+      if (gi.cols % 64 == 0) {
+        for (int i = 0; i < 2; ++i) {
+          void* xb = reinterpret_cast<__nv_bfloat16*>(h->X[i]) + gi.x_base;
+          if ((rc = encode_map_atoms(h, &maps[g * sm::kMapsPerGroup + 12 + i], xb, gi.cols, gi.rows, gi.ld, batch, 64,
+                                     2)))
+            return bail(rc);
+        }
       }
     }
     uint8_t* m = nullptr;
