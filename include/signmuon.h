@@ -56,6 +56,9 @@ typedef struct signmuon_ctx* signmuon_t;
 #define SIGNMUON_ACC_INT8    (1u << 3) /* signmuon_vote writes int8 sums (requires M <= 127) */
 #define SIGNMUON_ASYNC       (1u << 4) /* signmuon_step does not wait; signmuon_sync reports status */
 #define SIGNMUON_VOTE_ONLY   (1u << 5) /* allocate no step workspace: vote/pack/update calls only */
+#define SIGNMUON_KEEP_POLAR  (1u << 6) /* signmuon_step also writes U for signmuon_get_polar; without it
+                                          the last Newton-Schulz GEMM of a step writes only the one-bit
+                                          signs when every matrix has a multiple of 32 columns */
 
 /* ------------------------------------------------------------------------
  * signmuon_init -- plan the step and allocate its device state.
@@ -144,8 +147,11 @@ int signmuon_polar(signmuon_t h, const float* const* X, float* const* U);
 /* ------------------------------------------------------------------------
  * State access (device float[d] / uint8[ceil(d/8)] buffers of the caller).
  * get/set_momentum: worker m's momentum (checkpoint / resume).
- * get_polar: worker m's U from the last step.  get_signs: worker m's packed
- * bits from the last step.  get_direction: the last step's D.
+ * get_polar: worker m's U from the last step (or signmuon_polar call);
+ * SIGNMUON_E_UNSUPPORTED when the step did not keep it (handle made without
+ * SIGNMUON_KEEP_POLAR on shapes whose signs are packed inside the last
+ * Newton-Schulz GEMM).  get_signs: worker m's packed bits from the last
+ * step.  get_direction: the last step's D.
  * get_scales: host float[M*n_mats]: the last step's scale s per (worker,
  * matrix), worker-major (waits for the GPU).
  * ---------------------------------------------------------------------- */

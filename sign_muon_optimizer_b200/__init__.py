@@ -35,6 +35,7 @@ SIGNMUON_POST_POLAR = 1 << 2
 SIGNMUON_ACC_INT8 = 1 << 3
 SIGNMUON_ASYNC = 1 << 4
 SIGNMUON_VOTE_ONLY = 1 << 5
+SIGNMUON_KEEP_POLAR = 1 << 6
 
 EXPORTED = [
     "signmuon_init", "signmuon_step", "signmuon_step_host", "signmuon_vote", "signmuon_pack",

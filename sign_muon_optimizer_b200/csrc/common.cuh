@@ -103,9 +103,14 @@ struct GemmArgs {
   const float2* coef;
   float c0, c1;
   // final APPLY: fp32 flat output out + worker*out_stride + mat_off + r*cols + c
+  // (skipped when out is null), and, when out_bits is non-null, the one-bit
+  // signs (U >= 0) as LSB-first 32-bit words at out_bits + worker*bits_stride
+  // + flat/32 (every matrix has a multiple of 32 columns)
   float* out;
   int64_t out_stride;
   int final_out;
+  uint32_t* out_bits;
+  int64_t bits_stride;       // in 32-bit words
   int* err;
   int param_tables;                        // 1: the p* copies below are valid
   TileGroup ptiles[kParamGroups];
@@ -130,7 +135,7 @@ void launch_fro_finalize(cudaStream_t s, int n_probs, int n_mats, int M, const f
 void launch_pi_init(cudaStream_t s, int n_probs, const int64_t* uoff, const int* prob_g, float* u);
 void launch_pi_matvec(cudaStream_t s, const ProbRows* rows, int n_rows, const void* A, int a_bf16,
                       const int64_t* prob_a_off, const int* prob_g, const int* prob_gld,
-                      const int64_t* uoff, const float* u, float* y);
+                      const int64_t* uoff, const float* u, float* y, int max_g);
 void launch_pi_normalize(cudaStream_t s, int n_probs, const int64_t* uoff, const int* prob_g,
                          const float* y, float* u);
 void launch_pi_finalize(cudaStream_t s, int n_probs, const int64_t* uoff, const int* prob_g,

@@ -194,44 +194,77 @@ k_pi_matvec(const ProbRows* __restrict__ rows, const void* __restrict__ A,
             const int64_t* __restrict__ prob_a_off, const int* __restrict__ prob_g,
             const int* __restrict__ prob_gld, const int64_t* __restrict__ uoff,
             const float* __restrict__ u, float* __restrict__ y) {
+  // y[r] = sum_k A[r][k] u[k] for the block's kPiRows rows of one problem.
+  // u is staged in shared memory; each warp streams kRowsPerWarp rows at
+  // once (one 16-byte load per row and lane in flight per step) so that the
+  // HBM stream of A has enough loads in flight.
+  extern __shared__ float us[];
   const ProbRows pr = rows[blockIdx.x];
   const int p = pr.p;
   const int g = prob_g[p], gld = prob_gld[p];
   const float* up = u + uoff[p];
+  for (int k = threadIdx.x; k < g; k += kThreads) us[k] = up[k];
+  __syncthreads();
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  constexpr int kRowsPerWarp = kPiRows / (kThreads / 32);
-  for (int j = 0; j < kRowsPerWarp; ++j) {
-    const int r = pr.row0 + wid * kRowsPerWarp + j;
-    if (r >= g) break;
-    float acc = 0.f;
-    if (BF16) {
-      const __nv_bfloat16* a = reinterpret_cast<const __nv_bfloat16*>(A) + prob_a_off[p] + (int64_t)r * gld;
-      const int g8 = g & ~7;
-      for (int k = lane * 8; k < g8; k += 256) {
-        const uint4 raw = *reinterpret_cast<const uint4*>(a + k);
-        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+  constexpr int R = kPiRows / (kThreads / 32);
+  const int r0 = pr.row0 + wid * R;
+  float acc[R];
+#pragma unroll
+  for (int j = 0; j < R; ++j) acc[j] = 0.f;
+  if (BF16) {
+    const __nv_bfloat16* a0 = reinterpret_cast<const __nv_bfloat16*>(A) + prob_a_off[p] + (int64_t)r0 * gld;
+    const int g8 = g & ~7;
+    for (int k = lane * 8; k < g8; k += 256) {
+      uint4 raw[R];
+#pragma unroll
+      for (int j = 0; j < R; ++j)
+        raw[j] = (r0 + j < g) ? __ldcs(reinterpret_cast<const uint4*>(a0 + (int64_t)j * gld + k)) : make_uint4(0, 0, 0, 0);
+      const float4 u0 = *reinterpret_cast<const float4*>(us + k);
+      const float4 u1 = *reinterpret_cast<const float4*>(us + k + 4);
+      const float uv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+      for (int j = 0; j < R; ++j) {
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw[j]);
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
           const float2 f = __bfloat1622float2(h[t]);
-          acc = fmaf(f.x, up[k + 2 * t], acc);
-          acc = fmaf(f.y, up[k + 2 * t + 1], acc);
+          acc[j] = fmaf(f.x, uv[2 * t], acc[j]);
+          acc[j] = fmaf(f.y, uv[2 * t + 1], acc[j]);
         }
       }
-      for (int k = g8 + lane; k < g; k += 32) acc = fmaf(__bfloat162float(a[k]), up[k], acc);
-    } else {
-      const float* a = reinterpret_cast<const float*>(A) + prob_a_off[p] + (int64_t)r * gld;
-      const int g4 = g & ~3;
-      for (int k = lane * 4; k < g4; k += 128) {
-        const float4 f = ld4(a + k);
-        acc = fmaf(f.x, up[k], acc);
-        acc = fmaf(f.y, up[k + 1], acc);
-        acc = fmaf(f.z, up[k + 2], acc);
-        acc = fmaf(f.w, up[k + 3], acc);
-      }
-      for (int k = g4 + lane; k < g; k += 32) acc = fmaf(a[k], up[k], acc);
     }
-    acc = warp_sum(acc);
-    if (lane == 0) y[uoff[p] + r] = acc;
+    for (int k = g8 + lane; k < g; k += 32) {
+#pragma unroll
+      for (int j = 0; j < R; ++j)
+        if (r0 + j < g) acc[j] = fmaf(__bfloat162float(a0[(int64_t)j * gld + k]), us[k], acc[j]);
+    }
+  } else {
+    const float* a0 = reinterpret_cast<const float*>(A) + prob_a_off[p] + (int64_t)r0 * gld;
+    const int g4 = g & ~3;
+    for (int k = lane * 4; k < g4; k += 128) {
+      float4 f[R];
+#pragma unroll
+      for (int j = 0; j < R; ++j)
+        f[j] = (r0 + j < g) ? __ldcs(reinterpret_cast<const float4*>(a0 + (int64_t)j * gld + k)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float4 uv = *reinterpret_cast<const float4*>(us + k);
+#pragma unroll
+      for (int j = 0; j < R; ++j) {
+        acc[j] = fmaf(f[j].x, uv.x, acc[j]);
+        acc[j] = fmaf(f[j].y, uv.y, acc[j]);
+        acc[j] = fmaf(f[j].z, uv.z, acc[j]);
+        acc[j] = fmaf(f[j].w, uv.w, acc[j]);
+      }
+    }
+    for (int k = g4 + lane; k < g; k += 32) {
+#pragma unroll
+      for (int j = 0; j < R; ++j)
+        if (r0 + j < g) acc[j] = fmaf(a0[(int64_t)j * gld + k], us[k], acc[j]);
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < R; ++j) {
+    const float v = warp_sum(acc[j]);
+    if (lane == 0 && r0 + j < g) y[uoff[p] + r0 + j] = v;
   }
 }
 
@@ -524,12 +557,16 @@ void launch_pi_init(cudaStream_t s, int n_probs, const int64_t* uoff, const int*
 
 void launch_pi_matvec(cudaStream_t s, const ProbRows* rows, int n_rows, const void* A, int a_bf16,
                       const int64_t* prob_a_off, const int* prob_g, const int* prob_gld,
-                      const int64_t* uoff, const float* u, float* y) {
+                      const int64_t* uoff, const float* u, float* y, int max_g) {
   count_launch();
-  if (a_bf16)
-    k_pi_matvec<true><<<n_rows, kThreads, 0, s>>>(rows, A, prob_a_off, prob_g, prob_gld, uoff, u, y);
-  else
-    k_pi_matvec<false><<<n_rows, kThreads, 0, s>>>(rows, A, prob_a_off, prob_g, prob_gld, uoff, u, y);
+  const size_t smem = (size_t)max_g * sizeof(float);
+  if (a_bf16) {
+    if (smem > 48 * 1024) cudaFuncSetAttribute(k_pi_matvec<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    k_pi_matvec<true><<<n_rows, kThreads, smem, s>>>(rows, A, prob_a_off, prob_g, prob_gld, uoff, u, y);
+  } else {
+    if (smem > 48 * 1024) cudaFuncSetAttribute(k_pi_matvec<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    k_pi_matvec<false><<<n_rows, kThreads, smem, s>>>(rows, A, prob_a_off, prob_g, prob_gld, uoff, u, y);
+  }
 }
 
 void launch_pi_normalize(cudaStream_t s, int n_probs, const int64_t* uoff, const int* prob_g,

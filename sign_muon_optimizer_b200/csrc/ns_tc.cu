@@ -547,7 +547,16 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
         }
         if (final_out) {
           if (!live) return;
-          float* dst = a.out + (int64_t)w * a.out_stride + a.mat_off[mat] + (int64_t)row * gi.cols + col0;
+          const int64_t flat = a.mat_off[mat] + (int64_t)row * gi.cols + col0;
+          if (a.out_bits != nullptr) {
+            // the chunk's 32 signs are one LSB-first word of the bit stream
+            uint32_t word = 0;
+#pragma unroll
+            for (int u = 0; u < 32; ++u) word |= (v[u] >= 0.f ? 1u : 0u) << u;
+            a.out_bits[(int64_t)w * a.bits_stride + (flat >> 5)] = word;
+          }
+          if (a.out == nullptr) return;
+          float* dst = a.out + (int64_t)w * a.out_stride + flat;
           if (ncol == 32 && ((reinterpret_cast<uintptr_t>(dst) & 15u) == 0)) {
 #pragma unroll
             for (int u = 0; u < 8; ++u)

@@ -37,6 +37,7 @@ struct signmuon_ctx {
   cudaStream_t stream = nullptr;
   int device = 0, n_sm = 148;
   bool vote_only = false;
+  bool u_valid = true;          // U holds the last step's (or polar call's) polar factors
   // device plan tables
   sm::MatInfo* d_mats = nullptr;
   sm::GroupInfo* d_groups = nullptr;
@@ -243,7 +244,7 @@ void prof_collect(signmuon_t h) {
 // worker*out_stride.  kzero_in is the fp32 input used when K == 0.
 // ---------------------------------------------------------------------------
 void gemm(signmuon_t h, int op, int slot, int src, int nw, const float2* coef, float c0, float c1,
-          bool final_out, float* out, int64_t out_stride) {
+          bool final_out, float* out, int64_t out_stride, uint32_t* out_bits = nullptr, int64_t bits_stride = 0) {
   const Plan& p = h->plan;
   sm::GemmArgs a{};
   a.tiles = h->d_tiles[op][slot];
@@ -267,6 +268,8 @@ void gemm(signmuon_t h, int op, int slot, int src, int nw, const float2* coef, f
   a.out = out;
   a.out_stride = out_stride;
   a.final_out = final_out ? 1 : 0;
+  a.out_bits = out_bits;
+  a.bits_stride = bits_stride;
   a.err = h->status + 1;
   (void)nw;
   const auto& tg = p.tiles[op][slot].groups;
@@ -287,19 +290,30 @@ void power_iteration(signmuon_t h, int nw) {
   const int nprob = nw * p.n_mats;
   const int nrows = nw == 1 ? p.n_pi_rows_one : (int)p.pi_rows.size();
   ProfScope ps(h, 5);
+  int max_g = 1;
+  for (const sm::GroupInfo& gi : p.groups) max_g = gi.g > max_g ? gi.g : max_g;
   sm::launch_pi_init(h->stream, nprob, h->d_uoff, h->d_prob_g, h->pi_u);
   for (int it = 0; it < h->P; ++it) {
     sm::launch_pi_matvec(h->stream, h->d_pi_rows, nrows, h->A, p.fp32 ? 0 : 1, h->d_prob_aoff, h->d_prob_g,
-                         h->d_prob_gld, h->d_uoff, h->pi_u, h->pi_y);
+                         h->d_prob_gld, h->d_uoff, h->pi_u, h->pi_y, max_g);
     sm::launch_pi_normalize(h->stream, nprob, h->d_uoff, h->d_prob_g, h->pi_y, h->pi_u);
   }
   sm::launch_pi_matvec(h->stream, h->d_pi_rows, nrows, h->A, p.fp32 ? 0 : 1, h->d_prob_aoff, h->d_prob_g,
-                       h->d_prob_gld, h->d_uoff, h->pi_u, h->pi_y);
+                       h->d_prob_gld, h->d_uoff, h->pi_u, h->pi_y, max_g);
   sm::launch_pi_finalize(h->stream, nprob, h->d_uoff, h->d_prob_g, h->pi_u, h->pi_y, h->eps, p.quintic ? 1 : 0,
                          h->ns_a, h->ns_b, h->ns_c, h->scale_v, h->coef_apply, h->coef_square, h->status);
 }
 
-void run_ns(signmuon_t h, int nw, const sm::WorkerPtrs& kzero_in, float* out, int64_t out_stride) {
+bool signs_in_gemm(signmuon_t h) {
+  const Plan& p = h->plan;
+  if (p.fp32 || h->K == 0 || (p.nb_pad % 4) != 0) return false;
+  for (const sm::GroupInfo& gi : p.groups)
+    if (gi.cols % 32 != 0) return false;
+  return true;
+}
+
+void run_ns(signmuon_t h, int nw, const sm::WorkerPtrs& kzero_in, float* out, int64_t out_stride,
+            uint32_t* out_bits = nullptr, int64_t bits_stride = 0) {
   const Plan& p = h->plan;
   const int slot = nw == 1 ? 1 : 0;
   const bool spectral = h->scale == SIGNMUON_SCALE_SPECTRAL;
@@ -321,7 +335,7 @@ void run_ns(signmuon_t h, int nw, const sm::WorkerPtrs& kzero_in, float* out, in
       gemm(h, sm::OP_SQUARE, slot, cur, nw, k == 0 ? h->coef_square : nullptr, h->ns_b, h->ns_c, false, nullptr, 0);
     const bool last = (k == h->K - 1);
     gemm(h, sm::OP_APPLY, slot, cur, nw, k == 0 ? h->coef_apply : nullptr, h->ns_a, p.quintic ? 1.f : h->ns_b, last,
-         out, out_stride);
+         out, out_stride, last ? out_bits : nullptr, bits_stride);
     cur ^= 1;
   }
 }
@@ -565,8 +579,17 @@ int signmuon_step(signmuon_t h, float* W, const float* const* G, float eta) {
                         (int)p.chunks.size(), h->d_mats, h->d_groups, h->partials);
   }
   fro_finalize(h, h->M);
-  run_ns(h, h->M, strided_ptrs(h->Mom, p.dpad, h->M), h->U, p.dpad);
-  {
+  // The signs come out of the last Newton-Schulz GEMM itself when every
+  // matrix has a multiple of 32 columns (then each 32-column chunk of an
+  // output row is one aligned word of the bit stream; K > 0, bf16 path);
+  // U is written only when kept for get_polar.
+  const bool fused = signs_in_gemm(h);
+  h->u_valid = !fused || (h->flags & SIGNMUON_KEEP_POLAR) != 0;
+  if (fused) {
+    run_ns(h, h->M, strided_ptrs(h->Mom, p.dpad, h->M), h->u_valid ? h->U : nullptr, p.dpad,
+           reinterpret_cast<uint32_t*>(h->bits), p.nb_pad / 4);
+  } else {
+    run_ns(h, h->M, strided_ptrs(h->Mom, p.dpad, h->M), h->U, p.dpad);
     ProfScope ps(h, 6);
     sm::launch_pack(s, h->U, p.dpad, p.d, h->bits, p.nb_pad, h->M);
   }
@@ -678,6 +701,7 @@ int signmuon_polar(signmuon_t h, const float* const* X, float* const* U) {
                    h->partials);
   fro_finalize(h, h->M);
   run_ns(h, h->M, xp, h->U, p.dpad);
+  h->u_valid = true;
   for (int m = 0; m < h->M; ++m)
     CK(h, cudaMemcpyAsync(U[m], h->U + (int64_t)m * p.dpad, (size_t)p.d * 4, cudaMemcpyDeviceToDevice, s));
   return finish(h, (h->flags & SIGNMUON_ASYNC) == 0);
@@ -705,6 +729,10 @@ int signmuon_get_polar(signmuon_t h, int m, float* dst) {
   int rc = check_handle(h, true);
   if (rc) return rc;
   if (m < 0 || m >= h->M || !dst) return fail(h, SIGNMUON_E_INVALID, "bad worker index or null dst");
+  if (!h->u_valid)
+    return fail(h, SIGNMUON_E_UNSUPPORTED,
+                "the last step packed its signs inside the Newton-Schulz GEMM and kept no U; create the handle "
+                "with SIGNMUON_KEEP_POLAR");
   CK(h, cudaMemcpyAsync(dst, h->U + (int64_t)m * h->plan.dpad, (size_t)h->plan.d * 4, cudaMemcpyDeviceToDevice,
                         h->stream));
   return SIGNMUON_OK;

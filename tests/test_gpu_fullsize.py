@@ -47,7 +47,7 @@ def _mat(flat_dev, shapes, i):
 def _step_sampled(name, sample, post_polar):
     wl = synth.WORKLOADS[name]
     shapes, M = wl["shapes"], wl["M"]
-    flags = smo.SIGNMUON_POST_POLAR if post_polar else 0
+    flags = (smo.SIGNMUON_POST_POLAR if post_polar else 0) | smo.SIGNMUON_KEEP_POLAR
     opt = smo.SignMuon(shapes, M, beta=HP["beta"], lam=HP["lam"], K=wl["K"], eps=HP["eps"], scale=wl["scale"],
                        P=wl["P"], flags=flags)
     W = synth.device_weights0(shapes, config_id=41)

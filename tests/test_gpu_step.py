@@ -24,7 +24,8 @@ HP = dict(beta=0.9, lam=0.01, eta=0.02, eps=1e-7)
 
 
 def _flags(precision, post_polar=False, order="cubic"):
-    f = smo.SIGNMUON_NS_FP32 if precision == "fp32" else 0
+    # these tests read U back, so the step keeps it
+    f = (smo.SIGNMUON_NS_FP32 if precision == "fp32" else 0) | smo.SIGNMUON_KEEP_POLAR
     if post_polar:
         f |= smo.SIGNMUON_POST_POLAR
     if order == "quintic":
@@ -215,3 +216,53 @@ def test_step_host_matches_device_step():
     wh = w0.copy()
     b.step_host(wh, G, 0.02)
     assert np.array_equal(wh.view(np.uint32), host(W).view(np.uint32))
+
+
+@pytest.mark.parametrize("post_polar", [False, True])
+def test_signs_packed_in_gemm_match_kept_polar(post_polar):
+    """With every column count a multiple of 32 the step packs the signs in
+    the last Newton-Schulz GEMM; without SIGNMUON_KEEP_POLAR it writes no U.
+    Both handles run the same step: the packed signs, the direction and W
+    must be identical, the signs must be U >= 0 of the kept U, and get_polar
+    of the handle that kept nothing must refuse."""
+    shapes = [(256, 512), (512, 256), (96, 160), (384, 384)]
+    M, seed = 4, 23
+    base = smo.SIGNMUON_POST_POLAR if post_polar else 0
+    d = synth.numel(shapes)
+    w0 = synth.weights0(shapes, seed)
+    mom0 = synth.momentum0(shapes, M, seed, scale=0.5)
+    G = synth.gradients(shapes, M, 1.0, step=1, config_id=seed)
+    out = {}
+    for keep in (True, False):
+        h = smo.SignMuon(shapes, M, beta=HP["beta"], lam=HP["lam"], K=5, eps=HP["eps"], scale="spectral", P=2,
+                         flags=base | (smo.SIGNMUON_KEEP_POLAR if keep else 0))
+        for m in range(M):
+            h.set_momentum(m, dev(mom0[m]))
+        W = dev(w0)
+        h.step(W, [dev(g) for g in G], HP["eta"])
+        bits = []
+        for m in range(M):
+            b = torch.zeros(ref.packed_nbytes(d), dtype=torch.uint8, device="cuda")
+            h.get_signs(m, b)
+            bits.append(host(b))
+        Dg = torch.zeros(d, device="cuda")
+        h.get_direction(Dg)
+        U = []
+        if keep:
+            for m in range(M):
+                t = torch.zeros(d, device="cuda")
+                h.get_polar(m, t)
+                U.append(host(t))
+        else:
+            t = torch.zeros(d, device="cuda")
+            with pytest.raises(smo.SignMuonError) as ei:
+                h.get_polar(0, t)
+            assert ei.value.status == 7
+        out[keep] = dict(W=host(W), bits=bits, D=host(Dg), U=U)
+        h.close()
+    for m in range(M):
+        assert np.array_equal(out[True]["bits"][m], out[False]["bits"][m])
+        want = np.packbits(out[True]["U"][m] >= 0, bitorder="little")
+        assert np.array_equal(out[True]["bits"][m][: want.size], want)
+    assert np.array_equal(out[True]["D"], out[False]["D"])
+    assert np.array_equal(out[True]["W"].view(np.uint32), out[False]["W"].view(np.uint32))
