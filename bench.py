@@ -88,8 +88,9 @@ def hbm_bytes_per_step(shapes, M, P, post_polar):
         "momentum": d * (14.0 * M + 4.0),          # G r, Mom r+w, X w (bf16) per worker; W r once
         "pack": d * M * (4.0 + 1.0 / 8.0),          # U r (fp32), bits w
         "power_iter": (P + 1) * M * gram_bytes(shapes),
-        "vote": M * d / 8.0 + (4.0 * d if post_polar else 8.0 * d),  # bits r; D w, or W r+w
-        "stage": 6.0 * d,                           # D r (fp32), X w (bf16)
+        # bits r; with the post-vote polar the majority goes straight to the
+        # bf16 X of the polar step (2 B), else the update of W (8 B) is fused
+        "vote": M * d / 8.0 + (2.0 * d if post_polar else 8.0 * d),
         "update": 12.0 * d,                         # W r+w, D r
     }
     if post_polar:

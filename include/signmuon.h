@@ -190,10 +190,11 @@ int signmuon_plan(const int64_t* shapes, int n_mats, int M, int K, int scale, in
  * signmuon_profile_read() waits for the stream, adds up the elapsed times per
  * kind (ms[k], launches[k] for k < n) since the last read, and resets them.
  * Kinds: 0 momentum pass, 1 norm finalisation, 2/3/4 Newton-Schulz GEMMs
- * (Gram, quintic square, apply), 5 power iteration, 6 one-bit pack, 7 vote
- * (fused with the update or writing D), 8 staging of the majority, 9/10/11
- * post-vote Newton-Schulz GEMMs (Gram, square, apply), 12 update, 13 K=0
- * scaling. */
+ * (Gram, quintic square, apply), 5 power iteration, 6 one-bit pack (only
+ * when the signs are not packed inside the last GEMM), 7 vote (fused with the
+ * update, or with the staging of the majority for the post-vote polar step),
+ * 8 unused (kept for numbering), 9/10/11 post-vote Newton-Schulz GEMMs (Gram,
+ * square, apply), 12 update, 13 K=0 scaling. */
 #define SIGNMUON_PROF_KINDS 14
 int signmuon_profile(signmuon_t h, int enable);
 int signmuon_profile_read(signmuon_t h, double* ms, int64_t* launches, int n);

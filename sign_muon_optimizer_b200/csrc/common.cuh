@@ -152,6 +152,9 @@ void launch_vote_update(cudaStream_t s, const uint8_t* bits, int64_t bits_stride
                         float* W, float eta, const int* status);
 void launch_vote_major(cudaStream_t s, const uint8_t* bits, int64_t bits_stride, int M, int64_t d,
                        float* D);
+void launch_vote_stage(cudaStream_t s, const uint8_t* bits, int64_t bits_stride, int M, void* X, int x_bf16,
+                       const Chunk* chunks, int n_chunks, const MatInfo* mats, const GroupInfo* groups,
+                       float* partials, float* D);
 void launch_update(cudaStream_t s, float* W, const float* D, int64_t d, float eta,
                    const int* status);
 

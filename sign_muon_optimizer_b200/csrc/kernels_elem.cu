@@ -481,6 +481,103 @@ k_vote(WorkerPtrs signs, const uint8_t* __restrict__ bits, int64_t bits_stride, 
   }
 }
 
+// Majority of the packed signs staged straight into the Newton-Schulz input of
+// the post-vote polar step ([paper] §4, orthogonalising the aggregated
+// direction): per 4096-entry chunk of one matrix, the majority sgn(2c - M) of
+// every entry goes to X (bf16 or fp32, grouped layout) and, when D is
+// non-null, to D (fp32 flat); partials[chunk] gets the chunk's sum of
+// squares (its non-zero count) for the Frobenius scale and the finite check.
+__global__ void __launch_bounds__(kThreads)
+k_vote_stage(const uint8_t* __restrict__ bits, int64_t bits_stride, int M, void* __restrict__ X, int x_bf16,
+             const Chunk* __restrict__ chunks, const MatInfo* __restrict__ mats,
+             const GroupInfo* __restrict__ groups, float* __restrict__ partials, float* __restrict__ D) {
+  __shared__ float red[32];
+  const Chunk ch = chunks[blockIdx.x];
+  const MatInfo mi = mats[ch.mat];
+  const GroupInfo gi = groups[mi.group];
+  const int64_t base = mi.off + ch.start;
+  // vector path: whole bytes of the bit streams, 8-entry runs inside a row
+  const bool vec = ((base & 7) == 0) && ((ch.len & 7) == 0) && ((mi.cols & 7) == 0);
+  const bool bf = x_bf16 != 0;
+  const int64_t xb = gi.x_base + (int64_t)mi.q * gi.rows * gi.ld;
+  float ss = 0.f;
+  if (vec) {
+    // 8 consecutive entries per thread and step: one byte of every worker's
+    // stream, counted in two SWAR accumulators (byte lane i of lo / hi counts
+    // entry i / i + 4, 255 workers at a time); both steps' bytes are loaded
+    // before any is counted
+    constexpr int kV = kChunk / (kThreads * 8);
+    int64_t fe[kV];
+    bool on[kV];
+#pragma unroll
+    for (int j = 0; j < kV; ++j) {
+      const int e = (threadIdx.x + j * kThreads) * 8;
+      on[j] = e < ch.len;
+      fe[j] = base + e;
+    }
+    int cnt[kV][8];
+#pragma unroll
+    for (int j = 0; j < kV; ++j)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) cnt[j][i] = 0;
+    for (int m = 0; m < M;) {
+      const int end = min(M, m + 255);
+      uint32_t lo[kV], hi[kV];
+#pragma unroll
+      for (int j = 0; j < kV; ++j) lo[j] = hi[j] = 0;
+      for (; m < end; ++m) {
+        const uint8_t* bm = bits + (int64_t)m * bits_stride;
+#pragma unroll
+        for (int j = 0; j < kV; ++j) {
+          const uint32_t by = on[j] ? bm[fe[j] >> 3] : 0u;
+          lo[j] += ((by & 0xFu) * 0x00204081u) & 0x01010101u;
+          hi[j] += ((by >> 4) * 0x00204081u) & 0x01010101u;
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < kV; ++j)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          cnt[j][i] += (lo[j] >> (8 * i)) & 0xFF;
+          cnt[j][i + 4] += (hi[j] >> (8 * i)) & 0xFF;
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < kV; ++j) {
+      if (!on[j]) continue;
+      float v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        v[i] = (float)sgn(2 * cnt[j][i] - M);
+        ss += v[i] * v[i];
+      }
+      const float4 v0 = make_float4(v[0], v[1], v[2], v[3]), v1 = make_float4(v[4], v[5], v[6], v[7]);
+      if (D != nullptr) {
+        st4(D + fe[j], v0);
+        st4(D + fe[j] + 4, v1);
+      }
+      const int le = (int)(fe[j] - mi.off);
+      const int r = le / mi.cols, c = le - r * mi.cols;
+      store_x4(X, xb + (int64_t)r * gi.ld + c, v0, bf);
+      store_x4(X, xb + (int64_t)r * gi.ld + c + 4, v1, bf);
+    }
+  } else {
+    for (int e = threadIdx.x; e < ch.len; e += kThreads) {
+      const int64_t fe = base + e;
+      int c = 0;
+      for (int m = 0; m < M; ++m) c += (bits[(int64_t)m * bits_stride + (fe >> 3)] >> (fe & 7)) & 1;
+      const float v = (float)sgn(2 * c - M);
+      ss += v * v;
+      if (D != nullptr) D[fe] = v;
+      const int le = (int)(ch.start + e);
+      const int r = le / mi.cols, cc = le - r * mi.cols;
+      store_x(X, xb + (int64_t)r * gi.ld + cc, v, bf);
+    }
+  }
+  const float t = block_sum<float>(ss, red);
+  if (threadIdx.x == 0) partials[blockIdx.x] = t;
+}
+
 // W <- fl32(W - eta D), one rounding ([paper] Algorithm 1/2 update).
 __global__ void __launch_bounds__(kThreads)
 k_update(float* __restrict__ W, const float* __restrict__ D, int64_t d, float eta,
@@ -636,6 +733,14 @@ void launch_vote_major(cudaStream_t s, const uint8_t* bits, int64_t bits_stride,
   WorkerPtrs none{};
   k_vote<2, false><<<blocks, kThreads, smem, s>>>(none, bits, bits_stride, M, d, nullptr, nullptr,
                                                   nullptr, 0.f, D, nullptr);
+}
+
+void launch_vote_stage(cudaStream_t s, const uint8_t* bits, int64_t bits_stride, int M, void* X, int x_bf16,
+                       const Chunk* chunks, int n_chunks, const MatInfo* mats, const GroupInfo* groups,
+                       float* partials, float* D) {
+  if (n_chunks <= 0) return;
+  count_launch();
+  k_vote_stage<<<n_chunks, kThreads, 0, s>>>(bits, bits_stride, M, X, x_bf16, chunks, mats, groups, partials, D);
 }
 
 void launch_update(cudaStream_t s, float* W, const float* D, int64_t d, float eta,

@@ -546,28 +546,18 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
           }
         }
         if (final_out) {
-          if (!live) return;
-          const int64_t flat = a.mat_off[mat] + (int64_t)row * gi.cols + col0;
-          if (a.out_bits != nullptr) {
-            // the chunk's 32 signs are one LSB-first word of the bit stream
+          // fp32 results go back into rr for write_out_f32; the signs (when
+          // asked for) are one LSB-first word of the bit stream per chunk
+#pragma unroll
+          for (int u = 0; u < 32; ++u) rr[u] = __float_as_uint(v[u]);
+          if (live && a.out_bits != nullptr) {
+            const int64_t flat = a.mat_off[mat] + (int64_t)row * gi.cols + col0;
             uint32_t word = 0;
 #pragma unroll
             for (int u = 0; u < 32; ++u) word |= (v[u] >= 0.f ? 1u : 0u) << u;
             a.out_bits[(int64_t)w * a.bits_stride + (flat >> 5)] = word;
           }
-          if (a.out == nullptr) return;
-          float* dst = a.out + (int64_t)w * a.out_stride + flat;
-          if (ncol == 32 && ((reinterpret_cast<uintptr_t>(dst) & 15u) == 0)) {
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-              reinterpret_cast<float4*>(dst)[u] = make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
-          } else {
-            // fully unrolled with a guard: a loop bounded by ncol would index
-            // v dynamically and move it to local memory
-#pragma unroll
-            for (int u = 0; u < 32; ++u)
-              if (u < ncol) dst[u] = v[u];
-          }
+          (void)ncol;
           return;
         }
 #pragma unroll
@@ -586,6 +576,35 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
 #pragma unroll
           for (int u = 0; u < 32; ++u)
             if (u < ncol) A[(int64_t)(col0 + u) * gi.gld + row] = __float2bfloat16_rn(v[u]);
+        }
+      };
+      // fp32 output of one chunk (final APPLY): the warp's 32 rows x 32
+      // columns pass through the slice (one 128-byte swizzled row per lane),
+      // then each store instruction writes four whole 128-byte row segments
+      auto write_out_f32 = [&](int ch, uint32_t (&rr)[32]) {
+        __syncwarp();
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          sts128(slice + (uint32_t)(lane * 128 + ((u ^ (lane & 7)) * 16)),
+                 make_uint4(rr[4 * u], rr[4 * u + 1], rr[4 * u + 2], rr[4 * u + 3]));
+        __syncwarp();
+        const int uu = lane & 7;
+        const int colg = tc.n0 + ch * 32 + uu * 4;
+#pragma unroll 2
+        for (int it = 0; it < 8; ++it) {
+          const int rl = it * 4 + (lane >> 3);
+          const int rowg = rbase + q * 32 + rl;
+          if (rowg >= tc.Mdim || colg >= tc.Ndim) continue;
+          const uint4 val = lds128(slice + (uint32_t)(rl * 128 + ((uu ^ (rl & 7)) * 16)));
+          float* dst = a.out + (int64_t)w * a.out_stride + a.mat_off[mat] + (int64_t)rowg * gi.cols + colg;
+          if (colg + 3 < tc.Ndim && ((reinterpret_cast<uintptr_t>(dst) & 15u) == 0)) {
+            *reinterpret_cast<uint4*>(dst) = val;
+          } else {
+            const uint32_t e4[4] = {val.x, val.y, val.z, val.w};
+#pragma unroll
+            for (int t = 0; t < 4; ++t)
+              if (colg + t < tc.Ndim) dst[t] = __uint_as_float(e4[t]);
+          }
         }
       };
 #pragma unroll 1
@@ -614,6 +633,10 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
         }
         form(ch, r[0]);
         form(ch + 1, r[1]);
+        if (final_out && a.out != nullptr) {
+          write_out_f32(ch, r[0]);
+          write_out_f32(ch + 1, r[1]);
+        }
         // make the staged results visible to the TMA (async proxy), store
         // the atom (one 64 x 32 box in a bulk group of its own)
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

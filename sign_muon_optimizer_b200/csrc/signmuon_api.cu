@@ -594,15 +594,13 @@ int signmuon_step(signmuon_t h, float* W, const float* const* G, float eta) {
     sm::launch_pack(s, h->U, p.dpad, p.d, h->bits, p.nb_pad, h->M);
   }
   if (h->flags & SIGNMUON_POST_POLAR) {
-    {
-      ProfScope ps(h, 7);
-      sm::launch_vote_major(s, h->bits, p.nb_pad, h->M, p.d, h->D);
-    }
+    // the majority goes straight into the polar step's input (and into D
+    // only when K == 0, where the polar factor is the scaled input itself)
     const sm::WorkerPtrs dp = strided_ptrs(h->D, 0, 1);
     {
-      ProfScope ps(h, 8);
-      sm::launch_stage(s, dp, 1, h->X[0], p.fp32 ? 0 : 1, h->d_chunks, (int)p.chunks.size(), h->d_mats,
-                       h->d_groups, h->partials);
+      ProfScope ps(h, 7);
+      sm::launch_vote_stage(s, h->bits, p.nb_pad, h->M, h->X[0], p.fp32 ? 0 : 1, h->d_chunks, (int)p.chunks.size(),
+                            h->d_mats, h->d_groups, h->partials, h->K == 0 ? h->D : nullptr);
     }
     fro_finalize(h, 1);
     run_ns(h, 1, dp, h->D, 0);

@@ -84,7 +84,7 @@ def test_hbm_bytes_counts():
     assert d == 84_934_656
     assert b["momentum"] == d * 116          # W once + 8 x (G + Mom r/w + bf16 X)
     assert b["pack"] == d * 8 * 4.125        # fp32 U read + one bit written per worker
-    assert b["vote"] == d + 4 * d            # 8 bits per entry read, fp32 D written
+    assert b["vote"] == d + 2 * d            # 8 bits per entry read, bf16 X written
     assert b["power_iter"] == 3 * 9 * 48 * 768 * 768 * 2
 
 
