@@ -383,6 +383,93 @@ def run_ours(args):
     return 0
 
 
+def _events_time(fn, reps, stream):
+    """Mean ms of fn() over reps calls, CUDA events on the given stream,
+    after 3 warm-up calls."""
+    import torch
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def run_secondary(args):
+    """Secondary measurements (not the headline line): the LLaMA-layer vote
+    (vote GB/s), the Newton-Schulz sweep (NS TFLOP/s) and the ResNet-50 step
+    (steps/s), one JSON line each."""
+    import torch
+    import sign_muon_optimizer_b200 as smo
+    torch.cuda.set_device(0)
+    stream = torch.cuda.current_stream()
+    pk, pk_kind = peaks()
+    lines = []
+    if args.workload in ("llama_vote", "all"):
+        shapes = synth.LLAMA_LAYER_SHAPES
+        Mv = synth.WORKLOADS["llama_vote"]["M"]
+        d = synth.numel(shapes)
+        nb = (d + 7) // 8
+        g = torch.Generator(device="cuda")
+        g.manual_seed(4)
+        signs = [torch.randint(0, 256, (nb + 16,), generator=g, device="cuda", dtype=torch.uint8) for _ in range(Mv)]
+        for acc8 in (False, True):
+            h = smo.SignMuon(shapes, Mv, flags=smo.SIGNMUON_VOTE_ONLY | (smo.SIGNMUON_ACC_INT8 if acc8 else 0),
+                             stream=stream.cuda_stream)
+            sums = torch.empty(d, device="cuda", dtype=torch.int8 if acc8 else torch.int32)
+            maj = torch.empty(d, device="cuda", dtype=torch.int8)
+            ms = _events_time(lambda: h.vote(signs, d, sums, maj), 5, stream)
+            nbytes = Mv * d / 8.0 + (1.0 if acc8 else 4.0) * d + d
+            gbs = nbytes / (ms / 1e3) / 1e9
+            lines.append({"metric": "vote GB/s (LLaMA-layer shapes, M=16, " + ("int8" if acc8 else "int32") + " sums)",
+                          "value": gbs, "unit": "GB/s", "frac_of_hbm": gbs / pk["hbm_gbs"], "peak_kind": pk_kind,
+                          "ms": ms, "bytes": nbytes, "d": d, "M": Mv, "payload_bytes_per_worker": nb,
+                          "acc_dtype": "int8" if acc8 else "int32", "collective": "none (on-device vote)"})
+            h.close()
+            del sums, maj
+        del signs
+        torch.cuda.empty_cache()
+    if args.workload in ("ns_sweep", "all"):
+        for name, shp in synth.SWEEP_SHAPES.items():
+            Mw = 8
+            h = smo.SignMuon(shp, Mw, beta=0.9, lam=0.0, K=5, eps=1e-7, scale="spectral", P=2, flags=0,
+                             stream=stream.cuda_stream)
+            X = synth.device_gaussian(h.d, Mw, seed=5)
+            U = torch.empty_like(X)
+            xs, us = [X[m] for m in range(Mw)], [U[m] for m in range(Mw)]
+            ms = _events_time(lambda: h.polar(xs, us), 3, stream)
+            fl = sum(4.0 * min(r, c) ** 2 * max(r, c) for r, c in shp) * 5 * Mw
+            tf = fl / (ms / 1e3) / 1e12
+            lines.append({"metric": f"NS TFLOP/s ({name}, M=8, K=5 cubic bf16, spectral P=2)", "value": tf,
+                          "unit": "TFLOP/s", "frac_of_bf16_sustained": tf / pk["bf16_tflops_sustained"],
+                          "frac_of_bf16_burst": tf / pk["bf16_tflops"], "peak_kind": pk_kind, "ms": ms,
+                          "flops": fl})
+            h.close()
+            del X, U
+            torch.cuda.empty_cache()
+    if args.workload in ("resnet50", "all"):
+        wl = synth.WORKLOADS["resnet50"]
+        shp, Mr = wl["shapes"], wl["M"]
+        h = smo.SignMuon(shp, Mr, beta=HP["beta"], lam=HP["lam"], K=wl["K"], eps=HP["eps"], scale=wl["scale"],
+                         P=wl["P"], flags=0, stream=stream.cuda_stream)
+        W = synth.device_weights0(shp, config_id=2)
+        G = synth.device_gradients(shp, Mr, wl["sigma"], step=0, config_id=2)
+        gl = [G[m] for m in range(Mr)]
+        ms = _events_time(lambda: h.step(W, gl, HP["eta"]), 20, stream)
+        fl = ns_flops_per_step(shp, Mr, wl["K"], False)
+        lines.append({"metric": "Sign-Muon steps/s (ResNet-50 shapes, M=4)", "value": 1e3 / ms, "unit": "steps/s",
+                      "ms_per_step": ms, "ns_tflops_per_step": fl / 1e12, "d": synth.numel(shp)})
+        h.close()
+    for ln in lines:
+        print(json.dumps(ln), flush=True)
+    return 0
+
+
 def run_capture(args):
     """Profiler-capture mode (prints no bench line): the same step on the first
     L transformer layers of the nanoGPT shapes, M=8, a few steps."""
@@ -412,9 +499,13 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--capture-layers", type=int, default=0,
                     help="profiler capture mode on the first L layers; prints no bench line")
+    ap.add_argument("--workload", default="nanogpt", choices=["nanogpt", "llama_vote", "ns_sweep", "resnet50", "all"],
+                    help="nanogpt: the headline line; the others print secondary measurements only")
     args = ap.parse_args()
     if args.capture_layers > 0:
         return run_capture(args)
+    if args.workload != "nanogpt":
+        return run_secondary(args)
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":

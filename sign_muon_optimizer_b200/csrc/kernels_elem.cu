@@ -380,104 +380,226 @@ k_pack(const float* __restrict__ U, int64_t u_stride, int64_t d, uint8_t* __rest
 
 // ---------------------------------------------------------------------------
 // Majority vote ([paper] Algorithm 2: integer SUM of the signs then sign();
-// [blog]: ties give 0, sums lie in [-M, M]).  A block takes 1024 entries:
-// it stages the M workers' 128-byte slices in shared memory with 16-byte
-// loads, then each thread counts the +1 votes of 4 consecutive entries with
-// byte-lane counters (nibble * 0x00204081 & 0x01010101 spreads 4 bits into
-// 4 bytes) and writes 4 sums and 4 majority signs with vector stores.
-// ---------------------------------------------------------------------------
-constexpr int kVoteTile = 1024;
-
-struct BitsSrc {
-  const uint8_t* base;  // worker m at base + m*stride when ptrs == nullptr
-  int64_t stride;
-  const WorkerPtrs* ptrs;
-};
-
-__device__ __forceinline__ void count4(const uint32_t* sw, int M, int wi, int shift, int& c0,
-                                       int& c1, int& c2, int& c3) {
-  c0 = c1 = c2 = c3 = 0;
-  int m = 0;
-  while (m < M) {
-    const int end = min(M, m + 255);
-    uint32_t acc = 0;
-    for (; m < end; ++m) {
-      const uint32_t nib = (sw[m * 32 + wi] >> shift) & 0xFu;
-      acc += (nib * 0x00204081u) & 0x01010101u;
-    }
-    c0 += acc & 0xFF; c1 += (acc >> 8) & 0xFF; c2 += (acc >> 16) & 0xFF; c3 += acc >> 24;
-  }
-}
-
+// [blog]: ties give 0, sums lie in [-M, M]).
 __device__ __forceinline__ int sgn(int s) { return (s > 0) - (s < 0); }
 
 // MODE 0: API vote (sums + majority); 1: fused update of W; 2: write D = majority.
+// A warp takes 512 consecutive entries (4 blocks of 128) per step.  The 8
+// lanes of group j = lane / 8 share block j: each loads that block's 16 bytes
+// of every worker's stream (so one load instruction reads 64 contiguous
+// bytes per worker) and counts 4 of its 32 nibbles: lane g = lane % 8 takes
+// entries 32k + 4g .. 32k + 4g + 3 (k = 0..3), so that each store
+// instruction writes whole 128-byte lines.  Byte-lane counters: nibble *
+// 0x00204081 & 0x01010101 spreads 4 bits into 4 byte lanes, flushed every 248
+// workers so that no lane overflows; 8 workers' loads are in flight at once.
 template <int MODE, bool ACC8>
 __global__ void __launch_bounds__(kThreads)
 k_vote(WorkerPtrs signs, const uint8_t* __restrict__ bits, int64_t bits_stride, int M, int64_t d,
        void* __restrict__ sums, int8_t* __restrict__ maj, float* __restrict__ W, float eta,
        float* __restrict__ D, const int* __restrict__ status) {
-  extern __shared__ uint32_t sw[];  // [M][32]
   if (MODE == 1 && status != nullptr && (status[0] | status[1]) != 0) return;  // keep W on error
-  const int64_t n_full = d / kVoteTile;
-  for (int64_t t = blockIdx.x; t < n_full; t += gridDim.x) {
-    for (int idx = threadIdx.x; idx < M * 8; idx += kThreads) {
-      const int m = idx >> 3, v = idx & 7;
-      const uint8_t* src = (MODE == 0) ? reinterpret_cast<const uint8_t*>(signs.p[m]) : bits + (int64_t)m * bits_stride;
-      const uint4 x = reinterpret_cast<const uint4*>(src + t * 128)[v];
-      reinterpret_cast<uint4*>(sw + m * 32)[v] = x;
-    }
-    __syncthreads();
-    const int wi = threadIdx.x >> 3, shift = (threadIdx.x & 7) * 4;
-    int c0, c1, c2, c3;
-    count4(sw, M, wi, shift, c0, c1, c2, c3);
-    const int s0 = 2 * c0 - M, s1 = 2 * c1 - M, s2 = 2 * c2 - M, s3 = 2 * c3 - M;
-    const int64_t e = t * kVoteTile + threadIdx.x * 4;
-    if (MODE == 0) {
-      if (sums != nullptr) {
-        if (ACC8) {
-          char4 v = make_char4((signed char)s0, (signed char)s1, (signed char)s2, (signed char)s3);
-          *reinterpret_cast<char4*>(reinterpret_cast<int8_t*>(sums) + e) = v;
-        } else {
-          *reinterpret_cast<int4*>(reinterpret_cast<int32_t*>(sums) + e) = make_int4(s0, s1, s2, s3);
+  const int lane = threadIdx.x & 31;
+  const int64_t gw = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
+  const int64_t nw = ((int64_t)gridDim.x * kThreads) >> 5;
+  const int64_t nblk = d >> 7;                  // full 128-entry blocks
+  const int grp = lane >> 3, g = lane & 7, shift = 4 * g;
+  auto stream = [&](int m) {
+    return (MODE == 0) ? reinterpret_cast<const uint8_t*>(signs.p[m]) : bits + (int64_t)m * bits_stride;
+  };
+  for (int64_t st = gw; st * 4 < nblk; st += nw) {
+    const int64_t b = st * 4 + grp;               // this lane group's block
+    const bool on = b < nblk;
+    int cnt[4][4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) cnt[k][0] = cnt[k][1] = cnt[k][2] = cnt[k][3] = 0;
+    uint32_t acc[4] = {0u, 0u, 0u, 0u};
+    for (int m = 0; m < M; m += 8) {
+      uint4 wv[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        wv[i] = (on && m + i < M) ? __ldg(reinterpret_cast<const uint4*>(stream(m + i) + b * 16))
+                                  : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        acc[0] += (((wv[i].x >> shift) & 0xFu) * 0x00204081u) & 0x01010101u;
+        acc[1] += (((wv[i].y >> shift) & 0xFu) * 0x00204081u) & 0x01010101u;
+        acc[2] += (((wv[i].z >> shift) & 0xFu) * 0x00204081u) & 0x01010101u;
+        acc[3] += (((wv[i].w >> shift) & 0xFu) * 0x00204081u) & 0x01010101u;
+      }
+      if (((m + 8) % 248) == 0 || m + 8 >= M) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          cnt[k][0] += acc[k] & 0xFF;
+          cnt[k][1] += (acc[k] >> 8) & 0xFF;
+          cnt[k][2] += (acc[k] >> 16) & 0xFF;
+          cnt[k][3] += acc[k] >> 24;
+          acc[k] = 0;
         }
       }
-      if (maj != nullptr)
-        *reinterpret_cast<char4*>(maj + e) =
-            make_char4((signed char)sgn(s0), (signed char)sgn(s1), (signed char)sgn(s2), (signed char)sgn(s3));
-    } else if (MODE == 1) {
-      float4 w = ld4(W + e);
-      w.x = fmaf(-eta, (float)sgn(s0), w.x);
-      w.y = fmaf(-eta, (float)sgn(s1), w.y);
-      w.z = fmaf(-eta, (float)sgn(s2), w.z);
-      w.w = fmaf(-eta, (float)sgn(s3), w.w);
-      st4(W + e, w);
-    } else {
-      st4(D + e, make_float4((float)sgn(s0), (float)sgn(s1), (float)sgn(s2), (float)sgn(s3)));
     }
-    __syncthreads();
+    if (!on) continue;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int s0 = 2 * cnt[k][0] - M, s1 = 2 * cnt[k][1] - M, s2 = 2 * cnt[k][2] - M, s3 = 2 * cnt[k][3] - M;
+      const int64_t e = b * 128 + 32 * k + 4 * g;
+      if (MODE == 0) {
+        if (sums != nullptr) {
+          if (ACC8) {
+            char4 v = make_char4((signed char)s0, (signed char)s1, (signed char)s2, (signed char)s3);
+            *reinterpret_cast<char4*>(reinterpret_cast<int8_t*>(sums) + e) = v;
+          } else {
+            *reinterpret_cast<int4*>(reinterpret_cast<int32_t*>(sums) + e) = make_int4(s0, s1, s2, s3);
+          }
+        }
+        if (maj != nullptr)
+          *reinterpret_cast<char4*>(maj + e) =
+              make_char4((signed char)sgn(s0), (signed char)sgn(s1), (signed char)sgn(s2), (signed char)sgn(s3));
+      } else if (MODE == 1) {
+        float4 w = ld4(W + e);
+        w.x = fmaf(-eta, (float)sgn(s0), w.x);
+        w.y = fmaf(-eta, (float)sgn(s1), w.y);
+        w.z = fmaf(-eta, (float)sgn(s2), w.z);
+        w.w = fmaf(-eta, (float)sgn(s3), w.w);
+        st4(W + e, w);
+      } else {
+        st4(D + e, make_float4((float)sgn(s0), (float)sgn(s1), (float)sgn(s2), (float)sgn(s3)));
+      }
+    }
   }
-  // ragged tail (< 1024 entries): byte loads, one entry per thread
+  // ragged tail (< 128 entries): bit loads, one entry per thread
   if (blockIdx.x == gridDim.x - 1) {
-    for (int64_t e = n_full * kVoteTile + threadIdx.x; e < d; e += kThreads) {
+    for (int64_t e = nblk * 128 + threadIdx.x; e < d; e += kThreads) {
       int c = 0;
       for (int m = 0; m < M; ++m) {
         const uint8_t* src = (MODE == 0) ? reinterpret_cast<const uint8_t*>(signs.p[m]) : bits + (int64_t)m * bits_stride;
         c += (src[e >> 3] >> (e & 7)) & 1;
       }
-      const int s = 2 * c - M;
+      const int sm_ = 2 * c - M;
       if (MODE == 0) {
         if (sums != nullptr) {
-          if (ACC8) reinterpret_cast<int8_t*>(sums)[e] = (int8_t)s;
-          else reinterpret_cast<int32_t*>(sums)[e] = s;
+          if (ACC8) reinterpret_cast<int8_t*>(sums)[e] = (int8_t)sm_;
+          else reinterpret_cast<int32_t*>(sums)[e] = sm_;
         }
-        if (maj != nullptr) maj[e] = (int8_t)sgn(s);
+        if (maj != nullptr) maj[e] = (int8_t)sgn(sm_);
       } else if (MODE == 1) {
-        W[e] = fmaf(-eta, (float)sgn(s), W[e]);
+        W[e] = fmaf(-eta, (float)sgn(sm_), W[e]);
       } else {
-        D[e] = (float)sgn(s);
+        D[e] = (float)sgn(sm_);
       }
     }
+  }
+}
+
+// Streaming vote for M <= 255 (byte-lane counters): each warp takes tiles of 4096 consecutive entries (512 bytes of
+// every worker's stream).  The bytes come into shared memory by cp.async, 16
+// per lane (each load instruction reads 512 contiguous bytes of one stream),
+// kVoteBatch workers at a time, double-buffered so that the next batch is in
+// flight while this one is counted.  Lane t then counts entries 128 j + 4 t
+// .. + 3 for j = 0..31 (nibble t % 8 of word 4 j + t / 8, a shared-memory
+// broadcast among 8 lanes) into byte-lane counters, and writes each group of
+// 4 results with one vector store (the warp's stores are contiguous).
+constexpr int kVoteBatch = 8;
+constexpr int kVoteWarps = 4;                  // warps per block
+constexpr int kVoteTileB = 512;                // bytes of one stream per tile
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
+template <int MODE, bool ACC8>
+__global__ void __launch_bounds__(kVoteWarps * 32)
+k_vote_stream(WorkerPtrs signs, const uint8_t* __restrict__ bits, int64_t bits_stride, int M, int64_t ntiles,
+              void* __restrict__ sums, int8_t* __restrict__ maj, float* __restrict__ W, float eta,
+              float* __restrict__ D, const int* __restrict__ status) {
+  if (MODE == 1 && status != nullptr && (status[0] | status[1]) != 0) return;  // keep W on error
+  extern __shared__ __align__(16) uint8_t vsm[];   // [warp][2][kVoteBatch][512]
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int64_t gw = (int64_t)blockIdx.x * kVoteWarps + wid;
+  const int64_t nw = (int64_t)gridDim.x * kVoteWarps;
+  const uint32_t buf0 = (uint32_t)__cvta_generic_to_shared(vsm) + (uint32_t)wid * (2 * kVoteBatch * kVoteTileB);
+  const int nbatch = (M + kVoteBatch - 1) / kVoteBatch;
+  auto stream = [&](int m) {
+    return (MODE == 0) ? reinterpret_cast<const uint8_t*>(signs.p[m]) : bits + (int64_t)m * bits_stride;
+  };
+  // (tile, batch) work items of this warp, in order
+  int64_t tile = gw;
+  int batch = 0;
+  auto issue = [&](int64_t t, int bt, int buf) {
+    const uint32_t dst = buf0 + (uint32_t)buf * (kVoteBatch * kVoteTileB) + (uint32_t)lane * 16;
+#pragma unroll
+    for (int i = 0; i < kVoteBatch; ++i) {
+      const int m = bt * kVoteBatch + i;
+      if (m < M) cp_async16(dst + (uint32_t)i * kVoteTileB, stream(m) + t * kVoteTileB + lane * 16);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  if (tile >= ntiles) return;
+  issue(tile, 0, 0);
+  int cur = 0;
+  uint32_t acc[32];                            // byte lane i of acc[j]: entry 128 j + 4 lane + i
+#pragma unroll
+  for (int j = 0; j < 32; ++j) acc[j] = 0;
+  while (true) {
+    // the next work item goes out before this one is counted
+    int64_t ntile = tile;
+    int nbt = batch + 1;
+    if (nbt == nbatch) { nbt = 0; ntile += nw; }
+    if (ntile < ntiles) {
+      issue(ntile, nbt, cur ^ 1);
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+    } else {
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+    }
+    __syncwarp();
+    const uint32_t src = buf0 + (uint32_t)cur * (kVoteBatch * kVoteTileB);
+    const int nm = min(kVoteBatch, M - batch * kVoteBatch);
+    const int shift = (lane & 7) * 4;
+    for (int i = 0; i < nm; ++i) {
+      const uint32_t row = src + (uint32_t)i * kVoteTileB + (uint32_t)(lane >> 3) * 4;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        uint32_t w;
+        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w) : "r"(row + (uint32_t)j * 16));
+        acc[j] += ((w >> shift) & 0xFu) * 0x00204081u & 0x01010101u;
+      }
+    }
+    __syncwarp();
+    if (batch == nbatch - 1) {
+      // tile done: write its 4096 results
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const int c0 = acc[j] & 0xFF, c1 = (acc[j] >> 8) & 0xFF, c2 = (acc[j] >> 16) & 0xFF, c3 = acc[j] >> 24;
+        acc[j] = 0;
+        const int s0 = 2 * c0 - M, s1 = 2 * c1 - M, s2 = 2 * c2 - M, s3 = 2 * c3 - M;
+        const int64_t e = tile * 4096 + j * 128 + lane * 4;
+        if (MODE == 0) {
+          if (sums != nullptr) {
+            if (ACC8) {
+              *reinterpret_cast<char4*>(reinterpret_cast<int8_t*>(sums) + e) =
+                  make_char4((signed char)s0, (signed char)s1, (signed char)s2, (signed char)s3);
+            } else {
+              *reinterpret_cast<int4*>(reinterpret_cast<int32_t*>(sums) + e) = make_int4(s0, s1, s2, s3);
+            }
+          }
+          if (maj != nullptr)
+            *reinterpret_cast<char4*>(maj + e) =
+                make_char4((signed char)sgn(s0), (signed char)sgn(s1), (signed char)sgn(s2), (signed char)sgn(s3));
+        } else if (MODE == 1) {
+          float4 wv = ld4(W + e);
+          wv.x = fmaf(-eta, (float)sgn(s0), wv.x);
+          wv.y = fmaf(-eta, (float)sgn(s1), wv.y);
+          wv.z = fmaf(-eta, (float)sgn(s2), wv.z);
+          wv.w = fmaf(-eta, (float)sgn(s3), wv.w);
+          st4(W + e, wv);
+        } else {
+          st4(D + e, make_float4((float)sgn(s0), (float)sgn(s1), (float)sgn(s2), (float)sgn(s3)));
+        }
+      }
+    }
+    tile = ntile;
+    batch = nbt;
+    cur ^= 1;
+    if (tile >= ntiles) break;
   }
 }
 
@@ -699,40 +821,56 @@ void launch_pack(cudaStream_t s, const float* U, int64_t u_stride, int64_t d, ui
   k_pack<<<grid, kThreads, 0, s>>>(U, u_stride, d, out, out_stride);
 }
 
+// Full 4096-entry tiles by the streaming kernel (M <= 255), the rest (and
+// every entry for larger M) by the register kernel on offset pointers.
+template <int MODE, bool ACC8>
+void vote_dispatch(cudaStream_t s, WorkerPtrs signs, const uint8_t* bits, int64_t bits_stride, int M, int64_t d,
+                   void* sums, int8_t* maj, float* W, float eta, float* D, const int* status) {
+  int64_t done = 0;
+  if (M <= 255 && d >= 4096) {
+    const int64_t ntiles = d / 4096;
+    const size_t smem = (size_t)kVoteWarps * 2 * kVoteBatch * kVoteTileB;
+    const int64_t want = (ntiles + kVoteWarps - 1) / kVoteWarps;
+    const int64_t cap = (int64_t)num_sms() * 6;
+    const int blocks = (int)(want < cap ? want : cap);
+    count_launch();
+    k_vote_stream<MODE, ACC8><<<blocks, kVoteWarps * 32, smem, s>>>(signs, bits, bits_stride, M, ntiles, sums, maj, W,
+                                                                     eta, D, status);
+    done = ntiles * 4096;
+  }
+  const int64_t rest = d - done;
+  if (rest <= 0) return;
+  const int64_t boff = done / 8;  // byte offset in every stream (a multiple of 512)
+  WorkerPtrs sp = signs;
+  if (MODE == 0)
+    for (int m = 0; m < M; ++m) sp.p[m] = reinterpret_cast<const float*>(reinterpret_cast<const uint8_t*>(signs.p[m]) + boff);
+  void* sums2 = sums == nullptr ? nullptr : reinterpret_cast<uint8_t*>(sums) + done * (ACC8 ? 1 : 4);
+  count_launch();
+  const int blocks = stream_grid((rest / 512 + 8) / 8 + 1, 8);
+  k_vote<MODE, ACC8><<<blocks, kThreads, 0, s>>>(sp, bits == nullptr ? nullptr : bits + boff, bits_stride, M, rest, sums2,
+                                                 maj == nullptr ? nullptr : maj + done, W == nullptr ? nullptr : W + done,
+                                                 eta, D == nullptr ? nullptr : D + done, status);
+}
+
 void launch_vote(cudaStream_t s, const WorkerPtrs& signs, int M, int64_t d, void* sums, int acc8,
                  int8_t* majority) {
   if (d <= 0) return;
-  count_launch();
-  const int blocks = stream_grid(d / kVoteTile + 1, 8);
-  const size_t smem = (size_t)M * 32 * 4;
-  if (acc8)
-    k_vote<0, true><<<blocks, kThreads, smem, s>>>(signs, nullptr, 0, M, d, sums, majority, nullptr,
-                                                   0.f, nullptr, nullptr);
-  else
-    k_vote<0, false><<<blocks, kThreads, smem, s>>>(signs, nullptr, 0, M, d, sums, majority, nullptr,
-                                                    0.f, nullptr, nullptr);
+  if (acc8) vote_dispatch<0, true>(s, signs, nullptr, 0, M, d, sums, majority, nullptr, 0.f, nullptr, nullptr);
+  else vote_dispatch<0, false>(s, signs, nullptr, 0, M, d, sums, majority, nullptr, 0.f, nullptr, nullptr);
 }
 
 void launch_vote_update(cudaStream_t s, const uint8_t* bits, int64_t bits_stride, int M, int64_t d,
                         float* W, float eta, const int* status) {
   if (d <= 0) return;
-  count_launch();
-  const int blocks = stream_grid(d / kVoteTile + 1, 8);
-  const size_t smem = (size_t)M * 32 * 4;
   WorkerPtrs none{};
-  k_vote<1, false><<<blocks, kThreads, smem, s>>>(none, bits, bits_stride, M, d, nullptr, nullptr, W,
-                                                  eta, nullptr, status);
+  vote_dispatch<1, false>(s, none, bits, bits_stride, M, d, nullptr, nullptr, W, eta, nullptr, status);
 }
 
 void launch_vote_major(cudaStream_t s, const uint8_t* bits, int64_t bits_stride, int M, int64_t d,
                        float* D) {
   if (d <= 0) return;
-  count_launch();
-  const int blocks = stream_grid(d / kVoteTile + 1, 8);
-  const size_t smem = (size_t)M * 32 * 4;
   WorkerPtrs none{};
-  k_vote<2, false><<<blocks, kThreads, smem, s>>>(none, bits, bits_stride, M, d, nullptr, nullptr,
-                                                  nullptr, 0.f, D, nullptr);
+  vote_dispatch<2, false>(s, none, bits, bits_stride, M, d, nullptr, nullptr, nullptr, 0.f, D, nullptr);
 }
 
 void launch_vote_stage(cudaStream_t s, const uint8_t* bits, int64_t bits_stride, int M, void* X, int x_bf16,
