@@ -56,9 +56,12 @@ def test_vote_blog_worked_example():
     assert host(maj)[:4].reshape(2, 2).tolist() == g["majority"]
 
 
-@pytest.mark.parametrize("M", [1, 2, 3, 16, 127, 200])
-@pytest.mark.parametrize("d", [1, 7, 1024, 5000, 40 * 1024 + 3])
+@pytest.mark.parametrize("M", [1, 2, 3, 16, 127, 200, 256])
+@pytest.mark.parametrize("d", [1, 7, 1024, 5000, 8192, 40 * 1024 + 3])
 def test_vote_bit_exact(M, d):
+    # d = 8192: whole 4096-entry tiles only; 5000 and 40963: tiles plus a
+    # ragged rest; M = 256: above the byte-lane counters' range (all entries
+    # on the register kernel)
     bits = synth.bernoulli_bits(d, M, config_id=M * 1000 + d % 997)
     packed = [ref.pack_bits(b) for b in bits]
     want_sums = ref.vote_sums_from_bits(packed, d, "int32")
