@@ -410,8 +410,10 @@ def run_secondary(args):
     stream = torch.cuda.current_stream()
     pk, pk_kind = peaks()
     lines = []
-    if args.workload in ("llama_vote", "all"):
-        shapes = synth.LLAMA_LAYER_SHAPES
+    if args.workload in ("llama_vote", "vote_100m", "all"):
+        # vote_100m: the same kernel on one 1 x 100,000,000 matrix (a small
+        # case for profiler captures)
+        shapes = [(1, 100_000_000)] if args.workload == "vote_100m" else synth.LLAMA_LAYER_SHAPES
         Mv = synth.WORKLOADS["llama_vote"]["M"]
         d = synth.numel(shapes)
         nb = (d + 7) // 8
@@ -426,7 +428,8 @@ def run_secondary(args):
             ms = _events_time(lambda: h.vote(signs, d, sums, maj), 5, stream)
             nbytes = Mv * d / 8.0 + (1.0 if acc8 else 4.0) * d + d
             gbs = nbytes / (ms / 1e3) / 1e9
-            lines.append({"metric": "vote GB/s (LLaMA-layer shapes, M=16, " + ("int8" if acc8 else "int32") + " sums)",
+            shp_name = "1 x 100,000,000" if args.workload == "vote_100m" else "LLaMA-layer shapes"
+            lines.append({"metric": f"vote GB/s ({shp_name}, M=16, " + ("int8" if acc8 else "int32") + " sums)",
                           "value": gbs, "unit": "GB/s", "frac_of_hbm": gbs / pk["hbm_gbs"], "peak_kind": pk_kind,
                           "ms": ms, "bytes": nbytes, "d": d, "M": Mv, "payload_bytes_per_worker": nb,
                           "acc_dtype": "int8" if acc8 else "int32", "collective": "none (on-device vote)"})
@@ -499,7 +502,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--capture-layers", type=int, default=0,
                     help="profiler capture mode on the first L layers; prints no bench line")
-    ap.add_argument("--workload", default="nanogpt", choices=["nanogpt", "llama_vote", "ns_sweep", "resnet50", "all"],
+    ap.add_argument("--workload", default="nanogpt", choices=["nanogpt", "llama_vote", "vote_100m", "ns_sweep", "resnet50", "all"],
                     help="nanogpt: the headline line; the others print secondary measurements only")
     args = ap.parse_args()
     if args.capture_layers > 0:

@@ -626,8 +626,7 @@ k_vote_stage(const uint8_t* __restrict__ bits, int64_t bits_stride, int M, void*
   if (vec) {
     // 8 consecutive entries per thread and step: one byte of every worker's
     // stream, counted in two SWAR accumulators (byte lane i of lo / hi counts
-    // entry i / i + 4, 255 workers at a time); both steps' bytes are loaded
-    // before any is counted
+    // entry i / i + 4)
     constexpr int kV = kChunk / (kThreads * 8);
     int64_t fe[kV];
     bool on[kV];
@@ -642,27 +641,37 @@ k_vote_stage(const uint8_t* __restrict__ bits, int64_t bits_stride, int M, void*
     for (int j = 0; j < kV; ++j)
 #pragma unroll
       for (int i = 0; i < 8; ++i) cnt[j][i] = 0;
-    for (int m = 0; m < M;) {
-      const int end = min(M, m + 255);
-      uint32_t lo[kV], hi[kV];
+    // 8 workers' bytes are loaded before any is counted (one memory round
+    // trip per 8 workers, not one per worker); counters flushed every 248
+    uint32_t lo[kV], hi[kV];
 #pragma unroll
-      for (int j = 0; j < kV; ++j) lo[j] = hi[j] = 0;
-      for (; m < end; ++m) {
-        const uint8_t* bm = bits + (int64_t)m * bits_stride;
+    for (int j = 0; j < kV; ++j) lo[j] = hi[j] = 0;
+    for (int m = 0; m < M; m += 8) {
+      uint32_t by[8][kV];
 #pragma unroll
-        for (int j = 0; j < kV; ++j) {
-          const uint32_t by = on[j] ? bm[fe[j] >> 3] : 0u;
-          lo[j] += ((by & 0xFu) * 0x00204081u) & 0x01010101u;
-          hi[j] += ((by >> 4) * 0x00204081u) & 0x01010101u;
-        }
+      for (int i = 0; i < 8; ++i) {
+        const uint8_t* bm = bits + (int64_t)(m + i) * bits_stride;
+#pragma unroll
+        for (int j = 0; j < kV; ++j) by[i][j] = (m + i < M && on[j]) ? (uint32_t)bm[fe[j] >> 3] : 0u;
       }
 #pragma unroll
-      for (int j = 0; j < kV; ++j)
+      for (int i = 0; i < 8; ++i)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          cnt[j][i] += (lo[j] >> (8 * i)) & 0xFF;
-          cnt[j][i + 4] += (hi[j] >> (8 * i)) & 0xFF;
+        for (int j = 0; j < kV; ++j) {
+          lo[j] += ((by[i][j] & 0xFu) * 0x00204081u) & 0x01010101u;
+          hi[j] += ((by[i][j] >> 4) * 0x00204081u) & 0x01010101u;
         }
+      if (((m + 8) % 248) == 0 || m + 8 >= M) {
+#pragma unroll
+        for (int j = 0; j < kV; ++j) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            cnt[j][i] += (lo[j] >> (8 * i)) & 0xFF;
+            cnt[j][i + 4] += (hi[j] >> (8 * i)) & 0xFF;
+          }
+          lo[j] = hi[j] = 0;
+        }
+      }
     }
 #pragma unroll
     for (int j = 0; j < kV; ++j) {
