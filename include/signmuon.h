@@ -59,6 +59,18 @@ typedef struct signmuon_ctx* signmuon_t;
 #define SIGNMUON_KEEP_POLAR  (1u << 6) /* signmuon_step also writes U for signmuon_get_polar; without it
                                           the last Newton-Schulz GEMM of a step writes only the one-bit
                                           signs when every matrix has a multiple of 32 columns */
+/* Named variants ([paper] "SignMuon: 通信高效的分布式Muon优化" Algorithm 2, §4, Table 1):
+ * TIE_PLUS           a tied vote (sum 0, even M) gives +1 instead of 0 (Algorithm 2's sign
+ *                    default on the {-1, +1} wire); applies to signmuon_vote's majority and
+ *                    to the step.
+ * POLAR_AFTER_ONLY   the step signs the momentum itself and orthogonalises only after the
+ *                    vote (§4 "where to orthogonalise"); requires SIGNMUON_POST_POLAR.
+ * MUON_MEAN          the Muon baseline instead of Sign-Muon: D = PolarNS(mean of the M
+ *                    workers' momenta), W <- fl32(W - eta D); no signs, no vote; cannot be
+ *                    combined with POST_POLAR or POLAR_AFTER_ONLY. */
+#define SIGNMUON_TIE_PLUS          (1u << 7)
+#define SIGNMUON_POLAR_AFTER_ONLY  (1u << 8)
+#define SIGNMUON_MUON_MEAN         (1u << 9)
 
 /* ------------------------------------------------------------------------
  * signmuon_init -- plan the step and allocate its device state.
@@ -150,8 +162,9 @@ int signmuon_polar(signmuon_t h, const float* const* X, float* const* U);
  * get_polar: worker m's U from the last step (or signmuon_polar call);
  * SIGNMUON_E_UNSUPPORTED when the step did not keep it (handle made without
  * SIGNMUON_KEEP_POLAR on shapes whose signs are packed inside the last
- * Newton-Schulz GEMM).  get_signs: worker m's packed bits from the last
- * step.  get_direction: the last step's D.
+ * Newton-Schulz GEMM, and always with POLAR_AFTER_ONLY or MUON_MEAN).
+ * get_signs: worker m's packed bits from the last step (SIGNMUON_E_UNSUPPORTED
+ * with MUON_MEAN).  get_direction: the last step's D.
  * get_scales: host float[M*n_mats]: the last step's scale s per (worker,
  * matrix), worker-major (waits for the GPU).
  * ---------------------------------------------------------------------- */

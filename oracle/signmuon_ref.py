@@ -209,9 +209,16 @@ def vote_sums_ternary(sign_list):
     return total.astype(np.int32)
 
 
-def majority(sums):
-    """sign(sum) with a tie (sum 0) mapped to 0 (R7, [blog])."""
-    return sign_ternary(sums).astype(np.int8)
+def majority(sums, tie=0):
+    """sign(sum) with a tie (sum 0) mapped to 0 (R7, [blog]); with tie=+1 a
+    tie gives +1 instead, [paper] Algorithm 2's default for sign(0) on the
+    {-1, +1} wire (a named variant)."""
+    maj = sign_ternary(sums).astype(np.int8)
+    if tie == 1:
+        maj[np.asarray(sums) == 0] = 1
+    elif tie != 0:
+        raise ValueError("tie must be 0 or 1")
+    return maj
 
 
 # ---------------------------------------------------------------------------
@@ -261,36 +268,46 @@ def split(flat, shapes, offsets=None):
     return out
 
 
+def polar_flat(flat, shapes, K, eps, scale, P=1, order="cubic"):
+    """PolarNS of every matrix of a flat vector, returned flat (float64)."""
+    out = np.empty(int(np.asarray(flat).size), np.float64)
+    off = 0
+    for (r, c), mat in zip(shapes, split(np.asarray(flat, np.float64), shapes)):
+        out[off: off + r * c] = polar_ns(mat, K, eps, scale, P, order).ravel()
+        off += r * c
+    return out
+
+
 def step(W, G_list, mom_list, shapes, *, beta, lam, eta, K, eps, scale, P=1,
-         order="cubic", post_polar=False, acc="int32"):
+         order="cubic", post_polar=False, acc="int32", tie=0, pre_polar=True):
     """One distributed Sign-Muon step ([paper] Algorithm 2, with the vote of
     [blog] and the optional post-vote polar step of [paper] §4).
 
-    Returns a dict with the new momentum (float64), the polar factors U_m,
-    the packed bits, the vote sums, the majority, the direction D and the new
-    W (float32).  Inputs are flat vectors; momentum is float64 or float32.
+    Named variants: tie=1 sends a tied vote to +1 ([paper] Algorithm 2's
+    default); pre_polar=False signs the momentum itself and orthogonalises
+    only after the vote ([paper] §4 "where to orthogonalise", the
+    after-only placement; needs post_polar=True).
+
+    Returns a dict with the new momentum (float64), the polar factors U_m
+    (the momentum itself when pre_polar is False), the packed bits, the vote
+    sums, the majority, the direction D and the new W (float32).  Inputs are
+    flat vectors; momentum is float64 or float32.
     """
+    if not pre_polar and not post_polar:
+        raise ValueError("pre_polar=False needs post_polar=True")
     M = len(G_list)
     d = int(np.asarray(W).size)
     new_mom, U_list, packed = [], [], []
     for m in range(M):
         mom = momentum_update(mom_list[m], G_list[m], W, beta, lam)
         new_mom.append(mom)
-        u = np.empty(d, np.float64)
-        off = 0
-        for (r, c), mat in zip(shapes, split(mom, shapes)):
-            u[off: off + r * c] = polar_ns(mat, K, eps, scale, P, order).ravel()
-            off += r * c
+        u = polar_flat(mom, shapes, K, eps, scale, P, order) if pre_polar else np.asarray(mom, np.float64)
         U_list.append(u)
         packed.append(pack_bits(sign_bits(u)))
     sums = vote_sums_from_bits(packed, d, acc)
-    maj = majority(sums)
+    maj = majority(sums, tie)
     if post_polar:
-        D = np.empty(d, np.float64)
-        off = 0
-        for (r, c), mat in zip(shapes, split(maj.astype(np.float64), shapes)):
-            D[off: off + r * c] = polar_ns(mat, K, eps, scale, P, order).ravel()
-            off += r * c
+        D = polar_flat(maj.astype(np.float64), shapes, K, eps, scale, P, order)
         D32 = D.astype(np.float32)
     else:
         D = maj.astype(np.float64)
@@ -298,3 +315,16 @@ def step(W, G_list, mom_list, shapes, *, beta, lam, eta, K, eps, scale, P=1,
     W_new = update(W, D32, eta)
     return dict(mom=new_mom, U=U_list, packed=packed, sums=sums, majority=maj,
                 D=D, D32=D32, W=W_new)
+
+
+def muon_step(W, G_list, mom_list, shapes, *, beta, lam, eta, K, eps, scale, P=1, order="cubic"):
+    """The Muon baseline the pages compare against ([paper] §4 Muon update,
+    Table 1's "Muon" row): the workers' momenta are averaged (the all-reduce
+    of full-precision momentum) and the mean goes through one PolarNS per
+    matrix; W_new = fl32(W - eta * D) with D = PolarNS(mean Mom)."""
+    M = len(G_list)
+    new_mom = [momentum_update(mom_list[m], G_list[m], W, beta, lam) for m in range(M)]
+    mean = np.sum(np.stack([np.asarray(x, np.float64) for x in new_mom]), axis=0) / M
+    D = polar_flat(mean, shapes, K, eps, scale, P, order)
+    D32 = D.astype(np.float32)
+    return dict(mom=new_mom, mean=mean, D=D, D32=D32, W=update(W, D32, eta))

@@ -36,6 +36,9 @@ SIGNMUON_ACC_INT8 = 1 << 3
 SIGNMUON_ASYNC = 1 << 4
 SIGNMUON_VOTE_ONLY = 1 << 5
 SIGNMUON_KEEP_POLAR = 1 << 6
+SIGNMUON_TIE_PLUS = 1 << 7
+SIGNMUON_POLAR_AFTER_ONLY = 1 << 8
+SIGNMUON_MUON_MEAN = 1 << 9
 
 EXPORTED = [
     "signmuon_init", "signmuon_step", "signmuon_step_host", "signmuon_vote", "signmuon_pack",

@@ -147,12 +147,15 @@ void launch_scale_flat(cudaStream_t s, const WorkerPtrs& in, int M, float* out, 
 void launch_pack(cudaStream_t s, const float* U, int64_t u_stride, int64_t d, uint8_t* out,
                  int64_t out_stride, int M);
 void launch_vote(cudaStream_t s, const WorkerPtrs& signs, int M, int64_t d, void* sums, int acc8,
-                 int8_t* majority);
+                 int8_t* majority, int tie_plus);
 void launch_vote_update(cudaStream_t s, const uint8_t* bits, int64_t bits_stride, int M, int64_t d,
-                        float* W, float eta, const int* status);
+                        float* W, float eta, const int* status, int tie_plus);
 void launch_vote_major(cudaStream_t s, const uint8_t* bits, int64_t bits_stride, int M, int64_t d,
-                       float* D);
+                       float* D, int tie_plus);
 void launch_vote_stage(cudaStream_t s, const uint8_t* bits, int64_t bits_stride, int M, void* X, int x_bf16,
+                       const Chunk* chunks, int n_chunks, const MatInfo* mats, const GroupInfo* groups,
+                       float* partials, float* D, int tie_plus);
+void launch_mean_stage(cudaStream_t s, const float* Mom, int64_t mom_stride, int M, void* X, int x_bf16,
                        const Chunk* chunks, int n_chunks, const MatInfo* mats, const GroupInfo* groups,
                        float* partials, float* D);
 void launch_update(cudaStream_t s, float* W, const float* D, int64_t d, float eta,

@@ -382,6 +382,9 @@ k_pack(const float* __restrict__ U, int64_t u_stride, int64_t d, uint8_t* __rest
 // Majority vote ([paper] Algorithm 2: integer SUM of the signs then sign();
 // [blog]: ties give 0, sums lie in [-M, M]).
 __device__ __forceinline__ int sgn(int s) { return (s > 0) - (s < 0); }
+// majority of a vote sum: sign(s) with a tie sent to 0, or to +1 when
+// tie_plus is set ([paper] Algorithm 2's default, a named variant)
+__device__ __forceinline__ int vmaj(int s, int tie_plus) { return tie_plus ? (s >= 0 ? 1 : -1) : sgn(s); }
 
 // MODE 0: API vote (sums + majority); 1: fused update of W; 2: write D = majority.
 // A warp takes 512 consecutive entries (4 blocks of 128) per step.  The 8
@@ -396,7 +399,7 @@ template <int MODE, bool ACC8>
 __global__ void __launch_bounds__(kThreads)
 k_vote(WorkerPtrs signs, const uint8_t* __restrict__ bits, int64_t bits_stride, int M, int64_t d,
        void* __restrict__ sums, int8_t* __restrict__ maj, float* __restrict__ W, float eta,
-       float* __restrict__ D, const int* __restrict__ status) {
+       float* __restrict__ D, const int* __restrict__ status, int tie_plus) {
   if (MODE == 1 && status != nullptr && (status[0] | status[1]) != 0) return;  // keep W on error
   const int lane = threadIdx.x & 31;
   const int64_t gw = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
@@ -453,16 +456,16 @@ k_vote(WorkerPtrs signs, const uint8_t* __restrict__ bits, int64_t bits_stride, 
         }
         if (maj != nullptr)
           *reinterpret_cast<char4*>(maj + e) =
-              make_char4((signed char)sgn(s0), (signed char)sgn(s1), (signed char)sgn(s2), (signed char)sgn(s3));
+              make_char4((signed char)vmaj(s0, tie_plus), (signed char)vmaj(s1, tie_plus), (signed char)vmaj(s2, tie_plus), (signed char)vmaj(s3, tie_plus));
       } else if (MODE == 1) {
         float4 w = ld4(W + e);
-        w.x = fmaf(-eta, (float)sgn(s0), w.x);
-        w.y = fmaf(-eta, (float)sgn(s1), w.y);
-        w.z = fmaf(-eta, (float)sgn(s2), w.z);
-        w.w = fmaf(-eta, (float)sgn(s3), w.w);
+        w.x = fmaf(-eta, (float)vmaj(s0, tie_plus), w.x);
+        w.y = fmaf(-eta, (float)vmaj(s1, tie_plus), w.y);
+        w.z = fmaf(-eta, (float)vmaj(s2, tie_plus), w.z);
+        w.w = fmaf(-eta, (float)vmaj(s3, tie_plus), w.w);
         st4(W + e, w);
       } else {
-        st4(D + e, make_float4((float)sgn(s0), (float)sgn(s1), (float)sgn(s2), (float)sgn(s3)));
+        st4(D + e, make_float4((float)vmaj(s0, tie_plus), (float)vmaj(s1, tie_plus), (float)vmaj(s2, tie_plus), (float)vmaj(s3, tie_plus)));
       }
     }
   }
@@ -480,11 +483,11 @@ k_vote(WorkerPtrs signs, const uint8_t* __restrict__ bits, int64_t bits_stride, 
           if (ACC8) reinterpret_cast<int8_t*>(sums)[e] = (int8_t)sm_;
           else reinterpret_cast<int32_t*>(sums)[e] = sm_;
         }
-        if (maj != nullptr) maj[e] = (int8_t)sgn(sm_);
+        if (maj != nullptr) maj[e] = (int8_t)vmaj(sm_, tie_plus);
       } else if (MODE == 1) {
-        W[e] = fmaf(-eta, (float)sgn(sm_), W[e]);
+        W[e] = fmaf(-eta, (float)vmaj(sm_, tie_plus), W[e]);
       } else {
-        D[e] = (float)sgn(sm_);
+        D[e] = (float)vmaj(sm_, tie_plus);
       }
     }
   }
@@ -510,7 +513,7 @@ template <int MODE, bool ACC8>
 __global__ void __launch_bounds__(kVoteWarps * 32)
 k_vote_stream(WorkerPtrs signs, const uint8_t* __restrict__ bits, int64_t bits_stride, int M, int64_t ntiles,
               void* __restrict__ sums, int8_t* __restrict__ maj, float* __restrict__ W, float eta,
-              float* __restrict__ D, const int* __restrict__ status) {
+              float* __restrict__ D, const int* __restrict__ status, int tie_plus) {
   if (MODE == 1 && status != nullptr && (status[0] | status[1]) != 0) return;  // keep W on error
   extern __shared__ __align__(16) uint8_t vsm[];   // [warp][2][kVoteBatch][512]
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
@@ -583,16 +586,16 @@ k_vote_stream(WorkerPtrs signs, const uint8_t* __restrict__ bits, int64_t bits_s
           }
           if (maj != nullptr)
             *reinterpret_cast<char4*>(maj + e) =
-                make_char4((signed char)sgn(s0), (signed char)sgn(s1), (signed char)sgn(s2), (signed char)sgn(s3));
+                make_char4((signed char)vmaj(s0, tie_plus), (signed char)vmaj(s1, tie_plus), (signed char)vmaj(s2, tie_plus), (signed char)vmaj(s3, tie_plus));
         } else if (MODE == 1) {
           float4 wv = ld4(W + e);
-          wv.x = fmaf(-eta, (float)sgn(s0), wv.x);
-          wv.y = fmaf(-eta, (float)sgn(s1), wv.y);
-          wv.z = fmaf(-eta, (float)sgn(s2), wv.z);
-          wv.w = fmaf(-eta, (float)sgn(s3), wv.w);
+          wv.x = fmaf(-eta, (float)vmaj(s0, tie_plus), wv.x);
+          wv.y = fmaf(-eta, (float)vmaj(s1, tie_plus), wv.y);
+          wv.z = fmaf(-eta, (float)vmaj(s2, tie_plus), wv.z);
+          wv.w = fmaf(-eta, (float)vmaj(s3, tie_plus), wv.w);
           st4(W + e, wv);
         } else {
-          st4(D + e, make_float4((float)sgn(s0), (float)sgn(s1), (float)sgn(s2), (float)sgn(s3)));
+          st4(D + e, make_float4((float)vmaj(s0, tie_plus), (float)vmaj(s1, tie_plus), (float)vmaj(s2, tie_plus), (float)vmaj(s3, tie_plus)));
         }
       }
     }
@@ -612,7 +615,7 @@ k_vote_stream(WorkerPtrs signs, const uint8_t* __restrict__ bits, int64_t bits_s
 __global__ void __launch_bounds__(kThreads)
 k_vote_stage(const uint8_t* __restrict__ bits, int64_t bits_stride, int M, void* __restrict__ X, int x_bf16,
              const Chunk* __restrict__ chunks, const MatInfo* __restrict__ mats,
-             const GroupInfo* __restrict__ groups, float* __restrict__ partials, float* __restrict__ D) {
+             const GroupInfo* __restrict__ groups, float* __restrict__ partials, float* __restrict__ D, int tie_plus) {
   __shared__ float red[32];
   const Chunk ch = chunks[blockIdx.x];
   const MatInfo mi = mats[ch.mat];
@@ -679,7 +682,7 @@ k_vote_stage(const uint8_t* __restrict__ bits, int64_t bits_stride, int M, void*
       float v[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        v[i] = (float)sgn(2 * cnt[j][i] - M);
+        v[i] = (float)vmaj(2 * cnt[j][i] - M, tie_plus);
         ss += v[i] * v[i];
       }
       const float4 v0 = make_float4(v[0], v[1], v[2], v[3]), v1 = make_float4(v[4], v[5], v[6], v[7]);
@@ -697,12 +700,62 @@ k_vote_stage(const uint8_t* __restrict__ bits, int64_t bits_stride, int M, void*
       const int64_t fe = base + e;
       int c = 0;
       for (int m = 0; m < M; ++m) c += (bits[(int64_t)m * bits_stride + (fe >> 3)] >> (fe & 7)) & 1;
-      const float v = (float)sgn(2 * c - M);
+      const float v = (float)vmaj(2 * c - M, tie_plus);
       ss += v * v;
       if (D != nullptr) D[fe] = v;
       const int le = (int)(ch.start + e);
       const int r = le / mi.cols, cc = le - r * mi.cols;
       store_x(X, xb + (int64_t)r * gi.ld + cc, v, bf);
+    }
+  }
+  const float t = block_sum<float>(ss, red);
+  if (threadIdx.x == 0) partials[blockIdx.x] = t;
+}
+
+// Muon baseline ([paper] §4 Muon update, Table 1): the mean of the M
+// workers' momenta (summed in worker order in fp32, times 1/M) staged into
+// the Newton-Schulz input of one problem set, with its sum-of-squares
+// partials; the fp32 mean also goes to D when non-null (K == 0).
+__global__ void __launch_bounds__(kThreads)
+k_mean_stage(const float* __restrict__ Mom, int64_t mom_stride, int M, void* __restrict__ X, int x_bf16,
+             const Chunk* __restrict__ chunks, const MatInfo* __restrict__ mats,
+             const GroupInfo* __restrict__ groups, float* __restrict__ partials, float* __restrict__ D) {
+  __shared__ float red[32];
+  const Chunk ch = chunks[blockIdx.x];
+  const MatInfo mi = mats[ch.mat];
+  const GroupInfo gi = groups[mi.group];
+  const int64_t base = mi.off + ch.start;
+  const bool vec = ((base & 3) == 0) && ((ch.len & 3) == 0) && ((mi.cols & 3) == 0);
+  const bool bf = x_bf16 != 0;
+  const int64_t xb = gi.x_base + (int64_t)mi.q * gi.rows * gi.ld;
+  const float inv = 1.f / (float)M;
+  float ss = 0.f;
+  if (vec) {
+    for (int e = threadIdx.x * 4; e < ch.len; e += kThreads * 4) {
+      const int64_t fe = base + e;
+      float4 acc = ld4(Mom + fe);
+      for (int m = 1; m < M; ++m) {
+        const float4 v = ld4(Mom + (int64_t)m * mom_stride + fe);
+        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+      }
+      acc.x *= inv; acc.y *= inv; acc.z *= inv; acc.w *= inv;
+      ss += acc.x * acc.x + acc.y * acc.y + acc.z * acc.z + acc.w * acc.w;
+      if (D != nullptr) st4(D + fe, acc);
+      const int le = (int)(ch.start + e);
+      const int r = le / mi.cols, c = le - r * mi.cols;
+      store_x4(X, xb + (int64_t)r * gi.ld + c, acc, bf);
+    }
+  } else {
+    for (int e = threadIdx.x; e < ch.len; e += kThreads) {
+      const int64_t fe = base + e;
+      float acc = Mom[fe];
+      for (int m = 1; m < M; ++m) acc += Mom[(int64_t)m * mom_stride + fe];
+      acc *= inv;
+      ss += acc * acc;
+      if (D != nullptr) D[fe] = acc;
+      const int le = (int)(ch.start + e);
+      const int r = le / mi.cols, c = le - r * mi.cols;
+      store_x(X, xb + (int64_t)r * gi.ld + c, acc, bf);
     }
   }
   const float t = block_sum<float>(ss, red);
@@ -834,7 +887,7 @@ void launch_pack(cudaStream_t s, const float* U, int64_t u_stride, int64_t d, ui
 // every entry for larger M) by the register kernel on offset pointers.
 template <int MODE, bool ACC8>
 void vote_dispatch(cudaStream_t s, WorkerPtrs signs, const uint8_t* bits, int64_t bits_stride, int M, int64_t d,
-                   void* sums, int8_t* maj, float* W, float eta, float* D, const int* status) {
+                   void* sums, int8_t* maj, float* W, float eta, float* D, const int* status, int tie_plus) {
   int64_t done = 0;
   if (M <= 255 && d >= 4096) {
     const int64_t ntiles = d / 4096;
@@ -844,7 +897,7 @@ void vote_dispatch(cudaStream_t s, WorkerPtrs signs, const uint8_t* bits, int64_
     const int blocks = (int)(want < cap ? want : cap);
     count_launch();
     k_vote_stream<MODE, ACC8><<<blocks, kVoteWarps * 32, smem, s>>>(signs, bits, bits_stride, M, ntiles, sums, maj, W,
-                                                                     eta, D, status);
+                                                                     eta, D, status, tie_plus);
     done = ntiles * 4096;
   }
   const int64_t rest = d - done;
@@ -858,36 +911,45 @@ void vote_dispatch(cudaStream_t s, WorkerPtrs signs, const uint8_t* bits, int64_
   const int blocks = stream_grid((rest / 512 + 8) / 8 + 1, 8);
   k_vote<MODE, ACC8><<<blocks, kThreads, 0, s>>>(sp, bits == nullptr ? nullptr : bits + boff, bits_stride, M, rest, sums2,
                                                  maj == nullptr ? nullptr : maj + done, W == nullptr ? nullptr : W + done,
-                                                 eta, D == nullptr ? nullptr : D + done, status);
+                                                 eta, D == nullptr ? nullptr : D + done, status, tie_plus);
 }
 
 void launch_vote(cudaStream_t s, const WorkerPtrs& signs, int M, int64_t d, void* sums, int acc8,
-                 int8_t* majority) {
+                 int8_t* majority, int tie_plus) {
   if (d <= 0) return;
-  if (acc8) vote_dispatch<0, true>(s, signs, nullptr, 0, M, d, sums, majority, nullptr, 0.f, nullptr, nullptr);
-  else vote_dispatch<0, false>(s, signs, nullptr, 0, M, d, sums, majority, nullptr, 0.f, nullptr, nullptr);
+  if (acc8) vote_dispatch<0, true>(s, signs, nullptr, 0, M, d, sums, majority, nullptr, 0.f, nullptr, nullptr, tie_plus);
+  else vote_dispatch<0, false>(s, signs, nullptr, 0, M, d, sums, majority, nullptr, 0.f, nullptr, nullptr, tie_plus);
 }
 
 void launch_vote_update(cudaStream_t s, const uint8_t* bits, int64_t bits_stride, int M, int64_t d,
-                        float* W, float eta, const int* status) {
+                        float* W, float eta, const int* status, int tie_plus) {
   if (d <= 0) return;
   WorkerPtrs none{};
-  vote_dispatch<1, false>(s, none, bits, bits_stride, M, d, nullptr, nullptr, W, eta, nullptr, status);
+  vote_dispatch<1, false>(s, none, bits, bits_stride, M, d, nullptr, nullptr, W, eta, nullptr, status, tie_plus);
 }
 
 void launch_vote_major(cudaStream_t s, const uint8_t* bits, int64_t bits_stride, int M, int64_t d,
-                       float* D) {
+                       float* D, int tie_plus) {
   if (d <= 0) return;
   WorkerPtrs none{};
-  vote_dispatch<2, false>(s, none, bits, bits_stride, M, d, nullptr, nullptr, nullptr, 0.f, D, nullptr);
+  vote_dispatch<2, false>(s, none, bits, bits_stride, M, d, nullptr, nullptr, nullptr, 0.f, D, nullptr, tie_plus);
 }
 
 void launch_vote_stage(cudaStream_t s, const uint8_t* bits, int64_t bits_stride, int M, void* X, int x_bf16,
                        const Chunk* chunks, int n_chunks, const MatInfo* mats, const GroupInfo* groups,
+                       float* partials, float* D, int tie_plus) {
+  if (n_chunks <= 0) return;
+  count_launch();
+  k_vote_stage<<<n_chunks, kThreads, 0, s>>>(bits, bits_stride, M, X, x_bf16, chunks, mats, groups, partials, D,
+                                             tie_plus);
+}
+
+void launch_mean_stage(cudaStream_t s, const float* Mom, int64_t mom_stride, int M, void* X, int x_bf16,
+                       const Chunk* chunks, int n_chunks, const MatInfo* mats, const GroupInfo* groups,
                        float* partials, float* D) {
   if (n_chunks <= 0) return;
   count_launch();
-  k_vote_stage<<<n_chunks, kThreads, 0, s>>>(bits, bits_stride, M, X, x_bf16, chunks, mats, groups, partials, D);
+  k_mean_stage<<<n_chunks, kThreads, 0, s>>>(Mom, mom_stride, M, X, x_bf16, chunks, mats, groups, partials, D);
 }
 
 void launch_update(cudaStream_t s, float* W, const float* D, int64_t d, float eta,

@@ -38,6 +38,7 @@ struct signmuon_ctx {
   int device = 0, n_sm = 148;
   bool vote_only = false;
   bool u_valid = true;          // U holds the last step's (or polar call's) polar factors
+  bool bits_valid = true;       // bits hold the last step's packed signs
   // device plan tables
   sm::MatInfo* d_mats = nullptr;
   sm::GroupInfo* d_groups = nullptr;
@@ -426,6 +427,10 @@ int signmuon_init(signmuon_t* out, const int64_t* shapes, int n_mats, int M, flo
   if (!(beta >= 0.f && beta < 1.f)) return fail(nullptr, SIGNMUON_E_INVALID, "beta must be in [0, 1)");
   if (!(lambda >= 0.f)) return fail(nullptr, SIGNMUON_E_INVALID, "lambda must be >= 0");
   if (!(eps > 0.f)) return fail(nullptr, SIGNMUON_E_INVALID, "eps must be > 0");
+  if ((flags & SIGNMUON_POLAR_AFTER_ONLY) && !(flags & SIGNMUON_POST_POLAR))
+    return fail(nullptr, SIGNMUON_E_INVALID, "SIGNMUON_POLAR_AFTER_ONLY requires SIGNMUON_POST_POLAR");
+  if ((flags & SIGNMUON_MUON_MEAN) && (flags & (SIGNMUON_POST_POLAR | SIGNMUON_POLAR_AFTER_ONLY)))
+    return fail(nullptr, SIGNMUON_E_INVALID, "SIGNMUON_MUON_MEAN cannot be combined with the post-vote polar step");
   signmuon_t h = new (std::nothrow) signmuon_ctx();
   if (!h) return fail(nullptr, SIGNMUON_E_NOMEM, "host allocation failed");
   std::string err;
@@ -579,28 +584,52 @@ int signmuon_step(signmuon_t h, float* W, const float* const* G, float eta) {
                         (int)p.chunks.size(), h->d_mats, h->d_groups, h->partials);
   }
   fro_finalize(h, h->M);
-  // The signs come out of the last Newton-Schulz GEMM itself when every
-  // matrix has a multiple of 32 columns (then each 32-column chunk of an
-  // output row is one aligned word of the bit stream; K > 0, bf16 path);
-  // U is written only when kept for get_polar.
-  const bool fused = signs_in_gemm(h);
-  h->u_valid = !fused || (h->flags & SIGNMUON_KEEP_POLAR) != 0;
-  if (fused) {
-    run_ns(h, h->M, strided_ptrs(h->Mom, p.dpad, h->M), h->u_valid ? h->U : nullptr, p.dpad,
-           reinterpret_cast<uint32_t*>(h->bits), p.nb_pad / 4);
-  } else {
-    run_ns(h, h->M, strided_ptrs(h->Mom, p.dpad, h->M), h->U, p.dpad);
+  const int tie = (h->flags & SIGNMUON_TIE_PLUS) ? 1 : 0;
+  const sm::WorkerPtrs dp = strided_ptrs(h->D, 0, 1);
+  if (h->flags & SIGNMUON_MUON_MEAN) {
+    // Muon baseline: the workers' mean momentum through one PolarNS
+    h->u_valid = false;
+    h->bits_valid = false;
+    {
+      ProfScope ps(h, 8);
+      sm::launch_mean_stage(s, h->Mom, p.dpad, h->M, h->X[0], p.fp32 ? 0 : 1, h->d_chunks, (int)p.chunks.size(),
+                            h->d_mats, h->d_groups, h->partials, h->K == 0 ? h->D : nullptr);
+    }
+    fro_finalize(h, 1);
+    run_ns(h, 1, dp, h->D, 0);
+    ProfScope ps(h, 12);
+    sm::launch_update(s, W, h->D, p.d, eta, h->status);
+    return finish(h, (h->flags & SIGNMUON_ASYNC) == 0);
+  }
+  h->bits_valid = true;
+  if (h->flags & SIGNMUON_POLAR_AFTER_ONLY) {
+    // after-only placement: the signs of the momentum itself
+    h->u_valid = false;
     ProfScope ps(h, 6);
-    sm::launch_pack(s, h->U, p.dpad, p.d, h->bits, p.nb_pad, h->M);
+    sm::launch_pack(s, h->Mom, p.dpad, p.d, h->bits, p.nb_pad, h->M);
+  } else {
+    // The signs come out of the last Newton-Schulz GEMM itself when every
+    // matrix has a multiple of 32 columns (then each 32-column chunk of an
+    // output row is one aligned word of the bit stream; K > 0, bf16 path);
+    // U is written only when kept for get_polar.
+    const bool fused = signs_in_gemm(h);
+    h->u_valid = !fused || (h->flags & SIGNMUON_KEEP_POLAR) != 0;
+    if (fused) {
+      run_ns(h, h->M, strided_ptrs(h->Mom, p.dpad, h->M), h->u_valid ? h->U : nullptr, p.dpad,
+             reinterpret_cast<uint32_t*>(h->bits), p.nb_pad / 4);
+    } else {
+      run_ns(h, h->M, strided_ptrs(h->Mom, p.dpad, h->M), h->U, p.dpad);
+      ProfScope ps(h, 6);
+      sm::launch_pack(s, h->U, p.dpad, p.d, h->bits, p.nb_pad, h->M);
+    }
   }
   if (h->flags & SIGNMUON_POST_POLAR) {
     // the majority goes straight into the polar step's input (and into D
     // only when K == 0, where the polar factor is the scaled input itself)
-    const sm::WorkerPtrs dp = strided_ptrs(h->D, 0, 1);
     {
       ProfScope ps(h, 7);
       sm::launch_vote_stage(s, h->bits, p.nb_pad, h->M, h->X[0], p.fp32 ? 0 : 1, h->d_chunks, (int)p.chunks.size(),
-                            h->d_mats, h->d_groups, h->partials, h->K == 0 ? h->D : nullptr);
+                            h->d_mats, h->d_groups, h->partials, h->K == 0 ? h->D : nullptr, tie);
     }
     fro_finalize(h, 1);
     run_ns(h, 1, dp, h->D, 0);
@@ -608,7 +637,7 @@ int signmuon_step(signmuon_t h, float* W, const float* const* G, float eta) {
     sm::launch_update(s, W, h->D, p.d, eta, h->status);
   } else {
     ProfScope ps(h, 7);
-    sm::launch_vote_update(s, h->bits, p.nb_pad, h->M, p.d, W, eta, h->status);
+    sm::launch_vote_update(s, h->bits, p.nb_pad, h->M, p.d, W, eta, h->status, tie);
   }
   return finish(h, (h->flags & SIGNMUON_ASYNC) == 0);
 }
@@ -659,7 +688,8 @@ int signmuon_vote(signmuon_t h, const uint8_t* const* signs, int64_t d, void* su
     return fail(h, SIGNMUON_E_INVALID, "sums/majority must be 16-byte aligned");
   sm::WorkerPtrs sp{};
   for (int m = 0; m < h->M; ++m) sp.p[m] = reinterpret_cast<const float*>(signs[m]);
-  sm::launch_vote(h->stream, sp, h->M, d, sums, (h->flags & SIGNMUON_ACC_INT8) ? 1 : 0, majority);
+  sm::launch_vote(h->stream, sp, h->M, d, sums, (h->flags & SIGNMUON_ACC_INT8) ? 1 : 0, majority,
+                  (h->flags & SIGNMUON_TIE_PLUS) ? 1 : 0);
   CK(h, cudaGetLastError());
   return SIGNMUON_OK;
 }
@@ -740,6 +770,7 @@ int signmuon_get_signs(signmuon_t h, int m, uint8_t* dst) {
   int rc = check_handle(h, true);
   if (rc) return rc;
   if (m < 0 || m >= h->M || !dst) return fail(h, SIGNMUON_E_INVALID, "bad worker index or null dst");
+  if (!h->bits_valid) return fail(h, SIGNMUON_E_UNSUPPORTED, "a SIGNMUON_MUON_MEAN step packs no signs");
   CK(h, cudaMemcpyAsync(dst, h->bits + (int64_t)m * h->plan.nb_pad, (size_t)h->plan.nb, cudaMemcpyDeviceToDevice,
                         h->stream));
   return SIGNMUON_OK;
@@ -750,12 +781,12 @@ int signmuon_get_direction(signmuon_t h, float* dst) {
   if (rc) return rc;
   if (!dst || !aligned16(dst)) return fail(h, SIGNMUON_E_INVALID, "null or misaligned dst");
   const Plan& p = h->plan;
-  if (h->flags & SIGNMUON_POST_POLAR) {
+  if (h->flags & (SIGNMUON_POST_POLAR | SIGNMUON_MUON_MEAN)) {
     CK(h, cudaMemcpyAsync(dst, h->D, (size_t)p.d * 4, cudaMemcpyDeviceToDevice, h->stream));
   } else {
     // the step fuses the vote into the update; recompute the majority from
     // the last step's packed signs
-    sm::launch_vote_major(h->stream, h->bits, p.nb_pad, h->M, p.d, dst);
+    sm::launch_vote_major(h->stream, h->bits, p.nb_pad, h->M, p.d, dst, (h->flags & SIGNMUON_TIE_PLUS) ? 1 : 0);
     CK(h, cudaGetLastError());
   }
   return SIGNMUON_OK;

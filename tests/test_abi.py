@@ -73,3 +73,15 @@ def test_status_strings():
     import sign_muon_optimizer_b200 as smo
     for s in range(8):
         assert smo.signmuon_status_string(s)
+
+
+# POLAR_AFTER_ONLY (1 << 8) without POST_POLAR (1 << 2); MUON_MEAN (1 << 9)
+# with the post-vote polar step
+@pytest.mark.parametrize("flags", [1 << 8, (1 << 9) | (1 << 2), (1 << 9) | (1 << 8) | (1 << 2)])
+def test_init_rejects_variant_flag_combinations(flags):
+    # checked before any CUDA call: runs without a GPU
+    import sign_muon_optimizer_b200 as smo
+    assert smo.SIGNMUON_POLAR_AFTER_ONLY == 1 << 8 and smo.SIGNMUON_MUON_MEAN == 1 << 9
+    with pytest.raises(smo.SignMuonError) as e:
+        smo.SignMuon([(8, 8)], 2, flags=flags)
+    assert e.value.status == smo.SIGNMUON_E_INVALID

@@ -185,3 +185,20 @@ def test_gram_matches_bf16_product(precision, shapes):
             tol = (2.0 ** -7 if precision == "bf16" else 1e-5) * np.abs(want).max()
             bad = np.abs(got - want) > tol
             assert not bad.any(), f"{r}x{c} worker {m}: {bad.sum()} Gram entries off, rows {np.nonzero(bad)[0][:5]}"
+
+
+@pytest.mark.parametrize("M", [2, 4, 16])
+@pytest.mark.parametrize("d", [5000, 8192])
+def test_vote_tie_plus_bit_exact(M, d):
+    """Named variant: a tie gives +1 ([paper] Algorithm 2's default)."""
+    bits = synth.bernoulli_bits(d, M, config_id=7000 + M + d % 97)
+    packed = [ref.pack_bits(b) for b in bits]
+    want_sums = ref.vote_sums_from_bits(packed, d, "int32")
+    assert (want_sums == 0).any()
+    signs = [dev(np.concatenate([p, np.zeros(16, np.uint8)])) for p in packed]
+    h = smo.SignMuon([(1, d)], M, flags=smo.SIGNMUON_VOTE_ONLY | smo.SIGNMUON_TIE_PLUS)
+    sums = torch.zeros(d, dtype=torch.int32, device="cuda")
+    maj = torch.zeros(d, dtype=torch.int8, device="cuda")
+    h.vote(signs, d, sums, maj)
+    assert np.array_equal(host(sums), want_sums)
+    assert np.array_equal(host(maj), ref.majority(want_sums, tie=1))

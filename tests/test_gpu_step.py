@@ -33,9 +33,10 @@ def _flags(precision, post_polar=False, order="cubic"):
     return f
 
 
-def _run_one_step(shapes, M, sigma, K, scale, P, precision, post_polar, seed, order="cubic"):
+def _run_one_step(shapes, M, sigma, K, scale, P, precision, post_polar, seed, order="cubic", extra_flags=0,
+                  tie=0):
     h = smo.SignMuon(shapes, M, beta=HP["beta"], lam=HP["lam"], K=K, eps=HP["eps"], scale=scale, P=P,
-                     flags=_flags(precision, post_polar, order))
+                     flags=_flags(precision, post_polar, order) | extra_flags)
     d = h.d
     w0 = synth.weights0(shapes, seed)
     mom0 = synth.momentum0(shapes, M, seed, scale=0.5)
@@ -60,7 +61,7 @@ def _run_one_step(shapes, M, sigma, K, scale, P, precision, post_polar, seed, or
     gpu["D"] = host(D)
     gpu["scales"] = h.get_scales()
     want = ref.step(w0, G, mom0, shapes, beta=HP["beta"], lam=HP["lam"], eta=HP["eta"], K=K, eps=HP["eps"],
-                    scale=scale, P=P, order=order, post_polar=post_polar)
+                    scale=scale, P=P, order=order, post_polar=post_polar, tie=tie)
     want.update(mom0=mom0, G=G, w0=w0)
     return h, gpu, want
 
@@ -69,14 +70,17 @@ def _np_bits(packed, d):
     return np.unpackbits(np.asarray(packed, np.uint8), bitorder="little")[:d].astype(bool)
 
 
-def _np_majority(packed_list, d):
+def _np_majority(packed_list, d, tie=0):
     s = np.zeros(d, np.int64)
     for p in packed_list:
         s += 2 * _np_bits(p, d).astype(np.int64) - 1
-    return np.sign(s).astype(np.int8)
+    maj = np.sign(s).astype(np.int8)
+    if tie == 1:
+        maj[s == 0] = 1
+    return maj
 
 
-def _compare_step(shapes, M, gpu, want, precision, post_polar):
+def _compare_step(shapes, M, gpu, want, precision, post_polar, tie=0):
     d = synth.numel(shapes)
     for m in range(M):
         assert_momentum_close(gpu["mom"][m], want["mom0"][m], want["G"][m], want["w0"], HP["beta"], HP["lam"])
@@ -88,7 +92,7 @@ def _compare_step(shapes, M, gpu, want, precision, post_polar):
     agree = np.ones(d, bool)
     for m in range(M):
         agree &= _np_bits(gpu["bits"][m], d) == _np_bits(want["packed"][m], d)
-    gpu_maj = _np_majority(gpu["bits"], d)
+    gpu_maj = _np_majority(gpu["bits"], d, tie)
     assert np.array_equal(gpu_maj[agree], want["majority"][agree])
     assert (~agree).mean() <= M * 1e-3
     if not post_polar:
@@ -266,3 +270,99 @@ def test_signs_packed_in_gemm_match_kept_polar(post_polar):
         assert np.array_equal(out[True]["bits"][m][: want.size], want)
     assert np.array_equal(out[True]["D"], out[False]["D"])
     assert np.array_equal(out[True]["W"].view(np.uint32), out[False]["W"].view(np.uint32))
+
+
+@pytest.mark.parametrize("precision", ["fp32", "bf16"])
+@pytest.mark.parametrize("post_polar", [False, True])
+def test_step_tie_plus(precision, post_polar):
+    """Named variant: a tied vote gives +1 ([paper] Algorithm 2's default);
+    M = 4 so that ties occur.  With ties this frequent a sign within rounding
+    of zero flips a large matrix's majority somewhere, so the post-vote polar
+    factor is compared on the small matrices, whose majorities match."""
+    shapes = [(3, 5), (8, 16), (64, 96), (130, 70)]
+    M = 4
+    h, gpu, want = _run_one_step(shapes, M, 1.0, 5, "spectral", 2, precision, post_polar, seed=31,
+                                 extra_flags=smo.SIGNMUON_TIE_PLUS, tie=1)
+    assert (want["sums"] == 0).any()
+    _compare_step(shapes, M, gpu, want, precision, post_polar, tie=1)
+
+
+@pytest.mark.parametrize("precision", ["fp32", "bf16"])
+def test_step_polar_after_only(precision):
+    """Named variant: the signs of the momentum itself, orthogonalised only
+    after the vote ([paper] §4 placement)."""
+    shapes = [(64, 96), (130, 70), (96, 64)]
+    M, seed = 3, 37
+    d = synth.numel(shapes)
+    w0 = synth.weights0(shapes, seed)
+    mom0 = synth.momentum0(shapes, M, seed, scale=0.5)
+    G = synth.gradients(shapes, M, 1.0, step=1, config_id=seed)
+    h = smo.SignMuon(shapes, M, beta=HP["beta"], lam=HP["lam"], K=5, eps=HP["eps"], scale="spectral", P=2,
+                     flags=_flags(precision, True) | smo.SIGNMUON_POLAR_AFTER_ONLY)
+    for m in range(M):
+        h.set_momentum(m, dev(mom0[m]))
+    W = dev(w0)
+    h.step(W, [dev(g) for g in G], HP["eta"])
+    want = ref.step(w0, G, mom0, shapes, beta=HP["beta"], lam=HP["lam"], eta=HP["eta"], K=5, eps=HP["eps"],
+                    scale="spectral", P=2, post_polar=True, pre_polar=False)
+    agree = np.ones(d, bool)
+    bits = []
+    for m in range(M):
+        t = torch.zeros(d, device="cuda")
+        h.get_momentum(m, t)
+        mom = host(t)
+        assert_momentum_close(mom, mom0[m], G[m], w0, HP["beta"], HP["lam"])
+        b = torch.zeros(ref.packed_nbytes(d), dtype=torch.uint8, device="cuda")
+        h.get_signs(m, b)
+        bits.append(host(b))
+        # the packed signs are exactly those of the GPU's own momentum
+        assert np.array_equal(bits[m], np.packbits(mom >= 0, bitorder="little"))
+        agree &= _np_bits(bits[m], d) == _np_bits(want["packed"][m], d)
+    with pytest.raises(smo.SignMuonError) as ei:
+        h.get_polar(0, torch.zeros(d, device="cuda"))
+    assert ei.value.status == smo.SIGNMUON_E_UNSUPPORTED
+    assert (~agree).mean() <= M * 1e-4
+    gpu_maj = _np_majority(bits, d)
+    assert np.array_equal(gpu_maj[agree], want["majority"][agree])
+    Dg = torch.zeros(d, device="cuda")
+    h.get_direction(Dg)
+    D, Wn = host(Dg), host(W)
+    off = 0
+    compared = 0
+    for r, c in shapes:
+        sl = slice(off, off + r * c)
+        if np.array_equal(gpu_maj[sl], want["majority"][sl]):
+            assert_polar_close(D[sl], want["D"][sl], precision, f"after-only D {r}x{c}")
+            compared += 1
+        off += r * c
+    assert compared >= 1
+    # W is the single-rounding update with the GPU's own D
+    assert np.array_equal(Wn.view(np.uint32), ref.update(w0, D, HP["eta"]).view(np.uint32))
+
+
+@pytest.mark.parametrize("precision", ["fp32", "bf16"])
+@pytest.mark.parametrize("K", [0, 5])
+def test_step_muon_mean(precision, K):
+    """Muon baseline on the same kernels: D = PolarNS(mean momentum)."""
+    shapes = [(64, 96), (130, 70), (96, 64)]
+    M, seed = 3, 41
+    d = synth.numel(shapes)
+    w0 = synth.weights0(shapes, seed)
+    mom0 = synth.momentum0(shapes, M, seed, scale=0.5)
+    G = synth.gradients(shapes, M, 1.0, step=1, config_id=seed)
+    h = smo.SignMuon(shapes, M, beta=HP["beta"], lam=HP["lam"], K=K, eps=HP["eps"], scale="spectral", P=2,
+                     flags=_flags(precision) | smo.SIGNMUON_MUON_MEAN)
+    for m in range(M):
+        h.set_momentum(m, dev(mom0[m]))
+    W = dev(w0)
+    h.step(W, [dev(g) for g in G], HP["eta"])
+    want = ref.muon_step(w0, G, mom0, shapes, beta=HP["beta"], lam=HP["lam"], eta=HP["eta"], K=K, eps=HP["eps"],
+                         scale="spectral", P=2)
+    Dg = torch.zeros(d, device="cuda")
+    h.get_direction(Dg)
+    D = host(Dg)
+    assert_polar_close(D, want["D"], precision, "Muon D")
+    assert np.array_equal(host(W).view(np.uint32), ref.update(w0, D, HP["eta"]).view(np.uint32))
+    with pytest.raises(smo.SignMuonError) as ei:
+        h.get_signs(0, torch.zeros(ref.packed_nbytes(d), dtype=torch.uint8, device="cuda"))
+    assert ei.value.status == smo.SIGNMUON_E_UNSUPPORTED

@@ -373,3 +373,77 @@ def test_step_polar_of_orthogonal_gradients_and_post_polar():
     assert out["majority"].reshape(2, 2).tolist() == [[1, 1], [1, -1]]
     assert np.max(np.abs(out["D"].reshape(2, 2) - H * s1)) < 1e-14
     assert np.array_equal(out["W"], ref.update(W, out["D32"], 0.5))
+
+
+# ---------------------------------------------------------------------------
+# named variants ([paper] Algorithm 2's tie default, after-only polar, Muon)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 6, 7, 8])
+def test_tie_plus_brute_force_all_patterns(M):
+    # every pattern of M one-bit votes on one entry: the tie-to-+1 majority
+    # is +1 exactly when the +1 votes are at least half (counted bit by bit)
+    for pattern in range(1 << M):
+        plus = bin(pattern).count("1")
+        packed = [np.array([(pattern >> m) & 1], np.uint8) for m in range(M)]
+        sums = ref.vote_sums_from_bits(packed, 1, "int32")
+        want = 1 if 2 * plus >= M else -1
+        assert int(ref.majority(sums, tie=1)[0]) == want
+        if M % 2 == 1:  # no ties with an odd number of voters
+            assert int(ref.majority(sums, tie=1)[0]) == int(ref.majority(sums)[0])
+
+
+def test_tie_plus_in_the_step_moves_w_by_eta():
+    # two workers whose one-bit signs disagree everywhere: every entry ties;
+    # tie=0 leaves W alone, tie=+1 moves every entry by -eta
+    W = np.array([0.25, -0.5, 1.0, 0.0], np.float32)
+    g1 = np.array([1.0, -1.0, 1.0, -1.0])
+    out0 = ref.step(W, [g1, -g1], [np.zeros(4)] * 2, [(2, 2)], beta=0.0, lam=0.0, eta=0.125, K=0, eps=1e-7,
+                    scale="fro")
+    out1 = ref.step(W, [g1, -g1], [np.zeros(4)] * 2, [(2, 2)], beta=0.0, lam=0.0, eta=0.125, K=0, eps=1e-7,
+                    scale="fro", tie=1)
+    assert out0["sums"].tolist() == [0, 0, 0, 0]
+    assert np.array_equal(out0["W"], W)
+    assert out1["majority"].tolist() == [1, 1, 1, 1]
+    assert np.array_equal(out1["W"], (W - np.float32(0.125)).astype(np.float32))
+
+
+def test_after_only_polar_signs_the_momentum():
+    # pre_polar=False: the signs are those of the momentum itself; all three
+    # workers see sqrt(2) H (H orthogonal) so the majority is sign(H) and the
+    # post-vote polar of the +-1 matrix sqrt(2) H' is H' f^K(sqrt(2)/(2+eps))
+    H = np.array([[1.0, 1.0], [1.0, -1.0]]) / math.sqrt(2)
+    G = (math.sqrt(2) * H).ravel()
+    W = np.zeros(4, np.float32)
+    eps = 1e-7
+    out = ref.step(W, [G, G, G], [np.zeros(4)] * 3, [(2, 2)], beta=0.5, lam=0.0, eta=0.5, K=3, eps=eps,
+                   scale="fro", post_polar=True, pre_polar=False)
+    # momentum = (1 - beta) G: U is the momentum, unorthogonalised
+    assert np.max(np.abs(out["U"][0] - 0.5 * G)) < 1e-15
+    assert out["majority"].reshape(2, 2).tolist() == [[1, 1], [1, -1]]
+    s1 = _f_cubic(np.array([math.sqrt(2) / (2 + eps)]), 3)[0]
+    assert np.max(np.abs(out["D"].reshape(2, 2) - H * s1)) < 1e-14
+    with pytest.raises(ValueError):
+        ref.step(W, [G], [np.zeros(4)], [(2, 2)], beta=0.0, lam=0.0, eta=0.5, K=3, eps=eps, scale="fro",
+                 pre_polar=False)
+
+
+def test_muon_mean_closed_form():
+    # the momenta of 3 workers are 0.5*(a_m * H) with mean 0.5*H*mean(a);
+    # D = PolarNS(mean) = H f^K(|.|/(||.||_F+eps)) for the orthogonal H
+    H = np.array([[1.0, 1.0], [1.0, -1.0]]) / math.sqrt(2)
+    a = [1.0, 2.0, 6.0]
+    G = [(x * H).ravel() for x in a]
+    W = np.array([0.5, -0.25, 0.125, 1.0], np.float32)
+    eps = 1e-7
+    out = ref.muon_step(W, G, [np.zeros(4)] * 3, [(2, 2)], beta=0.5, lam=0.0, eta=0.25, K=4, eps=eps, scale="fro")
+    mean = 0.5 * np.mean(a)
+    assert np.max(np.abs(out["mean"] - mean * H.ravel())) < 1e-15
+    # ||mean*H||_F = mean*sqrt(2): singular values are mean each
+    s = _f_cubic(np.array([mean / (mean * math.sqrt(2) + eps)]), 4)[0]
+    assert np.max(np.abs(out["D"].reshape(2, 2) - H * s)) < 1e-14
+    assert np.array_equal(out["W"], ref.update(W, out["D32"], 0.25))
+    # one worker: Muon's direction is that worker's polar factor
+    one = ref.muon_step(W, G[:1], [np.zeros(4)], [(2, 2)], beta=0.5, lam=0.0, eta=0.25, K=4, eps=eps, scale="fro")
+    full = ref.step(W, G[:1], [np.zeros(4)], [(2, 2)], beta=0.5, lam=0.0, eta=0.25, K=4, eps=eps, scale="fro")
+    assert np.max(np.abs(one["D"] - full["U"][0])) < 1e-15
