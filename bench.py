@@ -371,7 +371,14 @@ def run_ours(args):
             "config": {"workload": WORKLOAD_DESC, "M": M, "d": D,
                        "l2": "inputs larger than L2: 2.72 GB of gradients per step, two alternating sets",
                        "parallelism": "replicas" if world > 1 else "single GPU"},
-            "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
+            "roofline": roofline,
+            # the same fraction against NVIDIA's nominal dense bf16 figure (context only)
+            "roofline_spec": {"peak": 2250.0, "unit": "TFLOP/s", "kind": "nominal dense bf16",
+                              "frac": (tflops / 2250.0) if tflops else None},
+            # the vote's payload as the pages count it (no network: M workers on one GPU)
+            "vote": {"payload_bytes_per_worker": (D + 7) // 8, "M": M, "acc_dtype": "int32 (byte-lane counters)",
+                     "collective": "none (on-device vote)"},
+            "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches, "clocks": clocks,
             "ns_tflops_per_step": flops / 1e12,
         }

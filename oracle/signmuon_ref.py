@@ -41,6 +41,16 @@ R7  Ties map to 0 ([blog]); the +1 policy of [paper] Algorithm 2 is not used.
 R8  Post-vote polar: D = PolarNS(majority as floats) with the same K, eps,
     scale and P; no second sign, no rescale.
 R9  Update: W_new = float32 nearest to (W - eta*D), one rounding.
+
+Named variants (each a flag of the CUDA path, pinned in the tests):
+
+* majority(sums, tie=1): a tie gives +1, [paper] Algorithm 2's default on the
+  {-1, +1} wire (pinned by brute force over all vote patterns).
+* step(..., pre_polar=False): the signs of the momentum itself, orthogonalised
+  only after the vote ([paper] §4, where to orthogonalise; closed-form pin).
+* muon_step: the Muon baseline the paper compares against (its §3 Muon update
+  applied to the workers' mean momentum; closed-form pin, and equal to a
+  worker's polar factor when M = 1).
 """
 from __future__ import annotations
 
