@@ -17,10 +17,7 @@
 
 namespace sm {
 
-// tensor-core GEMM pipeline depth and widest output tile (build-time knobs)
-#ifndef SM_TC_STAGES
-#define SM_TC_STAGES 4
-#endif
+// widest tensor-core output tile the planner may choose (build-time knob)
 #ifndef SM_TC_BN_MAX
 #define SM_TC_BN_MAX 256
 #endif

@@ -11,17 +11,19 @@
 // 2*128*BN*64 flops (a one-SM 128 x BN tile needs 48 KB).  Per CTA, 384
 // threads:
 //   warps 0..2  TMA producers taking turns over the k-blocks: bf16 boxes of
-//               64 columns (128-byte swizzle) into a 5-deep ring, one box per
+//               64 columns (128-byte swizzle) into a 6-deep ring, one box per
 //               lane; both CTAs' loads complete on the leader CTA's "full"
 //               barrier
 //   warp 3      allocates 512 TMEM columns (cta_group::2); in the leader CTA
 //               one lane issues tcgen05.mma.cta_group::2 (M=256, N=BN, K=16)
 //               and tcgen05.commit multicast to both CTAs' barriers
-//   warps 4..11 epilogue, each on its own 32-row x BN/2 slice of the tile:
-//               the slice of the affine operand (X for APPLY, A for SQUARE)
-//               comes into shared memory by TMA; tcgen05.ld 32x32b.x32 ->
-//               a*operand + b*acc -> bf16 results written over the operand
-//               in shared memory -> TMA store of the slice
+//   warps 4..11 epilogue, each on its own 32-row x BN/2 slice of the tile,
+//               one 32 x 64 atom at a time: the atom of the affine operand (X
+//               for APPLY, A for SQUARE) comes into shared memory by TMA;
+//               tcgen05.ld 32x32b.x32 -> a*operand + b*acc -> bf16 results
+//               written over the operand -> TMA store of the atom.  The last
+//               APPLY of a step writes sign bits (and U / D in fp32 only when
+//               asked for) instead.
 // The Gram matrix is symmetric: only tiles on or above the diagonal are
 // computed, and the epilogue also writes each off-diagonal tile transposed.
 // Every mbarrier wait is bounded (2 s): on expiry the CTA records
