@@ -181,18 +181,30 @@ def test_llama_layer_vote_full_size(acc8):
 @pytest.mark.parametrize("name,sample", [("batch64_1024", [0, 63]), ("batch256_512x2048", [0, 255])])
 @pytest.mark.parametrize("precision", ["bf16", "fp32"])
 def test_ns_sweep_sampled(name, sample, precision):
+    _ns_sweep_case(name, sample, precision, "cubic", 5, "spectral")
+
+
+# the sweep's other settings: quintic and K = 10 on the tensor cores (the
+# quintic with the Frobenius scale, which keeps every singular value of X0
+# inside the quintic's basin of convergence)
+@pytest.mark.parametrize("order,K,scale", [("quintic", 5, "fro"), ("cubic", 10, "spectral")])
+def test_ns_sweep_sampled_quintic_and_k10(order, K, scale):
+    _ns_sweep_case("batch64_1024", [0, 63], "bf16", order, K, scale)
+
+
+def _ns_sweep_case(name, sample, precision, order, K, scale):
     shapes = synth.SWEEP_SHAPES[name]
     M = 8
-    flags = smo.SIGNMUON_NS_FP32 if precision == "fp32" else 0
-    h = smo.SignMuon(shapes, M, beta=0.9, lam=0.0, K=5, eps=1e-7, scale="spectral", P=2, flags=flags)
+    flags = (smo.SIGNMUON_NS_FP32 if precision == "fp32" else 0) | (smo.SIGNMUON_NS_QUINTIC if order == "quintic" else 0)
+    h = smo.SignMuon(shapes, M, beta=0.9, lam=0.0, K=K, eps=1e-7, scale=scale, P=2, flags=flags)
     d = h.d
     X = list(synth.device_gaussian(d, M, seed=2024))
     U = [torch.empty_like(x) for x in X]
     h.polar(X, U)
     for m in (0, M - 1):
         for i in sample:
-            want = ref.polar_ns(_mat(X[m], shapes, i), 5, 1e-7, "spectral", 2)
-            assert_polar_close(_mat(U[m], shapes, i), want, precision, f"{name} worker {m} matrix {i}")
+            want = ref.polar_ns(_mat(X[m], shapes, i), K, 1e-7, scale, 2, order)
+            assert_polar_close(_mat(U[m], shapes, i), want, precision, f"{name} {order} K={K} worker {m} matrix {i}")
 
 
 def _hadamard_entry(i, j):
