@@ -75,7 +75,11 @@ k_momentum(WorkerPtrs G, const float* __restrict__ W, float* __restrict__ Mom, i
            float beta, float lambda, void* __restrict__ X, int x_bf16,
            const Chunk* __restrict__ chunks, const MatInfo* __restrict__ mats,
            const GroupInfo* __restrict__ groups, float* __restrict__ partials) {
-  __shared__ float red[32];
+  // per-(worker, warp) partial sums of squares: one block barrier at the
+  // end instead of two per worker, so that the warps run through the
+  // workers independently
+  __shared__ float red[kMaxWorkers * (kThreads / 32)];
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const Chunk ch = chunks[blockIdx.x];
   const MatInfo mi = mats[ch.mat];
   const GroupInfo gi = groups[mi.group];
@@ -132,8 +136,15 @@ k_momentum(WorkerPtrs G, const float* __restrict__ W, float* __restrict__ Mom, i
         store_x(X, xb + (int64_t)r * gi.ld + c, v, bf);
       }
     }
-    const float t = block_sum<float>(ss, red);
-    if (threadIdx.x == 0) partials[(int64_t)blockIdx.x * M + m] = t;
+    ss = warp_sum(ss);
+    if (lane == 0) red[m * (kThreads / 32) + wid] = ss;
+  }
+  __syncthreads();
+  for (int m = threadIdx.x; m < M; m += kThreads) {
+    float t = 0.f;
+#pragma unroll
+    for (int w = 0; w < kThreads / 32; ++w) t += red[m * (kThreads / 32) + w];
+    partials[(int64_t)blockIdx.x * M + m] = t;
   }
 }
 
