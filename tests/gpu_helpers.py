@@ -22,11 +22,12 @@ def host(t):
     return t.detach().cpu().numpy()
 
 
-def oracle_polar_flat(flat, shapes, K, eps, scale, P, order="cubic"):
+def oracle_polar_flat(flat, shapes, K, eps, scale, P, order="cubic", coeffs=None):
     out = np.empty(flat.size, np.float64)
     off = 0
     for r, c in shapes:
-        out[off: off + r * c] = ref.polar_ns(flat[off: off + r * c].reshape(r, c), K, eps, scale, P, order).ravel()
+        out[off: off + r * c] = ref.polar_ns(flat[off: off + r * c].reshape(r, c), K, eps, scale, P, order,
+                                             coeffs).ravel()
         off += r * c
     return out
 

@@ -107,16 +107,18 @@ def test_update_bit_exact(kind, d):
 SHAPES_SMALL = [(3, 5), (5, 3), (130, 70), (64, 147), (200, 200), (96, 300)]
 
 
-def _polar_case(shapes, M, K, scale, P, precision, order, seed):
+def _polar_case(shapes, M, K, scale, P, precision, order, seed, coeffs=None):
     flags = (smo.SIGNMUON_NS_FP32 if precision == "fp32" else 0) | (smo.SIGNMUON_NS_QUINTIC if order == "quintic" else 0)
     h = smo.SignMuon(shapes, M, beta=0.9, lam=0.0, K=K, eps=1e-7, scale=scale, P=P, flags=flags)
+    if coeffs is not None:
+        h.set_ns_coeffs(coeffs)
     xs = synth.gaussian_matrices(shapes, M, config_id=seed)
     X = [dev(x) for x in xs]
     U = [torch.zeros_like(x) for x in X]
     h.polar(X, U)
     worst = 0.0
     for m in range(M):
-        want = oracle_polar_flat(xs[m].astype(np.float64), shapes, K, 1e-7, scale, P, order)
+        want = oracle_polar_flat(xs[m].astype(np.float64), shapes, K, 1e-7, scale, P, order, coeffs)
         err, _, _ = assert_polar_close(host(U[m]), want, precision, f"worker {m}")
         worst = max(worst, err)
     return worst
@@ -132,6 +134,15 @@ def test_polar_cubic(precision, scale, P, K):
 @pytest.mark.parametrize("precision", ["fp32", "bf16"])
 def test_polar_quintic(precision):
     _polar_case(SHAPES_SMALL, 2, 5, "spectral", 2, precision, "quintic", seed=7)
+
+
+@pytest.mark.parametrize("precision", ["fp32", "bf16"])
+@pytest.mark.parametrize("order,coeffs", [("cubic", (1.75, -0.75)), ("quintic", (2.0, -1.5, 0.5))])
+def test_polar_custom_coefficients(precision, order, coeffs):
+    """signmuon_set_ns_coeffs: generic two- and three-coefficient iterations
+    against the oracle run with the same coefficients (both converge to the
+    polar factor: p(1) = 1 for each)."""
+    _polar_case(SHAPES_SMALL, 2, 4, "fro", 1, precision, order, seed=11, coeffs=coeffs)
 
 
 @pytest.mark.parametrize("precision", ["fp32", "bf16"])
