@@ -366,3 +366,68 @@ def test_step_muon_mean(precision, K):
     with pytest.raises(smo.SignMuonError) as ei:
         h.get_signs(0, torch.zeros(ref.packed_nbytes(d), dtype=torch.uint8, device="cuda"))
     assert ei.value.status == smo.SIGNMUON_E_UNSUPPORTED
+
+
+def test_async_step_matches_sync_and_defers_errors():
+    """SIGNMUON_ASYNC: the step returns without waiting and gives the same W
+    bit for bit; a non-finite gradient is reported by signmuon_sync (and
+    cleared by it), with W left untouched."""
+    shapes = [(64, 96), (96, 64)]
+    M, seed = 2, 51
+    w0 = synth.weights0(shapes, seed)
+    mom0 = synth.momentum0(shapes, M, seed, scale=0.5)
+    G = synth.gradients(shapes, M, 1.0, step=1, config_id=seed)
+    out = []
+    for flags in (0, smo.SIGNMUON_ASYNC):
+        h = smo.SignMuon(shapes, M, beta=HP["beta"], lam=HP["lam"], K=5, eps=HP["eps"], scale="spectral", P=2,
+                         flags=flags)
+        for m in range(M):
+            h.set_momentum(m, dev(mom0[m]))
+        W = dev(w0)
+        h.step(W, [dev(g) for g in G], HP["eta"])
+        h.sync()
+        out.append((h, host(W)))
+    assert np.array_equal(out[0][1].view(np.uint32), out[1][1].view(np.uint32))
+    ha = out[1][0]
+    bad = [g.copy() for g in G]
+    bad[0][5] = np.nan
+    W2 = dev(w0)
+    ha.step(W2, [dev(g) for g in bad], HP["eta"])   # no wait, no error yet
+    with pytest.raises(smo.SignMuonError) as ei:
+        ha.sync()
+    assert ei.value.status == smo.SIGNMUON_E_NONFINITE
+    assert np.array_equal(host(W2).view(np.uint32), w0.view(np.uint32))
+    ha.sync()  # the deferred error was cleared
+
+
+def test_profile_info_and_launch_counter():
+    """signmuon_profile / profile_read time every kernel kind of a step;
+    signmuon_kernel_launches counts the launches; signmuon_info reports the
+    handle's sizes."""
+    shapes = [(64, 96), (96, 64), (130, 70)]
+    M = 3
+    h = smo.SignMuon(shapes, M, beta=HP["beta"], lam=HP["lam"], K=5, eps=HP["eps"], scale="spectral", P=2,
+                     flags=smo.SIGNMUON_POST_POLAR)
+    d = h.d
+    info = smo.signmuon_info(h.h)
+    assert info["d"] == d == synth.numel(shapes)
+    assert info["packed_bytes"] == ref.packed_nbytes(d)
+    assert info["M"] == M and info["n_mats"] == len(shapes) and info["groups"] == 3
+    assert info["device_bytes"] > 0
+    W = dev(synth.weights0(shapes, 3))
+    G = [dev(g) for g in synth.gradients(shapes, M, 1.0, step=1, config_id=3)]
+    h.step(W, G, HP["eta"])
+    h.profile(True)
+    h.profile_read()
+    n0 = smo.signmuon_kernel_launches()
+    h.step(W, G, HP["eta"])
+    prof = h.profile_read()
+    h.profile(False)
+    n1 = smo.signmuon_kernel_launches()
+    want = dict(momentum=1, norm_finalize=2, ns_gram=5, ns_apply=5, power_iter=2, vote=1, post_gram=5,
+                post_apply=5, update=1)
+    for kind, n in want.items():
+        ms, cnt = prof[kind]
+        assert cnt == n, (kind, cnt)
+        assert ms > 0.0, kind
+    assert n1 - n0 >= sum(want.values())
