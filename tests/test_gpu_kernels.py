@@ -213,3 +213,20 @@ def test_vote_tie_plus_bit_exact(M, d):
     h.vote(signs, d, sums, maj)
     assert np.array_equal(host(sums), want_sums)
     assert np.array_equal(host(maj), ref.majority(want_sums, tie=1))
+
+
+def test_empty_calls_write_nothing():
+    """d = 0: vote, pack and update return at once and leave their outputs."""
+    h = _vote_handle(3)
+    signs = [torch.zeros(16, dtype=torch.uint8, device="cuda") for _ in range(3)]
+    sums = torch.full((4,), 7, dtype=torch.int32, device="cuda")
+    maj = torch.full((16,), 5, dtype=torch.int8, device="cuda")
+    h.vote(signs, 0, sums, maj)
+    assert host(sums).tolist() == [7] * 4 and (host(maj) == 5).all()
+    U = torch.ones(4, device="cuda")
+    out = torch.full((16,), 9, dtype=torch.uint8, device="cuda")
+    h.pack(U, 0, out)
+    assert (host(out) == 9).all()
+    W = torch.full((4,), 2.0, device="cuda")
+    h.apply_update(W, torch.ones(4, device="cuda"), 0, 0.5)
+    assert (host(W) == 2.0).all()

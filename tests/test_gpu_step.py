@@ -431,3 +431,39 @@ def test_profile_info_and_launch_counter():
         assert cnt == n, (kind, cnt)
         assert ms > 0.0, kind
     assert n1 - n0 >= sum(want.values())
+
+
+@pytest.mark.parametrize("precision", ["fp32", "bf16"])
+@pytest.mark.parametrize("post_polar", [False, True])
+def test_step_zero_gradients_degenerate(precision, post_polar):
+    """The degenerate case: zero weights, gradients and momentum.  The scale
+    is 0, X0 = 0/(0 + eps) = 0, so U = 0 exactly, every one-bit sign is +1
+    (reading R5), the majority is +1 and, without the post-vote polar step,
+    W moves to -eta exactly; with it D is the polar factor of the all-ones
+    matrix (its own rank-one direction)."""
+    shapes = [(64, 96), (96, 64)]
+    M = 3
+    d = synth.numel(shapes)
+    h = smo.SignMuon(shapes, M, beta=HP["beta"], lam=HP["lam"], K=5, eps=HP["eps"], scale="spectral", P=2,
+                     flags=_flags(precision, post_polar))
+    W = torch.zeros(d, device="cuda")
+    h.step(W, [torch.zeros(d, device="cuda") for _ in range(M)], HP["eta"])
+    z = np.zeros(d, np.float32)
+    want = ref.step(z, [z] * M, [z] * M, shapes, beta=HP["beta"], lam=HP["lam"], eta=HP["eta"], K=5, eps=HP["eps"],
+                    scale="spectral", P=2, post_polar=post_polar)
+    for m in range(M):
+        t = torch.ones(d, device="cuda")
+        h.get_polar(m, t)
+        assert not host(t).any()
+        b = torch.zeros(ref.packed_nbytes(d), dtype=torch.uint8, device="cuda")
+        h.get_signs(m, b)
+        assert np.array_equal(host(b), want["packed"][m])
+    Dg = torch.zeros(d, device="cuda")
+    h.get_direction(Dg)
+    D = host(Dg)
+    if post_polar:
+        assert_polar_close(D, want["D"], precision, "polar factor of the all-ones majority")
+        assert np.array_equal(host(W).view(np.uint32), ref.update(z, D, HP["eta"]).view(np.uint32))
+    else:
+        assert np.array_equal(D, np.ones(d, np.float32))
+        assert np.array_equal(host(W).view(np.uint32), want["W"].view(np.uint32))
