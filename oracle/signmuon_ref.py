@@ -37,7 +37,8 @@ R5  One-bit sign: bit = (U >= 0), so 0 and -0 send +1.  The ternary sign keeps
     sign(0) = 0 as in [paper] §3.
 R6  Packing: one flat bit stream over all matrices (shapes order, row-major),
     bit j of byte b is element 8b+j; ceil(d/8) bytes; pad bits 0.
-R7  Ties map to 0 ([blog]); the +1 policy of [paper] Algorithm 2 is not used.
+R7  Ties map to 0 ([blog]) by default; the +1 policy of [paper] Algorithm 2 is
+    the named variant majority(..., tie=1).
 R8  Post-vote polar: D = PolarNS(majority as floats) with the same K, eps,
     scale and P; no second sign, no rescale.
 R9  Update: W_new = float32 nearest to (W - eta*D), one rounding.
