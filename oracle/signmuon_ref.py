@@ -52,6 +52,15 @@ Named variants (each a flag of the CUDA path, pinned in the tests):
 * muon_step: the Muon baseline the paper compares against (its §3 Muon update
   applied to the workers' mean momentum; closed-form pin, and equal to a
   worker's polar factor when M = 1).
+* step(..., signs="ternary"): int8 signs in {-1, 0, +1}, d bytes per worker
+  ([paper] §3 sign(0) = 0; Algorithm 2's int8 all-reduce of d bytes), summed
+  as integers (pinned by brute force over all 3^M patterns, by the zero
+  momentum closed form, and by equality with the one-bit step when U has no
+  zeros).
+* step(..., normalize=True): D = majority / ||majority||_2 per matrix
+  ([paper] §4, the explicitly normalised sign step of the analysis), with the
+  norm estimated as PolarNS estimates its scale (pinned by exact singular
+  values of ternary matrices: rank-one sign patterns, signed permutations).
 """
 from __future__ import annotations
 
@@ -212,12 +221,20 @@ def vote_sums_from_bits(packed_list, d, acc="int32"):
     return total.astype(np.int8 if acc == "int8" else np.int32)
 
 
-def vote_sums_ternary(sign_list):
-    """Integer sum of ternary sign arrays (the [blog] worked example)."""
+def vote_sums_ternary(sign_list, acc="int32"):
+    """Integer sum of ternary sign arrays: the [blog] worked example, and the
+    int8 SUM all-reduce of [paper] Algorithm 2 whose payload is one byte per
+    entry and worker.  Entries must be -1, 0 or +1, so sums lie in [-M, M]."""
+    M = len(sign_list)
+    if acc == "int8" and M > 127:
+        raise AccumulatorOverflow(f"int8 sums overflow for M={M} > 127")
     total = np.zeros(np.shape(sign_list[0]), np.int64)
     for s in sign_list:
-        total += np.asarray(s, np.int64)
-    return total.astype(np.int32)
+        s = np.asarray(s, np.int64)
+        if np.any(np.abs(s) > 1):
+            raise ValueError("ternary signs must be -1, 0 or +1")
+        total += s
+    return total.astype(np.int8 if acc == "int8" else np.int32)
 
 
 def majority(sums, tie=0):
@@ -289,23 +306,55 @@ def polar_flat(flat, shapes, K, eps, scale, P=1, order="cubic"):
     return out
 
 
+def normalize_flat(flat, shapes, eps, scale, P=1):
+    """Each matrix of a flat vector divided by its norm: D_i / (s_i + eps).
+
+    [paper] §4 (single-worker variant) notes that the theory normalises the
+    sign matrix explicitly by its spectral norm, D / ||D||_2.  s_i is the same
+    scale estimate PolarNS uses for its input (reading R2 for spectral: P power
+    iterations on the wide orientation; the Frobenius norm for fro), and eps
+    keeps an all-zero majority at zero.  This is PolarNS with K = 0.
+    """
+    if scale not in ("fro", "spectral"):
+        raise ValueError(scale)
+    out = np.empty(int(np.asarray(flat).size), np.float64)
+    off = 0
+    for (r, c), mat in zip(shapes, split(np.asarray(flat, np.float64), shapes)):
+        x = mat.T if r > c else mat
+        s = frobenius_norm(x) if scale == "fro" else power_sigma(x, P)
+        out[off: off + r * c] = (mat / (s + float(eps))).ravel()
+        off += r * c
+    return out
+
+
 def step(W, G_list, mom_list, shapes, *, beta, lam, eta, K, eps, scale, P=1,
-         order="cubic", post_polar=False, acc="int32", tie=0, pre_polar=True):
+         order="cubic", post_polar=False, acc="int32", tie=0, pre_polar=True,
+         signs="bits", normalize=False):
     """One distributed Sign-Muon step ([paper] Algorithm 2, with the vote of
     [blog] and the optional post-vote polar step of [paper] §4).
 
     Named variants: tie=1 sends a tied vote to +1 ([paper] Algorithm 2's
     default); pre_polar=False signs the momentum itself and orthogonalises
     only after the vote ([paper] §4 "where to orthogonalise", the
-    after-only placement; needs post_polar=True).
+    after-only placement; needs post_polar=True); signs="ternary" sends
+    sign(U) in {-1, 0, +1}, one int8 per entry ([paper] §3 sign with
+    sign(0) = 0, and Algorithm 2's d-byte int8 all-reduce) instead of one bit;
+    normalize=True takes D = majority / ||majority||_2 per matrix ([paper] §4,
+    the explicitly normalised sign step of the analysis; cannot be combined
+    with post_polar).
 
     Returns a dict with the new momentum (float64), the polar factors U_m
-    (the momentum itself when pre_polar is False), the packed bits, the vote
-    sums, the majority, the direction D and the new W (float32).  Inputs are
-    flat vectors; momentum is float64 or float32.
+    (the momentum itself when pre_polar is False), the packed bits (the int8
+    ternary signs when signs="ternary"), the vote sums, the majority, the
+    direction D and the new W (float32).  Inputs are flat vectors; momentum
+    is float64 or float32.
     """
     if not pre_polar and not post_polar:
         raise ValueError("pre_polar=False needs post_polar=True")
+    if normalize and post_polar:
+        raise ValueError("normalize=True replaces the post-vote polar step")
+    if signs not in ("bits", "ternary"):
+        raise ValueError(signs)
     M = len(G_list)
     d = int(np.asarray(W).size)
     new_mom, U_list, packed = [], [], []
@@ -314,11 +363,20 @@ def step(W, G_list, mom_list, shapes, *, beta, lam, eta, K, eps, scale, P=1,
         new_mom.append(mom)
         u = polar_flat(mom, shapes, K, eps, scale, P, order) if pre_polar else np.asarray(mom, np.float64)
         U_list.append(u)
-        packed.append(pack_bits(sign_bits(u)))
-    sums = vote_sums_from_bits(packed, d, acc)
+        if signs == "ternary":
+            packed.append(sign_ternary(u).astype(np.int8))
+        else:
+            packed.append(pack_bits(sign_bits(u)))
+    if signs == "ternary":
+        sums = vote_sums_ternary(packed, acc)
+    else:
+        sums = vote_sums_from_bits(packed, d, acc)
     maj = majority(sums, tie)
     if post_polar:
         D = polar_flat(maj.astype(np.float64), shapes, K, eps, scale, P, order)
+        D32 = D.astype(np.float32)
+    elif normalize:
+        D = normalize_flat(maj.astype(np.float64), shapes, eps, scale, P)
         D32 = D.astype(np.float32)
     else:
         D = maj.astype(np.float64)

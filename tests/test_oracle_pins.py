@@ -447,3 +447,162 @@ def test_muon_mean_closed_form():
     one = ref.muon_step(W, G[:1], [np.zeros(4)], [(2, 2)], beta=0.5, lam=0.0, eta=0.25, K=4, eps=eps, scale="fro")
     full = ref.step(W, G[:1], [np.zeros(4)], [(2, 2)], beta=0.5, lam=0.0, eta=0.25, K=4, eps=eps, scale="fro")
     assert np.max(np.abs(one["D"] - full["U"][0])) < 1e-15
+
+
+# ---------------------------------------------------------------------------
+# ternary int8 signs ([paper] §3 sign(0) = 0; Algorithm 2's d-byte int8 SUM)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 6])
+def test_ternary_vote_brute_force_all_patterns(M):
+    # every pattern of M ternary votes on one entry, counted one by one
+    for pattern in itertools.product((-1, 0, 1), repeat=M):
+        plus = sum(1 for v in pattern if v == 1)
+        minus = sum(1 for v in pattern if v == -1)
+        signs = [np.array([v], np.int8) for v in pattern]
+        s32 = ref.vote_sums_ternary(signs, "int32")
+        s8 = ref.vote_sums_ternary(signs, "int8")
+        assert s32.dtype == np.int32 and s8.dtype == np.int8
+        assert int(s32[0]) == plus - minus == int(s8[0])
+        want0 = 1 if plus > minus else (-1 if minus > plus else 0)
+        want1 = 1 if plus >= minus else -1
+        assert int(ref.majority(s32)[0]) == want0
+        assert int(ref.majority(s32, tie=1)[0]) == want1
+
+
+def test_ternary_vote_guards():
+    with pytest.raises(ValueError):
+        ref.vote_sums_ternary([np.array([2], np.int8)])
+    with pytest.raises(ref.AccumulatorOverflow):
+        ref.vote_sums_ternary([np.zeros(3, np.int8)] * 128, "int8")
+    # 127 unanimous voters still fit an int8 accumulator
+    assert ref.vote_sums_ternary([np.ones(3, np.int8)] * 127, "int8").tolist() == [127] * 3
+
+
+def test_ternary_step_zero_momentum_closed_form():
+    # zero gradients and no weight decay: Mom = 0, so U = 0 (0 / (0 + eps),
+    # and NS keeps 0 at 0); the ternary signs are all 0, every sum is 0 and
+    # tie=0 leaves W alone, tie=+1 moves it by -eta, while the one-bit wire
+    # sends +1 (sign of 0 is +1 there) and moves it by -eta as well
+    W = np.array([0.5, -0.25, 2.0, 0.0, 1.0, -1.0], np.float32)
+    G = [np.zeros(6)] * 4
+    kw = dict(beta=0.9, lam=0.0, eta=0.125, K=3, eps=1e-7, scale="fro")
+    t0 = ref.step(W, G, [np.zeros(6)] * 4, [(2, 3)], signs="ternary", **kw)
+    t1 = ref.step(W, G, [np.zeros(6)] * 4, [(2, 3)], signs="ternary", tie=1, **kw)
+    b0 = ref.step(W, G, [np.zeros(6)] * 4, [(2, 3)], **kw)
+    assert all(np.array_equal(p, np.zeros(6, np.int8)) for p in t0["packed"])
+    assert t0["sums"].tolist() == [0] * 6 and t0["majority"].tolist() == [0] * 6
+    assert np.array_equal(t0["W"], W)
+    assert np.array_equal(t1["W"], (W - np.float32(0.125)).astype(np.float32))
+    assert b0["sums"].tolist() == [4] * 6
+    assert np.array_equal(b0["W"], t1["W"])
+
+
+def test_ternary_step_equals_one_bit_step_without_zeros():
+    # Gaussian gradients leave no exact zero in U: sign(U) in {-1, +1} and the
+    # two wires must carry the same vote (ternary sums = 2 popcount - M)
+    rng = np.random.default_rng(11)
+    shapes = [(4, 6), (5, 3)]
+    d = 24 + 15
+    W = (0.02 * rng.standard_normal(d)).astype(np.float32)
+    G = [rng.standard_normal(d) for _ in range(5)]
+    kw = dict(beta=0.9, lam=0.01, eta=0.02, K=3, eps=1e-7, scale="spectral", P=2)
+    t = ref.step(W, G, [np.zeros(d)] * 5, shapes, signs="ternary", **kw)
+    b = ref.step(W, G, [np.zeros(d)] * 5, shapes, **kw)
+    assert all(np.all(u != 0) for u in t["U"])
+    assert np.array_equal(t["sums"], b["sums"])
+    assert np.array_equal(t["majority"], b["majority"])
+    assert np.array_equal(t["W"], b["W"])
+    for m in range(5):
+        assert np.array_equal(ref.pack_bits(t["packed"][m] > 0), b["packed"][m])
+    tp = ref.step(W, G, [np.zeros(d)] * 5, shapes, signs="ternary", post_polar=True, **kw)
+    bp = ref.step(W, G, [np.zeros(d)] * 5, shapes, post_polar=True, **kw)
+    assert np.array_equal(tp["D32"], bp["D32"]) and np.array_equal(tp["W"], bp["W"])
+
+
+# ---------------------------------------------------------------------------
+# explicitly normalised sign step D / ||D||_2 ([paper] §4, single-worker notes)
+# ---------------------------------------------------------------------------
+
+def _sign_pattern_step(pattern, scale, P=2, M=3, eps=1e-7):
+    # M identical workers whose gradient is the pattern itself: the majority
+    # is the pattern (K = 0, positive scaling keeps every sign; the ternary
+    # wire keeps the pattern's zeros, which the one-bit wire would send as +1)
+    r, c = pattern.shape
+    W = np.zeros(r * c, np.float32)
+    G = [pattern.astype(np.float64).ravel()] * M
+    return ref.step(W, G, [np.zeros(r * c)] * M, [(r, c)], beta=0.5, lam=0.0, eta=0.25, K=0, eps=eps,
+                    scale=scale, P=P, normalize=True, signs="ternary")
+
+
+@pytest.mark.parametrize("rows,cols", [(3, 5), (5, 3), (4, 4)])
+def test_normalize_rank_one_sign_pattern(rows, cols):
+    # a = sign pattern with unequal +-1 counts (so ones . a != 0), b any signs:
+    # a b^T has the single singular value sqrt(rows*cols), and one power
+    # iteration from the all-ones start lands on it exactly
+    a = np.array([1, 1, -1, 1, 1][:rows], np.float64)
+    b = np.array([1, -1, -1, 1, -1][:cols], np.float64)
+    if rows == 4:
+        a = np.array([1, 1, 1, -1], np.float64)
+    pattern = np.outer(a, b)
+    eps = 1e-7
+    out = _sign_pattern_step(pattern, "spectral", P=1, eps=eps)
+    assert out["majority"].reshape(rows, cols).tolist() == pattern.astype(int).tolist()
+    want = pattern / (math.sqrt(rows * cols) + eps)
+    assert np.max(np.abs(out["D"].reshape(rows, cols) - want)) < 1e-15
+    assert np.array_equal(out["W"], ref.update(np.zeros(rows * cols, np.float32), out["D32"], 0.25))
+    # Frobenius: ||a b^T||_F = sqrt(rows*cols) as well
+    fro = _sign_pattern_step(pattern, "fro", eps=eps)
+    assert np.max(np.abs(fro["D"].reshape(rows, cols) - want)) < 1e-15
+
+
+@pytest.mark.parametrize("rows,cols", [(4, 4), (3, 6), (6, 3)])
+@pytest.mark.parametrize("P", [1, 2, 5])
+def test_normalize_signed_permutation(rows, cols, P):
+    # one +-1 per row (wide) or per column (tall) at distinct places: every
+    # singular value is 1, so D = pattern / (1 + eps) for any P
+    k = min(rows, cols)
+    perm = [2, 0, 3, 1, 5, 4][:k] if max(rows, cols) >= 6 else [2, 0, 3, 1][:k]
+    sgn = [1, -1, -1, 1, 1, -1]
+    pattern = np.zeros((rows, cols))
+    for i in range(k):
+        if rows <= cols:
+            pattern[i, perm[i] % cols] = sgn[i]
+        else:
+            pattern[perm[i] % rows, i] = sgn[i]
+    assert np.allclose(np.linalg.svd(pattern, compute_uv=False), 1.0)
+    eps = 1e-7
+    out = _sign_pattern_step(pattern, "spectral", P=P, eps=eps)
+    assert out["majority"].reshape(rows, cols).tolist() == pattern.astype(int).tolist()
+    assert np.max(np.abs(out["D"].reshape(rows, cols) - pattern / (1.0 + eps))) < 1e-15
+
+
+def test_normalize_against_exact_sigma_max():
+    # a sign pattern with a dominant rank-one part: many power iterations
+    # reach numpy's exact largest singular value of the majority matrix
+    rng = np.random.default_rng(5)
+    u, v = rng.standard_normal(7), rng.standard_normal(11)
+    pattern = np.sign(np.outer(u, v) + 0.3 * rng.standard_normal((7, 11)))
+    pattern[pattern == 0] = 1
+    out = _sign_pattern_step(pattern, "spectral", P=300, eps=1e-12)
+    smax = np.linalg.svd(out["majority"].reshape(7, 11).astype(np.float64), compute_uv=False)[0]
+    assert np.max(np.abs(out["D"].reshape(7, 11) * smax - pattern)) < 1e-9
+    fro = _sign_pattern_step(pattern, "fro", eps=1e-12)
+    assert np.max(np.abs(fro["D"].reshape(7, 11) * math.sqrt(77.0) - pattern)) < 1e-9
+
+
+def test_normalize_of_an_all_tied_vote_is_zero_and_guards():
+    # two workers with opposite signs everywhere: every entry ties, the
+    # majority is 0, and eps keeps D at 0 (no 0/0)
+    W = np.array([0.25, -0.5, 1.0, 0.0], np.float32)
+    g = np.array([1.0, -1.0, 2.0, -3.0])
+    out = ref.step(W, [g, -g], [np.zeros(4)] * 2, [(2, 2)], beta=0.0, lam=0.0, eta=0.5, K=2, eps=1e-7,
+                   scale="spectral", P=2, normalize=True)
+    assert out["majority"].tolist() == [0, 0, 0, 0]
+    assert np.array_equal(out["D"], np.zeros(4)) and np.array_equal(out["W"], W)
+    with pytest.raises(ValueError):
+        ref.step(W, [g], [np.zeros(4)], [(2, 2)], beta=0.0, lam=0.0, eta=0.5, K=2, eps=1e-7, scale="fro",
+                 normalize=True, post_polar=True)
+    with pytest.raises(ValueError):
+        ref.step(W, [g], [np.zeros(4)], [(2, 2)], beta=0.0, lam=0.0, eta=0.5, K=2, eps=1e-7, scale="fro",
+                 signs="trits")
