@@ -67,10 +67,21 @@ typedef struct signmuon_ctx* signmuon_t;
  *                    vote (§4 "where to orthogonalise"); requires SIGNMUON_POST_POLAR.
  * MUON_MEAN          the Muon baseline instead of Sign-Muon: D = PolarNS(mean of the M
  *                    workers' momenta), W <- fl32(W - eta D); no signs, no vote; cannot be
- *                    combined with POST_POLAR or POLAR_AFTER_ONLY. */
+ *                    combined with POST_POLAR, POLAR_AFTER_ONLY, TERNARY or NORMALIZED_SIGN.
+ * TERNARY            the step sends sign(U) in {-1, 0, +1} as one int8 per entry (d bytes
+ *                    per worker: §3's sign with sign(0) = 0, the payload of Algorithm 2's
+ *                    int8 SUM all-reduce) instead of one bit, and votes on the integer
+ *                    sums of those; U is always kept.  The handle holds M*d more bytes.
+ * NORMALIZED_SIGN    D = majority / (s + eps) per matrix, s the handle's scale estimate of
+ *                    the majority matrix (spectral: the P-step power-iteration estimate of
+ *                    ||majority||_2; fro: ||majority||_F) -- the explicitly normalised sign
+ *                    step of §4's analysis.  Cannot be combined with POST_POLAR (it is the
+ *                    post-vote step with no Newton-Schulz iteration). */
 #define SIGNMUON_TIE_PLUS          (1u << 7)
 #define SIGNMUON_POLAR_AFTER_ONLY  (1u << 8)
 #define SIGNMUON_MUON_MEAN         (1u << 9)
+#define SIGNMUON_TERNARY           (1u << 10)
+#define SIGNMUON_NORMALIZED_SIGN   (1u << 11)
 
 /* ------------------------------------------------------------------------
  * signmuon_init -- plan the step and allocate its device state.
@@ -102,9 +113,11 @@ int signmuon_init(signmuon_t* out, const int64_t* shapes, int n_mats, int M,
  *   G    host array of M device pointers, each float[d]: worker gradients.
  *   eta  step size.
  * Per worker: Mom_m <- beta*Mom_m + (1-beta)(G_m + lambda*W); U_m =
- * PolarNS(Mom_m) per matrix; bits_m = (U_m >= 0) packed LSB-first.  Then
- * sums = sum_m (2 bits_m - 1), majority = sign(sums) (0 on a tie), D =
- * majority or PolarNS(majority) per matrix.  Unless SIGNMUON_ASYNC, waits for
+ * PolarNS(Mom_m) per matrix; bits_m = (U_m >= 0) packed LSB-first (with
+ * SIGNMUON_TERNARY: t_m = sign(U_m) in {-1, 0, +1}, one int8 each).  Then
+ * sums = sum_m (2 bits_m - 1) (or sum_m t_m), majority = sign(sums) (0 on a
+ * tie), D = majority, PolarNS(majority) or majority / (s + eps) per matrix
+ * (SIGNMUON_POST_POLAR / SIGNMUON_NORMALIZED_SIGN).  Unless SIGNMUON_ASYNC, waits for
  * the GPU and returns E_NONFINITE when a momentum norm is NaN/Inf; W is then
  * left unchanged (the momentum keeps the non-finite values: restore it with
  * signmuon_set_momentum).
@@ -142,6 +155,30 @@ int signmuon_vote(signmuon_t h, const uint8_t* const* signs, int64_t d, void* su
 int signmuon_pack(signmuon_t h, const float* U, int64_t d, uint8_t* out);
 
 /* ------------------------------------------------------------------------
+ * signmuon_sign_ternary -- entrywise ternary sign of a flat float vector
+ * ([paper] §3: sign(0) = 0): out[i] = +1 if U[i] > 0, -1 if U[i] < 0, else 0
+ * (0, -0 and NaN give 0).  U device float[d]; out device int8[d]; both
+ * 16-byte aligned.  d >= 0.  Errors: E_INVALID.
+ * ---------------------------------------------------------------------- */
+int signmuon_sign_ternary(signmuon_t h, const float* U, int64_t d, int8_t* out);
+
+/* ------------------------------------------------------------------------
+ * signmuon_vote_ternary -- majority vote over M int8 ternary sign buffers
+ * ([paper] Algorithm 2's integer SUM of the workers' signs, d bytes per
+ * worker; [blog] "A tiny aggregation calculation": sums in [-M, M], ties to 0,
+ * or to +1 with SIGNMUON_TIE_PLUS).
+ *   signs     host array of M device pointers, each int8[d] with entries -1,
+ *             0 or +1 (other values give unspecified sums, never a fault),
+ *             16-byte aligned.
+ *   d         number of entries (>= 0).
+ *   sums      device int32[d] (int8[d] when SIGNMUON_ACC_INT8), may be NULL.
+ *   majority  device int8[d] in {-1, 0, +1}, may be NULL.
+ * Results are bit-exact integers.  Errors: E_INVALID (null or misaligned).
+ * ---------------------------------------------------------------------- */
+int signmuon_vote_ternary(signmuon_t h, const int8_t* const* signs, int64_t d, void* sums,
+                          int8_t* majority);
+
+/* ------------------------------------------------------------------------
  * signmuon_apply_update -- W <- fl32(W - eta*D), one rounding (fused
  * multiply-add), [paper] Algorithm 1/2 update.  W, D device float[d].
  * ---------------------------------------------------------------------- */
@@ -164,7 +201,9 @@ int signmuon_polar(signmuon_t h, const float* const* X, float* const* U);
  * SIGNMUON_KEEP_POLAR on shapes whose signs are packed inside the last
  * Newton-Schulz GEMM, and always with POLAR_AFTER_ONLY or MUON_MEAN).
  * get_signs: worker m's packed bits from the last step (SIGNMUON_E_UNSUPPORTED
- * with MUON_MEAN).  get_direction: the last step's D.
+ * with MUON_MEAN or TERNARY).  get_ternary_signs: worker m's int8[d] ternary
+ * signs from the last step (SIGNMUON_E_UNSUPPORTED unless TERNARY).
+ * get_direction: the last step's D.
  * get_scales: host float[M*n_mats]: the last step's scale s per (worker,
  * matrix), worker-major (waits for the GPU).
  * ---------------------------------------------------------------------- */
@@ -172,6 +211,7 @@ int signmuon_get_momentum(signmuon_t h, int m, float* dst);
 int signmuon_set_momentum(signmuon_t h, int m, const float* src);
 int signmuon_get_polar(signmuon_t h, int m, float* dst);
 int signmuon_get_signs(signmuon_t h, int m, uint8_t* dst);
+int signmuon_get_ternary_signs(signmuon_t h, int m, int8_t* dst);
 int signmuon_get_direction(signmuon_t h, float* dst);
 int signmuon_get_scales(signmuon_t h, float* dst_host);
 /* get_gram: the Gram matrix (g x g, g = min(rows, cols), row-major floats on
@@ -204,10 +244,11 @@ int signmuon_plan(const int64_t* shapes, int n_mats, int M, int K, int scale, in
  * kind (ms[k], launches[k] for k < n) since the last read, and resets them.
  * Kinds: 0 momentum pass, 1 norm finalisation, 2/3/4 Newton-Schulz GEMMs
  * (Gram, quintic square, apply), 5 power iteration, 6 one-bit pack (only
- * when the signs are not packed inside the last GEMM), 7 vote (fused with the
- * update, or with the staging of the majority for the post-vote polar step),
- * 8 unused (kept for numbering), 9/10/11 post-vote Newton-Schulz GEMMs (Gram,
- * square, apply), 12 update, 13 K=0 scaling. */
+ * when the signs are not packed inside the last GEMM) or ternary sign, 7 vote
+ * (fused with the update, or with the staging of the majority for the
+ * post-vote step), 8 staging of the mean momentum (MUON_MEAN), 9/10/11
+ * post-vote Newton-Schulz GEMMs (Gram, square, apply), 12 update, 13 K=0
+ * scaling. */
 #define SIGNMUON_PROF_KINDS 14
 int signmuon_profile(signmuon_t h, int enable);
 int signmuon_profile_read(signmuon_t h, double* ms, int64_t* launches, int n);

@@ -39,6 +39,8 @@ SIGNMUON_KEEP_POLAR = 1 << 6
 SIGNMUON_TIE_PLUS = 1 << 7
 SIGNMUON_POLAR_AFTER_ONLY = 1 << 8
 SIGNMUON_MUON_MEAN = 1 << 9
+SIGNMUON_TERNARY = 1 << 10
+SIGNMUON_NORMALIZED_SIGN = 1 << 11
 
 EXPORTED = [
     "signmuon_init", "signmuon_step", "signmuon_step_host", "signmuon_vote", "signmuon_pack",
@@ -47,7 +49,8 @@ EXPORTED = [
     "signmuon_set_ns_coeffs", "signmuon_sync", "signmuon_info", "signmuon_plan",
     "signmuon_kernel_launches", "signmuon_last_error", "signmuon_status_string", "signmuon_destroy",
     "signmuon_profile", "signmuon_profile_read", "signmuon_get_gram",
-    "signmuon_spectral_norm_noalloc",
+    "signmuon_spectral_norm_noalloc", "signmuon_sign_ternary", "signmuon_vote_ternary",
+    "signmuon_get_ternary_signs",
 ]
 PROF_KINDS = ["momentum", "norm_finalize", "ns_gram", "ns_square", "ns_apply", "power_iter", "pack",
               "vote", "stage", "post_gram", "post_square", "post_apply", "update", "k0_scale"]
@@ -71,6 +74,9 @@ def _load():
         "signmuon_step_host": (I, [P, P, PP, F]),
         "signmuon_vote": (I, [P, PP, I64, P, P]),
         "signmuon_pack": (I, [P, P, I64, P]),
+        "signmuon_sign_ternary": (I, [P, P, I64, P]),
+        "signmuon_vote_ternary": (I, [P, PP, I64, P, P]),
+        "signmuon_get_ternary_signs": (I, [P, I, P]),
         "signmuon_apply_update": (I, [P, P, P, I64, F]),
         "signmuon_polar": (I, [P, PP, PP]),
         "signmuon_get_momentum": (I, [P, I, P]),
@@ -171,6 +177,18 @@ def signmuon_vote(h, signs, d, sums=None, majority=None):
 
 def signmuon_pack(h, U, d, out):
     _check(h, _lib.signmuon_pack(h, _ptr(U), int(d), _ptr(out)))
+
+
+def signmuon_sign_ternary(h, U, d, out):
+    _check(h, _lib.signmuon_sign_ternary(h, _ptr(U), int(d), _ptr(out)))
+
+
+def signmuon_vote_ternary(h, signs, d, sums=None, majority=None):
+    _check(h, _lib.signmuon_vote_ternary(h, _ptr_array(signs), int(d), _ptr(sums), _ptr(majority)))
+
+
+def signmuon_get_ternary_signs(h, m, dst):
+    _check(h, _lib.signmuon_get_ternary_signs(h, int(m), _ptr(dst)))
 
 
 def signmuon_apply_update(h, W, D, d, eta):
@@ -297,6 +315,15 @@ class SignMuon:
 
     def pack(self, U, d, out):
         signmuon_pack(self.h, U, d, out)
+
+    def sign_ternary(self, U, d, out):
+        signmuon_sign_ternary(self.h, U, d, out)
+
+    def vote_ternary(self, signs, d, sums=None, majority=None):
+        signmuon_vote_ternary(self.h, signs, d, sums, majority)
+
+    def get_ternary_signs(self, m, dst):
+        signmuon_get_ternary_signs(self.h, m, dst)
 
     def apply_update(self, W, D, d, eta):
         signmuon_apply_update(self.h, W, D, d, eta)

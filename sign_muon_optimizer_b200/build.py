@@ -20,7 +20,8 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libsignmuon.so")
 
-SOURCES = ["kernels_elem.cu", "ns_simt.cu", "ns_tc.cu", "signmuon_api.cu", "noalloc.cu", "plan.cpp"]
+SOURCES = ["kernels_elem.cu", "kernels_ternary.cu", "ns_simt.cu", "ns_tc.cu", "signmuon_api.cu", "noalloc.cu",
+           "plan.cpp"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-I" + INCLUDE,
                      "--expt-relaxed-constexpr"]

@@ -118,6 +118,8 @@ struct GemmArgs {
 // ---- launch wrappers (host) ----------------------------------------------
 void count_launch();
 void set_global_error(const char* msg);  // text for signmuon_last_error(NULL)
+int num_sms();                                   // SMs of the current device
+int stream_grid(int64_t work_items, int per_sm); // min(work_items, SMs * per_sm), at least 1
 
 void launch_momentum(cudaStream_t s, const WorkerPtrs& G, const float* W, float* Mom, int64_t d,
                      int M, float beta, float lambda, void* X, int x_bf16, const Chunk* chunks,
@@ -157,6 +159,15 @@ void launch_mean_stage(cudaStream_t s, const float* Mom, int64_t mom_stride, int
                        float* partials, float* D);
 void launch_update(cudaStream_t s, float* W, const float* D, int64_t d, float eta,
                    const int* status);
+// int8 ternary sign wire (kernels_ternary.cu)
+void launch_sign8(cudaStream_t s, const float* U, int64_t u_stride, int64_t d, int8_t* out, int64_t out_stride,
+                  int M);
+void launch_vote_ternary(cudaStream_t s, const WorkerPtrs& signs, int M, int64_t d, void* sums, int acc8,
+                         int8_t* majority, int tie_plus);
+void launch_vote_ternary_update(cudaStream_t s, const int8_t* signs, int64_t stride, int M, int64_t d, float* W,
+                                float eta, const int* status, int tie_plus);
+void launch_vote_ternary_major(cudaStream_t s, const int8_t* signs, int64_t stride, int M, int64_t d, float* D,
+                               int tie_plus);
 
 void launch_gemm_simt(cudaStream_t s, const GemmArgs& a, int x_f32);
 int gemm_tc_smem_bytes();

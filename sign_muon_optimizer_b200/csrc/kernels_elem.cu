@@ -794,6 +794,9 @@ k_update(float* __restrict__ W, const float* __restrict__ D, int64_t d, float et
 }
 
 int g_num_sms = 0;
+
+}  // namespace
+
 int num_sms() {
   if (g_num_sms == 0) {
     int dev = 0;
@@ -809,8 +812,6 @@ int stream_grid(int64_t work_items, int per_sm) {
   if (work_items < 1) return 1;
   return (int)(work_items < cap ? work_items : cap);
 }
-
-}  // namespace
 
 // ---- launch wrappers --------------------------------------------------------
 

@@ -81,6 +81,19 @@ int make_plan(const int64_t* shapes, int n_mats, int M, int K, int scale, int P,
   if (K < 0) { *err = "K must be >= 0"; return SIGNMUON_E_INVALID; }
   if (scale != SIGNMUON_SCALE_FRO && scale != SIGNMUON_SCALE_SPECTRAL) { *err = "unknown scale"; return SIGNMUON_E_INVALID; }
   if (scale == SIGNMUON_SCALE_SPECTRAL && P < 1) { *err = "spectral scaling needs P >= 1"; return SIGNMUON_E_INVALID; }
+  if ((flags & SIGNMUON_POLAR_AFTER_ONLY) && !(flags & SIGNMUON_POST_POLAR)) {
+    *err = "SIGNMUON_POLAR_AFTER_ONLY requires SIGNMUON_POST_POLAR";
+    return SIGNMUON_E_INVALID;
+  }
+  if ((flags & SIGNMUON_MUON_MEAN) &&
+      (flags & (SIGNMUON_POST_POLAR | SIGNMUON_POLAR_AFTER_ONLY | SIGNMUON_TERNARY | SIGNMUON_NORMALIZED_SIGN))) {
+    *err = "SIGNMUON_MUON_MEAN sends no signs: it cannot be combined with the post-vote step or the sign wire flags";
+    return SIGNMUON_E_INVALID;
+  }
+  if ((flags & SIGNMUON_NORMALIZED_SIGN) && (flags & SIGNMUON_POST_POLAR)) {
+    *err = "SIGNMUON_NORMALIZED_SIGN replaces the post-vote polar step: drop SIGNMUON_POST_POLAR";
+    return SIGNMUON_E_INVALID;
+  }
   Plan& p = *plan;
   p = Plan();
   p.M = M;
@@ -188,6 +201,7 @@ int make_plan(const int64_t* shapes, int n_mats, int M, int K, int scale, int P,
     bytes += 2 * p.x_elems * esz;                         // X ping/pong
     bytes += p.a_elems * esz * (p.quintic ? 2 : 1);       // A (and B)
     bytes += (int64_t)M * p.nb_pad;                       // packed bits
+    if (flags & SIGNMUON_TERNARY) bytes += (int64_t)M * p.dpad;  // int8 ternary signs
     bytes += p.dpad * 4;                                  // D
     bytes += (int64_t)p.chunks.size() * M * 4;            // norm partials
     bytes += (int64_t)M * n_mats * (4 + 8 + 8);           // scales, coefficients

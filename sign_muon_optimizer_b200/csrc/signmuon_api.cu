@@ -6,8 +6,9 @@
 // Algorithm 2; the vote of [blog] "SignMuon: Matrix Directions, Majority
 // Votes, and the Actual Bytes Sent"):
 //   momentum pass -> Frobenius partials -> NS GEMMs (GRAM [-> power iteration]
-//   [-> SQUARE] -> APPLY) x K -> one-bit pack -> vote fused with the update,
-//   or vote -> stage -> NS x K -> update for the post-vote polar step.
+//   [-> SQUARE] -> APPLY) x K -> one-bit pack (or int8 ternary sign) -> vote
+//   fused with the update, or vote -> stage -> NS x K -> update for the
+//   post-vote polar step (K = 0 there for the normalised sign step).
 #include <cuda.h>
 
 #include <atomic>
@@ -39,6 +40,7 @@ struct signmuon_ctx {
   bool vote_only = false;
   bool u_valid = true;          // U holds the last step's (or polar call's) polar factors
   bool bits_valid = true;       // bits hold the last step's packed signs
+  bool t_valid = false;         // sign8 holds the last step's ternary signs
   // device plan tables
   sm::MatInfo* d_mats = nullptr;
   sm::GroupInfo* d_groups = nullptr;
@@ -61,6 +63,7 @@ struct signmuon_ctx {
   void* B = nullptr;
   float* U = nullptr;
   uint8_t* bits = nullptr;
+  int8_t* sign8 = nullptr;      // TERNARY: int8 signs, M x dpad bytes
   float* D = nullptr;
   float* partials = nullptr;
   float* scale_v = nullptr;
@@ -240,9 +243,10 @@ void prof_collect(signmuon_t h) {
 }
 
 // ---------------------------------------------------------------------------
-// PolarNS for nw workers whose X~ (unscaled) is staged in X[0]; the Frobenius
-// scale (if used) is already final.  Writes U (fp32, flat) to out +
-// worker*out_stride.  kzero_in is the fp32 input used when K == 0.
+// PolarNS with K iterations for nw workers whose X~ (unscaled) is staged in
+// X[0]; the Frobenius scale (if used) is already final.  Writes U (fp32,
+// flat) to out + worker*out_stride.  kzero_in is the fp32 input used when
+// K == 0.
 // ---------------------------------------------------------------------------
 void gemm(signmuon_t h, int op, int slot, int src, int nw, const float2* coef, float c0, float c1,
           bool final_out, float* out, int64_t out_stride, uint32_t* out_bits = nullptr, int64_t bits_stride = 0) {
@@ -313,12 +317,12 @@ bool signs_in_gemm(signmuon_t h) {
   return true;
 }
 
-void run_ns(signmuon_t h, int nw, const sm::WorkerPtrs& kzero_in, float* out, int64_t out_stride,
+void run_ns(signmuon_t h, int K, int nw, const sm::WorkerPtrs& kzero_in, float* out, int64_t out_stride,
             uint32_t* out_bits = nullptr, int64_t bits_stride = 0) {
   const Plan& p = h->plan;
   const int slot = nw == 1 ? 1 : 0;
   const bool spectral = h->scale == SIGNMUON_SCALE_SPECTRAL;
-  if (h->K == 0) {
+  if (K == 0) {
     if (spectral) {
       gemm(h, sm::OP_GRAM, slot, 0, nw, nullptr, 0.f, 0.f, false, nullptr, 0);
       power_iteration(h, nw);
@@ -329,12 +333,12 @@ void run_ns(signmuon_t h, int nw, const sm::WorkerPtrs& kzero_in, float* out, in
     return;
   }
   int cur = 0;
-  for (int k = 0; k < h->K; ++k) {
+  for (int k = 0; k < K; ++k) {
     gemm(h, sm::OP_GRAM, slot, cur, nw, nullptr, 0.f, 0.f, false, nullptr, 0);
     if (k == 0 && spectral) power_iteration(h, nw);
     if (p.quintic)
       gemm(h, sm::OP_SQUARE, slot, cur, nw, k == 0 ? h->coef_square : nullptr, h->ns_b, h->ns_c, false, nullptr, 0);
-    const bool last = (k == h->K - 1);
+    const bool last = (k == K - 1);
     gemm(h, sm::OP_APPLY, slot, cur, nw, k == 0 ? h->coef_apply : nullptr, h->ns_a, p.quintic ? 1.f : h->ns_b, last,
          out, out_stride, last ? out_bits : nullptr, bits_stride);
     cur ^= 1;
@@ -427,10 +431,6 @@ int signmuon_init(signmuon_t* out, const int64_t* shapes, int n_mats, int M, flo
   if (!(beta >= 0.f && beta < 1.f)) return fail(nullptr, SIGNMUON_E_INVALID, "beta must be in [0, 1)");
   if (!(lambda >= 0.f)) return fail(nullptr, SIGNMUON_E_INVALID, "lambda must be >= 0");
   if (!(eps > 0.f)) return fail(nullptr, SIGNMUON_E_INVALID, "eps must be > 0");
-  if ((flags & SIGNMUON_POLAR_AFTER_ONLY) && !(flags & SIGNMUON_POST_POLAR))
-    return fail(nullptr, SIGNMUON_E_INVALID, "SIGNMUON_POLAR_AFTER_ONLY requires SIGNMUON_POST_POLAR");
-  if ((flags & SIGNMUON_MUON_MEAN) && (flags & (SIGNMUON_POST_POLAR | SIGNMUON_POLAR_AFTER_ONLY)))
-    return fail(nullptr, SIGNMUON_E_INVALID, "SIGNMUON_MUON_MEAN cannot be combined with the post-vote polar step");
   signmuon_t h = new (std::nothrow) signmuon_ctx();
   if (!h) return fail(nullptr, SIGNMUON_E_NOMEM, "host allocation failed");
   std::string err;
@@ -500,6 +500,10 @@ int signmuon_init(signmuon_t* out, const int64_t* shapes, int n_mats, int M, flo
     }
   }
   if ((rc = dalloc(h, &h->bits, (int64_t)M * p.nb_pad))) return bail(rc);
+  if (flags & SIGNMUON_TERNARY) {
+    if ((rc = dalloc(h, &h->sign8, (int64_t)M * p.dpad))) return bail(rc);
+    if (cudaMemset(h->sign8, 0, (size_t)M * p.dpad) != cudaSuccess) return bail(fail(h, SIGNMUON_E_CUDA, "memset"));
+  }
   if ((rc = dalloc(h, &h->D, p.dpad))) return bail(rc);
   if ((rc = dalloc(h, &h->partials, (int64_t)p.chunks.size() * M))) return bail(rc);
   if ((rc = dalloc(h, &h->scale_v, (int64_t)M * p.n_mats))) return bail(rc);
@@ -596,48 +600,66 @@ int signmuon_step(signmuon_t h, float* W, const float* const* G, float eta) {
                             h->d_mats, h->d_groups, h->partials, h->K == 0 ? h->D : nullptr);
     }
     fro_finalize(h, 1);
-    run_ns(h, 1, dp, h->D, 0);
+    run_ns(h, h->K, 1, dp, h->D, 0);
     ProfScope ps(h, 12);
     sm::launch_update(s, W, h->D, p.d, eta, h->status);
     return finish(h, (h->flags & SIGNMUON_ASYNC) == 0);
   }
-  h->bits_valid = true;
+  // one bit per entry, or (TERNARY) one int8 sign in {-1, 0, +1}
+  const bool ternary = (h->flags & SIGNMUON_TERNARY) != 0;
+  h->bits_valid = !ternary;
+  h->t_valid = ternary;
   if (h->flags & SIGNMUON_POLAR_AFTER_ONLY) {
     // after-only placement: the signs of the momentum itself
     h->u_valid = false;
     ProfScope ps(h, 6);
-    sm::launch_pack(s, h->Mom, p.dpad, p.d, h->bits, p.nb_pad, h->M);
+    if (ternary) sm::launch_sign8(s, h->Mom, p.dpad, p.d, h->sign8, p.dpad, h->M);
+    else sm::launch_pack(s, h->Mom, p.dpad, p.d, h->bits, p.nb_pad, h->M);
   } else {
-    // The signs come out of the last Newton-Schulz GEMM itself when every
-    // matrix has a multiple of 32 columns (then each 32-column chunk of an
-    // output row is one aligned word of the bit stream; K > 0, bf16 path);
+    // The one-bit signs come out of the last Newton-Schulz GEMM itself when
+    // every matrix has a multiple of 32 columns (then each 32-column chunk of
+    // an output row is one aligned word of the bit stream; K > 0, bf16 path);
     // U is written only when kept for get_polar.
-    const bool fused = signs_in_gemm(h);
+    const bool fused = !ternary && signs_in_gemm(h);
     h->u_valid = !fused || (h->flags & SIGNMUON_KEEP_POLAR) != 0;
     if (fused) {
-      run_ns(h, h->M, strided_ptrs(h->Mom, p.dpad, h->M), h->u_valid ? h->U : nullptr, p.dpad,
+      run_ns(h, h->K, h->M, strided_ptrs(h->Mom, p.dpad, h->M), h->u_valid ? h->U : nullptr, p.dpad,
              reinterpret_cast<uint32_t*>(h->bits), p.nb_pad / 4);
     } else {
-      run_ns(h, h->M, strided_ptrs(h->Mom, p.dpad, h->M), h->U, p.dpad);
+      run_ns(h, h->K, h->M, strided_ptrs(h->Mom, p.dpad, h->M), h->U, p.dpad);
       ProfScope ps(h, 6);
-      sm::launch_pack(s, h->U, p.dpad, p.d, h->bits, p.nb_pad, h->M);
+      if (ternary) sm::launch_sign8(s, h->U, p.dpad, p.d, h->sign8, p.dpad, h->M);
+      else sm::launch_pack(s, h->U, p.dpad, p.d, h->bits, p.nb_pad, h->M);
     }
   }
-  if (h->flags & SIGNMUON_POST_POLAR) {
-    // the majority goes straight into the polar step's input (and into D
-    // only when K == 0, where the polar factor is the scaled input itself)
+  if (h->flags & (SIGNMUON_POST_POLAR | SIGNMUON_NORMALIZED_SIGN)) {
+    // post-vote step on the majority matrix: PolarNS with the handle's K, or
+    // (normalised sign step) with none, which leaves majority / (s + eps)
+    const int k_post = (h->flags & SIGNMUON_NORMALIZED_SIGN) ? 0 : h->K;
     {
       ProfScope ps(h, 7);
-      sm::launch_vote_stage(s, h->bits, p.nb_pad, h->M, h->X[0], p.fp32 ? 0 : 1, h->d_chunks, (int)p.chunks.size(),
-                            h->d_mats, h->d_groups, h->partials, h->K == 0 ? h->D : nullptr, tie);
+      if (ternary) {
+        // majority -> D, then D staged as the step's input (a one-worker
+        // mean, which is D itself) with its sum-of-squares partials
+        sm::launch_vote_ternary_major(s, h->sign8, p.dpad, h->M, p.d, h->D, tie);
+        sm::launch_mean_stage(s, h->D, 0, 1, h->X[0], p.fp32 ? 0 : 1, h->d_chunks, (int)p.chunks.size(), h->d_mats,
+                              h->d_groups, h->partials, nullptr);
+      } else {
+        // the majority goes straight into the step's input (and into D only
+        // when K == 0, where the result is the scaled input itself)
+        sm::launch_vote_stage(s, h->bits, p.nb_pad, h->M, h->X[0], p.fp32 ? 0 : 1, h->d_chunks,
+                              (int)p.chunks.size(), h->d_mats, h->d_groups, h->partials,
+                              k_post == 0 ? h->D : nullptr, tie);
+      }
     }
     fro_finalize(h, 1);
-    run_ns(h, 1, dp, h->D, 0);
+    run_ns(h, k_post, 1, dp, h->D, 0);
     ProfScope ps(h, 12);
     sm::launch_update(s, W, h->D, p.d, eta, h->status);
   } else {
     ProfScope ps(h, 7);
-    sm::launch_vote_update(s, h->bits, p.nb_pad, h->M, p.d, W, eta, h->status, tie);
+    if (ternary) sm::launch_vote_ternary_update(s, h->sign8, p.dpad, h->M, p.d, W, eta, h->status, tie);
+    else sm::launch_vote_update(s, h->bits, p.nb_pad, h->M, p.d, W, eta, h->status, tie);
   }
   return finish(h, (h->flags & SIGNMUON_ASYNC) == 0);
 }
@@ -704,6 +726,32 @@ int signmuon_pack(signmuon_t h, const float* U, int64_t d, uint8_t* out) {
   return SIGNMUON_OK;
 }
 
+int signmuon_sign_ternary(signmuon_t h, const float* U, int64_t d, int8_t* out) {
+  int rc = check_handle(h, false);
+  if (rc) return rc;
+  if (d < 0 || (d > 0 && (U == nullptr || out == nullptr))) return fail(h, SIGNMUON_E_INVALID, "bad sign arguments");
+  if (!aligned16(U) || !aligned16(out)) return fail(h, SIGNMUON_E_INVALID, "U/out must be 16-byte aligned");
+  sm::launch_sign8(h->stream, U, 0, d, out, 0, 1);
+  CK(h, cudaGetLastError());
+  return SIGNMUON_OK;
+}
+
+int signmuon_vote_ternary(signmuon_t h, const int8_t* const* signs, int64_t d, void* sums, int8_t* majority) {
+  int rc = check_handle(h, false);
+  if (rc) return rc;
+  if (d < 0 || signs == nullptr) return fail(h, SIGNMUON_E_INVALID, "bad vote arguments");
+  for (int m = 0; m < h->M; ++m)
+    if (signs[m] == nullptr || !aligned16(signs[m])) return fail(h, SIGNMUON_E_INVALID, "signs[m] null or misaligned");
+  if ((sums && !aligned16(sums)) || (majority && !aligned16(majority)))
+    return fail(h, SIGNMUON_E_INVALID, "sums/majority must be 16-byte aligned");
+  sm::WorkerPtrs sp{};
+  for (int m = 0; m < h->M; ++m) sp.p[m] = reinterpret_cast<const float*>(signs[m]);
+  sm::launch_vote_ternary(h->stream, sp, h->M, d, sums, (h->flags & SIGNMUON_ACC_INT8) ? 1 : 0, majority,
+                          (h->flags & SIGNMUON_TIE_PLUS) ? 1 : 0);
+  CK(h, cudaGetLastError());
+  return SIGNMUON_OK;
+}
+
 int signmuon_apply_update(signmuon_t h, float* W, const float* D, int64_t d, float eta) {
   int rc = check_handle(h, false);
   if (rc) return rc;
@@ -728,7 +776,7 @@ int signmuon_polar(signmuon_t h, const float* const* X, float* const* U) {
   sm::launch_stage(s, xp, h->M, h->X[0], p.fp32 ? 0 : 1, h->d_chunks, (int)p.chunks.size(), h->d_mats, h->d_groups,
                    h->partials);
   fro_finalize(h, h->M);
-  run_ns(h, h->M, xp, h->U, p.dpad);
+  run_ns(h, h->K, h->M, xp, h->U, p.dpad);
   h->u_valid = true;
   for (int m = 0; m < h->M; ++m)
     CK(h, cudaMemcpyAsync(U[m], h->U + (int64_t)m * p.dpad, (size_t)p.d * 4, cudaMemcpyDeviceToDevice, s));
@@ -770,8 +818,21 @@ int signmuon_get_signs(signmuon_t h, int m, uint8_t* dst) {
   int rc = check_handle(h, true);
   if (rc) return rc;
   if (m < 0 || m >= h->M || !dst) return fail(h, SIGNMUON_E_INVALID, "bad worker index or null dst");
-  if (!h->bits_valid) return fail(h, SIGNMUON_E_UNSUPPORTED, "a SIGNMUON_MUON_MEAN step packs no signs");
+  if (!h->bits_valid)
+    return fail(h, SIGNMUON_E_UNSUPPORTED,
+                (h->flags & SIGNMUON_TERNARY) ? "a SIGNMUON_TERNARY step sends int8 signs: use signmuon_get_ternary_signs"
+                                              : "a SIGNMUON_MUON_MEAN step packs no signs");
   CK(h, cudaMemcpyAsync(dst, h->bits + (int64_t)m * h->plan.nb_pad, (size_t)h->plan.nb, cudaMemcpyDeviceToDevice,
+                        h->stream));
+  return SIGNMUON_OK;
+}
+
+int signmuon_get_ternary_signs(signmuon_t h, int m, int8_t* dst) {
+  int rc = check_handle(h, true);
+  if (rc) return rc;
+  if (m < 0 || m >= h->M || !dst) return fail(h, SIGNMUON_E_INVALID, "bad worker index or null dst");
+  if (!h->t_valid) return fail(h, SIGNMUON_E_UNSUPPORTED, "no SIGNMUON_TERNARY step has run on this handle");
+  CK(h, cudaMemcpyAsync(dst, h->sign8 + (int64_t)m * h->plan.dpad, (size_t)h->plan.d, cudaMemcpyDeviceToDevice,
                         h->stream));
   return SIGNMUON_OK;
 }
@@ -781,8 +842,14 @@ int signmuon_get_direction(signmuon_t h, float* dst) {
   if (rc) return rc;
   if (!dst || !aligned16(dst)) return fail(h, SIGNMUON_E_INVALID, "null or misaligned dst");
   const Plan& p = h->plan;
-  if (h->flags & (SIGNMUON_POST_POLAR | SIGNMUON_MUON_MEAN)) {
+  if (h->flags & (SIGNMUON_POST_POLAR | SIGNMUON_MUON_MEAN | SIGNMUON_NORMALIZED_SIGN)) {
     CK(h, cudaMemcpyAsync(dst, h->D, (size_t)p.d * 4, cudaMemcpyDeviceToDevice, h->stream));
+  } else if (h->flags & SIGNMUON_TERNARY) {
+    // the step fuses the vote into the update; recompute the majority from
+    // the last step's ternary signs
+    sm::launch_vote_ternary_major(h->stream, h->sign8, p.dpad, h->M, p.d, dst,
+                                  (h->flags & SIGNMUON_TIE_PLUS) ? 1 : 0);
+    CK(h, cudaGetLastError());
   } else {
     // the step fuses the vote into the update; recompute the majority from
     // the last step's packed signs

@@ -135,6 +135,20 @@ def bernoulli_bits(d, M, config_id=0, lo=0.3, hi=0.7):
     return np.stack([rng(config_id, 0, "bits", m).random(d) < p for m in range(M)])
 
 
+def ternary_signs(d, M, config_id=0, p_zero=0.2, lo=0.3, hi=0.7):
+    """Ternary vote stress input: per entry p_i ~ U(lo, hi); each of M workers
+    independently sends 0 with probability p_zero, else +1 with probability
+    p_i and -1 otherwise.  Returns a (M, d) int8 array."""
+    p = rng(config_id, 0, "p").uniform(lo, hi, size=d)
+    out = np.empty((M, d), np.int8)
+    for m in range(M):
+        g = rng(config_id, 0, "bits", m)
+        z = g.random(d) < p_zero
+        plus = g.random(d) < p
+        out[m] = np.where(z, 0, np.where(plus, 1, -1)).astype(np.int8)
+    return out
+
+
 def ternary_direction(d, config_id=0, p_zero=0.1):
     """A direction with entries in {-1, 0, +1} (float32)."""
     g = rng(config_id, 0, "dir")

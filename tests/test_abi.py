@@ -76,12 +76,32 @@ def test_status_strings():
 
 
 # POLAR_AFTER_ONLY (1 << 8) without POST_POLAR (1 << 2); MUON_MEAN (1 << 9)
-# with the post-vote polar step
-@pytest.mark.parametrize("flags", [1 << 8, (1 << 9) | (1 << 2), (1 << 9) | (1 << 8) | (1 << 2)])
+# with the post-vote polar step or a sign wire flag (TERNARY 1 << 10,
+# NORMALIZED_SIGN 1 << 11); NORMALIZED_SIGN with POST_POLAR
+BAD_FLAG_SETS = [1 << 8, (1 << 9) | (1 << 2), (1 << 9) | (1 << 8) | (1 << 2), (1 << 9) | (1 << 10),
+                 (1 << 9) | (1 << 11), (1 << 11) | (1 << 2), (1 << 11) | (1 << 8) | (1 << 2)]
+
+
+@pytest.mark.parametrize("flags", BAD_FLAG_SETS)
 def test_init_rejects_variant_flag_combinations(flags):
     # checked before any CUDA call: runs without a GPU
     import sign_muon_optimizer_b200 as smo
     assert smo.SIGNMUON_POLAR_AFTER_ONLY == 1 << 8 and smo.SIGNMUON_MUON_MEAN == 1 << 9
+    assert smo.SIGNMUON_TERNARY == 1 << 10 and smo.SIGNMUON_NORMALIZED_SIGN == 1 << 11
     with pytest.raises(smo.SignMuonError) as e:
         smo.SignMuon([(8, 8)], 2, flags=flags)
     assert e.value.status == smo.SIGNMUON_E_INVALID
+    with pytest.raises(smo.SignMuonError) as e:
+        smo.signmuon_plan([(8, 8)], 2, flags=flags)
+    assert e.value.status == smo.SIGNMUON_E_INVALID
+
+
+def test_plan_accepts_the_sign_wire_variants_and_counts_ternary_bytes():
+    import sign_muon_optimizer_b200 as smo
+    shapes = [(8, 24), (40, 16)]
+    base = smo.signmuon_plan(shapes, 5, 5, "spectral", 2)
+    for flags in (1 << 10, 1 << 11, (1 << 10) | (1 << 11), (1 << 10) | (1 << 2), (1 << 10) | (1 << 8) | (1 << 2)):
+        p = smo.signmuon_plan(shapes, 5, 5, "spectral", 2, flags)
+        # one int8 per entry and worker, at the library's 64-entry padded stride
+        extra = 5 * ((p["d"] + 63) // 64 * 64) if flags & (1 << 10) else 0
+        assert p["device_bytes"] == base["device_bytes"] + extra
