@@ -42,6 +42,9 @@ R7  Ties map to 0 ([blog]) by default; the +1 policy of [paper] Algorithm 2 is
 R8  Post-vote polar: D = PolarNS(majority as floats) with the same K, eps,
     scale and P; no second sign, no rescale.
 R9  Update: W_new = float32 nearest to (W - eta*D), one rounding.
+R21 Warm-started power iteration (named variant): each problem's power
+    iteration starts from the iterate it ended with in the previous step;
+    a zero or non-finite stored iterate starts from ones/sqrt(m) as in R2.
 
 Named variants (each a flag of the CUDA path, pinned in the tests):
 
@@ -57,6 +60,10 @@ Named variants (each a flag of the CUDA path, pinned in the tests):
   as integers (pinned by brute force over all 3^M patterns, by the zero
   momentum closed form, and by equality with the one-bit step when U has no
   zeros).
+* step(..., warm={...}): warm-started power iterations (R21; [paper]
+  Algorithm 1's P with the iterate carried across steps).  On a constant
+  matrix, t warm steps of P iterations equal one cold start with P*t
+  iterations exactly (pinned), and a zero state restarts cold.
 * step(..., normalize=True): D = majority / ||majority||_2 per matrix
   ([paper] §4, the explicitly normalised sign step of the analysis), with the
   norm estimated as PolarNS estimates its scale (pinned by exact singular
@@ -98,18 +105,27 @@ def frobenius_norm(x):
     return math.sqrt(float(np.sum(x * x)))
 
 
-def power_sigma(x, P):
+def power_sigma(x, P, u0=None, return_u=False):
     """Estimate of the largest singular value of a wide X (m <= n) by P power
-    iterations on X X^T (reading R2; [paper] Algorithm 1 input P, §4)."""
+    iterations on X X^T (reading R2; [paper] Algorithm 1 input P, §4).
+
+    u0 is a warm start on the small side (reading R21): the iterate a previous
+    call ended with.  None, an all-zero or a non-finite u0 starts from
+    ones(m)/sqrt(m).  With return_u the final iterate comes back as well.
+    """
     x = np.asarray(x, np.float64)
     m = x.shape[0]
-    u = np.full(m, 1.0 / math.sqrt(m))
+    if u0 is not None and np.all(np.isfinite(u0)) and np.any(np.asarray(u0) != 0):
+        u = np.array(u0, np.float64)
+    else:
+        u = np.full(m, 1.0 / math.sqrt(m))
     for _ in range(int(P)):
         y = x @ (x.T @ u)
         nrm = math.sqrt(float(y @ y))
         u = y / nrm if nrm > 0.0 else np.zeros(m)
     z = x.T @ u
-    return math.sqrt(float(z @ z))
+    sigma = math.sqrt(float(z @ z))
+    return (sigma, u) if return_u else sigma
 
 
 def ns_iterate(x0, K, order="cubic", coeffs=None):
@@ -135,26 +151,31 @@ def ns_iterate(x0, K, order="cubic", coeffs=None):
     return x
 
 
-def polar_ns(mat, K, eps, scale, P=1, order="cubic", coeffs=None, return_scale=False):
+def polar_ns(mat, K, eps, scale, P=1, order="cubic", coeffs=None, return_scale=False, u0=None,
+             return_u=False):
     """PolarNS(Mat; K, eps, scale, P) of one matrix ([paper] Algorithm 1, §4).
 
     Works on the wide orientation (R1), divides by s + eps where s is the
     Frobenius norm or the power-iteration estimate of the spectral norm
     (R2, R3), runs K Newton-Schulz steps and returns the result in the
-    matrix's own orientation.
+    matrix's own orientation.  u0 warm-starts the power iteration (R21);
+    return_u returns (result, s, final iterate or None for fro).
     """
     mat = np.asarray(mat, np.float64)
     tall = mat.shape[0] > mat.shape[1]
     x = mat.T if tall else mat
+    u = None
     if scale == "fro":
         s = frobenius_norm(x)
     elif scale == "spectral":
-        s = power_sigma(x, P)
+        s, u = power_sigma(x, P, u0, return_u=True)
     else:
         raise ValueError(scale)
     x = x / (s + float(eps))
     x = ns_iterate(x, K, order, coeffs)
     out = x.T if tall else x
+    if return_u:
+        return out, s, u
     return (out, s) if return_scale else out
 
 
@@ -296,40 +317,52 @@ def split(flat, shapes, offsets=None):
     return out
 
 
-def polar_flat(flat, shapes, K, eps, scale, P=1, order="cubic"):
-    """PolarNS of every matrix of a flat vector, returned flat (float64)."""
+def polar_flat(flat, shapes, K, eps, scale, P=1, order="cubic", u0=None, return_u=False):
+    """PolarNS of every matrix of a flat vector, returned flat (float64).
+    u0: None or one warm start (or None) per matrix (R21); with return_u the
+    per-matrix final iterates come back too."""
     out = np.empty(int(np.asarray(flat).size), np.float64)
+    us = []
     off = 0
-    for (r, c), mat in zip(shapes, split(np.asarray(flat, np.float64), shapes)):
-        out[off: off + r * c] = polar_ns(mat, K, eps, scale, P, order).ravel()
+    for i, ((r, c), mat) in enumerate(zip(shapes, split(np.asarray(flat, np.float64), shapes))):
+        res, _, u = polar_ns(mat, K, eps, scale, P, order, u0=None if u0 is None else u0[i], return_u=True)
+        us.append(u)
+        out[off: off + r * c] = res.ravel()
         off += r * c
-    return out
+    return (out, us) if return_u else out
 
 
-def normalize_flat(flat, shapes, eps, scale, P=1):
+def normalize_flat(flat, shapes, eps, scale, P=1, u0=None, return_u=False):
     """Each matrix of a flat vector divided by its norm: D_i / (s_i + eps).
 
     [paper] §4 (single-worker variant) notes that the theory normalises the
     sign matrix explicitly by its spectral norm, D / ||D||_2.  s_i is the same
     scale estimate PolarNS uses for its input (reading R2 for spectral: P power
     iterations on the wide orientation; the Frobenius norm for fro), and eps
-    keeps an all-zero majority at zero.  This is PolarNS with K = 0.
+    keeps an all-zero majority at zero.  This is PolarNS with K = 0.  u0 and
+    return_u: per-matrix warm starts and final iterates, as in polar_flat.
     """
     if scale not in ("fro", "spectral"):
         raise ValueError(scale)
     out = np.empty(int(np.asarray(flat).size), np.float64)
+    us = []
     off = 0
-    for (r, c), mat in zip(shapes, split(np.asarray(flat, np.float64), shapes)):
+    for i, ((r, c), mat) in enumerate(zip(shapes, split(np.asarray(flat, np.float64), shapes))):
         x = mat.T if r > c else mat
-        s = frobenius_norm(x) if scale == "fro" else power_sigma(x, P)
+        u = None
+        if scale == "fro":
+            s = frobenius_norm(x)
+        else:
+            s, u = power_sigma(x, P, None if u0 is None else u0[i], return_u=True)
+        us.append(u)
         out[off: off + r * c] = (mat / (s + float(eps))).ravel()
         off += r * c
-    return out
+    return (out, us) if return_u else out
 
 
 def step(W, G_list, mom_list, shapes, *, beta, lam, eta, K, eps, scale, P=1,
          order="cubic", post_polar=False, acc="int32", tie=0, pre_polar=True,
-         signs="bits", normalize=False):
+         signs="bits", normalize=False, warm=None):
     """One distributed Sign-Muon step ([paper] Algorithm 2, with the vote of
     [blog] and the optional post-vote polar step of [paper] §4).
 
@@ -341,7 +374,11 @@ def step(W, G_list, mom_list, shapes, *, beta, lam, eta, K, eps, scale, P=1,
     sign(0) = 0, and Algorithm 2's d-byte int8 all-reduce) instead of one bit;
     normalize=True takes D = majority / ||majority||_2 per matrix ([paper] §4,
     the explicitly normalised sign step of the analysis; cannot be combined
-    with post_polar).
+    with post_polar); warm (a dict, {} on the first step) warm-starts every
+    power iteration from the previous step's final iterates (reading R21):
+    warm["workers"][m][i] for worker m's matrix i, warm["single"][i] for the
+    post-vote or normalised step's matrix i; the new state is returned as
+    out["warm"].
 
     Returns a dict with the new momentum (float64), the polar factors U_m
     (the momentum itself when pre_polar is False), the packed bits (the int8
@@ -357,11 +394,19 @@ def step(W, G_list, mom_list, shapes, *, beta, lam, eta, K, eps, scale, P=1,
         raise ValueError(signs)
     M = len(G_list)
     d = int(np.asarray(W).size)
+    wk = None if warm is None else warm.get("workers")
+    new_warm = None if warm is None else dict(workers=[None] * M, single=warm.get("single"))
     new_mom, U_list, packed = [], [], []
     for m in range(M):
         mom = momentum_update(mom_list[m], G_list[m], W, beta, lam)
         new_mom.append(mom)
-        u = polar_flat(mom, shapes, K, eps, scale, P, order) if pre_polar else np.asarray(mom, np.float64)
+        if pre_polar:
+            u, us = polar_flat(mom, shapes, K, eps, scale, P, order, u0=None if wk is None else wk[m],
+                               return_u=True)
+            if new_warm is not None:
+                new_warm["workers"][m] = us
+        else:
+            u = np.asarray(mom, np.float64)
         U_list.append(u)
         if signs == "ternary":
             packed.append(sign_ternary(u).astype(np.int8))
@@ -372,28 +417,36 @@ def step(W, G_list, mom_list, shapes, *, beta, lam, eta, K, eps, scale, P=1,
     else:
         sums = vote_sums_from_bits(packed, d, acc)
     maj = majority(sums, tie)
+    single = None if warm is None else warm.get("single")
     if post_polar:
-        D = polar_flat(maj.astype(np.float64), shapes, K, eps, scale, P, order)
+        D, us = polar_flat(maj.astype(np.float64), shapes, K, eps, scale, P, order, u0=single, return_u=True)
         D32 = D.astype(np.float32)
+        if new_warm is not None:
+            new_warm["single"] = us
     elif normalize:
-        D = normalize_flat(maj.astype(np.float64), shapes, eps, scale, P)
+        D, us = normalize_flat(maj.astype(np.float64), shapes, eps, scale, P, u0=single, return_u=True)
         D32 = D.astype(np.float32)
+        if new_warm is not None:
+            new_warm["single"] = us
     else:
         D = maj.astype(np.float64)
         D32 = maj.astype(np.float32)
     W_new = update(W, D32, eta)
     return dict(mom=new_mom, U=U_list, packed=packed, sums=sums, majority=maj,
-                D=D, D32=D32, W=W_new)
+                D=D, D32=D32, W=W_new, warm=new_warm)
 
 
-def muon_step(W, G_list, mom_list, shapes, *, beta, lam, eta, K, eps, scale, P=1, order="cubic"):
+def muon_step(W, G_list, mom_list, shapes, *, beta, lam, eta, K, eps, scale, P=1, order="cubic", warm=None):
     """The Muon baseline the pages compare against ([paper] §4 Muon update,
     Table 1's "Muon" row): the workers' momenta are averaged (the all-reduce
     of full-precision momentum) and the mean goes through one PolarNS per
-    matrix; W_new = fl32(W - eta * D) with D = PolarNS(mean Mom)."""
+    matrix; W_new = fl32(W - eta * D) with D = PolarNS(mean Mom).  warm as in
+    step (the mean's power iterations use warm["single"])."""
     M = len(G_list)
     new_mom = [momentum_update(mom_list[m], G_list[m], W, beta, lam) for m in range(M)]
     mean = np.sum(np.stack([np.asarray(x, np.float64) for x in new_mom]), axis=0) / M
-    D = polar_flat(mean, shapes, K, eps, scale, P, order)
+    D, us = polar_flat(mean, shapes, K, eps, scale, P, order, u0=None if warm is None else warm.get("single"),
+                       return_u=True)
     D32 = D.astype(np.float32)
-    return dict(mom=new_mom, mean=mean, D=D, D32=D32, W=update(W, D32, eta))
+    new_warm = None if warm is None else dict(workers=warm.get("workers"), single=us)
+    return dict(mom=new_mom, mean=mean, D=D, D32=D32, W=update(W, D32, eta), warm=new_warm)

@@ -606,3 +606,92 @@ def test_normalize_of_an_all_tied_vote_is_zero_and_guards():
     with pytest.raises(ValueError):
         ref.step(W, [g], [np.zeros(4)], [(2, 2)], beta=0.0, lam=0.0, eta=0.5, K=2, eps=1e-7, scale="fro",
                  signs="trits")
+
+
+# ---------------------------------------------------------------------------
+# warm-started power iteration (named variant: the iterate carried across steps)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("P", [1, 2])
+def test_warm_power_iteration_composes_with_cold_start(P):
+    # power iteration composes: t warm calls of P iterations on one matrix are
+    # the same arithmetic as one cold call of P*t iterations (bit for bit)
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal((6, 9))
+    u = None
+    for t in range(1, 6):
+        s_warm, u = ref.power_sigma(x, P, u, return_u=True)
+        s_cold, u_cold = ref.power_sigma(x, P * t, return_u=True)
+        assert s_warm == s_cold and np.array_equal(u, u_cold)
+    # and it converges to numpy's largest singular value
+    s_far, _ = ref.power_sigma(x, 400, return_u=True)
+    assert abs(s_far - np.linalg.svd(x, compute_uv=False)[0]) < 1e-12 * s_far
+
+
+def test_warm_power_iteration_fixed_point_and_restart():
+    # diag(5, 2, 1) padded wide: e1 is the top singular vector, so a warm
+    # start there gives sigma = 5 after one iteration; a zero or non-finite
+    # stored iterate restarts from ones/sqrt(m) exactly like a cold start
+    x = np.zeros((3, 5))
+    x[0, 0], x[1, 1], x[2, 2] = 5.0, 2.0, 1.0
+    s, u = ref.power_sigma(x, 1, np.array([1.0, 0.0, 0.0]), return_u=True)
+    assert s == 5.0 and np.array_equal(u, np.array([1.0, 0.0, 0.0]))
+    cold = ref.power_sigma(x, 2)
+    assert ref.power_sigma(x, 2, np.zeros(3)) == cold
+    assert ref.power_sigma(x, 2, np.array([np.nan, 1.0, 0.0])) == cold
+    # a zero matrix leaves a zero iterate behind, which the next call restarts
+    s0, u0 = ref.power_sigma(np.zeros((3, 5)), 2, return_u=True)
+    assert s0 == 0.0 and not u0.any()
+    assert ref.power_sigma(x, 2, u0) == cold
+
+
+@pytest.mark.parametrize("post_polar", [False, True])
+def test_warm_step_threads_the_state_per_worker_and_matrix(post_polar):
+    # beta = 0, lambda = 0 and one gradient per worker repeated every step:
+    # the momentum (so the Gram) is constant, and after t warm steps of P
+    # iterations each (worker, matrix) iterate equals a cold start with P*t
+    # iterations on that worker's matrix; the post-vote state does the same on
+    # the majority matrix, constant too because K = 0 makes the signs those of
+    # the momentum (with K > 0 the changing scale moves small entries of U)
+    rng = np.random.default_rng(9)
+    shapes = [(4, 7), (6, 3)]
+    d = 28 + 18
+    M, P = 3, 1
+    G = [rng.standard_normal(d) for _ in range(M)]
+    W = np.zeros(d, np.float32)
+    kw = dict(beta=0.0, lam=0.0, eta=0.01, K=0, eps=1e-7, scale="spectral", P=P, post_polar=post_polar)
+    warm = {}
+    maj0 = None
+    for t in range(1, 4):
+        out = ref.step(W, G, [np.zeros(d)] * M, shapes, warm=warm, **kw)
+        warm = out["warm"]
+        maj0 = out["majority"] if maj0 is None else maj0
+        assert np.array_equal(out["majority"], maj0)
+        for m in range(M):
+            for i, x in enumerate(ref.split(G[m], shapes)):
+                xw = x.T if x.shape[0] > x.shape[1] else x
+                _, u_cold = ref.power_sigma(xw, P * t, return_u=True)
+                assert np.array_equal(warm["workers"][m][i], u_cold)
+        if post_polar:
+            for i, x in enumerate(ref.split(out["majority"].astype(np.float64), shapes)):
+                xw = x.T if x.shape[0] > x.shape[1] else x
+                _, u_cold = ref.power_sigma(xw, P * t, return_u=True)
+                assert np.array_equal(warm["single"][i], u_cold)
+        else:
+            assert warm["single"] is None
+    # without warm the step keeps no state
+    assert ref.step(W, G, [np.zeros(d)] * M, shapes, **kw)["warm"] is None
+
+
+def test_warm_muon_step_uses_the_single_state():
+    rng = np.random.default_rng(13)
+    shapes = [(5, 8)]
+    G = [rng.standard_normal(40) for _ in range(2)]
+    W = np.zeros(40, np.float32)
+    kw = dict(beta=0.0, lam=0.0, eta=0.01, K=1, eps=1e-7, scale="spectral", P=2)
+    warm = {}
+    for t in range(1, 3):
+        out = ref.muon_step(W, G, [np.zeros(40)] * 2, shapes, warm=warm, **kw)
+        warm = out["warm"]
+        _, u_cold = ref.power_sigma(out["mean"].reshape(5, 8), 2 * t, return_u=True)
+        assert np.array_equal(warm["single"][0], u_cold)
