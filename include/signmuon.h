@@ -76,12 +76,20 @@ typedef struct signmuon_ctx* signmuon_t;
  *                    the majority matrix (spectral: the P-step power-iteration estimate of
  *                    ||majority||_2; fro: ||majority||_F) -- the explicitly normalised sign
  *                    step of §4's analysis.  Cannot be combined with POST_POLAR (it is the
- *                    post-vote step with no Newton-Schulz iteration). */
+ *                    post-vote step with no Newton-Schulz iteration).
+ * PI_WARM            each power iteration (spectral scale) starts from the iterate the same
+ *                    problem ended with in the previous call instead of ones/sqrt(m): one
+ *                    state per (worker, matrix) for the M-worker PolarNS (signmuon_step and
+ *                    signmuon_polar share it) and one per matrix for the post-vote,
+ *                    normalised-sign and Muon-baseline PolarNS.  A zero or non-finite state
+ *                    (the first call, a zero matrix, a failed step) starts cold.  The state
+ *                    is not part of get/set_momentum.  No effect with SIGNMUON_SCALE_FRO. */
 #define SIGNMUON_TIE_PLUS          (1u << 7)
 #define SIGNMUON_POLAR_AFTER_ONLY  (1u << 8)
 #define SIGNMUON_MUON_MEAN         (1u << 9)
 #define SIGNMUON_TERNARY           (1u << 10)
 #define SIGNMUON_NORMALIZED_SIGN   (1u << 11)
+#define SIGNMUON_PI_WARM           (1u << 12)
 
 /* ------------------------------------------------------------------------
  * signmuon_init -- plan the step and allocate its device state.

@@ -41,6 +41,7 @@ SIGNMUON_POLAR_AFTER_ONLY = 1 << 8
 SIGNMUON_MUON_MEAN = 1 << 9
 SIGNMUON_TERNARY = 1 << 10
 SIGNMUON_NORMALIZED_SIGN = 1 << 11
+SIGNMUON_PI_WARM = 1 << 12
 
 EXPORTED = [
     "signmuon_init", "signmuon_step", "signmuon_step_host", "signmuon_vote", "signmuon_pack",

@@ -131,7 +131,8 @@ void launch_fro_finalize(cudaStream_t s, int n_probs, int n_mats, int M, const f
                          const int* mat_chunk0, const int* mat_nchunks, int use_for_scale,
                          float eps, int quintic, float a, float b, float c, float* scale,
                          float2* coef_apply, float2* coef_square, int* status);
-void launch_pi_init(cudaStream_t s, int n_probs, const int64_t* uoff, const int* prob_g, float* u);
+// warm != 0: keep each problem's stored iterate when it is non-zero and finite
+void launch_pi_init(cudaStream_t s, int n_probs, const int64_t* uoff, const int* prob_g, float* u, int warm);
 void launch_pi_matvec(cudaStream_t s, const ProbRows* rows, int n_rows, const void* A, int a_bf16,
                       const int64_t* prob_a_off, const int* prob_g, const int* prob_gld,
                       const int64_t* uoff, const float* u, float* y, int max_g);

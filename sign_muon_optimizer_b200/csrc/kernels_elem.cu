@@ -190,13 +190,26 @@ k_fro_finalize(int n_mats, int M, const float* __restrict__ partials, const int*
 // normalisation by power iteration): u0 = ones/sqrt(g); u <- A~u/||A~u|| P
 // times; sigma^2 = u^T A~ u (= ||X~^T u||^2).  The Gram is the first
 // Newton-Schulz GEMM's output, so no extra pass over X is needed.
+// With warm set, a problem whose stored iterate (the one the previous call
+// ended with) is non-zero and finite starts from it instead of ones/sqrt(g).
 // ---------------------------------------------------------------------------
-__global__ void k_pi_init(const int64_t* __restrict__ uoff, const int* __restrict__ prob_g,
-                          float* __restrict__ u) {
+__global__ void __launch_bounds__(kThreads)
+k_pi_init(const int64_t* __restrict__ uoff, const int* __restrict__ prob_g, float* __restrict__ u, int warm) {
+  __shared__ double red[32];
+  __shared__ int keep;
   const int p = blockIdx.x;
   const int g = prob_g[p];
+  float* up = u + uoff[p];
+  if (warm) {
+    double s = 0.0;
+    for (int k = threadIdx.x; k < g; k += kThreads) s += (double)up[k] * (double)up[k];
+    const double t = block_sum<double>(s, red);
+    if (threadIdx.x == 0) keep = (t > 0.0 && isfinite(t)) ? 1 : 0;
+    __syncthreads();
+    if (keep) return;  // the whole block leaves together
+  }
   const float v = rsqrtf((float)g);
-  for (int k = threadIdx.x; k < g; k += blockDim.x) u[uoff[p] + k] = v;
+  for (int k = threadIdx.x; k < g; k += kThreads) up[k] = v;
 }
 
 template <bool BF16>
@@ -843,9 +856,9 @@ void launch_fro_finalize(cudaStream_t s, int n_probs, int n_mats, int M, const f
                                               coef_apply, coef_square, status);
 }
 
-void launch_pi_init(cudaStream_t s, int n_probs, const int64_t* uoff, const int* prob_g, float* u) {
+void launch_pi_init(cudaStream_t s, int n_probs, const int64_t* uoff, const int* prob_g, float* u, int warm) {
   count_launch();
-  k_pi_init<<<n_probs, kThreads, 0, s>>>(uoff, prob_g, u);
+  k_pi_init<<<n_probs, kThreads, 0, s>>>(uoff, prob_g, u, warm);
 }
 
 void launch_pi_matvec(cudaStream_t s, const ProbRows* rows, int n_rows, const void* A, int a_bf16,

@@ -191,7 +191,10 @@ int make_plan(const int64_t* shapes, int n_mats, int M, int K, int scale, int P,
       u += g.g;
       for (int r0 = 0; r0 < g.g; r0 += kPiRows) p.pi_rows.push_back(ProbRows{pid, r0});
     }
-    if (w == 0) p.n_pi_rows_one = (int)p.pi_rows.size();
+    if (w == 0) {
+      p.n_pi_rows_one = (int)p.pi_rows.size();
+      p.u_elems_one = u;
+    }
   }
   p.u_elems = u;
   const int64_t esz = p.fp32 ? 4 : 2;
@@ -206,6 +209,7 @@ int make_plan(const int64_t* shapes, int n_mats, int M, int K, int scale, int P,
     bytes += (int64_t)p.chunks.size() * M * 4;            // norm partials
     bytes += (int64_t)M * n_mats * (4 + 8 + 8);           // scales, coefficients
     bytes += 2 * p.u_elems * 4;                           // power-iteration vectors
+    if (flags & SIGNMUON_PI_WARM) bytes += p.u_elems_one * 4;  // warm state of one problem set
     bytes += (int64_t)p.groups.size() * 8 * 128;          // tensor maps
   }
   p.device_bytes = bytes;

@@ -40,6 +40,7 @@ struct Plan {
   std::vector<int> prob_g, prob_gld;
   std::vector<int64_t> prob_aoff;
   int64_t u_elems = 0;
+  int64_t u_elems_one = 0;  // power-iteration vector entries of worker 0 (one problem set)
   int64_t device_bytes = 0;  // everything the handle allocates
 };
 

@@ -69,7 +69,8 @@ struct signmuon_ctx {
   float* scale_v = nullptr;
   float2* coef_apply = nullptr;
   float2* coef_square = nullptr;
-  float* pi_u = nullptr;
+  float* pi_u = nullptr;        // power-iteration iterates of the M-worker problems (warm state)
+  float* pi_u1 = nullptr;       // PI_WARM: iterates of the one-problem-set PolarNS (warm state)
   float* pi_y = nullptr;
   int* status = nullptr;        // [0] non-finite flag, [1] kernel error code
   int* h_status = nullptr;      // pinned mirror
@@ -290,22 +291,28 @@ void gemm(signmuon_t h, int op, int slot, int src, int nw, const float2* coef, f
   else sm::launch_gemm_tc(h->stream, a, h->d_maps, h->n_sm);
 }
 
+// P power iterations on the Gram of nw problem sets.  With SIGNMUON_PI_WARM
+// each problem starts from the iterate it ended with last time: the M-worker
+// PolarNS (step or signmuon_polar) keeps its iterates in pi_u, the
+// one-problem-set PolarNS (post-vote, normalised sign, Muon mean) in pi_u1.
 void power_iteration(signmuon_t h, int nw) {
   const Plan& p = h->plan;
   const int nprob = nw * p.n_mats;
   const int nrows = nw == 1 ? p.n_pi_rows_one : (int)p.pi_rows.size();
+  const bool warm = (h->flags & SIGNMUON_PI_WARM) != 0;
+  float* u = (warm && nw == 1) ? h->pi_u1 : h->pi_u;
   ProfScope ps(h, 5);
   int max_g = 1;
   for (const sm::GroupInfo& gi : p.groups) max_g = gi.g > max_g ? gi.g : max_g;
-  sm::launch_pi_init(h->stream, nprob, h->d_uoff, h->d_prob_g, h->pi_u);
+  sm::launch_pi_init(h->stream, nprob, h->d_uoff, h->d_prob_g, u, warm ? 1 : 0);
   for (int it = 0; it < h->P; ++it) {
     sm::launch_pi_matvec(h->stream, h->d_pi_rows, nrows, h->A, p.fp32 ? 0 : 1, h->d_prob_aoff, h->d_prob_g,
-                         h->d_prob_gld, h->d_uoff, h->pi_u, h->pi_y, max_g);
-    sm::launch_pi_normalize(h->stream, nprob, h->d_uoff, h->d_prob_g, h->pi_y, h->pi_u);
+                         h->d_prob_gld, h->d_uoff, u, h->pi_y, max_g);
+    sm::launch_pi_normalize(h->stream, nprob, h->d_uoff, h->d_prob_g, h->pi_y, u);
   }
   sm::launch_pi_matvec(h->stream, h->d_pi_rows, nrows, h->A, p.fp32 ? 0 : 1, h->d_prob_aoff, h->d_prob_g,
-                       h->d_prob_gld, h->d_uoff, h->pi_u, h->pi_y, max_g);
-  sm::launch_pi_finalize(h->stream, nprob, h->d_uoff, h->d_prob_g, h->pi_u, h->pi_y, h->eps, p.quintic ? 1 : 0,
+                       h->d_prob_gld, h->d_uoff, u, h->pi_y, max_g);
+  sm::launch_pi_finalize(h->stream, nprob, h->d_uoff, h->d_prob_g, u, h->pi_y, h->eps, p.quintic ? 1 : 0,
                          h->ns_a, h->ns_b, h->ns_c, h->scale_v, h->coef_apply, h->coef_square, h->status);
 }
 
@@ -511,6 +518,13 @@ int signmuon_init(signmuon_t* out, const int64_t* shapes, int n_mats, int M, flo
   if ((rc = dalloc(h, &h->coef_square, (int64_t)M * p.n_mats))) return bail(rc);
   if ((rc = dalloc(h, &h->pi_u, p.u_elems))) return bail(rc);
   if ((rc = dalloc(h, &h->pi_y, p.u_elems))) return bail(rc);
+  if (flags & SIGNMUON_PI_WARM) {
+    // zero state: the first power iteration of every problem starts cold
+    if ((rc = dalloc(h, &h->pi_u1, p.u_elems_one))) return bail(rc);
+    if (cudaMemset(h->pi_u, 0, (size_t)p.u_elems * 4) != cudaSuccess ||
+        cudaMemset(h->pi_u1, 0, (size_t)p.u_elems_one * 4) != cudaSuccess)
+      return bail(fail(h, SIGNMUON_E_CUDA, "memset"));
+  }
   if (cudaMemset(h->Mom, 0, (size_t)M * p.dpad * 4) != cudaSuccess ||
       cudaMemset(h->bits, 0, (size_t)M * p.nb_pad) != cudaSuccess ||
       cudaMemset(h->scale_v, 0, (size_t)M * p.n_mats * 4) != cudaSuccess)

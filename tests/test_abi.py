@@ -105,3 +105,7 @@ def test_plan_accepts_the_sign_wire_variants_and_counts_ternary_bytes():
         # one int8 per entry and worker, at the library's 64-entry padded stride
         extra = 5 * ((p["d"] + 63) // 64 * 64) if flags & (1 << 10) else 0
         assert p["device_bytes"] == base["device_bytes"] + extra
+    # the warm power-iteration state of one problem set: min(rows, cols) floats per matrix
+    assert smo.SIGNMUON_PI_WARM == 1 << 12
+    p = smo.signmuon_plan(shapes, 5, 5, "spectral", 2, 1 << 12)
+    assert p["device_bytes"] == base["device_bytes"] + 4 * (8 + 16)
