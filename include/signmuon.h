@@ -133,6 +133,40 @@ int signmuon_init(signmuon_t* out, const int64_t* shapes, int n_mats, int M,
 int signmuon_step(signmuon_t h, float* W, const float* const* G, float eta);
 
 /* ------------------------------------------------------------------------
+ * signmuon_local_signs / signmuon_vote_step -- signmuon_step in two halves,
+ * so that the signs can cross a collective in between: each GPU holds some
+ * of the workers, all-gathers their signs, and every GPU votes and updates its
+ * own replica of W ([paper] Algorithm 2: local polar and sign, one exchange
+ * of the signs, local majority and update; [blog] "the actual bytes sent").
+ * signmuon_step(W, G) is signmuon_local_signs into the handle's own buffers
+ * followed by signmuon_vote_step over them, kernel for kernel.
+ *
+ * signmuon_local_signs: momentum, scale, PolarNS and signs of the handle's M
+ * workers; W is read (weight decay), not written.
+ *   W       device float[d].     G  host array of M device pointers, float[d].
+ *   signs   device buffer; worker m's signs at signs + m*stride: ceil(d/8)
+ *           packed bytes (LSB-first, as signmuon_pack), or d int8 ternary
+ *           signs with SIGNMUON_TERNARY.
+ *   stride  bytes between workers: a multiple of 16, at least one worker's
+ *           signs.
+ * Unless SIGNMUON_ASYNC, waits and returns E_NONFINITE when a momentum norm is
+ * NaN/Inf (the signs are then not valid: do not vote on them).  Not for
+ * MUON_MEAN handles (E_UNSUPPORTED).
+ *
+ * signmuon_vote_step: majority of M sign buffers at signs + j*stride (any M in
+ * 1..256, e.g. the all-gathered signs of every GPU's workers, in worker
+ * order), then the post-vote step the handle's flags ask for and W <-
+ * fl32(W - eta*D).  Vote-only handles may call it when they ask for no
+ * post-vote step.  Waits like signmuon_step.  After it, signmuon_get_direction
+ * gives D only for the post-vote steps (E_UNSUPPORTED when the vote was fused
+ * with the update).
+ * ---------------------------------------------------------------------- */
+int signmuon_local_signs(signmuon_t h, const float* W, const float* const* G, uint8_t* signs,
+                         int64_t stride);
+int signmuon_vote_step(signmuon_t h, float* W, const uint8_t* signs, int64_t stride, int M,
+                       float eta);
+
+/* ------------------------------------------------------------------------
  * signmuon_step_host -- signmuon_step on HOST buffers: copies W and the M
  * gradients to library-owned device buffers (allocated on first use),
  * runs the step and copies W back.  Always waits.  Pinned host memory gives
@@ -211,7 +245,8 @@ int signmuon_polar(signmuon_t h, const float* const* X, float* const* U);
  * get_signs: worker m's packed bits from the last step (SIGNMUON_E_UNSUPPORTED
  * with MUON_MEAN or TERNARY).  get_ternary_signs: worker m's int8[d] ternary
  * signs from the last step (SIGNMUON_E_UNSUPPORTED unless TERNARY).
- * get_direction: the last step's D.
+ * get_direction: the last step's D (E_UNSUPPORTED before the first step, and
+ * after a signmuon_vote_step whose vote was fused with the update).
  * get_scales: host float[M*n_mats]: the last step's scale s per (worker,
  * matrix), worker-major (waits for the GPU).
  * ---------------------------------------------------------------------- */

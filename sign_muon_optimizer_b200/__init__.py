@@ -51,7 +51,7 @@ EXPORTED = [
     "signmuon_kernel_launches", "signmuon_last_error", "signmuon_status_string", "signmuon_destroy",
     "signmuon_profile", "signmuon_profile_read", "signmuon_get_gram",
     "signmuon_spectral_norm_noalloc", "signmuon_sign_ternary", "signmuon_vote_ternary",
-    "signmuon_get_ternary_signs",
+    "signmuon_get_ternary_signs", "signmuon_local_signs", "signmuon_vote_step",
 ]
 PROF_KINDS = ["momentum", "norm_finalize", "ns_gram", "ns_square", "ns_apply", "power_iter", "pack",
               "vote", "stage", "post_gram", "post_square", "post_apply", "update", "k0_scale"]
@@ -78,6 +78,8 @@ def _load():
         "signmuon_sign_ternary": (I, [P, P, I64, P]),
         "signmuon_vote_ternary": (I, [P, PP, I64, P, P]),
         "signmuon_get_ternary_signs": (I, [P, I, P]),
+        "signmuon_local_signs": (I, [P, P, PP, P, I64]),
+        "signmuon_vote_step": (I, [P, P, P, I64, I, F]),
         "signmuon_apply_update": (I, [P, P, P, I64, F]),
         "signmuon_polar": (I, [P, PP, PP]),
         "signmuon_get_momentum": (I, [P, I, P]),
@@ -192,6 +194,14 @@ def signmuon_get_ternary_signs(h, m, dst):
     _check(h, _lib.signmuon_get_ternary_signs(h, int(m), _ptr(dst)))
 
 
+def signmuon_local_signs(h, W, G, signs, stride):
+    _check(h, _lib.signmuon_local_signs(h, _ptr(W), _ptr_array(G), _ptr(signs), int(stride)))
+
+
+def signmuon_vote_step(h, W, signs, stride, M, eta):
+    _check(h, _lib.signmuon_vote_step(h, _ptr(W), _ptr(signs), int(stride), int(M), float(eta)))
+
+
 def signmuon_apply_update(h, W, D, d, eta):
     _check(h, _lib.signmuon_apply_update(h, _ptr(W), _ptr(D), int(d), float(eta)))
 
@@ -301,6 +311,7 @@ class SignMuon:
                  stream=None):
         self.shapes = [(int(r), int(c)) for r, c in shapes]
         self.M = int(M)
+        self.flags = int(flags)
         self.h = signmuon_init(self.shapes, M, beta, lam, K, eps, scale, P, flags, stream)
         self.info = signmuon_info(self.h)
         self.d = self.info["d"]
@@ -325,6 +336,19 @@ class SignMuon:
 
     def get_ternary_signs(self, m, dst):
         signmuon_get_ternary_signs(self.h, m, dst)
+
+    def sign_stride(self):
+        """Bytes per worker in a sign buffer for local_signs / vote_step: the
+        packed bits (or, with SIGNMUON_TERNARY, the int8 signs) rounded up to
+        16."""
+        n = self.d if self.flags & SIGNMUON_TERNARY else (self.d + 7) // 8
+        return (n + 15) // 16 * 16
+
+    def local_signs(self, W, G, signs, stride=None):
+        signmuon_local_signs(self.h, W, G, signs, self.sign_stride() if stride is None else stride)
+
+    def vote_step(self, W, signs, M, eta, stride=None):
+        signmuon_vote_step(self.h, W, signs, self.sign_stride() if stride is None else stride, M, eta)
 
     def apply_update(self, W, D, d, eta):
         signmuon_apply_update(self.h, W, D, d, eta)

@@ -41,6 +41,7 @@ struct signmuon_ctx {
   bool u_valid = true;          // U holds the last step's (or polar call's) polar factors
   bool bits_valid = true;       // bits hold the last step's packed signs
   bool t_valid = false;         // sign8 holds the last step's ternary signs
+  bool dir_valid = false;       // get_direction can give the last step's D
   // device plan tables
   sm::MatInfo* d_mats = nullptr;
   sm::GroupInfo* d_groups = nullptr;
@@ -585,6 +586,83 @@ int signmuon_set_ns_coeffs(signmuon_t h, const float* c, int n) {
   return SIGNMUON_OK;
 }
 
+// The step in two parts, so that the signs can cross a collective in
+// between (one worker per GPU, [paper] Algorithm 2's exchange).
+// local_part: momentum -> scale -> PolarNS -> signs of the handle's M workers,
+// worker m's at dst + m*stride (packed bits, or int8 ternary signs).
+static void local_part(signmuon_t h, const float* W, const sm::WorkerPtrs& gp, uint8_t* dst, int64_t stride) {
+  const Plan& p = h->plan;
+  cudaStream_t s = h->stream;
+  {
+    ProfScope ps(h, 0);
+    sm::launch_momentum(s, gp, W, h->Mom, p.dpad, h->M, h->beta, h->lambda, h->X[0], p.fp32 ? 0 : 1, h->d_chunks,
+                        (int)p.chunks.size(), h->d_mats, h->d_groups, h->partials);
+  }
+  fro_finalize(h, h->M);
+  const bool ternary = (h->flags & SIGNMUON_TERNARY) != 0;
+  int8_t* dst8 = reinterpret_cast<int8_t*>(dst);
+  if (h->flags & SIGNMUON_POLAR_AFTER_ONLY) {
+    // after-only placement: the signs of the momentum itself
+    h->u_valid = false;
+    ProfScope ps(h, 6);
+    if (ternary) sm::launch_sign8(s, h->Mom, p.dpad, p.d, dst8, stride, h->M);
+    else sm::launch_pack(s, h->Mom, p.dpad, p.d, dst, stride, h->M);
+    return;
+  }
+  // The one-bit signs come out of the last Newton-Schulz GEMM itself when
+  // every matrix has a multiple of 32 columns (then each 32-column chunk of an
+  // output row is one aligned word of the bit stream; K > 0, bf16 path); U is
+  // written only when kept for get_polar.
+  const bool fused = !ternary && signs_in_gemm(h);
+  h->u_valid = !fused || (h->flags & SIGNMUON_KEEP_POLAR) != 0;
+  if (fused) {
+    run_ns(h, h->K, h->M, strided_ptrs(h->Mom, p.dpad, h->M), h->u_valid ? h->U : nullptr, p.dpad,
+           reinterpret_cast<uint32_t*>(dst), stride / 4);
+  } else {
+    run_ns(h, h->K, h->M, strided_ptrs(h->Mom, p.dpad, h->M), h->U, p.dpad);
+    ProfScope ps(h, 6);
+    if (ternary) sm::launch_sign8(s, h->U, p.dpad, p.d, dst8, stride, h->M);
+    else sm::launch_pack(s, h->U, p.dpad, p.d, dst, stride, h->M);
+  }
+}
+
+// vote_part: the majority of Mv sign buffers at src + j*stride, then the
+// post-vote step (PolarNS with the handle's K, or with none for the
+// normalised sign step) and the update, or the vote fused with the update.
+static void vote_part(signmuon_t h, float* W, const uint8_t* src, int64_t stride, int Mv, float eta) {
+  const Plan& p = h->plan;
+  cudaStream_t s = h->stream;
+  const int tie = (h->flags & SIGNMUON_TIE_PLUS) ? 1 : 0;
+  const bool ternary = (h->flags & SIGNMUON_TERNARY) != 0;
+  const int8_t* src8 = reinterpret_cast<const int8_t*>(src);
+  if (h->flags & (SIGNMUON_POST_POLAR | SIGNMUON_NORMALIZED_SIGN)) {
+    const int k_post = (h->flags & SIGNMUON_NORMALIZED_SIGN) ? 0 : h->K;
+    {
+      ProfScope ps(h, 7);
+      if (ternary) {
+        // majority -> D, then D staged as the step's input (a one-worker
+        // mean, which is D itself) with its sum-of-squares partials
+        sm::launch_vote_ternary_major(s, src8, stride, Mv, p.d, h->D, tie);
+        sm::launch_mean_stage(s, h->D, 0, 1, h->X[0], p.fp32 ? 0 : 1, h->d_chunks, (int)p.chunks.size(), h->d_mats,
+                              h->d_groups, h->partials, nullptr);
+      } else {
+        // the majority goes straight into the step's input (and into D only
+        // when K == 0, where the result is the scaled input itself)
+        sm::launch_vote_stage(s, src, stride, Mv, h->X[0], p.fp32 ? 0 : 1, h->d_chunks, (int)p.chunks.size(),
+                              h->d_mats, h->d_groups, h->partials, k_post == 0 ? h->D : nullptr, tie);
+      }
+    }
+    fro_finalize(h, 1);
+    run_ns(h, k_post, 1, strided_ptrs(h->D, 0, 1), h->D, 0);
+    ProfScope ps(h, 12);
+    sm::launch_update(s, W, h->D, p.d, eta, h->status);
+  } else {
+    ProfScope ps(h, 7);
+    if (ternary) sm::launch_vote_ternary_update(s, src8, stride, Mv, p.d, W, eta, h->status, tie);
+    else sm::launch_vote_update(s, src, stride, Mv, p.d, W, eta, h->status, tie);
+  }
+}
+
 int signmuon_step(signmuon_t h, float* W, const float* const* G, float eta) {
   int rc = check_handle(h, true);
   if (rc) return rc;
@@ -596,25 +674,24 @@ int signmuon_step(signmuon_t h, float* W, const float* const* G, float eta) {
   cudaStream_t s = h->stream;
   CK(h, cudaMemsetAsync(h->status, 0, 2 * sizeof(int), s));
   const sm::WorkerPtrs gp = worker_ptrs(G, h->M);
-  {
-    ProfScope ps(h, 0);
-    sm::launch_momentum(s, gp, W, h->Mom, p.dpad, h->M, h->beta, h->lambda, h->X[0], p.fp32 ? 0 : 1, h->d_chunks,
-                        (int)p.chunks.size(), h->d_mats, h->d_groups, h->partials);
-  }
-  fro_finalize(h, h->M);
-  const int tie = (h->flags & SIGNMUON_TIE_PLUS) ? 1 : 0;
-  const sm::WorkerPtrs dp = strided_ptrs(h->D, 0, 1);
   if (h->flags & SIGNMUON_MUON_MEAN) {
     // Muon baseline: the workers' mean momentum through one PolarNS
     h->u_valid = false;
     h->bits_valid = false;
+    h->dir_valid = true;
+    {
+      ProfScope ps(h, 0);
+      sm::launch_momentum(s, gp, W, h->Mom, p.dpad, h->M, h->beta, h->lambda, h->X[0], p.fp32 ? 0 : 1, h->d_chunks,
+                          (int)p.chunks.size(), h->d_mats, h->d_groups, h->partials);
+    }
+    fro_finalize(h, h->M);
     {
       ProfScope ps(h, 8);
       sm::launch_mean_stage(s, h->Mom, p.dpad, h->M, h->X[0], p.fp32 ? 0 : 1, h->d_chunks, (int)p.chunks.size(),
                             h->d_mats, h->d_groups, h->partials, h->K == 0 ? h->D : nullptr);
     }
     fro_finalize(h, 1);
-    run_ns(h, h->K, 1, dp, h->D, 0);
+    run_ns(h, h->K, 1, strided_ptrs(h->D, 0, 1), h->D, 0);
     ProfScope ps(h, 12);
     sm::launch_update(s, W, h->D, p.d, eta, h->status);
     return finish(h, (h->flags & SIGNMUON_ASYNC) == 0);
@@ -623,58 +700,50 @@ int signmuon_step(signmuon_t h, float* W, const float* const* G, float eta) {
   const bool ternary = (h->flags & SIGNMUON_TERNARY) != 0;
   h->bits_valid = !ternary;
   h->t_valid = ternary;
-  if (h->flags & SIGNMUON_POLAR_AFTER_ONLY) {
-    // after-only placement: the signs of the momentum itself
-    h->u_valid = false;
-    ProfScope ps(h, 6);
-    if (ternary) sm::launch_sign8(s, h->Mom, p.dpad, p.d, h->sign8, p.dpad, h->M);
-    else sm::launch_pack(s, h->Mom, p.dpad, p.d, h->bits, p.nb_pad, h->M);
-  } else {
-    // The one-bit signs come out of the last Newton-Schulz GEMM itself when
-    // every matrix has a multiple of 32 columns (then each 32-column chunk of
-    // an output row is one aligned word of the bit stream; K > 0, bf16 path);
-    // U is written only when kept for get_polar.
-    const bool fused = !ternary && signs_in_gemm(h);
-    h->u_valid = !fused || (h->flags & SIGNMUON_KEEP_POLAR) != 0;
-    if (fused) {
-      run_ns(h, h->K, h->M, strided_ptrs(h->Mom, p.dpad, h->M), h->u_valid ? h->U : nullptr, p.dpad,
-             reinterpret_cast<uint32_t*>(h->bits), p.nb_pad / 4);
-    } else {
-      run_ns(h, h->K, h->M, strided_ptrs(h->Mom, p.dpad, h->M), h->U, p.dpad);
-      ProfScope ps(h, 6);
-      if (ternary) sm::launch_sign8(s, h->U, p.dpad, p.d, h->sign8, p.dpad, h->M);
-      else sm::launch_pack(s, h->U, p.dpad, p.d, h->bits, p.nb_pad, h->M);
-    }
-  }
-  if (h->flags & (SIGNMUON_POST_POLAR | SIGNMUON_NORMALIZED_SIGN)) {
-    // post-vote step on the majority matrix: PolarNS with the handle's K, or
-    // (normalised sign step) with none, which leaves majority / (s + eps)
-    const int k_post = (h->flags & SIGNMUON_NORMALIZED_SIGN) ? 0 : h->K;
-    {
-      ProfScope ps(h, 7);
-      if (ternary) {
-        // majority -> D, then D staged as the step's input (a one-worker
-        // mean, which is D itself) with its sum-of-squares partials
-        sm::launch_vote_ternary_major(s, h->sign8, p.dpad, h->M, p.d, h->D, tie);
-        sm::launch_mean_stage(s, h->D, 0, 1, h->X[0], p.fp32 ? 0 : 1, h->d_chunks, (int)p.chunks.size(), h->d_mats,
-                              h->d_groups, h->partials, nullptr);
-      } else {
-        // the majority goes straight into the step's input (and into D only
-        // when K == 0, where the result is the scaled input itself)
-        sm::launch_vote_stage(s, h->bits, p.nb_pad, h->M, h->X[0], p.fp32 ? 0 : 1, h->d_chunks,
-                              (int)p.chunks.size(), h->d_mats, h->d_groups, h->partials,
-                              k_post == 0 ? h->D : nullptr, tie);
-      }
-    }
-    fro_finalize(h, 1);
-    run_ns(h, k_post, 1, dp, h->D, 0);
-    ProfScope ps(h, 12);
-    sm::launch_update(s, W, h->D, p.d, eta, h->status);
-  } else {
-    ProfScope ps(h, 7);
-    if (ternary) sm::launch_vote_ternary_update(s, h->sign8, p.dpad, h->M, p.d, W, eta, h->status, tie);
-    else sm::launch_vote_update(s, h->bits, p.nb_pad, h->M, p.d, W, eta, h->status, tie);
-  }
+  h->dir_valid = true;
+  uint8_t* own = ternary ? reinterpret_cast<uint8_t*>(h->sign8) : h->bits;
+  const int64_t own_stride = ternary ? p.dpad : p.nb_pad;
+  local_part(h, W, gp, own, own_stride);
+  vote_part(h, W, own, own_stride, h->M, eta);
+  return finish(h, (h->flags & SIGNMUON_ASYNC) == 0);
+}
+
+int signmuon_local_signs(signmuon_t h, const float* W, const float* const* G, uint8_t* signs, int64_t stride) {
+  int rc = check_handle(h, true);
+  if (rc) return rc;
+  const Plan& p = h->plan;
+  if (h->flags & SIGNMUON_MUON_MEAN) return fail(h, SIGNMUON_E_UNSUPPORTED, "a SIGNMUON_MUON_MEAN handle sends no signs");
+  if (W == nullptr || G == nullptr || signs == nullptr) return fail(h, SIGNMUON_E_INVALID, "null W, G or signs");
+  if (!aligned16(W) || !aligned16(signs)) return fail(h, SIGNMUON_E_INVALID, "W and signs must be 16-byte aligned");
+  for (int m = 0; m < h->M; ++m)
+    if (G[m] == nullptr || !aligned16(G[m])) return fail(h, SIGNMUON_E_INVALID, "G[m] null or not 16-byte aligned");
+  const int64_t need = (h->flags & SIGNMUON_TERNARY) ? p.d : p.nb;
+  if (stride < need || stride % 16 != 0)
+    return fail(h, SIGNMUON_E_INVALID, "stride must be a multiple of 16 bytes and hold one worker's signs");
+  CK(h, cudaMemsetAsync(h->status, 0, 2 * sizeof(int), h->stream));
+  // the handle's own sign buffers do not hold these signs
+  h->bits_valid = false;
+  h->t_valid = false;
+  h->dir_valid = false;
+  local_part(h, W, worker_ptrs(G, h->M), signs, stride);
+  return finish(h, (h->flags & SIGNMUON_ASYNC) == 0);
+}
+
+int signmuon_vote_step(signmuon_t h, float* W, const uint8_t* signs, int64_t stride, int M, float eta) {
+  const bool post = h != nullptr && (h->flags & (SIGNMUON_POST_POLAR | SIGNMUON_NORMALIZED_SIGN)) != 0;
+  int rc = check_handle(h, post);
+  if (rc) return rc;
+  const Plan& p = h->plan;
+  if (h->flags & SIGNMUON_MUON_MEAN) return fail(h, SIGNMUON_E_UNSUPPORTED, "a SIGNMUON_MUON_MEAN handle takes no vote");
+  if (M < 1 || M > sm::kMaxWorkers) return fail(h, SIGNMUON_E_INVALID, "M must be in [1, 256]");
+  if (W == nullptr || signs == nullptr) return fail(h, SIGNMUON_E_INVALID, "null W or signs");
+  if (!aligned16(W) || !aligned16(signs)) return fail(h, SIGNMUON_E_INVALID, "W and signs must be 16-byte aligned");
+  const int64_t need = (h->flags & SIGNMUON_TERNARY) ? p.d : p.nb;
+  if (stride < need || stride % 16 != 0)
+    return fail(h, SIGNMUON_E_INVALID, "stride must be a multiple of 16 bytes and hold one worker's signs");
+  CK(h, cudaMemsetAsync(h->status, 0, 2 * sizeof(int), h->stream));
+  h->dir_valid = post;  // D is kept only by the post-vote steps
+  vote_part(h, W, signs, stride, M, eta);
   return finish(h, (h->flags & SIGNMUON_ASYNC) == 0);
 }
 
@@ -834,8 +903,10 @@ int signmuon_get_signs(signmuon_t h, int m, uint8_t* dst) {
   if (m < 0 || m >= h->M || !dst) return fail(h, SIGNMUON_E_INVALID, "bad worker index or null dst");
   if (!h->bits_valid)
     return fail(h, SIGNMUON_E_UNSUPPORTED,
-                (h->flags & SIGNMUON_TERNARY) ? "a SIGNMUON_TERNARY step sends int8 signs: use signmuon_get_ternary_signs"
-                                              : "a SIGNMUON_MUON_MEAN step packs no signs");
+                (h->flags & SIGNMUON_TERNARY)     ? "a SIGNMUON_TERNARY step sends int8 signs: use signmuon_get_ternary_signs"
+                : (h->flags & SIGNMUON_MUON_MEAN) ? "a SIGNMUON_MUON_MEAN step packs no signs"
+                                                  : "no step has left its signs in the handle (signmuon_local_signs "
+                                                    "writes them to the caller's buffer)");
   CK(h, cudaMemcpyAsync(dst, h->bits + (int64_t)m * h->plan.nb_pad, (size_t)h->plan.nb, cudaMemcpyDeviceToDevice,
                         h->stream));
   return SIGNMUON_OK;
@@ -845,7 +916,8 @@ int signmuon_get_ternary_signs(signmuon_t h, int m, int8_t* dst) {
   int rc = check_handle(h, true);
   if (rc) return rc;
   if (m < 0 || m >= h->M || !dst) return fail(h, SIGNMUON_E_INVALID, "bad worker index or null dst");
-  if (!h->t_valid) return fail(h, SIGNMUON_E_UNSUPPORTED, "no SIGNMUON_TERNARY step has run on this handle");
+  if (!h->t_valid)
+    return fail(h, SIGNMUON_E_UNSUPPORTED, "no SIGNMUON_TERNARY step has left its signs in the handle");
   CK(h, cudaMemcpyAsync(dst, h->sign8 + (int64_t)m * h->plan.dpad, (size_t)h->plan.d, cudaMemcpyDeviceToDevice,
                         h->stream));
   return SIGNMUON_OK;
@@ -856,6 +928,9 @@ int signmuon_get_direction(signmuon_t h, float* dst) {
   if (rc) return rc;
   if (!dst || !aligned16(dst)) return fail(h, SIGNMUON_E_INVALID, "null or misaligned dst");
   const Plan& p = h->plan;
+  if (!h->dir_valid)
+    return fail(h, SIGNMUON_E_UNSUPPORTED,
+                "no D to give: no step yet, or the last vote (signmuon_vote_step) was fused with the update");
   if (h->flags & (SIGNMUON_POST_POLAR | SIGNMUON_MUON_MEAN | SIGNMUON_NORMALIZED_SIGN)) {
     CK(h, cudaMemcpyAsync(dst, h->D, (size_t)p.d * 4, cudaMemcpyDeviceToDevice, h->stream));
   } else if (h->flags & SIGNMUON_TERNARY) {

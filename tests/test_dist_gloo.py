@@ -1,0 +1,143 @@
+"""The multi-GPU driver's exchange (sign_muon_optimizer_b200.dist) on the CPU:
+world size 2 over gloo, with a stand-in for the library's two halves of the
+step (the signs are the one-bit signs of the gradients themselves, and the
+vote follows the oracle).  It checks what the driver itself adds: the
+rank-major worker order of the all-gather, identical W on every rank (and
+the replica check), and that a failure on one rank makes every rank raise
+without updating W and without hanging in a collective."""
+import datetime
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+import synth
+from oracle import signmuon_ref as ref
+
+SHAPES = [(6, 10), (9, 5)]
+M_LOCAL = 2
+
+
+class _StandIn:
+    """local_signs / vote_step / sign_stride with the library's layout."""
+
+    def __init__(self, fail=False):
+        self.d = synth.numel(SHAPES)
+        self.nb = ref.packed_nbytes(self.d)
+        self.fail = fail
+        self.seen = None
+
+    def sign_stride(self):
+        return (self.nb + 15) // 16 * 16
+
+    def local_signs(self, W, G, out, stride):
+        import sign_muon_optimizer_b200 as smo
+        if self.fail:
+            raise smo.SignMuonError(smo.SIGNMUON_E_NONFINITE, "planted failure")
+        for m, g in enumerate(G):
+            out[m * stride: m * stride + self.nb] = torch.from_numpy(ref.pack_bits(ref.sign_bits(g.numpy())))
+
+    def vote_step(self, W, signs, M, eta, stride):
+        self.seen = signs.clone()
+        packed = [signs[j * stride: j * stride + self.nb].numpy() for j in range(M)]
+        maj = ref.majority(ref.vote_sums_from_bits(packed, self.d))
+        W.copy_(torch.from_numpy(ref.update(W.numpy(), maj.astype(np.float32), eta)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank(rank, world, port, fail_rank, q):
+    import torch.distributed as dist
+
+    from sign_muon_optimizer_b200.dist import DistSignMuon
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        opt = _StandIn(fail=(rank == fail_rank))
+        drv = DistSignMuon(SHAPES, M_local=M_LOCAL, opt=opt, device="cpu")
+        W = torch.from_numpy(synth.weights0(SHAPES, 5))
+        G = synth.gradients(SHAPES, world * M_LOCAL, 1.0, step=1, config_id=5)
+        mine = [torch.from_numpy(g) for g in G[rank * M_LOCAL:(rank + 1) * M_LOCAL]]
+        raised = False
+        try:
+            drv.step(W, mine, 0.02)
+        except Exception as e:  # noqa: BLE001
+            raised = type(e).__name__
+        agree = drv.replicas_agree(W)
+        q.put((rank, W.numpy().copy(), None if opt.seen is None else opt.seen.numpy(), raised, agree,
+               drv.payload_bytes))
+    finally:
+        dist.destroy_process_group()
+
+
+def _run(fail_rank):
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank, args=(r, world, port, fail_rank, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    out = {}
+    for _ in range(world):
+        r, W, seen, raised, agree, payload = q.get(timeout=120)
+        out[r] = dict(W=W, seen=seen, raised=raised, agree=agree, payload=payload)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    return out
+
+
+def test_exchange_gathers_in_rank_order_and_replicas_agree():
+    out = _run(fail_rank=-1)
+    world = 2
+    M = world * M_LOCAL
+    G = synth.gradients(SHAPES, M, 1.0, step=1, config_id=5)
+    d = synth.numel(SHAPES)
+    nb = ref.packed_nbytes(d)
+    stride = (nb + 15) // 16 * 16
+    packed = [ref.pack_bits(ref.sign_bits(g)) for g in G]
+    w0 = synth.weights0(SHAPES, 5)
+    want = ref.update(w0, ref.majority(ref.vote_sums_from_bits(packed, d)).astype(np.float32), 0.02)
+    for r in range(world):
+        assert out[r]["raised"] is False
+        assert out[r]["agree"] is True
+        assert out[r]["payload"] == M_LOCAL * stride
+        assert np.array_equal(out[r]["W"].view(np.uint32), want.view(np.uint32))
+        for j in range(M):  # global worker j sits at slot j on every rank
+            assert np.array_equal(out[r]["seen"][j * stride: j * stride + nb], packed[j])
+
+
+def test_one_failing_rank_stops_every_rank_without_update():
+    out = _run(fail_rank=1)
+    w0 = synth.weights0(SHAPES, 5)
+    for r in range(2):
+        assert out[r]["raised"] == "SignMuonError"
+        assert out[r]["seen"] is None           # nobody voted
+        assert np.array_equal(out[r]["W"], w0)  # nobody updated
+        assert out[r]["agree"] is True
+
+
+def test_too_many_workers_is_rejected():
+    # 2 ranks x 200 workers exceed the vote's 256: checked before any collective
+    import torch.distributed as dist
+
+    from sign_muon_optimizer_b200.dist import DistSignMuon
+    port = _free_port()
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    store = dist.TCPStore("127.0.0.1", port, 1, True)
+    dist.init_process_group("gloo", store=store, rank=0, world_size=1)
+    try:
+        with pytest.raises(ValueError):
+            DistSignMuon(SHAPES, M_local=257, opt=_StandIn(), device="cpu")
+    finally:
+        dist.destroy_process_group()
