@@ -409,7 +409,8 @@ def _events_time(fn, reps, stream):
 
 def run_secondary(args):
     """Secondary measurements (not the headline line): the LLaMA-layer vote
-    (vote GB/s), the Newton-Schulz sweep (NS TFLOP/s) and the ResNet-50 step
+    (vote GB/s, one-bit and int8 ternary signs), the Newton-Schulz sweep (NS
+    TFLOP/s), the ResNet-50 step and the named variants of the nanoGPT step
     (steps/s), one JSON line each."""
     import torch
     import sign_muon_optimizer_b200 as smo
@@ -462,6 +463,58 @@ def run_secondary(args):
             h.close()
             del X, U
             torch.cuda.empty_cache()
+    if args.workload in ("ternary_vote", "all"):
+        # the int8 ternary wire's vote: d bytes per worker instead of d/8
+        shapes = synth.LLAMA_LAYER_SHAPES
+        Mv = synth.WORKLOADS["llama_vote"]["M"]
+        d = synth.numel(shapes)
+        g = torch.Generator(device="cuda")
+        g.manual_seed(6)
+        signs = [torch.randint(-1, 2, (d + 16,), generator=g, device="cuda", dtype=torch.int8) for _ in range(Mv)]
+        h = smo.SignMuon(shapes, Mv, flags=smo.SIGNMUON_VOTE_ONLY, stream=stream.cuda_stream)
+        sums = torch.empty(d, device="cuda", dtype=torch.int32)
+        maj = torch.empty(d, device="cuda", dtype=torch.int8)
+        ms = _events_time(lambda: h.vote_ternary(signs, d, sums, maj), 5, stream)
+        nbytes = Mv * d + 4.0 * d + d
+        gbs = nbytes / (ms / 1e3) / 1e9
+        lines.append({"metric": "ternary vote GB/s (LLaMA-layer shapes, M=16, int8 signs, int32 sums)", "value": gbs,
+                      "unit": "GB/s", "frac_of_hbm": gbs / pk["hbm_gbs"], "peak_kind": pk_kind, "ms": ms,
+                      "bytes": nbytes, "d": d, "M": Mv, "payload_bytes_per_worker": d, "acc_dtype": "int32",
+                      "collective": "none (on-device vote)"})
+        h.close()
+        del signs, sums, maj
+        torch.cuda.empty_cache()
+    if args.workload in ("variants", "all"):
+        # the named variants on the headline shapes (nanoGPT, M=8, K=5), one
+        # step each; split = local signs + vote step through a caller buffer
+        base = smo.SIGNMUON_POST_POLAR if WL["post_polar"] else 0
+        variants = [("sign-muon", base, WL["P"]), ("tie_plus", base | smo.SIGNMUON_TIE_PLUS, WL["P"]),
+                    ("ternary", base | smo.SIGNMUON_TERNARY, WL["P"]),
+                    ("normalized_sign", smo.SIGNMUON_NORMALIZED_SIGN, WL["P"]),
+                    ("after_only", smo.SIGNMUON_POST_POLAR | smo.SIGNMUON_POLAR_AFTER_ONLY, WL["P"]),
+                    ("muon_mean", smo.SIGNMUON_MUON_MEAN, WL["P"]),
+                    ("pi_warm_P1", base | smo.SIGNMUON_PI_WARM, 1), ("cold_P1", base, 1), ("split", base, WL["P"])]
+        W = synth.device_weights0(SHAPES, config_id=7)
+        G = synth.device_gradients(SHAPES, M, WL["sigma"], step=0, config_id=7)
+        gl = [G[m] for m in range(M)]
+        for name, flags, P in variants:
+            h = smo.SignMuon(SHAPES, M, beta=HP["beta"], lam=HP["lam"], K=K_NS, eps=HP["eps"], scale=WL["scale"],
+                             P=P, flags=flags, stream=stream.cuda_stream)
+            if name == "split":
+                buf = torch.empty(M * h.sign_stride(), dtype=torch.uint8, device="cuda")
+
+                def one():
+                    h.local_signs(W, gl, buf)
+                    h.vote_step(W, buf, M, HP["eta"])
+            else:
+                def one():
+                    h.step(W, gl, HP["eta"])
+            ms = _events_time(one, 10, stream)
+            lines.append({"metric": f"Sign-Muon steps/s (nanoGPT-124M shapes, M=8, variant {name})",
+                          "value": 1e3 / ms, "unit": "steps/s", "ms_per_step": ms, "flags": flags, "P": P})
+            h.close()
+        del W, G, gl
+        torch.cuda.empty_cache()
     if args.workload in ("resnet50", "all"):
         wl = synth.WORKLOADS["resnet50"]
         shp, Mr = wl["shapes"], wl["M"]
@@ -509,7 +562,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--capture-layers", type=int, default=0,
                     help="profiler capture mode on the first L layers; prints no bench line")
-    ap.add_argument("--workload", default="nanogpt", choices=["nanogpt", "llama_vote", "vote_100m", "ns_sweep", "resnet50", "all"],
+    ap.add_argument("--workload", default="nanogpt",
+                    choices=["nanogpt", "llama_vote", "vote_100m", "ns_sweep", "resnet50", "ternary_vote", "variants",
+                             "all"],
                     help="nanogpt: the headline line; the others print secondary measurements only")
     args = ap.parse_args()
     if args.capture_layers > 0:
