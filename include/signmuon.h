@@ -167,6 +167,21 @@ int signmuon_vote_step(signmuon_t h, float* W, const uint8_t* signs, int64_t str
                        float eta);
 
 /* ------------------------------------------------------------------------
+ * signmuon_sums_step -- the second half of the step when the vote sums arrive
+ * already added up: [paper] Algorithm 2's integer SUM all-reduce of the
+ * workers' signs (each GPU sums its own workers with signmuon_vote or
+ * signmuon_vote_ternary, an all-reduce adds the GPUs' sums).  majority =
+ * sign(sums) with the handle's tie rule, then the post-vote step the flags
+ * ask for and W <- fl32(W - eta*D).
+ *   W     device float[d].
+ *   sums  device int32[d], or int8[d] with SIGNMUON_ACC_INT8 (then at most 127
+ *         workers in all, so that no partial or total sum overflows); 16-byte
+ *         aligned.
+ * Waits like signmuon_step; signmuon_get_direction then gives D.
+ * ---------------------------------------------------------------------- */
+int signmuon_sums_step(signmuon_t h, float* W, const void* sums, float eta);
+
+/* ------------------------------------------------------------------------
  * signmuon_step_host -- signmuon_step on HOST buffers: copies W and the M
  * gradients to library-owned device buffers (allocated on first use),
  * runs the step and copies W back.  Always waits.  Pinned host memory gives

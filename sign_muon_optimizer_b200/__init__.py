@@ -51,7 +51,7 @@ EXPORTED = [
     "signmuon_kernel_launches", "signmuon_last_error", "signmuon_status_string", "signmuon_destroy",
     "signmuon_profile", "signmuon_profile_read", "signmuon_get_gram",
     "signmuon_spectral_norm_noalloc", "signmuon_sign_ternary", "signmuon_vote_ternary",
-    "signmuon_get_ternary_signs", "signmuon_local_signs", "signmuon_vote_step",
+    "signmuon_get_ternary_signs", "signmuon_local_signs", "signmuon_vote_step", "signmuon_sums_step",
 ]
 PROF_KINDS = ["momentum", "norm_finalize", "ns_gram", "ns_square", "ns_apply", "power_iter", "pack",
               "vote", "stage", "post_gram", "post_square", "post_apply", "update", "k0_scale"]
@@ -80,6 +80,7 @@ def _load():
         "signmuon_get_ternary_signs": (I, [P, I, P]),
         "signmuon_local_signs": (I, [P, P, PP, P, I64]),
         "signmuon_vote_step": (I, [P, P, P, I64, I, F]),
+        "signmuon_sums_step": (I, [P, P, P, F]),
         "signmuon_apply_update": (I, [P, P, P, I64, F]),
         "signmuon_polar": (I, [P, PP, PP]),
         "signmuon_get_momentum": (I, [P, I, P]),
@@ -200,6 +201,10 @@ def signmuon_local_signs(h, W, G, signs, stride):
 
 def signmuon_vote_step(h, W, signs, stride, M, eta):
     _check(h, _lib.signmuon_vote_step(h, _ptr(W), _ptr(signs), int(stride), int(M), float(eta)))
+
+
+def signmuon_sums_step(h, W, sums, eta):
+    _check(h, _lib.signmuon_sums_step(h, _ptr(W), _ptr(sums), float(eta)))
 
 
 def signmuon_apply_update(h, W, D, d, eta):
@@ -349,6 +354,9 @@ class SignMuon:
 
     def vote_step(self, W, signs, M, eta, stride=None):
         signmuon_vote_step(self.h, W, signs, self.sign_stride() if stride is None else stride, M, eta)
+
+    def sums_step(self, W, sums, eta):
+        signmuon_sums_step(self.h, W, sums, eta)
 
     def apply_update(self, W, D, d, eta):
         signmuon_apply_update(self.h, W, D, d, eta)

@@ -169,6 +169,8 @@ void launch_vote_ternary_update(cudaStream_t s, const int8_t* signs, int64_t str
                                 float eta, const int* status, int tie_plus);
 void launch_vote_ternary_major(cudaStream_t s, const int8_t* signs, int64_t stride, int M, int64_t d, float* D,
                                int tie_plus);
+// D = majority of int32 (or int8, acc8) vote sums
+void launch_sums_major(cudaStream_t s, const void* sums, int acc8, int64_t d, float* D, int tie_plus);
 
 void launch_gemm_simt(cudaStream_t s, const GemmArgs& a, int x_f32);
 int gemm_tc_smem_bytes();

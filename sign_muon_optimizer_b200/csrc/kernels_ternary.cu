@@ -1,6 +1,8 @@
 // kernels_ternary.cu -- the int8 ternary sign wire: sign(U) in {-1, 0, +1},
 // one byte per entry and worker, and the majority vote over M such buffers
-// (API form with int32 or int8 sums, fused with the update, or emitting D).
+// (API form with int32 or int8 sums, fused with the update, or emitting D);
+// and the majority of integer vote sums that arrive already added up (the
+// SUM all-reduce of the workers' signs).
 //
 // Sources, by page title:
 //   [paper] "SignMuon: 通信高效的分布式Muon优化" (a rendering of arXiv 2605.16311):
@@ -179,6 +181,33 @@ void vote_tern(cudaStream_t s, const WorkerPtrs& signs, int M, int64_t d, void* 
   k_vote_tern<MODE, ACC8><<<blocks, kTThreads, 0, s>>>(signs, M, d, sums, maj, W, eta, D, status, tie_plus);
 }
 
+// D = majority of integer vote sums (int32, or int8 when ACC8): four entries
+// per thread and step (one 16- or 4-byte load, one float4 store), the d % 4
+// tail entry by entry in the last block.  Host-checked: sums 16-byte aligned.
+template <bool ACC8>
+__global__ void __launch_bounds__(kTThreads)
+k_sums_major(const void* __restrict__ sums, int64_t d, float* __restrict__ D, int tie_plus) {
+  const int64_t n4 = d >> 2;
+  const int64_t stride = (int64_t)gridDim.x * kTThreads;
+  for (int64_t i = (int64_t)blockIdx.x * kTThreads + threadIdx.x; i < n4; i += stride) {
+    int s0, s1, s2, s3;
+    if (ACC8) {
+      const char4 v = reinterpret_cast<const char4*>(sums)[i];
+      s0 = v.x; s1 = v.y; s2 = v.z; s3 = v.w;
+    } else {
+      const int4 v = reinterpret_cast<const int4*>(sums)[i];
+      s0 = v.x; s1 = v.y; s2 = v.z; s3 = v.w;
+    }
+    reinterpret_cast<float4*>(D)[i] = make_float4((float)tmaj(s0, tie_plus), (float)tmaj(s1, tie_plus),
+                                                  (float)tmaj(s2, tie_plus), (float)tmaj(s3, tie_plus));
+  }
+  if (blockIdx.x == gridDim.x - 1)
+    for (int64_t e = 4 * n4 + threadIdx.x; e < d; e += kTThreads) {
+      const int sv = ACC8 ? (int)reinterpret_cast<const int8_t*>(sums)[e] : reinterpret_cast<const int32_t*>(sums)[e];
+      D[e] = (float)tmaj(sv, tie_plus);
+    }
+}
+
 WorkerPtrs strided_bytes(const int8_t* base, int64_t stride, int M) {
   WorkerPtrs w{};
   for (int m = 0; m < M; ++m) w.p[m] = reinterpret_cast<const float*>(base + (int64_t)m * stride);
@@ -217,6 +246,14 @@ void launch_vote_ternary_major(cudaStream_t s, const int8_t* signs, int64_t stri
   if (d <= 0) return;
   vote_tern<2, false>(s, strided_bytes(signs, stride, M), M, d, nullptr, nullptr, nullptr, 0.f, D, nullptr,
                       tie_plus);
+}
+
+void launch_sums_major(cudaStream_t s, const void* sums, int acc8, int64_t d, float* D, int tie_plus) {
+  if (d <= 0) return;
+  count_launch();
+  const int blocks = stream_grid(((d >> 2) + kTThreads - 1) / kTThreads, 8);
+  if (acc8) k_sums_major<true><<<blocks, kTThreads, 0, s>>>(sums, d, D, tie_plus);
+  else k_sums_major<false><<<blocks, kTThreads, 0, s>>>(sums, d, D, tie_plus);
 }
 
 }  // namespace sm

@@ -42,6 +42,7 @@ struct signmuon_ctx {
   bool bits_valid = true;       // bits hold the last step's packed signs
   bool t_valid = false;         // sign8 holds the last step's ternary signs
   bool dir_valid = false;       // get_direction can give the last step's D
+  bool dir_in_D = false;        // ... and it is in D (else: the majority of the handle's own signs)
   // device plan tables
   sm::MatInfo* d_mats = nullptr;
   sm::GroupInfo* d_groups = nullptr;
@@ -679,6 +680,7 @@ int signmuon_step(signmuon_t h, float* W, const float* const* G, float eta) {
     h->u_valid = false;
     h->bits_valid = false;
     h->dir_valid = true;
+    h->dir_in_D = true;
     {
       ProfScope ps(h, 0);
       sm::launch_momentum(s, gp, W, h->Mom, p.dpad, h->M, h->beta, h->lambda, h->X[0], p.fp32 ? 0 : 1, h->d_chunks,
@@ -701,6 +703,7 @@ int signmuon_step(signmuon_t h, float* W, const float* const* G, float eta) {
   h->bits_valid = !ternary;
   h->t_valid = ternary;
   h->dir_valid = true;
+  h->dir_in_D = (h->flags & (SIGNMUON_POST_POLAR | SIGNMUON_NORMALIZED_SIGN)) != 0;
   uint8_t* own = ternary ? reinterpret_cast<uint8_t*>(h->sign8) : h->bits;
   const int64_t own_stride = ternary ? p.dpad : p.nb_pad;
   local_part(h, W, gp, own, own_stride);
@@ -743,7 +746,43 @@ int signmuon_vote_step(signmuon_t h, float* W, const uint8_t* signs, int64_t str
     return fail(h, SIGNMUON_E_INVALID, "stride must be a multiple of 16 bytes and hold one worker's signs");
   CK(h, cudaMemsetAsync(h->status, 0, 2 * sizeof(int), h->stream));
   h->dir_valid = post;  // D is kept only by the post-vote steps
+  h->dir_in_D = post;
   vote_part(h, W, signs, stride, M, eta);
+  return finish(h, (h->flags & SIGNMUON_ASYNC) == 0);
+}
+
+int signmuon_sums_step(signmuon_t h, float* W, const void* sums, float eta) {
+  int rc = check_handle(h, true);
+  if (rc) return rc;
+  const Plan& p = h->plan;
+  if (h->flags & SIGNMUON_MUON_MEAN) return fail(h, SIGNMUON_E_UNSUPPORTED, "a SIGNMUON_MUON_MEAN handle takes no vote");
+  if (W == nullptr || sums == nullptr) return fail(h, SIGNMUON_E_INVALID, "null W or sums");
+  if (!aligned16(W) || !aligned16(sums)) return fail(h, SIGNMUON_E_INVALID, "W and sums must be 16-byte aligned");
+  cudaStream_t s = h->stream;
+  CK(h, cudaMemsetAsync(h->status, 0, 2 * sizeof(int), s));
+  const int tie = (h->flags & SIGNMUON_TIE_PLUS) ? 1 : 0;
+  {
+    // the majority into D; for the post-vote steps D is then staged as
+    // their input (a one-worker mean, which is D itself)
+    ProfScope ps(h, 7);
+    sm::launch_sums_major(s, sums, (h->flags & SIGNMUON_ACC_INT8) ? 1 : 0, p.d, h->D, tie);
+  }
+  if (h->flags & (SIGNMUON_POST_POLAR | SIGNMUON_NORMALIZED_SIGN)) {
+    const int k_post = (h->flags & SIGNMUON_NORMALIZED_SIGN) ? 0 : h->K;
+    {
+      ProfScope ps(h, 7);
+      sm::launch_mean_stage(s, h->D, 0, 1, h->X[0], p.fp32 ? 0 : 1, h->d_chunks, (int)p.chunks.size(), h->d_mats,
+                            h->d_groups, h->partials, nullptr);
+    }
+    fro_finalize(h, 1);
+    run_ns(h, k_post, 1, strided_ptrs(h->D, 0, 1), h->D, 0);
+  }
+  {
+    ProfScope ps(h, 12);
+    sm::launch_update(s, W, h->D, p.d, eta, h->status);
+  }
+  h->dir_valid = true;
+  h->dir_in_D = true;
   return finish(h, (h->flags & SIGNMUON_ASYNC) == 0);
 }
 
@@ -931,7 +970,7 @@ int signmuon_get_direction(signmuon_t h, float* dst) {
   if (!h->dir_valid)
     return fail(h, SIGNMUON_E_UNSUPPORTED,
                 "no D to give: no step yet, or the last vote (signmuon_vote_step) was fused with the update");
-  if (h->flags & (SIGNMUON_POST_POLAR | SIGNMUON_MUON_MEAN | SIGNMUON_NORMALIZED_SIGN)) {
+  if (h->dir_in_D) {
     CK(h, cudaMemcpyAsync(dst, h->D, (size_t)p.d * 4, cudaMemcpyDeviceToDevice, h->stream));
   } else if (h->flags & SIGNMUON_TERNARY) {
     // the step fuses the vote into the update; recompute the majority from

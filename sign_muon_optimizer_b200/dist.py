@@ -7,19 +7,28 @@ every worker takes the majority and updates its own copy of W.  [blog]
 the payload: ceil(d/8) bytes per worker for the packed bits, gathered from all
 ranks (an all-gather; every rank then votes locally).
 
+Two exchanges are offered:
+- "allgather": every rank gathers all workers' packed (or int8 ternary) signs
+  and votes over them.  The payload is M_local * ceil(d/8) bytes per rank.
+- "allreduce": each rank adds up its own workers' signs, and an integer SUM
+  all-reduce adds the ranks' sums (Algorithm 2's form).  The payload is d
+  bytes per rank with int8 sums (SIGNMUON_ACC_INT8, at most 127 workers in
+  all), or 4d with int32 sums.
+
 This module is plumbing only.  The arithmetic runs in libsignmuon.so:
-signmuon_local_signs before the exchange, and signmuon_vote_step after it.
-torch.distributed moves the bytes: one all-gather of the packed (or int8
-ternary) signs, plus one all-reduce of a status flag.  The flag lets every
-rank take the same collective path when one rank's momentum turns
-non-finite.  Ranks must call step() in lockstep, with the same shapes and flags.
+signmuon_local_signs before the exchange; after it, signmuon_vote_step, or
+signmuon_vote / signmuon_vote_ternary then signmuon_sums_step.
+torch.distributed moves the bytes, plus one all-reduce of a status flag.
+The flag lets every rank take the same collective path when one rank's
+momentum turns non-finite.  Ranks must call step() in lockstep, with the
+same shapes, flags and exchange.
 """
 from __future__ import annotations
 
 import torch
 import torch.distributed as dist
 
-from . import SIGNMUON_E_NONFINITE, SignMuon, SignMuonError
+from . import SIGNMUON_ACC_INT8, SIGNMUON_E_NONFINITE, SIGNMUON_TERNARY, SignMuon, SignMuonError
 
 
 class DistSignMuon:
@@ -28,12 +37,17 @@ class DistSignMuon:
     ``step(W, G, eta)`` takes this rank's replica of W (device float[d]) and
     its M_local gradients, and leaves W equal on every rank.  The global
     worker order is rank-major: rank r holds workers r*M_local ...
-    (r+1)*M_local - 1.  ``opt`` may be given to reuse an existing handle, or
-    any object with the same local_signs / vote_step / sign_stride methods.
+    (r+1)*M_local - 1.  ``exchange`` is "allgather" or "allreduce" (see the
+    module text).  ``opt`` may be given to reuse an existing handle, or any
+    object with the same methods (local_signs, vote_step, vote, vote_ternary,
+    sums_step, sign_stride) and attributes (d, flags).
     """
 
     def __init__(self, shapes, M_local=1, beta=0.9, lam=0.01, K=5, eps=1e-7, scale="fro", P=1, flags=0,
-                 group=None, device=None, opt=None):
+                 group=None, device=None, opt=None, exchange="allgather"):
+        if exchange not in ("allgather", "allreduce"):
+            raise ValueError(f"unknown exchange {exchange!r}")
+        self.exchange = exchange
         self.group = group
         self.world = dist.get_world_size(group)
         self.rank = dist.get_rank(group)
@@ -47,13 +61,24 @@ class DistSignMuon:
             device = torch.device("cuda", torch.cuda.current_device()) if torch.cuda.is_available() else "cpu"
         self.device = torch.device(device)
         self.local = torch.zeros(self.M_local * self.stride, dtype=torch.uint8, device=self.device)
-        self.gathered = torch.zeros(self.M * self.stride, dtype=torch.uint8, device=self.device)
         self._flag = torch.zeros(1, dtype=torch.int32, device=self.device)
+        flags = int(getattr(self.opt, "flags", flags))
+        self.ternary = bool(flags & SIGNMUON_TERNARY)
+        if exchange == "allgather":
+            self.gathered = torch.zeros(self.M * self.stride, dtype=torch.uint8, device=self.device)
+        else:
+            acc8 = bool(flags & SIGNMUON_ACC_INT8)
+            if acc8 and self.M > 127:
+                raise ValueError(f"int8 sums overflow for {self.M} workers (at most 127)")
+            self.sums = torch.zeros(int(self.opt.d), dtype=torch.int8 if acc8 else torch.int32, device=self.device)
+            self.views = [self.local[m * self.stride:] for m in range(self.M_local)]
 
     @property
     def payload_bytes(self):
-        """Bytes each rank contributes to the all-gather per step."""
-        return self.local.numel()
+        """Bytes each rank contributes to the exchange per step."""
+        if self.exchange == "allgather":
+            return self.local.numel()
+        return self.sums.numel() * self.sums.element_size()
 
     def step(self, W, G, eta):
         err = None
@@ -69,8 +94,17 @@ class DistSignMuon:
             if err is not None:
                 raise err
             raise SignMuonError(SIGNMUON_E_NONFINITE, "another rank's step failed; W was not updated")
-        dist.all_gather_into_tensor(self.gathered, self.local, group=self.group)
-        self.opt.vote_step(W, self.gathered, self.M, eta, self.stride)
+        if self.exchange == "allgather":
+            dist.all_gather_into_tensor(self.gathered, self.local, group=self.group)
+            self.opt.vote_step(W, self.gathered, self.M, eta, self.stride)
+            return
+        d = int(self.opt.d)
+        if self.ternary:
+            self.opt.vote_ternary(self.views, d, self.sums, None)
+        else:
+            self.opt.vote(self.views, d, self.sums, None)
+        dist.all_reduce(self.sums, op=dist.ReduceOp.SUM, group=self.group)
+        self.opt.sums_step(W, self.sums, eta)
 
     def replicas_agree(self, W):
         """True on every rank when the ranks' W agree (the [blog] replica

@@ -22,11 +22,13 @@ M_LOCAL = 2
 
 
 class _StandIn:
-    """local_signs / vote_step / sign_stride with the library's layout."""
+    """local_signs / vote_step / vote / sums_step / sign_stride with the
+    library's layout (int32 sums; flags 0)."""
 
     def __init__(self, fail=False):
         self.d = synth.numel(SHAPES)
         self.nb = ref.packed_nbytes(self.d)
+        self.flags = 0
         self.fail = fail
         self.seen = None
 
@@ -46,6 +48,14 @@ class _StandIn:
         maj = ref.majority(ref.vote_sums_from_bits(packed, self.d))
         W.copy_(torch.from_numpy(ref.update(W.numpy(), maj.astype(np.float32), eta)))
 
+    def vote(self, views, d, sums, majority):
+        sums.copy_(torch.from_numpy(ref.vote_sums_from_bits([v[: self.nb].numpy() for v in views], d)))
+
+    def sums_step(self, W, sums, eta):
+        self.seen = sums.clone()
+        maj = ref.majority(sums.numpy())
+        W.copy_(torch.from_numpy(ref.update(W.numpy(), maj.astype(np.float32), eta)))
+
 
 def _free_port():
     with socket.socket() as s:
@@ -53,7 +63,7 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def _rank(rank, world, port, fail_rank, q):
+def _rank(rank, world, port, fail_rank, q, exchange="allgather"):
     import torch.distributed as dist
 
     from sign_muon_optimizer_b200.dist import DistSignMuon
@@ -62,7 +72,7 @@ def _rank(rank, world, port, fail_rank, q):
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
     try:
         opt = _StandIn(fail=(rank == fail_rank))
-        drv = DistSignMuon(SHAPES, M_local=M_LOCAL, opt=opt, device="cpu")
+        drv = DistSignMuon(SHAPES, M_local=M_LOCAL, opt=opt, device="cpu", exchange=exchange)
         W = torch.from_numpy(synth.weights0(SHAPES, 5))
         G = synth.gradients(SHAPES, world * M_LOCAL, 1.0, step=1, config_id=5)
         mine = [torch.from_numpy(g) for g in G[rank * M_LOCAL:(rank + 1) * M_LOCAL]]
@@ -78,12 +88,12 @@ def _rank(rank, world, port, fail_rank, q):
         dist.destroy_process_group()
 
 
-def _run(fail_rank):
+def _run(fail_rank, exchange="allgather"):
     world = 2
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_rank, args=(r, world, port, fail_rank, q)) for r in range(world)]
+    procs = [ctx.Process(target=_rank, args=(r, world, port, fail_rank, q, exchange)) for r in range(world)]
     for p in procs:
         p.start()
     out = {}
@@ -116,8 +126,27 @@ def test_exchange_gathers_in_rank_order_and_replicas_agree():
             assert np.array_equal(out[r]["seen"][j * stride: j * stride + nb], packed[j])
 
 
-def test_one_failing_rank_stops_every_rank_without_update():
-    out = _run(fail_rank=1)
+def test_allreduce_exchange_adds_the_ranks_sums():
+    # each rank sums its own two workers' signs; the SUM all-reduce must give
+    # every rank the sums over all four workers, and the same W
+    out = _run(fail_rank=-1, exchange="allreduce")
+    M = 2 * M_LOCAL
+    G = synth.gradients(SHAPES, M, 1.0, step=1, config_id=5)
+    d = synth.numel(SHAPES)
+    packed = [ref.pack_bits(ref.sign_bits(g)) for g in G]
+    sums = ref.vote_sums_from_bits(packed, d)
+    w0 = synth.weights0(SHAPES, 5)
+    want = ref.update(w0, ref.majority(sums).astype(np.float32), 0.02)
+    for r in range(2):
+        assert out[r]["raised"] is False and out[r]["agree"] is True
+        assert out[r]["payload"] == 4 * d       # int32 sums
+        assert np.array_equal(out[r]["seen"], sums)
+        assert np.array_equal(out[r]["W"].view(np.uint32), want.view(np.uint32))
+
+
+@pytest.mark.parametrize("exchange", ["allgather", "allreduce"])
+def test_one_failing_rank_stops_every_rank_without_update(exchange):
+    out = _run(fail_rank=1, exchange=exchange)
     w0 = synth.weights0(SHAPES, 5)
     for r in range(2):
         assert out[r]["raised"] == "SignMuonError"

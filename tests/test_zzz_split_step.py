@@ -139,3 +139,61 @@ def test_split_argument_checks():
         with pytest.raises(smo.SignMuonError) as ei:
             call()
         assert ei.value.status == smo.SIGNMUON_E_UNSUPPORTED
+
+
+@pytest.mark.parametrize("case", ["bf16_fused", "post_polar", "ternary", "normalized_sign"])
+def test_sums_step_equals_the_step(case):
+    """[paper] Algorithm 2's form of the exchange: the workers' signs summed
+    (here by the library's own vote on one handle's buffer), then the majority
+    of the sums and the rest of the step; W and D bit for bit."""
+    shapes, flags = CASES[case]
+    M = 4
+    w0 = synth.weights0(shapes, 97)
+    whole, halves = _opt(shapes, M, flags), _opt(shapes, M, flags)
+    Wa, Wb = dev(w0), dev(w0)
+    stride = halves.sign_stride()
+    buf = torch.zeros(M * stride, dtype=torch.uint8, device="cuda")
+    sums = torch.zeros(halves.d, dtype=torch.int32, device="cuda")
+    views = [buf[m * stride:] for m in range(M)]
+    for step in (1, 2):
+        G = [dev(g) for g in synth.gradients(shapes, M, 1.0, step=step, config_id=97)]
+        whole.step(Wa, G, HP["eta"])
+        halves.local_signs(Wb, G, buf)
+        if flags & smo.SIGNMUON_TERNARY:
+            halves.vote_ternary(views, halves.d, sums, None)
+        else:
+            halves.vote(views, halves.d, sums, None)
+        halves.sums_step(Wb, sums, HP["eta"])
+        assert np.array_equal(_bits(Wa), _bits(Wb)), f"step {step}"
+    a, b = torch.zeros(whole.d, device="cuda"), torch.zeros(whole.d, device="cuda")
+    whole.get_direction(a)
+    halves.get_direction(b)
+    assert np.array_equal(_bits(a), _bits(b))
+
+
+@pytest.mark.parametrize("acc8", [False, True])
+def test_two_ranks_adding_their_sums_equal_one_handle(acc8):
+    """Two ranks each sum their own two workers' signs (int32, or int8 as
+    Algorithm 2's d-byte payload); the sums are added as the SUM all-reduce
+    would, and both ranks land on the W of one four-worker handle."""
+    shapes, flags = CASES["bf16_fused"]
+    flags |= smo.SIGNMUON_ACC_INT8 if acc8 else 0
+    M, ranks, per = 4, 2, 2
+    w0 = synth.weights0(shapes, 99)
+    single = _opt(shapes, M, flags)
+    parts = [_opt(shapes, per, flags) for _ in range(ranks)]
+    stride = single.sign_stride()
+    W, Wr = dev(w0), [dev(w0) for _ in range(ranks)]
+    dt = torch.int8 if acc8 else torch.int32
+    local = [torch.zeros(per * stride, dtype=torch.uint8, device="cuda") for _ in range(ranks)]
+    part_sums = [torch.zeros(single.d, dtype=dt, device="cuda") for _ in range(ranks)]
+    for step in (1, 2):
+        G = [dev(g) for g in synth.gradients(shapes, M, 1.0, step=step, config_id=99)]
+        single.step(W, G, HP["eta"])
+        for r in range(ranks):
+            parts[r].local_signs(Wr[r], G[r * per:(r + 1) * per], local[r])
+            parts[r].vote([local[r][m * stride:] for m in range(per)], single.d, part_sums[r], None)
+        total = part_sums[0] + part_sums[1]          # the all-reduce's sum
+        for r in range(ranks):
+            parts[r].sums_step(Wr[r], total, HP["eta"])
+            assert np.array_equal(_bits(Wr[r]), _bits(W)), f"rank {r}, step {step}"
