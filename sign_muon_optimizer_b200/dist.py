@@ -25,6 +25,9 @@ same shapes, flags and exchange.
 """
 from __future__ import annotations
 
+import time
+
+import numpy as np
 import torch
 import torch.distributed as dist
 
@@ -80,7 +83,17 @@ class DistSignMuon:
             return self.local.numel()
         return self.sums.numel() * self.sums.element_size()
 
-    def step(self, W, G, eta):
+    def step(self, W, G, eta, clocks=None):
+        """One step.  With a ``clocks`` dict, adds this step's phase times in
+        ms to its keys ([blog] "The experiment needs three clocks"; the
+        gradient clock is the caller's):
+        - local_ms: momentum, polar factor and signs, the status all-reduce,
+          and, for the all-reduce exchange, the local vote;
+        - exchange_ms: the all-gather or the SUM all-reduce;
+        - finish_ms: the vote or majority, the post-vote step and the update;
+        - total_ms: the whole step."""
+        clk = _PhaseClock(self.device) if clocks is not None else None
+        t0 = clk.mark() if clk else None
         err = None
         try:
             self.opt.local_signs(W, G, self.local, self.stride)
@@ -95,16 +108,25 @@ class DistSignMuon:
                 raise err
             raise SignMuonError(SIGNMUON_E_NONFINITE, "another rank's step failed; W was not updated")
         if self.exchange == "allgather":
+            t1 = clk.mark() if clk else None
             dist.all_gather_into_tensor(self.gathered, self.local, group=self.group)
+            t2 = clk.mark() if clk else None
             self.opt.vote_step(W, self.gathered, self.M, eta, self.stride)
-            return
-        d = int(self.opt.d)
-        if self.ternary:
-            self.opt.vote_ternary(self.views, d, self.sums, None)
         else:
-            self.opt.vote(self.views, d, self.sums, None)
-        dist.all_reduce(self.sums, op=dist.ReduceOp.SUM, group=self.group)
-        self.opt.sums_step(W, self.sums, eta)
+            d = int(self.opt.d)
+            if self.ternary:
+                self.opt.vote_ternary(self.views, d, self.sums, None)
+            else:
+                self.opt.vote(self.views, d, self.sums, None)
+            t1 = clk.mark() if clk else None
+            dist.all_reduce(self.sums, op=dist.ReduceOp.SUM, group=self.group)
+            t2 = clk.mark() if clk else None
+            self.opt.sums_step(W, self.sums, eta)
+        if clk:
+            t3 = clk.mark()
+            for key, a, b in (("local_ms", t0, t1), ("exchange_ms", t1, t2), ("finish_ms", t2, t3),
+                              ("total_ms", t0, t3)):
+                clocks[key] = clocks.get(key, 0.0) + clk.ms(a, b)
 
     def replicas_agree(self, W):
         """True on every rank when the ranks' W agree (the [blog] replica
@@ -117,3 +139,76 @@ class DistSignMuon:
         dist.all_reduce(lo, op=dist.ReduceOp.MIN, group=self.group)
         dist.all_reduce(hi, op=dist.ReduceOp.MAX, group=self.group)
         return bool(torch.equal(lo, hi))
+
+
+class _PhaseClock:
+    """Phase boundaries on the device (CUDA events on the current stream,
+    read after a synchronize) or, for a CPU device, on the host clock."""
+
+    def __init__(self, device):
+        self.cuda = torch.device(device).type == "cuda"
+
+    def mark(self):
+        if self.cuda:
+            e = torch.cuda.Event(enable_timing=True)
+            e.record()
+            return e
+        return time.perf_counter()
+
+    def ms(self, a, b):
+        if self.cuda:
+            b.synchronize()
+            return float(a.elapsed_time(b))
+        return (b - a) * 1e3
+
+
+def fit_alpha_beta(nbytes, seconds):
+    """Least-squares fit of the alpha-beta model t = alpha + beta * n ([paper]
+    §6: alpha the start-up latency in s, beta the time per byte in s/byte)
+    to collective timings at several message sizes."""
+    n = np.asarray(nbytes, np.float64)
+    t = np.asarray(seconds, np.float64)
+    A = np.stack([np.ones_like(n), n], axis=1)
+    (alpha, beta), *_ = np.linalg.lstsq(A, t, rcond=None)
+    return float(alpha), float(beta)
+
+
+def allreduce_time_model(alpha, beta, M, nbytes, rounds):
+    """[paper] §6 per-iteration estimate of one all-reduce over M ranks:
+    alpha * R(M) + 2 (1 - 1/M) * s * beta, with R(M) the rounds on the
+    critical path and s the payload in bytes."""
+    return alpha * rounds + 2.0 * (1.0 - 1.0 / M) * nbytes * beta
+
+
+def time_collective(kind, nbytes_list, reps=5, group=None, device="cpu"):
+    """Seconds per call of one collective at each message size, the max over
+    ranks: kind "allgather" (each rank gives n uint8 bytes) or "allreduce"
+    (a SUM over n int8 bytes).  One untimed call per size first."""
+    world = dist.get_world_size(group)
+    clk = _PhaseClock(device)
+    out = []
+    for n in nbytes_list:
+        n = int(n)
+        if kind == "allgather":
+            src = torch.zeros(n, dtype=torch.uint8, device=device)
+            dst = torch.zeros(n * world, dtype=torch.uint8, device=device)
+
+            def call():
+                dist.all_gather_into_tensor(dst, src, group=group)
+        elif kind == "allreduce":
+            buf = torch.zeros(n, dtype=torch.int8, device=device)
+
+            def call():
+                dist.all_reduce(buf, op=dist.ReduceOp.SUM, group=group)
+        else:
+            raise ValueError(kind)
+        call()
+        dist.barrier(group=group)
+        a = clk.mark()
+        for _ in range(reps):
+            call()
+        b = clk.mark()
+        t = torch.tensor([clk.ms(a, b) / 1e3 / reps], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX, group=group)
+        out.append(float(t.item()))
+    return out

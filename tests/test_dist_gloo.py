@@ -77,13 +77,14 @@ def _rank(rank, world, port, fail_rank, q, exchange="allgather"):
         G = synth.gradients(SHAPES, world * M_LOCAL, 1.0, step=1, config_id=5)
         mine = [torch.from_numpy(g) for g in G[rank * M_LOCAL:(rank + 1) * M_LOCAL]]
         raised = False
+        clocks = {}
         try:
-            drv.step(W, mine, 0.02)
+            drv.step(W, mine, 0.02, clocks=clocks)
         except Exception as e:  # noqa: BLE001
             raised = type(e).__name__
         agree = drv.replicas_agree(W)
         q.put((rank, W.numpy().copy(), None if opt.seen is None else opt.seen.numpy(), raised, agree,
-               drv.payload_bytes))
+               drv.payload_bytes, clocks))
     finally:
         dist.destroy_process_group()
 
@@ -98,8 +99,8 @@ def _run(fail_rank, exchange="allgather"):
         p.start()
     out = {}
     for _ in range(world):
-        r, W, seen, raised, agree, payload = q.get(timeout=120)
-        out[r] = dict(W=W, seen=seen, raised=raised, agree=agree, payload=payload)
+        r, W, seen, raised, agree, payload, clocks = q.get(timeout=120)
+        out[r] = dict(W=W, seen=seen, raised=raised, agree=agree, payload=payload, clocks=clocks)
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
@@ -124,6 +125,10 @@ def test_exchange_gathers_in_rank_order_and_replicas_agree():
         assert np.array_equal(out[r]["W"].view(np.uint32), want.view(np.uint32))
         for j in range(M):  # global worker j sits at slot j on every rank
             assert np.array_equal(out[r]["seen"][j * stride: j * stride + nb], packed[j])
+        c = out[r]["clocks"]
+        assert set(c) == {"local_ms", "exchange_ms", "finish_ms", "total_ms"}
+        assert all(v >= 0.0 for v in c.values())
+        assert abs(c["local_ms"] + c["exchange_ms"] + c["finish_ms"] - c["total_ms"]) <= 1e-6 * max(1.0, c["total_ms"])
 
 
 def test_allreduce_exchange_adds_the_ranks_sums():
@@ -153,6 +158,50 @@ def test_one_failing_rank_stops_every_rank_without_update(exchange):
         assert out[r]["seen"] is None           # nobody voted
         assert np.array_equal(out[r]["W"], w0)  # nobody updated
         assert out[r]["agree"] is True
+        assert out[r]["clocks"] == {}          # a failed step records no times
+
+
+def test_alpha_beta_fit_recovers_the_model():
+    from sign_muon_optimizer_b200.dist import allreduce_time_model, fit_alpha_beta
+    alpha, beta = 7.5e-6, 1.0 / 150e9
+    sizes = [1 << k for k in range(10, 31, 4)]
+    a, b = fit_alpha_beta(sizes, [alpha + beta * n for n in sizes])
+    assert abs(a - alpha) <= 1e-12 and abs(b - beta) <= 1e-9 * beta
+    # one rank moves nothing; the transfer term tends to 2 s beta for many ranks
+    assert allreduce_time_model(alpha, beta, 1, 1 << 20, 0) == 0.0
+    assert allreduce_time_model(alpha, beta, 1, 1 << 20, 3) == 3 * alpha
+    big = allreduce_time_model(alpha, beta, 10 ** 9, 1 << 20, 1)
+    assert abs(big - (alpha + 2 * (1 << 20) * beta)) <= 1e-9 * big
+
+
+def _time_rank(rank, world, port, q):
+    import torch.distributed as dist
+
+    from sign_muon_optimizer_b200.dist import time_collective
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        sizes = [1 << 10, 1 << 16, 1 << 20]
+        q.put((rank, time_collective("allgather", sizes, reps=2), time_collective("allreduce", sizes, reps=2)))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_collective_timings_are_the_max_over_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_time_rank, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = dict((r, (ag, ar)) for r, ag, ar in (q.get(timeout=120) for _ in range(2)))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert res[0] == res[1]                    # both ranks report the max
+    for ts in res[0]:
+        assert len(ts) == 3 and all(t > 0.0 for t in ts)
 
 
 def test_too_many_workers_is_rejected():
