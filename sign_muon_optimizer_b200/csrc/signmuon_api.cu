@@ -10,6 +10,7 @@
 //   fused with the update, or vote -> stage -> NS x K -> update for the
 //   post-vote polar step (K = 0 there for the normalised sign step).
 #include <cuda.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <atomic>
 #include <cstdio>
@@ -208,12 +209,28 @@ sm::WorkerPtrs strided_ptrs(const float* base, int64_t stride, int M) {
   return w;
 }
 
-// Record the event pair of one kernel launch of `kind` (no-op unless timing).
+// NVTX range names of the profiling kinds (signmuon_profile's numbering)
+const char* const kKindNames[SIGNMUON_PROF_KINDS] = {
+    "signmuon momentum",      "signmuon norm finalize",  "signmuon NS gram",       "signmuon NS square",
+    "signmuon NS apply",      "signmuon power iteration", "signmuon sign",         "signmuon vote",
+    "signmuon mean stage",    "signmuon post NS gram",    "signmuon post NS square", "signmuon post NS apply",
+    "signmuon update",        "signmuon K=0 scale"};
+
+// A host NVTX range for the lifetime of a scope (a no-op unless a tool such
+// as ncu --nvtx is attached).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+};
+
+// One kernel launch of `kind`: an NVTX range always, and the CUDA event pair
+// only while timing (signmuon_profile).
 struct ProfScope {
   signmuon_t h;
   int kind;
   cudaEvent_t e1 = nullptr;
-  ProfScope(signmuon_t h_, int kind_) : h(h_), kind(kind_) {
+  NvtxRange range;
+  ProfScope(signmuon_t h_, int kind_) : h(h_), kind(kind_), range(kKindNames[kind_]) {
     if (!h->prof) return;
     while (h->ev_pool.size() < h->ev_used + 2) {
       cudaEvent_t e;
@@ -665,6 +682,7 @@ static void vote_part(signmuon_t h, float* W, const uint8_t* src, int64_t stride
 }
 
 int signmuon_step(signmuon_t h, float* W, const float* const* G, float eta) {
+  NvtxRange range("signmuon_step");
   int rc = check_handle(h, true);
   if (rc) return rc;
   const Plan& p = h->plan;
@@ -712,6 +730,7 @@ int signmuon_step(signmuon_t h, float* W, const float* const* G, float eta) {
 }
 
 int signmuon_local_signs(signmuon_t h, const float* W, const float* const* G, uint8_t* signs, int64_t stride) {
+  NvtxRange range("signmuon_local_signs");
   int rc = check_handle(h, true);
   if (rc) return rc;
   const Plan& p = h->plan;
@@ -733,6 +752,7 @@ int signmuon_local_signs(signmuon_t h, const float* W, const float* const* G, ui
 }
 
 int signmuon_vote_step(signmuon_t h, float* W, const uint8_t* signs, int64_t stride, int M, float eta) {
+  NvtxRange range("signmuon_vote_step");
   const bool post = h != nullptr && (h->flags & (SIGNMUON_POST_POLAR | SIGNMUON_NORMALIZED_SIGN)) != 0;
   int rc = check_handle(h, post);
   if (rc) return rc;
@@ -752,6 +772,7 @@ int signmuon_vote_step(signmuon_t h, float* W, const uint8_t* signs, int64_t str
 }
 
 int signmuon_sums_step(signmuon_t h, float* W, const void* sums, float eta) {
+  NvtxRange range("signmuon_sums_step");
   int rc = check_handle(h, true);
   if (rc) return rc;
   const Plan& p = h->plan;
