@@ -284,7 +284,9 @@ int signmuon_get_gram(signmuon_t h, int m, int mat, float* dst_host);
 int signmuon_set_ns_coeffs(signmuon_t h, const float* coeffs, int n);
 
 /* Wait for the handle's stream; returns the first deferred error
- * (E_NONFINITE, E_TIMEOUT, E_CUDA) since the last sync, and clears it. */
+ * (E_NONFINITE, E_TIMEOUT, E_CUDA) since the last sync, and clears it.  Until
+ * then a deferred error stays set: later SIGNMUON_ASYNC calls on the handle
+ * run but leave W unchanged. */
 int signmuon_sync(signmuon_t h);
 
 /* Sizes: out[0]=d, out[1]=packed bytes per worker, out[2]=device bytes owned

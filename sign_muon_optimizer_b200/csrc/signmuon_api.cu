@@ -379,6 +379,15 @@ void fro_finalize(signmuon_t h, int nw) {
                           h->ns_c, h->scale_v, h->coef_apply, h->coef_square, h->status);
 }
 
+// Clear the device status at the start of a call, unless an asynchronous
+// call's status is still unread: then its flags stay set, so the update
+// kernels of this call leave W alone and signmuon_sync reports the first
+// error since the last sync.
+cudaError_t begin_status(signmuon_t h) {
+  if (h->pending) return cudaSuccess;
+  return cudaMemsetAsync(h->status, 0, 2 * sizeof(int), h->stream);
+}
+
 int finish(signmuon_t h, bool wait) {
   CK(h, cudaMemcpyAsync(h->h_status, h->status, 2 * sizeof(int), cudaMemcpyDeviceToHost, h->stream));
   CK(h, cudaGetLastError());
@@ -691,7 +700,7 @@ int signmuon_step(signmuon_t h, float* W, const float* const* G, float eta) {
   for (int m = 0; m < h->M; ++m)
     if (G[m] == nullptr || !aligned16(G[m])) return fail(h, SIGNMUON_E_INVALID, "G[m] null or not 16-byte aligned");
   cudaStream_t s = h->stream;
-  CK(h, cudaMemsetAsync(h->status, 0, 2 * sizeof(int), s));
+  CK(h, begin_status(h));
   const sm::WorkerPtrs gp = worker_ptrs(G, h->M);
   if (h->flags & SIGNMUON_MUON_MEAN) {
     // Muon baseline: the workers' mean momentum through one PolarNS
@@ -742,7 +751,7 @@ int signmuon_local_signs(signmuon_t h, const float* W, const float* const* G, ui
   const int64_t need = (h->flags & SIGNMUON_TERNARY) ? p.d : p.nb;
   if (stride < need || stride % 16 != 0)
     return fail(h, SIGNMUON_E_INVALID, "stride must be a multiple of 16 bytes and hold one worker's signs");
-  CK(h, cudaMemsetAsync(h->status, 0, 2 * sizeof(int), h->stream));
+  CK(h, begin_status(h));
   // the handle's own sign buffers do not hold these signs
   h->bits_valid = false;
   h->t_valid = false;
@@ -764,7 +773,7 @@ int signmuon_vote_step(signmuon_t h, float* W, const uint8_t* signs, int64_t str
   const int64_t need = (h->flags & SIGNMUON_TERNARY) ? p.d : p.nb;
   if (stride < need || stride % 16 != 0)
     return fail(h, SIGNMUON_E_INVALID, "stride must be a multiple of 16 bytes and hold one worker's signs");
-  CK(h, cudaMemsetAsync(h->status, 0, 2 * sizeof(int), h->stream));
+  CK(h, begin_status(h));
   h->dir_valid = post;  // D is kept only by the post-vote steps
   h->dir_in_D = post;
   vote_part(h, W, signs, stride, M, eta);
@@ -780,7 +789,7 @@ int signmuon_sums_step(signmuon_t h, float* W, const void* sums, float eta) {
   if (W == nullptr || sums == nullptr) return fail(h, SIGNMUON_E_INVALID, "null W or sums");
   if (!aligned16(W) || !aligned16(sums)) return fail(h, SIGNMUON_E_INVALID, "W and sums must be 16-byte aligned");
   cudaStream_t s = h->stream;
-  CK(h, cudaMemsetAsync(h->status, 0, 2 * sizeof(int), s));
+  CK(h, begin_status(h));
   const int tie = (h->flags & SIGNMUON_TIE_PLUS) ? 1 : 0;
   {
     // the majority into D; for the post-vote steps D is then staged as
@@ -914,7 +923,7 @@ int signmuon_polar(signmuon_t h, const float* const* X, float* const* U) {
     if (!X[m] || !U[m] || !aligned16(X[m]) || !aligned16(U[m]))
       return fail(h, SIGNMUON_E_INVALID, "X[m]/U[m] null or misaligned");
   cudaStream_t s = h->stream;
-  CK(h, cudaMemsetAsync(h->status, 0, 2 * sizeof(int), s));
+  CK(h, begin_status(h));
   const sm::WorkerPtrs xp = worker_ptrs(X, h->M);
   sm::launch_stage(s, xp, h->M, h->X[0], p.fp32 ? 0 : 1, h->d_chunks, (int)p.chunks.size(), h->d_mats, h->d_groups,
                    h->partials);
