@@ -263,7 +263,9 @@ int signmuon_polar(signmuon_t h, const float* const* X, float* const* U);
  * get_direction: the last step's D (E_UNSUPPORTED before the first step, and
  * after a signmuon_vote_step whose vote was fused with the update).
  * get_scales: host float[M*n_mats]: the last step's scale s per (worker,
- * matrix), worker-major (waits for the GPU).
+ * matrix), worker-major (waits for the GPU).  A post-vote step (POST_POLAR,
+ * NORMALIZED_SIGN, MUON_MEAN) writes its own scales, those of the majority
+ * (or mean) matrices, into worker 0's row.
  * ---------------------------------------------------------------------- */
 int signmuon_get_momentum(signmuon_t h, int m, float* dst);
 int signmuon_set_momentum(signmuon_t h, int m, const float* src);
@@ -275,7 +277,8 @@ int signmuon_get_scales(signmuon_t h, float* dst_host);
 /* get_gram: the Gram matrix (g x g, g = min(rows, cols), row-major floats on
  * the host) that the last Newton-Schulz iteration of worker m used for
  * matrix `mat`: X X^T of the wide orientation; after one iteration it is the
- * unscaled Gram of the staged momentum (waits for the GPU). */
+ * unscaled Gram of the staged momentum (waits for the GPU).  After a post-vote
+ * step, worker 0's slot holds the post-vote step's Gram. */
 int signmuon_get_gram(signmuon_t h, int m, int mat, float* dst_host);
 
 /* Newton-Schulz coefficients: n=2 (a, b) for X <- aX + b(XX^T)X ([paper] §3
