@@ -40,8 +40,13 @@ R6  Packing: one flat bit stream over all matrices (shapes order, row-major),
 R7  Ties map to 0 ([blog]) by default; the +1 policy of [paper] Algorithm 2 is
     the named variant majority(..., tie=1).
 R8  Post-vote polar: D = PolarNS(majority as floats) with the same K, eps,
-    scale and P; no second sign, no rescale.
+    scale and P; no second sign, no rescale.  The pages fix neither where this
+    step sits nor its scale, so beyond the PolarNS arithmetic (pinned by the
+    closed forms) its parity is unpinned.
 R9  Update: W_new = float32 nearest to (W - eta*D), one rounding.
+R19 Ternary wire (named variant): sign(U) in {-1, 0, +1}, one int8 per entry.
+R20 Normalised sign step (named variant): D = majority / (s + eps) per matrix,
+    s the scale PolarNS would use (R2 for spectral, the Frobenius norm for fro).
 R21 Warm-started power iteration (named variant): each problem's power
     iteration starts from the iterate it ended with in the previous step;
     a zero or non-finite stored iterate starts from ones/sqrt(m) as in R2.
