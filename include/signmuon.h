@@ -301,6 +301,17 @@ int signmuon_info(signmuon_t h, int64_t* out, int n);
 int signmuon_plan(const int64_t* shapes, int n_mats, int M, int K, int scale, int P,
                   unsigned flags, int64_t* out, int n);
 
+/* Host-only: the plan's tables as JSON text, for inspection and for checking
+ * the planner without a GPU.  The tables are the shape groups and their
+ * buffer bases, the matrices, the 4096-entry chunks of the elementwise
+ * kernels, the GEMM tile lists per op (Gram, quintic square, apply) for M
+ * workers and for one, the power-iteration row blocks and vector offsets, and
+ * the buffer sizes.  *need receives the text's size in bytes, with the
+ * terminating NUL.  buf may be NULL to ask for the size; a non-NULL buf
+ * shorter than that returns E_INVALID.  Validates like signmuon_init. */
+int signmuon_plan_tables(const int64_t* shapes, int n_mats, int M, int K, int scale, int P,
+                         unsigned flags, char* buf, int64_t cap, int64_t* need);
+
 /* Per-kernel timing.  signmuon_profile(h, 1) makes the following calls record
  * a CUDA event pair around every kernel they launch on the handle's stream;
  * signmuon_profile_read() waits for the stream, adds up the elapsed times per

@@ -52,6 +52,7 @@ EXPORTED = [
     "signmuon_profile", "signmuon_profile_read", "signmuon_get_gram",
     "signmuon_spectral_norm_noalloc", "signmuon_sign_ternary", "signmuon_vote_ternary",
     "signmuon_get_ternary_signs", "signmuon_local_signs", "signmuon_vote_step", "signmuon_sums_step",
+    "signmuon_plan_tables",
 ]
 PROF_KINDS = ["momentum", "norm_finalize", "ns_gram", "ns_square", "ns_apply", "power_iter", "pack",
               "vote", "stage", "post_gram", "post_square", "post_apply", "update", "k0_scale"]
@@ -81,6 +82,8 @@ def _load():
         "signmuon_local_signs": (I, [P, P, PP, P, I64]),
         "signmuon_vote_step": (I, [P, P, P, I64, I, F]),
         "signmuon_sums_step": (I, [P, P, P, F]),
+        "signmuon_plan_tables": (I, [ctypes.POINTER(I64), I, I, I, I, I, U, ctypes.c_char_p, I64,
+                                     ctypes.POINTER(I64)]),
         "signmuon_apply_update": (I, [P, P, P, I64, F]),
         "signmuon_polar": (I, [P, PP, PP]),
         "signmuon_get_momentum": (I, [P, I, P]),
@@ -277,6 +280,20 @@ def signmuon_plan(shapes, M, K=5, scale=SIGNMUON_SCALE_FRO, P=1, flags=0):
     out = (ctypes.c_int64 * 6)()
     _check(None, _lib.signmuon_plan(arr, n, int(M), int(K), int(scale), int(P), int(flags), out, 6))
     return dict(zip(["d", "packed_bytes", "device_bytes", "groups", "M", "n_mats"], list(out)))
+
+
+def signmuon_plan_tables(shapes, M, K=5, scale=SIGNMUON_SCALE_FRO, P=1, flags=0):
+    """The plan's tables (host only) as a dict parsed from the library's JSON."""
+    import json
+    if isinstance(scale, str):
+        scale = {"fro": SIGNMUON_SCALE_FRO, "spectral": SIGNMUON_SCALE_SPECTRAL}[scale]
+    arr, n = _shapes_arr(shapes)
+    need = ctypes.c_int64(0)
+    args = (arr, n, int(M), int(K), int(scale), int(P), int(flags))
+    _check(None, _lib.signmuon_plan_tables(*args, None, 0, ctypes.byref(need)))
+    buf = ctypes.create_string_buffer(need.value)
+    _check(None, _lib.signmuon_plan_tables(*args, buf, need.value, ctypes.byref(need)))
+    return json.loads(buf.value.decode())
 
 
 def signmuon_kernel_launches():

@@ -15,8 +15,10 @@
 #include <atomic>
 #include <cstdio>
 #include <cstring>
+#include <initializer_list>
 #include <new>
 #include <string>
+#include <utility>
 #include <vector>
 
 #include "../../include/signmuon.h"
@@ -447,6 +449,89 @@ int signmuon_plan(const int64_t* shapes, int n_mats, int M, int K, int scale, in
   const int rc = sm::make_plan(shapes, n_mats, M, K, scale, P, flags, &p, &err);
   if (rc) return fail(nullptr, rc, err);
   if (out) fill_info(p, out, n);
+  return SIGNMUON_OK;
+}
+
+int signmuon_plan_tables(const int64_t* shapes, int n_mats, int M, int K, int scale, int P, unsigned flags,
+                         char* buf, int64_t cap, int64_t* need) {
+  Plan p;
+  std::string err;
+  const int rc = sm::make_plan(shapes, n_mats, M, K, scale, P, flags, &p, &err);
+  if (rc) return fail(nullptr, rc, err);
+  std::string j;
+  j.reserve(1 << 16);
+  auto num = [&](int64_t v) { j += std::to_string(v); };
+  auto list = [&](const char* name, auto n, auto item) {
+    j += '"';
+    j += name;
+    j += "\":[";
+    for (size_t i = 0; i < (size_t)n; ++i) {
+      if (i) j += ',';
+      item(i);
+    }
+    j += "],";
+  };
+  auto tuple = [&](std::initializer_list<int64_t> v) {
+    j += '[';
+    bool first = true;
+    for (int64_t x : v) {
+      if (!first) j += ',';
+      first = false;
+      num(x);
+    }
+    j += ']';
+  };
+  j += "{";
+  const std::pair<const char*, int64_t> scalars[] = {
+      {"d", p.d}, {"dpad", p.dpad}, {"nb", p.nb}, {"nb_pad", p.nb_pad}, {"x_elems", p.x_elems},
+      {"a_elems", p.a_elems}, {"u_elems", p.u_elems}, {"u_elems_one", p.u_elems_one},
+      {"n_pi_rows_one", p.n_pi_rows_one}, {"M", p.M}, {"n_mats", p.n_mats}, {"fp32", p.fp32 ? 1 : 0},
+      {"quintic", p.quintic ? 1 : 0}, {"device_bytes", p.device_bytes}};
+  for (const auto& kv : scalars) {
+    j += '"';
+    j += kv.first;
+    j += "\":";
+    num(kv.second);
+    j += ',';
+  }
+  list("groups", p.groups.size(), [&](size_t i) {
+    const sm::GroupInfo& g = p.groups[i];
+    tuple({g.rows, g.cols, g.ld, g.g, g.gld, g.wide, g.count, g.first, g.x_base, g.a_base});
+  });
+  list("mats", p.mats.size(), [&](size_t i) {
+    const sm::MatInfo& m = p.mats[i];
+    tuple({m.off, m.rows, m.cols, m.group, m.q});
+  });
+  list("group_mats", p.group_mats.size(), [&](size_t i) { num(p.group_mats[i]); });
+  list("chunks", p.chunks.size(), [&](size_t i) {
+    const sm::Chunk& c = p.chunks[i];
+    tuple({c.mat, c.len, c.start});
+  });
+  list("mat_chunk0", p.mat_chunk0.size(), [&](size_t i) { num(p.mat_chunk0[i]); });
+  list("mat_nchunks", p.mat_nchunks.size(), [&](size_t i) { num(p.mat_nchunks[i]); });
+  list("tiles", 6, [&](size_t k) {
+    const sm::TileTable& t = p.tiles[k / 2][k % 2];
+    j += "{\"total\":";
+    num(t.total);
+    j += ",\"groups\":[";
+    for (size_t i = 0; i < t.groups.size(); ++i) {
+      const sm::TileGroup& x = t.groups[i];
+      if (i) j += ',';
+      tuple({x.group, x.Mdim, x.Ndim, x.Kdim, x.BM, x.BN, x.sym, x.tiles_m, x.tiles_n, x.batch, x.tile_start});
+    }
+    j += "]}";
+  });
+  list("pi_rows", p.pi_rows.size(), [&](size_t i) { tuple({p.pi_rows[i].p, p.pi_rows[i].row0}); });
+  list("uoff", p.uoff.size(), [&](size_t i) { num(p.uoff[i]); });
+  list("prob_g", p.prob_g.size(), [&](size_t i) { num(p.prob_g[i]); });
+  list("prob_gld", p.prob_gld.size(), [&](size_t i) { num(p.prob_gld[i]); });
+  list("prob_aoff", p.prob_aoff.size(), [&](size_t i) { num(p.prob_aoff[i]); });
+  j.back() = '}';
+  const int64_t n = (int64_t)j.size() + 1;
+  if (need) *need = n;
+  if (buf == nullptr) return SIGNMUON_OK;
+  if (cap < n) return fail(nullptr, SIGNMUON_E_INVALID, "buffer too small: " + std::to_string(n) + " bytes needed");
+  std::memcpy(buf, j.c_str(), (size_t)n);
   return SIGNMUON_OK;
 }
 

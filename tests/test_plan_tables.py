@@ -1,0 +1,158 @@
+"""The planner's tables (signmuon_plan_tables, host only) against the layout
+rules the kernels rely on, for random mixes of matrix shapes, worker counts
+and precision flags (hypothesis, derandomized):
+
+- every X / A region and power-iteration vector lies inside its buffer, and
+  none overlaps another;
+- every base and row stride keeps rows on 16-byte boundaries (the TMA rule);
+- the 4096-entry chunks cover each matrix exactly once, in order;
+- the GEMM tile lists have the tile counts their shapes need, for every
+  operation, for M workers and for one.
+
+A planner mistake here would be an out-of-range access on the GPU."""
+import pytest
+
+hyp = pytest.importorskip("hypothesis")
+from hypothesis import given, settings  # noqa: E402
+from hypothesis import strategies as st  # noqa: E402
+
+import sign_muon_optimizer_b200 as smo  # noqa: E402
+
+GRAM, SQUARE, APPLY = 0, 1, 2
+
+
+def _ceil(a, b):
+    return -(-a // b)
+
+
+def _disjoint_inside(regions, limit):
+    regions = sorted((s, e) for s, e in regions if e > s)
+    end = 0
+    for s, e in regions:
+        assert s >= end, f"overlap at {s}"
+        end = e
+    assert end <= limit
+
+
+def _check(shapes, M, flags, spectral):
+    t = smo.signmuon_plan_tables(shapes, M, 5, "spectral" if spectral else "fro", 2, flags)
+    fp32 = bool(flags & smo.SIGNMUON_NS_FP32)
+    d = sum(r * c for r, c in shapes)
+    assert t["d"] == d and t["dpad"] >= d and t["dpad"] % 64 == 0
+    assert t["nb"] == _ceil(d, 8) and t["nb_pad"] >= t["nb"] and t["nb_pad"] % 16 == 0
+    assert t["device_bytes"] == smo.signmuon_plan(shapes, M, 5, "spectral" if spectral else "fro", 2,
+                                                  flags)["device_bytes"]
+
+    # shape groups, in order of first appearance
+    distinct = list(dict.fromkeys(shapes))
+    groups = t["groups"]
+    assert [(g[0], g[1]) for g in groups] == distinct
+    first = 0
+    for (rows, cols, ld, g, gld, wide, count, gfirst, x_base, a_base) in groups:
+        assert ld == _ceil(cols, 8) * 8 and g == min(rows, cols) and gld == _ceil(g, 8) * 8
+        assert wide == (1 if rows <= cols else 0) and count == shapes.count((rows, cols))
+        assert gfirst == first
+        first += count
+        assert x_base % 8 == 0 and a_base % 8 == 0      # 16-byte aligned bf16 bases
+    _disjoint_inside([(g[8], g[8] + M * g[6] * g[0] * g[2]) for g in groups], t["x_elems"])
+    _disjoint_inside([(g[9], g[9] + M * g[6] * g[3] * g[4]) for g in groups], t["a_elems"])
+
+    # matrices and their place in the flat vector and in their group
+    off, seen = 0, {}
+    for i, (moff, rows, cols, gi, q) in enumerate(t["mats"]):
+        assert (rows, cols) == shapes[i] and moff == off
+        assert groups[gi][0:2] == [rows, cols] and q == seen.get(gi, 0)
+        assert t["group_mats"][groups[gi][7] + q] == i
+        seen[gi] = q + 1
+        off += rows * cols
+
+    # chunks of the elementwise kernels: each matrix exactly once, in order
+    chunks = t["chunks"]
+    for i, (r, c) in enumerate(shapes):
+        c0, nc = t["mat_chunk0"][i], t["mat_nchunks"][i]
+        assert nc == _ceil(r * c, 4096)
+        pos = 0
+        for mat, ln, start in chunks[c0:c0 + nc]:
+            assert mat == i and start == pos and 0 < ln <= 4096
+            pos += ln
+        assert pos == r * c
+    assert sum(t["mat_nchunks"]) == len(chunks)
+
+    # GEMM tile lists
+    for op in (GRAM, SQUARE, APPLY):
+        for slot, nw in ((0, M), (1, 1)):
+            table = t["tiles"][2 * op + slot]
+            tg = table["groups"]
+            assert sorted(x[0] for x in tg) == list(range(len(groups)))
+            start = 0
+            for (gi, Md, Nd, Kd, BM, BN, sym, tm, tn, batch, tstart) in tg:
+                rows, cols, _, g = groups[gi][:4]
+                if op == GRAM:
+                    assert (Md, Nd, Kd) == (g, g, max(rows, cols))
+                elif op == SQUARE:
+                    assert (Md, Nd, Kd) == (g, g, g)
+                else:
+                    assert (Md, Nd, Kd) == (rows, cols, g)
+                if fp32:
+                    assert (BM, BN) == (128, 128) and sym == 0
+                else:
+                    assert BM == 256 and BN in (128, 256)
+                    assert sym == (1 if (op == GRAM and BN == 256) else 0)
+                assert tm == _ceil(Md, BM) and tn == _ceil(Nd, BN)
+                assert batch == nw * groups[gi][6] and tstart == start
+                per = tm * (tm + 1) // 2 if sym else tm * tn
+                start += per * batch
+            assert table["total"] == start
+
+    # power iteration: problem p = worker * n_mats + matrix
+    n = len(shapes)
+    gs = [min(r, c) for r, c in shapes]
+    assert t["prob_g"] == gs * M
+    assert t["u_elems_one"] == sum(gs) and t["u_elems"] == M * sum(gs)
+    _disjoint_inside([(u, u + g) for u, g in zip(t["uoff"], t["prob_g"])], t["u_elems"])
+    for p, aoff in enumerate(t["prob_aoff"]):
+        w, i = divmod(p, n)
+        mat = t["mats"][i]
+        grp = groups[mat[3]]
+        assert aoff == grp[9] + (w * grp[6] + mat[4]) * grp[3] * grp[4]
+        assert t["prob_gld"][p] == grp[4]
+    rows_of = {}
+    for k, (p, r0) in enumerate(t["pi_rows"]):
+        rows_of.setdefault(p, []).append(r0)
+        if k < t["n_pi_rows_one"]:
+            assert p < n                           # worker 0's blocks come first
+    for p in range(M * n):
+        assert rows_of[p] == list(range(0, t["prob_g"][p], 32))
+
+
+shape = st.tuples(st.integers(1, 300), st.integers(1, 300))
+
+
+@settings(max_examples=120, deadline=None, derandomize=True)
+@given(st.lists(shape, min_size=1, max_size=5), st.integers(0, 3), st.integers(1, 9), st.integers(0, 7),
+       st.booleans())
+def test_plan_tables_follow_the_layout_rules(base, repeat, M, fl, spectral):
+    shapes = base + base[:repeat]                  # repeated shapes share a group
+    flags = ((smo.SIGNMUON_NS_FP32 if fl & 1 else 0) | (smo.SIGNMUON_NS_QUINTIC if fl & 2 else 0)
+             | (smo.SIGNMUON_POST_POLAR if fl & 4 else 0))
+    _check(shapes, M, flags, spectral)
+
+
+@pytest.mark.parametrize("name", ["nanogpt", "resnet50"])
+def test_plan_tables_of_the_bench_workloads(name):
+    import synth
+    wl = synth.WORKLOADS[name]
+    _check([tuple(s) for s in wl["shapes"]], wl["M"], smo.SIGNMUON_POST_POLAR, True)
+
+
+def test_plan_tables_size_query_and_errors():
+    import ctypes
+    arr = (ctypes.c_int64 * 2)(4, 6)
+    need = ctypes.c_int64(0)
+    assert smo._lib.signmuon_plan_tables(arr, 1, 2, 5, 0, 1, 0, None, 0, ctypes.byref(need)) == 0
+    assert need.value > 2
+    small = ctypes.create_string_buffer(8)
+    assert smo._lib.signmuon_plan_tables(arr, 1, 2, 5, 0, 1, 0, small, 8, ctypes.byref(need)) == \
+        smo.SIGNMUON_E_INVALID
+    with pytest.raises(smo.SignMuonError):
+        smo.signmuon_plan_tables([(0, 4)], 2)
