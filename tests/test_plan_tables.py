@@ -110,6 +110,9 @@ def _check(shapes, M, flags, spectral):
     assert t["prob_g"] == gs * M
     assert t["u_elems_one"] == sum(gs) and t["u_elems"] == M * sum(gs)
     _disjoint_inside([(u, u + g) for u, g in zip(t["uoff"], t["prob_g"])], t["u_elems"])
+    # the one-problem-set power iteration (worker 0's offsets) also runs on the
+    # warm-start buffer of u_elems_one floats
+    _disjoint_inside([(u, u + g) for u, g in zip(t["uoff"][:n], t["prob_g"][:n])], t["u_elems_one"])
     for p, aoff in enumerate(t["prob_aoff"]):
         w, i = divmod(p, n)
         mat = t["mats"][i]
