@@ -82,8 +82,9 @@ typedef struct signmuon_ctx* signmuon_t;
  *                    state per (worker, matrix) for the M-worker PolarNS (signmuon_step and
  *                    signmuon_polar share it) and one per matrix for the post-vote,
  *                    normalised-sign and Muon-baseline PolarNS.  A zero or non-finite state
- *                    (the first call, a zero matrix, a failed step) starts cold.  The state
- *                    is not part of get/set_momentum.  No effect with SIGNMUON_SCALE_FRO. */
+ *                    (the first call, a zero matrix, a failed step) starts cold.  A
+ *                    checkpoint saves the state with signmuon_get/set_pi_state (it is not
+ *                    part of get/set_momentum).  No effect with SIGNMUON_SCALE_FRO. */
 #define SIGNMUON_TIE_PLUS          (1u << 7)
 #define SIGNMUON_POLAR_AFTER_ONLY  (1u << 8)
 #define SIGNMUON_MUON_MEAN         (1u << 9)
@@ -269,6 +270,14 @@ int signmuon_polar(signmuon_t h, const float* const* X, float* const* U);
  * ---------------------------------------------------------------------- */
 int signmuon_get_momentum(signmuon_t h, int m, float* dst);
 int signmuon_set_momentum(signmuon_t h, int m, const float* src);
+/* The warm power-iteration state of a SIGNMUON_PI_WARM handle, the rest of
+ * what a checkpoint needs besides W and the momentum: which = 0 for the
+ * M-worker problems (signmuon_info out[6] floats), 1 for the one-problem-set
+ * PolarNS (out[7] floats).  dst / src are device float buffers of that size.
+ * A zero state makes the next power iteration start cold.  E_UNSUPPORTED
+ * without SIGNMUON_PI_WARM. */
+int signmuon_get_pi_state(signmuon_t h, int which, float* dst);
+int signmuon_set_pi_state(signmuon_t h, int which, const float* src);
 int signmuon_get_polar(signmuon_t h, int m, float* dst);
 int signmuon_get_signs(signmuon_t h, int m, uint8_t* dst);
 int signmuon_get_ternary_signs(signmuon_t h, int m, int8_t* dst);
@@ -293,7 +302,9 @@ int signmuon_set_ns_coeffs(signmuon_t h, const float* coeffs, int n);
 int signmuon_sync(signmuon_t h);
 
 /* Sizes: out[0]=d, out[1]=packed bytes per worker, out[2]=device bytes owned
- * by the handle, out[3]=number of shape groups, out[4]=M, out[5]=n_mats. */
+ * by the handle, out[3]=number of shape groups, out[4]=M, out[5]=n_mats,
+ * out[6]=power-iteration state floats of the M-worker problems,
+ * out[7]=those of one problem set (n <= 8 values are written). */
 int signmuon_info(signmuon_t h, int64_t* out, int n);
 
 /* Host-only planning (no GPU needed): same outputs as signmuon_info for a

@@ -52,7 +52,7 @@ EXPORTED = [
     "signmuon_profile", "signmuon_profile_read", "signmuon_get_gram",
     "signmuon_spectral_norm_noalloc", "signmuon_sign_ternary", "signmuon_vote_ternary",
     "signmuon_get_ternary_signs", "signmuon_local_signs", "signmuon_vote_step", "signmuon_sums_step",
-    "signmuon_plan_tables",
+    "signmuon_plan_tables", "signmuon_get_pi_state", "signmuon_set_pi_state",
 ]
 PROF_KINDS = ["momentum", "norm_finalize", "ns_gram", "ns_square", "ns_apply", "power_iter", "pack",
               "vote", "stage", "post_gram", "post_square", "post_apply", "update", "k0_scale"]
@@ -79,6 +79,8 @@ def _load():
         "signmuon_sign_ternary": (I, [P, P, I64, P]),
         "signmuon_vote_ternary": (I, [P, PP, I64, P, P]),
         "signmuon_get_ternary_signs": (I, [P, I, P]),
+        "signmuon_get_pi_state": (I, [P, I, P]),
+        "signmuon_set_pi_state": (I, [P, I, P]),
         "signmuon_local_signs": (I, [P, P, PP, P, I64]),
         "signmuon_vote_step": (I, [P, P, P, I64, I, F]),
         "signmuon_sums_step": (I, [P, P, P, F]),
@@ -226,6 +228,14 @@ def signmuon_set_momentum(h, m, src):
     _check(h, _lib.signmuon_set_momentum(h, int(m), _ptr(src)))
 
 
+def signmuon_get_pi_state(h, which, dst):
+    _check(h, _lib.signmuon_get_pi_state(h, int(which), _ptr(dst)))
+
+
+def signmuon_set_pi_state(h, which, src):
+    _check(h, _lib.signmuon_set_pi_state(h, int(which), _ptr(src)))
+
+
 def signmuon_get_polar(h, m, dst):
     _check(h, _lib.signmuon_get_polar(h, int(m), _ptr(dst)))
 
@@ -267,19 +277,22 @@ def signmuon_sync(h):
     _check(h, _lib.signmuon_sync(h))
 
 
+INFO_KEYS = ["d", "packed_bytes", "device_bytes", "groups", "M", "n_mats", "pi_state_workers", "pi_state_single"]
+
+
 def signmuon_info(h):
-    out = (ctypes.c_int64 * 6)()
-    _check(h, _lib.signmuon_info(h, out, 6))
-    return dict(zip(["d", "packed_bytes", "device_bytes", "groups", "M", "n_mats"], list(out)))
+    out = (ctypes.c_int64 * 8)()
+    _check(h, _lib.signmuon_info(h, out, 8))
+    return dict(zip(INFO_KEYS, list(out)))
 
 
 def signmuon_plan(shapes, M, K=5, scale=SIGNMUON_SCALE_FRO, P=1, flags=0):
     if isinstance(scale, str):
         scale = {"fro": SIGNMUON_SCALE_FRO, "spectral": SIGNMUON_SCALE_SPECTRAL}[scale]
     arr, n = _shapes_arr(shapes)
-    out = (ctypes.c_int64 * 6)()
-    _check(None, _lib.signmuon_plan(arr, n, int(M), int(K), int(scale), int(P), int(flags), out, 6))
-    return dict(zip(["d", "packed_bytes", "device_bytes", "groups", "M", "n_mats"], list(out)))
+    out = (ctypes.c_int64 * 8)()
+    _check(None, _lib.signmuon_plan(arr, n, int(M), int(K), int(scale), int(P), int(flags), out, 8))
+    return dict(zip(INFO_KEYS, list(out)))
 
 
 def signmuon_plan_tables(shapes, M, K=5, scale=SIGNMUON_SCALE_FRO, P=1, flags=0):
@@ -389,6 +402,12 @@ class SignMuon:
 
     def get_polar(self, m, dst):
         signmuon_get_polar(self.h, m, dst)
+
+    def get_pi_state(self, which, dst):
+        signmuon_get_pi_state(self.h, which, dst)
+
+    def set_pi_state(self, which, src):
+        signmuon_set_pi_state(self.h, which, src)
 
     def get_signs(self, m, dst):
         signmuon_get_signs(self.h, m, dst)

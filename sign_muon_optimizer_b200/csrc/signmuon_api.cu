@@ -438,8 +438,8 @@ const char* signmuon_last_error(signmuon_t h) { return h ? h->err.c_str() : g_no
 int64_t signmuon_kernel_launches(void) { return sm::g_launches.load(); }
 
 static void fill_info(const Plan& p, int64_t* out, int n) {
-  const int64_t v[6] = {p.d, p.nb, p.device_bytes, (int64_t)p.groups.size(), p.M, p.n_mats};
-  for (int i = 0; i < n && i < 6; ++i) out[i] = v[i];
+  const int64_t v[8] = {p.d, p.nb, p.device_bytes, (int64_t)p.groups.size(), p.M, p.n_mats, p.u_elems, p.u_elems_one};
+  for (int i = 0; i < n && i < 8; ++i) out[i] = v[i];
 }
 
 int signmuon_plan(const int64_t* shapes, int n_mats, int M, int K, int scale, int P, unsigned flags,
@@ -1035,6 +1035,43 @@ int signmuon_set_momentum(signmuon_t h, int m, const float* src) {
   if (m < 0 || m >= h->M || !src) return fail(h, SIGNMUON_E_INVALID, "bad worker index or null src");
   CK(h, cudaMemcpyAsync(h->Mom + (int64_t)m * h->plan.dpad, src, (size_t)h->plan.d * 4, cudaMemcpyDeviceToDevice,
                         h->stream));
+  return SIGNMUON_OK;
+}
+
+// the warm power-iteration state: which = 0 (M-worker problems), 1 (one problem set)
+static int pi_state_buffer(signmuon_t h, int which, float** buf, int64_t* n) {
+  if (!(h->flags & SIGNMUON_PI_WARM)) return fail(h, SIGNMUON_E_UNSUPPORTED, "the handle has no SIGNMUON_PI_WARM state");
+  if (which == 0) {
+    *buf = h->pi_u;
+    *n = h->plan.u_elems;
+  } else if (which == 1) {
+    *buf = h->pi_u1;
+    *n = h->plan.u_elems_one;
+  } else {
+    return fail(h, SIGNMUON_E_INVALID, "which must be 0 (workers) or 1 (one problem set)");
+  }
+  return SIGNMUON_OK;
+}
+
+int signmuon_get_pi_state(signmuon_t h, int which, float* dst) {
+  int rc = check_handle(h, true);
+  if (rc) return rc;
+  float* buf = nullptr;
+  int64_t n = 0;
+  if ((rc = pi_state_buffer(h, which, &buf, &n))) return rc;
+  if (!dst) return fail(h, SIGNMUON_E_INVALID, "null dst");
+  CK(h, cudaMemcpyAsync(dst, buf, (size_t)n * 4, cudaMemcpyDeviceToDevice, h->stream));
+  return SIGNMUON_OK;
+}
+
+int signmuon_set_pi_state(signmuon_t h, int which, const float* src) {
+  int rc = check_handle(h, true);
+  if (rc) return rc;
+  float* buf = nullptr;
+  int64_t n = 0;
+  if ((rc = pi_state_buffer(h, which, &buf, &n))) return rc;
+  if (!src) return fail(h, SIGNMUON_E_INVALID, "null src");
+  CK(h, cudaMemcpyAsync(buf, src, (size_t)n * 4, cudaMemcpyDeviceToDevice, h->stream));
   return SIGNMUON_OK;
 }
 

@@ -100,3 +100,58 @@ def test_warm_state_restarts_after_a_zero_matrix(precision):
     cold = _handle(M, 3, 2, precision)
     cold.step(torch.zeros(d, device="cuda"), G, 0.01)
     assert np.array_equal(h.get_scales(), cold.get_scales())
+
+
+@pytest.mark.parametrize("precision", ["fp32", "bf16"])
+def test_warm_checkpoint_resume_bit_exact(precision):
+    """A warm-started handle's checkpoint is W, the momentum and the
+    power-iteration state (signmuon_get/set_pi_state): two steps, a save,
+    and two more on a fresh handle equal four straight steps bit for bit;
+    restoring only the momentum restarts the power iteration cold."""
+    M, K, P, seed = 2, 3, 1, 87
+    flags = smo.SIGNMUON_PI_WARM | smo.SIGNMUON_POST_POLAR
+    d = synth.numel(SHAPES)
+
+    def grads(step):
+        return [dev(g) for g in synth.gradients(SHAPES, M, 1.0, step=step, config_id=seed)]
+
+    straight = _handle(M, K, P, precision, flags, beta=0.9)
+    Wa = dev(synth.weights0(SHAPES, seed))
+    for step in range(1, 5):
+        straight.step(Wa, grads(step), 0.01)
+
+    first = _handle(M, K, P, precision, flags, beta=0.9)
+    Wb = dev(synth.weights0(SHAPES, seed))
+    for step in (1, 2):
+        first.step(Wb, grads(step), 0.01)
+    info = smo.signmuon_info(first.h)
+    assert info["pi_state_workers"] == M * sum(min(r, c) for r, c in SHAPES)
+    assert info["pi_state_single"] == sum(min(r, c) for r, c in SHAPES)
+    mom = [torch.zeros(d, device="cuda") for _ in range(M)]
+    for m in range(M):
+        first.get_momentum(m, mom[m])
+    s0 = torch.zeros(info["pi_state_workers"], device="cuda")
+    s1 = torch.zeros(info["pi_state_single"], device="cuda")
+    first.get_pi_state(0, s0)
+    first.get_pi_state(1, s1)
+    W_saved = Wb.clone()
+
+    resumed = _handle(M, K, P, precision, flags, beta=0.9)
+    cold = _handle(M, K, P, precision, flags, beta=0.9)
+    W_cold = W_saved.clone()
+    for m in range(M):
+        resumed.set_momentum(m, mom[m])
+        cold.set_momentum(m, mom[m])
+    resumed.set_pi_state(0, s0)
+    resumed.set_pi_state(1, s1)
+    for step in (3, 4):
+        resumed.step(W_saved, grads(step), 0.01)
+        cold.step(W_cold, grads(step), 0.01)
+    assert np.array_equal(host(W_saved).view(np.uint32), host(Wa).view(np.uint32))
+    assert np.array_equal(resumed.get_scales(), straight.get_scales())
+    assert not np.array_equal(cold.get_scales(), straight.get_scales())
+    # a handle without the flag has no state to give
+    plain = _handle(M, K, P, precision)
+    with pytest.raises(smo.SignMuonError) as ei:
+        plain.get_pi_state(0, s0)
+    assert ei.value.status == smo.SIGNMUON_E_UNSUPPORTED
