@@ -14,6 +14,9 @@
 //          tall: Aop = X (K-major), Bop(k,j) = P[j][k] (K-major), M = rows, N = cols
 // where P is A (cubic) or B (quintic).  "K-major" means consecutive k are
 // adjacent in memory; "MN-major" means consecutive i (or j) are.
+//
+// The functions below are host-callable too, so that a CPU program can check
+// the decoding against the planner's tile lists.
 #pragma once
 #include "common.cuh"
 
@@ -27,14 +30,14 @@ struct TileCoord {
   int Mdim, Ndim, Kdim, BN;
 };
 
-__device__ __forceinline__ const TileGroup* tile_table(const GemmArgs& a) {
+__host__ __device__ __forceinline__ const TileGroup* tile_table(const GemmArgs& a) {
   return a.param_tables ? a.ptiles : a.tiles;
 }
-__device__ __forceinline__ const GroupInfo& group_info(const GemmArgs& a, int g) {
+__host__ __device__ __forceinline__ const GroupInfo& group_info(const GemmArgs& a, int g) {
   return a.param_tables ? a.pgroups[g] : a.groups[g];
 }
 
-__device__ __forceinline__ TileCoord decode_tile(const GemmArgs& a, int tile) {
+__host__ __device__ __forceinline__ TileCoord decode_tile(const GemmArgs& a, int tile) {
   const TileGroup* tiles = tile_table(a);
   int t = 0;
   while (t + 1 < a.n_tile_groups && tiles[t + 1].tile_start <= tile) ++t;
@@ -68,7 +71,7 @@ __device__ __forceinline__ TileCoord decode_tile(const GemmArgs& a, int tile) {
 }
 
 // problem id p = worker*n_mats + matrix, used for the per-problem coefficients
-__device__ __forceinline__ int problem_id(const GemmArgs& a, const GroupInfo& gi, int b, int* mat_out) {
+__host__ __device__ __forceinline__ int problem_id(const GemmArgs& a, const GroupInfo& gi, int b, int* mat_out) {
   const int w = b / gi.count;
   const int q = b - w * gi.count;
   const int mat = a.param_tables ? a.pgroup_mats[gi.first + q] : a.group_mats[gi.first + q];
@@ -77,8 +80,8 @@ __device__ __forceinline__ int problem_id(const GemmArgs& a, const GroupInfo& gi
 }
 
 // operand majorness (1 = MN-major) for an op/orientation
-__device__ __forceinline__ int a_is_mn(int op, int wide) { return (op == OP_GRAM && !wide) ? 1 : 0; }
-__device__ __forceinline__ int b_is_mn(int op, int wide) {
+__host__ __device__ __forceinline__ int a_is_mn(int op, int wide) { return (op == OP_GRAM && !wide) ? 1 : 0; }
+__host__ __device__ __forceinline__ int b_is_mn(int op, int wide) {
   return ((op == OP_GRAM && !wide) || (op == OP_APPLY && wide)) ? 1 : 0;
 }
 
