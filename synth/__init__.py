@@ -9,7 +9,7 @@ stay independent of one another.
 Workload shapes are stand-ins for the pages' models (the datasets and trained
 weights are not used; only the weight shapes are):
 
-* ``config1``: one 256x128 matrix, 3 workers, noise scale 0.5.
+* ``small_256x128``: one 256x128 matrix, 3 workers, noise scale 0.5.
 * ``resnet50``: the 54 conv/fc weights of ResNet-50, each conv flattened to
   out x (in*kh*kw), in torchvision module order (25,502,912 weights).
 * ``nanogpt``: 12 transformer layers x {qkv 2304x768, attn proj 768x768,
@@ -50,7 +50,7 @@ def _resnet50_shapes():
 RESNET50_SHAPES = _resnet50_shapes()
 NANOGPT_SHAPES = [(2304, 768), (768, 768), (3072, 768), (768, 3072)] * 12
 LLAMA_LAYER_SHAPES = [(4096, 4096)] * 32 + [(11008, 4096)] * 4
-CONFIG1_SHAPES = [(256, 128)]
+SMALL_256x128_SHAPES = [(256, 128)]
 SWEEP_SHAPES = {
     "single_8192": [(8192, 8192)],
     "batch64_1024": [(1024, 1024)] * 64,
@@ -58,10 +58,11 @@ SWEEP_SHAPES = {
 }
 
 # Per-workload run parameters (hyper-parameters not given for a workload take
-# config 1's values: beta=0.9, lambda=0.01, eta=0.02, eps=1e-7).
+# the small 256x128 workload's values: beta=0.9, lambda=0.01, eta=0.02,
+# eps=1e-7).
 WORKLOADS = {
-    "config1": dict(shapes=CONFIG1_SHAPES, M=3, sigma=0.5, K=5, scale="fro", P=1,
-                    order="cubic", precision="fp32", post_polar=False, steps=10),
+    "small_256x128": dict(shapes=SMALL_256x128_SHAPES, M=3, sigma=0.5, K=5, scale="fro", P=1,
+                          order="cubic", precision="fp32", post_polar=False, steps=10),
     "resnet50": dict(shapes=RESNET50_SHAPES, M=4, sigma=1.0, K=5, scale="spectral", P=2,
                      order="cubic", precision="bf16", post_polar=False, steps=20),
     "nanogpt": dict(shapes=NANOGPT_SHAPES, M=8, sigma=2.0, K=5, scale="spectral", P=2,

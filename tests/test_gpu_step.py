@@ -115,8 +115,8 @@ def _compare_step(shapes, M, gpu, want, precision, post_polar, tie=0):
 
 
 @pytest.mark.parametrize("precision", ["fp32", "bf16"])
-def test_step_config1_single(precision):
-    shapes = synth.CONFIG1_SHAPES
+def test_step_small_256x128_single(precision):
+    shapes = synth.SMALL_256x128_SHAPES
     h, gpu, want = _run_one_step(shapes, 3, 0.5, 5, "fro", 1, precision, False, seed=1)
     _compare_step(shapes, 3, gpu, want, precision, False)
 
@@ -136,11 +136,11 @@ def test_step_quintic_fp32():
     _compare_step(shapes, 2, gpu, want, "fp32", False)
 
 
-def test_step_config1_ten_steps_drift():
-    """Config 1 end to end: 10 steps on the GPU (fp32 NS) and in the oracle,
+def test_step_small_256x128_ten_steps_drift():
+    """The small 256x128 workload end to end: 10 steps on the GPU (fp32 NS) and in the oracle,
     each from its own state; the trajectories may part only where a sign was
     within rounding of zero."""
-    shapes = synth.CONFIG1_SHAPES
+    shapes = synth.SMALL_256x128_SHAPES
     M = 3
     h = smo.SignMuon(shapes, M, beta=HP["beta"], lam=HP["lam"], K=5, eps=HP["eps"], scale="fro",
                      flags=smo.SIGNMUON_NS_FP32)
