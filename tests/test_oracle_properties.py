@@ -101,3 +101,38 @@ def test_polar_of_a_well_conditioned_matrix_reaches_the_svd_factor(r, c, seed):
     assert np.max(np.abs(got - polar)) < 1e-9
     # the signs of the result are what the one-bit and ternary paths send
     assert np.array_equal(ref.sign_bits(got), got >= 0)
+
+
+@SLOW
+@given(st.integers(2, 5), st.integers(0, 2 ** 31 - 1), st.booleans(), st.sampled_from(["bits", "ternary"]))
+def test_step_is_symmetric_in_the_workers(M, seed, post_polar, signs):
+    # the vote is a sum: any order of the workers gives the same W and D
+    rng = np.random.default_rng(seed)
+    shapes = [(3, 5), (4, 2)]
+    d = 15 + 8
+    W = (0.02 * rng.standard_normal(d)).astype(np.float32)
+    G = [rng.standard_normal(d) for _ in range(M)]
+    mom = [0.3 * rng.standard_normal(d) for _ in range(M)]
+    kw = dict(beta=0.9, lam=0.01, eta=0.02, K=3, eps=1e-7, scale="spectral", P=2, post_polar=post_polar,
+              signs=signs)
+    a = ref.step(W, G, mom, shapes, **kw)
+    perm = rng.permutation(M)
+    b = ref.step(W, [G[i] for i in perm], [mom[i] for i in perm], shapes, **kw)
+    assert np.array_equal(a["sums"], b["sums"]) and np.array_equal(a["W"], b["W"])
+    assert np.array_equal(a["D32"], b["D32"])
+
+
+@SLOW
+@given(st.integers(1, 6), st.integers(0, 2 ** 31 - 1), st.sampled_from([0, 1]))
+def test_identical_workers_vote_like_one(M, seed, tie):
+    # M copies of one worker: every sum is +-M (or 0 only where its ternary
+    # sign is 0), so the majority, D and W are the one-worker step's
+    rng = np.random.default_rng(seed)
+    shapes = [(5, 3)]
+    W = (0.02 * rng.standard_normal(15)).astype(np.float32)
+    g = rng.standard_normal(15)
+    kw = dict(beta=0.5, lam=0.01, eta=0.05, K=2, eps=1e-7, scale="fro", tie=tie)
+    one = ref.step(W, [g], [np.zeros(15)], shapes, **kw)
+    many = ref.step(W, [g] * M, [np.zeros(15)] * M, shapes, **kw)
+    assert np.array_equal(many["sums"], M * one["sums"])
+    assert np.array_equal(many["majority"], one["majority"]) and np.array_equal(many["W"], one["W"])
