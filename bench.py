@@ -531,6 +531,52 @@ def run_secondary(args):
     return 0
 
 
+def run_collectives(args):
+    """The exchange of the multi-GPU step on its own (one JSON line from rank
+    0; run under torchrun with N >= 2): the all-gather of packed signs and
+    the SUM all-reduce of int8 sums timed over NCCL at message sizes from
+    1 KB to 256 MB (max over ranks), the alpha-beta fit t = alpha + beta * n
+    of each, and the fitted time of the nanoGPT payloads (ceil(d/8) bytes
+    per rank gathered, d int8 bytes reduced) next to a direct measurement."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    from sign_muon_optimizer_b200.dist import fit_alpha_beta, time_collective
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world < 2:
+        print(json.dumps({"metric": "exchange alpha-beta fit", "unavailable": "needs 2 or more ranks (torchrun)"}),
+              flush=True)
+        return 0
+    if torch.cuda.is_available():
+        torch.cuda.set_device(local)
+        device = f"cuda:{local}"
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        sizes = [1 << k for k in range(10, 29, 2)]
+    else:  # the same exchange over gloo on the host (a check of this code path)
+        device = "cpu"
+        dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=120))
+        sizes = [1 << k for k in range(10, 21, 2)]
+    packed, sums8 = (D + 7) // 8, D
+    out = {"metric": "exchange alpha-beta fit", "n_gpus": world, "device": device, "sizes_bytes": sizes}
+    for kind, payload in (("allgather", packed), ("allreduce", sums8)):
+        ts = time_collective(kind, sizes, reps=5, device=device)
+        alpha, beta = fit_alpha_beta(sizes, ts)
+        direct = time_collective(kind, [payload], reps=2, device=device)[0]
+        out[kind] = {"seconds": ts, "alpha_s": alpha, "beta_s_per_byte": beta,
+                     "GB_per_s": (1.0 / beta / 1e9) if beta > 0 else None,
+                     "nanogpt_payload_bytes": payload, "fitted_s": alpha + beta * payload, "measured_s": direct}
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    dist.barrier()
+    dist.destroy_process_group()
+    return 0
+
+
 def run_capture(args):
     """Profiler-capture mode (prints no bench line): the same step on the first
     L transformer layers of the nanoGPT shapes, M=8, a few steps."""
@@ -562,11 +608,13 @@ def main():
                     help="profiler capture mode on the first L layers; prints no bench line")
     ap.add_argument("--workload", default="nanogpt",
                     choices=["nanogpt", "llama_vote", "vote_100m", "ns_sweep", "resnet50", "ternary_vote", "variants",
-                             "all"],
+                             "collectives", "all"],
                     help="nanogpt: the headline line; the others print secondary measurements only")
     args = ap.parse_args()
     if args.capture_layers > 0:
         return run_capture(args)
+    if args.workload == "collectives":
+        return run_collectives(args)
     if args.workload != "nanogpt":
         return run_secondary(args)
     if args.warmup < 3:

@@ -90,3 +90,36 @@ def test_hbm_bytes_counts():
 
 def test_cpu_sample_is_one_144th():
     assert bench.CPU_SCALE == 144.0
+
+
+def _collectives_rank(rank, world, port, q):
+    import contextlib
+    import io
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    buf = io.StringIO()
+    with contextlib.redirect_stdout(buf):
+        rc = bench.run_collectives(None)
+    q.put((rank, rc, buf.getvalue()))
+
+
+def test_collectives_workload_over_gloo_world2():
+    """bench.py --workload collectives on two host ranks (gloo): one JSON line
+    from rank 0 with an alpha-beta fit per exchange."""
+    import json
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_collectives_rank, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = dict((r, (rc, out)) for r, rc, out in (q.get(timeout=300) for _ in range(2)))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert res[0][0] == 0 and res[1][0] == 0 and res[1][1] == ""
+    line = json.loads(res[0][1].strip().splitlines()[-1])
+    assert line["n_gpus"] == 2 and line["device"] == "cpu"
+    for kind in ("allgather", "allreduce"):
+        assert len(line[kind]["seconds"]) == len(line["sizes_bytes"])
+        assert line[kind]["measured_s"] > 0 and line[kind]["nanogpt_payload_bytes"] > 0
