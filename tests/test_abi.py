@@ -109,3 +109,50 @@ def test_plan_accepts_the_sign_wire_variants_and_counts_ternary_bytes():
     assert smo.SIGNMUON_PI_WARM == 1 << 12
     p = smo.signmuon_plan(shapes, 5, 5, "spectral", 2, 1 << 12)
     assert p["device_bytes"] == base["device_bytes"] + 4 * (8 + 16)
+
+
+_NULL_HANDLE_CALLS = """
+import ctypes, sys
+sys.path.insert(0, {root!r})
+import sign_muon_optimizer_b200 as smo
+L = smo._lib
+pp = (ctypes.c_void_p * 1)()
+calls = {{
+    "signmuon_step": (None, None, pp, 0.1), "signmuon_step_host": (None, None, pp, 0.1),
+    "signmuon_local_signs": (None, None, pp, None, 16), "signmuon_vote_step": (None, None, None, 16, 2, 0.1),
+    "signmuon_sums_step": (None, None, None, 0.1), "signmuon_vote": (None, pp, 8, None, None),
+    "signmuon_vote_ternary": (None, pp, 8, None, None), "signmuon_pack": (None, None, 8, None),
+    "signmuon_sign_ternary": (None, None, 8, None), "signmuon_apply_update": (None, None, None, 8, 0.1),
+    "signmuon_polar": (None, pp, pp), "signmuon_get_momentum": (None, 0, None),
+    "signmuon_set_momentum": (None, 0, None), "signmuon_get_pi_state": (None, 0, None),
+    "signmuon_set_pi_state": (None, 0, None), "signmuon_get_polar": (None, 0, None),
+    "signmuon_get_signs": (None, 0, None), "signmuon_get_ternary_signs": (None, 0, None),
+    "signmuon_get_direction": (None, None), "signmuon_get_scales": (None, None),
+    "signmuon_set_ns_coeffs": (None, None, 2), "signmuon_sync": (None,), "signmuon_info": (None, None, 6),
+    "signmuon_profile": (None, 1), "signmuon_profile_read": (None, None, None, 1),
+    "signmuon_get_gram": (None, 0, 0, None),
+}}
+bad = []
+for name, args in calls.items():
+    rc = getattr(L, name)(*args)
+    if rc != smo.SIGNMUON_E_INVALID or not L.signmuon_last_error(None):
+        bad.append((name, rc))
+L.signmuon_destroy(None)
+print("BAD", bad) if bad else print("ALL", len(calls))
+"""
+
+
+def test_every_entry_point_rejects_a_null_handle():
+    # in a child process, so that a crash would fail this test, not the run
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    res = subprocess.run([sys.executable, "-c", _NULL_HANDLE_CALLS.format(root=root)], capture_output=True,
+                         text=True, timeout=120)
+    assert res.returncode == 0, res.stderr[-2000:]
+    assert res.stdout.strip().startswith("ALL"), res.stdout
+    import sign_muon_optimizer_b200 as smo
+    declared = [n for n in smo.EXPORTED if n not in (
+        "signmuon_init", "signmuon_plan", "signmuon_plan_tables", "signmuon_kernel_launches",
+        "signmuon_last_error", "signmuon_status_string", "signmuon_destroy", "signmuon_spectral_norm_noalloc")]
+    assert int(res.stdout.split()[1]) == len(declared)   # every handle-taking call is covered
