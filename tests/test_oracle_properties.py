@@ -136,3 +136,24 @@ def test_identical_workers_vote_like_one(M, seed, tie):
     many = ref.step(W, [g] * M, [np.zeros(15)] * M, shapes, **kw)
     assert np.array_equal(many["sums"], M * one["sums"])
     assert np.array_equal(many["majority"], one["majority"]) and np.array_equal(many["W"], one["W"])
+
+
+@SLOW
+@given(st.integers(1, 7), st.integers(1, 7), st.integers(1, 4), st.integers(0, 2 ** 31 - 1))
+def test_normalised_sign_step_norm_bounds(r, c, P, seed):
+    # D = maj / (s + eps): the power-iteration estimate never exceeds sigma_max,
+    # so the spectral-normalised D has ||D||_2 >= 1 - eps/sigma (any P); the
+    # Frobenius norm bounds sigma_max from above, so that D has ||D||_2 < 1
+    rng = np.random.default_rng(seed)
+    maj = rng.integers(-1, 2, size=(r, c)).astype(np.float64)
+    if not maj.any():
+        maj[0, 0] = 1.0
+    eps = 1e-9
+    for scale in ("spectral", "fro"):
+        D = ref.normalize_flat(maj.ravel(), [(r, c)], eps, scale, P).reshape(r, c)
+        n2 = np.linalg.svd(D, compute_uv=False)[0]
+        if scale == "spectral":
+            assert n2 >= 1.0 - 1e-6
+        else:
+            assert n2 <= 1.0
+        assert np.array_equal(np.sign(D), maj)      # a positive rescaling only
