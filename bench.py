@@ -443,24 +443,35 @@ def run_secondary(args):
             del sums, maj
         del signs
         torch.cuda.empty_cache()
-    if args.workload in ("ns_sweep", "all"):
-        for name, shp in synth.SWEEP_SHAPES.items():
-            Mw = 8
-            h = smo.SignMuon(shp, Mw, beta=0.9, lam=0.0, K=5, eps=1e-7, scale="spectral", P=2, flags=0,
-                             stream=stream.cuda_stream)
-            X = synth.device_gaussian(h.d, Mw, seed=5)
-            U = torch.empty_like(X)
-            xs, us = [X[m] for m in range(Mw)], [U[m] for m in range(Mw)]
-            ms = _events_time(lambda: h.polar(xs, us), 3, stream)
-            fl = sum(4.0 * min(r, c) ** 2 * max(r, c) for r, c in shp) * 5 * Mw
-            tf = fl / (ms / 1e3) / 1e12
-            lines.append({"metric": f"NS TFLOP/s ({name}, M=8, K=5 cubic bf16, spectral P=2)", "value": tf,
-                          "unit": "TFLOP/s", "frac_of_bf16_sustained": tf / pk["bf16_tflops_sustained"],
-                          "frac_of_bf16_burst": tf / pk["bf16_tflops"], "peak_kind": pk_kind, "ms": ms,
-                          "flops": fl})
-            h.close()
-            del X, U
-            torch.cuda.empty_cache()
+    if args.workload in ("ns_sweep", "ns_sweep_full", "all"):
+        # ns_sweep: K = 5 cubic bf16; ns_sweep_full adds K = 10, quintic and
+        # the fp32 SIMT path (the sweep's full grid)
+        grid = [(5, "cubic", "bf16")]
+        if args.workload == "ns_sweep_full":
+            grid += [(10, "cubic", "bf16"), (5, "quintic", "bf16"), (5, "cubic", "fp32")]
+        for K, order, prec in grid:
+            for name, shp in synth.SWEEP_SHAPES.items():
+                Mw = 8
+                fl_ns = (smo.SIGNMUON_NS_QUINTIC if order == "quintic" else 0) | \
+                        (smo.SIGNMUON_NS_FP32 if prec == "fp32" else 0)
+                h = smo.SignMuon(shp, Mw, beta=0.9, lam=0.0, K=K, eps=1e-7, scale="spectral", P=2, flags=fl_ns,
+                                 stream=stream.cuda_stream)
+                X = synth.device_gaussian(h.d, Mw, seed=5)
+                U = torch.empty_like(X)
+                xs, us = [X[m] for m in range(Mw)], [U[m] for m in range(Mw)]
+                ms = _events_time(lambda: h.polar(xs, us), 3, stream)
+                # cubic 4 m^2 n per iteration; quintic adds the 2 m^3 of A^2
+                per_it = sum(4.0 * min(r, c) ** 2 * max(r, c) + (2.0 * min(r, c) ** 3 if order == "quintic" else 0.0)
+                             for r, c in shp)
+                fl = per_it * K * Mw
+                tf = fl / (ms / 1e3) / 1e12
+                lines.append({"metric": f"NS TFLOP/s ({name}, M=8, K={K} {order} {prec}, spectral P=2)", "value": tf,
+                              "unit": "TFLOP/s", "frac_of_bf16_sustained": tf / pk["bf16_tflops_sustained"],
+                              "frac_of_bf16_burst": tf / pk["bf16_tflops"], "peak_kind": pk_kind, "ms": ms,
+                              "flops": fl})
+                h.close()
+                del X, U
+                torch.cuda.empty_cache()
     if args.workload in ("ternary_vote", "all"):
         # the int8 ternary wire's vote: d bytes per worker instead of d/8
         shapes = synth.LLAMA_LAYER_SHAPES
@@ -607,8 +618,8 @@ def main():
     ap.add_argument("--capture-layers", type=int, default=0,
                     help="profiler capture mode on the first L layers; prints no bench line")
     ap.add_argument("--workload", default="nanogpt",
-                    choices=["nanogpt", "llama_vote", "vote_100m", "ns_sweep", "resnet50", "ternary_vote", "variants",
-                             "collectives", "all"],
+                    choices=["nanogpt", "llama_vote", "vote_100m", "ns_sweep", "ns_sweep_full", "resnet50",
+                             "ternary_vote", "variants", "collectives", "all"],
                     help="nanogpt: the headline line; the others print secondary measurements only")
     args = ap.parse_args()
     if args.capture_layers > 0:
