@@ -53,8 +53,10 @@ typedef struct signmuon_ctx* signmuon_t;
 #define SIGNMUON_NS_FP32     (1u << 0) /* fp32 Newton-Schulz (SIMT) instead of bf16 tcgen05 tensor cores */
 #define SIGNMUON_NS_QUINTIC  (1u << 1) /* quintic NS X(15/8 I - 10/8 X^T X + 3/8 (X^T X)^2) */
 #define SIGNMUON_POST_POLAR  (1u << 2) /* post-vote local polar step: D = PolarNS(majority) */
-#define SIGNMUON_ACC_INT8    (1u << 3) /* signmuon_vote writes int8 sums (requires M <= 127) */
-#define SIGNMUON_ASYNC       (1u << 4) /* signmuon_step does not wait; signmuon_sync reports status */
+#define SIGNMUON_ACC_INT8    (1u << 3) /* int8 vote sums: signmuon_vote / signmuon_vote_ternary write
+                                          them and signmuon_sums_step reads them (M <= 127) */
+#define SIGNMUON_ASYNC       (1u << 4) /* step, polar, local_signs, vote_step and sums_step do not
+                                          wait; signmuon_sync reports their status */
 #define SIGNMUON_VOTE_ONLY   (1u << 5) /* allocate no step workspace: vote/pack/update calls only */
 #define SIGNMUON_KEEP_POLAR  (1u << 6) /* signmuon_step also writes U for signmuon_get_polar; without it
                                           the last Newton-Schulz GEMM of a step writes only the one-bit
