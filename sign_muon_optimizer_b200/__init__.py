@@ -347,7 +347,10 @@ class SignMuon:
         self.shapes = [(int(r), int(c)) for r, c in shapes]
         self.M = int(M)
         self.flags = int(flags)
-        self.h = signmuon_init(self.shapes, M, beta, lam, K, eps, scale, P, flags, stream)
+        # the CUDA stream the handle enqueues on (a cudaStream_t as an int; 0
+        # or None for the legacy default stream)
+        self.stream = stream if stream is not None else _default_stream()
+        self.h = signmuon_init(self.shapes, M, beta, lam, K, eps, scale, P, flags, self.stream)
         self.info = signmuon_info(self.h)
         self.d = self.info["d"]
 

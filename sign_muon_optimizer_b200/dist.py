@@ -25,6 +25,7 @@ same shapes, flags and exchange.
 """
 from __future__ import annotations
 
+import contextlib
 import time
 
 import numpy as np
@@ -65,6 +66,14 @@ class DistSignMuon:
         self.device = torch.device(device)
         self.local = torch.zeros(self.M_local * self.stride, dtype=torch.uint8, device=self.device)
         self._flag = torch.zeros(1, dtype=torch.int32, device=self.device)
+        # torch orders its collectives after the current stream; make that the
+        # handle's stream, so that the exchange waits for the library's kernels
+        # and the vote after it waits for the exchange
+        self._stream = None
+        if self.device.type == "cuda":
+            ptr = getattr(self.opt, "stream", None)
+            self._stream = (torch.cuda.ExternalStream(ptr, device=self.device) if ptr
+                            else torch.cuda.default_stream(self.device))
         flags = int(getattr(self.opt, "flags", flags))
         self.ternary = bool(flags & SIGNMUON_TERNARY)
         if exchange == "allgather":
@@ -92,6 +101,10 @@ class DistSignMuon:
         - exchange_ms: the all-gather or the SUM all-reduce;
         - finish_ms: the vote or majority, the post-vote step and the update;
         - total_ms: the whole step."""
+        with torch.cuda.stream(self._stream) if self._stream is not None else contextlib.nullcontext():
+            self._step(W, G, eta, clocks)
+
+    def _step(self, W, G, eta, clocks):
         clk = _PhaseClock(self.device) if clocks is not None else None
         t0 = clk.mark() if clk else None
         err = None
