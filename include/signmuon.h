@@ -19,6 +19,9 @@
  *     are flattened to out x (in*kh*kw) by the caller.
  *   - Work is enqueued on the CUDA stream given at init.  Calls return without
  *     waiting for the GPU, except where a call says otherwise.
+ *   - A handle belongs to the device that was current at signmuon_init.  A
+ *     call on it makes that device current while it runs and gives the
+ *     caller's current device back before it returns.
  *   - The caller owns W, G, signs, sums, majority and every buffer it passes;
  *     the library owns the momentum, the Newton-Schulz workspace and the
  *     packed sign buffers of the step.

@@ -404,11 +404,30 @@ int finish(signmuon_t h, bool wait) {
   return SIGNMUON_OK;
 }
 
+// Makes the handle's device current for the duration of one entry point and
+// gives the caller's current device back on return, so that a call on a
+// handle of another GPU leaves the caller's device selection as it was.
+struct DeviceGuard {
+  int saved = -1;
+  explicit DeviceGuard(signmuon_t h) {
+    if (h == nullptr) return;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+      cudaGetLastError();
+      dev = -1;
+    }
+    if (dev != h->device && cudaSetDevice(h->device) == cudaSuccess) saved = dev;
+  }
+  ~DeviceGuard() {
+    if (saved >= 0) cudaSetDevice(saved);
+  }
+  DeviceGuard(const DeviceGuard&) = delete;
+  DeviceGuard& operator=(const DeviceGuard&) = delete;
+};
+
 int check_handle(signmuon_t h, bool need_step) {
   if (h == nullptr) return fail(nullptr, SIGNMUON_E_INVALID, "null handle");
   if (need_step && h->vote_only) return fail(h, SIGNMUON_E_UNSUPPORTED, "handle was created with SIGNMUON_VOTE_ONLY");
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev != h->device) cudaSetDevice(h->device);
   return SIGNMUON_OK;
 }
 
@@ -537,6 +556,7 @@ int signmuon_plan_tables(const int64_t* shapes, int n_mats, int M, int K, int sc
 
 void signmuon_destroy(signmuon_t h) {
   if (!h) return;
+  DeviceGuard dev_guard(h);
   cudaStreamSynchronize(h->stream);
   for (cudaEvent_t e : h->ev_pool) cudaEventDestroy(e);
   for (void* q : h->allocs) cudaFree(q);
@@ -685,6 +705,7 @@ int signmuon_init(signmuon_t* out, const int64_t* shapes, int n_mats, int M, flo
 }
 
 int signmuon_set_ns_coeffs(signmuon_t h, const float* c, int n) {
+  DeviceGuard dev_guard(h);
   int rc = check_handle(h, false);
   if (rc) return rc;
   if (c == nullptr) return fail(h, SIGNMUON_E_INVALID, "null coefficients");
@@ -777,6 +798,7 @@ static void vote_part(signmuon_t h, float* W, const uint8_t* src, int64_t stride
 
 int signmuon_step(signmuon_t h, float* W, const float* const* G, float eta) {
   NvtxRange range("signmuon_step");
+  DeviceGuard dev_guard(h);
   int rc = check_handle(h, true);
   if (rc) return rc;
   const Plan& p = h->plan;
@@ -825,6 +847,7 @@ int signmuon_step(signmuon_t h, float* W, const float* const* G, float eta) {
 
 int signmuon_local_signs(signmuon_t h, const float* W, const float* const* G, uint8_t* signs, int64_t stride) {
   NvtxRange range("signmuon_local_signs");
+  DeviceGuard dev_guard(h);
   int rc = check_handle(h, true);
   if (rc) return rc;
   const Plan& p = h->plan;
@@ -848,6 +871,7 @@ int signmuon_local_signs(signmuon_t h, const float* W, const float* const* G, ui
 int signmuon_vote_step(signmuon_t h, float* W, const uint8_t* signs, int64_t stride, int M, float eta) {
   NvtxRange range("signmuon_vote_step");
   const bool post = h != nullptr && (h->flags & (SIGNMUON_POST_POLAR | SIGNMUON_NORMALIZED_SIGN)) != 0;
+  DeviceGuard dev_guard(h);
   int rc = check_handle(h, post);
   if (rc) return rc;
   const Plan& p = h->plan;
@@ -867,6 +891,7 @@ int signmuon_vote_step(signmuon_t h, float* W, const uint8_t* signs, int64_t str
 
 int signmuon_sums_step(signmuon_t h, float* W, const void* sums, float eta) {
   NvtxRange range("signmuon_sums_step");
+  DeviceGuard dev_guard(h);
   int rc = check_handle(h, true);
   if (rc) return rc;
   const Plan& p = h->plan;
@@ -902,6 +927,7 @@ int signmuon_sums_step(signmuon_t h, float* W, const void* sums, float eta) {
 }
 
 int signmuon_step_host(signmuon_t h, float* W_host, const float* const* G_host, float eta) {
+  DeviceGuard dev_guard(h);
   int rc = check_handle(h, true);
   if (rc) return rc;
   const Plan& p = h->plan;
@@ -929,6 +955,7 @@ int signmuon_step_host(signmuon_t h, float* W_host, const float* const* G_host, 
 
 int signmuon_sync(signmuon_t h) {
   if (h == nullptr) return fail(nullptr, SIGNMUON_E_INVALID, "null handle");
+  DeviceGuard dev_guard(h);
   CK(h, cudaStreamSynchronize(h->stream));
   if (!h->pending) return SIGNMUON_OK;
   h->pending = false;
@@ -938,6 +965,7 @@ int signmuon_sync(signmuon_t h) {
 }
 
 int signmuon_vote(signmuon_t h, const uint8_t* const* signs, int64_t d, void* sums, int8_t* majority) {
+  DeviceGuard dev_guard(h);
   int rc = check_handle(h, false);
   if (rc) return rc;
   if (d < 0 || signs == nullptr) return fail(h, SIGNMUON_E_INVALID, "bad vote arguments");
@@ -954,6 +982,7 @@ int signmuon_vote(signmuon_t h, const uint8_t* const* signs, int64_t d, void* su
 }
 
 int signmuon_pack(signmuon_t h, const float* U, int64_t d, uint8_t* out) {
+  DeviceGuard dev_guard(h);
   int rc = check_handle(h, false);
   if (rc) return rc;
   if (d < 0 || (d > 0 && (U == nullptr || out == nullptr))) return fail(h, SIGNMUON_E_INVALID, "bad pack arguments");
@@ -964,6 +993,7 @@ int signmuon_pack(signmuon_t h, const float* U, int64_t d, uint8_t* out) {
 }
 
 int signmuon_sign_ternary(signmuon_t h, const float* U, int64_t d, int8_t* out) {
+  DeviceGuard dev_guard(h);
   int rc = check_handle(h, false);
   if (rc) return rc;
   if (d < 0 || (d > 0 && (U == nullptr || out == nullptr))) return fail(h, SIGNMUON_E_INVALID, "bad sign arguments");
@@ -974,6 +1004,7 @@ int signmuon_sign_ternary(signmuon_t h, const float* U, int64_t d, int8_t* out) 
 }
 
 int signmuon_vote_ternary(signmuon_t h, const int8_t* const* signs, int64_t d, void* sums, int8_t* majority) {
+  DeviceGuard dev_guard(h);
   int rc = check_handle(h, false);
   if (rc) return rc;
   if (d < 0 || signs == nullptr) return fail(h, SIGNMUON_E_INVALID, "bad vote arguments");
@@ -990,6 +1021,7 @@ int signmuon_vote_ternary(signmuon_t h, const int8_t* const* signs, int64_t d, v
 }
 
 int signmuon_apply_update(signmuon_t h, float* W, const float* D, int64_t d, float eta) {
+  DeviceGuard dev_guard(h);
   int rc = check_handle(h, false);
   if (rc) return rc;
   if (d < 0 || (d > 0 && (W == nullptr || D == nullptr))) return fail(h, SIGNMUON_E_INVALID, "bad update arguments");
@@ -1000,6 +1032,7 @@ int signmuon_apply_update(signmuon_t h, float* W, const float* D, int64_t d, flo
 }
 
 int signmuon_polar(signmuon_t h, const float* const* X, float* const* U) {
+  DeviceGuard dev_guard(h);
   int rc = check_handle(h, true);
   if (rc) return rc;
   const Plan& p = h->plan;
@@ -1021,6 +1054,7 @@ int signmuon_polar(signmuon_t h, const float* const* X, float* const* U) {
 }
 
 int signmuon_get_momentum(signmuon_t h, int m, float* dst) {
+  DeviceGuard dev_guard(h);
   int rc = check_handle(h, true);
   if (rc) return rc;
   if (m < 0 || m >= h->M || !dst) return fail(h, SIGNMUON_E_INVALID, "bad worker index or null dst");
@@ -1030,6 +1064,7 @@ int signmuon_get_momentum(signmuon_t h, int m, float* dst) {
 }
 
 int signmuon_set_momentum(signmuon_t h, int m, const float* src) {
+  DeviceGuard dev_guard(h);
   int rc = check_handle(h, true);
   if (rc) return rc;
   if (m < 0 || m >= h->M || !src) return fail(h, SIGNMUON_E_INVALID, "bad worker index or null src");
@@ -1054,6 +1089,7 @@ static int pi_state_buffer(signmuon_t h, int which, float** buf, int64_t* n) {
 }
 
 int signmuon_get_pi_state(signmuon_t h, int which, float* dst) {
+  DeviceGuard dev_guard(h);
   int rc = check_handle(h, true);
   if (rc) return rc;
   float* buf = nullptr;
@@ -1065,6 +1101,7 @@ int signmuon_get_pi_state(signmuon_t h, int which, float* dst) {
 }
 
 int signmuon_set_pi_state(signmuon_t h, int which, const float* src) {
+  DeviceGuard dev_guard(h);
   int rc = check_handle(h, true);
   if (rc) return rc;
   float* buf = nullptr;
@@ -1076,6 +1113,7 @@ int signmuon_set_pi_state(signmuon_t h, int which, const float* src) {
 }
 
 int signmuon_get_polar(signmuon_t h, int m, float* dst) {
+  DeviceGuard dev_guard(h);
   int rc = check_handle(h, true);
   if (rc) return rc;
   if (m < 0 || m >= h->M || !dst) return fail(h, SIGNMUON_E_INVALID, "bad worker index or null dst");
@@ -1089,6 +1127,7 @@ int signmuon_get_polar(signmuon_t h, int m, float* dst) {
 }
 
 int signmuon_get_signs(signmuon_t h, int m, uint8_t* dst) {
+  DeviceGuard dev_guard(h);
   int rc = check_handle(h, true);
   if (rc) return rc;
   if (m < 0 || m >= h->M || !dst) return fail(h, SIGNMUON_E_INVALID, "bad worker index or null dst");
@@ -1104,6 +1143,7 @@ int signmuon_get_signs(signmuon_t h, int m, uint8_t* dst) {
 }
 
 int signmuon_get_ternary_signs(signmuon_t h, int m, int8_t* dst) {
+  DeviceGuard dev_guard(h);
   int rc = check_handle(h, true);
   if (rc) return rc;
   if (m < 0 || m >= h->M || !dst) return fail(h, SIGNMUON_E_INVALID, "bad worker index or null dst");
@@ -1115,6 +1155,7 @@ int signmuon_get_ternary_signs(signmuon_t h, int m, int8_t* dst) {
 }
 
 int signmuon_get_direction(signmuon_t h, float* dst) {
+  DeviceGuard dev_guard(h);
   int rc = check_handle(h, true);
   if (rc) return rc;
   if (!dst || !aligned16(dst)) return fail(h, SIGNMUON_E_INVALID, "null or misaligned dst");
@@ -1140,6 +1181,7 @@ int signmuon_get_direction(signmuon_t h, float* dst) {
 }
 
 int signmuon_get_scales(signmuon_t h, float* dst_host) {
+  DeviceGuard dev_guard(h);
   int rc = check_handle(h, true);
   if (rc) return rc;
   if (!dst_host) return fail(h, SIGNMUON_E_INVALID, "null dst");
@@ -1150,6 +1192,7 @@ int signmuon_get_scales(signmuon_t h, float* dst_host) {
 
 int signmuon_profile(signmuon_t h, int enable) {
   if (h == nullptr) return fail(nullptr, SIGNMUON_E_INVALID, "null handle");
+  DeviceGuard dev_guard(h);
   prof_collect(h);
   h->prof = enable != 0;
   return SIGNMUON_OK;
@@ -1157,6 +1200,7 @@ int signmuon_profile(signmuon_t h, int enable) {
 
 int signmuon_profile_read(signmuon_t h, double* ms, int64_t* launches, int n) {
   if (h == nullptr) return fail(nullptr, SIGNMUON_E_INVALID, "null handle");
+  DeviceGuard dev_guard(h);
   prof_collect(h);
   for (int k = 0; k < n && k < SIGNMUON_PROF_KINDS; ++k) {
     if (ms) ms[k] = h->prof_ms[k];
@@ -1168,6 +1212,7 @@ int signmuon_profile_read(signmuon_t h, double* ms, int64_t* launches, int n) {
 }
 
 int signmuon_get_gram(signmuon_t h, int m, int mat, float* dst_host) {
+  DeviceGuard dev_guard(h);
   int rc = check_handle(h, true);
   if (rc) return rc;
   const Plan& p = h->plan;

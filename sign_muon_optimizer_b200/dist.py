@@ -32,7 +32,7 @@ import numpy as np
 import torch
 import torch.distributed as dist
 
-from . import SIGNMUON_ACC_INT8, SIGNMUON_E_NONFINITE, SIGNMUON_TERNARY, SignMuon, SignMuonError
+from . import SIGNMUON_ACC_INT8, SIGNMUON_ASYNC, SIGNMUON_E_NONFINITE, SIGNMUON_TERNARY, SignMuon, SignMuonError
 
 
 class DistSignMuon:
@@ -44,7 +44,10 @@ class DistSignMuon:
     (r+1)*M_local - 1.  ``exchange`` is "allgather" or "allreduce" (see the
     module text).  ``opt`` may be given to reuse an existing handle, or any
     object with the same methods (local_signs, vote_step, vote, vote_ternary,
-    sums_step, sign_stride) and attributes (d, flags).
+    sums_step, sign_stride, and sync for a handle made with SIGNMUON_ASYNC)
+    and attributes (d, flags).  With SIGNMUON_ASYNC every step waits for the
+    local half's status before the exchange, so that a failed rank stops all
+    ranks as it does without the flag.
     """
 
     def __init__(self, shapes, M_local=1, beta=0.9, lam=0.01, K=5, eps=1e-7, scale="fro", P=1, flags=0,
@@ -76,6 +79,10 @@ class DistSignMuon:
                             else torch.cuda.default_stream(self.device))
         flags = int(getattr(self.opt, "flags", flags))
         self.ternary = bool(flags & SIGNMUON_TERNARY)
+        # An asynchronous handle returns from local_signs before its status is
+        # known; the status all-reduce must carry that status, so the step
+        # waits for it (signmuon_sync) before the flag is set.
+        self.async_status = bool(flags & SIGNMUON_ASYNC)
         if exchange == "allgather":
             self.gathered = torch.zeros(self.M * self.stride, dtype=torch.uint8, device=self.device)
         else:
@@ -110,6 +117,10 @@ class DistSignMuon:
         err = None
         try:
             self.opt.local_signs(W, G, self.local, self.stride)
+            if self.async_status:
+                # raises the deferred error of this call (or of an earlier
+                # asynchronous call on the handle) before the flag is set
+                self.opt.sync()
             self._flag.fill_(1)
         except SignMuonError as e:
             err = e

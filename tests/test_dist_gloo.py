@@ -25,11 +25,16 @@ class _StandIn:
     """local_signs / vote_step / vote / sums_step / sign_stride with the
     library's layout (int32 sums; flags 0)."""
 
-    def __init__(self, fail=False):
+    def __init__(self, fail=False, deferred=False):
+        import sign_muon_optimizer_b200 as smo
         self.d = synth.numel(SHAPES)
         self.nb = ref.packed_nbytes(self.d)
-        self.flags = 0
+        # deferred: behave like a handle made with SIGNMUON_ASYNC, whose
+        # local_signs returns OK and whose sync() reports the failure
+        self.flags = smo.SIGNMUON_ASYNC if deferred else 0
         self.fail = fail
+        self.deferred = deferred
+        self.pending = False
         self.seen = None
 
     def sign_stride(self):
@@ -37,10 +42,17 @@ class _StandIn:
 
     def local_signs(self, W, G, out, stride):
         import sign_muon_optimizer_b200 as smo
-        if self.fail:
+        if self.fail and not self.deferred:
             raise smo.SignMuonError(smo.SIGNMUON_E_NONFINITE, "planted failure")
+        self.pending = self.fail
         for m, g in enumerate(G):
             out[m * stride: m * stride + self.nb] = torch.from_numpy(ref.pack_bits(ref.sign_bits(g.numpy())))
+
+    def sync(self):
+        import sign_muon_optimizer_b200 as smo
+        if self.pending:
+            self.pending = False
+            raise smo.SignMuonError(smo.SIGNMUON_E_NONFINITE, "planted deferred failure")
 
     def vote_step(self, W, signs, M, eta, stride):
         self.seen = signs.clone()
@@ -63,7 +75,7 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def _rank(rank, world, port, fail_rank, q, exchange="allgather"):
+def _rank(rank, world, port, fail_rank, q, exchange="allgather", deferred=False):
     import torch.distributed as dist
 
     from sign_muon_optimizer_b200.dist import DistSignMuon
@@ -71,7 +83,7 @@ def _rank(rank, world, port, fail_rank, q, exchange="allgather"):
     os.environ["MASTER_PORT"] = str(port)
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
     try:
-        opt = _StandIn(fail=(rank == fail_rank))
+        opt = _StandIn(fail=(rank == fail_rank), deferred=deferred)
         drv = DistSignMuon(SHAPES, M_local=M_LOCAL, opt=opt, device="cpu", exchange=exchange)
         W = torch.from_numpy(synth.weights0(SHAPES, 5))
         G = synth.gradients(SHAPES, world * M_LOCAL, 1.0, step=1, config_id=5)
@@ -89,12 +101,12 @@ def _rank(rank, world, port, fail_rank, q, exchange="allgather"):
         dist.destroy_process_group()
 
 
-def _run(fail_rank, exchange="allgather"):
+def _run(fail_rank, exchange="allgather", deferred=False):
     world = 2
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_rank, args=(r, world, port, fail_rank, q, exchange)) for r in range(world)]
+    procs = [ctx.Process(target=_rank, args=(r, world, port, fail_rank, q, exchange, deferred)) for r in range(world)]
     for p in procs:
         p.start()
     out = {}
@@ -149,9 +161,12 @@ def test_allreduce_exchange_adds_the_ranks_sums():
         assert np.array_equal(out[r]["W"].view(np.uint32), want.view(np.uint32))
 
 
+@pytest.mark.parametrize("deferred", [False, True])
 @pytest.mark.parametrize("exchange", ["allgather", "allreduce"])
-def test_one_failing_rank_stops_every_rank_without_update(exchange):
-    out = _run(fail_rank=1, exchange=exchange)
+def test_one_failing_rank_stops_every_rank_without_update(exchange, deferred):
+    # deferred: the failing rank's handle is asynchronous, so its local half
+    # returns OK and only its sync() reports the failure
+    out = _run(fail_rank=1, exchange=exchange, deferred=deferred)
     w0 = synth.weights0(SHAPES, 5)
     for r in range(2):
         assert out[r]["raised"] == "SignMuonError"
