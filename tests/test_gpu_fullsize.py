@@ -13,10 +13,15 @@ invariants over the whole output:
 * LLaMA-layer vote, d = 717,225,984, M=16: sampled entries bit-exact
   (int32 and int8 sums, majority); range, parity and sign invariants over
   every entry.
+* nanoGPT in the benchmark's exact configuration (signs packed inside the
+  last GEMM, no U written): packed bits, vote, post-vote D and W on sampled
+  matrices of three layers; and the signSGD baseline (K = 0) at full size.
 * NS sweep shapes: sampled problems of 64 x 1024^2 and 256 x 512x2048
-  against the oracle; one 8192^2 matrix with a known polar factor (a
-  normalised Sylvester-Hadamard matrix times a diagonal times a signed
-  permutation), compared entry by entry.
+  against the oracle over the whole grid (K in {5, 10}, cubic and quintic,
+  bf16 and fp32), and the M = 8 vote on the sweep's results; one 8192^2
+  matrix with a known polar factor (a normalised Sylvester-Hadamard matrix
+  times a diagonal times a signed permutation), compared entry by entry over
+  the same grid.
 Inputs are seeded synthetic data; large ones are drawn on the device by the
 synth module (torch Philox) and the sampled parts read back for the oracle.
 """
@@ -99,6 +104,130 @@ def _step_sampled(name, sample, post_polar):
 def test_nanogpt_step_full_size_sampled():
     shapes = synth.NANOGPT_SHAPES
     _step_sampled("nanogpt", [0, 1, 2, 3, len(shapes) - 1], post_polar=True)
+
+
+def _unpack_range(packed_dev, off, n):
+    """Bits off .. off+n of a device bit stream (off and n multiples of 8)."""
+    assert off % 8 == 0 and n % 8 == 0
+    b = packed_dev[off // 8: (off + n) // 8].cpu().numpy()
+    return np.unpackbits(b, bitorder="little").astype(bool)
+
+
+def test_nanogpt_bench_configuration_full_size():
+    """The exact configuration the benchmark times: SIGNMUON_POST_POLAR only,
+    so the last Newton-Schulz GEMM writes the one-bit signs of its epilogue
+    straight into the packed buffers and no U at all (384 problems, M = 8).
+    Checked on sampled matrices of three layers against the oracle: every
+    worker's packed bits (sign disagreement <= 1e-3 of the entries above the
+    magnitude mask), the vote (exact wherever every worker's sign agrees), the
+    post-vote polar D against the oracle's PolarNS of the GPU's own majority
+    (the teacher-forced global step), and W bit-exact given the GPU's D."""
+    wl = synth.WORKLOADS["nanogpt"]
+    shapes, M = wl["shapes"], wl["M"]
+    opt = smo.SignMuon(shapes, M, beta=HP["beta"], lam=HP["lam"], K=wl["K"], eps=HP["eps"], scale=wl["scale"],
+                       P=wl["P"], flags=smo.SIGNMUON_POST_POLAR)
+    W = synth.device_weights0(shapes, config_id=43)
+    W0 = W.clone()
+    G = synth.device_gradients(shapes, M, wl["sigma"], step=0, config_id=43)
+    opt.step(W, [G[m] for m in range(M)], HP["eta"])
+    d = opt.d
+    # no U is kept in this configuration
+    with pytest.raises(smo.SignMuonError):
+        opt.get_polar(0, torch.empty(d, device="cuda"))
+    nb = (d + 7) // 8
+    bits = []
+    for m in range(M):
+        b = torch.zeros(nb, dtype=torch.uint8, device="cuda")
+        opt.get_signs(m, b)
+        bits.append(b)
+    Dg = torch.empty(d, device="cuda")
+    opt.get_direction(Dg)
+    offs = synth.flat_offsets(shapes)
+    sample = [0, 1, 2, 3, 24, 25, 26, 27, len(shapes) - 4, len(shapes) - 3, len(shapes) - 2, len(shapes) - 1]
+    for i in sample:
+        r, c = shapes[i]
+        w0 = _mat(W0, shapes, i).astype(np.float32)
+        agree = np.ones(r * c, bool)
+        ref_bits, gpu_bits = [], []
+        for m in range(M):
+            g = _mat(G[m], shapes, i)
+            mom = ref.momentum_update(np.zeros_like(g), g, w0, HP["beta"], HP["lam"])
+            u = ref.polar_ns(mom, wl["K"], HP["eps"], wl["scale"], wl["P"]).ravel()
+            rb = ref.sign_bits(u)
+            gb = _unpack_range(bits[m], offs[i], r * c)
+            thr = 1e-3 * np.max(np.abs(u))
+            dis = int(((rb != gb) & (np.abs(u) > thr)).sum())
+            assert dis <= 1e-3 * int((np.abs(u) > thr).sum()), f"matrix {i} worker {m}: {dis} sign disagreements"
+            agree &= rb == gb
+            ref_bits.append(rb)
+            gpu_bits.append(gb)
+        ref_maj = np.sign(sum(2 * b.astype(np.int64) - 1 for b in ref_bits))
+        gpu_maj = np.sign(sum(2 * b.astype(np.int64) - 1 for b in gpu_bits))
+        assert np.array_equal(gpu_maj[agree], ref_maj[agree]), f"matrix {i}: vote differs on agreed entries"
+        assert (~agree).mean() <= M * 1e-3
+        # the post-vote polar step of the GPU's own majority
+        d_ref = ref.polar_ns(gpu_maj.reshape(r, c).astype(np.float64), wl["K"], HP["eps"], wl["scale"], wl["P"])
+        d_gpu = _mat(Dg, shapes, i)
+        assert_polar_close(d_gpu, d_ref, "bf16", f"post-vote D of matrix {i} ({r}x{c})")
+        # W moved by exactly one rounding of -eta * D
+        w_ref = ref.update(w0.ravel(), d_gpu.ravel().astype(np.float32), HP["eta"])
+        w_gpu = _mat(W, shapes, i).astype(np.float32).ravel()
+        assert np.array_equal(w_gpu.view(np.uint32), w_ref.view(np.uint32)), f"matrix {i}: W not bit-exact"
+    # over every entry: W = W0 - eta * D to within one float32 rounding
+    expect = W0.double() - float(np.float32(HP["eta"])) * Dg.double()
+    ulp = torch.abs(expect.float()).double() * 2.0 ** -23
+    assert bool((torch.abs(W.double() - expect) <= ulp).all())
+
+
+def test_nanogpt_signsgd_k0_full_size():
+    """The signSGD member of the comparison family at the headline size: K = 0
+    (no Newton-Schulz, the one-bit signs of the scaled momentum), no post-vote
+    step, M = 8.  Sampled matrices against the oracle: bits where |Mom| is
+    above the mask, the vote wherever every worker agrees, and W bit-exact
+    wherever the direction agrees."""
+    wl = synth.WORKLOADS["nanogpt"]
+    shapes, M = wl["shapes"], wl["M"]
+    opt = smo.SignMuon(shapes, M, beta=HP["beta"], lam=HP["lam"], K=0, eps=HP["eps"], scale="fro", flags=0)
+    W = synth.device_weights0(shapes, config_id=44)
+    W0 = W.clone()
+    G = synth.device_gradients(shapes, M, wl["sigma"], step=0, config_id=44)
+    opt.step(W, [G[m] for m in range(M)], HP["eta"])
+    d = opt.d
+    nb = (d + 7) // 8
+    bits = []
+    for m in range(M):
+        b = torch.zeros(nb, dtype=torch.uint8, device="cuda")
+        opt.get_signs(m, b)
+        bits.append(b)
+    Dg = torch.empty(d, device="cuda")
+    opt.get_direction(Dg)
+    offs = synth.flat_offsets(shapes)
+    for i in [0, 1, 2, 3, len(shapes) - 1]:
+        r, c = shapes[i]
+        w0 = _mat(W0, shapes, i).astype(np.float32)
+        agree = np.ones(r * c, bool)
+        ref_bits, gpu_bits = [], []
+        for m in range(M):
+            g = _mat(G[m], shapes, i)
+            mom = ref.momentum_update(np.zeros_like(g), g, w0, HP["beta"], HP["lam"])
+            u = ref.polar_ns(mom, 0, HP["eps"], "fro").ravel()
+            rb = ref.sign_bits(u)
+            gb = _unpack_range(bits[m], offs[i], r * c)
+            thr = 1e-3 * np.max(np.abs(u))
+            dis = int(((rb != gb) & (np.abs(u) > thr)).sum())
+            assert dis == 0, f"matrix {i} worker {m}: {dis} sign disagreements above the mask"
+            agree &= rb == gb
+            ref_bits.append(rb)
+            gpu_bits.append(gb)
+        ref_maj = np.sign(sum(2 * b.astype(np.int64) - 1 for b in ref_bits))
+        gpu_maj = np.sign(sum(2 * b.astype(np.int64) - 1 for b in gpu_bits))
+        assert np.array_equal(gpu_maj[agree], ref_maj[agree])
+        d_gpu = _mat(Dg, shapes, i).ravel()
+        assert np.array_equal(d_gpu, gpu_maj.astype(np.float64)), "D is the GPU's own majority"
+        w_ref = ref.update(w0.ravel(), ref_maj.astype(np.float32), HP["eta"])
+        w_gpu = _mat(W, shapes, i).astype(np.float32).ravel()
+        assert np.array_equal(w_gpu[agree].view(np.uint32), w_ref[agree].view(np.uint32))
+        assert (~agree).mean() <= M * 1e-3
 
 
 @pytest.mark.parametrize("i", [0, 1, 2, 3])
@@ -184,12 +313,74 @@ def test_ns_sweep_sampled(name, sample, precision):
     _ns_sweep_case(name, sample, precision, "cubic", 5, "spectral")
 
 
-# the sweep's other settings: quintic and K = 10 on the tensor cores (the
-# quintic with the Frobenius scale, which keeps every singular value of X0
-# inside the quintic's basin of convergence)
-@pytest.mark.parametrize("order,K,scale", [("quintic", 5, "fro"), ("cubic", 10, "spectral")])
-def test_ns_sweep_sampled_quintic_and_k10(order, K, scale):
-    _ns_sweep_case("batch64_1024", [0, 63], "bf16", order, K, scale)
+# the rest of the sweep's grid: K in {5, 10}, cubic and quintic, bf16 and
+# fp32, on both batched shapes (the quintic with the Frobenius scale, which
+# keeps every singular value of X0 inside the quintic's basin of convergence)
+@pytest.mark.parametrize("name,sample", [("batch64_1024", [0, 63]), ("batch256_512x2048", [0, 255])])
+@pytest.mark.parametrize("order,K,scale,precision", [
+    ("quintic", 5, "fro", "bf16"), ("quintic", 5, "fro", "fp32"), ("cubic", 10, "spectral", "bf16"),
+    ("cubic", 10, "spectral", "fp32"), ("quintic", 10, "fro", "bf16"), ("quintic", 10, "fro", "fp32")])
+def test_ns_sweep_sampled_grid(name, sample, order, K, scale, precision):
+    _ns_sweep_case(name, sample[:1] if precision == "fp32" else sample, precision, order, K, scale)
+
+
+@pytest.mark.parametrize("name,sample", [("batch64_1024", [0, 63]), ("batch256_512x2048", [0, 255])])
+def test_ns_sweep_m8_vote_on_the_results(name, sample):
+    """The sweep's M = 8 vote on its results: every worker's PolarNS output
+    (bf16, K = 5 cubic, spectral P = 2) packed to one bit per entry and voted
+    on the device.  The packed bits equal the signs of the GPU's U (bit for
+    bit, sampled matrices); the sums and majority equal the oracle's vote on
+    those bits at sampled entries over the whole vector (bit-exact); the
+    range, parity and sign invariants hold for every entry; and against the
+    oracle's own polar factors the majority agrees wherever every worker's
+    sign does."""
+    shapes = synth.SWEEP_SHAPES[name]
+    M = 8
+    h = smo.SignMuon(shapes, M, beta=0.9, lam=0.0, K=5, eps=1e-7, scale="spectral", P=2)
+    d = h.d
+    X = list(synth.device_gaussian(d, M, seed=2025))
+    U = [torch.empty_like(x) for x in X]
+    h.polar(X, U)
+    nb = (d + 7) // 8
+    bits = [torch.zeros(nb + 16, dtype=torch.uint8, device="cuda") for _ in range(M)]
+    for m in range(M):
+        h.pack(U[m], d, bits[m])
+    sums = torch.empty(d, dtype=torch.int32, device="cuda")
+    maj = torch.empty(d, dtype=torch.int8, device="cuda")
+    h.vote(bits, d, sums, maj)
+    torch.cuda.synchronize()
+    assert int(sums.min()) >= -M and int(sums.max()) <= M
+    assert bool(((sums + M) % 2 == 0).all())
+    assert torch.equal(torch.sign(sums).to(torch.int8), maj)
+    offs = synth.flat_offsets(shapes)
+    for i in sample:
+        r, c = shapes[i]
+        agree = np.ones(r * c, bool)
+        ref_bits, gpu_bits = [], []
+        for m in range(M):
+            gb = _unpack_range(bits[m], offs[i], r * c)
+            assert np.array_equal(gb, _mat(U[m], shapes, i).ravel() >= 0), f"matrix {i} worker {m}: pack"
+            u = ref.polar_ns(_mat(X[m], shapes, i), 5, 1e-7, "spectral", 2).ravel()
+            rb = ref.sign_bits(u)
+            agree &= rb == gb
+            ref_bits.append(rb)
+            gpu_bits.append(gb)
+        ref_maj = np.sign(sum(2 * b.astype(np.int64) - 1 for b in ref_bits))
+        got = maj[offs[i]: offs[i] + r * c].cpu().numpy()
+        assert np.array_equal(got[agree], ref_maj[agree]), f"matrix {i}: majority differs on agreed entries"
+        assert (~agree).mean() <= M * 1e-3
+    # sampled entries over the whole vector against the oracle's vote on the GPU's bits
+    rs = np.random.default_rng(11)
+    idx = np.unique(np.concatenate([rs.integers(0, d, 8192), np.arange(d - 1024, d)]))
+    words = np.unique(idx // 8)
+    wdev = torch.from_numpy(words).cuda()
+    packed = [b[wdev].cpu().numpy() for b in bits]
+    local = {w: k for k, w in enumerate(words)}
+    sub = np.array([local[i // 8] * 8 + (i % 8) for i in idx])
+    want = ref.vote_sums_from_bits(packed, len(words) * 8, "int32")[sub]
+    idev = torch.from_numpy(idx).cuda()
+    assert np.array_equal(sums[idev].cpu().numpy().astype(np.int64), want.astype(np.int64))
+    assert np.array_equal(maj[idev].cpu().numpy(), ref.majority(want))
 
 
 def _ns_sweep_case(name, sample, precision, order, K, scale):
@@ -212,7 +403,9 @@ def _hadamard_entry(i, j):
     return 1 - 2 * (np.bitwise_count(np.asarray(i) & np.asarray(j)).astype(np.int64) & 1)
 
 
-@pytest.mark.parametrize("order,K,precision", [("cubic", 5, "fp32"), ("quintic", 5, "fp32"), ("cubic", 10, "bf16")])
+@pytest.mark.parametrize("order,K,precision", [
+    ("cubic", 5, "fp32"), ("quintic", 5, "fp32"), ("cubic", 10, "fp32"), ("quintic", 10, "fp32"),
+    ("cubic", 5, "bf16"), ("quintic", 5, "bf16"), ("cubic", 10, "bf16"), ("quintic", 10, "bf16")])
 def test_ns_sweep_8192_known_polar_factor(order, K, precision):
     n = 8192
     rs = np.random.default_rng(8192)

@@ -467,3 +467,63 @@ def test_step_zero_gradients_degenerate(precision, post_polar):
     else:
         assert np.array_equal(D, np.ones(d, np.float32))
         assert np.array_equal(host(W).view(np.uint32), want["W"].view(np.uint32))
+
+
+@pytest.mark.parametrize("precision", ["fp32", "bf16"])
+@pytest.mark.parametrize("scale,P", [("fro", 1), ("spectral", 2)])
+def test_step_signsgd_k0(precision, scale, P):
+    """The signSGD baseline of the comparison family ([paper] Table 1's
+    SignSGD row, §3's sign vote): K = 0 Newton-Schulz iterations, so U is the
+    scaled momentum and the vote runs on sign(Mom); no post-vote step.  An
+    even M makes ties occur; they must map to 0.  Momentum, U, bits, the vote
+    on agreed entries and W where D agrees, as for the other steps."""
+    shapes = [(3, 5), (130, 70), (64, 147), (96, 300)]
+    M = 4
+    h, gpu, want = _run_one_step(shapes, M, 1.0, 0, scale, P, precision, False, seed=31)
+    _compare_step(shapes, M, gpu, want, precision, False)
+    d = synth.numel(shapes)
+    # with K = 0 the signs are those of the momentum itself (U = Mom / (s + eps))
+    for m in range(M):
+        mom = np.asarray(gpu["mom"][m])
+        assert np.array_equal(_np_bits(gpu["bits"][m], d), mom >= 0)
+    # ties occurred and went to 0
+    assert (_np_majority(gpu["bits"], d) == 0).any()
+
+
+def test_step_signsgd_k0_without_kept_polar():
+    """K = 0 with the flags a caller of the baseline would use (no
+    SIGNMUON_KEEP_POLAR): the packed signs come from the pack kernel of the
+    scaled momentum and must equal the signs of the GPU's own momentum bit for
+    bit; W moves by the vote of those signs."""
+    shapes = [(130, 70), (96, 300), (256, 128)]
+    M = 6
+    h = smo.SignMuon(shapes, M, beta=HP["beta"], lam=HP["lam"], K=0, eps=HP["eps"], scale="fro", P=1, flags=0)
+    d = h.d
+    w0 = synth.weights0(shapes, 33)
+    mom0 = synth.momentum0(shapes, M, 33, scale=0.5)
+    G = synth.gradients(shapes, M, 1.0, step=1, config_id=33)
+    for m in range(M):
+        h.set_momentum(m, dev(mom0[m]))
+    W = dev(w0)
+    h.step(W, [dev(g) for g in G], HP["eta"])
+    bits, moms = [], []
+    for m in range(M):
+        t = torch.zeros(d, device="cuda")
+        h.get_momentum(m, t)
+        moms.append(host(t))
+        b = torch.zeros(ref.packed_nbytes(d), dtype=torch.uint8, device="cuda")
+        h.get_signs(m, b)
+        bits.append(host(b))
+        assert np.array_equal(bits[m], ref.pack_bits(ref.sign_bits(moms[m])))
+    maj = ref.majority(ref.vote_sums_from_bits(bits, d))
+    assert (maj == 0).any()
+    want_w = ref.update(w0, maj.astype(np.float32), HP["eta"])
+    assert np.array_equal(host(W).view(np.uint32), want_w.view(np.uint32))
+    # and the oracle's own step agrees wherever every worker's sign agrees
+    want = ref.step(w0, G, mom0, shapes, beta=HP["beta"], lam=HP["lam"], eta=HP["eta"], K=0, eps=HP["eps"],
+                    scale="fro", P=1)
+    agree = np.ones(d, bool)
+    for m in range(M):
+        agree &= _np_bits(bits[m], d) == _np_bits(want["packed"][m], d)
+    assert np.array_equal(maj[agree], want["majority"][agree])
+    assert (~agree).mean() <= M * 1e-3

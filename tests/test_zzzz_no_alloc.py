@@ -5,12 +5,15 @@ graph capture, frameworks that own all device memory, real-time paths).  Its
 result must equal, within the fp32 tolerance of the other parity tests, the
 spectral scale that the regular entry points compute for the same matrix
 (signmuon_polar with SIGNMUON_NS_FP32 and spectral scaling, read back with
-signmuon_get_scales).  This file is collected last on purpose.
+signmuon_get_scales), and the oracle's power iteration in float64.  The size
+limit is checked on both sides of the bound.  This file is collected last on
+purpose.
 """
 import numpy as np
 import pytest
 
 import synth
+from oracle import signmuon_ref as ref
 
 pytestmark = pytest.mark.gpu
 
@@ -44,6 +47,10 @@ def test_noalloc_matches_existing_entry_point_two_calls_in_a_row(P):
     for (r, c), x, g in zip(shapes, xs, got):
         want = _existing_sigma((r, c), x, P)
         assert abs(g - want) <= REL_TOL * want, f"{r}x{c} P={P}: {g} vs {want}"
+        # the same estimate in float64 by the oracle (wide orientation)
+        xw = x.reshape(r, c).astype(np.float64)
+        exact = ref.power_sigma(xw if r <= c else xw.T, P)
+        assert abs(g - exact) <= REL_TOL * exact, f"{r}x{c} P={P}: {g} vs oracle {exact}"
 
 
 def test_noalloc_allocates_nothing_after_setup():
@@ -68,3 +75,29 @@ def test_noalloc_rejects_sizes_beyond_the_scratch():
         smo.signmuon_spectral_norm_noalloc(x, 400_000, 400_000, 2, sig)
     assert e.value.status == smo.SIGNMUON_E_INVALID
     assert "static scratch" in smo.signmuon_last_error(None)
+
+
+@pytest.mark.parametrize("rows,cols,P", [(1, 1048574, 2), (1048574, 1, 1)])
+def test_noalloc_accepts_the_largest_size(rows, cols, P):
+    """max(rows, cols) + 2 * min(rows, cols) equal to the scratch's 1,048,576
+    floats is accepted, in both orientations.  A single row or column has one
+    singular value, its 2-norm, which every power iteration returns."""
+    n = rows * cols
+    x = torch.randn(n, device="cuda", generator=torch.Generator(device="cuda").manual_seed(77))
+    sig = torch.zeros(4, device="cuda")
+    smo.signmuon_spectral_norm_noalloc(x, rows, cols, P, sig)
+    torch.cuda.synchronize()
+    got = float(sig[0].item())
+    want = float(np.linalg.norm(x.double().cpu().numpy()))
+    assert abs(got - want) <= REL_TOL * want, f"{rows}x{cols}: {got} vs {want}"
+
+
+@pytest.mark.parametrize("rows,cols", [(1, 1048575), (1048575, 1), (349527, 349525)])
+def test_noalloc_rejects_one_past_the_largest_size(rows, cols):
+    x = torch.zeros(16, device="cuda")
+    sig = torch.full((4,), -1.0, device="cuda")
+    with pytest.raises(smo.SignMuonError) as e:
+        smo.signmuon_spectral_norm_noalloc(x, rows, cols, 1, sig)
+    assert e.value.status == smo.SIGNMUON_E_INVALID
+    torch.cuda.synchronize()
+    assert float(sig[0].item()) == -1.0  # nothing was launched
