@@ -89,15 +89,16 @@ QUINTIC = (15.0 / 8.0, -10.0 / 8.0, 3.0 / 8.0)  # reading R4
 # 1. weight decay + momentum
 # ---------------------------------------------------------------------------
 
-def momentum_update(mom, g, w, beta, lam):
+def momentum_update(mom, g, w, beta, lam, dtype=np.float64):
     """Coupled weight decay then an exponential moving average.
 
     [paper] Algorithm 1 and Algorithm 2: the decayed gradient is
     G~ = G + lambda*W, and the new momentum is beta*Mom + (1-beta)*G~
-    (momentum starts at zero).
+    (momentum starts at zero).  dtype: the arithmetic (float64 for parity;
+    float32 only for the timed CPU baseline).
     """
-    g_tilde = np.asarray(g, np.float64) + float(lam) * np.asarray(w, np.float64)
-    return float(beta) * np.asarray(mom, np.float64) + (1.0 - float(beta)) * g_tilde
+    g_tilde = np.asarray(g, dtype) + float(lam) * np.asarray(w, dtype)
+    return float(beta) * np.asarray(mom, dtype) + (1.0 - float(beta)) * g_tilde
 
 
 # ---------------------------------------------------------------------------
@@ -110,7 +111,7 @@ def frobenius_norm(x):
     return math.sqrt(float(np.sum(x * x)))
 
 
-def power_sigma(x, P, u0=None, return_u=False):
+def power_sigma(x, P, u0=None, return_u=False, dtype=np.float64):
     """Estimate of the largest singular value of a wide X (m <= n) by P power
     iterations on X X^T (reading R2; [paper] Algorithm 1 input P, §4).
 
@@ -118,29 +119,29 @@ def power_sigma(x, P, u0=None, return_u=False):
     call ended with.  None, an all-zero or a non-finite u0 starts from
     ones(m)/sqrt(m).  With return_u the final iterate comes back as well.
     """
-    x = np.asarray(x, np.float64)
+    x = np.asarray(x, dtype)
     m = x.shape[0]
     if u0 is not None and np.all(np.isfinite(u0)) and np.any(np.asarray(u0) != 0):
-        u = np.array(u0, np.float64)
+        u = np.array(u0, dtype)
     else:
-        u = np.full(m, 1.0 / math.sqrt(m))
+        u = np.full(m, 1.0 / math.sqrt(m), dtype)
     for _ in range(int(P)):
         y = x @ (x.T @ u)
         nrm = math.sqrt(float(y @ y))
-        u = y / nrm if nrm > 0.0 else np.zeros(m)
+        u = y / nrm if nrm > 0.0 else np.zeros(m, dtype)
     z = x.T @ u
     sigma = math.sqrt(float(z @ z))
     return (sigma, u) if return_u else sigma
 
 
-def ns_iterate(x0, K, order="cubic", coeffs=None):
+def ns_iterate(x0, K, order="cubic", coeffs=None, dtype=np.float64):
     """K Newton-Schulz steps on a wide X (m <= n).
 
     With A = X X^T, the step X(aI + b X^T X) equals aX + b A X ([paper] §3,
     two-coefficient form; §4, cubic a=3/2, b=-1/2).  The quintic step (reading
     R4) is aX + (bA + cA^2) X.
     """
-    x = np.asarray(x0, np.float64)
+    x = np.asarray(x0, dtype)
     if order == "cubic":
         a, b = coeffs if coeffs is not None else CUBIC
         for _ in range(int(K)):
@@ -157,7 +158,7 @@ def ns_iterate(x0, K, order="cubic", coeffs=None):
 
 
 def polar_ns(mat, K, eps, scale, P=1, order="cubic", coeffs=None, return_scale=False, u0=None,
-             return_u=False):
+             return_u=False, dtype=np.float64):
     """PolarNS(Mat; K, eps, scale, P) of one matrix ([paper] Algorithm 1, §4).
 
     Works on the wide orientation (R1), divides by s + eps where s is the
@@ -166,18 +167,18 @@ def polar_ns(mat, K, eps, scale, P=1, order="cubic", coeffs=None, return_scale=F
     matrix's own orientation.  u0 warm-starts the power iteration (R21);
     return_u returns (result, s, final iterate or None for fro).
     """
-    mat = np.asarray(mat, np.float64)
+    mat = np.asarray(mat, dtype)
     tall = mat.shape[0] > mat.shape[1]
     x = mat.T if tall else mat
     u = None
     if scale == "fro":
         s = frobenius_norm(x)
     elif scale == "spectral":
-        s, u = power_sigma(x, P, u0, return_u=True)
+        s, u = power_sigma(x, P, u0, return_u=True, dtype=dtype)
     else:
         raise ValueError(scale)
     x = x / (s + float(eps))
-    x = ns_iterate(x, K, order, coeffs)
+    x = ns_iterate(x, K, order, coeffs, dtype=dtype)
     out = x.T if tall else x
     if return_u:
         return out, s, u
@@ -322,15 +323,17 @@ def split(flat, shapes, offsets=None):
     return out
 
 
-def polar_flat(flat, shapes, K, eps, scale, P=1, order="cubic", u0=None, return_u=False):
-    """PolarNS of every matrix of a flat vector, returned flat (float64).
-    u0: None or one warm start (or None) per matrix (R21); with return_u the
-    per-matrix final iterates come back too."""
-    out = np.empty(int(np.asarray(flat).size), np.float64)
+def polar_flat(flat, shapes, K, eps, scale, P=1, order="cubic", u0=None, return_u=False, dtype=np.float64):
+    """PolarNS of every matrix of a flat vector, returned flat (in dtype,
+    float64 unless asked otherwise).  u0: None or one warm start (or None)
+    per matrix (R21); with return_u the per-matrix final iterates come back
+    too."""
+    out = np.empty(int(np.asarray(flat).size), dtype)
     us = []
     off = 0
-    for i, ((r, c), mat) in enumerate(zip(shapes, split(np.asarray(flat, np.float64), shapes))):
-        res, _, u = polar_ns(mat, K, eps, scale, P, order, u0=None if u0 is None else u0[i], return_u=True)
+    for i, ((r, c), mat) in enumerate(zip(shapes, split(np.asarray(flat, dtype), shapes))):
+        res, _, u = polar_ns(mat, K, eps, scale, P, order, u0=None if u0 is None else u0[i], return_u=True,
+                             dtype=dtype)
         us.append(u)
         out[off: off + r * c] = res.ravel()
         off += r * c
@@ -367,7 +370,7 @@ def normalize_flat(flat, shapes, eps, scale, P=1, u0=None, return_u=False):
 
 def step(W, G_list, mom_list, shapes, *, beta, lam, eta, K, eps, scale, P=1,
          order="cubic", post_polar=False, acc="int32", tie=0, pre_polar=True,
-         signs="bits", normalize=False, warm=None):
+         signs="bits", normalize=False, warm=None, dtype=np.float64):
     """One distributed Sign-Muon step ([paper] Algorithm 2, with the vote of
     [blog] and the optional post-vote polar step of [paper] §4).
 
@@ -383,7 +386,9 @@ def step(W, G_list, mom_list, shapes, *, beta, lam, eta, K, eps, scale, P=1,
     power iteration from the previous step's final iterates (reading R21):
     warm["workers"][m][i] for worker m's matrix i, warm["single"][i] for the
     post-vote or normalised step's matrix i; the new state is returned as
-    out["warm"].
+    out["warm"].  dtype: the arithmetic of the momentum and both PolarNS
+    steps (float64, the parity mode; float32 only for the timed CPU
+    baseline); the vote and the update are exact either way.
 
     Returns a dict with the new momentum (float64), the polar factors U_m
     (the momentum itself when pre_polar is False), the packed bits (the int8
@@ -403,11 +408,11 @@ def step(W, G_list, mom_list, shapes, *, beta, lam, eta, K, eps, scale, P=1,
     new_warm = None if warm is None else dict(workers=[None] * M, single=warm.get("single"))
     new_mom, U_list, packed = [], [], []
     for m in range(M):
-        mom = momentum_update(mom_list[m], G_list[m], W, beta, lam)
+        mom = momentum_update(mom_list[m], G_list[m], W, beta, lam, dtype=dtype)
         new_mom.append(mom)
         if pre_polar:
             u, us = polar_flat(mom, shapes, K, eps, scale, P, order, u0=None if wk is None else wk[m],
-                               return_u=True)
+                               return_u=True, dtype=dtype)
             if new_warm is not None:
                 new_warm["workers"][m] = us
         else:
@@ -424,7 +429,8 @@ def step(W, G_list, mom_list, shapes, *, beta, lam, eta, K, eps, scale, P=1,
     maj = majority(sums, tie)
     single = None if warm is None else warm.get("single")
     if post_polar:
-        D, us = polar_flat(maj.astype(np.float64), shapes, K, eps, scale, P, order, u0=single, return_u=True)
+        D, us = polar_flat(maj.astype(dtype), shapes, K, eps, scale, P, order, u0=single, return_u=True,
+                           dtype=dtype)
         D32 = D.astype(np.float32)
         if new_warm is not None:
             new_warm["single"] = us

@@ -13,6 +13,7 @@ from fractions import Fraction
 import numpy as np
 import pytest
 
+import synth
 from oracle import signmuon_ref as ref
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
@@ -695,3 +696,23 @@ def test_warm_muon_step_uses_the_single_state():
         warm = out["warm"]
         _, u_cold = ref.power_sigma(out["mean"].reshape(5, 8), 2 * t, return_u=True)
         assert np.array_equal(warm["single"][0], u_cold)
+
+
+def test_float32_mode_matches_float64_within_the_fp32_tolerance():
+    """The oracle's float32 mode (timed as the CPU baseline) against its
+    float64 parity mode on the small 256x128 workload and a post-vote step:
+    the polar factors within the fp32 polar tolerance (1e-4), the momentum
+    within float32 rounding, and the float32 arithmetic really in float32."""
+    shapes = [(256, 128), (96, 300)]
+    M = 3
+    w0 = synth.weights0(shapes, 71)
+    G = synth.gradients(shapes, M, 0.5, step=1, config_id=71)
+    mom0 = synth.momentum0(shapes, M, 71, scale=0.5)
+    kw = dict(beta=0.9, lam=0.01, eta=0.02, K=5, eps=1e-7, scale="spectral", P=2, post_polar=True)
+    a = ref.step(w0, G, mom0, shapes, **kw)
+    b = ref.step(w0, G, mom0, shapes, dtype=np.float32, **kw)
+    for m in range(M):
+        assert b["mom"][m].dtype == np.float32 and b["U"][m].dtype == np.float32
+        assert np.max(np.abs(b["mom"][m] - a["mom"][m])) <= 4 * 2.0 ** -24 * np.max(np.abs(a["mom"][m])) * 4
+        assert np.max(np.abs(b["U"][m] - a["U"][m])) <= 1e-4
+    assert np.max(np.abs(b["D"] - a["D"])) <= 1e-4
