@@ -44,6 +44,9 @@ WORKLOAD_DESC = ("nanoGPT-124M weight shapes: 12 x {2304x768, 768x768, 3072x768,
 
 # per-(GPU) fallback peaks, used only when MEASURED_PEAKS.json is absent
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# fp32 FMA peak of the CUDA cores (the fp32 Newton-Schulz path runs there):
+# 148 SMs x 128 fp32 lanes x 2 flops x 1.965 GHz
+FP32_SIMT_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
 def peaks():
@@ -186,12 +189,16 @@ def gpu_smi_id(dev_index):
 # ---------------------------------------------------------------------------
 # CPU oracle (baseline leg and --impl reference)
 # ---------------------------------------------------------------------------
-def cpu_oracle_sample(step_idx=0):
+def cpu_oracle_sample(step_idx=0, precision="float32"):
     """One oracle step on the 768x768 attention projection of one layer for
     all 8 workers, including power iteration and the post-vote polar step;
     returns seconds.  Every nanoGPT matrix has 768 as its small side, so both
     the Newton-Schulz flops and the elementwise work of a matrix scale with
-    its element count: this sample is exactly 1/144 of one whole step."""
+    its element count: this sample is exactly 1/144 of one whole step.
+    precision: the oracle's arithmetic, float32 (the baseline) or float64
+    (its parity mode)."""
+    import numpy as np
+
     from oracle import signmuon_ref as ref
     shapes = [SHAPES[1]]
     w = synth.weights0(shapes, 3)
@@ -199,7 +206,7 @@ def cpu_oracle_sample(step_idx=0):
     mom = synth.momentum0(shapes, M, 3, scale=0.5)
     t0 = time.perf_counter()
     ref.step(w, G, mom, shapes, beta=HP["beta"], lam=HP["lam"], eta=HP["eta"], K=K_NS, eps=HP["eps"],
-             scale=WL["scale"], P=WL["P"], post_polar=WL["post_polar"])
+             scale=WL["scale"], P=WL["P"], post_polar=WL["post_polar"], dtype=getattr(np, precision))
     return time.perf_counter() - t0
 
 
@@ -219,7 +226,7 @@ def cpu_threads():
 
 CPU_SAMPLE = ("the 768x768 attention projection of one layer (589,824 weights, 1/144 of the model's "
               "weights and Newton-Schulz flops) x 8 workers, full oracle step incl. power iteration and "
-              "post-vote polar, numpy float64; steps/s scaled by 1/144 to the whole model")
+              "post-vote polar, numpy float32 (float64 beside it); steps/s scaled by 1/144 to the whole model")
 
 
 def run_reference(args):
@@ -229,20 +236,150 @@ def run_reference(args):
     for i in range(args.warmup):
         cpu_oracle_sample(i)
     times = [cpu_oracle_sample(args.warmup + i) for i in range(args.steps)]
-    per_step = CPU_SCALE * sum(times) / len(times)
-    value = 1.0 / per_step
+    sample_s = sum(times) / len(times)
+    # each timed step is the 1/144 sample; the value is the whole workload's
+    # rate, extrapolated by that factor (ms_per_step is what was timed)
+    value = 1.0 / (CPU_SCALE * sample_s)
     cores = cpu_threads()
+    extrap = f"x{CPU_SCALE:.0f}: value = 1 / ({CPU_SCALE:.0f} x the timed sample's mean seconds)"
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step * 1e3, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sample_s * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": WORKLOAD_DESC, "sample": CPU_SAMPLE},
+        "sample": {"ms_per_sample_step": sample_s * 1e3, "fraction_of_step": 1.0 / CPU_SCALE,
+                   "extrapolated": extrap},
         "cpu_baseline": {"value": value, "unit": "steps/s", "cores": cores, "kind": "oracle",
-                         "sample": CPU_SAMPLE},
+                         "sample": CPU_SAMPLE, "precision": "float32", "extrapolated": extrap},
         "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+# ---------------------------------------------------------------------------
+# the other configurations: short timed passes, each with its roofline
+# fraction (folded into the headline line, and printed by --workload)
+# ---------------------------------------------------------------------------
+SWEEP_GRID = [(5, "cubic", "bf16"), (10, "cubic", "bf16"), (5, "quintic", "bf16"), (10, "quintic", "bf16"),
+              (5, "cubic", "fp32"), (10, "cubic", "fp32"), (5, "quintic", "fp32"), (10, "quintic", "fp32")]
+
+
+def _events_time(fn, reps, stream, warm=3):
+    """Mean ms of fn() over reps calls, CUDA events on the given stream,
+    after `warm` warm-up calls."""
+    import torch
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def measure_resnet50(smo, stream, pk, steps=20):
+    """The ResNet-50 step (M=4, K=5 cubic bf16, spectral P=2): steps/s, and
+    its Newton-Schulz GEMMs' TFLOP/s from the library's per-kernel events."""
+    import torch
+    wl = synth.WORKLOADS["resnet50"]
+    shp, Mr = wl["shapes"], wl["M"]
+    h = smo.SignMuon(shp, Mr, beta=HP["beta"], lam=HP["lam"], K=wl["K"], eps=HP["eps"], scale=wl["scale"],
+                     P=wl["P"], flags=0, stream=stream.cuda_stream)
+    W = synth.device_weights0(shp, config_id=2)
+    G = synth.device_gradients(shp, Mr, wl["sigma"], step=0, config_id=2)
+    gl = [G[m] for m in range(Mr)]
+    ms = _events_time(lambda: h.step(W, gl, HP["eta"]), steps, stream)
+    h.profile(True)
+    h.profile_read()
+    for _ in range(steps):
+        h.step(W, gl, HP["eta"])
+    prof = h.profile_read()
+    h.profile(False)
+    fl = ns_flops_per_step(shp, Mr, wl["K"], False)
+    gemm_ms = sum(prof[k][0] for k in ("ns_gram", "ns_square", "ns_apply")) / steps
+    tf = fl / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else None
+    h.close()
+    del W, G, gl
+    torch.cuda.empty_cache()
+    return {"metric": "Sign-Muon steps/s (ResNet-50 shapes, M=4, K=5 cubic bf16, spectral P=2)",
+            "value": 1e3 / ms, "unit": "steps/s", "ms_per_step": ms, "d": synth.numel(shp),
+            "ns_tflops_per_step": fl / 1e12, "ns_ms_per_step": gemm_ms,
+            "ns_TFLOP/s": tf, "ns_frac_of_bf16_burst": (tf / pk["bf16_tflops"]) if tf else None,
+            "ns_share_of_step": gemm_ms / ms}
+
+
+def measure_llama_vote(smo, stream, pk, shapes=None, reps=5):
+    """The LLaMA-layer vote stress (M=16 packed one-bit buffers, d =
+    717,225,984): int32 and int8 sums + int8 majority, GB/s of algorithmic
+    bytes (M d/8 read, 4d or d sums and d majority written)."""
+    import torch
+    shapes = shapes or synth.LLAMA_LAYER_SHAPES
+    Mv = synth.WORKLOADS["llama_vote"]["M"]
+    d = synth.numel(shapes)
+    nb = (d + 7) // 8
+    g = torch.Generator(device="cuda")
+    g.manual_seed(4)
+    signs = [torch.randint(0, 256, (nb + 16,), generator=g, device="cuda", dtype=torch.uint8) for _ in range(Mv)]
+    out = []
+    for acc8 in (False, True):
+        h = smo.SignMuon(shapes, Mv, flags=smo.SIGNMUON_VOTE_ONLY | (smo.SIGNMUON_ACC_INT8 if acc8 else 0),
+                         stream=stream.cuda_stream)
+        sums = torch.empty(d, device="cuda", dtype=torch.int8 if acc8 else torch.int32)
+        maj = torch.empty(d, device="cuda", dtype=torch.int8)
+        ms = _events_time(lambda: h.vote(signs, d, sums, maj), reps, stream)
+        nbytes = Mv * d / 8.0 + (1.0 if acc8 else 4.0) * d + d
+        gbs = nbytes / (ms / 1e3) / 1e9
+        out.append({"acc_dtype": "int8" if acc8 else "int32", "GB/s": gbs, "frac_of_hbm": gbs / pk["hbm_gbs"],
+                    "ms": ms, "bytes": nbytes, "d": d, "M": Mv, "payload_bytes_per_worker": nb})
+        h.close()
+        del sums, maj
+    del signs
+    torch.cuda.empty_cache()
+    return out
+
+
+def measure_ns_sweep(smo, stream, pk, grid=SWEEP_GRID):
+    """The Newton-Schulz sweep: TFLOP/s of PolarNS (spectral P=2) on one
+    8192^2 matrix, 64 x 1024^2 and 256 x 512x2048, M=8 workers of Gaussian
+    input, over K in {5, 10}, cubic and quintic, bf16 (tcgen05) and fp32
+    (SIMT).  Flops per iteration and matrix: 4 m^2 n (cubic), 4 m^2 n + 2 m^3
+    (quintic), m = min dim, n = max dim.  The fp32 8192^2 case is timed with
+    one worker (one 8192^2 matrix already fills the GPU with tiles) to bound
+    the run; its flop rate is per worker like the others."""
+    import torch
+    out = []
+    for K, order, prec in grid:
+        for name, shp in synth.SWEEP_SHAPES.items():
+            Mw = 1 if (prec == "fp32" and name == "single_8192") else 8
+            fl_ns = (smo.SIGNMUON_NS_QUINTIC if order == "quintic" else 0) | \
+                    (smo.SIGNMUON_NS_FP32 if prec == "fp32" else 0)
+            h = smo.SignMuon(shp, Mw, beta=0.9, lam=0.0, K=K, eps=1e-7, scale="spectral", P=2, flags=fl_ns,
+                             stream=stream.cuda_stream)
+            X = synth.device_gaussian(h.d, Mw, seed=5)
+            U = torch.empty_like(X)
+            xs, us = [X[m] for m in range(Mw)], [U[m] for m in range(Mw)]
+            reps, warm = (3, 1) if prec == "bf16" else (1, 1)
+            ms = _events_time(lambda: h.polar(xs, us), reps, stream, warm=warm)
+            per_it = sum(4.0 * min(r, c) ** 2 * max(r, c) + (2.0 * min(r, c) ** 3 if order == "quintic" else 0.0)
+                         for r, c in shp)
+            fl = per_it * K * Mw
+            tf = fl / (ms / 1e3) / 1e12
+            e = {"shape": name, "K": K, "order": order, "precision": prec, "M": Mw, "TFLOP/s": tf, "ms": ms,
+                 "flops": fl}
+            if prec == "bf16":
+                e["frac_of_bf16_burst"] = tf / pk["bf16_tflops"]
+            else:
+                e["frac_of_fp32_simt_peak"] = tf / FP32_SIMT_PEAK_TFLOPS
+            out.append(e)
+            h.close()
+            del X, U, xs, us
+            torch.cuda.empty_cache()
+    return out
 
 
 # ---------------------------------------------------------------------------
@@ -262,7 +399,11 @@ def run_ours(args):
     import sign_muon_optimizer_b200 as smo
 
     stream = torch.cuda.current_stream()
-    flags = smo.SIGNMUON_POST_POLAR if WL["post_polar"] else 0
+    # SIGNMUON_ASYNC: the step does not wait for the GPU after each call; the
+    # device still checks the momentum norms every step (a non-finite one
+    # leaves W untouched) and signmuon_sync reads that status once, inside
+    # the timed region
+    flags = (smo.SIGNMUON_POST_POLAR if WL["post_polar"] else 0) | smo.SIGNMUON_ASYNC
     opt = smo.SignMuon(SHAPES, M, beta=HP["beta"], lam=HP["lam"], K=K_NS, eps=HP["eps"], scale=WL["scale"],
                        P=WL["P"], flags=flags, stream=stream.cuda_stream)
     W = synth.device_weights0(SHAPES, config_id=3 + rank)
@@ -272,8 +413,7 @@ def run_ours(args):
 
     for i in range(args.warmup):
         opt.step(W, gptrs[i % 2], HP["eta"])
-    opt.profile(True)
-    opt.profile_read()
+    opt.sync()
     launches0 = smo.signmuon_kernel_launches()
     sampler = ClockSampler(gpu_smi_id(local))
     sampler.start()
@@ -286,15 +426,23 @@ def run_ours(args):
     ev0.record(stream)
     for i in range(args.steps):
         opt.step(W, gptrs[i % 2], HP["eta"])
+    opt.sync()   # raises if any timed step saw a non-finite momentum norm
     ev1.record(stream)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
     launches = smo.signmuon_kernel_launches() - launches0
+    ms = max_over_ranks(ev0.elapsed_time(ev1), "cuda")
+    # per-kernel breakdown: the same steps again with an event pair around
+    # every launch (outside the timed region: the events serialise the stream)
+    opt.profile(True)
+    opt.profile_read()
+    for i in range(args.steps):
+        opt.step(W, gptrs[i % 2], HP["eta"])
+    opt.sync()
     prof = opt.profile_read()
     opt.profile(False)
-    ms = max_over_ranks(ev0.elapsed_time(ev1), "cuda")
     ms_per_step = ms / args.steps
     value = job_throughput(world, args.steps, ms)
 
@@ -305,13 +453,17 @@ def run_ours(args):
     gemm_ms = sum(prof[k][0] for k in gemm_kinds)
     gemm_launches = sum(prof[k][1] for k in gemm_kinds)
     tflops = flops * steps / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else None
-    peak_tc = pk["bf16_tflops_sustained"]
+    # the timed region is a fraction of a second: the burst peak is the
+    # denominator (the sustained figure is for seconds-long loops)
+    peak_tc = pk["bf16_tflops"]
     roofline = {"kernel": "k_gemm_tc (grouped Newton-Schulz GEMM, tcgen05)", "bound": "tensor",
                 "achieved": tflops, "peak": peak_tc, "unit": "TFLOP/s",
                 "frac": (tflops / peak_tc) if tflops else None, "traffic": gemm_traffic_from_profile(),
-                "peak_kind": f"bf16 sustained, {pk_kind}",
+                "peak_kind": f"bf16 burst, {pk_kind}",
                 "flops_per_launch": flops / max(1, gemm_launches / steps),
-                "avg_launch_ms": gemm_ms / max(1, gemm_launches)}
+                "avg_launch_ms": gemm_ms / max(1, gemm_launches),
+                "timed_region_ms": ms,
+                "frac_of_sustained": (tflops / pk["bf16_tflops_sustained"]) if tflops else None}
     hbm = hbm_bytes_per_step(SHAPES, M, WL["P"], WL["post_polar"])
     kernels = {}
     for kind, (kms, n) in prof.items():
@@ -323,7 +475,7 @@ def run_ours(args):
             f = 0.5 * ns_flops_per_step(SHAPES, 0 if kind.startswith("post") else M, K_NS,
                                         kind.startswith("post"))
             e["TFLOP/s"] = f / (kms / steps / 1e3) / 1e12
-            e["frac_of_bf16_peak"] = e["TFLOP/s"] / peak_tc
+            e["frac_of_bf16_burst"] = e["TFLOP/s"] / peak_tc
         elif kind in hbm:
             e["GB/s"] = hbm[kind] / (kms / steps / 1e3) / 1e9
             e["frac_of_hbm"] = e["GB/s"] / pk["hbm_gbs"]
@@ -355,11 +507,22 @@ def run_ours(args):
                "api": "signmuon_step_host (pinned host W and G)"}
         del Gh, Wh
 
+    # the other configurations (N = 1 only: the scaling runs time the headline alone)
+    extras = None
+    if rank == 0 and world == 1 and not args.no_extras:
+        extras = {"resnet50": measure_resnet50(smo, stream, pk),
+                  "llama_vote": measure_llama_vote(smo, stream, pk),
+                  "ns_sweep": measure_ns_sweep(smo, stream, pk)}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        t = 0.5 * (cpu_oracle_sample(0) + cpu_oracle_sample(1))
-        cpu = {"value": 1.0 / (CPU_SCALE * t), "unit": "steps/s", "cores": cpu_threads(), "kind": "oracle",
-               "sample": CPU_SAMPLE}
+        t32 = 0.5 * (cpu_oracle_sample(0, "float32") + cpu_oracle_sample(1, "float32"))
+        t64 = 0.5 * (cpu_oracle_sample(0, "float64") + cpu_oracle_sample(1, "float64"))
+        cpu = {"value": 1.0 / (CPU_SCALE * t32), "unit": "steps/s", "cores": cpu_threads(), "kind": "oracle",
+               "sample": CPU_SAMPLE, "precision": "float32",
+               "extrapolated": f"x{CPU_SCALE:.0f}: the sample's mean seconds times {CPU_SCALE:.0f}",
+               "sample_s": t32,
+               "float64": {"value": 1.0 / (CPU_SCALE * t64), "unit": "steps/s", "sample_s": t64}}
 
     if rank == 0:
         line = {
@@ -367,6 +530,7 @@ def run_ours(args):
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": WORKLOAD_DESC, "M": M, "d": D,
+                       "api": "signmuon_step with SIGNMUON_ASYNC; signmuon_sync once at the end of the timed steps",
                        "l2": "inputs larger than L2: 2.72 GB of gradients per step, two alternating sets",
                        "parallelism": "replicas" if world > 1 else "single GPU"},
             "roofline": roofline,
@@ -379,6 +543,7 @@ def run_ours(args):
             "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches, "clocks": clocks,
             "ns_tflops_per_step": flops / 1e12,
+            "workloads": extras,
         }
         print(json.dumps(line), flush=True)
     opt.close()
@@ -386,23 +551,6 @@ def run_ours(args):
         dist.barrier()
         dist.destroy_process_group()
     return 0
-
-
-def _events_time(fn, reps, stream):
-    """Mean ms of fn() over reps calls, CUDA events on the given stream,
-    after 3 warm-up calls."""
-    import torch
-    for _ in range(3):
-        fn()
-    torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(reps):
-        fn()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    return e0.elapsed_time(e1) / reps
 
 
 def run_secondary(args):
@@ -419,59 +567,18 @@ def run_secondary(args):
     if args.workload in ("llama_vote", "vote_100m", "all"):
         # vote_100m: the same kernel on one 1 x 100,000,000 matrix (a small
         # case for profiler captures)
-        shapes = [(1, 100_000_000)] if args.workload == "vote_100m" else synth.LLAMA_LAYER_SHAPES
-        Mv = synth.WORKLOADS["llama_vote"]["M"]
-        d = synth.numel(shapes)
-        nb = (d + 7) // 8
-        g = torch.Generator(device="cuda")
-        g.manual_seed(4)
-        signs = [torch.randint(0, 256, (nb + 16,), generator=g, device="cuda", dtype=torch.uint8) for _ in range(Mv)]
-        for acc8 in (False, True):
-            h = smo.SignMuon(shapes, Mv, flags=smo.SIGNMUON_VOTE_ONLY | (smo.SIGNMUON_ACC_INT8 if acc8 else 0),
-                             stream=stream.cuda_stream)
-            sums = torch.empty(d, device="cuda", dtype=torch.int8 if acc8 else torch.int32)
-            maj = torch.empty(d, device="cuda", dtype=torch.int8)
-            ms = _events_time(lambda: h.vote(signs, d, sums, maj), 5, stream)
-            nbytes = Mv * d / 8.0 + (1.0 if acc8 else 4.0) * d + d
-            gbs = nbytes / (ms / 1e3) / 1e9
-            shp_name = "1 x 100,000,000" if args.workload == "vote_100m" else "LLaMA-layer shapes"
-            lines.append({"metric": f"vote GB/s ({shp_name}, M=16, " + ("int8" if acc8 else "int32") + " sums)",
-                          "value": gbs, "unit": "GB/s", "frac_of_hbm": gbs / pk["hbm_gbs"], "peak_kind": pk_kind,
-                          "ms": ms, "bytes": nbytes, "d": d, "M": Mv, "payload_bytes_per_worker": nb,
-                          "acc_dtype": "int8" if acc8 else "int32", "collective": "none (on-device vote)"})
-            h.close()
-            del sums, maj
-        del signs
-        torch.cuda.empty_cache()
+        small = args.workload == "vote_100m"
+        shp_name = "1 x 100,000,000" if small else "LLaMA-layer shapes"
+        for e in measure_llama_vote(smo, stream, pk, [(1, 100_000_000)] if small else None):
+            lines.append(dict({"metric": f"vote GB/s ({shp_name}, M=16, {e['acc_dtype']} sums)", "value": e["GB/s"],
+                               "unit": "GB/s", "peak_kind": pk_kind, "collective": "none (on-device vote)"}, **e))
     if args.workload in ("ns_sweep", "ns_sweep_full", "all"):
-        # ns_sweep: K = 5 cubic bf16; ns_sweep_full adds K = 10, quintic and
-        # the fp32 SIMT path (the sweep's full grid)
-        grid = [(5, "cubic", "bf16")]
-        if args.workload == "ns_sweep_full":
-            grid += [(10, "cubic", "bf16"), (5, "quintic", "bf16"), (5, "cubic", "fp32")]
-        for K, order, prec in grid:
-            for name, shp in synth.SWEEP_SHAPES.items():
-                Mw = 8
-                fl_ns = (smo.SIGNMUON_NS_QUINTIC if order == "quintic" else 0) | \
-                        (smo.SIGNMUON_NS_FP32 if prec == "fp32" else 0)
-                h = smo.SignMuon(shp, Mw, beta=0.9, lam=0.0, K=K, eps=1e-7, scale="spectral", P=2, flags=fl_ns,
-                                 stream=stream.cuda_stream)
-                X = synth.device_gaussian(h.d, Mw, seed=5)
-                U = torch.empty_like(X)
-                xs, us = [X[m] for m in range(Mw)], [U[m] for m in range(Mw)]
-                ms = _events_time(lambda: h.polar(xs, us), 3, stream)
-                # cubic 4 m^2 n per iteration; quintic adds the 2 m^3 of A^2
-                per_it = sum(4.0 * min(r, c) ** 2 * max(r, c) + (2.0 * min(r, c) ** 3 if order == "quintic" else 0.0)
-                             for r, c in shp)
-                fl = per_it * K * Mw
-                tf = fl / (ms / 1e3) / 1e12
-                lines.append({"metric": f"NS TFLOP/s ({name}, M=8, K={K} {order} {prec}, spectral P=2)", "value": tf,
-                              "unit": "TFLOP/s", "frac_of_bf16_sustained": tf / pk["bf16_tflops_sustained"],
-                              "frac_of_bf16_burst": tf / pk["bf16_tflops"], "peak_kind": pk_kind, "ms": ms,
-                              "flops": fl})
-                h.close()
-                del X, U
-                torch.cuda.empty_cache()
+        # ns_sweep: K = 5 cubic bf16; ns_sweep_full: the sweep's whole grid
+        grid = SWEEP_GRID if args.workload == "ns_sweep_full" else [(5, "cubic", "bf16")]
+        for e in measure_ns_sweep(smo, stream, pk, grid):
+            lines.append(dict({"metric": f"NS TFLOP/s ({e['shape']}, M={e['M']}, K={e['K']} {e['order']} "
+                                         f"{e['precision']}, spectral P=2)", "value": e["TFLOP/s"],
+                               "unit": "TFLOP/s", "peak_kind": pk_kind}, **e))
     if args.workload in ("ternary_vote", "all"):
         # the int8 ternary wire's vote: d bytes per worker instead of d/8
         shapes = synth.LLAMA_LAYER_SHAPES
@@ -525,18 +632,7 @@ def run_secondary(args):
         del W, G, gl
         torch.cuda.empty_cache()
     if args.workload in ("resnet50", "all"):
-        wl = synth.WORKLOADS["resnet50"]
-        shp, Mr = wl["shapes"], wl["M"]
-        h = smo.SignMuon(shp, Mr, beta=HP["beta"], lam=HP["lam"], K=wl["K"], eps=HP["eps"], scale=wl["scale"],
-                         P=wl["P"], flags=0, stream=stream.cuda_stream)
-        W = synth.device_weights0(shp, config_id=2)
-        G = synth.device_gradients(shp, Mr, wl["sigma"], step=0, config_id=2)
-        gl = [G[m] for m in range(Mr)]
-        ms = _events_time(lambda: h.step(W, gl, HP["eta"]), 20, stream)
-        fl = ns_flops_per_step(shp, Mr, wl["K"], False)
-        lines.append({"metric": "Sign-Muon steps/s (ResNet-50 shapes, M=4)", "value": 1e3 / ms, "unit": "steps/s",
-                      "ms_per_step": ms, "ns_tflops_per_step": fl / 1e12, "d": synth.numel(shp)})
-        h.close()
+        lines.append(measure_resnet50(smo, stream, pk))
     for ln in lines:
         print(json.dumps(ln), flush=True)
     return 0
@@ -590,11 +686,18 @@ def run_collectives(args):
 
 def run_capture(args):
     """Profiler-capture mode (prints no bench line): the same step on the first
-    L transformer layers of the nanoGPT shapes, M=8, a few steps."""
+    L transformer layers of the nanoGPT shapes, M=8, a few steps.  Variants:
+    "ternary" sends int8 ternary signs (the sign8 and ternary vote kernels);
+    "unpacked" adds a 48-column matrix, so that no sign can be packed inside
+    the GEMM and the pack kernel runs."""
     import torch
     import sign_muon_optimizer_b200 as smo
     shapes = SHAPES[: 4 * args.capture_layers]
     flags = smo.SIGNMUON_POST_POLAR if WL["post_polar"] else 0
+    if args.capture_variant == "ternary":
+        flags |= smo.SIGNMUON_TERNARY
+    elif args.capture_variant == "unpacked":
+        shapes = shapes + [(768, 48)]
     opt = smo.SignMuon(shapes, M, beta=HP["beta"], lam=HP["lam"], K=K_NS, eps=HP["eps"], scale=WL["scale"],
                        P=WL["P"], flags=flags)
     W = synth.device_weights0(shapes, config_id=3)
@@ -615,8 +718,11 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the short passes of the ResNet-50, LLaMA-layer vote and NS sweep configurations")
     ap.add_argument("--capture-layers", type=int, default=0,
                     help="profiler capture mode on the first L layers; prints no bench line")
+    ap.add_argument("--capture-variant", default="nanogpt", choices=["nanogpt", "ternary", "unpacked"])
     ap.add_argument("--workload", default="nanogpt",
                     choices=["nanogpt", "llama_vote", "vote_100m", "ns_sweep", "ns_sweep_full", "resnet50",
                              "ternary_vote", "variants", "collectives", "all"],
