@@ -74,9 +74,9 @@ enum GemmOp { OP_GRAM = 0, OP_SQUARE = 1, OP_APPLY = 2 };
 // parameters (read through the constant cache; a per-tile decode from global
 // memory is a chain of dependent loads).
 constexpr int kParamGroups = 24;
-// TMA tensor maps per shape group (bf16 path): X ping/pong, A, B with 64-row,
-// 128-row and 32-row boxes, and X ping/pong as 4-D atom views with two-atom
-// operand boxes.
+// TMA tensor maps per shape group (bf16 path): X ping/pong, A, B with 64-row
+// and 128-row boxes, X ping/pong as 4-D atom views with two-atom operand
+// boxes, and X ping/pong, A, B with 32-row boxes (an epilogue warp's atom).
 constexpr int kMapsPerGroup = 14;
 constexpr int kParamMats = 64;
 
@@ -115,6 +115,32 @@ struct GemmArgs {
   int pgroup_mats[kParamMats];
 };
 
+// ---- programmatic dependent launch -----------------------------------------
+// Every kernel of the step is launched with programmatic stream
+// serialization, so that it can be scheduled while the kernel before it on
+// the stream is finishing; it starts with griddep_wait() (no global memory is
+// read or written before the previous kernel has completed and its writes are
+// visible), then lets the next kernel be scheduled.  Outside such a launch
+// both instructions do nothing.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+}
+
 // ---- launch wrappers (host) ----------------------------------------------
 void count_launch();
 void set_global_error(const char* msg);  // text for signmuon_last_error(NULL)
@@ -148,13 +174,17 @@ void launch_pack(cudaStream_t s, const float* U, int64_t u_stride, int64_t d, ui
                  int64_t out_stride, int M);
 void launch_vote(cudaStream_t s, const WorkerPtrs& signs, int M, int64_t d, void* sums, int acc8,
                  int8_t* majority, int tie_plus);
-void launch_vote_update(cudaStream_t s, const uint8_t* bits, int64_t bits_stride, int M, int64_t d,
-                        float* W, float eta, const int* status, int tie_plus);
-void launch_vote_major(cudaStream_t s, const uint8_t* bits, int64_t bits_stride, int M, int64_t d,
-                       float* D, int tie_plus);
-void launch_vote_stage(cudaStream_t s, const uint8_t* bits, int64_t bits_stride, int M, void* X, int x_bf16,
+// The vote kernels take worker m's packed signs at signs.p[m]: this GPU's
+// memory or a peer's mapped over NVLink (16-byte aligned, ceil(d/8) bytes
+// padded to a multiple of 16).
+void launch_vote_update(cudaStream_t s, const WorkerPtrs& signs, int M, int64_t d, float* W, float eta,
+                        const int* status, int tie_plus);
+void launch_vote_major(cudaStream_t s, const WorkerPtrs& signs, int M, int64_t d, float* D, int tie_plus);
+// streamable: every matrix starts at a multiple of 128 entries and has a
+// multiple of 8 columns (the streaming kernel's layout rule)
+void launch_vote_stage(cudaStream_t s, const WorkerPtrs& signs, int M, void* X, int x_bf16,
                        const Chunk* chunks, int n_chunks, const MatInfo* mats, const GroupInfo* groups,
-                       float* partials, float* D, int tie_plus);
+                       float* partials, float* D, int tie_plus, int streamable);
 void launch_mean_stage(cudaStream_t s, const float* Mom, int64_t mom_stride, int M, void* X, int x_bf16,
                        const Chunk* chunks, int n_chunks, const MatInfo* mats, const GroupInfo* groups,
                        float* partials, float* D);
@@ -165,10 +195,9 @@ void launch_sign8(cudaStream_t s, const float* U, int64_t u_stride, int64_t d, i
                   int M);
 void launch_vote_ternary(cudaStream_t s, const WorkerPtrs& signs, int M, int64_t d, void* sums, int acc8,
                          int8_t* majority, int tie_plus);
-void launch_vote_ternary_update(cudaStream_t s, const int8_t* signs, int64_t stride, int M, int64_t d, float* W,
-                                float eta, const int* status, int tie_plus);
-void launch_vote_ternary_major(cudaStream_t s, const int8_t* signs, int64_t stride, int M, int64_t d, float* D,
-                               int tie_plus);
+void launch_vote_ternary_update(cudaStream_t s, const WorkerPtrs& signs, int M, int64_t d, float* W, float eta,
+                                const int* status, int tie_plus);
+void launch_vote_ternary_major(cudaStream_t s, const WorkerPtrs& signs, int M, int64_t d, float* D, int tie_plus);
 // D = majority of int32 (or int8, acc8) vote sums
 void launch_sums_major(cudaStream_t s, const void* sums, int acc8, int64_t d, float* D, int tie_plus);
 

@@ -75,6 +75,8 @@ k_momentum(WorkerPtrs G, const float* __restrict__ W, float* __restrict__ Mom, i
            float beta, float lambda, void* __restrict__ X, int x_bf16,
            const Chunk* __restrict__ chunks, const MatInfo* __restrict__ mats,
            const GroupInfo* __restrict__ groups, float* __restrict__ partials) {
+  griddep_wait();
+  griddep_launch();
   // per-(worker, warp) partial sums of squares: one block barrier at the
   // end instead of two per worker, so that the warps run through the
   // workers independently
@@ -167,6 +169,8 @@ k_fro_finalize(int n_mats, int M, const float* __restrict__ partials, const int*
                const int* __restrict__ mat_nchunks, int use_for_scale, float eps, int quintic,
                float a, float b, float c, float* __restrict__ scale, float2* coef_apply,
                float2* coef_square, int* status) {
+  griddep_wait();
+  griddep_launch();
   __shared__ double red[32];
   const int p = blockIdx.x;
   const int w = p / n_mats, i = p - w * n_mats;
@@ -195,6 +199,8 @@ k_fro_finalize(int n_mats, int M, const float* __restrict__ partials, const int*
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kThreads)
 k_pi_init(const int64_t* __restrict__ uoff, const int* __restrict__ prob_g, float* __restrict__ u, int warm) {
+  griddep_wait();
+  griddep_launch();
   __shared__ double red[32];
   __shared__ int keep;
   const int p = blockIdx.x;
@@ -218,6 +224,8 @@ k_pi_matvec(const ProbRows* __restrict__ rows, const void* __restrict__ A,
             const int64_t* __restrict__ prob_a_off, const int* __restrict__ prob_g,
             const int* __restrict__ prob_gld, const int64_t* __restrict__ uoff,
             const float* __restrict__ u, float* __restrict__ y) {
+  griddep_wait();
+  griddep_launch();
   // y[r] = sum_k A[r][k] u[k] for the block's kPiRows rows of one problem.
   // u is staged in shared memory; each warp streams kRowsPerWarp rows at
   // once (one 16-byte load per row and lane in flight per step) so that the
@@ -238,22 +246,34 @@ k_pi_matvec(const ProbRows* __restrict__ rows, const void* __restrict__ A,
   if (BF16) {
     const __nv_bfloat16* a0 = reinterpret_cast<const __nv_bfloat16*>(A) + prob_a_off[p] + (int64_t)r0 * gld;
     const int g8 = g & ~7;
-    for (int k = lane * 8; k < g8; k += 256) {
-      uint4 raw[R];
+    // R rows x 4 column blocks of 256: all their 16-byte loads are in flight
+    // before the first FMA (one round trip per 1024 columns, not per 256)
+    for (int k0 = 0; k0 < g8; k0 += 4 * 256) {
+      uint4 raw[R][4];
 #pragma unroll
       for (int j = 0; j < R; ++j)
-        raw[j] = (r0 + j < g) ? __ldcs(reinterpret_cast<const uint4*>(a0 + (int64_t)j * gld + k)) : make_uint4(0, 0, 0, 0);
-      const float4 u0 = *reinterpret_cast<const float4*>(us + k);
-      const float4 u1 = *reinterpret_cast<const float4*>(us + k + 4);
-      const float uv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
 #pragma unroll
-      for (int j = 0; j < R; ++j) {
-        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw[j]);
+        for (int c = 0; c < 4; ++c) {
+          const int k = k0 + c * 256 + lane * 8;
+          raw[j][c] = (r0 + j < g && k < g8) ? __ldcs(reinterpret_cast<const uint4*>(a0 + (int64_t)j * gld + k))
+                                             : make_uint4(0, 0, 0, 0);
+        }
 #pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          const float2 f = __bfloat1622float2(h[t]);
-          acc[j] = fmaf(f.x, uv[2 * t], acc[j]);
-          acc[j] = fmaf(f.y, uv[2 * t + 1], acc[j]);
+      for (int c = 0; c < 4; ++c) {
+        const int k = k0 + c * 256 + lane * 8;
+        if (k >= g8) break;
+        const float4 u0 = *reinterpret_cast<const float4*>(us + k);
+        const float4 u1 = *reinterpret_cast<const float4*>(us + k + 4);
+        const float uv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+        for (int j = 0; j < R; ++j) {
+          const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw[j][c]);
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const float2 f = __bfloat1622float2(h[t]);
+            acc[j] = fmaf(f.x, uv[2 * t], acc[j]);
+            acc[j] = fmaf(f.y, uv[2 * t + 1], acc[j]);
+          }
         }
       }
     }
@@ -295,6 +315,8 @@ k_pi_matvec(const ProbRows* __restrict__ rows, const void* __restrict__ A,
 __global__ void __launch_bounds__(kThreads)
 k_pi_normalize(const int64_t* __restrict__ uoff, const int* __restrict__ prob_g,
                const float* __restrict__ y, float* __restrict__ u) {
+  griddep_wait();
+  griddep_launch();
   __shared__ double red[32];
   __shared__ float inv;
   const int p = blockIdx.x;
@@ -313,6 +335,8 @@ k_pi_finalize(const int64_t* __restrict__ uoff, const int* __restrict__ prob_g,
               const float* __restrict__ u, const float* __restrict__ y, float eps, int quintic,
               float a, float b, float c, float* __restrict__ scale, float2* coef_apply,
               float2* coef_square, int* status) {
+  griddep_wait();
+  griddep_launch();
   __shared__ double red[32];
   const int p = blockIdx.x;
   const int g = prob_g[p];
@@ -332,6 +356,8 @@ __global__ void __launch_bounds__(kThreads)
 k_scale_flat(WorkerPtrs in, float* __restrict__ out, int64_t out_stride,
              const Chunk* __restrict__ chunks, const MatInfo* __restrict__ mats, int n_mats,
              const float* __restrict__ scale, float eps) {
+  griddep_wait();
+  griddep_launch();
   const Chunk ch = chunks[blockIdx.x];
   const int w = blockIdx.y;
   const MatInfo mi = mats[ch.mat];
@@ -359,6 +385,8 @@ __device__ __forceinline__ uint32_t spread8(uint32_t x) {  // bit i -> bit 4i
 __global__ void __launch_bounds__(kThreads)
 k_pack(const float* __restrict__ U, int64_t u_stride, int64_t d, uint8_t* __restrict__ out,
        int64_t out_stride) {
+  griddep_wait();
+  griddep_launch();
   const int w = blockIdx.y;
   U += (int64_t)w * u_stride;
   out += (int64_t)w * out_stride;
@@ -421,18 +449,18 @@ __device__ __forceinline__ int vmaj(int s, int tie_plus) { return tie_plus ? (s 
 // workers so that no lane overflows; 8 workers' loads are in flight at once.
 template <int MODE, bool ACC8>
 __global__ void __launch_bounds__(kThreads)
-k_vote(WorkerPtrs signs, const uint8_t* __restrict__ bits, int64_t bits_stride, int M, int64_t d,
+k_vote(WorkerPtrs signs, int M, int64_t d,
        void* __restrict__ sums, int8_t* __restrict__ maj, float* __restrict__ W, float eta,
        float* __restrict__ D, const int* __restrict__ status, int tie_plus) {
+  griddep_wait();
+  griddep_launch();
   if (MODE == 1 && status != nullptr && (status[0] | status[1]) != 0) return;  // keep W on error
   const int lane = threadIdx.x & 31;
   const int64_t gw = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
   const int64_t nw = ((int64_t)gridDim.x * kThreads) >> 5;
   const int64_t nblk = d >> 7;                  // full 128-entry blocks
   const int grp = lane >> 3, g = lane & 7, shift = 4 * g;
-  auto stream = [&](int m) {
-    return (MODE == 0) ? reinterpret_cast<const uint8_t*>(signs.p[m]) : bits + (int64_t)m * bits_stride;
-  };
+  auto stream = [&](int m) { return reinterpret_cast<const uint8_t*>(signs.p[m]); };
   for (int64_t st = gw; st * 4 < nblk; st += nw) {
     const int64_t b = st * 4 + grp;               // this lane group's block
     const bool on = b < nblk;
@@ -498,7 +526,7 @@ k_vote(WorkerPtrs signs, const uint8_t* __restrict__ bits, int64_t bits_stride, 
     for (int64_t e = nblk * 128 + threadIdx.x; e < d; e += kThreads) {
       int c = 0;
       for (int m = 0; m < M; ++m) {
-        const uint8_t* src = (MODE == 0) ? reinterpret_cast<const uint8_t*>(signs.p[m]) : bits + (int64_t)m * bits_stride;
+        const uint8_t* src = reinterpret_cast<const uint8_t*>(signs.p[m]);
         c += (src[e >> 3] >> (e & 7)) & 1;
       }
       const int sm_ = 2 * c - M;
@@ -533,11 +561,29 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
 
+// MODE 3 (staging of the post-vote polar step's input): the work items are
+// the plan's chunks instead of flat tiles.  Chunk c covers entries base ..
+// base + len - 1 of the flat vector (base = its matrix's offset + its start,
+// a multiple of 128; len <= 4096); its majorities go to the bf16 X of the
+// one-problem-set Newton-Schulz input, which for a matrix with a multiple of
+// 8 columns is the chunk's contiguous range starting at xb + start, and
+// partials[c] receives the chunk's count of non-zero majorities (its sum of
+// squares).
+struct VoteStage {
+  __nv_bfloat16* X;
+  const Chunk* chunks;
+  const MatInfo* mats;
+  const GroupInfo* groups;
+  float* partials;
+};
+
 template <int MODE, bool ACC8>
 __global__ void __launch_bounds__(kVoteWarps * 32)
-k_vote_stream(WorkerPtrs signs, const uint8_t* __restrict__ bits, int64_t bits_stride, int M, int64_t ntiles,
+k_vote_stream(WorkerPtrs signs, int M, int64_t ntiles,
               void* __restrict__ sums, int8_t* __restrict__ maj, float* __restrict__ W, float eta,
-              float* __restrict__ D, const int* __restrict__ status, int tie_plus) {
+              float* __restrict__ D, const int* __restrict__ status, int tie_plus, VoteStage st) {
+  griddep_wait();
+  griddep_launch();
   if (MODE == 1 && status != nullptr && (status[0] | status[1]) != 0) return;  // keep W on error
   extern __shared__ __align__(16) uint8_t vsm[];   // [warp][2][kVoteBatch][512]
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
@@ -545,27 +591,46 @@ k_vote_stream(WorkerPtrs signs, const uint8_t* __restrict__ bits, int64_t bits_s
   const int64_t nw = (int64_t)gridDim.x * kVoteWarps;
   const uint32_t buf0 = (uint32_t)__cvta_generic_to_shared(vsm) + (uint32_t)wid * (2 * kVoteBatch * kVoteTileB);
   const int nbatch = (M + kVoteBatch - 1) / kVoteBatch;
-  auto stream = [&](int m) {
-    return (MODE == 0) ? reinterpret_cast<const uint8_t*>(signs.p[m]) : bits + (int64_t)m * bits_stride;
-  };
+  auto stream = [&](int m) { return reinterpret_cast<const uint8_t*>(signs.p[m]); };
   // (tile, batch) work items of this warp, in order
   int64_t tile = gw;
   int batch = 0;
+  // flat start and length of work item t (a whole tile, or one chunk)
+  auto item_base = [&](int64_t t) -> int64_t {
+    if (MODE == 3) {
+      const Chunk c = st.chunks[t];
+      return st.mats[c.mat].off + c.start;
+    }
+    return t * 4096;
+  };
+  auto item_len = [&](int64_t t) -> int { return MODE == 3 ? st.chunks[t].len : 4096; };
   auto issue = [&](int64_t t, int bt, int buf) {
     const uint32_t dst = buf0 + (uint32_t)buf * (kVoteBatch * kVoteTileB) + (uint32_t)lane * 16;
+    const int64_t boff = item_base(t) >> 3;
+    // a lane's 16 bytes hold entries 128 lane .. 128 lane + 127 of the item;
+    // pieces wholly past a short chunk's end are not read
+    const bool live = MODE != 3 || lane * 128 < item_len(t);
 #pragma unroll
     for (int i = 0; i < kVoteBatch; ++i) {
       const int m = bt * kVoteBatch + i;
-      if (m < M) cp_async16(dst + (uint32_t)i * kVoteTileB, stream(m) + t * kVoteTileB + lane * 16);
+      if (m < M && live) cp_async16(dst + (uint32_t)i * kVoteTileB, stream(m) + boff + lane * 16);
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
   };
   if (tile >= ntiles) return;
   issue(tile, 0, 0);
   int cur = 0;
-  uint32_t acc[32];                            // byte lane i of acc[j]: entry 128 j + 4 lane + i
+  // Counting: lane t counts the 128 entries it loaded itself (entries 128 t ..
+  // 128 t + 127 of the item, four 32-bit words of every stream).  Bit g + 4 q
+  // of word w goes to nibble q of the vertical counter nib[w][g] (one
+  // shift-and-add per 8 entries and worker); after each batch of <= 8 workers
+  // the nibbles move into byte counters: byte b of cb[w][g][0] counts entry
+  // 32 w + 8 b + g, of cb[w][g][1] entry 32 w + 8 b + 4 + g.
+  uint32_t cb[4][4][2];
 #pragma unroll
-  for (int j = 0; j < 32; ++j) acc[j] = 0;
+  for (int w = 0; w < 4; ++w)
+#pragma unroll
+    for (int g = 0; g < 4; ++g) cb[w][g][0] = cb[w][g][1] = 0;
   while (true) {
     // the next work item goes out before this one is counted
     int64_t ntile = tile;
@@ -580,23 +645,97 @@ k_vote_stream(WorkerPtrs signs, const uint8_t* __restrict__ bits, int64_t bits_s
     __syncwarp();
     const uint32_t src = buf0 + (uint32_t)cur * (kVoteBatch * kVoteTileB);
     const int nm = min(kVoteBatch, M - batch * kVoteBatch);
-    const int shift = (lane & 7) * 4;
-    for (int i = 0; i < nm; ++i) {
-      const uint32_t row = src + (uint32_t)i * kVoteTileB + (uint32_t)(lane >> 3) * 4;
+    {
+      uint32_t nib[4][4];
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        uint32_t w;
-        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w) : "r"(row + (uint32_t)j * 16));
-        acc[j] += ((w >> shift) & 0xFu) * 0x00204081u & 0x01010101u;
+      for (int w = 0; w < 4; ++w)
+#pragma unroll
+        for (int g = 0; g < 4; ++g) nib[w][g] = 0;
+      for (int i = 0; i < nm; ++i) {
+        uint32_t v[4];
+        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3])
+                     : "r"(src + (uint32_t)i * kVoteTileB + (uint32_t)lane * 16));
+#pragma unroll
+        for (int w = 0; w < 4; ++w)
+#pragma unroll
+          for (int g = 0; g < 4; ++g) nib[w][g] += (v[w] >> g) & 0x11111111u;
       }
+#pragma unroll
+      for (int w = 0; w < 4; ++w)
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          cb[w][g][0] += nib[w][g] & 0x0F0F0F0Fu;
+          cb[w][g][1] += (nib[w][g] >> 4) & 0x0F0F0F0Fu;
+        }
     }
     __syncwarp();
+    uint32_t acc[32];   // byte lane i of acc[j]: the count of entry 128 j + 4 lane + i
     if (batch == nbatch - 1) {
+      // Byte counts in entry order for this lane's 128 entries: word 8 w + 2 b
+      // + h holds entries 32 w + 8 b + 4 h .. + 3 (a 4 x 4 byte transpose of
+      // cb[w][0..3][h]), written to row `lane` of the (consumed) batch buffer
+      // with an XOR swizzle; column reads then give lane t the words of
+      // entries 128 j + 4 t .. + 3, so that each warp store below writes
+      // consecutive entries.  Both passes are free of bank conflicts.
+      const uint32_t tr = src;   // 32 x 32 words = 4 KB of the buffer just counted
+#pragma unroll
+      for (int w = 0; w < 4; ++w)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t t0 = __byte_perm(cb[w][0][h], cb[w][1][h], 0x5140);
+          const uint32_t t1 = __byte_perm(cb[w][0][h], cb[w][1][h], 0x7362);
+          const uint32_t t2 = __byte_perm(cb[w][2][h], cb[w][3][h], 0x5140);
+          const uint32_t t3 = __byte_perm(cb[w][2][h], cb[w][3][h], 0x7362);
+          const uint32_t o[4] = {__byte_perm(t0, t2, 0x5410), __byte_perm(t0, t2, 0x7632),
+                                 __byte_perm(t1, t3, 0x5410), __byte_perm(t1, t3, 0x7632)};
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            const int k = 8 * w + 2 * b + h;
+            asm volatile("st.shared.u32 [%0], %1;" ::"r"(tr + (uint32_t)(lane * 32 + (k ^ lane)) * 4), "r"(o[b])
+                         : "memory");
+          }
+          cb[w][0][h] = cb[w][1][h] = cb[w][2][h] = cb[w][3][h] = 0;
+        }
+      __syncwarp();
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(acc[j]) : "r"(tr + (uint32_t)(j * 32 + (lane ^ j)) * 4) : "memory");
+      __syncwarp();
+    }
+    if (batch == nbatch - 1 && MODE == 3) {
+      // chunk done: its majorities into X (4 bf16 per lane and step, so each
+      // warp store writes 256 contiguous bytes) and D, its non-zero count
+      const Chunk ch = st.chunks[tile];
+      const MatInfo mi = st.mats[ch.mat];
+      const GroupInfo gi = st.groups[mi.group];
+      __nv_bfloat16* xo = st.X + gi.x_base + (int64_t)mi.q * gi.rows * gi.ld + ch.start;
+      const int64_t fb = mi.off + ch.start;
+      int nz = 0;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const int c0 = acc[j] & 0xFF, c1 = (acc[j] >> 8) & 0xFF, c2 = (acc[j] >> 16) & 0xFF, c3 = acc[j] >> 24;
+        const int e = j * 128 + lane * 4;
+        if (e < ch.len) {
+          const int v0 = vmaj(2 * c0 - M, tie_plus), v1 = vmaj(2 * c1 - M, tie_plus);
+          const int v2 = vmaj(2 * c2 - M, tie_plus), v3 = vmaj(2 * c3 - M, tie_plus);
+          nz += (v0 != 0) + (v1 != 0) + (v2 != 0) + (v3 != 0);
+          const __nv_bfloat162 lo = __floats2bfloat162_rn((float)v0, (float)v1);
+          const __nv_bfloat162 hi = __floats2bfloat162_rn((float)v2, (float)v3);
+          uint2 u;
+          u.x = *reinterpret_cast<const uint32_t*>(&lo);
+          u.y = *reinterpret_cast<const uint32_t*>(&hi);
+          *reinterpret_cast<uint2*>(xo + e) = u;
+          if (D != nullptr) st4(D + fb + e, make_float4((float)v0, (float)v1, (float)v2, (float)v3));
+        }
+      }
+      nz = __reduce_add_sync(0xffffffffu, nz);
+      if (lane == 0) st.partials[tile] = (float)nz;
+    } else if (batch == nbatch - 1) {
       // tile done: write its 4096 results
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
         const int c0 = acc[j] & 0xFF, c1 = (acc[j] >> 8) & 0xFF, c2 = (acc[j] >> 16) & 0xFF, c3 = acc[j] >> 24;
-        acc[j] = 0;
         const int s0 = 2 * c0 - M, s1 = 2 * c1 - M, s2 = 2 * c2 - M, s3 = 2 * c3 - M;
         const int64_t e = tile * 4096 + j * 128 + lane * 4;
         if (MODE == 0) {
@@ -637,9 +776,11 @@ k_vote_stream(WorkerPtrs signs, const uint8_t* __restrict__ bits, int64_t bits_s
 // non-null, to D (fp32 flat); partials[chunk] gets the chunk's sum of
 // squares (its non-zero count) for the Frobenius scale and the finite check.
 __global__ void __launch_bounds__(kThreads)
-k_vote_stage(const uint8_t* __restrict__ bits, int64_t bits_stride, int M, void* __restrict__ X, int x_bf16,
+k_vote_stage(WorkerPtrs signs, int M, void* __restrict__ X, int x_bf16,
              const Chunk* __restrict__ chunks, const MatInfo* __restrict__ mats,
              const GroupInfo* __restrict__ groups, float* __restrict__ partials, float* __restrict__ D, int tie_plus) {
+  griddep_wait();
+  griddep_launch();
   __shared__ float red[32];
   const Chunk ch = chunks[blockIdx.x];
   const MatInfo mi = mats[ch.mat];
@@ -677,7 +818,7 @@ k_vote_stage(const uint8_t* __restrict__ bits, int64_t bits_stride, int M, void*
       uint32_t by[8][kV];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const uint8_t* bm = bits + (int64_t)(m + i) * bits_stride;
+        const uint8_t* bm = (m + i < M) ? reinterpret_cast<const uint8_t*>(signs.p[m + i]) : nullptr;
 #pragma unroll
         for (int j = 0; j < kV; ++j) by[i][j] = (m + i < M && on[j]) ? (uint32_t)bm[fe[j] >> 3] : 0u;
       }
@@ -723,7 +864,7 @@ k_vote_stage(const uint8_t* __restrict__ bits, int64_t bits_stride, int M, void*
     for (int e = threadIdx.x; e < ch.len; e += kThreads) {
       const int64_t fe = base + e;
       int c = 0;
-      for (int m = 0; m < M; ++m) c += (bits[(int64_t)m * bits_stride + (fe >> 3)] >> (fe & 7)) & 1;
+      for (int m = 0; m < M; ++m) c += (reinterpret_cast<const uint8_t*>(signs.p[m])[fe >> 3] >> (fe & 7)) & 1;
       const float v = (float)vmaj(2 * c - M, tie_plus);
       ss += v * v;
       if (D != nullptr) D[fe] = v;
@@ -744,6 +885,8 @@ __global__ void __launch_bounds__(kThreads)
 k_mean_stage(const float* __restrict__ Mom, int64_t mom_stride, int M, void* __restrict__ X, int x_bf16,
              const Chunk* __restrict__ chunks, const MatInfo* __restrict__ mats,
              const GroupInfo* __restrict__ groups, float* __restrict__ partials, float* __restrict__ D) {
+  griddep_wait();
+  griddep_launch();
   __shared__ float red[32];
   const Chunk ch = chunks[blockIdx.x];
   const MatInfo mi = mats[ch.mat];
@@ -790,6 +933,8 @@ k_mean_stage(const float* __restrict__ Mom, int64_t mom_stride, int M, void* __r
 __global__ void __launch_bounds__(kThreads)
 k_update(float* __restrict__ W, const float* __restrict__ D, int64_t d, float eta,
          const int* __restrict__ status) {
+  griddep_wait();
+  griddep_launch();
   if (status != nullptr && (status[0] | status[1]) != 0) return;  // keep W on error
   const int64_t n4 = d >> 2;
   const int64_t stride = (int64_t)gridDim.x * kThreads;
@@ -833,7 +978,7 @@ void launch_momentum(cudaStream_t s, const WorkerPtrs& G, const float* W, float*
                      int n_chunks, const MatInfo* mats, const GroupInfo* groups, float* partials) {
   if (n_chunks <= 0) return;
   count_launch();
-  k_momentum<true><<<n_chunks, kThreads, 0, s>>>(G, W, Mom, d, M, beta, lambda, X, x_bf16, chunks,
+  launch_pdl(k_momentum<true>, dim3(n_chunks), dim3(kThreads), 0, s, G, W, Mom, d, M, beta, lambda, X, x_bf16, chunks,
                                                  mats, groups, partials);
 }
 
@@ -842,7 +987,7 @@ void launch_stage(cudaStream_t s, const WorkerPtrs& in, int M, void* X, int x_bf
                   float* partials) {
   if (n_chunks <= 0) return;
   count_launch();
-  k_momentum<false><<<n_chunks, kThreads, 0, s>>>(in, nullptr, nullptr, 0, M, 0.f, 0.f, X, x_bf16,
+  launch_pdl(k_momentum<false>, dim3(n_chunks), dim3(kThreads), 0, s, in, nullptr, nullptr, 0, M, 0.f, 0.f, X, x_bf16,
                                                   chunks, mats, groups, partials);
 }
 
@@ -851,14 +996,14 @@ void launch_fro_finalize(cudaStream_t s, int n_probs, int n_mats, int M, const f
                          float eps, int quintic, float a, float b, float c, float* scale,
                          float2* coef_apply, float2* coef_square, int* status) {
   count_launch();
-  k_fro_finalize<<<n_probs, kThreads, 0, s>>>(n_mats, M, partials, mat_chunk0, mat_nchunks,
+  launch_pdl(k_fro_finalize, dim3(n_probs), dim3(kThreads), 0, s, n_mats, M, partials, mat_chunk0, mat_nchunks,
                                               use_for_scale, eps, quintic, a, b, c, scale,
                                               coef_apply, coef_square, status);
 }
 
 void launch_pi_init(cudaStream_t s, int n_probs, const int64_t* uoff, const int* prob_g, float* u, int warm) {
   count_launch();
-  k_pi_init<<<n_probs, kThreads, 0, s>>>(uoff, prob_g, u, warm);
+  launch_pdl(k_pi_init, dim3(n_probs), dim3(kThreads), 0, s, uoff, prob_g, u, warm);
 }
 
 void launch_pi_matvec(cudaStream_t s, const ProbRows* rows, int n_rows, const void* A, int a_bf16,
@@ -868,24 +1013,24 @@ void launch_pi_matvec(cudaStream_t s, const ProbRows* rows, int n_rows, const vo
   const size_t smem = (size_t)max_g * sizeof(float);
   if (a_bf16) {
     if (smem > 48 * 1024) cudaFuncSetAttribute(k_pi_matvec<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    k_pi_matvec<true><<<n_rows, kThreads, smem, s>>>(rows, A, prob_a_off, prob_g, prob_gld, uoff, u, y);
+    launch_pdl(k_pi_matvec<true>, dim3(n_rows), dim3(kThreads), smem, s, rows, A, prob_a_off, prob_g, prob_gld, uoff, u, y);
   } else {
     if (smem > 48 * 1024) cudaFuncSetAttribute(k_pi_matvec<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    k_pi_matvec<false><<<n_rows, kThreads, smem, s>>>(rows, A, prob_a_off, prob_g, prob_gld, uoff, u, y);
+    launch_pdl(k_pi_matvec<false>, dim3(n_rows), dim3(kThreads), smem, s, rows, A, prob_a_off, prob_g, prob_gld, uoff, u, y);
   }
 }
 
 void launch_pi_normalize(cudaStream_t s, int n_probs, const int64_t* uoff, const int* prob_g,
                          const float* y, float* u) {
   count_launch();
-  k_pi_normalize<<<n_probs, kThreads, 0, s>>>(uoff, prob_g, y, u);
+  launch_pdl(k_pi_normalize, dim3(n_probs), dim3(kThreads), 0, s, uoff, prob_g, y, u);
 }
 
 void launch_pi_finalize(cudaStream_t s, int n_probs, const int64_t* uoff, const int* prob_g,
                         const float* u, const float* y, float eps, int quintic, float a, float b,
                         float c, float* scale, float2* coef_apply, float2* coef_square, int* status) {
   count_launch();
-  k_pi_finalize<<<n_probs, kThreads, 0, s>>>(uoff, prob_g, u, y, eps, quintic, a, b, c, scale,
+  launch_pdl(k_pi_finalize, dim3(n_probs), dim3(kThreads), 0, s, uoff, prob_g, u, y, eps, quintic, a, b, c, scale,
                                              coef_apply, coef_square, status);
 }
 
@@ -895,7 +1040,7 @@ void launch_scale_flat(cudaStream_t s, const WorkerPtrs& in, int M, float* out, 
   if (n_chunks <= 0) return;
   count_launch();
   dim3 grid(n_chunks, M);
-  k_scale_flat<<<grid, kThreads, 0, s>>>(in, out, out_stride, chunks, mats, n_mats, scale, eps);
+  launch_pdl(k_scale_flat, dim3(grid), dim3(kThreads), 0, s, in, out, out_stride, chunks, mats, n_mats, scale, eps);
 }
 
 void launch_pack(cudaStream_t s, const float* U, int64_t u_stride, int64_t d, uint8_t* out,
@@ -905,14 +1050,16 @@ void launch_pack(cudaStream_t s, const float* U, int64_t u_stride, int64_t d, ui
   const int64_t warps = (d + 1023) / 1024;
   const int blocks = stream_grid((warps + 7) / 8, 16);
   dim3 grid(blocks, M);
-  k_pack<<<grid, kThreads, 0, s>>>(U, u_stride, d, out, out_stride);
+  launch_pdl(k_pack, dim3(grid), dim3(kThreads), 0, s, U, u_stride, d, out, out_stride);
 }
 
 // Full 4096-entry tiles by the streaming kernel (M <= 255), the rest (and
 // every entry for larger M) by the register kernel on offset pointers.
+// Worker m's packed signs start at signs.p[m] (16-byte aligned), which may
+// be this GPU's memory or a peer's mapped over NVLink.
 template <int MODE, bool ACC8>
-void vote_dispatch(cudaStream_t s, WorkerPtrs signs, const uint8_t* bits, int64_t bits_stride, int M, int64_t d,
-                   void* sums, int8_t* maj, float* W, float eta, float* D, const int* status, int tie_plus) {
+void vote_dispatch(cudaStream_t s, const WorkerPtrs& signs, int M, int64_t d, void* sums, int8_t* maj, float* W,
+                   float eta, float* D, const int* status, int tie_plus) {
   int64_t done = 0;
   if (M <= 255 && d >= 4096) {
     const int64_t ntiles = d / 4096;
@@ -921,52 +1068,59 @@ void vote_dispatch(cudaStream_t s, WorkerPtrs signs, const uint8_t* bits, int64_
     const int64_t cap = (int64_t)num_sms() * 6;
     const int blocks = (int)(want < cap ? want : cap);
     count_launch();
-    k_vote_stream<MODE, ACC8><<<blocks, kVoteWarps * 32, smem, s>>>(signs, bits, bits_stride, M, ntiles, sums, maj, W,
-                                                                     eta, D, status, tie_plus);
+    launch_pdl(k_vote_stream<MODE, ACC8>, dim3(blocks), dim3(kVoteWarps * 32), smem, s, signs, M, ntiles, sums, maj,
+               W, eta, D, status, tie_plus, VoteStage{});
     done = ntiles * 4096;
   }
   const int64_t rest = d - done;
   if (rest <= 0) return;
   const int64_t boff = done / 8;  // byte offset in every stream (a multiple of 512)
   WorkerPtrs sp = signs;
-  if (MODE == 0)
-    for (int m = 0; m < M; ++m) sp.p[m] = reinterpret_cast<const float*>(reinterpret_cast<const uint8_t*>(signs.p[m]) + boff);
+  for (int m = 0; m < M; ++m) sp.p[m] = reinterpret_cast<const float*>(reinterpret_cast<const uint8_t*>(signs.p[m]) + boff);
   void* sums2 = sums == nullptr ? nullptr : reinterpret_cast<uint8_t*>(sums) + done * (ACC8 ? 1 : 4);
   count_launch();
   const int blocks = stream_grid((rest / 512 + 8) / 8 + 1, 8);
-  k_vote<MODE, ACC8><<<blocks, kThreads, 0, s>>>(sp, bits == nullptr ? nullptr : bits + boff, bits_stride, M, rest, sums2,
-                                                 maj == nullptr ? nullptr : maj + done, W == nullptr ? nullptr : W + done,
-                                                 eta, D == nullptr ? nullptr : D + done, status, tie_plus);
+  launch_pdl(k_vote<MODE, ACC8>, dim3(blocks), dim3(kThreads), 0, s, sp, M, rest, sums2,
+             maj == nullptr ? nullptr : maj + done, W == nullptr ? nullptr : W + done, eta,
+             D == nullptr ? nullptr : D + done, status, tie_plus);
 }
 
 void launch_vote(cudaStream_t s, const WorkerPtrs& signs, int M, int64_t d, void* sums, int acc8,
                  int8_t* majority, int tie_plus) {
   if (d <= 0) return;
-  if (acc8) vote_dispatch<0, true>(s, signs, nullptr, 0, M, d, sums, majority, nullptr, 0.f, nullptr, nullptr, tie_plus);
-  else vote_dispatch<0, false>(s, signs, nullptr, 0, M, d, sums, majority, nullptr, 0.f, nullptr, nullptr, tie_plus);
+  if (acc8) vote_dispatch<0, true>(s, signs, M, d, sums, majority, nullptr, 0.f, nullptr, nullptr, tie_plus);
+  else vote_dispatch<0, false>(s, signs, M, d, sums, majority, nullptr, 0.f, nullptr, nullptr, tie_plus);
 }
 
-void launch_vote_update(cudaStream_t s, const uint8_t* bits, int64_t bits_stride, int M, int64_t d,
-                        float* W, float eta, const int* status, int tie_plus) {
+void launch_vote_update(cudaStream_t s, const WorkerPtrs& signs, int M, int64_t d, float* W, float eta,
+                        const int* status, int tie_plus) {
   if (d <= 0) return;
-  WorkerPtrs none{};
-  vote_dispatch<1, false>(s, none, bits, bits_stride, M, d, nullptr, nullptr, W, eta, nullptr, status, tie_plus);
+  vote_dispatch<1, false>(s, signs, M, d, nullptr, nullptr, W, eta, nullptr, status, tie_plus);
 }
 
-void launch_vote_major(cudaStream_t s, const uint8_t* bits, int64_t bits_stride, int M, int64_t d,
-                       float* D, int tie_plus) {
+void launch_vote_major(cudaStream_t s, const WorkerPtrs& signs, int M, int64_t d, float* D, int tie_plus) {
   if (d <= 0) return;
-  WorkerPtrs none{};
-  vote_dispatch<2, false>(s, none, bits, bits_stride, M, d, nullptr, nullptr, nullptr, 0.f, D, nullptr, tie_plus);
+  vote_dispatch<2, false>(s, signs, M, d, nullptr, nullptr, nullptr, 0.f, D, nullptr, tie_plus);
 }
 
-void launch_vote_stage(cudaStream_t s, const uint8_t* bits, int64_t bits_stride, int M, void* X, int x_bf16,
+void launch_vote_stage(cudaStream_t s, const WorkerPtrs& signs, int M, void* X, int x_bf16,
                        const Chunk* chunks, int n_chunks, const MatInfo* mats, const GroupInfo* groups,
-                       float* partials, float* D, int tie_plus) {
+                       float* partials, float* D, int tie_plus, int streamable) {
   if (n_chunks <= 0) return;
   count_launch();
-  k_vote_stage<<<n_chunks, kThreads, 0, s>>>(bits, bits_stride, M, X, x_bf16, chunks, mats, groups, partials, D,
-                                             tie_plus);
+  if (streamable && x_bf16 && M <= 255) {
+    // one warp per chunk, the next chunk's bytes in flight while one is counted
+    const size_t smem = (size_t)kVoteWarps * 2 * kVoteBatch * kVoteTileB;
+    const int64_t want = ((int64_t)n_chunks + kVoteWarps - 1) / kVoteWarps;
+    const int64_t cap = (int64_t)num_sms() * 6;
+    const int blocks = (int)(want < cap ? want : cap);
+    const VoteStage st{reinterpret_cast<__nv_bfloat16*>(X), chunks, mats, groups, partials};
+    launch_pdl(k_vote_stream<3, false>, dim3(blocks), dim3(kVoteWarps * 32), smem, s, signs, M, (int64_t)n_chunks,
+               nullptr, nullptr, nullptr, 0.f, D, nullptr, tie_plus, st);
+    return;
+  }
+  launch_pdl(k_vote_stage, dim3(n_chunks), dim3(kThreads), 0, s, signs, M, X, x_bf16, chunks, mats, groups, partials,
+             D, tie_plus);
 }
 
 void launch_mean_stage(cudaStream_t s, const float* Mom, int64_t mom_stride, int M, void* X, int x_bf16,
@@ -974,7 +1128,7 @@ void launch_mean_stage(cudaStream_t s, const float* Mom, int64_t mom_stride, int
                        float* partials, float* D) {
   if (n_chunks <= 0) return;
   count_launch();
-  k_mean_stage<<<n_chunks, kThreads, 0, s>>>(Mom, mom_stride, M, X, x_bf16, chunks, mats, groups, partials, D);
+  launch_pdl(k_mean_stage, dim3(n_chunks), dim3(kThreads), 0, s, Mom, mom_stride, M, X, x_bf16, chunks, mats, groups, partials, D);
 }
 
 void launch_update(cudaStream_t s, float* W, const float* D, int64_t d, float eta,
@@ -982,7 +1136,7 @@ void launch_update(cudaStream_t s, float* W, const float* D, int64_t d, float et
   if (d <= 0) return;
   count_launch();
   const int blocks = stream_grid((d / 4 + kThreads - 1) / kThreads + 1, 8);
-  k_update<<<blocks, kThreads, 0, s>>>(W, D, d, eta, status);
+  launch_pdl(k_update, dim3(blocks), dim3(kThreads), 0, s, W, D, d, eta, status);
 }
 
 }  // namespace sm

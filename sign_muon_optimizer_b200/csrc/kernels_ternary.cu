@@ -44,6 +44,8 @@ __device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kTThreads)
 k_sign8(const float* __restrict__ U, int64_t u_stride, int64_t d, int8_t* __restrict__ out, int64_t out_stride) {
+  griddep_wait();
+  griddep_launch();
   const int w = blockIdx.y;
   U += (int64_t)w * u_stride;
   out += (int64_t)w * out_stride;
@@ -82,6 +84,8 @@ __global__ void __launch_bounds__(kTThreads)
 k_vote_tern(WorkerPtrs signs, int M, int64_t d, void* __restrict__ sums, int8_t* __restrict__ maj,
             float* __restrict__ W, float eta, float* __restrict__ D, const int* __restrict__ status,
             int tie_plus) {
+  griddep_wait();
+  griddep_launch();
   if (MODE == 1 && status != nullptr && (status[0] | status[1]) != 0) return;
   const int64_t n16 = d >> 4;
   const int64_t stride = (int64_t)gridDim.x * kTThreads;
@@ -178,7 +182,7 @@ void vote_tern(cudaStream_t s, const WorkerPtrs& signs, int M, int64_t d, void* 
                float eta, float* D, const int* status, int tie_plus) {
   count_launch();
   const int blocks = stream_grid(((d >> 4) + kTThreads - 1) / kTThreads, 8);
-  k_vote_tern<MODE, ACC8><<<blocks, kTThreads, 0, s>>>(signs, M, d, sums, maj, W, eta, D, status, tie_plus);
+  launch_pdl(k_vote_tern<MODE, ACC8>, dim3(blocks), dim3(kTThreads), 0, s, signs, M, d, sums, maj, W, eta, D, status, tie_plus);
 }
 
 // D = majority of integer vote sums (int32, or int8 when ACC8): four entries
@@ -187,6 +191,8 @@ void vote_tern(cudaStream_t s, const WorkerPtrs& signs, int M, int64_t d, void* 
 template <bool ACC8>
 __global__ void __launch_bounds__(kTThreads)
 k_sums_major(const void* __restrict__ sums, int64_t d, float* __restrict__ D, int tie_plus) {
+  griddep_wait();
+  griddep_launch();
   const int64_t n4 = d >> 2;
   const int64_t stride = (int64_t)gridDim.x * kTThreads;
   for (int64_t i = (int64_t)blockIdx.x * kTThreads + threadIdx.x; i < n4; i += stride) {
@@ -208,12 +214,6 @@ k_sums_major(const void* __restrict__ sums, int64_t d, float* __restrict__ D, in
     }
 }
 
-WorkerPtrs strided_bytes(const int8_t* base, int64_t stride, int M) {
-  WorkerPtrs w{};
-  for (int m = 0; m < M; ++m) w.p[m] = reinterpret_cast<const float*>(base + (int64_t)m * stride);
-  return w;
-}
-
 }  // namespace
 
 // ---- launch wrappers --------------------------------------------------------
@@ -224,7 +224,7 @@ void launch_sign8(cudaStream_t s, const float* U, int64_t u_stride, int64_t d, i
   count_launch();
   const int blocks = stream_grid(((d >> 4) + kTThreads - 1) / kTThreads, 8);
   dim3 grid(blocks, M);
-  k_sign8<<<grid, kTThreads, 0, s>>>(U, u_stride, d, out, out_stride);
+  launch_pdl(k_sign8, dim3(grid), dim3(kTThreads), 0, s, U, u_stride, d, out, out_stride);
 }
 
 void launch_vote_ternary(cudaStream_t s, const WorkerPtrs& signs, int M, int64_t d, void* sums, int acc8,
@@ -234,26 +234,23 @@ void launch_vote_ternary(cudaStream_t s, const WorkerPtrs& signs, int M, int64_t
   else vote_tern<0, false>(s, signs, M, d, sums, majority, nullptr, 0.f, nullptr, nullptr, tie_plus);
 }
 
-void launch_vote_ternary_update(cudaStream_t s, const int8_t* signs, int64_t stride, int M, int64_t d, float* W,
-                                float eta, const int* status, int tie_plus) {
+void launch_vote_ternary_update(cudaStream_t s, const WorkerPtrs& signs, int M, int64_t d, float* W, float eta,
+                                const int* status, int tie_plus) {
   if (d <= 0) return;
-  vote_tern<1, false>(s, strided_bytes(signs, stride, M), M, d, nullptr, nullptr, W, eta, nullptr, status,
-                      tie_plus);
+  vote_tern<1, false>(s, signs, M, d, nullptr, nullptr, W, eta, nullptr, status, tie_plus);
 }
 
-void launch_vote_ternary_major(cudaStream_t s, const int8_t* signs, int64_t stride, int M, int64_t d, float* D,
-                               int tie_plus) {
+void launch_vote_ternary_major(cudaStream_t s, const WorkerPtrs& signs, int M, int64_t d, float* D, int tie_plus) {
   if (d <= 0) return;
-  vote_tern<2, false>(s, strided_bytes(signs, stride, M), M, d, nullptr, nullptr, nullptr, 0.f, D, nullptr,
-                      tie_plus);
+  vote_tern<2, false>(s, signs, M, d, nullptr, nullptr, nullptr, 0.f, D, nullptr, tie_plus);
 }
 
 void launch_sums_major(cudaStream_t s, const void* sums, int acc8, int64_t d, float* D, int tie_plus) {
   if (d <= 0) return;
   count_launch();
   const int blocks = stream_grid(((d >> 2) + kTThreads - 1) / kTThreads, 8);
-  if (acc8) k_sums_major<true><<<blocks, kTThreads, 0, s>>>(sums, d, D, tie_plus);
-  else k_sums_major<false><<<blocks, kTThreads, 0, s>>>(sums, d, D, tie_plus);
+  if (acc8) launch_pdl(k_sums_major<true>, dim3(blocks), dim3(kTThreads), 0, s, sums, d, D, tie_plus);
+  else launch_pdl(k_sums_major<false>, dim3(blocks), dim3(kTThreads), 0, s, sums, d, D, tie_plus);
 }
 
 }  // namespace sm

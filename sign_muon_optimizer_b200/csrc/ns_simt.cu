@@ -74,6 +74,8 @@ __device__ __forceinline__ void store_slab(const Operand& o, float (*s)[TM + 4],
 
 __global__ void __launch_bounds__(NT)
 k_gemm_simt(const __grid_constant__ GemmArgs a) {
+  griddep_wait();
+  griddep_launch();
   __shared__ __align__(16) float As[2][TK][TM + 4];
   __shared__ __align__(16) float Bs[2][TK][TN + 4];
 
@@ -183,7 +185,7 @@ k_gemm_simt(const __grid_constant__ GemmArgs a) {
 void launch_gemm_simt(cudaStream_t s, const GemmArgs& a, int /*x_f32*/) {
   if (a.total_tiles <= 0) return;
   count_launch();
-  k_gemm_simt<<<a.total_tiles, NT, 0, s>>>(a);
+  launch_pdl(k_gemm_simt, dim3(a.total_tiles), dim3(NT), 0, s, a);
 }
 
 }  // namespace sm

@@ -11,19 +11,20 @@
 // 2*128*BN*64 flops (a one-SM 128 x BN tile needs 48 KB).  Per CTA, 384
 // threads:
 //   warps 0..2  TMA producers taking turns over the k-blocks: bf16 boxes of
-//               64 columns (128-byte swizzle) into a 6-deep ring, one box per
+//               64 columns (128-byte swizzle) into a 7-stage ring (6 for
+//               APPLY and SQUARE, whose epilogue takes the last), one box per
 //               lane; both CTAs' loads complete on the leader CTA's "full"
 //               barrier
 //   warp 3      allocates 512 TMEM columns (cta_group::2); in the leader CTA
 //               one lane issues tcgen05.mma.cta_group::2 (M=256, N=BN, K=16)
 //               and tcgen05.commit multicast to both CTAs' barriers
-//   warps 4..11 epilogue, each on its own 32-row x BN/2 slice of the tile,
-//               one 32 x 64 atom at a time: the atom of the affine operand (X
-//               for APPLY, A for SQUARE) comes into shared memory by TMA;
-//               tcgen05.ld 32x32b.x32 -> a*operand + b*acc -> bf16 results
-//               written over the operand -> TMA store of the atom.  The last
-//               APPLY of a step writes sign bits (and U / D in fp32 only when
-//               asked for) instead.
+//   warps 4..11 epilogue, each on its own 32-row x BN/2 slice of the tile:
+//               per 32-column chunk tcgen05.ld 32x32b.x32 -> (APPLY, SQUARE)
+//               a*operand + b*acc, the operand's 32 x 64 atom brought into a
+//               4 KB shared-memory slice by TMA -> bf16 results stored
+//               straight to global memory (64 bytes per lane and row, no
+//               shared memory).  The last APPLY of a step writes sign bits
+//               (and U / D in fp32 only when asked for) instead.
 // The Gram matrix is symmetric: only tiles on or above the diagonal are
 // computed, and the epilogue also writes each off-diagonal tile transposed.
 // Every mbarrier wait is bounded (2 s): on expiry the CTA records
@@ -40,13 +41,17 @@ constexpr int BOX_BYTES = 64 * 64 * 2;                  // one 64x64 bf16 TMA bo
 constexpr int A_BYTES = 128 * BK * 2;                   // 16 KB: this CTA's 128 rows of A
 constexpr int B_BYTES = 128 * BK * 2;                   // 16 KB: this CTA's BN/2 <= 128 rows of B
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int EPI_BYTES = 8 * 32 * 64 * 2;              // 32 KB: one 32x64 atom per epilogue warp
-// Shared memory: a 6-deep operand ring and the epilogue's staging atoms
-// (224 KB).  The ring depth is what hides the operand latency: a freed stage
-// is refilled ~2,500 cycles later under load, against ~650 cycles of MMA work
-// per stage.
-constexpr int RING = 6, RING_MAX = RING;
-constexpr int DATA_BYTES = RING * STAGE_BYTES + EPI_BYTES;
+// Shared memory: a 7-stage operand ring (224 KB) and the barriers.  The ring
+// depth is what hides the operand latency: a freed stage is refilled ~2,500
+// cycles later under load, against 500-700 cycles of MMA work per stage.  The
+// ring's TMA writes and the tensor cores' operand reads already take about
+// all of the SM's shared-memory bandwidth at full MMA rate, so the epilogue
+// stores its results straight to global memory; only the affine operand of
+// APPLY and SQUARE passes through shared memory (TMA in, one read), in the
+// last stage's 32 KB, which those launches take out of the ring.
+constexpr int RING = 7, RING_MAX = RING;
+constexpr int EPI_SLICE = 32 * 64 * 2;                  // 4 KB: one 32 x 64 operand atom per epilogue warp
+constexpr int DATA_BYTES = RING * STAGE_BYTES;
 constexpr int TMEM_COLS = 512;
 // Warp roles.  A warp completes only about one TMA load instruction every
 // 500-700 cycles however many it has in flight, while the lanes of one
@@ -108,15 +113,6 @@ __device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cl_addr) {
 __device__ __forceinline__ void mbar_expect_tx_relaxed(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.relaxed.cta.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
 }
-// shared-memory 16-byte load / store by shared-window address
-__device__ __forceinline__ uint4 lds128(uint32_t addr) {
-  uint4 v;
-  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
-  return v;
-}
-__device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
-  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
-}
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -159,18 +155,13 @@ __device__ __forceinline__ void tma_load_pair(uint32_t dst, const void* map, uin
       ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar_cl)
       : "memory");
 }
-// 2-SM TMA load of a 4-D box (the two-atom views of slots 12/13)
+// 2-SM TMA load of a 4-D box (the two-atom views of slots 8/9)
 __device__ __forceinline__ void tma_load_pair4(uint32_t dst, const void* map, uint32_t bar_cl, int x, int y, int z,
                                                int w) {
   asm volatile(
       "cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], [%6];"
       ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(bar_cl)
       : "memory");
-}
-__device__ __forceinline__ void tma_store3(const void* map, uint32_t src, int x, int y, int z) {
-  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%1, %2, %3}], [%4];"
-               ::"l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(src)
-               : "memory");
 }
 // plain one-CTA TMA load completing on this CTA's barrier
 __device__ __forceinline__ void tma_load_local(uint32_t dst, const void* map, uint32_t bar, int x, int y, int z) {
@@ -232,25 +223,76 @@ __device__ __forceinline__ uint32_t instr_desc(int a_mn, int b_mn, int n) {
          ((uint32_t)(n >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
 }
 
+// ---- the epilogue's direct global accesses --------------------------------
+__device__ __forceinline__ void stg_v8(void* p, const uint32_t* w) {
+  asm volatile("st.global.v8.u32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
+               ::"l"(p), "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+               : "memory");
+}
+// the first n (1..32) of 32 bf16 (pairs in w) to one row at p (16-byte aligned)
+__device__ __forceinline__ void store_row_chunk(__nv_bfloat16* p, int n, const uint32_t (&w)[16]) {
+  if (n >= 32 && (reinterpret_cast<uintptr_t>(p) & 31u) == 0) {
+    stg_v8(p, &w[0]);
+    stg_v8(p + 16, &w[8]);
+    return;
+  }
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    if (8 * g + 8 <= n) {
+      *reinterpret_cast<uint4*>(p + 8 * g) = make_uint4(w[4 * g], w[4 * g + 1], w[4 * g + 2], w[4 * g + 3]);
+    } else {
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (8 * g + u < n) {
+          const uint32_t pair = w[4 * g + u / 2];
+          const unsigned short h = (u & 1) ? (unsigned short)(pair >> 16) : (unsigned short)(pair & 0xFFFFu);
+          reinterpret_cast<unsigned short*>(p)[8 * g + u] = h;
+        }
+      }
+    }
+  }
+}
+// the first n (1..32) of 32 floats to p (any 4-byte alignment)
+__device__ __forceinline__ void store_row_f32(float* p, int n, const float (&v)[32]) {
+  const uintptr_t al = reinterpret_cast<uintptr_t>(p);
+  if (n >= 32 && (al & 31u) == 0) {
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      uint32_t w8[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) w8[u] = __float_as_uint(v[8 * g + u]);
+      stg_v8(p + 8 * g, w8);
+    }
+    return;
+  }
+  if ((al & 15u) == 0) {
+#pragma unroll
+    for (int g = 0; g < 8; ++g) {
+      if (4 * g + 4 <= n) {
+        *reinterpret_cast<float4*>(p + 4 * g) = make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+      } else {
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (4 * g + u < n) p[4 * g + u] = v[4 * g + u];
+      }
+    }
+    return;
+  }
+#pragma unroll
+  for (int u = 0; u < 32; ++u)
+    if (u < n) p[u] = v[u];
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
 }
-__device__ __forceinline__ void unpack_bf16x8(uint4 u, float* f) {
-  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 t = __bfloat1622float2(h[i]);
-    f[2 * i] = t.x;
-    f[2 * i + 1] = t.y;
-  }
-}
 // Tensor-map slots per group: 0/1 = X ping/pong, 2 = A, 3 = B, with 64-row
-// boxes; the same four with 128-row boxes at slot + 4 and with 32-row boxes
-// (an epilogue warp's atom) at slot + 8.  When X's column count is a
-// multiple of 64, slots 12/13 hold X ping/pong as 4-D views (64-column atom,
-// row, atom index, matrix) with a box of two atoms x 64 rows: an MN-major
-// operand half of a k-block in one request.
+// boxes; the same four with 128-row boxes at slot + 4.  When X's column
+// count is a multiple of 64, slots 8/9 hold X ping/pong as 4-D views
+// (64-column atom, row, atom index, matrix) with a box of two atoms x 64
+// rows: an MN-major operand half of a k-block in one request.  Slots 10..13
+// hold the first four with 32-row boxes (an epilogue warp's operand atom).
 __device__ __forceinline__ const CUtensorMap* map_at(const CUtensorMap* maps, int group, int slot) {
   return maps + group * kMapsPerGroup + slot;
 }
@@ -263,8 +305,9 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* gbase = smem_raw + (base - raw);
   const int op = a.op;
-  const int nst = RING;                                        // operand ring depth
-  const uint32_t epi0 = base + nst * STAGE_BYTES;              // staging tile
+  const bool affine = op != OP_GRAM;                           // epilogue reads an operand
+  const int nst = affine ? RING - 1 : RING;                    // operand ring depth
+  const uint32_t epi0 = base + (RING - 1) * STAGE_BYTES;       // operand slices (affine)
   uint64_t* bars = reinterpret_cast<uint64_t*>(gbase + DATA_BYTES);
   // bars: full[RING_MAX], empty[RING_MAX], tmem_full[2], tmem_empty[2],
   // epi_full[8] (one per epilogue warp)
@@ -303,6 +346,10 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
   __syncthreads();
   cluster_sync();   // the peer's barriers are initialised before any remote arrive
   tc_fence_after();
+  // the prologue above touches no global memory: it overlaps the end of the
+  // previous kernel on the stream
+  griddep_wait();
+  griddep_launch();
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp < NPROD) {
@@ -342,7 +389,7 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
       // atoms when X's column count is a multiple of 64, else as one 64x64
       // box per 64 MN indices.
       const bool x4 = (gi.cols % 64) == 0;
-      const CUtensorMap* mX4 = map_at(maps, tc.group, 12 + a.map_src);
+      const CUtensorMap* mX4 = map_at(maps, tc.group, 8 + a.map_src);
       const int nA = amn ? (x4 ? 1 : 2) : 1;
       const int nB = bmn ? ((x4 && hb == 128) ? 1 : hb / 64) : 1;
       const bool box_a = lane < nA, box_b = !box_a && lane < nA + nB;
@@ -396,6 +443,12 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
         const uint64_t t0 = globaltimer();
         while (!mbar_try_wait(full_bar(s), par) && globaltimer() - t0 < kTimeoutNs) {}
       }
+    } else if (!ok && lane == 0 && issued != 0) {
+      // The peer CTA's loads complete on the leader's barriers, which this
+      // CTA cannot wait on: give the loads it issued time to land (a load
+      // takes microseconds; 50 us is a bound on a live memory system).
+      const uint64_t t0 = globaltimer();
+      while (globaltimer() - t0 < 50000ull) {}
     }
   } else if (warp == MMA_WARP) {
     // ---------------- MMA issuer (leader CTA) ----------------
@@ -408,6 +461,7 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
       int last_acc = 0;
       uint32_t last_acc_par = 0;
       bool ok = true;
+      bool pending_mma = false;     // MMAs issued since the last accumulator commit
       // the next tile is decoded while the current one's first MMAs run, so
       // that a tile boundary costs the MMA queue no decode time
       TileCoord tn = decode_tile(a, cid < a.total_tiles ? cid : 0);
@@ -431,16 +485,26 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
             const uint64_t bd = bmn ? desc_mnmajor(sb + kk * 2048) : desc_kmajor(sb + kk * 32);
             tc_mma(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
           }
+          pending_mma = true;
           tc_commit_pair(empty_bar(stage));
           if (++stage == nst) { stage = 0; phase ^= 1u; }
           if (kb == 0 && tile + ncl < a.total_tiles) tn = decode_tile(a, tile + ncl);
         }
         if (!ok) break;
         tc_commit_pair(tfull_bar(acc));
+        pending_mma = false;
         committed++;
         last_acc = acc;
         last_acc_par = acc_phase;
         if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      }
+      if (!ok && pending_mma) {
+        // a tile aborted after some of its MMAs went out: commit them too, so
+        // that the wait below covers every MMA before TMEM is freed
+        tc_commit_pair(tfull_bar(acc));
+        committed++;
+        last_acc = acc;
+        last_acc_par = acc_phase;
       }
       if (!ok && committed > 0) {
         const uint64_t t0 = globaltimer();
@@ -448,35 +512,35 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
       }
     }
   } else {
-    // ---------------- epilogue (warps 6..13, both CTAs) ----------------
-    // Warp e = warp - 6 owns rows 32*q .. 32*q+31 of the CTA's 128 (its TMEM
-    // lane quarter q = warp % 4) and the column half e / 4 of the tile, i.e.
-    // one 32-row slice of one or two 64-column atoms of the staging tile
-    // (swizzled box layout [atom][128 rows][128 B]).  Each warp runs on its
-    // own: it TMA-loads its slice of the affine operand (X for APPLY, A for
-    // SQUARE), drains its accumulator slice, writes bf16 results over the
-    // operand and TMA-stores the slice, with no barrier between warps.
+    // ---------------- epilogue (warps 4..11, both CTAs) ----------------
+    // Warp e = warp - 4 owns rows 32 q .. 32 q + 31 of the CTA's 128 (its TMEM
+    // lane quarter q = warp % 4; lane i holds row 32 q + i) and the column
+    // half e / 4 of the tile, i.e. BN/64 chunks of 32 columns.  It uses no
+    // shared memory, which the operand ring and the tensor cores keep busy:
+    // the affine operand of all its chunks (X for APPLY, A for SQUARE) is
+    // loaded into registers before the accumulator is ready; then, chunk by
+    // chunk, tcgen05.ld 32x32b.x32, the fp32 combination c0 * operand +
+    // c1 * acc, and 64 contiguous bytes of bf16 per lane stored straight to
+    // global memory (two 32-byte stores when aligned).  The last APPLY of a
+    // step writes the sign bits (and U / D in fp32 only when asked for).
     const int e = warp - EPI_WARP0;
     const int q = warp & 3;                // TMEM lane quarter this warp may access
     const int half = e >> 2;               // column half of the tile
-    const int rloc = q * 32 + lane;        // row within this CTA's 128 rows
-    const bool affine = op != OP_GRAM;
     const bool final_out = (op == OP_APPLY) && a.final_out;
     const uint32_t tempty_leader0 = leader_addr(tempty_bar(0));
     const uint32_t tempty_leader1 = leader_addr(tempty_bar(1));
+    __nv_bfloat16* dst_base =
+        reinterpret_cast<__nv_bfloat16*>(op == OP_GRAM ? a.A : (op == OP_SQUARE ? a.B : a.X_dst));
+    // This warp's operand slice: one 32-row x 64-column atom (128-byte rows,
+    // 128-byte swizzle) of the affine operand at a time, by TMA.
+    const uint32_t slice = epi0 + (uint32_t)e * EPI_SLICE;
     const uint32_t my_efull = efull_bar(e);
-    // This warp's staging slice is one atom, 32 rows x 64 columns (4 KB,
-    // 128-byte rows, swizzled); the warp's 64- or 128-column part of a tile
-    // passes through it one atom at a time.
-    const uint32_t slice = epi0 + (uint32_t)e * 4096u;
-    const int opnd_slot = (op == OP_SQUARE) ? 2 : a.map_src;
-    const int dst_slot = (op == OP_GRAM) ? 2 : (op == OP_SQUARE ? 3 : a.map_dst);
-    // atom i (of this warp's part) of a tile's affine operand, 64 x 32 box
+    const int opnd_slot = 10 + ((op == OP_SQUARE) ? 2 : a.map_src);
     auto load_operand = [&](const TileCoord& t2, int i) {
-      const int j = half * (t2.BN / 128) + i;
+      const int j = half * (t2.BN / 128) + i;   // atom index within the tile
       if (lane == 0) {
-        mbar_expect_tx_relaxed(my_efull, 4096u);
-        tma_load_local(slice, map_at(maps, t2.group, 8 + opnd_slot), my_efull, t2.n0 + 64 * j,
+        mbar_expect_tx_relaxed(my_efull, (uint32_t)EPI_SLICE);
+        tma_load_local(slice, map_at(maps, t2.group, opnd_slot), my_efull, t2.n0 + 64 * j,
                        t2.m0 + 128 * (int)rank + 32 * q, t2.b);
       }
     };
@@ -486,24 +550,11 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
       load_operand(decode_tile(a, cid), 0);
       load_pending = true;
     }
-    // lane 0 waits for my operand barrier; false if the wait gave up
-    auto wait_operand = [&]() {
-      int okw = 1;
-      if (lane == 0) okw = mbar_wait(my_efull, e_par, abort_flag, a.err) ? 1 : 0;
-      okw = __shfl_sync(0xffffffffu, okw, 0);
-      if (okw) {
-        e_par ^= 1u;
-        load_pending = false;
-      }
-      return okw != 0;
-    };
     int acc = 0;
     uint32_t acc_phase = 0;
-    bool alive = true;
-    for (int tile = cid; tile < a.total_tiles && alive; tile += ncl) {
+    for (int tile = cid; tile < a.total_tiles; tile += ncl) {
       const TileCoord tc = decode_tile(a, tile);
       const bool more = tile + ncl < a.total_tiles;
-      const TileCoord tnext = decode_tile(a, more ? tile + ncl : tile);
       const GroupInfo gi = group_info(a, tc.group);
       int mat = 0;
       const int p = problem_id(a, gi, tc.b, &mat);
@@ -513,13 +564,16 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
         c0 = cf.x;
         c1 = cf.y;
       }
-      const int rbase = tc.m0 + 128 * (int)rank;
-      const int row = rbase + rloc;
+      const int row = tc.m0 + 128 * (int)rank + q * 32 + lane;
       const bool row_ok = row < tc.Mdim;
-      const int64_t aoff = gi.a_base + (int64_t)tc.b * gi.g * gi.gld;
+      const int atoms = tc.BN / 128;                  // 64-column atoms of this warp (1 or 2)
+      const int ch0 = half * (tc.BN / 64);            // first 32-column chunk of this warp
+      // X (APPLY) rows have stride ld; the Gram A and the quintic B stride gld
+      const bool on_x = op == OP_APPLY;
+      const int64_t ldm = on_x ? gi.ld : gi.gld;
+      const int64_t mrow = (on_x ? gi.x_base + (int64_t)tc.b * gi.rows * gi.ld
+                                 : gi.a_base + (int64_t)tc.b * gi.g * gi.gld) + (int64_t)row * ldm;
       const int w = tc.b / gi.count;
-      const int atoms = tc.BN / 128;                 // atoms of this warp
-      const int ch0 = half * (tc.BN / 64);           // first 32-column chunk
       int okw = 1;
       if (lane == 0) okw = mbar_wait(tfull_bar(acc), acc_phase, abort_flag, a.err) ? 1 : 0;
       okw = __shfl_sync(0xffffffffu, okw, 0);
@@ -528,144 +582,98 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
       // symmetric Gram: an off-diagonal tile is also written transposed
       const bool mirror = (op == OP_GRAM) && (tc.n0 != tc.m0);
       const uint32_t tm_row = tmem_base + (uint32_t)(acc * 256) + ((uint32_t)(q * 32) << 16);
-      // results of one 32-column chunk from its accumulator registers
-      auto form = [&](int ch, uint32_t (&rr)[32]) {
-        float v[32];
-#pragma unroll
-        for (int u = 0; u < 32; ++u) v[u] = __uint_as_float(rr[u]);
-        const int col0 = tc.n0 + ch * 32;
-        const bool live = row_ok && col0 < tc.Ndim;
-        const int ncol = live ? min(32, tc.Ndim - col0) : 0;
-        const uint32_t rowa = slice + (uint32_t)(lane * 128);
-        if (affine) {
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const uint4 xo = lds128(rowa + (uint32_t)((((ch & 1) * 4 + u) ^ (lane & 7)) * 16));
-            float xv[8];
-            unpack_bf16x8(xo, xv);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) v[8 * u + i] = fmaf(c0, xv[i], c1 * v[8 * u + i]);
-          }
-        }
-        if (final_out) {
-          // fp32 results go back into rr for write_out_f32; the signs (when
-          // asked for) are one LSB-first word of the bit stream per chunk
-#pragma unroll
-          for (int u = 0; u < 32; ++u) rr[u] = __float_as_uint(v[u]);
-          if (live && a.out_bits != nullptr) {
-            const int64_t flat = a.mat_off[mat] + (int64_t)row * gi.cols + col0;
-            uint32_t word = 0;
-#pragma unroll
-            for (int u = 0; u < 32; ++u) word |= (v[u] >= 0.f ? 1u : 0u) << u;
-            a.out_bits[(int64_t)w * a.bits_stride + (flat >> 5)] = word;
-          }
-          (void)ncol;
-          return;
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int unit = ((ch & 1) * 4 + u) ^ (lane & 7);
-          uint4 o;
-          o.x = pack_bf16x2(v[8 * u + 0], v[8 * u + 1]);
-          o.y = pack_bf16x2(v[8 * u + 2], v[8 * u + 3]);
-          o.z = pack_bf16x2(v[8 * u + 4], v[8 * u + 5]);
-          o.w = pack_bf16x2(v[8 * u + 6], v[8 * u + 7]);
-          sts128(rowa + (uint32_t)(unit * 16), o);
-        }
-        if (mirror && live) {
-          // lanes hold consecutive rows: each store below is 64 contiguous bytes
-          __nv_bfloat16* A = reinterpret_cast<__nv_bfloat16*>(a.A) + aoff;
-#pragma unroll
-          for (int u = 0; u < 32; ++u)
-            if (u < ncol) A[(int64_t)(col0 + u) * gi.gld + row] = __float2bfloat16_rn(v[u]);
-        }
-      };
-      // fp32 output of one chunk (final APPLY): the warp's 32 rows x 32
-      // columns pass through the slice (one 128-byte swizzled row per lane),
-      // then each store instruction writes four whole 128-byte row segments
-      auto write_out_f32 = [&](int ch, uint32_t (&rr)[32]) {
-        __syncwarp();
-#pragma unroll
-        for (int u = 0; u < 8; ++u)
-          sts128(slice + (uint32_t)(lane * 128 + ((u ^ (lane & 7)) * 16)),
-                 make_uint4(rr[4 * u], rr[4 * u + 1], rr[4 * u + 2], rr[4 * u + 3]));
-        __syncwarp();
-        const int uu = lane & 7;
-        const int colg = tc.n0 + ch * 32 + uu * 4;
-#pragma unroll 2
-        for (int it = 0; it < 8; ++it) {
-          const int rl = it * 4 + (lane >> 3);
-          const int rowg = rbase + q * 32 + rl;
-          if (rowg >= tc.Mdim || colg >= tc.Ndim) continue;
-          const uint4 val = lds128(slice + (uint32_t)(rl * 128 + ((uu ^ (rl & 7)) * 16)));
-          float* dst = a.out + (int64_t)w * a.out_stride + a.mat_off[mat] + (int64_t)rowg * gi.cols + colg;
-          if (colg + 3 < tc.Ndim && ((reinterpret_cast<uintptr_t>(dst) & 15u) == 0)) {
-            *reinterpret_cast<uint4*>(dst) = val;
-          } else {
-            const uint32_t e4[4] = {val.x, val.y, val.z, val.w};
-#pragma unroll
-            for (int t = 0; t < 4; ++t)
-              if (colg + t < tc.Ndim) dst[t] = __uint_as_float(e4[t]);
-          }
-        }
-      };
+      bool alive = true;
 #pragma unroll 1
       for (int i = 0; i < atoms; ++i) {
-        const int ch = ch0 + 2 * i;
-        // the atom's operand has landed (affine); the slice is free of my
-        // previous store (Gram)
         if (affine) {
-          if (!wait_operand()) { alive = false; break; }
-        } else {
-          asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-          __syncwarp();
+          // the atom's operand has landed
+          int okw2 = 1;
+          if (lane == 0) okw2 = mbar_wait(my_efull, e_par, abort_flag, a.err) ? 1 : 0;
+          okw2 = __shfl_sync(0xffffffffu, okw2, 0);
+          if (!okw2) { alive = false; break; }
+          e_par ^= 1u;
+          load_pending = false;
         }
-        // two 32-column chunks per TMEM round trip; the accumulator slice is
-        // released after its last TMEM load
-        uint32_t r[2][32];
-        tmem_ld32_async(tm_row + (uint32_t)(ch * 32), r[0]);
-        tmem_ld32_async(tm_row + (uint32_t)((ch + 1) * 32), r[1]);
-        tmem_wait_ld();
-        reg_fence(r[0]);
-        reg_fence(r[1]);
-        if (i + 1 == atoms) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive_cluster_relaxed(acc == 0 ? tempty_leader0 : tempty_leader1);
-        }
-        form(ch, r[0]);
-        form(ch + 1, r[1]);
-        if (final_out && a.out != nullptr) {
-          write_out_f32(ch, r[0]);
-          write_out_f32(ch + 1, r[1]);
-        }
-        // make the staged results visible to the TMA (async proxy), store
-        // the atom (one 64 x 32 box in a bulk group of its own)
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        __syncwarp();
-        if (!final_out && lane == 0) {
-          const int x = tc.n0 + 64 * (half * atoms + i), y = rbase + 32 * q;
-          if (y < tc.Mdim && x < tc.Ndim) {
-            tma_store3(map_at(maps, tc.group, 8 + dst_slot), slice, x, y, tc.b);
-            asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+#pragma unroll
+        for (int hc = 0; hc < 2; ++hc) {
+          const int ch = ch0 + 2 * i + hc;
+          const int col0 = tc.n0 + ch * 32;
+          uint32_t r[32];
+          tmem_ld32_async(tm_row + (uint32_t)(ch * 32), r);
+          tmem_wait_ld();
+          reg_fence(r);
+          if (i + 1 == atoms && hc == 1) {
+            // the accumulator slice is free once its last TMEM load is done
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster_relaxed(acc == 0 ? tempty_leader0 : tempty_leader1);
+          }
+          float v[32];
+#pragma unroll
+          for (int u = 0; u < 32; ++u) v[u] = __uint_as_float(r[u]);
+          if (affine) {
+            // this lane's row of the chunk: 4 swizzled 16-byte units of the atom
+            const uint32_t rowa = slice + (uint32_t)(lane * 128);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              uint4 xo;
+              asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                           : "=r"(xo.x), "=r"(xo.y), "=r"(xo.z), "=r"(xo.w)
+                           : "r"(rowa + (uint32_t)(((hc * 4 + u) ^ (lane & 7)) * 16)));
+              const uint32_t xw[4] = {xo.x, xo.y, xo.z, xo.w};
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xw[k]));
+                v[8 * u + 2 * k] = fmaf(c0, x.x, c1 * v[8 * u + 2 * k]);
+                v[8 * u + 2 * k + 1] = fmaf(c0, x.y, c1 * v[8 * u + 2 * k + 1]);
+              }
+            }
+          }
+          const bool live = row_ok && col0 < tc.Ndim;
+          const int ncol = live ? min(32, tc.Ndim - col0) : 0;
+          if (final_out) {
+            if (live && a.out_bits != nullptr) {
+              // one LSB-first word of the bit stream (every matrix has a
+              // multiple of 32 columns when the signs are packed here)
+              const int64_t flat = a.mat_off[mat] + (int64_t)row * gi.cols + col0;
+              uint32_t word = 0;
+#pragma unroll
+              for (int u = 0; u < 32; ++u) word |= (v[u] >= 0.f ? 1u : 0u) << u;
+              a.out_bits[(int64_t)w * a.bits_stride + (flat >> 5)] = word;
+            }
+            if (live && a.out != nullptr) {
+              float* dst = a.out + (int64_t)w * a.out_stride + a.mat_off[mat] + (int64_t)row * gi.cols + col0;
+              store_row_f32(dst, ncol, v);
+            }
+            continue;
+          }
+          uint32_t ow[16];
+#pragma unroll
+          for (int k = 0; k < 16; ++k) ow[k] = pack_bf16x2(v[2 * k], v[2 * k + 1]);
+          if (live) store_row_chunk(dst_base + mrow + col0, ncol, ow);
+          if (mirror && live) {
+            // lanes hold consecutive rows: each store below is 64 contiguous bytes
+            __nv_bfloat16* At = reinterpret_cast<__nv_bfloat16*>(a.A) + gi.a_base + (int64_t)tc.b * gi.g * gi.gld;
+#pragma unroll
+            for (int u = 0; u < 32; ++u)
+              if (u < ncol) At[(int64_t)(col0 + u) * gi.gld + row] = __float2bfloat16_rn(v[u]);
           }
         }
         if (affine) {
-          // the slice takes the next operand atom once my store has read it
-          if (!final_out) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+          // the slice takes the next atom once every lane has read this one
           __syncwarp();
           if (i + 1 < atoms) {
             load_operand(tc, i + 1);
             load_pending = true;
           } else if (more) {
-            load_operand(tnext, 0);
+            load_operand(decode_tile(a, tile + ncl), 0);
             load_pending = true;
           }
         }
       }
+      if (!alive) break;
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
-    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
     if (load_pending && lane == 0) {
       // a wait gave up with an operand load in flight: let it land
       const uint64_t t0 = globaltimer();
@@ -695,7 +703,7 @@ void launch_gemm_tc(cudaStream_t s, const GemmArgs& a, const void* maps, int n_s
   count_launch();
   const int pairs = n_sm / 2;
   const int clusters = a.total_tiles < pairs ? a.total_tiles : pairs;
-  k_gemm_tc<<<2 * clusters, NTHREADS, SMEM_BYTES, s>>>(a, reinterpret_cast<const CUtensorMap*>(maps));
+  launch_pdl(k_gemm_tc, dim3(2 * clusters), dim3(NTHREADS), SMEM_BYTES, s, a, reinterpret_cast<const CUtensorMap*>(maps));
 }
 
 }  // namespace sm

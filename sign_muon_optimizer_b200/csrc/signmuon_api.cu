@@ -211,6 +211,13 @@ sm::WorkerPtrs strided_ptrs(const float* base, int64_t stride, int M) {
   return w;
 }
 
+// worker m's sign buffer at base + m * stride bytes
+sm::WorkerPtrs byte_ptrs(const uint8_t* base, int64_t stride, int M) {
+  sm::WorkerPtrs w{};
+  for (int m = 0; m < M; ++m) w.p[m] = reinterpret_cast<const float*>(base + (int64_t)m * stride);
+  return w;
+}
+
 // NVTX range names of the profiling kinds (signmuon_profile's numbering)
 const char* const kKindNames[SIGNMUON_PROF_KINDS] = {
     "signmuon momentum",      "signmuon norm finalize",  "signmuon NS gram",       "signmuon NS square",
@@ -335,6 +342,16 @@ void power_iteration(signmuon_t h, int nw) {
                        h->d_prob_gld, h->d_uoff, u, h->pi_y, max_g);
   sm::launch_pi_finalize(h->stream, nprob, h->d_uoff, h->d_prob_g, u, h->pi_y, h->eps, p.quintic ? 1 : 0,
                          h->ns_a, h->ns_b, h->ns_c, h->scale_v, h->coef_apply, h->coef_square, h->status);
+}
+
+// The streaming vote kernel stages the post-vote input when every matrix
+// starts at a multiple of 128 entries (16-byte aligned in every bit stream)
+// and has a multiple of 8 columns (its rows are unpadded in X, so a chunk's
+// range is contiguous there).
+bool stage_streamable(signmuon_t h) {
+  for (const sm::MatInfo& mi : h->plan.mats)
+    if ((mi.off % 128) != 0 || (mi.cols % 8) != 0) return false;
+  return true;
 }
 
 bool signs_in_gemm(signmuon_t h) {
@@ -664,9 +681,9 @@ int signmuon_init(signmuon_t* out, const int64_t* shapes, int n_mats, int M, flo
     return bail(fail(h, SIGNMUON_E_CUDA, "memset"));
   if (!p.fp32) {
     // per group: slots 0..3 = X ping, X pong, A, B with 64-row boxes;
-    // slots 4..7 = the same tensors with 128-row boxes; slots 8..11 with
-    // 32-row boxes; when X's column count is a multiple of 64, X ping/pong
-    // as 4-D atom views with 2-atom x 64-row boxes at 12/13
+    // slots 4..7 = the same tensors with 128-row boxes; when X's column
+    // count is a multiple of 64, X ping/pong as 4-D atom views with 2-atom x
+    // 64-row boxes at 8/9; slots 10..13 = the first four with 32-row boxes
     std::vector<CUtensorMap> maps(p.groups.size() * sm::kMapsPerGroup);
     std::memset(maps.data(), 0, maps.size() * sizeof(CUtensorMap));
     for (size_t g = 0; g < p.groups.size(); ++g) {
@@ -674,7 +691,7 @@ int signmuon_init(signmuon_t* out, const int64_t* shapes, int n_mats, int M, flo
       const int batch = M * gi.count;
       for (int box = 0; box < 3; ++box) {
         const int br = box == 0 ? 64 : (box == 1 ? 128 : 32);
-        CUtensorMap* mm = &maps[g * sm::kMapsPerGroup + 4 * box];
+        CUtensorMap* mm = &maps[g * sm::kMapsPerGroup + (box == 2 ? 10 : 4 * box)];
         for (int i = 0; i < 2; ++i) {
           void* xb = reinterpret_cast<__nv_bfloat16*>(h->X[i]) + gi.x_base;
           if ((rc = encode_map(h, &mm[i], xb, gi.cols, gi.rows, gi.ld, batch, br))) return bail(rc);
@@ -687,7 +704,7 @@ int signmuon_init(signmuon_t* out, const int64_t* shapes, int n_mats, int M, flo
       if (gi.cols % 64 == 0) {
         for (int i = 0; i < 2; ++i) {
           void* xb = reinterpret_cast<__nv_bfloat16*>(h->X[i]) + gi.x_base;
-          if ((rc = encode_map_atoms(h, &maps[g * sm::kMapsPerGroup + 12 + i], xb, gi.cols, gi.rows, gi.ld, batch, 64,
+          if ((rc = encode_map_atoms(h, &maps[g * sm::kMapsPerGroup + 8 + i], xb, gi.cols, gi.rows, gi.ld, batch, 64,
                                      2)))
             return bail(rc);
         }
@@ -759,15 +776,15 @@ static void local_part(signmuon_t h, const float* W, const sm::WorkerPtrs& gp, u
   }
 }
 
-// vote_part: the majority of Mv sign buffers at src + j*stride, then the
-// post-vote step (PolarNS with the handle's K, or with none for the
-// normalised sign step) and the update, or the vote fused with the update.
-static void vote_part(signmuon_t h, float* W, const uint8_t* src, int64_t stride, int Mv, float eta) {
+// vote_part: the majority of Mv sign buffers (worker j's at src.p[j], this
+// GPU's memory or a peer's), then the post-vote step (PolarNS with the
+// handle's K, or with none for the normalised sign step) and the update, or
+// the vote fused with the update.
+static void vote_part(signmuon_t h, float* W, const sm::WorkerPtrs& src, int Mv, float eta) {
   const Plan& p = h->plan;
   cudaStream_t s = h->stream;
   const int tie = (h->flags & SIGNMUON_TIE_PLUS) ? 1 : 0;
   const bool ternary = (h->flags & SIGNMUON_TERNARY) != 0;
-  const int8_t* src8 = reinterpret_cast<const int8_t*>(src);
   if (h->flags & (SIGNMUON_POST_POLAR | SIGNMUON_NORMALIZED_SIGN)) {
     const int k_post = (h->flags & SIGNMUON_NORMALIZED_SIGN) ? 0 : h->K;
     {
@@ -775,14 +792,15 @@ static void vote_part(signmuon_t h, float* W, const uint8_t* src, int64_t stride
       if (ternary) {
         // majority -> D, then D staged as the step's input (a one-worker
         // mean, which is D itself) with its sum-of-squares partials
-        sm::launch_vote_ternary_major(s, src8, stride, Mv, p.d, h->D, tie);
+        sm::launch_vote_ternary_major(s, src, Mv, p.d, h->D, tie);
         sm::launch_mean_stage(s, h->D, 0, 1, h->X[0], p.fp32 ? 0 : 1, h->d_chunks, (int)p.chunks.size(), h->d_mats,
                               h->d_groups, h->partials, nullptr);
       } else {
         // the majority goes straight into the step's input (and into D only
         // when K == 0, where the result is the scaled input itself)
-        sm::launch_vote_stage(s, src, stride, Mv, h->X[0], p.fp32 ? 0 : 1, h->d_chunks, (int)p.chunks.size(),
-                              h->d_mats, h->d_groups, h->partials, k_post == 0 ? h->D : nullptr, tie);
+        sm::launch_vote_stage(s, src, Mv, h->X[0], p.fp32 ? 0 : 1, h->d_chunks, (int)p.chunks.size(),
+                              h->d_mats, h->d_groups, h->partials, k_post == 0 ? h->D : nullptr, tie,
+                              stage_streamable(h) ? 1 : 0);
       }
     }
     fro_finalize(h, 1);
@@ -791,8 +809,8 @@ static void vote_part(signmuon_t h, float* W, const uint8_t* src, int64_t stride
     sm::launch_update(s, W, h->D, p.d, eta, h->status);
   } else {
     ProfScope ps(h, 7);
-    if (ternary) sm::launch_vote_ternary_update(s, src8, stride, Mv, p.d, W, eta, h->status, tie);
-    else sm::launch_vote_update(s, src, stride, Mv, p.d, W, eta, h->status, tie);
+    if (ternary) sm::launch_vote_ternary_update(s, src, Mv, p.d, W, eta, h->status, tie);
+    else sm::launch_vote_update(s, src, Mv, p.d, W, eta, h->status, tie);
   }
 }
 
@@ -841,7 +859,7 @@ int signmuon_step(signmuon_t h, float* W, const float* const* G, float eta) {
   uint8_t* own = ternary ? reinterpret_cast<uint8_t*>(h->sign8) : h->bits;
   const int64_t own_stride = ternary ? p.dpad : p.nb_pad;
   local_part(h, W, gp, own, own_stride);
-  vote_part(h, W, own, own_stride, h->M, eta);
+  vote_part(h, W, byte_ptrs(own, own_stride, h->M), h->M, eta);
   return finish(h, (h->flags & SIGNMUON_ASYNC) == 0);
 }
 
@@ -885,7 +903,29 @@ int signmuon_vote_step(signmuon_t h, float* W, const uint8_t* signs, int64_t str
   CK(h, begin_status(h));
   h->dir_valid = post;  // D is kept only by the post-vote steps
   h->dir_in_D = post;
-  vote_part(h, W, signs, stride, M, eta);
+  vote_part(h, W, byte_ptrs(signs, stride, M), M, eta);
+  return finish(h, (h->flags & SIGNMUON_ASYNC) == 0);
+}
+
+int signmuon_vote_step_ptrs(signmuon_t h, float* W, const uint8_t* const* signs, int M, float eta) {
+  NvtxRange range("signmuon_vote_step_ptrs");
+  const bool post = h != nullptr && (h->flags & (SIGNMUON_POST_POLAR | SIGNMUON_NORMALIZED_SIGN)) != 0;
+  DeviceGuard dev_guard(h);
+  int rc = check_handle(h, post);
+  if (rc) return rc;
+  if (h->flags & SIGNMUON_MUON_MEAN) return fail(h, SIGNMUON_E_UNSUPPORTED, "a SIGNMUON_MUON_MEAN handle takes no vote");
+  if (M < 1 || M > sm::kMaxWorkers) return fail(h, SIGNMUON_E_INVALID, "M must be in [1, 256]");
+  if (W == nullptr || signs == nullptr) return fail(h, SIGNMUON_E_INVALID, "null W or signs");
+  if (!aligned16(W)) return fail(h, SIGNMUON_E_INVALID, "W must be 16-byte aligned");
+  for (int m = 0; m < M; ++m)
+    if (signs[m] == nullptr || !aligned16(signs[m]))
+      return fail(h, SIGNMUON_E_INVALID, "signs[m] null or not 16-byte aligned");
+  CK(h, begin_status(h));
+  h->dir_valid = post;
+  h->dir_in_D = post;
+  sm::WorkerPtrs sp{};
+  for (int m = 0; m < M; ++m) sp.p[m] = reinterpret_cast<const float*>(signs[m]);
+  vote_part(h, W, sp, M, eta);
   return finish(h, (h->flags & SIGNMUON_ASYNC) == 0);
 }
 
@@ -951,6 +991,66 @@ int signmuon_step_host(signmuon_t h, float* W_host, const float* const* G_host, 
   if (rc) return rc;
   CK(h, cudaMemcpyAsync(W_host, h->hw_W, (size_t)p.d * 4, cudaMemcpyDeviceToHost, s));
   return signmuon_sync(h);
+}
+
+// ---- CUDA IPC: map a buffer of one process into another (peer GPUs) ------
+namespace {
+typedef CUresult (*AddrRangeFn)(CUdeviceptr*, size_t*, CUdeviceptr);
+AddrRangeFn get_addr_range() {
+  static AddrRangeFn fn = nullptr;
+  if (!fn) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<AddrRangeFn>(f);
+  }
+  return fn;
+}
+}  // namespace
+
+int signmuon_ipc_get_handle(const void* dev_ptr, void* handle, int64_t* offset) {
+  if (dev_ptr == nullptr || handle == nullptr || offset == nullptr)
+    return fail(nullptr, SIGNMUON_E_INVALID, "ipc_get_handle: null pointer");
+  AddrRangeFn range = get_addr_range();
+  if (!range) return fail(nullptr, SIGNMUON_E_CUDA, "cuMemGetAddressRange is not available from the driver");
+  CUdeviceptr base = 0;
+  size_t size = 0;
+  if (range(&base, &size, reinterpret_cast<CUdeviceptr>(dev_ptr)) != CUDA_SUCCESS)
+    return fail(nullptr, SIGNMUON_E_INVALID, "ipc_get_handle: not a device allocation");
+  cudaIpcMemHandle_t hd;
+  const cudaError_t e = cudaIpcGetMemHandle(&hd, reinterpret_cast<void*>(base));
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(nullptr, SIGNMUON_E_CUDA, std::string("cudaIpcGetMemHandle: ") + cudaGetErrorString(e));
+  }
+  static_assert(sizeof(cudaIpcMemHandle_t) == SIGNMUON_IPC_HANDLE_BYTES, "IPC handle size");
+  std::memcpy(handle, &hd, sizeof(hd));
+  *offset = (int64_t)(reinterpret_cast<uintptr_t>(dev_ptr) - (uintptr_t)base);
+  return SIGNMUON_OK;
+}
+
+int signmuon_ipc_open(const void* handle, void** base) {
+  if (handle == nullptr || base == nullptr) return fail(nullptr, SIGNMUON_E_INVALID, "ipc_open: null pointer");
+  cudaIpcMemHandle_t hd;
+  std::memcpy(&hd, handle, sizeof(hd));
+  *base = nullptr;
+  const cudaError_t e = cudaIpcOpenMemHandle(base, hd, cudaIpcMemLazyEnablePeerAccess);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(nullptr, SIGNMUON_E_CUDA, std::string("cudaIpcOpenMemHandle: ") + cudaGetErrorString(e));
+  }
+  return SIGNMUON_OK;
+}
+
+int signmuon_ipc_close(void* base) {
+  if (base == nullptr) return fail(nullptr, SIGNMUON_E_INVALID, "ipc_close: null pointer");
+  const cudaError_t e = cudaIpcCloseMemHandle(base);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(nullptr, SIGNMUON_E_CUDA, std::string("cudaIpcCloseMemHandle: ") + cudaGetErrorString(e));
+  }
+  return SIGNMUON_OK;
 }
 
 int signmuon_sync(signmuon_t h) {
@@ -1168,13 +1268,14 @@ int signmuon_get_direction(signmuon_t h, float* dst) {
   } else if (h->flags & SIGNMUON_TERNARY) {
     // the step fuses the vote into the update; recompute the majority from
     // the last step's ternary signs
-    sm::launch_vote_ternary_major(h->stream, h->sign8, p.dpad, h->M, p.d, dst,
-                                  (h->flags & SIGNMUON_TIE_PLUS) ? 1 : 0);
+    sm::launch_vote_ternary_major(h->stream, byte_ptrs(reinterpret_cast<const uint8_t*>(h->sign8), p.dpad, h->M),
+                                  h->M, p.d, dst, (h->flags & SIGNMUON_TIE_PLUS) ? 1 : 0);
     CK(h, cudaGetLastError());
   } else {
     // the step fuses the vote into the update; recompute the majority from
     // the last step's packed signs
-    sm::launch_vote_major(h->stream, h->bits, p.nb_pad, h->M, p.d, dst, (h->flags & SIGNMUON_TIE_PLUS) ? 1 : 0);
+    sm::launch_vote_major(h->stream, byte_ptrs(h->bits, p.nb_pad, h->M), h->M, p.d, dst,
+                          (h->flags & SIGNMUON_TIE_PLUS) ? 1 : 0);
     CK(h, cudaGetLastError());
   }
   return SIGNMUON_OK;

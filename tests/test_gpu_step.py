@@ -62,7 +62,7 @@ def _run_one_step(shapes, M, sigma, K, scale, P, precision, post_polar, seed, or
     gpu["scales"] = h.get_scales()
     want = ref.step(w0, G, mom0, shapes, beta=HP["beta"], lam=HP["lam"], eta=HP["eta"], K=K, eps=HP["eps"],
                     scale=scale, P=P, order=order, post_polar=post_polar, tie=tie)
-    want.update(mom0=mom0, G=G, w0=w0)
+    want.update(mom0=mom0, G=G, w0=w0, K=K, scale=scale, P=P, order=order)
     return h, gpu, want
 
 
@@ -105,6 +105,10 @@ def _compare_step(shapes, M, gpu, want, precision, post_polar, tie=0):
         compared = 0
         for r, c in shapes:
             sl = slice(off, off + r * c)
+            # every matrix: D is the PolarNS of the GPU's own majority
+            teacher = ref.polar_ns(gpu_maj[sl].reshape(r, c).astype(np.float64), want["K"], HP["eps"],
+                                   want["scale"], want["P"], want["order"]).ravel()
+            assert_polar_close(gpu["D"][sl], teacher, precision, f"post-polar D of the GPU majority {r}x{c}")
             if np.array_equal(gpu_maj[sl], want["majority"][sl]):
                 assert_polar_close(gpu["D"][sl], want["D"][sl], precision, f"post-polar D {r}x{c}")
                 tol = HP["eta"] * (2e-2 if precision == "bf16" else 1e-4) + 1e-6
@@ -128,6 +132,18 @@ def test_step_ragged_post_polar(precision, scale, P):
     M = 4  # even: ties occur and must map to zero
     h, gpu, want = _run_one_step(shapes, M, 1.0, 5, scale, P, precision, True, seed=3)
     _compare_step(shapes, M, gpu, want, precision, True)
+
+
+@pytest.mark.parametrize("M", [3, 4, 9])
+def test_step_post_polar_streamed_stage(M):
+    """Shapes whose matrices start at multiples of 128 entries and have a
+    multiple of 8 columns: the majority is staged into the post-vote input by
+    the streaming vote kernel, one warp per chunk.  Ragged chunks (512 and 64
+    entries, the last below one lane's 128), odd and even M, and a second
+    batch of workers (M = 9)."""
+    shapes = [(136, 64), (64, 200), (128, 128), (96, 136), (8, 8)]
+    h, gpu, want = _run_one_step(shapes, M, 1.0, 5, "spectral", 2, "bf16", True, seed=37)
+    _compare_step(shapes, M, gpu, want, "bf16", True)
 
 
 def test_step_quintic_fp32():
