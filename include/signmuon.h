@@ -173,6 +173,44 @@ int signmuon_vote_step(signmuon_t h, float* W, const uint8_t* signs, int64_t str
                        float eta);
 
 /* ------------------------------------------------------------------------
+ * signmuon_vote_step_ptrs -- signmuon_vote_step with worker j's signs at
+ * signs[j] instead of signs + j*stride: on a node of GPUs each rank maps the
+ * other ranks' sign buffers into its address space (signmuon_ipc_open) and
+ * the vote kernel reads their packed bits over NVLink directly, with no
+ * all-gather copy in between ([paper] Algorithm 2's one exchange of the
+ * signs; [blog] "One bit of information is not automatically a one-bit
+ * all-reduce").
+ *   signs  host array of M device pointers (this GPU's memory or a peer's
+ *          mapped by signmuon_ipc_open), each 16-byte aligned, each holding
+ *          one worker's ceil(d/8) packed bytes (d int8 signs with
+ *          SIGNMUON_TERNARY) padded to a multiple of 16; every buffer must
+ *          hold its signs when the call's kernels run (the caller orders the
+ *          writers and this call, e.g. by a collective in between).
+ *   M      1..256 workers, in worker order.
+ * Otherwise as signmuon_vote_step.  Errors: E_INVALID (null or misaligned),
+ * E_UNSUPPORTED (MUON_MEAN, or a vote-only handle with a post-vote step).
+ * ---------------------------------------------------------------------- */
+int signmuon_vote_step_ptrs(signmuon_t h, float* W, const uint8_t* const* signs, int M, float eta);
+
+/* ------------------------------------------------------------------------
+ * CUDA IPC for the exchange between GPUs (no counterpart on the pages: the
+ * plumbing that lets signmuon_vote_step_ptrs read a peer's sign buffer).
+ * signmuon_ipc_get_handle: the IPC handle (SIGNMUON_IPC_HANDLE_BYTES bytes,
+ *   written to `handle`) of the device allocation that contains dev_ptr, and
+ *   dev_ptr's byte offset in it (to *offset); send both to the peer.
+ * signmuon_ipc_open: map a peer's allocation (handle from another process)
+ *   into this process on the current device; *base receives its address here
+ *   (add the offset).  Peer access is enabled as needed.
+ * signmuon_ipc_close: unmap a base pointer returned by signmuon_ipc_open.
+ * Errors: E_INVALID (null pointers, not a device allocation), E_CUDA (the
+ * runtime refused: see signmuon_last_error(NULL)).
+ * ---------------------------------------------------------------------- */
+#define SIGNMUON_IPC_HANDLE_BYTES 64
+int signmuon_ipc_get_handle(const void* dev_ptr, void* handle, int64_t* offset);
+int signmuon_ipc_open(const void* handle, void** base);
+int signmuon_ipc_close(void* base);
+
+/* ------------------------------------------------------------------------
  * signmuon_sums_step -- the second half of the step when the vote sums arrive
  * already added up: [paper] Algorithm 2's integer SUM all-reduce of the
  * workers' signs (each GPU sums its own workers with signmuon_vote or

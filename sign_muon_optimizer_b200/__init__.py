@@ -52,7 +52,8 @@ EXPORTED = [
     "signmuon_profile", "signmuon_profile_read", "signmuon_get_gram",
     "signmuon_spectral_norm_noalloc", "signmuon_sign_ternary", "signmuon_vote_ternary",
     "signmuon_get_ternary_signs", "signmuon_local_signs", "signmuon_vote_step", "signmuon_sums_step",
-    "signmuon_plan_tables", "signmuon_get_pi_state", "signmuon_set_pi_state",
+    "signmuon_plan_tables", "signmuon_get_pi_state", "signmuon_set_pi_state", "signmuon_vote_step_ptrs",
+    "signmuon_ipc_get_handle", "signmuon_ipc_open", "signmuon_ipc_close",
 ]
 PROF_KINDS = ["momentum", "norm_finalize", "ns_gram", "ns_square", "ns_apply", "power_iter", "pack",
               "vote", "stage", "post_gram", "post_square", "post_apply", "update", "k0_scale"]
@@ -83,6 +84,10 @@ def _load():
         "signmuon_set_pi_state": (I, [P, I, P]),
         "signmuon_local_signs": (I, [P, P, PP, P, I64]),
         "signmuon_vote_step": (I, [P, P, P, I64, I, F]),
+        "signmuon_vote_step_ptrs": (I, [P, P, PP, I, F]),
+        "signmuon_ipc_get_handle": (I, [P, P, ctypes.POINTER(I64)]),
+        "signmuon_ipc_open": (I, [P, ctypes.POINTER(P)]),
+        "signmuon_ipc_close": (I, [P]),
         "signmuon_sums_step": (I, [P, P, P, F]),
         "signmuon_plan_tables": (I, [ctypes.POINTER(I64), I, I, I, I, I, U, ctypes.c_char_p, I64,
                                      ctypes.POINTER(I64)]),
@@ -206,6 +211,36 @@ def signmuon_local_signs(h, W, G, signs, stride):
 
 def signmuon_vote_step(h, W, signs, stride, M, eta):
     _check(h, _lib.signmuon_vote_step(h, _ptr(W), _ptr(signs), int(stride), int(M), float(eta)))
+
+
+def signmuon_vote_step_ptrs(h, W, signs, eta):
+    """signs: one device pointer (int or tensor) per worker, in worker order."""
+    _check(h, _lib.signmuon_vote_step_ptrs(h, _ptr(W), _ptr_array(signs), len(signs), float(eta)))
+
+
+SIGNMUON_IPC_HANDLE_BYTES = 64
+
+
+def signmuon_ipc_get_handle(dev_ptr):
+    """(handle bytes, byte offset of dev_ptr in its allocation)."""
+    buf = ctypes.create_string_buffer(SIGNMUON_IPC_HANDLE_BYTES)
+    off = ctypes.c_int64()
+    _check(None, _lib.signmuon_ipc_get_handle(_ptr(dev_ptr), buf, ctypes.byref(off)))
+    return buf.raw, int(off.value)
+
+
+def signmuon_ipc_open(handle):
+    """Base address, in this process, of a peer's allocation."""
+    if len(handle) != SIGNMUON_IPC_HANDLE_BYTES:
+        raise ValueError("an IPC handle has 64 bytes")
+    base = ctypes.c_void_p()
+    _check(None, _lib.signmuon_ipc_open(ctypes.create_string_buffer(bytes(handle), SIGNMUON_IPC_HANDLE_BYTES),
+                                        ctypes.byref(base)))
+    return int(base.value)
+
+
+def signmuon_ipc_close(base):
+    _check(None, _lib.signmuon_ipc_close(_ptr(base)))
 
 
 def signmuon_sums_step(h, W, sums, eta):
@@ -387,6 +422,9 @@ class SignMuon:
 
     def vote_step(self, W, signs, M, eta, stride=None):
         signmuon_vote_step(self.h, W, signs, self.sign_stride() if stride is None else stride, M, eta)
+
+    def vote_step_ptrs(self, W, signs, eta):
+        signmuon_vote_step_ptrs(self.h, W, signs, eta)
 
     def sums_step(self, W, sums, eta):
         signmuon_sums_step(self.h, W, sums, eta)

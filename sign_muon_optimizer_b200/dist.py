@@ -7,13 +7,20 @@ every worker takes the majority and updates its own copy of W.  [blog]
 the payload: ceil(d/8) bytes per worker for the packed bits, gathered from all
 ranks (an all-gather; every rank then votes locally).
 
-Two exchanges are offered:
+Three exchanges are offered:
 - "allgather": every rank gathers all workers' packed (or int8 ternary) signs
   and votes over them.  The payload is M_local * ceil(d/8) bytes per rank.
 - "allreduce": each rank adds up its own workers' signs, and an integer SUM
   all-reduce adds the ranks' sums (Algorithm 2's form).  The payload is d
   bytes per rank with int8 sums (SIGNMUON_ACC_INT8, at most 127 workers in
   all), or 4d with int32 sums.
+- "peer": no data collective at all.  Each rank's sign buffers are mapped
+  into every other rank once (CUDA IPC); every step the vote kernel reads
+  all ranks' packed bits directly, over NVLink for the peers' (loads only, no
+  multicast).  The buffers alternate between two slots from step to step, so
+  that the status all-reduce of a step, which every rank enters only after
+  its previous vote finished, is the only synchronisation needed: a rank
+  writes slot t % 2 at step t while its peers may still read slot (t-1) % 2.
 
 This module is plumbing only.  The arithmetic runs in libsignmuon.so:
 signmuon_local_signs before the exchange; after it, signmuon_vote_step, or
@@ -32,7 +39,8 @@ import numpy as np
 import torch
 import torch.distributed as dist
 
-from . import SIGNMUON_ACC_INT8, SIGNMUON_ASYNC, SIGNMUON_E_NONFINITE, SIGNMUON_TERNARY, SignMuon, SignMuonError
+from . import (SIGNMUON_ACC_INT8, SIGNMUON_ASYNC, SIGNMUON_E_NONFINITE, SIGNMUON_TERNARY, SignMuon, SignMuonError,
+               signmuon_ipc_close, signmuon_ipc_get_handle, signmuon_ipc_open)
 
 
 class DistSignMuon:
@@ -43,16 +51,18 @@ class DistSignMuon:
     worker order is rank-major: rank r holds workers r*M_local ...
     (r+1)*M_local - 1.  ``exchange`` is "allgather" or "allreduce" (see the
     module text).  ``opt`` may be given to reuse an existing handle, or any
-    object with the same methods (local_signs, vote_step, vote, vote_ternary,
-    sums_step, sign_stride, and sync for a handle made with SIGNMUON_ASYNC)
-    and attributes (d, flags).  With SIGNMUON_ASYNC every step waits for the
+    object with the same methods (local_signs, vote_step, vote_step_ptrs,
+    vote, vote_ternary, sums_step, sign_stride, and sync for a handle made
+    with SIGNMUON_ASYNC) and attributes (d, flags).  ``ipc`` replaces the CUDA
+    IPC mapping of the "peer" exchange (an object with alloc, handle,
+    address, open and close).  With SIGNMUON_ASYNC every step waits for the
     local half's status before the exchange, so that a failed rank stops all
     ranks as it does without the flag.
     """
 
     def __init__(self, shapes, M_local=1, beta=0.9, lam=0.01, K=5, eps=1e-7, scale="fro", P=1, flags=0,
-                 group=None, device=None, opt=None, exchange="allgather"):
-        if exchange not in ("allgather", "allreduce"):
+                 group=None, device=None, opt=None, exchange="allgather", ipc=None):
+        if exchange not in ("allgather", "allreduce", "peer"):
             raise ValueError(f"unknown exchange {exchange!r}")
         self.exchange = exchange
         self.group = group
@@ -85,6 +95,20 @@ class DistSignMuon:
         self.async_status = bool(flags & SIGNMUON_ASYNC)
         if exchange == "allgather":
             self.gathered = torch.zeros(self.M * self.stride, dtype=torch.uint8, device=self.device)
+        elif exchange == "peer":
+            self.ipc = ipc if ipc is not None else _CudaIpc()
+            self.slots = [self.ipc.alloc(self.M_local * self.stride, self.device) for _ in range(2)]
+            mine = [self.ipc.handle(b) for b in self.slots]
+            everyone = [None] * self.world
+            dist.all_gather_object(everyone, mine, group=self.group)
+            # slot_ptr[r][k]: the address, in this process, of rank r's slot k
+            self.slot_ptr = []
+            for r in range(self.world):
+                if r == self.rank:
+                    self.slot_ptr.append([self.ipc.address(b) for b in self.slots])
+                else:
+                    self.slot_ptr.append([self.ipc.open(hd) for hd in everyone[r]])
+            self.t = 0
         else:
             acc8 = bool(flags & SIGNMUON_ACC_INT8)
             if acc8 and self.M > 127:
@@ -94,10 +118,20 @@ class DistSignMuon:
 
     @property
     def payload_bytes(self):
-        """Bytes each rank contributes to the exchange per step."""
-        if self.exchange == "allgather":
+        """Bytes each rank contributes to the exchange per step (for "peer",
+        the bytes of its signs that every other rank reads)."""
+        if self.exchange in ("allgather", "peer"):
             return self.local.numel()
         return self.sums.numel() * self.sums.element_size()
+
+    def close(self):
+        """Unmap the peers' sign buffers ("peer" exchange)."""
+        if self.exchange == "peer":
+            for r, ptrs in enumerate(self.slot_ptr):
+                if r != self.rank:
+                    for p in ptrs:
+                        self.ipc.close(p)
+            self.slot_ptr = []
 
     def step(self, W, G, eta, clocks=None):
         """One step.  With a ``clocks`` dict, adds this step's phase times in
@@ -115,8 +149,14 @@ class DistSignMuon:
         clk = _PhaseClock(self.device) if clocks is not None else None
         t0 = clk.mark() if clk else None
         err = None
+        if self.exchange == "peer":
+            slot = self.t % 2
+            self.t += 1
+            own = self.slots[slot]
+        else:
+            own = self.local
         try:
-            self.opt.local_signs(W, G, self.local, self.stride)
+            self.opt.local_signs(W, G, own, self.stride)
             if self.async_status:
                 # raises the deferred error of this call (or of an earlier
                 # asynchronous call on the handle) before the flag is set
@@ -136,6 +176,12 @@ class DistSignMuon:
             dist.all_gather_into_tensor(self.gathered, self.local, group=self.group)
             t2 = clk.mark() if clk else None
             self.opt.vote_step(W, self.gathered, self.M, eta, self.stride)
+        elif self.exchange == "peer":
+            # every rank's signs of this step are complete (the all-reduce
+            # above); the vote reads them where they are, rank-major
+            t1 = t2 = clk.mark() if clk else None
+            ptrs = [self.slot_ptr[r][slot] + m * self.stride for r in range(self.world) for m in range(self.M_local)]
+            self.opt.vote_step_ptrs(W, ptrs, eta)
         else:
             d = int(self.opt.d)
             if self.ternary:
@@ -163,6 +209,32 @@ class DistSignMuon:
         dist.all_reduce(lo, op=dist.ReduceOp.MIN, group=self.group)
         dist.all_reduce(hi, op=dist.ReduceOp.MAX, group=self.group)
         return bool(torch.equal(lo, hi))
+
+
+class _CudaIpc:
+    """The sign buffers of the "peer" exchange: device allocations whose CUDA
+    IPC handles the other ranks open (libsignmuon's signmuon_ipc_* calls)."""
+
+    def alloc(self, nbytes, device):
+        return torch.zeros(nbytes, dtype=torch.uint8, device=device)
+
+    def handle(self, buf):
+        return signmuon_ipc_get_handle(buf.data_ptr())
+
+    def address(self, buf):
+        return buf.data_ptr()
+
+    def open(self, hd):
+        handle, offset = hd
+        base = signmuon_ipc_open(handle)
+        self._bases = getattr(self, "_bases", {})
+        self._bases[base + offset] = base
+        return base + offset
+
+    def close(self, ptr):
+        base = self._bases.pop(ptr, None)
+        if base is not None:
+            signmuon_ipc_close(base)
 
 
 class _PhaseClock:

@@ -130,10 +130,17 @@ calls = {{
     "signmuon_get_direction": (None, None), "signmuon_get_scales": (None, None),
     "signmuon_set_ns_coeffs": (None, None, 2), "signmuon_sync": (None,), "signmuon_info": (None, None, 6),
     "signmuon_profile": (None, 1), "signmuon_profile_read": (None, None, None, 1),
-    "signmuon_get_gram": (None, 0, 0, None),
+    "signmuon_get_gram": (None, 0, 0, None), "signmuon_vote_step_ptrs": (None, None, pp, 2, 0.1),
 }}
 bad = []
 for name, args in calls.items():
+    rc = getattr(L, name)(*args)
+    if rc != smo.SIGNMUON_E_INVALID or not L.signmuon_last_error(None):
+        bad.append((name, rc))
+# the handle-free IPC calls reject null pointers the same way
+off = ctypes.c_int64()
+for name, args in {{"signmuon_ipc_get_handle": (None, None, ctypes.byref(off)), "signmuon_ipc_open": (None, None),
+                    "signmuon_ipc_close": (None,)}}.items():
     rc = getattr(L, name)(*args)
     if rc != smo.SIGNMUON_E_INVALID or not L.signmuon_last_error(None):
         bad.append((name, rc))
@@ -154,5 +161,6 @@ def test_every_entry_point_rejects_a_null_handle():
     import sign_muon_optimizer_b200 as smo
     declared = [n for n in smo.EXPORTED if n not in (
         "signmuon_init", "signmuon_plan", "signmuon_plan_tables", "signmuon_kernel_launches",
-        "signmuon_last_error", "signmuon_status_string", "signmuon_destroy", "signmuon_spectral_norm_noalloc")]
+        "signmuon_last_error", "signmuon_status_string", "signmuon_destroy", "signmuon_spectral_norm_noalloc",
+        "signmuon_ipc_get_handle", "signmuon_ipc_open", "signmuon_ipc_close")]
     assert int(res.stdout.split()[1]) == len(declared)   # every handle-taking call is covered

@@ -60,6 +60,14 @@ class _StandIn:
         maj = ref.majority(ref.vote_sums_from_bits(packed, self.d))
         W.copy_(torch.from_numpy(ref.update(W.numpy(), maj.astype(np.float32), eta)))
 
+    def vote_step_ptrs(self, W, ptrs, eta):
+        # the stand-in's "device pointers" are host addresses (file mappings)
+        import ctypes
+        packed = [np.frombuffer(ctypes.string_at(p, self.nb), dtype=np.uint8) for p in ptrs]
+        self.seen = torch.from_numpy(np.concatenate(packed))
+        maj = ref.majority(ref.vote_sums_from_bits(packed, self.d))
+        W.copy_(torch.from_numpy(ref.update(W.numpy(), maj.astype(np.float32), eta)))
+
     def vote(self, views, d, sums, majority):
         sums.copy_(torch.from_numpy(ref.vote_sums_from_bits([v[: self.nb].numpy() for v in views], d)))
 
@@ -69,13 +77,45 @@ class _StandIn:
         W.copy_(torch.from_numpy(ref.update(W.numpy(), maj.astype(np.float32), eta)))
 
 
+class _FileIpc:
+    """Stand-in for the CUDA IPC mapping of the "peer" exchange: each rank's
+    buffers are shared files, mapped by every rank; a handle is the file name."""
+
+    def __init__(self, root, rank):
+        self.root, self.rank, self.n, self.keep = root, rank, 0, []
+
+    def alloc(self, nbytes, device):
+        path = os.path.join(self.root, f"rank{self.rank}_buf{self.n}")
+        self.n += 1
+        mm = np.memmap(path, dtype=np.uint8, mode="w+", shape=(nbytes,))
+        self.keep.append(mm)
+        t = torch.from_numpy(mm)
+        t.path = path
+        return t
+
+    def handle(self, buf):
+        return (buf.path, int(buf.numel()))
+
+    def address(self, buf):
+        return buf.data_ptr()
+
+    def open(self, hd):
+        path, n = hd
+        mm = np.memmap(path, dtype=np.uint8, mode="r", shape=(n,))
+        self.keep.append(mm)
+        return mm.ctypes.data
+
+    def close(self, ptr):
+        pass
+
+
 def _free_port():
     with socket.socket() as s:
         s.bind(("127.0.0.1", 0))
         return s.getsockname()[1]
 
 
-def _rank(rank, world, port, fail_rank, q, exchange="allgather", deferred=False):
+def _rank(rank, world, port, fail_rank, q, exchange="allgather", deferred=False, root=None, steps=1):
     import torch.distributed as dist
 
     from sign_muon_optimizer_b200.dist import DistSignMuon
@@ -84,16 +124,19 @@ def _rank(rank, world, port, fail_rank, q, exchange="allgather", deferred=False)
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
     try:
         opt = _StandIn(fail=(rank == fail_rank), deferred=deferred)
-        drv = DistSignMuon(SHAPES, M_local=M_LOCAL, opt=opt, device="cpu", exchange=exchange)
+        ipc = _FileIpc(root, rank) if exchange == "peer" else None
+        drv = DistSignMuon(SHAPES, M_local=M_LOCAL, opt=opt, device="cpu", exchange=exchange, ipc=ipc)
         W = torch.from_numpy(synth.weights0(SHAPES, 5))
-        G = synth.gradients(SHAPES, world * M_LOCAL, 1.0, step=1, config_id=5)
-        mine = [torch.from_numpy(g) for g in G[rank * M_LOCAL:(rank + 1) * M_LOCAL]]
         raised = False
         clocks = {}
-        try:
-            drv.step(W, mine, 0.02, clocks=clocks)
-        except Exception as e:  # noqa: BLE001
-            raised = type(e).__name__
+        for step in range(1, steps + 1):
+            G = synth.gradients(SHAPES, world * M_LOCAL, 1.0, step=step, config_id=5)
+            mine = [torch.from_numpy(g) for g in G[rank * M_LOCAL:(rank + 1) * M_LOCAL]]
+            try:
+                drv.step(W, mine, 0.02, clocks=clocks)
+            except Exception as e:  # noqa: BLE001
+                raised = type(e).__name__
+                break
         agree = drv.replicas_agree(W)
         q.put((rank, W.numpy().copy(), None if opt.seen is None else opt.seen.numpy(), raised, agree,
                drv.payload_bytes, clocks))
@@ -101,12 +144,13 @@ def _rank(rank, world, port, fail_rank, q, exchange="allgather", deferred=False)
         dist.destroy_process_group()
 
 
-def _run(fail_rank, exchange="allgather", deferred=False):
+def _run(fail_rank, exchange="allgather", deferred=False, root=None, steps=1):
     world = 2
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_rank, args=(r, world, port, fail_rank, q, exchange, deferred)) for r in range(world)]
+    procs = [ctx.Process(target=_rank, args=(r, world, port, fail_rank, q, exchange, deferred, root, steps))
+             for r in range(world)]
     for p in procs:
         p.start()
     out = {}
@@ -161,12 +205,37 @@ def test_allreduce_exchange_adds_the_ranks_sums():
         assert np.array_equal(out[r]["W"].view(np.uint32), want.view(np.uint32))
 
 
+def test_peer_exchange_votes_on_every_ranks_mapped_signs(tmp_path):
+    """The "peer" exchange: no data collective, each rank's sign buffers are
+    mapped by the other rank (here files stand in for CUDA IPC), the vote
+    reads all four workers' signs in rank-major order, and the two buffer
+    slots alternate: three steps must give both ranks the W of the oracle's
+    three sequential votes."""
+    out = _run(fail_rank=-1, exchange="peer", root=str(tmp_path), steps=3)
+    M = 2 * M_LOCAL
+    d = synth.numel(SHAPES)
+    nb = ref.packed_nbytes(d)
+    w = synth.weights0(SHAPES, 5)
+    for step in (1, 2, 3):
+        G = synth.gradients(SHAPES, M, 1.0, step=step, config_id=5)
+        packed = [ref.pack_bits(ref.sign_bits(g)) for g in G]
+        w = ref.update(w, ref.majority(ref.vote_sums_from_bits(packed, d)).astype(np.float32), 0.02)
+    stride = (nb + 15) // 16 * 16
+    for r in range(2):
+        assert out[r]["raised"] is False and out[r]["agree"] is True
+        assert out[r]["payload"] == M_LOCAL * stride
+        assert np.array_equal(out[r]["W"].view(np.uint32), w.view(np.uint32))
+        # the last vote saw worker j's signs at slot j (rank-major)
+        for j in range(M):
+            assert np.array_equal(out[r]["seen"][j * nb:(j + 1) * nb], packed[j])
+
+
 @pytest.mark.parametrize("deferred", [False, True])
-@pytest.mark.parametrize("exchange", ["allgather", "allreduce"])
-def test_one_failing_rank_stops_every_rank_without_update(exchange, deferred):
+@pytest.mark.parametrize("exchange", ["allgather", "allreduce", "peer"])
+def test_one_failing_rank_stops_every_rank_without_update(exchange, deferred, tmp_path):
     # deferred: the failing rank's handle is asynchronous, so its local half
     # returns OK and only its sync() reports the failure
-    out = _run(fail_rank=1, exchange=exchange, deferred=deferred)
+    out = _run(fail_rank=1, exchange=exchange, deferred=deferred, root=str(tmp_path))
     w0 = synth.weights0(SHAPES, 5)
     for r in range(2):
         assert out[r]["raised"] == "SignMuonError"

@@ -197,3 +197,111 @@ def test_two_ranks_adding_their_sums_equal_one_handle(acc8):
         for r in range(ranks):
             parts[r].sums_step(Wr[r], total, HP["eta"])
             assert np.array_equal(_bits(Wr[r]), _bits(W)), f"rank {r}, step {step}"
+
+
+@pytest.mark.parametrize("case", sorted(CASES))
+def test_vote_step_ptrs_equals_the_step(case):
+    """signmuon_vote_step_ptrs: every worker's signs in a buffer of its own,
+    reached through a list of pointers (as the peers' mapped buffers are on a
+    node of GPUs), two ranks' handles emulated one after the other: W of both
+    ranks equals one four-worker handle's, bit for bit, for two steps."""
+    shapes, flags = CASES[case]
+    M, ranks, per = 4, 2, 2
+    w0 = synth.weights0(shapes, 101)
+    single = _opt(shapes, M, flags)
+    parts = [_opt(shapes, per, flags) for _ in range(ranks)]
+    stride = single.sign_stride()
+    W, Wr = dev(w0), [dev(w0) for _ in range(ranks)]
+    # separate allocations, one per rank, with 16 bytes in front so that no
+    # buffer starts where an allocation starts
+    raw = [torch.zeros(per * stride + 16, dtype=torch.uint8, device="cuda") for _ in range(ranks)]
+    local = [b[16:] for b in raw]
+    ptrs = [local[r].data_ptr() + m * stride for r in range(ranks) for m in range(per)]
+    for step in (1, 2):
+        G = [dev(g) for g in synth.gradients(shapes, M, 1.0, step=step, config_id=101)]
+        single.step(W, G, HP["eta"])
+        for r in range(ranks):
+            parts[r].local_signs(Wr[r], G[r * per:(r + 1) * per], local[r])
+        for r in range(ranks):
+            parts[r].vote_step_ptrs(Wr[r], ptrs, HP["eta"])
+            assert np.array_equal(_bits(Wr[r]), _bits(W)), f"rank {r}, step {step}"
+    if flags & (smo.SIGNMUON_POST_POLAR | smo.SIGNMUON_NORMALIZED_SIGN):
+        a, b = torch.zeros(single.d, device="cuda"), torch.zeros(single.d, device="cuda")
+        single.get_direction(a)
+        parts[1].get_direction(b)
+        assert np.array_equal(_bits(a), _bits(b))
+
+
+def test_vote_step_ptrs_argument_checks():
+    shapes = FUSED
+    opt = _opt(shapes, 2, 0)
+    W = torch.zeros(opt.d, device="cuda")
+    buf = torch.zeros(2 * opt.sign_stride() + 64, dtype=torch.uint8, device="cuda")
+    good = [buf.data_ptr(), buf.data_ptr() + opt.sign_stride()]
+    for ptrs in ([], [buf.data_ptr(), buf.data_ptr() + 8], [buf.data_ptr(), 0], [buf.data_ptr()] * 257):
+        with pytest.raises(smo.SignMuonError) as ei:
+            opt.vote_step_ptrs(W, ptrs, 0.1)
+        assert ei.value.status == smo.SIGNMUON_E_INVALID
+    muon = _opt(shapes, 2, smo.SIGNMUON_MUON_MEAN)
+    with pytest.raises(smo.SignMuonError) as ei:
+        muon.vote_step_ptrs(W, good, 0.1)
+    assert ei.value.status == smo.SIGNMUON_E_UNSUPPORTED
+
+
+def _peer_rank(rank, world, port, shapes, flags, q):
+    """One rank of the "peer" exchange on the one GPU of this run: its sign
+    buffers are mapped into the other process by CUDA IPC and the vote kernel
+    reads them there (on a node, over NVLink).  No kernel waits for another
+    rank: the ranks meet only in the host-side status all-reduce."""
+    import datetime
+    import os
+
+    import torch.distributed as dist
+
+    import sign_muon_optimizer_b200 as smo_r
+    from sign_muon_optimizer_b200.dist import DistSignMuon
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    torch.cuda.set_device(0)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        per = 2
+        opt = smo_r.SignMuon(shapes, per, beta=HP["beta"], lam=HP["lam"], K=5, eps=HP["eps"], scale="spectral", P=2,
+                             flags=flags)
+        drv = DistSignMuon(shapes, M_local=per, opt=opt, device="cuda", exchange="peer")
+        W = torch.from_numpy(synth.weights0(shapes, 103)).cuda()
+        for step in (1, 2, 3):
+            G = synth.gradients(shapes, world * per, 1.0, step=step, config_id=103)
+            drv.step(W, [torch.from_numpy(g).cuda() for g in G[rank * per:(rank + 1) * per]], HP["eta"])
+        torch.cuda.synchronize()
+        q.put((rank, W.cpu().numpy().copy(), drv.replicas_agree(W)))
+        drv.close()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("case", ["bf16_fused", "post_polar"])
+def test_peer_exchange_through_cuda_ipc_equals_one_handle(case):
+    import socket
+
+    import torch.multiprocessing as mp
+    shapes, flags = CASES[case]
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_peer_rank, args=(r, 2, port, shapes, flags, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    got = dict((r, (w, agree)) for r, w, agree in (q.get(timeout=300) for _ in range(2)))
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    single = _opt(shapes, 4, flags)
+    W = dev(synth.weights0(shapes, 103))
+    for step in (1, 2, 3):
+        single.step(W, [dev(g) for g in synth.gradients(shapes, 4, 1.0, step=step, config_id=103)], HP["eta"])
+    for r in range(2):
+        assert got[r][1] is True
+        assert np.array_equal(got[r][0].view(np.uint32), _bits(W)), f"rank {r}"
