@@ -246,34 +246,22 @@ k_pi_matvec(const ProbRows* __restrict__ rows, const void* __restrict__ A,
   if (BF16) {
     const __nv_bfloat16* a0 = reinterpret_cast<const __nv_bfloat16*>(A) + prob_a_off[p] + (int64_t)r0 * gld;
     const int g8 = g & ~7;
-    // R rows x 4 column blocks of 256: all their 16-byte loads are in flight
-    // before the first FMA (one round trip per 1024 columns, not per 256)
-    for (int k0 = 0; k0 < g8; k0 += 4 * 256) {
-      uint4 raw[R][4];
+    for (int k = lane * 8; k < g8; k += 256) {
+      uint4 raw[R];
 #pragma unroll
       for (int j = 0; j < R; ++j)
+        raw[j] = (r0 + j < g) ? __ldcs(reinterpret_cast<const uint4*>(a0 + (int64_t)j * gld + k)) : make_uint4(0, 0, 0, 0);
+      const float4 u0 = *reinterpret_cast<const float4*>(us + k);
+      const float4 u1 = *reinterpret_cast<const float4*>(us + k + 4);
+      const float uv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int k = k0 + c * 256 + lane * 8;
-          raw[j][c] = (r0 + j < g && k < g8) ? __ldcs(reinterpret_cast<const uint4*>(a0 + (int64_t)j * gld + k))
-                                             : make_uint4(0, 0, 0, 0);
-        }
+      for (int j = 0; j < R; ++j) {
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw[j]);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int k = k0 + c * 256 + lane * 8;
-        if (k >= g8) break;
-        const float4 u0 = *reinterpret_cast<const float4*>(us + k);
-        const float4 u1 = *reinterpret_cast<const float4*>(us + k + 4);
-        const float uv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-#pragma unroll
-        for (int j = 0; j < R; ++j) {
-          const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw[j][c]);
-#pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            const float2 f = __bfloat1622float2(h[t]);
-            acc[j] = fmaf(f.x, uv[2 * t], acc[j]);
-            acc[j] = fmaf(f.y, uv[2 * t + 1], acc[j]);
-          }
+        for (int t = 0; t < 4; ++t) {
+          const float2 f = __bfloat1622float2(h[t]);
+          acc[j] = fmaf(f.x, uv[2 * t], acc[j]);
+          acc[j] = fmaf(f.y, uv[2 * t + 1], acc[j]);
         }
       }
     }
@@ -545,6 +533,25 @@ k_vote(WorkerPtrs signs, int M, int64_t d,
   }
 }
 
+// Byte-lane helpers of the vote's output: x holds four counts c (one per byte,
+// c <= M <= 255).
+// 2c - M per byte, modulo 256 (an exact int8 when M <= 127): 2c <= 254 has no
+// carry out of its byte, and the subtraction borrows nothing across bytes.
+__device__ __forceinline__ uint32_t swar_twice_minus(uint32_t x, int M) {
+  const uint32_t a = x << 1, b = (uint32_t)M * 0x01010101u, H = 0x80808080u;
+  return ((a | H) - (b & ~H)) ^ ((a ^ ~b) & H);
+}
+// sign(2c - M) per byte as int8 (+1 = 0x01, -1 = 0xFF, a tie 0x00, or 0x01
+// with tie_plus): c > M/2 <=> c + 127 - floor(M/2) has bit 7 set, and c < M/2
+// <=> c + 128 - ceil(M/2) has not (neither sum leaves its byte for M <= 255).
+__device__ __forceinline__ uint32_t swar_majority(uint32_t x, int M, int tie_plus) {
+  const uint32_t H = 0x80808080u;
+  const uint32_t gt = (x + (uint32_t)(127 - M / 2) * 0x01010101u) & H;
+  const uint32_t lt = ~(x + (uint32_t)(128 - (M + 1) / 2) * 0x01010101u) & H;
+  if (tie_plus) return ((lt >> 7) * 0xFEu) + 0x01010101u;
+  return (gt >> 7) | ((lt >> 7) * 0xFFu);
+}
+
 // Streaming vote for M <= 255 (byte-lane counters): each warp takes tiles of 4096 consecutive entries (512 bytes of
 // every worker's stream).  The bytes come into shared memory by cp.async, 16
 // per lane (each load instruction reads 512 contiguous bytes of one stream),
@@ -714,19 +721,23 @@ k_vote_stream(WorkerPtrs signs, int M, int64_t ntiles,
       int nz = 0;
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
-        const int c0 = acc[j] & 0xFF, c1 = (acc[j] >> 8) & 0xFF, c2 = (acc[j] >> 16) & 0xFF, c3 = acc[j] >> 24;
         const int e = j * 128 + lane * 4;
         if (e < ch.len) {
-          const int v0 = vmaj(2 * c0 - M, tie_plus), v1 = vmaj(2 * c1 - M, tie_plus);
-          const int v2 = vmaj(2 * c2 - M, tie_plus), v3 = vmaj(2 * c3 - M, tie_plus);
-          nz += (v0 != 0) + (v1 != 0) + (v2 != 0) + (v3 != 0);
-          const __nv_bfloat162 lo = __floats2bfloat162_rn((float)v0, (float)v1);
-          const __nv_bfloat162 hi = __floats2bfloat162_rn((float)v2, (float)v3);
+          // the four majorities as int8 byte lanes (0x01, 0xFF or 0), then as
+          // bf16 pairs: +1 = 0x3F80, -1 = 0xBF80, 0 = 0 (sign at bit 15 of a half)
+          const uint32_t mj = swar_majority(acc[j], M, tie_plus);
+          const uint32_t nzb = (mj | (mj << 7)) & 0x80808080u;    // bit 7 of a non-zero byte
+          const uint32_t sgn = mj & 0x80808080u;                  // bit 7 of a -1 byte
+          nz += __popc(nzb);
           uint2 u;
-          u.x = *reinterpret_cast<const uint32_t*>(&lo);
-          u.y = *reinterpret_cast<const uint32_t*>(&hi);
+          u.x = ((__byte_perm(nzb, 0, 0x1404) >> 15) * 0xFFFFu & 0x3F803F80u) | __byte_perm(sgn, 0, 0x1404);
+          u.y = ((__byte_perm(nzb, 0, 0x3424) >> 15) * 0xFFFFu & 0x3F803F80u) | __byte_perm(sgn, 0, 0x3424);
           *reinterpret_cast<uint2*>(xo + e) = u;
-          if (D != nullptr) st4(D + fb + e, make_float4((float)v0, (float)v1, (float)v2, (float)v3));
+          if (D != nullptr) {
+            const int c0 = acc[j] & 0xFF, c1 = (acc[j] >> 8) & 0xFF, c2 = (acc[j] >> 16) & 0xFF, c3 = acc[j] >> 24;
+            st4(D + fb + e, make_float4((float)vmaj(2 * c0 - M, tie_plus), (float)vmaj(2 * c1 - M, tie_plus),
+                                        (float)vmaj(2 * c2 - M, tie_plus), (float)vmaj(2 * c3 - M, tie_plus)));
+          }
         }
       }
       nz = __reduce_add_sync(0xffffffffu, nz);
@@ -739,17 +750,21 @@ k_vote_stream(WorkerPtrs signs, int M, int64_t ntiles,
         const int s0 = 2 * c0 - M, s1 = 2 * c1 - M, s2 = 2 * c2 - M, s3 = 2 * c3 - M;
         const int64_t e = tile * 4096 + j * 128 + lane * 4;
         if (MODE == 0) {
+          // the four results in byte lanes at once (acc[j] holds 4 counts c <= M)
           if (sums != nullptr) {
             if (ACC8) {
-              *reinterpret_cast<char4*>(reinterpret_cast<int8_t*>(sums) + e) =
-                  make_char4((signed char)s0, (signed char)s1, (signed char)s2, (signed char)s3);
+              // 2c - M mod 256 per byte: exact, since M <= 127 on this path
+              *reinterpret_cast<uint32_t*>(reinterpret_cast<int8_t*>(sums) + e) = swar_twice_minus(acc[j], M);
+            } else if (M <= 127) {
+              // the same exact int8 sums, sign-extended to int32
+              const uint32_t s8 = swar_twice_minus(acc[j], M);
+              *reinterpret_cast<int4*>(reinterpret_cast<int32_t*>(sums) + e) =
+                  make_int4((int)(s8 << 24) >> 24, (int)(s8 << 16) >> 24, (int)(s8 << 8) >> 24, (int)s8 >> 24);
             } else {
               *reinterpret_cast<int4*>(reinterpret_cast<int32_t*>(sums) + e) = make_int4(s0, s1, s2, s3);
             }
           }
-          if (maj != nullptr)
-            *reinterpret_cast<char4*>(maj + e) =
-                make_char4((signed char)vmaj(s0, tie_plus), (signed char)vmaj(s1, tie_plus), (signed char)vmaj(s2, tie_plus), (signed char)vmaj(s3, tie_plus));
+          if (maj != nullptr) *reinterpret_cast<uint32_t*>(maj + e) = swar_majority(acc[j], M, tie_plus);
         } else if (MODE == 1) {
           float4 wv = ld4(W + e);
           wv.x = fmaf(-eta, (float)vmaj(s0, tie_plus), wv.x);
