@@ -329,8 +329,10 @@ int signmuon_get_scales(signmuon_t h, float* dst_host);
 /* get_gram: the Gram matrix (g x g, g = min(rows, cols), row-major floats on
  * the host) that the last Newton-Schulz iteration of worker m used for
  * matrix `mat`: X X^T of the wide orientation; after one iteration it is the
- * unscaled Gram of the staged momentum (waits for the GPU).  After a post-vote
- * step, worker 0's slot holds the post-vote step's Gram. */
+ * unscaled Gram of the staged momentum (waits for the GPU).  On the bf16 path
+ * with the cubic polynomial, iterations after the first store the apply's
+ * whole operator a I + b X X^T there instead (the a X term folded into it).
+ * After a post-vote step, worker 0's slot holds the post-vote step's. */
 int signmuon_get_gram(signmuon_t h, int m, int mat, float* dst_host);
 
 /* Newton-Schulz coefficients: n=2 (a, b) for X <- aX + b(XX^T)X ([paper] §3

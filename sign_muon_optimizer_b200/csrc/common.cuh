@@ -96,9 +96,14 @@ struct GemmArgs {
   void* B;                   // quintic polynomial buffer
   int p_from_b;              // APPLY multiplies by B (quintic) instead of A
   int map_src, map_dst;      // tensor-map slots of X_src / X_dst (TMA path)
-  // epilogue coefficients: per-problem float2 when coef is non-null, else (c0, c1)
+  // epilogue coefficients: per-problem float2 when coef is non-null, else (c0, c1).
+  //   GRAM:   out = c1 acc + cdiag [row == col]
+  //   SQUARE: out = c0 A + c1 acc + cdiag [row == col]
+  //   APPLY:  out = c0 X + c1 acc, or (plain) out = acc
   const float2* coef;
   float c0, c1;
+  float cdiag;
+  int plain;                 // APPLY without the affine operand (its operator already holds a I)
   // final APPLY: fp32 flat output out + worker*out_stride + mat_off + r*cols + c
   // (skipped when out is null), and, when out_bits is non-null, the one-bit
   // signs (U >= 0) as LSB-first 32-bit words at out_bits + worker*bits_stride

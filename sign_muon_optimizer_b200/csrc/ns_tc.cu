@@ -305,7 +305,7 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* gbase = smem_raw + (base - raw);
   const int op = a.op;
-  const bool affine = op != OP_GRAM;                           // epilogue reads an operand
+  const bool affine = op == OP_SQUARE || (op == OP_APPLY && !a.plain);  // epilogue reads an operand
   const int nst = affine ? RING - 1 : RING;                    // operand ring depth
   const uint32_t epi0 = base + (RING - 1) * STAGE_BYTES;       // operand slices (affine)
   uint64_t* bars = reinterpret_cast<uint64_t*>(gbase + DATA_BYTES);
@@ -628,6 +628,17 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
                 v[8 * u + 2 * k + 1] = fmaf(c0, x.y, c1 * v[8 * u + 2 * k + 1]);
               }
             }
+          }
+          if (op == OP_GRAM) {
+#pragma unroll
+            for (int u = 0; u < 32; ++u) v[u] *= c1;
+          }
+          if (a.cdiag != 0.f && row >= col0 && row < col0 + 32) {
+            // the a I term of the apply's operator: the chunk holds this row's
+            // diagonal entry (any tile the diagonal crosses, 256 x 128 ones too)
+#pragma unroll
+            for (int u = 0; u < 32; ++u)
+              if (col0 + u == row) v[u] += a.cdiag;
           }
           const bool live = row_ok && col0 < tc.Ndim;
           const int ncol = live ? min(32, tc.Ndim - col0) : 0;

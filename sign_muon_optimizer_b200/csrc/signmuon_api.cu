@@ -278,7 +278,8 @@ void prof_collect(signmuon_t h) {
 // K == 0.
 // ---------------------------------------------------------------------------
 void gemm(signmuon_t h, int op, int slot, int src, int nw, const float2* coef, float c0, float c1,
-          bool final_out, float* out, int64_t out_stride, uint32_t* out_bits = nullptr, int64_t bits_stride = 0) {
+          bool final_out, float* out, int64_t out_stride, uint32_t* out_bits = nullptr, int64_t bits_stride = 0,
+          float cdiag = 0.f, bool plain = false) {
   const Plan& p = h->plan;
   sm::GemmArgs a{};
   a.tiles = h->d_tiles[op][slot];
@@ -299,6 +300,8 @@ void gemm(signmuon_t h, int op, int slot, int src, int nw, const float2* coef, f
   a.coef = coef;
   a.c0 = c0;
   a.c1 = c1;
+  a.cdiag = cdiag;
+  a.plain = plain ? 1 : 0;
   a.out = out;
   a.out_stride = out_stride;
   a.final_out = final_out ? 1 : 0;
@@ -369,7 +372,7 @@ void run_ns(signmuon_t h, int K, int nw, const sm::WorkerPtrs& kzero_in, float* 
   const bool spectral = h->scale == SIGNMUON_SCALE_SPECTRAL;
   if (K == 0) {
     if (spectral) {
-      gemm(h, sm::OP_GRAM, slot, 0, nw, nullptr, 0.f, 0.f, false, nullptr, 0);
+      gemm(h, sm::OP_GRAM, slot, 0, nw, nullptr, 0.f, 1.f, false, nullptr, 0);
       power_iteration(h, nw);
     }
     ProfScope ps(h, 13);
@@ -377,15 +380,30 @@ void run_ns(signmuon_t h, int K, int nw, const sm::WorkerPtrs& kzero_in, float* 
                           p.n_mats, h->scale_v, h->eps);
     return;
   }
+  // After the first iteration (bf16 path) the a X term joins the apply's
+  // operator: the Gram GEMM writes P = b A + a I (cubic) or the square GEMM
+  // B = b A + c A^2 + a I (quintic), and the apply is a plain GEMM X' = P X
+  // (X P for the tall orientation) whose epilogue reads no operand.  The
+  // first iteration keeps the affine epilogue: its coefficients carry the
+  // scale, which the power iteration takes from that iteration's pure Gram.
   int cur = 0;
   for (int k = 0; k < K; ++k) {
-    gemm(h, sm::OP_GRAM, slot, cur, nw, nullptr, 0.f, 0.f, false, nullptr, 0);
+    const bool fold = !p.fp32 && k > 0;
+    const bool last = (k == K - 1);
+    if (fold && !p.quintic)
+      gemm(h, sm::OP_GRAM, slot, cur, nw, nullptr, 0.f, h->ns_b, false, nullptr, 0, nullptr, 0, h->ns_a);
+    else
+      gemm(h, sm::OP_GRAM, slot, cur, nw, nullptr, 0.f, 1.f, false, nullptr, 0);
     if (k == 0 && spectral) power_iteration(h, nw);
     if (p.quintic)
-      gemm(h, sm::OP_SQUARE, slot, cur, nw, k == 0 ? h->coef_square : nullptr, h->ns_b, h->ns_c, false, nullptr, 0);
-    const bool last = (k == K - 1);
-    gemm(h, sm::OP_APPLY, slot, cur, nw, k == 0 ? h->coef_apply : nullptr, h->ns_a, p.quintic ? 1.f : h->ns_b, last,
-         out, out_stride, last ? out_bits : nullptr, bits_stride);
+      gemm(h, sm::OP_SQUARE, slot, cur, nw, k == 0 ? h->coef_square : nullptr, h->ns_b, h->ns_c, false, nullptr, 0,
+           nullptr, 0, fold ? h->ns_a : 0.f);
+    if (fold)
+      gemm(h, sm::OP_APPLY, slot, cur, nw, nullptr, 0.f, 1.f, last, out, out_stride, last ? out_bits : nullptr,
+           bits_stride, 0.f, true);
+    else
+      gemm(h, sm::OP_APPLY, slot, cur, nw, k == 0 ? h->coef_apply : nullptr, h->ns_a, p.quintic ? 1.f : h->ns_b,
+           last, out, out_stride, last ? out_bits : nullptr, bits_stride);
     cur ^= 1;
   }
 }
