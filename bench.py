@@ -78,8 +78,10 @@ def ns_flops_per_step(shapes, M, K, post_polar):
     return per_worker * (M + (1 if post_polar else 0))
 
 
-def gram_bytes(shapes):
-    return sum(2.0 * min(r, c) ** 2 for r, c in shapes)
+def gram_sym_bytes(shapes):
+    """bf16 bytes of the entries on and above each Gram's diagonal: what a
+    pass of the power iteration must read of the symmetric Gram."""
+    return sum(2.0 * min(r, c) * (min(r, c) + 1) / 2 for r, c in shapes)
 
 
 def hbm_bytes_per_step(shapes, M, P, post_polar):
@@ -88,14 +90,14 @@ def hbm_bytes_per_step(shapes, M, P, post_polar):
     b = {
         "momentum": d * (14.0 * M + 4.0),          # G r, Mom r+w, X w (bf16) per worker; W r once
         "pack": d * M * (4.0 + 1.0 / 8.0),          # U r (fp32), bits w
-        "power_iter": (P + 1) * M * gram_bytes(shapes),
+        "power_iter": (P + 1) * M * gram_sym_bytes(shapes),
         # bits r; with the post-vote polar the majority goes straight to the
         # bf16 X of the polar step (2 B), else the update of W (8 B) is fused
         "vote": M * d / 8.0 + (2.0 * d if post_polar else 8.0 * d),
         "update": 12.0 * d,                         # W r+w, D r
     }
     if post_polar:
-        b["power_iter"] += (P + 1) * gram_bytes(shapes)
+        b["power_iter"] += (P + 1) * gram_sym_bytes(shapes)
     return b
 
 
@@ -345,6 +347,47 @@ def measure_llama_vote(smo, stream, pk, shapes=None, reps=5):
     return out
 
 
+def measure_cublas_same_shapes(stream, pk, shapes=None, M=8, reps=5):
+    """cuBLAS (torch.bmm, bf16 in, fp32 accumulation, bf16 out) on the
+    bench step's own Newton-Schulz GEMM shapes, for comparison with the
+    library's tcgen05 kernel: per shape group, the Gram X X^T and the apply
+    A X of all M workers' matrices as one batched call each.  TFLOP/s counts
+    2 m^2 n per matrix for both (the algorithmic figure the library's own
+    per-kernel numbers use; cuBLAS computes the whole Gram)."""
+    import torch
+    shapes = shapes or SHAPES
+    groups = {}
+    for r, c in shapes:
+        key = (min(r, c), max(r, c))
+        groups[key] = groups.get(key, 0) + 1
+    g = torch.Generator(device="cuda")
+    g.manual_seed(6)
+    res = {"gram_ms": 0.0, "apply_ms": 0.0, "flops": 0.0, "groups": []}
+    for (m, n), cnt in sorted(groups.items()):
+        b = cnt * M
+        X = torch.randn(b, m, n, generator=g, device="cuda", dtype=torch.float32).to(torch.bfloat16)
+        A = torch.empty(b, m, m, device="cuda", dtype=torch.bfloat16)
+        Y = torch.empty_like(X)
+        XT = X.transpose(1, 2)
+        tg = _events_time(lambda: torch.bmm(X, XT, out=A), reps, stream)
+        ta = _events_time(lambda: torch.bmm(A, X, out=Y), reps, stream)
+        fl = 2.0 * m * m * n * b
+        res["gram_ms"] += tg
+        res["apply_ms"] += ta
+        res["flops"] += fl
+        res["groups"].append({"m": m, "n": n, "batch": b, "gram_TFLOP/s": fl / (tg / 1e3) / 1e12,
+                              "apply_TFLOP/s": fl / (ta / 1e3) / 1e12})
+        del X, A, Y, XT
+    torch.cuda.empty_cache()
+    for k in ("gram", "apply"):
+        tf = res["flops"] / (res[k + "_ms"] / 1e3) / 1e12
+        res[k + "_TFLOP/s"] = tf
+        res[k + "_frac_of_bf16_burst"] = tf / pk["bf16_tflops"]
+    res["note"] = ("torch.bmm on the same (m, n) groups, M = %d workers per call; one Newton-Schulz iteration's "
+                   "two GEMMs" % M)
+    return res
+
+
 def measure_ns_sweep(smo, stream, pk, grid=SWEEP_GRID):
     """The Newton-Schulz sweep: TFLOP/s of PolarNS (spectral P=2) on one
     8192^2 matrix, 64 x 1024^2 and 256 x 512x2048, M=8 workers of Gaussian
@@ -514,7 +557,8 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_extras:
         extras = {"resnet50": measure_resnet50(smo, stream, pk),
                   "llama_vote": measure_llama_vote(smo, stream, pk),
-                  "ns_sweep": measure_ns_sweep(smo, stream, pk)}
+                  "ns_sweep": measure_ns_sweep(smo, stream, pk),
+                  "cublas_same_shapes": measure_cublas_same_shapes(stream, pk)}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -635,6 +679,10 @@ def run_secondary(args):
         torch.cuda.empty_cache()
     if args.workload in ("resnet50", "all"):
         lines.append(measure_resnet50(smo, stream, pk))
+    if args.workload in ("cublas", "all"):
+        c = measure_cublas_same_shapes(stream, pk)
+        lines.append(dict({"metric": "cuBLAS TFLOP/s on the nanoGPT step's Newton-Schulz shapes (M=8, bf16)",
+                           "value": c["apply_TFLOP/s"], "unit": "TFLOP/s", "peak_kind": pk_kind}, **c))
     for ln in lines:
         print(json.dumps(ln), flush=True)
     return 0
@@ -727,7 +775,7 @@ def main():
     ap.add_argument("--capture-variant", default="nanogpt", choices=["nanogpt", "ternary", "unpacked"])
     ap.add_argument("--workload", default="nanogpt",
                     choices=["nanogpt", "llama_vote", "vote_100m", "ns_sweep", "ns_sweep_full", "resnet50",
-                             "ternary_vote", "variants", "collectives", "all"],
+                             "ternary_vote", "variants", "collectives", "cublas", "all"],
                     help="nanogpt: the headline line; the others print secondary measurements only")
     args = ap.parse_args()
     if args.capture_layers > 0:

@@ -47,11 +47,39 @@ struct Chunk {        // a piece of one matrix for the flat elementwise kernels
 };
 constexpr int kChunk = 4096;
 
-struct ProbRows {     // a block of Gram rows for the power-iteration matvec
+// Power iteration on a symmetric Gram: a 128 x 128 tiling of each problem's
+// g x g matrix; a pass visits the tiles (bi, bj) with bi <= bj only.
+constexpr int kPiTile = 128;
+struct PiTile {       // one upper-triangle tile of one problem: all that its block needs
+  int64_t aoff;       // the problem's Gram (elements of A)
+  int64_t uoff;       // its vectors (g entries)
+  int64_t poff;       // its partial sums (nt * nt * 128 entries, nt = ceil(g / 128))
   int p;              // problem id (worker*n_mats + mat)
-  int row0;
+  int g, gld;         // Gram side and row stride
+  int bi, bj;         // row and column slice, bi <= bj
+  int soff;           // index of the problem's first slice
 };
-constexpr int kPiRows = 32;
+struct PiSlice {      // one 128-row slice of one problem's iterate
+  int64_t uoff;
+  int64_t poff;
+  int p, g;
+  int bi;
+  int soff;           // index of the problem's first slice
+};
+struct PiReduce {     // what k_pi_reduce writes besides y
+  int last;           // the last pass: sigma^2 = u^T y, then the scale
+  const float* u;     // (last) the normalised iterate y came from
+  double* sq;         // per slice: ||y_slice||^2, or (last) u_slice . y_slice
+  int* counters;      // per problem, zero between launches
+  float* inv;         // (not last) per problem: 1 / ||y||, or 0 for a zero y
+  float eps;
+  int quintic;
+  float a, b, c;
+  float* scale;
+  float2* coef_apply;
+  float2* coef_square;
+  int* status;
+};
 
 struct WorkerPtrs {   // per-worker device pointers passed by value
   const float* p[kMaxWorkers];
@@ -150,7 +178,12 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
 void count_launch();
 void set_global_error(const char* msg);  // text for signmuon_last_error(NULL)
 int num_sms();                                   // SMs of the current device
-int stream_grid(int64_t work_items, int per_sm); // min(work_items, SMs * per_sm), at least 1
+// Blocks that the current device keeps resident per SM for a kernel launched
+// with `threads` threads and `smem` bytes of dynamic shared memory (at least 1).
+int resident_per_sm(const void* kernel, int threads, size_t smem);
+// Grid of a grid-stride kernel: min(work_items, SMs * min(per_sm, resident
+// blocks per SM)), at least 1 -- one full wave, never a partial second one.
+int stream_grid(const void* kernel, int threads, size_t smem, int64_t work_items, int per_sm);
 
 void launch_momentum(cudaStream_t s, const WorkerPtrs& G, const float* W, float* Mom, int64_t d,
                      int M, float beta, float lambda, void* X, int x_bf16, const Chunk* chunks,
@@ -164,14 +197,15 @@ void launch_fro_finalize(cudaStream_t s, int n_probs, int n_mats, int M, const f
                          float2* coef_apply, float2* coef_square, int* status);
 // warm != 0: keep each problem's stored iterate when it is non-zero and finite
 void launch_pi_init(cudaStream_t s, int n_probs, const int64_t* uoff, const int* prob_g, float* u, int warm);
-void launch_pi_matvec(cudaStream_t s, const ProbRows* rows, int n_rows, const void* A, int a_bf16,
-                      const int64_t* prob_a_off, const int* prob_g, const int* prob_gld,
-                      const int64_t* uoff, const float* u, float* y, int max_g);
-void launch_pi_normalize(cudaStream_t s, int n_probs, const int64_t* uoff, const int* prob_g,
-                         const float* y, float* u);
-void launch_pi_finalize(cudaStream_t s, int n_probs, const int64_t* uoff, const int* prob_g,
-                        const float* u, const float* y, float eps, int quintic, float a, float b,
-                        float c, float* scale, float2* coef_apply, float2* coef_square, int* status);
+// one pass over the upper-triangle tiles, one block per tile: partial sums
+// of A v, v = src (fold = 0) or v = src * inv[p] (fold = 1, which also stores
+// v into u)
+void launch_pi_tiles(cudaStream_t s, const PiTile* tiles, int n_tiles, const void* A, int a_bf16,
+                     const float* src, const float* inv, float* u, float* part, int fold);
+// y = the sum of each slice's partials in a fixed order; per problem 1 / ||y||
+// or, with r.last, sigma^2 = u^T y and the problem's scale and coefficients
+void launch_pi_reduce(cudaStream_t s, const PiSlice* slices, int n_slices, const float* part, float* y,
+                      const PiReduce& r);
 void launch_scale_flat(cudaStream_t s, const WorkerPtrs& in, int M, float* out, int64_t out_stride,
                        const Chunk* chunks, int n_chunks, const MatInfo* mats, int n_mats,
                        const float* scale, float eps);
@@ -185,11 +219,13 @@ void launch_vote(cudaStream_t s, const WorkerPtrs& signs, int M, int64_t d, void
 void launch_vote_update(cudaStream_t s, const WorkerPtrs& signs, int M, int64_t d, float* W, float eta,
                         const int* status, int tie_plus);
 void launch_vote_major(cudaStream_t s, const WorkerPtrs& signs, int M, int64_t d, float* D, int tie_plus);
-// streamable: every matrix starts at a multiple of 128 entries and has a
-// multiple of 8 columns (the streaming kernel's layout rule)
+// stage_off (two int64 per chunk: flat offset, offset in a one-problem-set
+// X) selects the streaming kernel; pass it only when every matrix starts at a
+// multiple of 128 entries and has a multiple of 8 columns (its layout rule),
+// else NULL
 void launch_vote_stage(cudaStream_t s, const WorkerPtrs& signs, int M, void* X, int x_bf16,
                        const Chunk* chunks, int n_chunks, const MatInfo* mats, const GroupInfo* groups,
-                       float* partials, float* D, int tie_plus, int streamable);
+                       float* partials, float* D, int tie_plus, const int64_t* stage_off);
 void launch_mean_stage(cudaStream_t s, const float* Mom, int64_t mom_stride, int M, void* X, int x_bf16,
                        const Chunk* chunks, int n_chunks, const MatInfo* mats, const GroupInfo* groups,
                        float* partials, float* D);

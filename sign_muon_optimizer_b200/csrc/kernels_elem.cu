@@ -9,6 +9,9 @@
 #include "common.cuh"
 
 #include <cmath>
+#include <map>
+#include <mutex>
+#include <tuple>
 
 namespace sm {
 
@@ -42,6 +45,11 @@ __device__ T block_sum(T v, T* red) {
     t = (sizeof(T) == 8) ? (T)warp_sum_d((double)t) : (T)warp_sum((float)t);
   }
   return t;  // valid in thread 0
+}
+
+// 16-byte global -> shared copy that bypasses the registers (and L1)
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
 
 __device__ __forceinline__ void store_x(void* X, int64_t idx, float v, bool bf16) {
@@ -196,6 +204,19 @@ k_fro_finalize(int n_mats, int M, const float* __restrict__ partials, const int*
 // Newton-Schulz GEMM's output, so no extra pass over X is needed.
 // With warm set, a problem whose stored iterate (the one the previous call
 // ended with) is non-zero and finite starts from it instead of ones/sqrt(g).
+//
+// A~ is symmetric, so a pass reads only the tiles (I, J), I <= J, of a
+// 128 x 128 tiling: an off-diagonal tile gives A_IJ v_J to y_I (its row sums)
+// and A_IJ^T v_I to y_J (its column sums), a diagonal tile A_II v_I.  A block
+// takes one tile; each contribution has its own slot in a partial-sum buffer
+// (slot K of slice I comes from the tile that pairs slices I and K), and
+// k_pi_reduce adds the slots of a slice in slot order, so the result does not
+// depend on the schedule.  A diagonal tile reads its upper triangle only (its rows give
+// the entries on and above the diagonal, its columns the ones above), so a
+// pass reads about g (g + 1) / 2 of the g^2 entries.  The normalisation of
+// an iterate is folded into the passes: the reduction's last block per
+// problem forms 1/||y||, and the next pass scales y by it while staging it;
+// after the last pass it forms sigma^2 = u^T y and the scale instead.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kThreads)
 k_pi_init(const int64_t* __restrict__ uoff, const int* __restrict__ prob_g, float* __restrict__ u, int warm) {
@@ -218,125 +239,230 @@ k_pi_init(const int64_t* __restrict__ uoff, const int* __restrict__ prob_g, floa
   for (int k = threadIdx.x; k < g; k += kThreads) up[k] = v;
 }
 
+// A lane's share of a 128 x 128 tile: NL 16-byte vectors of columns cl ..
+// cl + V - 1, one per tile row rw, rw + RPS, ...
+template <bool BF16>
+struct PiLane {
+  static constexpr int T = kPiTile;
+  static constexpr int V = BF16 ? 8 : 4;            // entries per 16-byte vector
+  static constexpr int LPR = T / V;                 // lanes per tile row: 16 or 32
+  static constexpr int RPS = 32 / LPR;              // tile rows per warp step: 2 or 1
+  static constexpr int RPW = T / (kThreads / 32);   // tile rows per warp
+  static constexpr int NL = RPW / RPS;              // vectors per lane: 8 or 16
+  static constexpr int ROWB = T * (BF16 ? 2 : 4);   // bytes of a tile row
+  static constexpr int TILEB = T * ROWB;            // 32 KB or 64 KB
+};
+
+// Two fp32 FMAs in one instruction (PTX fma.rn.f32x2, sm_100): the same
+// correctly rounded a * b + c per lane as fmaf.
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;"
+      : "=l"(r)
+      : "l"(*reinterpret_cast<const uint64_t*>(&a)), "l"(*reinterpret_cast<const uint64_t*>(&b)),
+        "l"(*reinterpret_cast<const uint64_t*>(&c)));
+  return *reinterpret_cast<const float2*>(&r);
+}
+
+// Sums of one tile out of shared memory: this lane's partial of each of its
+// rows (over its V columns) into rowp[r], its column partials into cacc
+// (pairs).  With MASK, entries past row or column g (whose vectors were not
+// loaded) and, on a diagonal tile, below the diagonal count as zero, and the
+// diagonal itself only in the row sums.
+template <bool BF16, bool MASK>
+__device__ __forceinline__ void pi_tile_sums(const uint8_t* tile, int rw, int cl, int rows_left, int nvalid,
+                                             bool diag, const float2* vjr, const float* vi, float* rowp,
+                                             float2* cacc) {
+  using L = PiLane<BF16>;
+#pragma unroll
+  for (int j = 0; j < L::NL; ++j) {
+    const int r = rw + j * L::RPS;
+    const uint4 raw = *reinterpret_cast<const uint4*>(tile + r * L::ROWB + cl * (BF16 ? 2 : 4));
+    float2 a[L::V / 2];
+    if (BF16) {
+      const uint32_t* w = reinterpret_cast<const uint32_t*>(&raw);
+#pragma unroll
+      for (int t = 0; t < L::V / 2; ++t)  // bf16 -> fp32 is a 16-bit shift
+        a[t] = make_float2(__uint_as_float(w[t] << 16), __uint_as_float(w[t] & 0xFFFF0000u));
+    } else {
+      const float2* fv = reinterpret_cast<const float2*>(&raw);
+#pragma unroll
+      for (int t = 0; t < L::V / 2; ++t) a[t] = fv[t];
+    }
+    int lo = 0;
+    if (MASK) {
+      lo = diag ? r - cl : 0;  // entries e < lo lie below the diagonal
+      const bool live = r < rows_left;
+#pragma unroll
+      for (int t = 0; t < L::V / 2; ++t) {
+        a[t].x = (live && 2 * t < nvalid && 2 * t >= lo) ? a[t].x : 0.f;
+        a[t].y = (live && 2 * t + 1 < nvalid && 2 * t + 1 >= lo) ? a[t].y : 0.f;
+      }
+    }
+    float2 sr = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int t = 0; t < L::V / 2; ++t) sr = fma2(a[t], vjr[t], sr);
+    rowp[r] = sr.x + sr.y;
+    const float2 vr = make_float2(vi[r], vi[r]);
+#pragma unroll
+    for (int t = 0; t < L::V / 2; ++t) {
+      float2 ac = a[t];
+      if (MASK && diag) {
+        if (2 * t == lo) ac.x = 0.f;
+        if (2 * t + 1 == lo) ac.y = 0.f;
+      }
+      cacc[t] = fma2(ac, vr, cacc[t]);
+    }
+  }
+}
+
+// One block per tile (I, J), I <= J: the tile comes into shared memory by
+// cp.async (vectors past row or column g, and on a diagonal tile the ones
+// wholly below the diagonal, are not read) while v_I and v_J are staged.
+// Its row sums go to slot J of slice I, its column sums (J > I) to slot I of
+// slice J; a diagonal tile adds its column sums to its row sums.
 template <bool BF16>
 __global__ void __launch_bounds__(kThreads)
-k_pi_matvec(const ProbRows* __restrict__ rows, const void* __restrict__ A,
-            const int64_t* __restrict__ prob_a_off, const int* __restrict__ prob_g,
-            const int* __restrict__ prob_gld, const int64_t* __restrict__ uoff,
-            const float* __restrict__ u, float* __restrict__ y) {
+k_pi_tiles(const PiTile* __restrict__ tiles, const void* __restrict__ A, const float* __restrict__ src,
+           const float* __restrict__ inv, float* __restrict__ u, float* __restrict__ part, int fold) {
   griddep_wait();
   griddep_launch();
-  // y[r] = sum_k A[r][k] u[k] for the block's kPiRows rows of one problem.
-  // u is staged in shared memory; each warp streams kRowsPerWarp rows at
-  // once (one 16-byte load per row and lane in flight per step) so that the
-  // HBM stream of A has enough loads in flight.
-  extern __shared__ float us[];
-  const ProbRows pr = rows[blockIdx.x];
-  const int p = pr.p;
-  const int g = prob_g[p], gld = prob_gld[p];
-  const float* up = u + uoff[p];
-  for (int k = threadIdx.x; k < g; k += kThreads) us[k] = up[k];
-  __syncthreads();
+  using L = PiLane<BF16>;
+  constexpr int T = kPiTile;
+  constexpr int esz = BF16 ? 2 : 4;
+  static_assert(kThreads == 2 * T, "one staging thread per entry of v_I and v_J");
+  __shared__ float vi[T], vj[T];
+  __shared__ float cols_s[kThreads / 32][T];     // warp w's column sums
+  __shared__ float rowp[L::LPR * (T + 1)];       // [c][r]: row r over column group c (stride T + 1)
+  extern __shared__ __align__(16) uint8_t pi_tile_smem[];   // the tile
+  const PiTile tl = tiles[blockIdx.x];
+  const int g = tl.g, I = tl.bi, J = tl.bj;
+  const bool diag = I == J;
+  const int nt = (g + T - 1) / T;
+  const int r0 = I * T, c0 = J * T, rows_left = g - r0;
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  constexpr int R = kPiRows / (kThreads / 32);
-  const int r0 = pr.row0 + wid * R;
-  float acc[R];
+  const int cl = (lane % L::LPR) * L::V;        // this lane's first column in the tile
+  const int rw = wid * L::RPW + lane / L::LPR;  // its first tile row
+  const int nvalid = g - (c0 + cl);             // entries of its vector inside the matrix
+  {
+    // A is g x gld with gld a multiple of 8, so a 16-byte vector that starts
+    // inside a row stays inside it
+    const char* src_a = reinterpret_cast<const char*>(A) + (tl.aoff + (int64_t)r0 * tl.gld + c0 + cl) * esz;
+    const int64_t row_bytes = (int64_t)tl.gld * esz;
+    const uint32_t dst = (uint32_t)__cvta_generic_to_shared(pi_tile_smem) + (uint32_t)(cl * esz);
 #pragma unroll
-  for (int j = 0; j < R; ++j) acc[j] = 0.f;
-  if (BF16) {
-    const __nv_bfloat16* a0 = reinterpret_cast<const __nv_bfloat16*>(A) + prob_a_off[p] + (int64_t)r0 * gld;
-    const int g8 = g & ~7;
-    for (int k = lane * 8; k < g8; k += 256) {
-      uint4 raw[R];
-#pragma unroll
-      for (int j = 0; j < R; ++j)
-        raw[j] = (r0 + j < g) ? __ldcs(reinterpret_cast<const uint4*>(a0 + (int64_t)j * gld + k)) : make_uint4(0, 0, 0, 0);
-      const float4 u0 = *reinterpret_cast<const float4*>(us + k);
-      const float4 u1 = *reinterpret_cast<const float4*>(us + k + 4);
-      const float uv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-#pragma unroll
-      for (int j = 0; j < R; ++j) {
-        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw[j]);
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          const float2 f = __bfloat1622float2(h[t]);
-          acc[j] = fmaf(f.x, uv[2 * t], acc[j]);
-          acc[j] = fmaf(f.y, uv[2 * t + 1], acc[j]);
-        }
-      }
+    for (int j = 0; j < L::NL; ++j) {
+      const int r = rw + j * L::RPS;
+      if (r < rows_left && nvalid > 0 && (!diag || cl + L::V - 1 >= r))
+        cp_async16(dst + (uint32_t)(r * L::ROWB), src_a + (int64_t)r * row_bytes);
     }
-    for (int k = g8 + lane; k < g; k += 32) {
-#pragma unroll
-      for (int j = 0; j < R; ++j)
-        if (r0 + j < g) acc[j] = fmaf(__bfloat162float(a0[(int64_t)j * gld + k]), us[k], acc[j]);
-    }
-  } else {
-    const float* a0 = reinterpret_cast<const float*>(A) + prob_a_off[p] + (int64_t)r0 * gld;
-    const int g4 = g & ~3;
-    for (int k = lane * 4; k < g4; k += 128) {
-      float4 f[R];
-#pragma unroll
-      for (int j = 0; j < R; ++j)
-        f[j] = (r0 + j < g) ? __ldcs(reinterpret_cast<const float4*>(a0 + (int64_t)j * gld + k)) : make_float4(0.f, 0.f, 0.f, 0.f);
-      const float4 uv = *reinterpret_cast<const float4*>(us + k);
-#pragma unroll
-      for (int j = 0; j < R; ++j) {
-        acc[j] = fmaf(f[j].x, uv.x, acc[j]);
-        acc[j] = fmaf(f[j].y, uv.y, acc[j]);
-        acc[j] = fmaf(f[j].z, uv.z, acc[j]);
-        acc[j] = fmaf(f[j].w, uv.w, acc[j]);
-      }
-    }
-    for (int k = g4 + lane; k < g; k += 32) {
-#pragma unroll
-      for (int j = 0; j < R; ++j)
-        if (r0 + j < g) acc[j] = fmaf(a0[(int64_t)j * gld + k], us[k], acc[j]);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  }
+  {
+    const float sc = fold ? inv[tl.p] : 1.f;
+    const int k = threadIdx.x & (T - 1);
+    if (threadIdx.x < T) {
+      const float v = (r0 + k < g) ? src[tl.uoff + r0 + k] * sc : 0.f;
+      vi[k] = v;
+      if (fold && diag && r0 + k < g) u[tl.uoff + r0 + k] = v;  // the normalised iterate, once per slice
+    } else {
+      vj[k] = (c0 + k < g) ? src[tl.uoff + c0 + k] * sc : 0.f;
     }
   }
-#pragma unroll
-  for (int j = 0; j < R; ++j) {
-    const float v = warp_sum(acc[j]);
-    if (lane == 0 && r0 + j < g) y[uoff[p] + r0 + j] = v;
-  }
-}
-
-__global__ void __launch_bounds__(kThreads)
-k_pi_normalize(const int64_t* __restrict__ uoff, const int* __restrict__ prob_g,
-               const float* __restrict__ y, float* __restrict__ u) {
-  griddep_wait();
-  griddep_launch();
-  __shared__ double red[32];
-  __shared__ float inv;
-  const int p = blockIdx.x;
-  const int g = prob_g[p];
-  const float* yp = y + uoff[p];
-  double s = 0.0;
-  for (int k = threadIdx.x; k < g; k += kThreads) s += (double)yp[k] * (double)yp[k];
-  const double t = block_sum<double>(s, red);
-  if (threadIdx.x == 0) inv = (t > 0.0) ? (float)(1.0 / sqrt(t)) : 0.f;  // a zero iterate stays zero
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
   __syncthreads();
-  for (int k = threadIdx.x; k < g; k += kThreads) u[uoff[p] + k] = yp[k] * inv;
+  float2 vjr[L::V / 2], cacc[L::V / 2];
+#pragma unroll
+  for (int t = 0; t < L::V / 2; ++t) {
+    vjr[t] = make_float2(vj[cl + 2 * t], vj[cl + 2 * t + 1]);
+    cacc[t] = make_float2(0.f, 0.f);
+  }
+  float* rowp_c = rowp + (lane % L::LPR) * (T + 1);
+  if (diag || rows_left < T || c0 + T > g)   // block-uniform
+    pi_tile_sums<BF16, true>(pi_tile_smem, rw, cl, rows_left, nvalid, diag, vjr, vi, rowp_c, cacc);
+  else
+    pi_tile_sums<BF16, false>(pi_tile_smem, rw, cl, rows_left, nvalid, false, vjr, vi, rowp_c, cacc);
+  if (L::RPS == 2) {
+#pragma unroll
+    for (int t = 0; t < L::V / 2; ++t) {
+      cacc[t].x += __shfl_xor_sync(0xffffffffu, cacc[t].x, 16);
+      cacc[t].y += __shfl_xor_sync(0xffffffffu, cacc[t].y, 16);
+    }
+  }
+  if (lane < L::LPR) {
+#pragma unroll
+    for (int t = 0; t < L::V / 2; ++t) {
+      cols_s[wid][cl + 2 * t] = cacc[t].x;
+      cols_s[wid][cl + 2 * t + 1] = cacc[t].y;
+    }
+  }
+  __syncthreads();
+  float* pp = part + tl.poff;
+  const int64_t gp = (int64_t)nt * T;
+  const int k = threadIdx.x & (T - 1);
+  float cs = 0.f;
+  if (diag || threadIdx.x >= T) {
+#pragma unroll
+    for (int w = 0; w < kThreads / 32; ++w) cs += cols_s[w][k];
+  }
+  if (threadIdx.x < T) {
+    float rs = 0.f;
+#pragma unroll
+    for (int c = 0; c < L::LPR; ++c) rs += rowp[c * (T + 1) + k];
+    // slice I, slot J: the row sums (a diagonal tile adds its column sums,
+    // the mirror of its strict upper triangle)
+    pp[(int64_t)J * gp + r0 + k] = diag ? rs + cs : rs;
+  } else if (!diag) {
+    pp[(int64_t)I * gp + c0 + k] = cs;  // slice J, slot I
+  }
 }
 
-__global__ void __launch_bounds__(kThreads)
-k_pi_finalize(const int64_t* __restrict__ uoff, const int* __restrict__ prob_g,
-              const float* __restrict__ u, const float* __restrict__ y, float eps, int quintic,
-              float a, float b, float c, float* __restrict__ scale, float2* coef_apply,
-              float2* coef_square, int* status) {
+// One block per 128-row slice: y = its nt slots added in slot order,
+// ||y_slice||^2 (or, on the last pass, u_slice . y_slice) in fp64; the
+// problem's last slice to finish adds the slices' figures in slice order:
+// 1 / ||y|| for the next pass, or sigma^2 = u^T y and the scale.
+__global__ void __launch_bounds__(kPiTile)
+k_pi_reduce(const PiSlice* __restrict__ slices, const float* __restrict__ part, float* __restrict__ y,
+            PiReduce rd) {
   griddep_wait();
   griddep_launch();
+  constexpr int T = kPiTile;
   __shared__ double red[32];
-  const int p = blockIdx.x;
-  const int g = prob_g[p];
-  double s = 0.0;
-  for (int k = threadIdx.x; k < g; k += kThreads) s += (double)u[uoff[p] + k] * (double)y[uoff[p] + k];
-  const double t = block_sum<double>(s, red);
-  if (threadIdx.x == 0) {
-    const float sc = (float)sqrt(fmax(t, 0.0));
-    if (!isfinite(t)) atomicOr(status, 1);
-    scale[p] = sc;
-    set_coefs(p, 1.f / (sc + eps), quintic, a, b, c, coef_apply, coef_square);
+  __shared__ int is_last;
+  const PiSlice sl = slices[blockIdx.x];
+  const int g = sl.g;
+  const int nt = (g + T - 1) / T;
+  const int64_t gp = (int64_t)nt * T;
+  const int r = sl.bi * T + threadIdx.x;
+  const float* pp = part + sl.poff + r;
+  float v = 0.f;
+#pragma unroll 8
+  for (int k = 0; k < nt; ++k) v += pp[(int64_t)k * gp];
+  double acc = 0.0;
+  if (r < g) {
+    y[sl.uoff + r] = v;
+    acc = rd.last ? (double)rd.u[sl.uoff + r] * (double)v : (double)v * (double)v;
   }
+  const double t = block_sum<double>(acc, red);
+  if (threadIdx.x == 0) {
+    rd.sq[sl.soff + sl.bi] = t;
+    __threadfence();
+    is_last = (atomicAdd(&rd.counters[sl.p], 1) == nt - 1);
+  }
+  __syncthreads();
+  if (!is_last || threadIdx.x != 0) return;
+  __threadfence();
+  double tt = 0.0;
+  for (int i = 0; i < nt; ++i) tt += __ldcg(rd.sq + sl.soff + i);
+  rd.counters[sl.p] = 0;
+  if (!rd.last) {
+    rd.inv[sl.p] = (tt > 0.0) ? (float)(1.0 / sqrt(tt)) : 0.f;  // a zero iterate stays zero
+    return;
+  }
+  const float scv = (float)sqrt(fmax(tt, 0.0));
+  if (!isfinite(tt)) atomicOr(rd.status, 1);
+  rd.scale[sl.p] = scv;
+  set_coefs(sl.p, 1.f / (scv + rd.eps), rd.quintic, rd.a, rd.b, rd.c, rd.coef_apply, rd.coef_square);
 }
 
 // K = 0: U = X0 = in / (s + eps) straight from the fp32 input.
@@ -552,6 +678,16 @@ __device__ __forceinline__ uint32_t swar_majority(uint32_t x, int M, int tie_plu
   return (gt >> 7) | ((lt >> 7) * 0xFFu);
 }
 
+// PTX prmt in its default mode with b = 0: byte n of the result is byte
+// (SEL >> 4n) & 7 of {a, b} (a = bytes 0-3), and bit 3 of that selector
+// nibble replicates the selected byte's top bit over the result byte.
+template <uint32_t SEL>
+__device__ __forceinline__ uint32_t prmt_sx(uint32_t a) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, 0, %2;" : "=r"(r) : "r"(a), "n"(SEL));
+  return r;
+}
+
 // Streaming vote for M <= 255 (byte-lane counters): each warp takes tiles of 4096 consecutive entries (512 bytes of
 // every worker's stream).  The bytes come into shared memory by cp.async, 16
 // per lane (each load instruction reads 512 contiguous bytes of one stream),
@@ -564,33 +700,31 @@ constexpr int kVoteBatch = 8;
 constexpr int kVoteWarps = 4;                  // warps per block
 constexpr int kVoteTileB = 512;                // bytes of one stream per tile
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
 
 // MODE 3 (staging of the post-vote polar step's input): the work items are
 // the plan's chunks instead of flat tiles.  Chunk c covers entries base ..
 // base + len - 1 of the flat vector (base = its matrix's offset + its start,
 // a multiple of 128; len <= 4096); its majorities go to the bf16 X of the
 // one-problem-set Newton-Schulz input, which for a matrix with a multiple of
-// 8 columns is the chunk's contiguous range starting at xb + start, and
+// 8 columns is the chunk's contiguous range starting at its X offset, and
 // partials[c] receives the chunk's count of non-zero majorities (its sum of
-// squares).
+// squares).  off[c] = (base, X offset), precomputed so that a chunk's bytes
+// can be requested after a single table load.
 struct VoteStage {
   __nv_bfloat16* X;
   const Chunk* chunks;
-  const MatInfo* mats;
-  const GroupInfo* groups;
+  const longlong2* off;
   float* partials;
 };
 
 template <int MODE, bool ACC8>
-__global__ void __launch_bounds__(kVoteWarps * 32)
+__global__ void __launch_bounds__(kVoteWarps * 32, 6)
 k_vote_stream(WorkerPtrs signs, int M, int64_t ntiles,
               void* __restrict__ sums, int8_t* __restrict__ maj, float* __restrict__ W, float eta,
               float* __restrict__ D, const int* __restrict__ status, int tie_plus, VoteStage st) {
   griddep_wait();
   griddep_launch();
+  constexpr bool STAGE = MODE >= 3;  // chunks of the post-vote input (MODE 4 also writes D)
   if (MODE == 1 && status != nullptr && (status[0] | status[1]) != 0) return;  // keep W on error
   extern __shared__ __align__(16) uint8_t vsm[];   // [warp][2][kVoteBatch][512]
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
@@ -604,19 +738,16 @@ k_vote_stream(WorkerPtrs signs, int M, int64_t ntiles,
   int batch = 0;
   // flat start and length of work item t (a whole tile, or one chunk)
   auto item_base = [&](int64_t t) -> int64_t {
-    if (MODE == 3) {
-      const Chunk c = st.chunks[t];
-      return st.mats[c.mat].off + c.start;
-    }
+    if (STAGE) return st.off[t].x;
     return t * 4096;
   };
-  auto item_len = [&](int64_t t) -> int { return MODE == 3 ? st.chunks[t].len : 4096; };
+  auto item_len = [&](int64_t t) -> int { return STAGE ? st.chunks[t].len : 4096; };
   auto issue = [&](int64_t t, int bt, int buf) {
     const uint32_t dst = buf0 + (uint32_t)buf * (kVoteBatch * kVoteTileB) + (uint32_t)lane * 16;
     const int64_t boff = item_base(t) >> 3;
     // a lane's 16 bytes hold entries 128 lane .. 128 lane + 127 of the item;
     // pieces wholly past a short chunk's end are not read
-    const bool live = MODE != 3 || lane * 128 < item_len(t);
+    const bool live = !STAGE || lane * 128 < item_len(t);
 #pragma unroll
     for (int i = 0; i < kVoteBatch; ++i) {
       const int m = bt * kVoteBatch + i;
@@ -710,31 +841,35 @@ k_vote_stream(WorkerPtrs signs, int M, int64_t ntiles,
         asm volatile("ld.shared.u32 %0, [%1];" : "=r"(acc[j]) : "r"(tr + (uint32_t)(j * 32 + (lane ^ j)) * 4) : "memory");
       __syncwarp();
     }
-    if (batch == nbatch - 1 && MODE == 3) {
+    if (batch == nbatch - 1 && STAGE) {
       // chunk done: its majorities into X (4 bf16 per lane and step, so each
-      // warp store writes 256 contiguous bytes) and D, its non-zero count
-      const Chunk ch = st.chunks[tile];
-      const MatInfo mi = st.mats[ch.mat];
-      const GroupInfo gi = st.groups[mi.group];
-      __nv_bfloat16* xo = st.X + gi.x_base + (int64_t)mi.q * gi.rows * gi.ld + ch.start;
-      const int64_t fb = mi.off + ch.start;
+      // warp store writes 256 contiguous bytes) and (MODE 4) D, its non-zero
+      // count
+      const longlong2 o = st.off[tile];
+      const int len = st.chunks[tile].len;
+      __nv_bfloat16* xo = st.X + o.y;
+      const int64_t fb = o.x;
+      const uint32_t H = 0x80808080u;
+      const uint32_t kgt = (uint32_t)(127 - M / 2) * 0x01010101u;
+      const uint32_t klt = (uint32_t)(128 - (M + 1) / 2) * 0x01010101u;
       int nz = 0;
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
         const int e = j * 128 + lane * 4;
-        if (e < ch.len) {
-          // the four majorities as int8 byte lanes (0x01, 0xFF or 0), then as
-          // bf16 pairs: +1 = 0x3F80, -1 = 0xBF80, 0 = 0 (sign at bit 15 of a half)
-          const uint32_t mj = swar_majority(acc[j], M, tie_plus);
-          const uint32_t nzb = (mj | (mj << 7)) & 0x80808080u;    // bit 7 of a non-zero byte
-          const uint32_t sgn = mj & 0x80808080u;                  // bit 7 of a -1 byte
-          nz += __popc(nzb);
+        if (e < len) {
+          // per byte lane (count c): bit 7 of neg when c < M/2 (majority -1),
+          // of nzm when the majority is not 0 (c > M/2 too; every entry with
+          // tie_plus); as bf16 pairs +1 = 0x3F80, -1 = 0xBF80, 0 = 0
+          const uint32_t x = acc[j];
+          const uint32_t neg = ~(x + klt) & H;
+          const uint32_t nzm = tie_plus ? H : (((x + kgt) & H) | neg);
+          nz += __popc(nzm);
           uint2 u;
-          u.x = ((__byte_perm(nzb, 0, 0x1404) >> 15) * 0xFFFFu & 0x3F803F80u) | __byte_perm(sgn, 0, 0x1404);
-          u.y = ((__byte_perm(nzb, 0, 0x3424) >> 15) * 0xFFFFu & 0x3F803F80u) | __byte_perm(sgn, 0, 0x3424);
+          u.x = (prmt_sx<0x9988>(nzm) & 0x3F803F80u) | (prmt_sx<0x9988>(neg) & 0x80008000u);
+          u.y = (prmt_sx<0xBBAA>(nzm) & 0x3F803F80u) | (prmt_sx<0xBBAA>(neg) & 0x80008000u);
           *reinterpret_cast<uint2*>(xo + e) = u;
-          if (D != nullptr) {
-            const int c0 = acc[j] & 0xFF, c1 = (acc[j] >> 8) & 0xFF, c2 = (acc[j] >> 16) & 0xFF, c3 = acc[j] >> 24;
+          if (MODE == 4) {
+            const int c0 = x & 0xFF, c1 = (x >> 8) & 0xFF, c2 = (x >> 16) & 0xFF, c3 = x >> 24;
             st4(D + fb + e, make_float4((float)vmaj(2 * c0 - M, tie_plus), (float)vmaj(2 * c1 - M, tie_plus),
                                         (float)vmaj(2 * c2 - M, tie_plus), (float)vmaj(2 * c3 - M, tie_plus)));
           }
@@ -742,7 +877,7 @@ k_vote_stream(WorkerPtrs signs, int M, int64_t ntiles,
       }
       nz = __reduce_add_sync(0xffffffffu, nz);
       if (lane == 0) st.partials[tile] = (float)nz;
-    } else if (batch == nbatch - 1) {
+    } else if (!STAGE && batch == nbatch - 1) {
       // tile done: write its 4096 results
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
@@ -980,8 +1115,27 @@ int num_sms() {
   return g_num_sms;
 }
 
-int stream_grid(int64_t work_items, int per_sm) {
-  const int64_t cap = (int64_t)num_sms() * per_sm;
+int resident_per_sm(const void* kernel, int threads, size_t smem) {
+  // looked up once per (kernel, block shape); launches come from one host
+  // thread per handle, but handles may live on several threads
+  static std::mutex mu;
+  static std::map<std::tuple<const void*, int, size_t>, int> cache;
+  const auto key = std::make_tuple(kernel, threads, smem);
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = cache.find(key);
+  if (it != cache.end()) return it->second;
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, smem) != cudaSuccess || n < 1) {
+    cudaGetLastError();
+    n = 1;
+  }
+  cache[key] = n;
+  return n;
+}
+
+int stream_grid(const void* kernel, int threads, size_t smem, int64_t work_items, int per_sm) {
+  const int fit = resident_per_sm(kernel, threads, smem);
+  const int64_t cap = (int64_t)num_sms() * (per_sm < fit ? per_sm : fit);
   if (work_items < 1) return 1;
   return (int)(work_items < cap ? work_items : cap);
 }
@@ -1021,32 +1175,26 @@ void launch_pi_init(cudaStream_t s, int n_probs, const int64_t* uoff, const int*
   launch_pdl(k_pi_init, dim3(n_probs), dim3(kThreads), 0, s, uoff, prob_g, u, warm);
 }
 
-void launch_pi_matvec(cudaStream_t s, const ProbRows* rows, int n_rows, const void* A, int a_bf16,
-                      const int64_t* prob_a_off, const int* prob_g, const int* prob_gld,
-                      const int64_t* uoff, const float* u, float* y, int max_g) {
+void launch_pi_tiles(cudaStream_t s, const PiTile* tiles, int n_tiles, const void* A, int a_bf16,
+                     const float* src, const float* inv, float* u, float* part, int fold) {
+  if (n_tiles <= 0) return;
   count_launch();
-  const size_t smem = (size_t)max_g * sizeof(float);
   if (a_bf16) {
-    if (smem > 48 * 1024) cudaFuncSetAttribute(k_pi_matvec<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    launch_pdl(k_pi_matvec<true>, dim3(n_rows), dim3(kThreads), smem, s, rows, A, prob_a_off, prob_g, prob_gld, uoff, u, y);
+    const size_t smem = (size_t)PiLane<true>::TILEB;
+    launch_pdl(k_pi_tiles<true>, dim3(n_tiles), dim3(kThreads), smem, s, tiles, A, src, inv, u, part, fold);
   } else {
-    if (smem > 48 * 1024) cudaFuncSetAttribute(k_pi_matvec<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    launch_pdl(k_pi_matvec<false>, dim3(n_rows), dim3(kThreads), smem, s, rows, A, prob_a_off, prob_g, prob_gld, uoff, u, y);
+    // 64 KB of dynamic shared memory needs the opt-in (per device)
+    const size_t smem = (size_t)PiLane<false>::TILEB;
+    cudaFuncSetAttribute(k_pi_tiles<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    launch_pdl(k_pi_tiles<false>, dim3(n_tiles), dim3(kThreads), smem, s, tiles, A, src, inv, u, part, fold);
   }
 }
 
-void launch_pi_normalize(cudaStream_t s, int n_probs, const int64_t* uoff, const int* prob_g,
-                         const float* y, float* u) {
+void launch_pi_reduce(cudaStream_t s, const PiSlice* slices, int n_slices, const float* part, float* y,
+                      const PiReduce& r) {
+  if (n_slices <= 0) return;
   count_launch();
-  launch_pdl(k_pi_normalize, dim3(n_probs), dim3(kThreads), 0, s, uoff, prob_g, y, u);
-}
-
-void launch_pi_finalize(cudaStream_t s, int n_probs, const int64_t* uoff, const int* prob_g,
-                        const float* u, const float* y, float eps, int quintic, float a, float b,
-                        float c, float* scale, float2* coef_apply, float2* coef_square, int* status) {
-  count_launch();
-  launch_pdl(k_pi_finalize, dim3(n_probs), dim3(kThreads), 0, s, uoff, prob_g, u, y, eps, quintic, a, b, c, scale,
-                                             coef_apply, coef_square, status);
+  launch_pdl(k_pi_reduce, dim3(n_slices), dim3(kPiTile), 0, s, slices, part, y, r);
 }
 
 void launch_scale_flat(cudaStream_t s, const WorkerPtrs& in, int M, float* out, int64_t out_stride,
@@ -1063,7 +1211,7 @@ void launch_pack(cudaStream_t s, const float* U, int64_t u_stride, int64_t d, ui
   if (d <= 0) return;
   count_launch();
   const int64_t warps = (d + 1023) / 1024;
-  const int blocks = stream_grid((warps + 7) / 8, 16);
+  const int blocks = stream_grid((const void*)k_pack, kThreads, 0, (warps + 7) / 8, 16);
   dim3 grid(blocks, M);
   launch_pdl(k_pack, dim3(grid), dim3(kThreads), 0, s, U, u_stride, d, out, out_stride);
 }
@@ -1079,9 +1227,8 @@ void vote_dispatch(cudaStream_t s, const WorkerPtrs& signs, int M, int64_t d, vo
   if (M <= 255 && d >= 4096) {
     const int64_t ntiles = d / 4096;
     const size_t smem = (size_t)kVoteWarps * 2 * kVoteBatch * kVoteTileB;
-    const int64_t want = (ntiles + kVoteWarps - 1) / kVoteWarps;
-    const int64_t cap = (int64_t)num_sms() * 6;
-    const int blocks = (int)(want < cap ? want : cap);
+    const int blocks = stream_grid((const void*)k_vote_stream<MODE, ACC8>, kVoteWarps * 32, smem,
+                                   (ntiles + kVoteWarps - 1) / kVoteWarps, 8);
     count_launch();
     launch_pdl(k_vote_stream<MODE, ACC8>, dim3(blocks), dim3(kVoteWarps * 32), smem, s, signs, M, ntiles, sums, maj,
                W, eta, D, status, tie_plus, VoteStage{});
@@ -1094,7 +1241,7 @@ void vote_dispatch(cudaStream_t s, const WorkerPtrs& signs, int M, int64_t d, vo
   for (int m = 0; m < M; ++m) sp.p[m] = reinterpret_cast<const float*>(reinterpret_cast<const uint8_t*>(signs.p[m]) + boff);
   void* sums2 = sums == nullptr ? nullptr : reinterpret_cast<uint8_t*>(sums) + done * (ACC8 ? 1 : 4);
   count_launch();
-  const int blocks = stream_grid((rest / 512 + 8) / 8 + 1, 8);
+  const int blocks = stream_grid((const void*)k_vote<MODE, ACC8>, kThreads, 0, (rest / 512 + 8) / 8 + 1, 8);
   launch_pdl(k_vote<MODE, ACC8>, dim3(blocks), dim3(kThreads), 0, s, sp, M, rest, sums2,
              maj == nullptr ? nullptr : maj + done, W == nullptr ? nullptr : W + done, eta,
              D == nullptr ? nullptr : D + done, status, tie_plus);
@@ -1120,18 +1267,24 @@ void launch_vote_major(cudaStream_t s, const WorkerPtrs& signs, int M, int64_t d
 
 void launch_vote_stage(cudaStream_t s, const WorkerPtrs& signs, int M, void* X, int x_bf16,
                        const Chunk* chunks, int n_chunks, const MatInfo* mats, const GroupInfo* groups,
-                       float* partials, float* D, int tie_plus, int streamable) {
+                       float* partials, float* D, int tie_plus, const int64_t* stage_off) {
   if (n_chunks <= 0) return;
   count_launch();
-  if (streamable && x_bf16 && M <= 255) {
+  if (stage_off != nullptr && x_bf16 && M <= 255) {
     // one warp per chunk, the next chunk's bytes in flight while one is counted
     const size_t smem = (size_t)kVoteWarps * 2 * kVoteBatch * kVoteTileB;
-    const int64_t want = ((int64_t)n_chunks + kVoteWarps - 1) / kVoteWarps;
-    const int64_t cap = (int64_t)num_sms() * 6;
-    const int blocks = (int)(want < cap ? want : cap);
-    const VoteStage st{reinterpret_cast<__nv_bfloat16*>(X), chunks, mats, groups, partials};
-    launch_pdl(k_vote_stream<3, false>, dim3(blocks), dim3(kVoteWarps * 32), smem, s, signs, M, (int64_t)n_chunks,
-               nullptr, nullptr, nullptr, 0.f, D, nullptr, tie_plus, st);
+    const VoteStage st{reinterpret_cast<__nv_bfloat16*>(X), chunks, reinterpret_cast<const longlong2*>(stage_off),
+                       partials};
+    const int64_t warps = ((int64_t)n_chunks + kVoteWarps - 1) / kVoteWarps;
+    if (D == nullptr) {
+      const int blocks = stream_grid((const void*)k_vote_stream<3, false>, kVoteWarps * 32, smem, warps, 8);
+      launch_pdl(k_vote_stream<3, false>, dim3(blocks), dim3(kVoteWarps * 32), smem, s, signs, M, (int64_t)n_chunks,
+                 nullptr, nullptr, nullptr, 0.f, nullptr, nullptr, tie_plus, st);
+    } else {
+      const int blocks = stream_grid((const void*)k_vote_stream<4, false>, kVoteWarps * 32, smem, warps, 8);
+      launch_pdl(k_vote_stream<4, false>, dim3(blocks), dim3(kVoteWarps * 32), smem, s, signs, M, (int64_t)n_chunks,
+                 nullptr, nullptr, nullptr, 0.f, D, nullptr, tie_plus, st);
+    }
     return;
   }
   launch_pdl(k_vote_stage, dim3(n_chunks), dim3(kThreads), 0, s, signs, M, X, x_bf16, chunks, mats, groups, partials,
@@ -1150,7 +1303,7 @@ void launch_update(cudaStream_t s, float* W, const float* D, int64_t d, float et
                    const int* status) {
   if (d <= 0) return;
   count_launch();
-  const int blocks = stream_grid((d / 4 + kThreads - 1) / kThreads + 1, 8);
+  const int blocks = stream_grid((const void*)k_update, kThreads, 0, (d / 4 + kThreads - 1) / kThreads + 1, 8);
   launch_pdl(k_update, dim3(blocks), dim3(kThreads), 0, s, W, D, d, eta, status);
 }
 

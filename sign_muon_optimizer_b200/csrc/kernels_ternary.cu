@@ -181,7 +181,8 @@ template <int MODE, bool ACC8>
 void vote_tern(cudaStream_t s, const WorkerPtrs& signs, int M, int64_t d, void* sums, int8_t* maj, float* W,
                float eta, float* D, const int* status, int tie_plus) {
   count_launch();
-  const int blocks = stream_grid(((d >> 4) + kTThreads - 1) / kTThreads, 8);
+  const int blocks = stream_grid((const void*)k_vote_tern<MODE, ACC8>, kTThreads, 0,
+                                 ((d >> 4) + kTThreads - 1) / kTThreads, 8);
   launch_pdl(k_vote_tern<MODE, ACC8>, dim3(blocks), dim3(kTThreads), 0, s, signs, M, d, sums, maj, W, eta, D, status, tie_plus);
 }
 
@@ -222,7 +223,7 @@ void launch_sign8(cudaStream_t s, const float* U, int64_t u_stride, int64_t d, i
                   int M) {
   if (d <= 0 || M <= 0) return;
   count_launch();
-  const int blocks = stream_grid(((d >> 4) + kTThreads - 1) / kTThreads, 8);
+  const int blocks = stream_grid((const void*)k_sign8, kTThreads, 0, ((d >> 4) + kTThreads - 1) / kTThreads, 8);
   dim3 grid(blocks, M);
   launch_pdl(k_sign8, dim3(grid), dim3(kTThreads), 0, s, U, u_stride, d, out, out_stride);
 }
@@ -248,7 +249,8 @@ void launch_vote_ternary_major(cudaStream_t s, const WorkerPtrs& signs, int M, i
 void launch_sums_major(cudaStream_t s, const void* sums, int acc8, int64_t d, float* D, int tie_plus) {
   if (d <= 0) return;
   count_launch();
-  const int blocks = stream_grid(((d >> 2) + kTThreads - 1) / kTThreads, 8);
+  const int blocks = acc8 ? stream_grid((const void*)k_sums_major<true>, kTThreads, 0, ((d >> 2) + kTThreads - 1) / kTThreads, 8)
+                         : stream_grid((const void*)k_sums_major<false>, kTThreads, 0, ((d >> 2) + kTThreads - 1) / kTThreads, 8);
   if (acc8) launch_pdl(k_sums_major<true>, dim3(blocks), dim3(kTThreads), 0, s, sums, d, D, tie_plus);
   else launch_pdl(k_sums_major<false>, dim3(blocks), dim3(kTThreads), 0, s, sums, d, D, tie_plus);
 }

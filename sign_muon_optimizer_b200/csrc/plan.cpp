@@ -170,6 +170,11 @@ int make_plan(const int64_t* shapes, int n_mats, int M, int K, int scale, int P,
       c.start = s;
       c.len = (int)std::min<int64_t>(kChunk, n - s);
       p.chunks.push_back(c);
+      // flat offset of the chunk, and its offset in a one-problem-set X
+      // when the matrix's rows are unpadded there
+      const GroupInfo& g = p.groups[p.mats[i].group];
+      p.stage_off.push_back(p.mats[i].off + s);
+      p.stage_off.push_back(g.x_base + (int64_t)p.mats[i].q * g.rows * g.ld + s);
     }
     p.mat_nchunks[i] = (int)p.chunks.size() - p.mat_chunk0[i];
   }
@@ -178,24 +183,35 @@ int make_plan(const int64_t* shapes, int n_mats, int M, int K, int scale, int P,
     build_tiles(p, op, 1, &p.tiles[op][1]);
   }
   // power iteration tables (worker-major problems so worker 0 is a prefix)
-  int64_t u = 0;
+  int64_t u = 0, part = 0;
   for (int w = 0; w < M; ++w) {
     for (int i = 0; i < n_mats; ++i) {
       const MatInfo& mi = p.mats[i];
       const GroupInfo& g = p.groups[mi.group];
       const int pid = w * n_mats + i;
+      const int nt = (int)((g.g + kPiTile - 1) / kPiTile);
       p.uoff.push_back(u);
+      p.poff.push_back(part);
       p.prob_g.push_back(g.g);
       p.prob_gld.push_back(g.gld);
       p.prob_aoff.push_back(g.a_base + (int64_t)(w * g.count + mi.q) * g.g * g.gld);
+      const int soff = (int)p.pi_slices.size();
+      p.soff.push_back(soff);
+      for (int bi = 0; bi < nt; ++bi) {
+        p.pi_slices.push_back(PiSlice{u, part, pid, g.g, bi, soff});
+        for (int bj = bi; bj < nt; ++bj)
+          p.pi_tiles.push_back(PiTile{p.prob_aoff.back(), u, part, pid, g.g, g.gld, bi, bj, soff});
+      }
       u += g.g;
-      for (int r0 = 0; r0 < g.g; r0 += kPiRows) p.pi_rows.push_back(ProbRows{pid, r0});
+      part += (int64_t)nt * nt * kPiTile;
     }
     if (w == 0) {
-      p.n_pi_rows_one = (int)p.pi_rows.size();
+      p.n_pi_tiles_one = (int)p.pi_tiles.size();
+      p.n_pi_slices_one = (int)p.pi_slices.size();
       p.u_elems_one = u;
     }
   }
+  p.part_elems = part;
   p.u_elems = u;
   const int64_t esz = p.fp32 ? 4 : 2;
   int64_t bytes = 0;
@@ -209,6 +225,9 @@ int make_plan(const int64_t* shapes, int n_mats, int M, int K, int scale, int P,
     bytes += (int64_t)p.chunks.size() * M * 4;            // norm partials
     bytes += (int64_t)M * n_mats * (4 + 8 + 8);           // scales, coefficients
     bytes += 2 * p.u_elems * 4;                           // power-iteration vectors
+    bytes += p.part_elems * 4;                            // power-iteration partial sums
+    bytes += (int64_t)p.pi_slices.size() * 8;             // per-slice figures
+    bytes += (int64_t)M * n_mats * 8;                     // per-problem counters, 1/||y||
     if (flags & SIGNMUON_PI_WARM) bytes += p.u_elems_one * 4;  // warm state of one problem set
     bytes += (int64_t)p.groups.size() * 8 * 128;          // tensor maps
   }

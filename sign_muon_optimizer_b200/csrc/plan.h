@@ -1,5 +1,5 @@
 // plan.h -- host-side planning of one Sign-Muon handle: shape groups, chunk
-// lists, grouped GEMM tile lists, power-iteration row blocks and buffer
+// lists, grouped GEMM tile lists, power-iteration tiles and buffer
 // sizes.  Pure host code (no CUDA calls), so that it can be checked without a
 // GPU through signmuon_plan().
 #pragma once
@@ -29,14 +29,20 @@ struct Plan {
   std::vector<int64_t> mat_off;
   std::vector<Chunk> chunks;
   std::vector<int> mat_chunk0, mat_nchunks;
+  std::vector<int64_t> stage_off;  // per chunk: flat offset, offset in a one-problem-set X
   int64_t x_elems = 0;  // elements of one grouped X buffer (all workers)
   int64_t a_elems = 0;  // elements of the grouped A (and B) buffer
   // tile lists: [op][0 = all M workers, 1 = one worker]
   TileTable tiles[3][2];
   // power iteration: problems p = worker*n_mats + mat (worker-major)
-  std::vector<ProbRows> pi_rows;
-  int n_pi_rows_one = 0;  // rows blocks of worker 0 (prefix)
+  std::vector<PiTile> pi_tiles;    // the 128 x 128 tiles on and above each Gram's diagonal
+  std::vector<PiSlice> pi_slices;  // 128-row slices of every problem
+  int n_pi_tiles_one = 0;          // tiles of worker 0's problems (prefix)
+  int n_pi_slices_one = 0;         // slices of worker 0's problems (prefix)
+  std::vector<int> soff;           // first slice of each problem
   std::vector<int64_t> uoff;
+  std::vector<int64_t> poff;       // partial-sum offsets (nt^2 * 128 entries per problem)
+  int64_t part_elems = 0;
   std::vector<int> prob_g, prob_gld;
   std::vector<int64_t> prob_aoff;
   int64_t u_elems = 0;

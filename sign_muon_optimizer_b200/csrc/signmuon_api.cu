@@ -54,8 +54,10 @@ struct signmuon_ctx {
   sm::Chunk* d_chunks = nullptr;
   int* d_mat_chunk0 = nullptr;
   int* d_mat_nchunks = nullptr;
+  int64_t* d_stage_off = nullptr;
   sm::TileGroup* d_tiles[3][2] = {{nullptr}};
-  sm::ProbRows* d_pi_rows = nullptr;
+  sm::PiTile* d_pi_tiles = nullptr;
+  sm::PiSlice* d_pi_slices = nullptr;
   int64_t* d_uoff = nullptr;
   int* d_prob_g = nullptr;
   int* d_prob_gld = nullptr;
@@ -77,6 +79,10 @@ struct signmuon_ctx {
   float* pi_u = nullptr;        // power-iteration iterates of the M-worker problems (warm state)
   float* pi_u1 = nullptr;       // PI_WARM: iterates of the one-problem-set PolarNS (warm state)
   float* pi_y = nullptr;
+  float* pi_part = nullptr;     // per-tile partial sums of A v
+  float* pi_inv = nullptr;      // per-problem 1/||y|| between passes
+  double* pi_sq = nullptr;      // per-slice ||y||^2 or u.y
+  int* pi_cnt = nullptr;        // per-problem slice counters (zero between launches)
   int* status = nullptr;        // [0] non-finite flag, [1] kernel error code
   int* h_status = nullptr;      // pinned mirror
   bool pending = false;         // an async step's status not yet read
@@ -329,22 +335,24 @@ void gemm(signmuon_t h, int op, int slot, int src, int nw, const float2* coef, f
 void power_iteration(signmuon_t h, int nw) {
   const Plan& p = h->plan;
   const int nprob = nw * p.n_mats;
-  const int nrows = nw == 1 ? p.n_pi_rows_one : (int)p.pi_rows.size();
+  const int ntiles = nw == 1 ? p.n_pi_tiles_one : (int)p.pi_tiles.size();
   const bool warm = (h->flags & SIGNMUON_PI_WARM) != 0;
   float* u = (warm && nw == 1) ? h->pi_u1 : h->pi_u;
+  const int bf16 = p.fp32 ? 0 : 1;
   ProfScope ps(h, 5);
-  int max_g = 1;
-  for (const sm::GroupInfo& gi : p.groups) max_g = gi.g > max_g ? gi.g : max_g;
+  const int nslices = nw == 1 ? p.n_pi_slices_one : (int)p.pi_slices.size();
+  const sm::PiReduce mid{0, u, h->pi_sq, h->pi_cnt, h->pi_inv, h->eps, p.quintic ? 1 : 0, h->ns_a, h->ns_b,
+                         h->ns_c, h->scale_v, h->coef_apply, h->coef_square, h->status};
+  sm::PiReduce fin = mid;
+  fin.last = 1;
+  // u0; then y = A u0; then P times y = A (y / ||y||), storing y / ||y|| as u
   sm::launch_pi_init(h->stream, nprob, h->d_uoff, h->d_prob_g, u, warm ? 1 : 0);
+  sm::launch_pi_tiles(h->stream, h->d_pi_tiles, ntiles, h->A, bf16, u, nullptr, u, h->pi_part, 0);
   for (int it = 0; it < h->P; ++it) {
-    sm::launch_pi_matvec(h->stream, h->d_pi_rows, nrows, h->A, p.fp32 ? 0 : 1, h->d_prob_aoff, h->d_prob_g,
-                         h->d_prob_gld, h->d_uoff, u, h->pi_y, max_g);
-    sm::launch_pi_normalize(h->stream, nprob, h->d_uoff, h->d_prob_g, h->pi_y, u);
+    sm::launch_pi_reduce(h->stream, h->d_pi_slices, nslices, h->pi_part, h->pi_y, mid);
+    sm::launch_pi_tiles(h->stream, h->d_pi_tiles, ntiles, h->A, bf16, h->pi_y, h->pi_inv, u, h->pi_part, 1);
   }
-  sm::launch_pi_matvec(h->stream, h->d_pi_rows, nrows, h->A, p.fp32 ? 0 : 1, h->d_prob_aoff, h->d_prob_g,
-                       h->d_prob_gld, h->d_uoff, u, h->pi_y, max_g);
-  sm::launch_pi_finalize(h->stream, nprob, h->d_uoff, h->d_prob_g, u, h->pi_y, h->eps, p.quintic ? 1 : 0,
-                         h->ns_a, h->ns_b, h->ns_c, h->scale_v, h->coef_apply, h->coef_square, h->status);
+  sm::launch_pi_reduce(h->stream, h->d_pi_slices, nslices, h->pi_part, h->pi_y, fin);
 }
 
 // The streaming vote kernel stages the post-vote input when every matrix
@@ -539,7 +547,9 @@ int signmuon_plan_tables(const int64_t* shapes, int n_mats, int M, int K, int sc
   const std::pair<const char*, int64_t> scalars[] = {
       {"d", p.d}, {"dpad", p.dpad}, {"nb", p.nb}, {"nb_pad", p.nb_pad}, {"x_elems", p.x_elems},
       {"a_elems", p.a_elems}, {"u_elems", p.u_elems}, {"u_elems_one", p.u_elems_one},
-      {"n_pi_rows_one", p.n_pi_rows_one}, {"M", p.M}, {"n_mats", p.n_mats}, {"fp32", p.fp32 ? 1 : 0},
+      {"n_pi_tiles_one", p.n_pi_tiles_one},
+      {"n_pi_slices", (int64_t)p.pi_slices.size()}, {"n_pi_slices_one", p.n_pi_slices_one},
+      {"part_elems", p.part_elems}, {"M", p.M}, {"n_mats", p.n_mats}, {"fp32", p.fp32 ? 1 : 0},
       {"quintic", p.quintic ? 1 : 0}, {"device_bytes", p.device_bytes}};
   for (const auto& kv : scalars) {
     j += '"';
@@ -575,8 +585,13 @@ int signmuon_plan_tables(const int64_t* shapes, int n_mats, int M, int K, int sc
     }
     j += "]}";
   });
-  list("pi_rows", p.pi_rows.size(), [&](size_t i) { tuple({p.pi_rows[i].p, p.pi_rows[i].row0}); });
+  list("pi_tiles", p.pi_tiles.size(), [&](size_t i) {
+    const sm::PiTile& t = p.pi_tiles[i];
+    tuple({t.p, t.bi, t.bj, t.aoff, t.uoff, t.poff, t.g, t.gld, t.soff});
+  });
   list("uoff", p.uoff.size(), [&](size_t i) { num(p.uoff[i]); });
+  list("poff", p.poff.size(), [&](size_t i) { num(p.poff[i]); });
+  list("soff", p.soff.size(), [&](size_t i) { num(p.soff[i]); });
   list("prob_g", p.prob_g.size(), [&](size_t i) { num(p.prob_g[i]); });
   list("prob_gld", p.prob_gld.size(), [&](size_t i) { num(p.prob_gld[i]); });
   list("prob_aoff", p.prob_aoff.size(), [&](size_t i) { num(p.prob_aoff[i]); });
@@ -647,10 +662,12 @@ int signmuon_init(signmuon_t* out, const int64_t* shapes, int n_mats, int M, flo
   if ((rc = upload(h, &h->d_chunks, p.chunks))) return bail(rc);
   if ((rc = upload(h, &h->d_mat_chunk0, p.mat_chunk0))) return bail(rc);
   if ((rc = upload(h, &h->d_mat_nchunks, p.mat_nchunks))) return bail(rc);
+  if ((rc = upload(h, &h->d_stage_off, p.stage_off))) return bail(rc);
   for (int op = 0; op < 3; ++op)
     for (int s = 0; s < 2; ++s)
       if ((rc = upload(h, &h->d_tiles[op][s], p.tiles[op][s].groups))) return bail(rc);
-  if ((rc = upload(h, &h->d_pi_rows, p.pi_rows))) return bail(rc);
+  if ((rc = upload(h, &h->d_pi_tiles, p.pi_tiles))) return bail(rc);
+  if ((rc = upload(h, &h->d_pi_slices, p.pi_slices))) return bail(rc);
   if ((rc = upload(h, &h->d_uoff, p.uoff))) return bail(rc);
   if ((rc = upload(h, &h->d_prob_g, p.prob_g))) return bail(rc);
   if ((rc = upload(h, &h->d_prob_gld, p.prob_gld))) return bail(rc);
@@ -686,6 +703,12 @@ int signmuon_init(signmuon_t* out, const int64_t* shapes, int n_mats, int M, flo
   if ((rc = dalloc(h, &h->coef_square, (int64_t)M * p.n_mats))) return bail(rc);
   if ((rc = dalloc(h, &h->pi_u, p.u_elems))) return bail(rc);
   if ((rc = dalloc(h, &h->pi_y, p.u_elems))) return bail(rc);
+  if ((rc = dalloc(h, &h->pi_part, p.part_elems))) return bail(rc);
+  if ((rc = dalloc(h, &h->pi_cnt, (int64_t)M * p.n_mats))) return bail(rc);
+  if ((rc = dalloc(h, &h->pi_inv, (int64_t)M * p.n_mats))) return bail(rc);
+  if ((rc = dalloc(h, &h->pi_sq, (int64_t)p.pi_slices.size()))) return bail(rc);
+  if (cudaMemset(h->pi_cnt, 0, (size_t)M * p.n_mats * sizeof(int)) != cudaSuccess)
+    return bail(fail(h, SIGNMUON_E_CUDA, "memset"));
   if (flags & SIGNMUON_PI_WARM) {
     // zero state: the first power iteration of every problem starts cold
     if ((rc = dalloc(h, &h->pi_u1, p.u_elems_one))) return bail(rc);
@@ -818,7 +841,7 @@ static void vote_part(signmuon_t h, float* W, const sm::WorkerPtrs& src, int Mv,
         // when K == 0, where the result is the scaled input itself)
         sm::launch_vote_stage(s, src, Mv, h->X[0], p.fp32 ? 0 : 1, h->d_chunks, (int)p.chunks.size(),
                               h->d_mats, h->d_groups, h->partials, k_post == 0 ? h->D : nullptr, tie,
-                              stage_streamable(h) ? 1 : 0);
+                              stage_streamable(h) ? h->d_stage_off : nullptr);
       }
     }
     fro_finalize(h, 1);

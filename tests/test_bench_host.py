@@ -85,7 +85,9 @@ def test_hbm_bytes_counts():
     assert b["momentum"] == d * 116          # W once + 8 x (G + Mom r/w + bf16 X)
     assert b["pack"] == d * 8 * 4.125        # fp32 U read + one bit written per worker
     assert b["vote"] == d + 2 * d            # 8 bits per entry read, bf16 X written
-    assert b["power_iter"] == 3 * 9 * 48 * 768 * 768 * 2
+    # 3 passes (P = 2), 8 workers + the post-vote set, 48 Grams of side 768:
+    # the bf16 entries on and above the diagonal of the symmetric Gram
+    assert b["power_iter"] == 3 * 9 * 48 * (768 * 769 // 2) * 2
 
 
 def test_cpu_sample_is_one_144th():

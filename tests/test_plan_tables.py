@@ -119,13 +119,26 @@ def _check(shapes, M, flags, spectral):
         grp = groups[mat[3]]
         assert aoff == grp[9] + (w * grp[6] + mat[4]) * grp[3] * grp[4]
         assert t["prob_gld"][p] == grp[4]
-    rows_of = {}
-    for k, (p, r0) in enumerate(t["pi_rows"]):
-        rows_of.setdefault(p, []).append(r0)
-        if k < t["n_pi_rows_one"]:
-            assert p < n                           # worker 0's blocks come first
+    # symmetric power iteration: the 128 x 128 tiles on and above each Gram's
+    # diagonal, each once and carrying its problem's offsets (one table load
+    # per block); 128-row slices numbered per problem from soff; partial-sum
+    # slots (nt x nt x 128 per problem) disjoint
+    tiles_of = {}
+    for k, (p, bi, bj, aoff, uoff, poff, g, gld, soff) in enumerate(t["pi_tiles"]):
+        tiles_of.setdefault(p, []).append((bi, bj))
+        assert (k < t["n_pi_tiles_one"]) == (p < n)        # worker 0's tiles come first
+        assert (aoff, uoff, poff, g, gld, soff) == (t["prob_aoff"][p], t["uoff"][p], t["poff"][p],
+                                                    t["prob_g"][p], t["prob_gld"][p], t["soff"][p])
+    spans, slices = [], []
     for p in range(M * n):
-        assert rows_of[p] == list(range(0, t["prob_g"][p], 32))
+        nt = _ceil(t["prob_g"][p], 128)
+        assert sorted(tiles_of[p]) == [(i, j) for i in range(nt) for j in range(i, nt)]
+        spans.append((t["poff"][p], t["poff"][p] + nt * nt * 128))
+        slices.append((t["soff"][p], t["soff"][p] + nt))
+    _disjoint_inside(slices, t["n_pi_slices"])
+    assert sum(e - s for s, e in slices) == t["n_pi_slices"]
+    _disjoint_inside(spans, t["part_elems"])
+    assert t["part_elems"] == sum(_ceil(g, 128) ** 2 * 128 for g in t["prob_g"])
 
 
 shape = st.tuples(st.integers(1, 300), st.integers(1, 300))
