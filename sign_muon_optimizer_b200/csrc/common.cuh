@@ -57,7 +57,7 @@ struct PiTile {       // one upper-triangle tile of one problem: all that its bl
   int p;              // problem id (worker*n_mats + mat)
   int g, gld;         // Gram side and row stride
   int bi, bj;         // row and column slice, bi <= bj
-  int soff;           // index of the problem's first slice
+  int pad;
 };
 struct PiSlice {      // one 128-row slice of one problem's iterate
   int64_t uoff;

@@ -200,7 +200,7 @@ int make_plan(const int64_t* shapes, int n_mats, int M, int K, int scale, int P,
       for (int bi = 0; bi < nt; ++bi) {
         p.pi_slices.push_back(PiSlice{u, part, pid, g.g, bi, soff});
         for (int bj = bi; bj < nt; ++bj)
-          p.pi_tiles.push_back(PiTile{p.prob_aoff.back(), u, part, pid, g.g, g.gld, bi, bj, soff});
+          p.pi_tiles.push_back(PiTile{p.prob_aoff.back(), u, part, pid, g.g, g.gld, bi, bj, 0});
       }
       u += g.g;
       part += (int64_t)nt * nt * kPiTile;

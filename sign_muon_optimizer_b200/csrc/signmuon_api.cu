@@ -587,7 +587,11 @@ int signmuon_plan_tables(const int64_t* shapes, int n_mats, int M, int K, int sc
   });
   list("pi_tiles", p.pi_tiles.size(), [&](size_t i) {
     const sm::PiTile& t = p.pi_tiles[i];
-    tuple({t.p, t.bi, t.bj, t.aoff, t.uoff, t.poff, t.g, t.gld, t.soff});
+    tuple({t.p, t.bi, t.bj, t.aoff, t.uoff, t.poff, t.g, t.gld});
+  });
+  list("pi_slices", p.pi_slices.size(), [&](size_t i) {
+    const sm::PiSlice& t = p.pi_slices[i];
+    tuple({t.p, t.bi, t.uoff, t.poff, t.g, t.soff});
   });
   list("uoff", p.uoff.size(), [&](size_t i) { num(p.uoff[i]); });
   list("poff", p.poff.size(), [&](size_t i) { num(p.poff[i]); });

@@ -123,20 +123,24 @@ def _check(shapes, M, flags, spectral):
     # diagonal, each once and carrying its problem's offsets (one table load
     # per block); 128-row slices numbered per problem from soff; partial-sum
     # slots (nt x nt x 128 per problem) disjoint
-    tiles_of = {}
-    for k, (p, bi, bj, aoff, uoff, poff, g, gld, soff) in enumerate(t["pi_tiles"]):
+    tiles_of, slices_of = {}, {}
+    for k, (p, bi, bj, aoff, uoff, poff, g, gld) in enumerate(t["pi_tiles"]):
         tiles_of.setdefault(p, []).append((bi, bj))
         assert (k < t["n_pi_tiles_one"]) == (p < n)        # worker 0's tiles come first
-        assert (aoff, uoff, poff, g, gld, soff) == (t["prob_aoff"][p], t["uoff"][p], t["poff"][p],
-                                                    t["prob_g"][p], t["prob_gld"][p], t["soff"][p])
-    spans, slices = [], []
+        assert (aoff, uoff, poff, g, gld) == (t["prob_aoff"][p], t["uoff"][p], t["poff"][p],
+                                              t["prob_g"][p], t["prob_gld"][p])
+    for k, (p, bi, uoff, poff, g, soff) in enumerate(t["pi_slices"]):
+        slices_of.setdefault(p, []).append(bi)
+        assert (k < t["n_pi_slices_one"]) == (p < n)       # and its slices
+        assert (uoff, poff, g, soff) == (t["uoff"][p], t["poff"][p], t["prob_g"][p], t["soff"][p])
+        assert k == soff + bi                              # a problem's slices are contiguous
+    spans = []
     for p in range(M * n):
         nt = _ceil(t["prob_g"][p], 128)
         assert sorted(tiles_of[p]) == [(i, j) for i in range(nt) for j in range(i, nt)]
+        assert slices_of[p] == list(range(nt))
         spans.append((t["poff"][p], t["poff"][p] + nt * nt * 128))
-        slices.append((t["soff"][p], t["soff"][p] + nt))
-    _disjoint_inside(slices, t["n_pi_slices"])
-    assert sum(e - s for s, e in slices) == t["n_pi_slices"]
+    assert t["n_pi_slices"] == len(t["pi_slices"])
     _disjoint_inside(spans, t["part_elems"])
     assert t["part_elems"] == sum(_ceil(g, 128) ** 2 * 128 for g in t["prob_g"])
 
