@@ -210,13 +210,14 @@ k_fro_finalize(int n_mats, int M, const float* __restrict__ partials, const int*
 // and A_IJ^T v_I to y_J (its column sums), a diagonal tile A_II v_I.  A block
 // takes one tile; each contribution has its own slot in a partial-sum buffer
 // (slot K of slice I comes from the tile that pairs slices I and K), and
-// k_pi_reduce adds the slots of a slice in slot order, so the result does not
-// depend on the schedule.  A diagonal tile reads its upper triangle only (its rows give
-// the entries on and above the diagonal, its columns the ones above), so a
-// pass reads about g (g + 1) / 2 of the g^2 entries.  The normalisation of
-// an iterate is folded into the passes: the reduction's last block per
-// problem forms 1/||y||, and the next pass scales y by it while staging it;
-// after the last pass it forms sigma^2 = u^T y and the scale instead.
+// k_pi_reduce adds the slots of a slice in slot order, so the result does
+// not depend on the schedule.  A diagonal tile reads its upper triangle only
+// (its rows give the entries on and above the diagonal, its columns the ones
+// above), so a pass reads about g (g + 1) / 2 of the g^2 entries.  The
+// normalisation of an iterate is folded into the passes: the reduction's
+// last block per problem forms 1/||y||, and the next pass scales y by it
+// while staging it; after the last pass it forms sigma^2 = u^T y and the
+// scale instead.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kThreads)
 k_pi_init(const int64_t* __restrict__ uoff, const int* __restrict__ prob_g, float* __restrict__ u, int warm) {
