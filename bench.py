@@ -78,6 +78,18 @@ def ns_flops_per_step(shapes, M, K, post_polar):
     return per_worker * (M + (1 if post_polar else 0))
 
 
+def ns_kind_flops(shapes, nw, K, gram_ns):
+    """Algorithmic flops of each Newton-Schulz GEMM kind for nw problem sets
+    (cubic), as the handle runs them.  On X: K x (Gram X X^T, 2 m^2 n;
+    apply A X, 2 m^2 n).  In Gram space: one Gram, 3K - 3 products of m x m
+    matrices (2 m^3 each) and one apply (2 m^2 n)."""
+    mn = sum(2.0 * min(r, c) ** 2 * max(r, c) for r, c in shapes) * nw
+    mmm = sum(2.0 * min(r, c) ** 3 for r, c in shapes) * nw
+    if gram_ns:
+        return {"gram": mn, "square": (3 * K - 3) * mmm, "apply": mn}
+    return {"gram": K * mn, "square": 0.0, "apply": K * mn}
+
+
 def gram_sym_bytes(shapes):
     """bf16 bytes of the entries on and above each Gram's diagonal: what a
     pass of the power iteration must read of the symmetric Gram."""
@@ -304,7 +316,8 @@ def measure_resnet50(smo, stream, pk, steps=20):
         h.step(W, gl, HP["eta"])
     prof = h.profile_read()
     h.profile(False)
-    fl = ns_flops_per_step(shp, Mr, wl["K"], False)
+    gram_ns = bool(smo.signmuon_plan_tables(shp, Mr, wl["K"], wl["scale"], wl["P"], 0)["gram_ns"])
+    fl = sum(ns_kind_flops(shp, Mr, wl["K"], gram_ns).values())
     gemm_ms = sum(prof[k][0] for k in ("ns_gram", "ns_square", "ns_apply")) / steps
     tf = fl / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else None
     h.close()
@@ -312,7 +325,7 @@ def measure_resnet50(smo, stream, pk, steps=20):
     torch.cuda.empty_cache()
     return {"metric": "Sign-Muon steps/s (ResNet-50 shapes, M=4, K=5 cubic bf16, spectral P=2)",
             "value": 1e3 / ms, "unit": "steps/s", "ms_per_step": ms, "d": synth.numel(shp),
-            "ns_tflops_per_step": fl / 1e12, "ns_ms_per_step": gemm_ms,
+            "ns_tflops_per_step": fl / 1e12, "ns_ms_per_step": gemm_ms, "ns_form": "gram space" if gram_ns else "x space",
             "ns_TFLOP/s": tf, "ns_frac_of_bf16_burst": (tf / pk["bf16_tflops"]) if tf else None,
             "ns_share_of_step": gemm_ms / ms}
 
@@ -425,12 +438,16 @@ def measure_ns_sweep(smo, stream, pk, grid=SWEEP_GRID):
             xs, us = [X[m] for m in range(Mw)], [U[m] for m in range(Mw)]
             reps, warm = (3, 1) if prec == "bf16" else (1, 1)
             ms = _events_time(lambda: h.polar(xs, us), reps, stream, warm=warm)
-            per_it = sum(4.0 * min(r, c) ** 2 * max(r, c) + (2.0 * min(r, c) ** 3 if order == "quintic" else 0.0)
-                         for r, c in shp)
-            fl = per_it * K * Mw
+            gram_ns = bool(smo.signmuon_plan_tables(shp, Mw, K, "spectral", 2, fl_ns)["gram_ns"])
+            if gram_ns:
+                fl = sum(ns_kind_flops(shp, Mw, K, True).values())
+            else:
+                per_it = sum(4.0 * min(r, c) ** 2 * max(r, c) + (2.0 * min(r, c) ** 3 if order == "quintic" else 0.0)
+                             for r, c in shp)
+                fl = per_it * K * Mw
             tf = fl / (ms / 1e3) / 1e12
             e = {"shape": name, "K": K, "order": order, "precision": prec, "M": Mw, "TFLOP/s": tf, "ms": ms,
-                 "flops": fl}
+                 "flops": fl, "ns_form": "gram space" if gram_ns else "x space"}
             if prec == "bf16":
                 e["frac_of_bf16_burst"] = tf / pk["bf16_tflops"]
             else:
@@ -508,7 +525,11 @@ def run_ours(args):
 
     pk, pk_kind = peaks()
     steps = args.steps
-    flops = ns_flops_per_step(SHAPES, M, K_NS, WL["post_polar"])
+    gram_ns = bool(smo.signmuon_plan_tables(SHAPES, M, K_NS, WL["scale"], WL["P"], flags)["gram_ns"])
+    kind_fl = {"ns_" + k: v for k, v in ns_kind_flops(SHAPES, M, K_NS, gram_ns).items()}
+    if WL["post_polar"]:
+        kind_fl.update({"post_" + k: v for k, v in ns_kind_flops(SHAPES, 1, K_NS, gram_ns).items()})
+    flops = sum(kind_fl.values())                 # as run: X space or Gram space
     gemm_kinds = ["ns_gram", "ns_square", "ns_apply", "post_gram", "post_square", "post_apply"]
     gemm_ms = sum(prof[k][0] for k in gemm_kinds)
     gemm_launches = sum(prof[k][1] for k in gemm_kinds)
@@ -531,11 +552,9 @@ def run_ours(args):
             continue
         e = {"ms_per_step": kms / steps, "launches_per_step": n / steps}
         if kind in gemm_kinds:
-            # cubic: the Gram and the apply GEMM each do half of the 4 m^2 n flops
-            f = 0.5 * ns_flops_per_step(SHAPES, 0 if kind.startswith("post") else M, K_NS,
-                                        kind.startswith("post"))
-            e["TFLOP/s"] = f / (kms / steps / 1e3) / 1e12
-            e["frac_of_bf16_burst"] = e["TFLOP/s"] / peak_tc
+            if kind_fl.get(kind):
+                e["TFLOP/s"] = kind_fl[kind] / (kms / steps / 1e3) / 1e12
+                e["frac_of_bf16_burst"] = e["TFLOP/s"] / peak_tc
         elif kind in hbm:
             e["GB/s"] = hbm[kind] / (kms / steps / 1e3) / 1e9
             e["frac_of_hbm"] = e["GB/s"] / pk["hbm_gbs"]
@@ -612,6 +631,10 @@ def run_ours(args):
             "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches, "clocks": clocks,
             "ns_tflops_per_step": flops / 1e12,
+            # the Newton-Schulz form the planner chose, and the flops the same
+            # iteration would take on X (context for the Gram-space form)
+            "ns_form": "gram space" if gram_ns else "x space",
+            "ns_tflops_per_step_on_x": ns_flops_per_step(SHAPES, M, K_NS, WL["post_polar"]) / 1e12,
             "workloads": extras,
         }
         print(json.dumps(line), flush=True)
@@ -678,7 +701,8 @@ def run_secondary(args):
                     ("normalized_sign", smo.SIGNMUON_NORMALIZED_SIGN, WL["P"]),
                     ("after_only", smo.SIGNMUON_POST_POLAR | smo.SIGNMUON_POLAR_AFTER_ONLY, WL["P"]),
                     ("muon_mean", smo.SIGNMUON_MUON_MEAN, WL["P"]),
-                    ("pi_warm_P1", base | smo.SIGNMUON_PI_WARM, 1), ("cold_P1", base, 1), ("split", base, WL["P"])]
+                    ("pi_warm_P1", base | smo.SIGNMUON_PI_WARM, 1), ("cold_P1", base, 1), ("split", base, WL["P"]),
+                    ("gram_space_ns", base | smo.SIGNMUON_NS_GRAM, WL["P"])]
         W = synth.device_weights0(SHAPES, config_id=7)
         G = synth.device_gradients(SHAPES, M, WL["sigma"], step=0, config_id=7)
         gl = [G[m] for m in range(M)]

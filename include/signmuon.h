@@ -96,6 +96,16 @@ typedef struct signmuon_ctx* signmuon_t;
 #define SIGNMUON_TERNARY           (1u << 10)
 #define SIGNMUON_NORMALIZED_SIGN   (1u << 11)
 #define SIGNMUON_PI_WARM           (1u << 12)
+/* NS_GRAM: run the bf16 cubic Newton-Schulz iteration in Gram space when that
+ * needs at least 15 % fewer tensor-core flops (every matrix with m >= 256, n
+ * well above m, K >= 2): A0 = X0 X0^T, then per iteration the m x m products
+ * A_{k+1} = P_k A_k P_k and Q_{k+1} = P_k Q_k with P_k = a I + b A_k (all
+ * polynomials in A0, so they commute), and one final X_K = Q_K X0.  In exact
+ * arithmetic both give the same X_K.  In bf16 the Gram-space iterates carry the
+ * squared spectrum and the iteration does not correct its own rounding: the
+ * polar error stays within 1.2x of the iteration on X, but the signs of the
+ * smallest entries flip several times more often, so the default iterates on X. */
+#define SIGNMUON_NS_GRAM           (1u << 13)
 
 /* ------------------------------------------------------------------------
  * signmuon_init -- plan the step and allocate its device state.
@@ -331,8 +341,10 @@ int signmuon_get_scales(signmuon_t h, float* dst_host);
  * matrix `mat`: X X^T of the wide orientation; after one iteration it is the
  * unscaled Gram of the staged momentum (waits for the GPU).  On the bf16 path
  * with the cubic polynomial, iterations after the first store the apply's
- * whole operator a I + b X X^T there instead (the a X term folded into it).
- * After a post-vote step, worker 0's slot holds the post-vote step's. */
+ * whole operator a I + b X X^T there instead (the a X term folded into it);
+ * a handle that iterates in Gram space (SIGNMUON_NS_GRAM)
+ * leaves one of the iteration's m x m iterates A_k there.  After a post-vote
+ * step, worker 0's slot holds the post-vote step's. */
 int signmuon_get_gram(signmuon_t h, int m, int mat, float* dst_host);
 
 /* Newton-Schulz coefficients: n=2 (a, b) for X <- aX + b(XX^T)X ([paper] §3

@@ -42,6 +42,7 @@ SIGNMUON_MUON_MEAN = 1 << 9
 SIGNMUON_TERNARY = 1 << 10
 SIGNMUON_NORMALIZED_SIGN = 1 << 11
 SIGNMUON_PI_WARM = 1 << 12
+SIGNMUON_NS_GRAM = 1 << 13
 
 EXPORTED = [
     "signmuon_init", "signmuon_step", "signmuon_step_host", "signmuon_vote", "signmuon_pack",

@@ -78,6 +78,7 @@ struct PiReduce {     // what k_pi_reduce writes besides y
   float* scale;
   float2* coef_apply;
   float2* coef_square;
+  float2* coef_gram;  // Gram-space start (null when the handle iterates on X)
   int* status;
 };
 
@@ -103,9 +104,19 @@ enum GemmOp { OP_GRAM = 0, OP_SQUARE = 1, OP_APPLY = 2 };
 // memory is a chain of dependent loads).
 constexpr int kParamGroups = 24;
 // TMA tensor maps per shape group (bf16 path): X ping/pong, A, B with 64-row
-// and 128-row boxes, X ping/pong as 4-D atom views with two-atom operand
-// boxes, and X ping/pong, A, B with 32-row boxes (an epilogue warp's atom).
-constexpr int kMapsPerGroup = 14;
+// and 128-row boxes (slots 0..3, 4..7), X ping/pong as 4-D atom views with
+// two-atom operand boxes (8, 9), and X ping/pong, A, B with 32-row boxes (an
+// epilogue warp's atom; 10..13); then the m x m buffers of the Gram-space
+// iteration, A2, Q0 and Q1, each with 64-, 128- and 32-row boxes (14..22).
+constexpr int kMapsPerGroup = 23;
+// m x m bf16 buffers addressed by index: 0 = A, 1 = B, 2 = A2, 3 = Q0, 4 = Q1
+enum MmBuf { MM_A = 0, MM_B = 1, MM_A2 = 2, MM_Q0 = 3, MM_Q1 = 4 };
+// tensor-map slot of m x m buffer `buf` with 64- (box 0), 128- (box 1) or
+// 32-row (box 2) boxes
+__host__ __device__ __forceinline__ int mm_slot(int buf, int box) {
+  if (buf <= MM_B) return box == 0 ? 2 + buf : (box == 1 ? 6 + buf : 12 + buf);
+  return 14 + 3 * (buf - MM_A2) + box;
+}
 constexpr int kParamMats = 64;
 
 // Arguments of one grouped Newton-Schulz GEMM launch (both precisions).
@@ -122,11 +133,18 @@ struct GemmArgs {
   void* X_dst;               // X buffer written by a non-final APPLY
   void* A;                   // Gram buffer
   void* B;                   // quintic polynomial buffer
-  int p_from_b;              // APPLY multiplies by B (quintic) instead of A
+  int p_from_b;              // APPLY multiplies by B (quintic) instead of A (fp32 path)
+  // bf16 path: APPLY's operator is m x m buffer p_buf; SQUARE computes
+  // L R^T (= L R, both symmetric) with L = buffer sq_l and R = buffer sq_r,
+  // its affine operand is R, and it writes sq_out (an m x m buffer)
+  int p_buf;
+  int sq_l, sq_r;
+  void* sq_out;
+  int sym_exact;             // symmetric outputs stored exactly symmetric (diagonal tiles too)
   int map_src, map_dst;      // tensor-map slots of X_src / X_dst (TMA path)
   // epilogue coefficients: per-problem float2 when coef is non-null, else (c0, c1).
   //   GRAM:   out = c1 acc + cdiag [row == col]
-  //   SQUARE: out = c0 A + c1 acc + cdiag [row == col]
+  //   SQUARE: out = c0 R + c1 acc + cdiag [row == col]  (R = A on the fp32 path)
   //   APPLY:  out = c0 X + c1 acc, or (plain) out = acc
   const float2* coef;
   float c0, c1;
@@ -194,7 +212,10 @@ void launch_stage(cudaStream_t s, const WorkerPtrs& in, int M, void* X, int x_bf
 void launch_fro_finalize(cudaStream_t s, int n_probs, int n_mats, int M, const float* partials,
                          const int* mat_chunk0, const int* mat_nchunks, int use_for_scale,
                          float eps, int quintic, float a, float b, float c, float* scale,
-                         float2* coef_apply, float2* coef_square, int* status);
+                         float2* coef_apply, float2* coef_square, float2* coef_gram, int* status);
+// Gram space: Q1 = coef[p].x I + coef[p].y A per problem (bf16 m x m buffers)
+void launch_gram_q1(cudaStream_t s, int n_probs, const void* A, void* Q, const int64_t* prob_aoff,
+                    const int* prob_g, const int* prob_gld, const float2* coef, int max_g, int max_gld);
 // warm != 0: keep each problem's stored iterate when it is non-zero and finite
 void launch_pi_init(cudaStream_t s, int n_probs, const int64_t* uoff, const int* prob_g, float* u, int warm);
 // one pass over the upper-triangle tiles, one block per tile: partial sums

@@ -8,6 +8,7 @@
 //   [blog]  "SignMuon: Matrix Directions, Majority Votes, and the Actual Bytes Sent"
 #include "common.cuh"
 
+#include <algorithm>
 #include <cmath>
 #include <map>
 #include <mutex>
@@ -159,12 +160,19 @@ k_momentum(WorkerPtrs G, const float* __restrict__ W, float* __restrict__ Mom, i
 }
 
 __device__ __forceinline__ void set_coefs(int p, float cc, int quintic, float a, float b, float c,
-                                          float2* coef_apply, float2* coef_square) {
+                                          float2* coef_apply, float2* coef_square, float2* coef_gram) {
   // Iteration 0 runs on the unscaled X~ and Gram A~ = X~ X~^T.  With X0 = cc X~:
   //   cubic:   X1 = a cc X~ + b cc^3 A~ X~
   //   quintic: B = b cc^2 A~ + c cc^4 A~^2;  X1 = cc (a X~ + B X~)
+  // and in Gram space (cubic, A0 = cc^2 A~): Q1 = a cc I + b cc^3 A~ (the
+  // apply coefficients), T0 = a cc^2 A~ + b cc^4 A~^2 (coef_square), and
+  // A1 = a T0 + b cc^2 A~ T0 (coef_gram)
   if (!quintic) {
     coef_apply[p] = make_float2(a * cc, b * cc * cc * cc);
+    if (coef_gram != nullptr) {
+      coef_square[p] = make_float2(a * cc * cc, b * cc * cc * cc * cc);
+      coef_gram[p] = make_float2(a, b * cc * cc);
+    }
   } else {
     coef_square[p] = make_float2(b * cc * cc, c * cc * cc * cc * cc);
     coef_apply[p] = make_float2(a * cc, cc);
@@ -176,7 +184,7 @@ __global__ void __launch_bounds__(kThreads)
 k_fro_finalize(int n_mats, int M, const float* __restrict__ partials, const int* __restrict__ mat_chunk0,
                const int* __restrict__ mat_nchunks, int use_for_scale, float eps, int quintic,
                float a, float b, float c, float* __restrict__ scale, float2* coef_apply,
-               float2* coef_square, int* status) {
+               float2* coef_square, float2* coef_gram, int* status) {
   griddep_wait();
   griddep_launch();
   __shared__ double red[32];
@@ -191,7 +199,7 @@ k_fro_finalize(int n_mats, int M, const float* __restrict__ partials, const int*
     if (use_for_scale) {
       const float sc = (float)sqrt(t);
       scale[p] = sc;
-      set_coefs(p, 1.f / (sc + eps), quintic, a, b, c, coef_apply, coef_square);
+      set_coefs(p, 1.f / (sc + eps), quintic, a, b, c, coef_apply, coef_square, coef_gram);
     }
   }
 }
@@ -463,7 +471,8 @@ k_pi_reduce(const PiSlice* __restrict__ slices, const float* __restrict__ part, 
   const float scv = (float)sqrt(fmax(tt, 0.0));
   if (!isfinite(tt)) atomicOr(rd.status, 1);
   rd.scale[sl.p] = scv;
-  set_coefs(sl.p, 1.f / (scv + rd.eps), rd.quintic, rd.a, rd.b, rd.c, rd.coef_apply, rd.coef_square);
+  set_coefs(sl.p, 1.f / (scv + rd.eps), rd.quintic, rd.a, rd.b, rd.c, rd.coef_apply, rd.coef_square,
+            rd.coef_gram);
 }
 
 // K = 0: U = X0 = in / (s + eps) straight from the fp32 input.
@@ -1164,11 +1173,53 @@ void launch_stage(cudaStream_t s, const WorkerPtrs& in, int M, void* X, int x_bf
 void launch_fro_finalize(cudaStream_t s, int n_probs, int n_mats, int M, const float* partials,
                          const int* mat_chunk0, const int* mat_nchunks, int use_for_scale,
                          float eps, int quintic, float a, float b, float c, float* scale,
-                         float2* coef_apply, float2* coef_square, int* status) {
+                         float2* coef_apply, float2* coef_square, float2* coef_gram, int* status) {
   count_launch();
   launch_pdl(k_fro_finalize, dim3(n_probs), dim3(kThreads), 0, s, n_mats, M, partials, mat_chunk0, mat_nchunks,
-                                              use_for_scale, eps, quintic, a, b, c, scale,
-                                              coef_apply, coef_square, status);
+             use_for_scale, eps, quintic, a, b, c, scale, coef_apply, coef_square, coef_gram, status);
+}
+
+// Gram space: Q1 = alpha I + beta A~ per problem, (alpha, beta) = coef[p]
+// (the cubic iteration 0's apply coefficients, a cc and b cc^3), over the
+// whole g x gld rows of each problem's m x m buffer.  8 bf16 per thread.
+__global__ void __launch_bounds__(kThreads)
+k_gram_q1(const __nv_bfloat16* __restrict__ A, __nv_bfloat16* __restrict__ Q, const int64_t* __restrict__ prob_aoff,
+          const int* __restrict__ prob_g, const int* __restrict__ prob_gld, const float2* __restrict__ coef) {
+  griddep_wait();
+  griddep_launch();
+  const int p = blockIdx.y;
+  const int g = prob_g[p], gld = prob_gld[p];
+  const int64_t base = prob_aoff[p];
+  const float2 cf = coef[p];
+  const int64_t n8 = (int64_t)g * gld / 8;   // gld is a multiple of 8
+  for (int64_t v = (int64_t)blockIdx.x * kThreads + threadIdx.x; v < n8; v += (int64_t)gridDim.x * kThreads) {
+    const int64_t e = 8 * v;
+    const int r = (int)(e / gld), c0 = (int)(e - (int64_t)r * gld);
+    const uint4 raw = *reinterpret_cast<const uint4*>(A + base + e);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+    uint4 out;
+    uint32_t* o = reinterpret_cast<uint32_t*>(&out);
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const float2 f = __bfloat1622float2(h[t]);
+      float x = cf.y * f.x, y = cf.y * f.y;
+      if (c0 + 2 * t == r) x += cf.x;
+      if (c0 + 2 * t + 1 == r) y += cf.x;
+      const __nv_bfloat162 q = __floats2bfloat162_rn(x, y);
+      o[t] = *reinterpret_cast<const uint32_t*>(&q);
+    }
+    *reinterpret_cast<uint4*>(Q + base + e) = out;
+  }
+}
+
+void launch_gram_q1(cudaStream_t s, int n_probs, const void* A, void* Q, const int64_t* prob_aoff,
+                    const int* prob_g, const int* prob_gld, const float2* coef, int max_g, int max_gld) {
+  if (n_probs <= 0) return;
+  count_launch();
+  const int64_t n8 = (int64_t)max_g * max_gld / 8;
+  const int bx = (int)std::min<int64_t>((n8 + kThreads - 1) / kThreads, 64);
+  launch_pdl(k_gram_q1, dim3(bx, n_probs), dim3(kThreads), 0, s, reinterpret_cast<const __nv_bfloat16*>(A),
+             reinterpret_cast<__nv_bfloat16*>(Q), prob_aoff, prob_g, prob_gld, coef);
 }
 
 void launch_pi_init(cudaStream_t s, int n_probs, const int64_t* uoff, const int* prob_g, float* u, int warm) {

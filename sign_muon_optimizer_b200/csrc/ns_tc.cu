@@ -293,6 +293,8 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
 // (64-column atom, row, atom index, matrix) with a box of two atoms x 64
 // rows: an MN-major operand half of a k-block in one request.  Slots 10..13
 // hold the first four with 32-row boxes (an epilogue warp's operand atom).
+// The m x m buffers (A, B and the Gram-space A2, Q0, Q1) are addressed by
+// mm_slot(buffer, box).
 __device__ __forceinline__ const CUtensorMap* map_at(const CUtensorMap* maps, int group, int slot) {
   return maps + group * kMapsPerGroup + slot;
 }
@@ -368,17 +370,24 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
       const GroupInfo gi = group_info(a, tc.group);
       const int nk = (tc.Kdim + BK - 1) / BK;
       const int amn = a_is_mn(op, gi.wide), bmn = b_is_mn(op, gi.wide);
-      const CUtensorMap* mA;
-      const CUtensorMap* mB;
+      // each operand's map with 64-row boxes, and with 128-row boxes
+      const CUtensorMap *mA, *mB, *mA128, *mB128;
       if (op == OP_GRAM) {
         mA = mB = map_at(maps, tc.group, a.map_src);
+        mA128 = mB128 = map128(mA);
       } else if (op == OP_SQUARE) {
-        mA = mB = map_at(maps, tc.group, 2);
+        mA = map_at(maps, tc.group, mm_slot(a.sq_l, 0));
+        mA128 = map_at(maps, tc.group, mm_slot(a.sq_l, 1));
+        mB = map_at(maps, tc.group, mm_slot(a.sq_r, 0));
+        mB128 = map_at(maps, tc.group, mm_slot(a.sq_r, 1));
       } else {
-        const CUtensorMap* mP = map_at(maps, tc.group, a.p_from_b ? 3 : 2);
+        const CUtensorMap* mP = map_at(maps, tc.group, mm_slot(a.p_buf, 0));
+        const CUtensorMap* mP128 = map_at(maps, tc.group, mm_slot(a.p_buf, 1));
         const CUtensorMap* mX = map_at(maps, tc.group, a.map_src);
         mA = gi.wide ? mP : mX;
         mB = gi.wide ? mX : mP;
+        mA128 = gi.wide ? mP128 : map128(mX);
+        mB128 = gi.wide ? map128(mX) : mP128;
       }
       const int a0 = tc.m0 + 128 * (int)rank;          // this CTA's A rows
       const int hb = tc.BN / 2;                        // this CTA's B rows
@@ -400,7 +409,7 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
       if (box_a) {
         lmn = amn;
         l4 = amn && x4;
-        lmap = l4 ? mX4 : (amn ? mA : map128(mA));
+        lmap = l4 ? mX4 : (amn ? mA : mA128);
         loff = (uint32_t)lane * BOX_BYTES;
         lx = a0 + 64 * lane;
         ly = a0;
@@ -408,7 +417,7 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
         const int i = lane - nA;
         lmn = bmn;
         l4 = bmn && x4 && hb == 128;
-        lmap = l4 ? mX4 : (bmn ? mB : (hb == 128 ? map128(mB) : mB));
+        lmap = l4 ? mX4 : (bmn ? mB : (hb == 128 ? mB128 : mB));
         loff = A_BYTES + (uint32_t)i * BOX_BYTES;
         lx = b0 + 64 * i;
         ly = b0;
@@ -517,7 +526,7 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
     // lane quarter q = warp % 4; lane i holds row 32 q + i) and the column
     // half e / 4 of the tile, i.e. BN/64 chunks of 32 columns.  It uses no
     // shared memory, which the operand ring and the tensor cores keep busy:
-    // the affine operand of all its chunks (X for APPLY, A for SQUARE) is
+    // the affine operand of all its chunks (X for APPLY, R for SQUARE) is
     // loaded into registers before the accumulator is ready; then, chunk by
     // chunk, tcgen05.ld 32x32b.x32, the fp32 combination c0 * operand +
     // c1 * acc, and 64 contiguous bytes of bf16 per lane stored straight to
@@ -530,12 +539,12 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
     const uint32_t tempty_leader0 = leader_addr(tempty_bar(0));
     const uint32_t tempty_leader1 = leader_addr(tempty_bar(1));
     __nv_bfloat16* dst_base =
-        reinterpret_cast<__nv_bfloat16*>(op == OP_GRAM ? a.A : (op == OP_SQUARE ? a.B : a.X_dst));
+        reinterpret_cast<__nv_bfloat16*>(op == OP_GRAM ? a.A : (op == OP_SQUARE ? a.sq_out : a.X_dst));
     // This warp's operand slice: one 32-row x 64-column atom (128-byte rows,
     // 128-byte swizzle) of the affine operand at a time, by TMA.
     const uint32_t slice = epi0 + (uint32_t)e * EPI_SLICE;
     const uint32_t my_efull = efull_bar(e);
-    const int opnd_slot = 10 + ((op == OP_SQUARE) ? 2 : a.map_src);
+    const int opnd_slot = (op == OP_SQUARE) ? mm_slot(a.sq_r, 2) : 10 + a.map_src;
     auto load_operand = [&](const TileCoord& t2, int i) {
       const int j = half * (t2.BN / 128) + i;   // atom index within the tile
       if (lane == 0) {
@@ -579,8 +588,13 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
       okw = __shfl_sync(0xffffffffu, okw, 0);
       if (!okw) break;
       tc_fence_after();
-      // symmetric Gram: an off-diagonal tile is also written transposed
-      const bool mirror = (op == OP_GRAM) && (tc.n0 != tc.m0);
+      // Symmetric output (the Gram, and the m x m products of symmetric
+      // operands that commute): an off-diagonal tile is also written
+      // transposed.  With sym_exact a diagonal tile writes its entries on and
+      // above the diagonal and their mirror, so that the stored matrix is
+      // exactly symmetric: a later SQUARE multiplies by R^T, which must equal R.
+      const bool sym_out = (op != OP_APPLY) && tc.sym;
+      const bool diag_tile = sym_out && a.sym_exact && (tc.n0 == tc.m0);
       const uint32_t tm_row = tmem_base + (uint32_t)(acc * 256) + ((uint32_t)(q * 32) << 16);
       bool alive = true;
 #pragma unroll 1
@@ -661,13 +675,24 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
           uint32_t ow[16];
 #pragma unroll
           for (int k = 0; k < 16; ++k) ow[k] = pack_bf16x2(v[2 * k], v[2 * k + 1]);
-          if (live) store_row_chunk(dst_base + mrow + col0, ncol, ow);
-          if (mirror && live) {
+          if (live) {
+            if (!diag_tile || col0 > row) {
+              store_row_chunk(dst_base + mrow + col0, ncol, ow);
+            } else if (col0 + 31 >= row) {
+              // the chunk crosses the diagonal: only the entries on or above it
+#pragma unroll
+              for (int u = 0; u < 32; ++u)
+                if (u < ncol && col0 + u >= row) dst_base[mrow + col0 + u] = __float2bfloat16_rn(v[u]);
+            }
+            // (a chunk wholly below the diagonal comes from the mirror of the lanes above)
+          }
+          if (sym_out && live && (tc.n0 != tc.m0 || (diag_tile && col0 + 31 > row))) {
             // lanes hold consecutive rows: each store below is 64 contiguous bytes
-            __nv_bfloat16* At = reinterpret_cast<__nv_bfloat16*>(a.A) + gi.a_base + (int64_t)tc.b * gi.g * gi.gld;
+            __nv_bfloat16* At = dst_base + gi.a_base + (int64_t)tc.b * gi.g * gi.gld;
 #pragma unroll
             for (int u = 0; u < 32; ++u)
-              if (u < ncol) At[(int64_t)(col0 + u) * gi.gld + row] = __float2bfloat16_rn(v[u]);
+              if (u < ncol && (!diag_tile || col0 + u > row))
+                At[(int64_t)(col0 + u) * gi.gld + row] = __float2bfloat16_rn(v[u]);
           }
         }
         if (affine) {

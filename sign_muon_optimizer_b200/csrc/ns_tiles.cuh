@@ -28,6 +28,7 @@ struct TileCoord {
   int b;         // problem within the group (worker*count + q)
   int m0, n0;    // tile origin in the output
   int Mdim, Ndim, Kdim, BN;
+  int sym;       // only tiles on or above the diagonal run (symmetric output)
 };
 
 __host__ __device__ __forceinline__ const TileGroup* tile_table(const GemmArgs& a) {
@@ -67,6 +68,7 @@ __host__ __device__ __forceinline__ TileCoord decode_tile(const GemmArgs& a, int
   c.Ndim = tg.Ndim;
   c.Kdim = tg.Kdim;
   c.BN = tg.BN;
+  c.sym = tg.sym;
   return c;
 }
 

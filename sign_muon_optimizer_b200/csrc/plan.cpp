@@ -34,7 +34,10 @@ int pick_bn(int n) {
   return best;
 }
 
-void build_tiles(Plan& p, int op, int nw, TileTable* tt) {
+// force_sym: square 256 x 256 tiles for GRAM and SQUARE (the Gram-space
+// iteration needs their outputs exactly symmetric, which the upper-triangle
+// tiles and their mirror give)
+void build_tiles(Plan& p, int op, int nw, TileTable* tt, bool force_sym = false) {
   std::vector<TileGroup> v;
   for (int gidx = 0; gidx < (int)p.groups.size(); ++gidx) {
     const GroupInfo& g = p.groups[gidx];
@@ -51,11 +54,12 @@ void build_tiles(Plan& p, int op, int nw, TileTable* tt) {
       t.Kdim = g.g;
     }
     t.BM = p.fp32 ? 128 : 256;
-    t.BN = p.fp32 ? 128 : pick_bn(t.Ndim);
+    t.BN = p.fp32 ? 128 : ((force_sym && op != OP_APPLY) ? 256 : pick_bn(t.Ndim));
     t.tiles_m = (t.Mdim + t.BM - 1) / t.BM;
     t.tiles_n = (t.Ndim + t.BN - 1) / t.BN;
-    // the Gram X X^T is symmetric: with square tiles only the upper ones run
-    t.sym = (op == OP_GRAM && !p.fp32 && t.BM == t.BN) ? 1 : 0;
+    // the Gram X X^T, and the square's products of commuting symmetric m x m
+    // matrices, are symmetric: with square tiles only the upper ones run
+    t.sym = ((op == OP_GRAM || op == OP_SQUARE) && !p.fp32 && t.BM == t.BN) ? 1 : 0;
     t.batch = nw * g.count;
     v.push_back(t);
   }
@@ -69,6 +73,16 @@ void build_tiles(Plan& p, int op, int nw, TileTable* tt) {
   }
   tt->groups = v;
   tt->total = start;
+}
+
+// flops of every tile of a launch as it runs (2 BM BN K per tile)
+double tile_flops(const TileTable& tt) {
+  double f = 0.0;
+  for (const TileGroup& t : tt.groups) {
+    const int per = t.sym ? t.tiles_m * (t.tiles_m + 1) / 2 : t.tiles_m * t.tiles_n;
+    f += 2.0 * t.BM * t.BN * t.Kdim * (double)per * t.batch;
+  }
+  return f;
 }
 
 }  // namespace
@@ -182,6 +196,33 @@ int make_plan(const int64_t* shapes, int n_mats, int M, int K, int scale, int P,
     build_tiles(p, op, M, &p.tiles[op][0]);
     build_tiles(p, op, 1, &p.tiles[op][1]);
   }
+  // X space: K x (Gram + apply).  Gram space: one Gram, 3K - 3 m x m products
+  // (T_k = a A_k + b A_k^2, A_{k+1} = a T_k + b A_k T_k, Q_{k+1} = a Q_k + b A_k Q_k)
+  // and one apply.  Tile flops, counted as the tiles run; with SIGNMUON_NS_GRAM
+  // the Gram-space form is taken when it saves more than 15 % (its extra
+  // launches and its elementwise start cost a little) and every Gram side is
+  // at least 256:
+  // small Grams gain little time, and rounding their squared spectrum to
+  // bf16 flips twice as many of the smallest entries' signs.
+  bool big = true;
+  for (const GroupInfo& g : p.groups) big = big && g.g >= 256;
+  if ((flags & SIGNMUON_NS_GRAM) && !p.fp32 && !p.quintic && K >= 2 && big) {
+    // both forms counted with the Gram on square tiles, as Gram space runs it
+    TileTable gram[2], square[2];
+    for (int s = 0; s < 2; ++s) {
+      build_tiles(p, OP_GRAM, s == 0 ? M : 1, &gram[s], true);
+      build_tiles(p, OP_SQUARE, s == 0 ? M : 1, &square[s], true);
+    }
+    const double xs = K * (tile_flops(gram[0]) + tile_flops(p.tiles[OP_APPLY][0]));
+    const double gs = tile_flops(gram[0]) + (3.0 * K - 3.0) * tile_flops(square[0]) + tile_flops(p.tiles[OP_APPLY][0]);
+    p.gram_ns = gs < 0.85 * xs;
+    if (p.gram_ns) {
+      for (int s = 0; s < 2; ++s) {
+        p.tiles[OP_GRAM][s] = gram[s];
+        p.tiles[OP_SQUARE][s] = square[s];
+      }
+    }
+  }
   // power iteration tables (worker-major problems so worker 0 is a prefix)
   int64_t u = 0, part = 0;
   for (int w = 0; w < M; ++w) {
@@ -219,6 +260,7 @@ int make_plan(const int64_t* shapes, int n_mats, int M, int K, int scale, int P,
     bytes += 2 * (int64_t)M * p.dpad * 4;                 // momentum, U
     bytes += 2 * p.x_elems * esz;                         // X ping/pong
     bytes += p.a_elems * esz * (p.quintic ? 2 : 1);       // A (and B)
+    if (p.gram_ns) bytes += p.a_elems * esz * 4;          // B, A2, Q0, Q1 of the Gram-space iteration
     bytes += (int64_t)M * p.nb_pad;                       // packed bits
     if (flags & SIGNMUON_TERNARY) bytes += (int64_t)M * p.dpad;  // int8 ternary signs
     bytes += p.dpad * 4;                                  // D
@@ -229,7 +271,7 @@ int make_plan(const int64_t* shapes, int n_mats, int M, int K, int scale, int P,
     bytes += (int64_t)p.pi_slices.size() * 8;             // per-slice figures
     bytes += (int64_t)M * n_mats * 8;                     // per-problem counters, 1/||y||
     if (flags & SIGNMUON_PI_WARM) bytes += p.u_elems_one * 4;  // warm state of one problem set
-    bytes += (int64_t)p.groups.size() * 8 * 128;          // tensor maps
+    bytes += (int64_t)p.groups.size() * kMapsPerGroup * 128;  // tensor maps
   }
   p.device_bytes = bytes;
   (void)K;

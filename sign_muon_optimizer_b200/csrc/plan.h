@@ -19,6 +19,10 @@ struct TileTable {
 struct Plan {
   int M = 0, n_mats = 0;
   bool fp32 = false, quintic = false;
+  // bf16 cubic Newton-Schulz in Gram space (m x m products, one final X
+  // product) rather than on X: with SIGNMUON_NS_GRAM, when it needs fewer
+  // tile flops
+  bool gram_ns = false;
   int64_t d = 0;        // parameters
   int64_t dpad = 0;     // stride of the library's flat per-worker vectors
   int64_t nb = 0;       // ceil(d/8) packed bytes per worker

@@ -12,6 +12,7 @@
 #include <cuda.h>
 #include <nvtx3/nvToolsExt.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cstdio>
 #include <cstring>
@@ -68,6 +69,8 @@ struct signmuon_ctx {
   void* X[2] = {nullptr, nullptr};
   void* A = nullptr;
   void* B = nullptr;
+  void* A2 = nullptr;           // Gram space: the second A buffer and the Q pair
+  void* Q[2] = {nullptr, nullptr};
   float* U = nullptr;
   uint8_t* bits = nullptr;
   int8_t* sign8 = nullptr;      // TERNARY: int8 signs, M x dpad bytes
@@ -76,6 +79,7 @@ struct signmuon_ctx {
   float* scale_v = nullptr;
   float2* coef_apply = nullptr;
   float2* coef_square = nullptr;
+  float2* coef_gram = nullptr;  // Gram space: A1 = a T0 + b cc^2 A~ T0
   float* pi_u = nullptr;        // power-iteration iterates of the M-worker problems (warm state)
   float* pi_u1 = nullptr;       // PI_WARM: iterates of the one-problem-set PolarNS (warm state)
   float* pi_y = nullptr;
@@ -283,9 +287,24 @@ void prof_collect(signmuon_t h) {
 // flat) to out + worker*out_stride.  kzero_in is the fp32 input used when
 // K == 0.
 // ---------------------------------------------------------------------------
+// m x m bf16 buffer by index (sm::MmBuf)
+void* mm_ptr(signmuon_t h, int buf) {
+  switch (buf) {
+    case sm::MM_A: return h->A;
+    case sm::MM_B: return h->B;
+    case sm::MM_A2: return h->A2;
+    case sm::MM_Q0: return h->Q[0];
+    default: return h->Q[1];
+  }
+}
+
+// One grouped GEMM launch.  SQUARE (bf16): out buffer sq_out = c0 R + c1 L R
+// + cdiag I with L = buffer sq_l, R = buffer sq_r; APPLY multiplies X by
+// buffer p_buf (default: B for quintic, else A).
 void gemm(signmuon_t h, int op, int slot, int src, int nw, const float2* coef, float c0, float c1,
           bool final_out, float* out, int64_t out_stride, uint32_t* out_bits = nullptr, int64_t bits_stride = 0,
-          float cdiag = 0.f, bool plain = false) {
+          float cdiag = 0.f, bool plain = false, int sq_l = sm::MM_A, int sq_r = sm::MM_A, int sq_out = sm::MM_B,
+          int p_buf = -1) {
   const Plan& p = h->plan;
   sm::GemmArgs a{};
   a.tiles = h->d_tiles[op][slot];
@@ -301,6 +320,11 @@ void gemm(signmuon_t h, int op, int slot, int src, int nw, const float2* coef, f
   a.A = h->A;
   a.B = h->B;
   a.p_from_b = (op == sm::OP_APPLY && p.quintic) ? 1 : 0;
+  a.p_buf = p_buf >= 0 ? p_buf : (a.p_from_b ? sm::MM_B : sm::MM_A);
+  a.sq_l = sq_l;
+  a.sq_r = sq_r;
+  a.sq_out = mm_ptr(h, sq_out);
+  a.sym_exact = p.gram_ns ? 1 : 0;
   a.map_src = src;
   a.map_dst = src ^ 1;
   a.coef = coef;
@@ -342,7 +366,7 @@ void power_iteration(signmuon_t h, int nw) {
   ProfScope ps(h, 5);
   const int nslices = nw == 1 ? p.n_pi_slices_one : (int)p.pi_slices.size();
   const sm::PiReduce mid{0, u, h->pi_sq, h->pi_cnt, h->pi_inv, h->eps, p.quintic ? 1 : 0, h->ns_a, h->ns_b,
-                         h->ns_c, h->scale_v, h->coef_apply, h->coef_square, h->status};
+                         h->ns_c, h->scale_v, h->coef_apply, h->coef_square, h->coef_gram, h->status};
   sm::PiReduce fin = mid;
   fin.last = 1;
   // u0; then y = A u0; then P times y = A (y / ||y||), storing y / ||y|| as u
@@ -388,6 +412,50 @@ void run_ns(signmuon_t h, int K, int nw, const sm::WorkerPtrs& kzero_in, float* 
                           p.n_mats, h->scale_v, h->eps);
     return;
   }
+  if (p.gram_ns && K >= 2) {
+    // The same iteration in Gram space (bf16 cubic): with P_k = a I + b A_k,
+    // A_{k+1} = P_k A_k P_k and Q_{k+1} = P_k Q_k, all polynomials in
+    // A0 = cc^2 A~, so every product commutes and is symmetric:
+    //   T_k     = a A_k + b A_k^2          (square: L = R = A_k)
+    //   A_{k+1} = a T_k + b A_k T_k        (L = A_k, R = T_k)
+    //   Q_{k+1} = a Q_k + b A_k Q_k        (L = A_k, R = Q_k)
+    // from Q1 = cc P_0 = a cc I + b cc^3 A~, then X_K = Q_K X~ once.  Iteration
+    // 0 works on the unscaled Gram (the power iteration's input), its scale
+    // in per-problem coefficients.
+    gemm(h, sm::OP_GRAM, slot, 0, nw, nullptr, 0.f, 1.f, false, nullptr, 0);
+    if (spectral) power_iteration(h, nw);
+    {
+      ProfScope ps(h, nw == 1 ? 10 : 3);
+      int max_g = 1, max_gld = 8;
+      for (const sm::GroupInfo& gi : p.groups) {
+        max_g = std::max(max_g, gi.g);
+        max_gld = std::max(max_gld, gi.gld);
+      }
+      sm::launch_gram_q1(h->stream, nw * p.n_mats, h->A, h->Q[0], h->d_prob_aoff, h->d_prob_g, h->d_prob_gld,
+                         h->coef_apply, max_g, max_gld);
+    }
+    const float a = h->ns_a, b = h->ns_b;
+    gemm(h, sm::OP_SQUARE, slot, 0, nw, h->coef_square, 0.f, 0.f, false, nullptr, 0, nullptr, 0, 0.f, false,
+         sm::MM_A, sm::MM_A, sm::MM_B);                                             // T0
+    gemm(h, sm::OP_SQUARE, slot, 0, nw, h->coef_gram, 0.f, 0.f, false, nullptr, 0, nullptr, 0, 0.f, false,
+         sm::MM_A, sm::MM_B, sm::MM_A2);                                            // A1
+    int acur = sm::MM_A2, aoth = sm::MM_A, qcur = sm::MM_Q0, qoth = sm::MM_Q1;
+    for (int k = 1; k < K; ++k) {
+      gemm(h, sm::OP_SQUARE, slot, 0, nw, nullptr, a, b, false, nullptr, 0, nullptr, 0, 0.f, false, acur, qcur,
+           qoth);                                                                   // Q_{k+1}
+      if (k + 1 < K) {
+        gemm(h, sm::OP_SQUARE, slot, 0, nw, nullptr, a, b, false, nullptr, 0, nullptr, 0, 0.f, false, acur, acur,
+             sm::MM_B);                                                             // T_k
+        gemm(h, sm::OP_SQUARE, slot, 0, nw, nullptr, a, b, false, nullptr, 0, nullptr, 0, 0.f, false, acur,
+             sm::MM_B, aoth);                                                       // A_{k+1}
+        std::swap(acur, aoth);
+      }
+      std::swap(qcur, qoth);
+    }
+    gemm(h, sm::OP_APPLY, slot, 0, nw, nullptr, 0.f, 1.f, true, out, out_stride, out_bits, bits_stride, 0.f, true,
+         sm::MM_A, sm::MM_A, sm::MM_B, qcur);                                       // X_K = Q_K X~
+    return;
+  }
   // After the first iteration (bf16 path) the a X term joins the apply's
   // operator: the Gram GEMM writes P = b A + a I (cubic) or the square GEMM
   // B = b A + c A^2 + a I (quintic), and the apply is a plain GEMM X' = P X
@@ -421,7 +489,7 @@ void fro_finalize(signmuon_t h, int nw) {
   ProfScope ps(h, 1);
   sm::launch_fro_finalize(h->stream, nw * p.n_mats, p.n_mats, nw, h->partials, h->d_mat_chunk0, h->d_mat_nchunks,
                           h->scale == SIGNMUON_SCALE_FRO ? 1 : 0, h->eps, p.quintic ? 1 : 0, h->ns_a, h->ns_b,
-                          h->ns_c, h->scale_v, h->coef_apply, h->coef_square, h->status);
+                          h->ns_c, h->scale_v, h->coef_apply, h->coef_square, h->coef_gram, h->status);
 }
 
 // Clear the device status at the start of a call, unless an asynchronous
@@ -550,7 +618,7 @@ int signmuon_plan_tables(const int64_t* shapes, int n_mats, int M, int K, int sc
       {"n_pi_tiles_one", p.n_pi_tiles_one},
       {"n_pi_slices", (int64_t)p.pi_slices.size()}, {"n_pi_slices_one", p.n_pi_slices_one},
       {"part_elems", p.part_elems}, {"M", p.M}, {"n_mats", p.n_mats}, {"fp32", p.fp32 ? 1 : 0},
-      {"quintic", p.quintic ? 1 : 0}, {"device_bytes", p.device_bytes}};
+      {"quintic", p.quintic ? 1 : 0}, {"gram_ns", p.gram_ns ? 1 : 0}, {"device_bytes", p.device_bytes}};
   for (const auto& kv : scalars) {
     j += '"';
     j += kv.first;
@@ -688,11 +756,19 @@ int signmuon_init(signmuon_t* out, const int64_t* shapes, int n_mats, int M, flo
     uint8_t* x = nullptr;
     if ((rc = dalloc(h, &x, p.a_elems * esz))) return bail(rc);
     h->A = x;
-    if (p.quintic) {
+    if (p.quintic || p.gram_ns) {
       if ((rc = dalloc(h, &x, p.a_elems * esz))) return bail(rc);
       h->B = x;
     } else {
       h->B = h->A;
+    }
+    if (p.gram_ns) {
+      if ((rc = dalloc(h, &x, p.a_elems * esz))) return bail(rc);
+      h->A2 = x;
+      for (int i = 0; i < 2; ++i) {
+        if ((rc = dalloc(h, &x, p.a_elems * esz))) return bail(rc);
+        h->Q[i] = x;
+      }
     }
   }
   if ((rc = dalloc(h, &h->bits, (int64_t)M * p.nb_pad))) return bail(rc);
@@ -705,6 +781,7 @@ int signmuon_init(signmuon_t* out, const int64_t* shapes, int n_mats, int M, flo
   if ((rc = dalloc(h, &h->scale_v, (int64_t)M * p.n_mats))) return bail(rc);
   if ((rc = dalloc(h, &h->coef_apply, (int64_t)M * p.n_mats))) return bail(rc);
   if ((rc = dalloc(h, &h->coef_square, (int64_t)M * p.n_mats))) return bail(rc);
+  if (p.gram_ns && (rc = dalloc(h, &h->coef_gram, (int64_t)M * p.n_mats))) return bail(rc);
   if ((rc = dalloc(h, &h->pi_u, p.u_elems))) return bail(rc);
   if ((rc = dalloc(h, &h->pi_y, p.u_elems))) return bail(rc);
   if ((rc = dalloc(h, &h->pi_part, p.part_elems))) return bail(rc);
@@ -728,7 +805,8 @@ int signmuon_init(signmuon_t* out, const int64_t* shapes, int n_mats, int M, flo
     // per group: slots 0..3 = X ping, X pong, A, B with 64-row boxes;
     // slots 4..7 = the same tensors with 128-row boxes; when X's column
     // count is a multiple of 64, X ping/pong as 4-D atom views with 2-atom x
-    // 64-row boxes at 8/9; slots 10..13 = the first four with 32-row boxes
+    // 64-row boxes at 8/9; slots 10..13 = the first four with 32-row boxes;
+    // Gram space: A2, Q0, Q1 with 64-, 128- and 32-row boxes at 14..22
     std::vector<CUtensorMap> maps(p.groups.size() * sm::kMapsPerGroup);
     std::memset(maps.data(), 0, maps.size() * sizeof(CUtensorMap));
     for (size_t g = 0; g < p.groups.size(); ++g) {
@@ -745,6 +823,14 @@ int signmuon_init(signmuon_t* out, const int64_t* shapes, int n_mats, int M, flo
         void* bb = reinterpret_cast<__nv_bfloat16*>(h->B) + gi.a_base;
         if ((rc = encode_map(h, &mm[2], ab, gi.g, gi.g, gi.gld, batch, br))) return bail(rc);
         if ((rc = encode_map(h, &mm[3], bb, gi.g, gi.g, gi.gld, batch, br))) return bail(rc);
+        if (p.gram_ns) {
+          void* const gbuf[3] = {h->A2, h->Q[0], h->Q[1]};
+          for (int j = 0; j < 3; ++j) {
+            void* base = reinterpret_cast<__nv_bfloat16*>(gbuf[j]) + gi.a_base;
+            CUtensorMap* gm = &maps[g * sm::kMapsPerGroup + sm::mm_slot(sm::MM_A2 + j, box)];
+            if ((rc = encode_map(h, gm, base, gi.g, gi.g, gi.gld, batch, br))) return bail(rc);
+          }
+        }
       }
       if (gi.cols % 64 == 0) {
         for (int i = 0; i < 2; ++i) {

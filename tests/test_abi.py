@@ -107,6 +107,7 @@ def test_plan_accepts_the_sign_wire_variants_and_counts_ternary_bytes():
         assert p["device_bytes"] == base["device_bytes"] + extra
     # the warm power-iteration state of one problem set: min(rows, cols) floats per matrix
     assert smo.SIGNMUON_PI_WARM == 1 << 12
+    assert smo.SIGNMUON_NS_GRAM == 1 << 13
     p = smo.signmuon_plan(shapes, 5, 5, "spectral", 2, 1 << 12)
     assert p["device_bytes"] == base["device_bytes"] + 4 * (8 + 16)
 

@@ -78,6 +78,18 @@ def test_nanogpt_flop_count():
     assert bench.ns_flops_per_step(synth.NANOGPT_SHAPES, 8, 5, False) == 8 * 1_304_596_316_160
 
 
+def test_ns_kind_flops_x_and_gram_space():
+    # one 768 x 3072 matrix, K = 5, one problem set: on X five Grams and five
+    # applies of 2 m^2 n; in Gram space one of each plus 12 m x m products
+    m, n = 768, 3072
+    x = bench.ns_kind_flops([(m, n)], 1, 5, False)
+    g = bench.ns_kind_flops([(n, m)], 1, 5, True)
+    assert x == {"gram": 5 * 2 * m * m * n, "square": 0, "apply": 5 * 2 * m * m * n}
+    assert g == {"gram": 2 * m * m * n, "square": 12 * 2 * m ** 3, "apply": 2 * m * m * n}
+    assert sum(g.values()) <= 0.5 * sum(x.values())     # 40 m^3 against 80 m^3 at n = 4 m
+    assert bench.ns_kind_flops([(m, n)], 8, 5, True)["square"] == 8 * g["square"]
+
+
 def test_hbm_bytes_counts():
     d = synth.numel(synth.NANOGPT_SHAPES)
     b = bench.hbm_bytes_per_step(synth.NANOGPT_SHAPES, 8, 2, True)

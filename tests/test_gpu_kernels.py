@@ -107,8 +107,11 @@ def test_update_bit_exact(kind, d):
 SHAPES_SMALL = [(3, 5), (5, 3), (130, 70), (64, 147), (200, 200), (96, 300)]
 
 
-def _polar_case(shapes, M, K, scale, P, precision, order, seed, coeffs=None):
+def _polar_case(shapes, M, K, scale, P, precision, order, seed, coeffs=None, extra=0, want_gram_ns=None):
     flags = (smo.SIGNMUON_NS_FP32 if precision == "fp32" else 0) | (smo.SIGNMUON_NS_QUINTIC if order == "quintic" else 0)
+    flags |= extra
+    if want_gram_ns is not None:
+        assert smo.signmuon_plan_tables(shapes, M, K, scale, P, flags)["gram_ns"] == want_gram_ns
     h = smo.SignMuon(shapes, M, beta=0.9, lam=0.0, K=K, eps=1e-7, scale=scale, P=P, flags=flags)
     if coeffs is not None:
         h.set_ns_coeffs(coeffs)
@@ -143,6 +146,19 @@ def test_polar_custom_coefficients(precision, order, coeffs):
     against the oracle run with the same coefficients (both converge to the
     polar factor: p(1) = 1 for each)."""
     _polar_case(SHAPES_SMALL, 2, 4, "fro", 1, precision, order, seed=11, coeffs=coeffs)
+
+
+@pytest.mark.parametrize("gram", [True, False])
+@pytest.mark.parametrize("K", [2, 3, 5])
+@pytest.mark.parametrize("scale,P", [("fro", 1), ("spectral", 2)])
+def test_polar_gram_space(gram, K, scale, P):
+    """bf16 cubic PolarNS in Gram space (SIGNMUON_NS_GRAM, taken for matrices
+    with n well above m) and, by default, on X: both against the oracle's
+    iteration on X, on multi-tile Grams with ragged edges (m = 300, 768, 520)
+    in both orientations."""
+    shapes = [(300, 1000), (3072, 768), (520, 1600)]
+    _polar_case(shapes, 2, K, scale, P, "bf16", "cubic", seed=300 + K,
+                extra=smo.SIGNMUON_NS_GRAM if gram else 0, want_gram_ns=1 if gram else 0)
 
 
 @pytest.mark.parametrize("precision", ["fp32", "bf16"])

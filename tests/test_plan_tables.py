@@ -36,6 +36,7 @@ def _disjoint_inside(regions, limit):
 
 def _check(shapes, M, flags, spectral):
     t = smo.signmuon_plan_tables(shapes, M, 5, "spectral" if spectral else "fro", 2, flags)
+    t["_K"], t["_gram"] = 5, bool(flags & smo.SIGNMUON_NS_GRAM)
     fp32 = bool(flags & smo.SIGNMUON_NS_FP32)
     d = sum(r * c for r, c in shapes)
     assert t["d"] == d and t["dpad"] >= d and t["dpad"] % 64 == 0
@@ -97,12 +98,38 @@ def _check(shapes, M, flags, spectral):
                     assert (BM, BN) == (128, 128) and sym == 0
                 else:
                     assert BM == 256 and BN in (128, 256)
-                    assert sym == (1 if (op == GRAM and BN == 256) else 0)
+                    assert sym == (1 if (op in (GRAM, SQUARE) and BN == 256) else 0)
                 assert tm == _ceil(Md, BM) and tn == _ceil(Nd, BN)
                 assert batch == nw * groups[gi][6] and tstart == start
                 per = tm * (tm + 1) // 2 if sym else tm * tn
                 start += per * batch
             assert table["total"] == start
+
+    # X space or Gram space (bf16 cubic, K >= 2): the form with fewer tile
+    # flops, both counted with the Gram and the m x m products on square
+    # 256 x 256 upper-triangle tiles (Gram space runs them so: its stored
+    # iterates must be exactly symmetric)
+    K = t.get("_K")
+    if K is not None and not fp32:
+        def sym_flops(kdim):
+            return sum(2 * 256 * 256 * kdim(g) * (_ceil(g[3], 256) * (_ceil(g[3], 256) + 1) // 2) * M * g[6]
+                       for g in groups)
+        apply_f = 0
+        for (gi, Md, Nd, Kd, BM, BN, sym, tm, tn, batch, tstart) in t["tiles"][2 * APPLY]["groups"]:
+            apply_f += 2 * BM * BN * Kd * tm * tn * batch
+        gram_f = sym_flops(lambda g: max(g[0], g[1]))
+        sq_f = sym_flops(lambda g: g[3])
+        xs = K * (gram_f + apply_f)
+        gs = gram_f + (3 * K - 3) * sq_f + apply_f
+        big = all(g[3] >= 256 for g in groups)
+        want = (not t["quintic"]) and K >= 2 and big and t.get("_gram") and gs < 0.85 * xs
+        assert t["gram_ns"] == (1 if want else 0)
+        if want:
+            for op in (GRAM, SQUARE):
+                for slot in (0, 1):
+                    assert all(x[4] == 256 and x[5] == 256 and x[6] == 1 for x in t["tiles"][2 * op + slot]["groups"])
+    elif K is not None:
+        assert t["gram_ns"] == 0
 
     # power iteration: problem p = worker * n_mats + matrix
     n = len(shapes)
@@ -163,6 +190,29 @@ def test_plan_tables_of_the_bench_workloads(name):
     import synth
     wl = synth.WORKLOADS[name]
     _check([tuple(s) for s in wl["shapes"]], wl["M"], smo.SIGNMUON_POST_POLAR, True)
+
+
+def test_gram_space_choice():
+    """With SIGNMUON_NS_GRAM the nanoGPT set (every matrix 768 x n, n = 768..3072)
+    runs its bf16 cubic iteration in Gram space; without the flag, and for
+    square matrices, Grams under 256, quintic, fp32 and K < 2, it stays on X."""
+    import synth
+    shp = [tuple(s) for s in synth.NANOGPT_SHAPES]
+    G = smo.SIGNMUON_NS_GRAM
+    plan = lambda shapes, K=5, flags=G: smo.signmuon_plan_tables(shapes, 8, K, "spectral", 2, flags)["gram_ns"]
+    assert plan(shp) == 1
+    assert plan(shp, flags=0) == 0                                    # the default iterates on X
+    assert plan([(768, 3072)]) == 1 and plan([(3072, 768)]) == 1     # either orientation
+    assert plan([(768, 768)]) == 0 and plan([(1024, 1024)]) == 0     # square: more flops in Gram space
+    assert plan([(128, 256), (96, 300)]) == 0                         # small Grams stay on X
+    assert plan([(768, 3072), (200, 3000)]) == 0                      # ... every one of them
+    assert plan(shp, K=1) == 0
+    assert plan(shp, flags=G | smo.SIGNMUON_NS_QUINTIC) == 0
+    assert plan(shp, flags=G | smo.SIGNMUON_NS_FP32) == 0
+    # the extra m x m buffers (B, A2, Q0, Q1) are part of the device bytes
+    t1 = smo.signmuon_plan_tables(shp, 8, 5, "spectral", 2, G)
+    t2 = smo.signmuon_plan_tables(shp, 8, 5, "spectral", 2, 0)
+    assert t1["device_bytes"] - t2["device_bytes"] == 4 * t1["a_elems"] * 2
 
 
 def test_plan_tables_size_query_and_errors():
