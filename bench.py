@@ -580,10 +580,27 @@ def run_ours(args):
         ev1.record(stream)
         torch.cuda.synchronize()
         wall = time.perf_counter() - t0
+        opt.sync()
         ems = max_over_ranks(max(ev0.elapsed_time(ev1), wall * 1e3), "cuda")
+        # the copy link alone: the same host-to-device bytes as plain pinned copies
+        h2d = (M + 1) * D * 4
+        dst = torch.empty(D, dtype=torch.float32, device="cuda")
+        dst.copy_(Gh[0], non_blocking=True)
+        torch.cuda.synchronize()
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        c0.record()
+        for src in [Wh] + Gh:
+            dst.copy_(src, non_blocking=True)
+        c1.record()
+        torch.cuda.synchronize()
+        h2d_gbs = h2d / (c0.elapsed_time(c1) / 1e3) / 1e9
+        del dst
         e2e = {"value": job_throughput(world, args.e2e_steps, ems), "unit": "steps/s",
-               "h2d_bytes_per_step": (M + 1) * D * 4, "d2h_bytes_per_step": D * 4,
-               "api": "signmuon_step_host (pinned host W and G)"}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": D * 4,
+               "h2d_copy_GBps": h2d_gbs, "copy_bound_steps_per_s": h2d_gbs * 1e9 / h2d,
+               "api": "signmuon_step_host (pinned host W and G) with SIGNMUON_ASYNC: each step's gradients "
+                      "come in on a copy stream while the step before runs and its W goes back; "
+                      "copy_bound_steps_per_s = the host-to-device bytes alone at the rate of plain pinned copies"}
         del Gh, Wh
 
     # the other configurations (N = 1 only: the scaling runs time the headline alone)
@@ -813,7 +830,7 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-steps", type=int, default=6)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the short passes of the ResNet-50, LLaMA-layer vote and NS sweep configurations")

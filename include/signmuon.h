@@ -237,9 +237,18 @@ int signmuon_sums_step(signmuon_t h, float* W, const void* sums, float eta);
 
 /* ------------------------------------------------------------------------
  * signmuon_step_host -- signmuon_step on HOST buffers: copies W and the M
- * gradients to library-owned device buffers (allocated on first use),
- * runs the step and copies W back.  Always waits.  Pinned host memory gives
- * full copy bandwidth.
+ * gradients to library-owned device buffers (allocated on first use: W and
+ * two sets of M gradients), runs the step and copies W back.  Pinned host
+ * memory gives full copy bandwidth.
+ *   W_host     float[d], read and then overwritten with the updated weights.
+ *   G_host     host array of M pointers, each float[d]; only read.
+ * The gradients come in on a second stream of the library's, alternating
+ * between the two device sets.  Without SIGNMUON_ASYNC the call waits and
+ * returns the step's status.  With it the call returns once the copies and
+ * the step are queued, and the next call's gradients come in while this
+ * step runs and W goes back; W_host and every G_host[m] must then stay
+ * valid and unchanged until signmuon_sync (a W_host shared by consecutive
+ * calls is fine: each call reads it after the call before has written it).
  * ---------------------------------------------------------------------- */
 int signmuon_step_host(signmuon_t h, float* W_host, const float* const* G_host, float eta);
 

@@ -90,9 +90,14 @@ struct signmuon_ctx {
   int* status = nullptr;        // [0] non-finite flag, [1] kernel error code
   int* h_status = nullptr;      // pinned mirror
   bool pending = false;         // an async step's status not yet read
-  // step_host staging
+  // step_host staging: W, and two gradient buffers so that a call's
+  // gradients can come in (on the copy stream) while the step before runs
   float* hw_W = nullptr;
-  float* hw_G = nullptr;
+  float* hw_G[2] = {nullptr, nullptr};
+  int hw_next = 0;                      // the gradient buffer of the next call
+  cudaStream_t copy_stream = nullptr;
+  cudaEvent_t g_ready[2] = {nullptr, nullptr};   // buffer b holds its call's gradients
+  cudaEvent_t g_free[2] = {nullptr, nullptr};    // the step that read buffer b is done
   std::vector<void*> allocs;
   int64_t bytes = 0;
   std::string err;
@@ -680,6 +685,14 @@ void signmuon_destroy(signmuon_t h) {
   if (!h) return;
   DeviceGuard dev_guard(h);
   cudaStreamSynchronize(h->stream);
+  if (h->copy_stream) {
+    cudaStreamSynchronize(h->copy_stream);
+    cudaStreamDestroy(h->copy_stream);
+  }
+  for (int b = 0; b < 2; ++b) {
+    if (h->g_ready[b]) cudaEventDestroy(h->g_ready[b]);
+    if (h->g_free[b]) cudaEventDestroy(h->g_free[b]);
+  }
   for (cudaEvent_t e : h->ev_pool) cudaEventDestroy(e);
   for (void* q : h->allocs) cudaFree(q);
   if (h->h_status) cudaFreeHost(h->h_status);
@@ -1103,25 +1116,45 @@ int signmuon_step_host(signmuon_t h, float* W_host, const float* const* G_host, 
   if (rc) return rc;
   const Plan& p = h->plan;
   if (W_host == nullptr || G_host == nullptr) return fail(h, SIGNMUON_E_INVALID, "null W or G");
-  if (!h->hw_W) {
-    if ((rc = dalloc(h, &h->hw_W, p.dpad))) return rc;
-    if ((rc = dalloc(h, &h->hw_G, (int64_t)h->M * p.dpad))) return rc;
+  for (int m = 0; m < h->M; ++m)
+    if (G_host[m] == nullptr) return fail(h, SIGNMUON_E_INVALID, "null G[m]");
+  // first use: each piece is made once, so a call after a failed one
+  // finishes the set-up
+  if (!h->hw_W && (rc = dalloc(h, &h->hw_W, p.dpad))) return rc;
+  for (int b = 0; b < 2; ++b)
+    if (!h->hw_G[b] && (rc = dalloc(h, &h->hw_G[b], (int64_t)h->M * p.dpad))) return rc;
+  if (!h->copy_stream) CK(h, cudaStreamCreateWithFlags(&h->copy_stream, cudaStreamNonBlocking));
+  for (int b = 0; b < 2; ++b) {
+    if (!h->g_ready[b]) CK(h, cudaEventCreateWithFlags(&h->g_ready[b], cudaEventDisableTiming));
+    if (!h->g_free[b]) {
+      CK(h, cudaEventCreateWithFlags(&h->g_free[b], cudaEventDisableTiming));
+      CK(h, cudaEventRecord(h->g_free[b], h->stream));
+    }
   }
-  cudaStream_t s = h->stream;
-  CK(h, cudaMemcpyAsync(h->hw_W, W_host, (size_t)p.d * 4, cudaMemcpyHostToDevice, s));
+  const int b = h->hw_next;
+  h->hw_next ^= 1;
+  cudaStream_t s = h->stream, cs = h->copy_stream;
+  // the gradients into buffer b on the copy stream, once the step that read
+  // it last (two calls ago) is done; with SIGNMUON_ASYNC they come in while
+  // the step of the call before still runs
+  CK(h, cudaStreamWaitEvent(cs, h->g_free[b], 0));
   std::vector<const float*> gd(h->M);
   for (int m = 0; m < h->M; ++m) {
-    if (G_host[m] == nullptr) return fail(h, SIGNMUON_E_INVALID, "null G[m]");
-    gd[m] = h->hw_G + (int64_t)m * p.dpad;
-    CK(h, cudaMemcpyAsync(const_cast<float*>(gd[m]), G_host[m], (size_t)p.d * 4, cudaMemcpyHostToDevice, s));
+    gd[m] = h->hw_G[b] + (int64_t)m * p.dpad;
+    CK(h, cudaMemcpyAsync(const_cast<float*>(gd[m]), G_host[m], (size_t)p.d * 4, cudaMemcpyHostToDevice, cs));
   }
+  CK(h, cudaEventRecord(h->g_ready[b], cs));
+  // W after the previous call's copy back (stream order), then the step
+  CK(h, cudaMemcpyAsync(h->hw_W, W_host, (size_t)p.d * 4, cudaMemcpyHostToDevice, s));
+  CK(h, cudaStreamWaitEvent(s, h->g_ready[b], 0));
   const unsigned saved = h->flags;
   h->flags |= SIGNMUON_ASYNC;
   rc = signmuon_step(h, h->hw_W, gd.data(), eta);
   h->flags = saved;
   if (rc) return rc;
+  CK(h, cudaEventRecord(h->g_free[b], s));
   CK(h, cudaMemcpyAsync(W_host, h->hw_W, (size_t)p.d * 4, cudaMemcpyDeviceToHost, s));
-  return signmuon_sync(h);
+  return (h->flags & SIGNMUON_ASYNC) ? SIGNMUON_OK : signmuon_sync(h);
 }
 
 // ---- CUDA IPC: map a buffer of one process into another (peer GPUs) ------

@@ -238,6 +238,42 @@ def test_step_host_matches_device_step():
     assert np.array_equal(wh.view(np.uint32), host(W).view(np.uint32))
 
 
+@pytest.mark.parametrize("pinned", [True, False])
+def test_step_host_async_pipeline_matches_device_steps(pinned):
+    """SIGNMUON_ASYNC step_host calls queued back to back (each call's
+    gradients come in on the copy stream, alternating between two device
+    sets, while the step before runs): after one sync, W and the momenta are
+    bit-identical to the same steps on device buffers, for gradients that
+    differ from call to call and one W host buffer shared by all calls."""
+    shapes = [(256, 512), (96, 160), (130, 70)]
+    M, T = 3, 5
+    w0 = synth.weights0(shapes, 41)
+    grads = [synth.gradients(shapes, M, 1.0, step=t, config_id=41) for t in range(T)]
+    kw = dict(beta=HP["beta"], lam=HP["lam"], K=3, eps=HP["eps"], scale="spectral", P=2,
+              flags=smo.SIGNMUON_POST_POLAR)
+    a = smo.SignMuon(shapes, M, **kw)
+    W = dev(w0)
+    for t in range(T):
+        a.step(W, [dev(g) for g in grads[t]], 0.02)
+    b = smo.SignMuon(shapes, M, **dict(kw, flags=kw["flags"] | smo.SIGNMUON_ASYNC))
+    if pinned:
+        wt = torch.from_numpy(w0.copy()).pin_memory()
+        gts = [[torch.from_numpy(g).pin_memory() for g in grads[t]] for t in range(T)]
+        wh, gh = wt.numpy(), [[g.numpy() for g in gt] for gt in gts]
+    else:
+        wh, gh = w0.copy(), [[g.copy() for g in grads[t]] for t in range(T)]
+    for t in range(T):
+        b.step_host(wh, gh[t], 0.02)
+    b.sync()
+    assert np.array_equal(wh.view(np.uint32), host(W).view(np.uint32))
+    for m in range(M):
+        x = torch.zeros(a.d, device="cuda")
+        y = torch.zeros(a.d, device="cuda")
+        a.get_momentum(m, x)
+        b.get_momentum(m, y)
+        assert torch.equal(x, y)
+
+
 @pytest.mark.parametrize("post_polar", [False, True])
 def test_signs_packed_in_gemm_match_kept_polar(post_polar):
     """With every column count a multiple of 32 the step packs the signs in
