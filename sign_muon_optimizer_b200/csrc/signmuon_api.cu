@@ -98,6 +98,8 @@ struct signmuon_ctx {
   cudaStream_t copy_stream = nullptr;
   cudaEvent_t g_ready[2] = {nullptr, nullptr};   // buffer b holds its call's gradients
   cudaEvent_t g_free[2] = {nullptr, nullptr};    // the step that read buffer b is done
+  cudaEvent_t w_ready = nullptr;                 // W of the current call is on the device
+  cudaEvent_t w_free = nullptr;                  // the previous call's W has gone back
   std::vector<void*> allocs;
   int64_t bytes = 0;
   std::string err;
@@ -693,6 +695,8 @@ void signmuon_destroy(signmuon_t h) {
     if (h->g_ready[b]) cudaEventDestroy(h->g_ready[b]);
     if (h->g_free[b]) cudaEventDestroy(h->g_free[b]);
   }
+  if (h->w_ready) cudaEventDestroy(h->w_ready);
+  if (h->w_free) cudaEventDestroy(h->w_free);
   for (cudaEvent_t e : h->ev_pool) cudaEventDestroy(e);
   for (void* q : h->allocs) cudaFree(q);
   if (h->h_status) cudaFreeHost(h->h_status);
@@ -1124,19 +1128,23 @@ int signmuon_step_host(signmuon_t h, float* W_host, const float* const* G_host, 
   for (int b = 0; b < 2; ++b)
     if (!h->hw_G[b] && (rc = dalloc(h, &h->hw_G[b], (int64_t)h->M * p.dpad))) return rc;
   if (!h->copy_stream) CK(h, cudaStreamCreateWithFlags(&h->copy_stream, cudaStreamNonBlocking));
-  for (int b = 0; b < 2; ++b) {
-    if (!h->g_ready[b]) CK(h, cudaEventCreateWithFlags(&h->g_ready[b], cudaEventDisableTiming));
-    if (!h->g_free[b]) {
-      CK(h, cudaEventCreateWithFlags(&h->g_free[b], cudaEventDisableTiming));
-      CK(h, cudaEventRecord(h->g_free[b], h->stream));
-    }
-  }
+  auto make_event = [&](cudaEvent_t* e, bool record) -> int {
+    if (*e) return SIGNMUON_OK;
+    CK(h, cudaEventCreateWithFlags(e, cudaEventDisableTiming));
+    if (record) CK(h, cudaEventRecord(*e, h->stream));
+    return SIGNMUON_OK;
+  };
+  for (int b = 0; b < 2; ++b)
+    if ((rc = make_event(&h->g_ready[b], false)) || (rc = make_event(&h->g_free[b], true))) return rc;
+  if ((rc = make_event(&h->w_ready, false)) || (rc = make_event(&h->w_free, true))) return rc;
   const int b = h->hw_next;
   h->hw_next ^= 1;
   cudaStream_t s = h->stream, cs = h->copy_stream;
-  // the gradients into buffer b on the copy stream, once the step that read
-  // it last (two calls ago) is done; with SIGNMUON_ASYNC they come in while
-  // the step of the call before still runs
+  // Every host-to-device copy goes on the copy stream: first the gradients
+  // into buffer b, once the step that read it last (two calls ago) is done;
+  // then W, once the previous call's W has gone back to the host.  With
+  // SIGNMUON_ASYNC the gradients come in while the step of the call before
+  // still runs, so the host-to-device link stays busy.
   CK(h, cudaStreamWaitEvent(cs, h->g_free[b], 0));
   std::vector<const float*> gd(h->M);
   for (int m = 0; m < h->M; ++m) {
@@ -1144,9 +1152,11 @@ int signmuon_step_host(signmuon_t h, float* W_host, const float* const* G_host, 
     CK(h, cudaMemcpyAsync(const_cast<float*>(gd[m]), G_host[m], (size_t)p.d * 4, cudaMemcpyHostToDevice, cs));
   }
   CK(h, cudaEventRecord(h->g_ready[b], cs));
-  // W after the previous call's copy back (stream order), then the step
-  CK(h, cudaMemcpyAsync(h->hw_W, W_host, (size_t)p.d * 4, cudaMemcpyHostToDevice, s));
+  CK(h, cudaStreamWaitEvent(cs, h->w_free, 0));
+  CK(h, cudaMemcpyAsync(h->hw_W, W_host, (size_t)p.d * 4, cudaMemcpyHostToDevice, cs));
+  CK(h, cudaEventRecord(h->w_ready, cs));
   CK(h, cudaStreamWaitEvent(s, h->g_ready[b], 0));
+  CK(h, cudaStreamWaitEvent(s, h->w_ready, 0));
   const unsigned saved = h->flags;
   h->flags |= SIGNMUON_ASYNC;
   rc = signmuon_step(h, h->hw_W, gd.data(), eta);
@@ -1154,6 +1164,7 @@ int signmuon_step_host(signmuon_t h, float* W_host, const float* const* G_host, 
   if (rc) return rc;
   CK(h, cudaEventRecord(h->g_free[b], s));
   CK(h, cudaMemcpyAsync(W_host, h->hw_W, (size_t)p.d * 4, cudaMemcpyDeviceToHost, s));
+  CK(h, cudaEventRecord(h->w_free, s));
   return (h->flags & SIGNMUON_ASYNC) ? SIGNMUON_OK : signmuon_sync(h);
 }
 
