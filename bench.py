@@ -719,25 +719,43 @@ def run_secondary(args):
                     ("after_only", smo.SIGNMUON_POST_POLAR | smo.SIGNMUON_POLAR_AFTER_ONLY, WL["P"]),
                     ("muon_mean", smo.SIGNMUON_MUON_MEAN, WL["P"]),
                     ("pi_warm_P1", base | smo.SIGNMUON_PI_WARM, 1), ("cold_P1", base, 1), ("split", base, WL["P"]),
-                    ("gram_space_ns", base | smo.SIGNMUON_NS_GRAM, WL["P"])]
+                    ("gram_space_ns", base | smo.SIGNMUON_NS_GRAM, WL["P"]),
+                    ("cuda_graph", base | smo.SIGNMUON_ASYNC, WL["P"])]
         W = synth.device_weights0(SHAPES, config_id=7)
         G = synth.device_gradients(SHAPES, M, WL["sigma"], step=0, config_id=7)
         gl = [G[m] for m in range(M)]
         for name, flags, P in variants:
+            # a graph is captured on a stream of its own (not the legacy default stream)
+            vs = torch.cuda.Stream() if name == "cuda_graph" else stream
             h = smo.SignMuon(SHAPES, M, beta=HP["beta"], lam=HP["lam"], K=K_NS, eps=HP["eps"], scale=WL["scale"],
-                             P=P, flags=flags, stream=stream.cuda_stream)
+                             P=P, flags=flags, stream=vs.cuda_stream)
             if name == "split":
                 buf = torch.empty(M * h.sign_stride(), dtype=torch.uint8, device="cuda")
 
                 def one():
                     h.local_signs(W, gl, buf)
                     h.vote_step(W, buf, M, HP["eta"])
+            elif name == "cuda_graph":
+                # the whole step captured once on the handle's stream, then replayed
+                h.step(W, gl, HP["eta"])
+                h.sync()
+                torch.cuda.synchronize()
+                graph = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(graph, stream=vs):
+                    h.step(W, gl, HP["eta"])
+
+                def one():
+                    with torch.cuda.stream(vs):
+                        graph.replay()
             else:
                 def one():
                     h.step(W, gl, HP["eta"])
-            ms = _events_time(one, 10, stream)
+            ms = _events_time(one, 10, vs)
             lines.append({"metric": f"Sign-Muon steps/s (nanoGPT-124M shapes, M=8, variant {name})",
                           "value": 1e3 / ms, "unit": "steps/s", "ms_per_step": ms, "flags": flags, "P": P})
+            if name == "cuda_graph":
+                h.sync()
+                del graph
             h.close()
         del W, G, gl
         torch.cuda.empty_cache()

@@ -59,7 +59,10 @@ typedef struct signmuon_ctx* signmuon_t;
 #define SIGNMUON_ACC_INT8    (1u << 3) /* int8 vote sums: signmuon_vote / signmuon_vote_ternary write
                                           them and signmuon_sums_step reads them (M <= 127) */
 #define SIGNMUON_ASYNC       (1u << 4) /* step, polar, local_signs, vote_step and sums_step do not
-                                          wait; signmuon_sync reports their status */
+                                          wait; signmuon_sync reports their status.  Such a step
+                                          makes no host synchronisation and no allocation, so it
+                                          can be captured into a CUDA graph on the handle's stream
+                                          (its pointers and eta are then fixed by the capture) */
 #define SIGNMUON_VOTE_ONLY   (1u << 5) /* allocate no step workspace: vote/pack/update calls only */
 #define SIGNMUON_KEEP_POLAR  (1u << 6) /* signmuon_step also writes U for signmuon_get_polar; without it
                                           the last Newton-Schulz GEMM of a step writes only the one-bit
