@@ -124,6 +124,10 @@ struct GemmArgs {
   const TileGroup* tiles;
   int n_tile_groups;
   int total_tiles;
+  // tensor-core launch: null for round robin (cluster c takes tiles c,
+  // c + clusters, ...), else [start of each cluster's list (clusters + 1
+  // entries), then the lists] from tile_schedule
+  const int* sched;
   const GroupInfo* groups;
   const int* group_mats;     // matrices of each group, in order
   const int64_t* mat_off;    // flat offset of each matrix

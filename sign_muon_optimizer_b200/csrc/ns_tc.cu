@@ -295,6 +295,17 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
 // hold the first four with 32-row boxes (an epilogue warp's operand atom).
 // The m x m buffers (A, B and the Gram-space A2, Q0, Q1) are addressed by
 // mm_slot(buffer, box).
+// The i-th tile of cluster cid (of ncl), or -1 past its last: round robin
+// over the launch's tile list, or the cluster's own list of a schedule.
+__device__ __forceinline__ int tile_at(const GemmArgs& a, int cid, int ncl, int i) {
+  if (a.sched == nullptr) {
+    const int t = cid + i * ncl;
+    return t < a.total_tiles ? t : -1;
+  }
+  const int s = __ldg(a.sched + cid) + i;
+  return s < __ldg(a.sched + cid + 1) ? __ldg(a.sched + ncl + 1 + s) : -1;
+}
+
 __device__ __forceinline__ const CUtensorMap* map_at(const CUtensorMap* maps, int group, int slot) {
   return maps + group * kMapsPerGroup + slot;
 }
@@ -365,7 +376,7 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
     uint32_t phase = 0;
     uint32_t issued = 0, last_par = 0;   // lane 0: stages this warp loaded, their parity
     bool ok = true;
-    for (int tile = cid; tile < a.total_tiles && ok; tile += ncl) {
+    for (int ti = 0, tile = tile_at(a, cid, ncl, 0); tile >= 0 && ok; tile = tile_at(a, cid, ncl, ++ti)) {
       const TileCoord tc = decode_tile(a, tile);
       const GroupInfo gi = group_info(a, tc.group);
       const int nk = (tc.Kdim + BK - 1) / BK;
@@ -473,8 +484,9 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
       bool pending_mma = false;     // MMAs issued since the last accumulator commit
       // the next tile is decoded while the current one's first MMAs run, so
       // that a tile boundary costs the MMA queue no decode time
-      TileCoord tn = decode_tile(a, cid < a.total_tiles ? cid : 0);
-      for (int tile = cid; tile < a.total_tiles && ok; tile += ncl) {
+      const int tile0 = tile_at(a, cid, ncl, 0);
+      TileCoord tn = decode_tile(a, tile0 >= 0 ? tile0 : 0);
+      for (int ti = 0, tile = tile0; tile >= 0 && ok; tile = tile_at(a, cid, ncl, ++ti)) {
         const TileCoord tc = tn;
         const GroupInfo gi = group_info(a, tc.group);
         const int nk = (tc.Kdim + BK - 1) / BK;
@@ -497,7 +509,10 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
           pending_mma = true;
           tc_commit_pair(empty_bar(stage));
           if (++stage == nst) { stage = 0; phase ^= 1u; }
-          if (kb == 0 && tile + ncl < a.total_tiles) tn = decode_tile(a, tile + ncl);
+          if (kb == 0) {
+            const int t2 = tile_at(a, cid, ncl, ti + 1);
+            if (t2 >= 0) tn = decode_tile(a, t2);
+          }
         }
         if (!ok) break;
         tc_commit_pair(tfull_bar(acc));
@@ -555,15 +570,17 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
     };
     uint32_t e_par = 0;          // phase of my operand barrier
     bool load_pending = false;   // an operand load is in flight
-    if (affine && cid < a.total_tiles) {
-      load_operand(decode_tile(a, cid), 0);
+    const int tile0 = tile_at(a, cid, ncl, 0);
+    if (affine && tile0 >= 0) {
+      load_operand(decode_tile(a, tile0), 0);
       load_pending = true;
     }
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int tile = cid; tile < a.total_tiles; tile += ncl) {
+    for (int it = 0, tile = tile0; tile >= 0; tile = tile_at(a, cid, ncl, ++it)) {
       const TileCoord tc = decode_tile(a, tile);
-      const bool more = tile + ncl < a.total_tiles;
+      const int tile_next = tile_at(a, cid, ncl, it + 1);
+      const bool more = tile_next >= 0;
       const GroupInfo gi = group_info(a, tc.group);
       int mat = 0;
       const int p = problem_id(a, gi, tc.b, &mat);
@@ -702,7 +719,7 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
             load_operand(tc, i + 1);
             load_pending = true;
           } else if (more) {
-            load_operand(decode_tile(a, tile + ncl), 0);
+            load_operand(decode_tile(a, tile_next), 0);
             load_pending = true;
           }
         }

@@ -4,6 +4,7 @@
 #include <algorithm>
 #include <climits>
 #include <map>
+#include <queue>
 #include <utility>
 
 #include "../../include/signmuon.h"
@@ -86,6 +87,46 @@ double tile_flops(const TileTable& tt) {
 }
 
 }  // namespace
+
+std::vector<int> tile_schedule(const TileTable& tt, int ncl, double* rr, double* greedy) {
+  std::vector<int> out;
+  if (rr) *rr = 0.0;
+  if (greedy) *greedy = 0.0;
+  if (tt.total <= 0 || ncl <= 0) return out;
+  std::vector<double> cost((size_t)tt.total);
+  for (const TileGroup& t : tt.groups) {
+    const int per = t.sym ? t.tiles_m * (t.tiles_m + 1) / 2 : t.tiles_m * t.tiles_n;
+    const double c = (double)((t.Kdim + 63) / 64) + 3.0;
+    for (int i = 0; i < per * t.batch; ++i) cost[(size_t)t.tile_start + i] = c;
+  }
+  std::vector<double> load_rr((size_t)ncl, 0.0), load_g((size_t)ncl, 0.0);
+  std::vector<std::vector<int>> lists((size_t)ncl);
+  // (load, cluster): the least-loaded cluster first, ties to the lower index
+  std::priority_queue<std::pair<double, int>, std::vector<std::pair<double, int>>, std::greater<>> q;
+  for (int c = 0; c < ncl; ++c) q.push({0.0, c});
+  for (int t = 0; t < tt.total; ++t) {
+    load_rr[(size_t)(t % ncl)] += cost[(size_t)t];
+    const auto [l, c] = q.top();
+    q.pop();
+    lists[(size_t)c].push_back(t);
+    load_g[(size_t)c] = l + cost[(size_t)t];
+    q.push({load_g[(size_t)c], c});
+  }
+  const double m_rr = *std::max_element(load_rr.begin(), load_rr.end());
+  const double m_g = *std::max_element(load_g.begin(), load_g.end());
+  if (rr) *rr = m_rr;
+  if (greedy) *greedy = m_g;
+  if (!(m_g < 0.97 * m_rr)) return out;
+  out.reserve((size_t)(ncl + 1 + tt.total));
+  int start = 0;
+  for (int c = 0; c < ncl; ++c) {
+    out.push_back(start);
+    start += (int)lists[(size_t)c].size();
+  }
+  out.push_back(start);
+  for (int c = 0; c < ncl; ++c) out.insert(out.end(), lists[(size_t)c].begin(), lists[(size_t)c].end());
+  return out;
+}
 
 int make_plan(const int64_t* shapes, int n_mats, int M, int K, int scale, int P, unsigned flags,
               Plan* plan, std::string* err) {

@@ -58,4 +58,15 @@ struct Plan {
 int make_plan(const int64_t* shapes, int n_mats, int M, int K, int scale, int P, unsigned flags,
               Plan* plan, std::string* err);
 
+// Tile schedule of one tensor-core GEMM launch over ncl clusters.  The
+// kernel's default is round robin (cluster c takes tiles c, c + ncl, ...).
+// With tiles of very different depth (the launch's list runs deepest first)
+// a greedy list schedule -- each tile, in list order, to the cluster with
+// the least work so far, a tile costing ceil(K / 64) + 3 k-blocks -- ends
+// sooner.  Returns the table [start of cluster 0 .. ncl (ncl + 1 entries),
+// then the clusters' tiles one after another], or an empty vector when the
+// greedy schedule's longest cluster is not at least 3 % shorter than round
+// robin's.  *rr and *greedy (if non-null) get the two makespans in k-blocks.
+std::vector<int> tile_schedule(const TileTable& tt, int ncl, double* rr, double* greedy);
+
 }  // namespace sm

@@ -57,6 +57,7 @@ struct signmuon_ctx {
   int* d_mat_nchunks = nullptr;
   int64_t* d_stage_off = nullptr;
   sm::TileGroup* d_tiles[3][2] = {{nullptr}};
+  int* d_sched[3][2] = {{nullptr}};   // tensor-core tile schedules (null: round robin)
   sm::PiTile* d_pi_tiles = nullptr;
   sm::PiSlice* d_pi_slices = nullptr;
   int64_t* d_uoff = nullptr;
@@ -315,6 +316,7 @@ void gemm(signmuon_t h, int op, int slot, int src, int nw, const float2* coef, f
   const Plan& p = h->plan;
   sm::GemmArgs a{};
   a.tiles = h->d_tiles[op][slot];
+  a.sched = h->d_sched[op][slot];
   a.n_tile_groups = (int)p.tiles[op][slot].groups.size();
   a.total_tiles = p.tiles[op][slot].total;
   a.groups = h->d_groups;
@@ -658,6 +660,22 @@ int signmuon_plan_tables(const int64_t* shapes, int n_mats, int M, int K, int sc
       if (i) j += ',';
       tuple({x.group, x.Mdim, x.Ndim, x.Kdim, x.BM, x.BN, x.sym, x.tiles_m, x.tiles_n, x.batch, x.tile_start});
     }
+    // the tensor-core launch's schedule for a 148-SM B200 (74 clusters),
+    // empty for round robin, and both makespans in k-blocks
+    const int ncl = std::min(t.total, 74);
+    double rr = 0.0, greedy = 0.0;
+    const std::vector<int> sched = sm::tile_schedule(t, ncl, &rr, &greedy);
+    j += "],\"clusters\":";
+    num(ncl);
+    j += ",\"makespan_rr\":";
+    num((int64_t)rr);
+    j += ",\"makespan_greedy\":";
+    num((int64_t)greedy);
+    j += ",\"sched\":[";
+    for (size_t i = 0; i < sched.size(); ++i) {
+      if (i) j += ',';
+      num(sched[i]);
+    }
     j += "]}";
   });
   list("pi_tiles", p.pi_tiles.size(), [&](size_t i) {
@@ -753,8 +771,16 @@ int signmuon_init(signmuon_t* out, const int64_t* shapes, int n_mats, int M, flo
   if ((rc = upload(h, &h->d_mat_nchunks, p.mat_nchunks))) return bail(rc);
   if ((rc = upload(h, &h->d_stage_off, p.stage_off))) return bail(rc);
   for (int op = 0; op < 3; ++op)
-    for (int s = 0; s < 2; ++s)
+    for (int s = 0; s < 2; ++s) {
       if ((rc = upload(h, &h->d_tiles[op][s], p.tiles[op][s].groups))) return bail(rc);
+      // a launch of the tensor-core kernel runs min(tiles, SMs / 2) clusters
+      const int total = p.tiles[op][s].total;
+      const int ncl = std::min(total, h->n_sm / 2);
+      if (!p.fp32 && ncl > 0) {
+        const std::vector<int> sched = sm::tile_schedule(p.tiles[op][s], ncl, nullptr, nullptr);
+        if (!sched.empty() && (rc = upload(h, &h->d_sched[op][s], sched))) return bail(rc);
+      }
+    }
   if ((rc = upload(h, &h->d_pi_tiles, p.pi_tiles))) return bail(rc);
   if ((rc = upload(h, &h->d_pi_slices, p.pi_slices))) return bail(rc);
   if ((rc = upload(h, &h->d_uoff, p.uoff))) return bail(rc);
