@@ -223,8 +223,8 @@ void launch_gram_q1(cudaStream_t s, int n_probs, const void* A, void* Q, const i
 // warm != 0: keep each problem's stored iterate when it is non-zero and finite
 void launch_pi_init(cudaStream_t s, int n_probs, const int64_t* uoff, const int* prob_g, float* u, int warm);
 // one pass over the upper-triangle tiles, one block per tile: partial sums
-// of A v, v = src (fold = 0) or v = src * inv[p] (fold = 1, which also stores
-// v into u)
+// of A v, v = src (fold = 0; src == nullptr: v = ones / sqrt(g)) or
+// v = src * inv[p] (fold = 1, which also stores v into u)
 void launch_pi_tiles(cudaStream_t s, const PiTile* tiles, int n_tiles, const void* A, int a_bf16,
                      const float* src, const float* inv, float* u, float* part, int fold);
 // y = the sum of each slice's partials in a fixed order; per problem 1 / ||y||

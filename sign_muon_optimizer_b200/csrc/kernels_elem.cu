@@ -368,14 +368,16 @@ k_pi_tiles(const PiTile* __restrict__ tiles, const void* __restrict__ A, const f
     asm volatile("cp.async.commit_group;" ::: "memory");
   }
   {
+    // src == nullptr: a cold start, v = u0 = ones / sqrt(g) (no stored vector)
     const float sc = fold ? inv[tl.p] : 1.f;
+    const float v0 = rsqrtf((float)g);
     const int k = threadIdx.x & (T - 1);
     if (threadIdx.x < T) {
-      const float v = (r0 + k < g) ? src[tl.uoff + r0 + k] * sc : 0.f;
+      const float v = (r0 + k < g) ? (src ? src[tl.uoff + r0 + k] * sc : v0) : 0.f;
       vi[k] = v;
       if (fold && diag && r0 + k < g) u[tl.uoff + r0 + k] = v;  // the normalised iterate, once per slice
     } else {
-      vj[k] = (c0 + k < g) ? src[tl.uoff + c0 + k] * sc : 0.f;
+      vj[k] = (c0 + k < g) ? (src ? src[tl.uoff + c0 + k] * sc : v0) : 0.f;
     }
   }
   asm volatile("cp.async.wait_group 0;" ::: "memory");

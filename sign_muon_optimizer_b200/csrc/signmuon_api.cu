@@ -378,9 +378,11 @@ void power_iteration(signmuon_t h, int nw) {
                          h->ns_c, h->scale_v, h->coef_apply, h->coef_square, h->coef_gram, h->status};
   sm::PiReduce fin = mid;
   fin.last = 1;
-  // u0; then y = A u0; then P times y = A (y / ||y||), storing y / ||y|| as u
-  sm::launch_pi_init(h->stream, nprob, h->d_uoff, h->d_prob_g, u, warm ? 1 : 0);
-  sm::launch_pi_tiles(h->stream, h->d_pi_tiles, ntiles, h->A, bf16, u, nullptr, u, h->pi_part, 0);
+  // y = A u0 (a cold start stages u0 = ones / sqrt(g) in the first pass
+  // itself; a warm one keeps the stored iterate when it is usable); then P
+  // times y = A (y / ||y||), storing y / ||y|| as u
+  if (warm) sm::launch_pi_init(h->stream, nprob, h->d_uoff, h->d_prob_g, u, 1);
+  sm::launch_pi_tiles(h->stream, h->d_pi_tiles, ntiles, h->A, bf16, warm ? u : nullptr, nullptr, u, h->pi_part, 0);
   for (int it = 0; it < h->P; ++it) {
     sm::launch_pi_reduce(h->stream, h->d_pi_slices, nslices, h->pi_part, h->pi_y, mid);
     sm::launch_pi_tiles(h->stream, h->d_pi_tiles, ntiles, h->A, bf16, h->pi_y, h->pi_inv, u, h->pi_part, 1);
