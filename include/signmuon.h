@@ -385,7 +385,8 @@ int signmuon_plan(const int64_t* shapes, int n_mats, int M, int K, int scale, in
  * the planner without a GPU.  The tables are the shape groups and their
  * buffer bases, the matrices, the 4096-entry chunks of the elementwise
  * kernels, the GEMM tile lists per op (Gram, quintic square, apply) for M
- * workers and for one, the power-iteration tiles (the 128 x 128 tiles on and
+ * workers and for one, each with its tensor-core schedule for a 148-SM B200
+ * (empty for round robin) and both makespans, the power-iteration tiles (the 128 x 128 tiles on and
  * above each Gram's diagonal), row slices, vector and partial-sum offsets, and
  * the buffer sizes.  *need receives the text's size in bytes, with the
  * terminating NUL.  buf may be NULL to ask for the size; a non-NULL buf
