@@ -146,6 +146,20 @@ def test_step_post_polar_streamed_stage(M):
     _compare_step(shapes, M, gpu, want, "bf16", True)
 
 
+@pytest.mark.parametrize("M", [1, 2])
+@pytest.mark.parametrize("post_polar", [False, True])
+def test_step_one_and_two_workers(M, post_polar):
+    """The vote's two smallest cases: one worker (the majority is its own
+    sign, no tie possible) and two (every disagreement is a tie and maps to
+    zero), with and without the post-vote polar step.  With so few workers
+    no other vote hides a sign that rounding flipped, so the comparison runs
+    on the fp32 path, where the majority of a whole matrix can match the
+    oracle's exactly (the post-vote check needs one such matrix)."""
+    shapes = [(130, 70), (64, 147), (96, 300), (8, 8)]
+    h, gpu, want = _run_one_step(shapes, M, 1.0, 5, "spectral", 2, "fp32", post_polar, seed=61 + M)
+    _compare_step(shapes, M, gpu, want, "fp32", post_polar)
+
+
 def test_step_quintic_fp32():
     shapes = [(64, 96), (96, 64)]
     h, gpu, want = _run_one_step(shapes, 2, 1.0, 3, "spectral", 2, "fp32", False, seed=5, order="quintic")
