@@ -163,6 +163,10 @@ struct GemmArgs {
   int final_out;
   uint32_t* out_bits;
   int64_t bits_stride;       // in 32-bit words
+  // (bf16 path) when non-null, the ternary signs sign(U) in {-1, 0, +1} as
+  // int8 at out_sign8 + worker*sign8_stride + flat index
+  int8_t* out_sign8;
+  int64_t sign8_stride;
   int* err;
   int param_tables;                        // 1: the p* copies below are valid
   TileGroup ptiles[kParamGroups];

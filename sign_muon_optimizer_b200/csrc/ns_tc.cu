@@ -253,6 +253,29 @@ __device__ __forceinline__ void store_row_chunk(__nv_bfloat16* p, int n, const u
   }
 }
 // the first n (1..32) of 32 floats to p (any 4-byte alignment)
+// The ternary signs (v > 0) - (v < 0) of a chunk's n <= 32 entries as int8
+// (0 for a zero or NaN, as the ternary sign kernel gives them).
+__device__ __forceinline__ int8_t tsign8(float f) { return (int8_t)((f > 0.f) - (f < 0.f)); }
+__device__ __forceinline__ void store_row_sign8(int8_t* p, int n, const float (&v)[32]) {
+  if (n >= 32 && (reinterpret_cast<uintptr_t>(p) & 15u) == 0) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint32_t w[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int e = 16 * h + 4 * k;
+        w[k] = (uint32_t)(uint8_t)tsign8(v[e]) | (uint32_t)(uint8_t)tsign8(v[e + 1]) << 8 |
+               (uint32_t)(uint8_t)tsign8(v[e + 2]) << 16 | (uint32_t)(uint8_t)tsign8(v[e + 3]) << 24;
+      }
+      *reinterpret_cast<uint4*>(p + 16 * h) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    return;
+  }
+#pragma unroll
+  for (int u = 0; u < 32; ++u)
+    if (u < n) p[u] = tsign8(v[u]);
+}
+
 __device__ __forceinline__ void store_row_f32(float* p, int n, const float (&v)[32]) {
   const uintptr_t al = reinterpret_cast<uintptr_t>(p);
   if (n >= 32 && (al & 31u) == 0) {
@@ -682,6 +705,10 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
 #pragma unroll
               for (int u = 0; u < 32; ++u) word |= (v[u] >= 0.f ? 1u : 0u) << u;
               a.out_bits[(int64_t)w * a.bits_stride + (flat >> 5)] = word;
+            }
+            if (live && a.out_sign8 != nullptr) {
+              store_row_sign8(a.out_sign8 + (int64_t)w * a.sign8_stride + a.mat_off[mat] + (int64_t)row * gi.cols + col0,
+                              ncol, v);
             }
             if (live && a.out != nullptr) {
               float* dst = a.out + (int64_t)w * a.out_stride + a.mat_off[mat] + (int64_t)row * gi.cols + col0;

@@ -91,6 +91,10 @@ struct signmuon_ctx {
   int* status = nullptr;        // [0] non-finite flag, [1] kernel error code
   int* h_status = nullptr;      // pinned mirror
   bool pending = false;         // an async step's status not yet read
+  // the ternary signs of the step's last Newton-Schulz GEMM (bf16 path): set
+  // by local_part around its run_ns, read by gemm() for the final apply
+  int8_t* final_sign8 = nullptr;
+  int64_t final_sign8_stride = 0;
   // step_host staging: W, and two gradient buffers so that a call's
   // gradients can come in (on the copy stream) while the step before runs
   float* hw_W = nullptr;
@@ -346,6 +350,10 @@ void gemm(signmuon_t h, int op, int slot, int src, int nw, const float2* coef, f
   a.final_out = final_out ? 1 : 0;
   a.out_bits = out_bits;
   a.bits_stride = bits_stride;
+  if (final_out && op == sm::OP_APPLY) {
+    a.out_sign8 = h->final_sign8;
+    a.sign8_stride = h->final_sign8_stride;
+  }
   a.err = h->status + 1;
   (void)nw;
   const auto& tg = p.tiles[op][slot].groups;
@@ -939,11 +947,20 @@ static void local_part(signmuon_t h, const float* W, const sm::WorkerPtrs& gp, u
   // every matrix has a multiple of 32 columns (then each 32-column chunk of an
   // output row is one aligned word of the bit stream; K > 0, bf16 path); U is
   // written only when kept for get_polar.
+  // The int8 ternary signs come out of the last GEMM on the bf16 path (any
+  // shapes: a chunk's 32 signs are stored bytewise where unaligned).
   const bool fused = !ternary && signs_in_gemm(h);
-  h->u_valid = !fused || (h->flags & SIGNMUON_KEEP_POLAR) != 0;
+  const bool fused8 = ternary && !p.fp32 && h->K > 0;
+  h->u_valid = !(fused || fused8) || (h->flags & SIGNMUON_KEEP_POLAR) != 0;
   if (fused) {
     run_ns(h, h->K, h->M, strided_ptrs(h->Mom, p.dpad, h->M), h->u_valid ? h->U : nullptr, p.dpad,
            reinterpret_cast<uint32_t*>(dst), stride / 4);
+  } else if (fused8) {
+    h->final_sign8 = dst8;
+    h->final_sign8_stride = stride;
+    run_ns(h, h->K, h->M, strided_ptrs(h->Mom, p.dpad, h->M), h->u_valid ? h->U : nullptr, p.dpad);
+    h->final_sign8 = nullptr;
+    h->final_sign8_stride = 0;
   } else {
     run_ns(h, h->K, h->M, strided_ptrs(h->Mom, p.dpad, h->M), h->U, p.dpad);
     ProfScope ps(h, 6);

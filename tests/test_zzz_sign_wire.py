@@ -101,6 +101,8 @@ def test_vote_ternary_blog_worked_example_and_empty():
 
 def _ternary_step(shapes, M, K, scale, P, precision, extra, seed, tie=0):
     flags = smo.SIGNMUON_TERNARY | (smo.SIGNMUON_NS_FP32 if precision == "fp32" else 0) | extra
+    if not extra & smo.SIGNMUON_POLAR_AFTER_ONLY:
+        flags |= smo.SIGNMUON_KEEP_POLAR   # U is read back below
     if tie:
         flags |= smo.SIGNMUON_TIE_PLUS
     h = smo.SignMuon(shapes, M, beta=HP["beta"], lam=HP["lam"], K=K, eps=HP["eps"], scale=scale, P=P, flags=flags)
@@ -320,3 +322,51 @@ def test_step_normalized_sign_closed_forms(precision):
         assert np.array_equal(got == 0, p == 0), f"permutation {r}x{c}: zeros moved"
         assert np.max(np.abs(got - p / (1.0 + eps))) <= 1e-5, f"permutation {r}x{c}"
         off += r * c
+
+
+@pytest.mark.parametrize("post_polar", [False, True])
+def test_ternary_signs_in_gemm_match_kept_polar(post_polar):
+    """On the bf16 path the int8 ternary signs come out of the last
+    Newton-Schulz GEMM's epilogue, and U is written only with
+    SIGNMUON_KEEP_POLAR.  Two handles, one keeping U, run the same step:
+    their signs, directions and W must be identical, the signs must be
+    sign(U) of the kept U (0 for an exact zero), and get_polar of the handle
+    that kept nothing must refuse.  Ragged shapes: rows whose 32-column
+    chunks start at unaligned flat offsets take the bytewise stores."""
+    shapes = [(3, 5), (130, 70), (64, 147), (96, 300), (256, 512)]
+    M, seed = 4, 83
+    base = smo.SIGNMUON_TERNARY | (smo.SIGNMUON_POST_POLAR if post_polar else 0)
+    d = synth.numel(shapes)
+    w0 = synth.weights0(shapes, seed)
+    mom0 = synth.momentum0(shapes, M, seed, scale=0.5)
+    G = synth.gradients(shapes, M, 1.0, step=1, config_id=seed)
+    out = {}
+    for keep in (True, False):
+        h = smo.SignMuon(shapes, M, beta=HP["beta"], lam=HP["lam"], K=5, eps=HP["eps"], scale="spectral", P=2,
+                         flags=base | (smo.SIGNMUON_KEEP_POLAR if keep else 0))
+        for m in range(M):
+            h.set_momentum(m, dev(mom0[m]))
+        W = dev(w0)
+        h.step(W, [dev(g) for g in G], HP["eta"])
+        t = []
+        for m in range(M):
+            s = torch.full((d,), 7, dtype=torch.int8, device="cuda")
+            h.get_ternary_signs(m, s)
+            t.append(host(s))
+        D = torch.zeros(d, device="cuda")
+        h.get_direction(D)
+        U = []
+        if keep:
+            for m in range(M):
+                x = torch.zeros(d, device="cuda")
+                h.get_polar(m, x)
+                U.append(host(x))
+        else:
+            with pytest.raises(smo.SignMuonError):
+                h.get_polar(0, torch.zeros(d, device="cuda"))
+        out[keep] = dict(t=t, D=host(D), W=host(W), U=U)
+    for m in range(M):
+        assert np.array_equal(out[True]["t"][m], out[False]["t"][m])
+        assert np.array_equal(out[True]["t"][m], np.sign(out[True]["U"][m]).astype(np.int8))
+    assert np.array_equal(out[True]["D"].view(np.uint32), out[False]["D"].view(np.uint32))
+    assert np.array_equal(out[True]["W"].view(np.uint32), out[False]["W"].view(np.uint32))
