@@ -65,8 +65,8 @@ typedef struct signmuon_ctx* signmuon_t;
                                           (its pointers and eta are then fixed by the capture) */
 #define SIGNMUON_VOTE_ONLY   (1u << 5) /* allocate no step workspace: vote/pack/update calls only */
 #define SIGNMUON_KEEP_POLAR  (1u << 6) /* signmuon_step also writes U for signmuon_get_polar; without it
-                                          the last Newton-Schulz GEMM of a step writes only the one-bit
-                                          signs when every matrix has a multiple of 32 columns */
+                                          the last Newton-Schulz GEMM of a bf16 step (K > 0) writes
+                                          only the signs (one-bit, or int8 with SIGNMUON_TERNARY) */
 /* Named variants ([paper] "SignMuon: 通信高效的分布式Muon优化" Algorithm 2, §4, Table 1):
  * TIE_PLUS           a tied vote (sum 0, even M) gives +1 instead of 0 (Algorithm 2's sign
  *                    default on the {-1, +1} wire); applies to signmuon_vote's majority and

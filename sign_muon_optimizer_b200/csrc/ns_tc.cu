@@ -698,13 +698,22 @@ k_gemm_tc(const __grid_constant__ GemmArgs a, const CUtensorMap* __restrict__ ma
           const int ncol = live ? min(32, tc.Ndim - col0) : 0;
           if (final_out) {
             if (live && a.out_bits != nullptr) {
-              // one LSB-first word of the bit stream (every matrix has a
-              // multiple of 32 columns when the signs are packed here)
+              // the chunk's ncol signs (U >= 0), LSB-first from its flat
+              // index: one word of the bit stream when that is a multiple of
+              // 32 and the chunk is whole, else OR-ed into the two words it
+              // straddles (the buffer was zeroed for such shapes)
               const int64_t flat = a.mat_off[mat] + (int64_t)row * gi.cols + col0;
               uint32_t word = 0;
 #pragma unroll
-              for (int u = 0; u < 32; ++u) word |= (v[u] >= 0.f ? 1u : 0u) << u;
-              a.out_bits[(int64_t)w * a.bits_stride + (flat >> 5)] = word;
+              for (int u = 0; u < 32; ++u) word |= (u < ncol && v[u] >= 0.f ? 1u : 0u) << u;
+              uint32_t* wp = a.out_bits + (int64_t)w * a.bits_stride + (flat >> 5);
+              const int sh = (int)(flat & 31);
+              if (sh == 0 && ncol == 32) {
+                *wp = word;
+              } else {
+                atomicOr(wp, word << sh);
+                if (sh != 0 && ncol + sh > 32) atomicOr(wp + 1, word >> (32 - sh));
+              }
             }
             if (live && a.out_sign8 != nullptr) {
               store_row_sign8(a.out_sign8 + (int64_t)w * a.sign8_stride + a.mat_off[mat] + (int64_t)row * gi.cols + col0,

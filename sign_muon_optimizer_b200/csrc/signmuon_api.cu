@@ -408,12 +408,20 @@ bool stage_streamable(signmuon_t h) {
   return true;
 }
 
+// The one-bit signs come out of the last Newton-Schulz GEMM on the bf16
+// path (K > 0).  Every 32-column chunk of an output row is then one aligned
+// word of the bit stream when every matrix has a multiple of 32 columns;
+// otherwise chunks that straddle words OR their bits in, and the buffer is
+// zeroed first (signs_ragged).
 bool signs_in_gemm(signmuon_t h) {
   const Plan& p = h->plan;
-  if (p.fp32 || h->K == 0 || (p.nb_pad % 4) != 0) return false;
-  for (const sm::GroupInfo& gi : p.groups)
-    if (gi.cols % 32 != 0) return false;
-  return true;
+  return !p.fp32 && h->K > 0 && (p.nb_pad % 4) == 0;
+}
+
+bool signs_ragged(signmuon_t h) {
+  for (const sm::GroupInfo& gi : h->plan.groups)
+    if (gi.cols % 32 != 0) return true;
+  return false;
 }
 
 void run_ns(signmuon_t h, int K, int nw, const sm::WorkerPtrs& kzero_in, float* out, int64_t out_stride,
@@ -943,16 +951,16 @@ static void local_part(signmuon_t h, const float* W, const sm::WorkerPtrs& gp, u
     else sm::launch_pack(s, h->Mom, p.dpad, p.d, dst, stride, h->M);
     return;
   }
-  // The one-bit signs come out of the last Newton-Schulz GEMM itself when
-  // every matrix has a multiple of 32 columns (then each 32-column chunk of an
-  // output row is one aligned word of the bit stream; K > 0, bf16 path); U is
-  // written only when kept for get_polar.
+  // The one-bit signs come out of the last Newton-Schulz GEMM itself (K > 0,
+  // bf16 path, see signs_in_gemm); U is written only when kept for get_polar.
   // The int8 ternary signs come out of the last GEMM on the bf16 path (any
   // shapes: a chunk's 32 signs are stored bytewise where unaligned).
   const bool fused = !ternary && signs_in_gemm(h);
   const bool fused8 = ternary && !p.fp32 && h->K > 0;
   h->u_valid = !(fused || fused8) || (h->flags & SIGNMUON_KEEP_POLAR) != 0;
   if (fused) {
+    // (an error here is the runtime's last error, which the step's status read reports)
+    if (signs_ragged(h)) cudaMemsetAsync(dst, 0, (size_t)h->M * (size_t)stride, s);
     run_ns(h, h->K, h->M, strided_ptrs(h->Mom, p.dpad, h->M), h->u_valid ? h->U : nullptr, p.dpad,
            reinterpret_cast<uint32_t*>(dst), stride / 4);
   } else if (fused8) {

@@ -288,14 +288,18 @@ def test_step_host_async_pipeline_matches_device_steps(pinned):
         assert torch.equal(x, y)
 
 
+@pytest.mark.parametrize("ragged", [False, True])
 @pytest.mark.parametrize("post_polar", [False, True])
-def test_signs_packed_in_gemm_match_kept_polar(post_polar):
-    """With every column count a multiple of 32 the step packs the signs in
-    the last Newton-Schulz GEMM; without SIGNMUON_KEEP_POLAR it writes no U.
+def test_signs_packed_in_gemm_match_kept_polar(post_polar, ragged):
+    """The bf16 step packs the one-bit signs in the last Newton-Schulz GEMM;
+    without SIGNMUON_KEEP_POLAR it writes no U.  With every column count a
+    multiple of 32 each 32-column chunk is one word of the bit stream; with
+    ragged column counts chunks straddle words and OR their bits into both.
     Both handles run the same step: the packed signs, the direction and W
     must be identical, the signs must be U >= 0 of the kept U, and get_polar
     of the handle that kept nothing must refuse."""
-    shapes = [(256, 512), (512, 256), (96, 160), (384, 384)]
+    shapes = ([(3, 5), (130, 70), (64, 147), (96, 300), (256, 512), (33, 31)] if ragged
+              else [(256, 512), (512, 256), (96, 160), (384, 384)])
     M, seed = 4, 23
     base = smo.SIGNMUON_POST_POLAR if post_polar else 0
     d = synth.numel(shapes)
