@@ -167,7 +167,9 @@ int signmuon_step(signmuon_t h, float* W, const float* const* G, float eta);
  *           packed bytes (LSB-first, as signmuon_pack), or d int8 ternary
  *           signs with SIGNMUON_TERNARY.
  *   stride  bytes between workers: a multiple of 16, at least one worker's
- *           signs.
+ *           signs.  The call may zero the whole M*stride bytes (packed signs
+ *           of matrices whose column counts are not multiples of 32 are OR-ed
+ *           into a zeroed buffer).
  * Unless SIGNMUON_ASYNC, waits and returns E_NONFINITE when a momentum norm is
  * NaN/Inf (the signs are then not valid: do not vote on them).  Not for
  * MUON_MEAN handles (E_UNSUPPORTED).
