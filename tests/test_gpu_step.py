@@ -288,7 +288,7 @@ def test_step_host_async_pipeline_matches_device_steps(pinned):
         assert torch.equal(x, y)
 
 
-@pytest.mark.parametrize("ragged", [False, True])
+@pytest.mark.parametrize("ragged", [False, True, "gram"])
 @pytest.mark.parametrize("post_polar", [False, True])
 def test_signs_packed_in_gemm_match_kept_polar(post_polar, ragged):
     """The bf16 step packs the one-bit signs in the last Newton-Schulz GEMM;
@@ -298,10 +298,18 @@ def test_signs_packed_in_gemm_match_kept_polar(post_polar, ragged):
     Both handles run the same step: the packed signs, the direction and W
     must be identical, the signs must be U >= 0 of the kept U, and get_polar
     of the handle that kept nothing must refuse."""
-    shapes = ([(3, 5), (130, 70), (64, 147), (96, 300), (256, 512), (33, 31)] if ragged
-              else [(256, 512), (512, 256), (96, 160), (384, 384)])
+    if ragged == "gram":
+        # SIGNMUON_NS_GRAM: the final product X_K = Q_K X0 packs the signs
+        # (1000 columns: ragged chunks)
+        shapes = [(300, 1000), (3072, 768), (520, 1600)]
+    elif ragged:
+        shapes = [(3, 5), (130, 70), (64, 147), (96, 300), (256, 512), (33, 31)]
+    else:
+        shapes = [(256, 512), (512, 256), (96, 160), (384, 384)]
     M, seed = 4, 23
-    base = smo.SIGNMUON_POST_POLAR if post_polar else 0
+    base = (smo.SIGNMUON_POST_POLAR if post_polar else 0) | (smo.SIGNMUON_NS_GRAM if ragged == "gram" else 0)
+    if ragged == "gram":
+        assert smo.signmuon_plan_tables(shapes, M, 5, "spectral", 2, base)["gram_ns"] == 1
     d = synth.numel(shapes)
     w0 = synth.weights0(shapes, seed)
     mom0 = synth.momentum0(shapes, M, seed, scale=0.5)
