@@ -819,16 +819,20 @@ def run_collectives(args):
 def run_capture(args):
     """Profiler-capture mode (prints no bench line): the same step on the first
     L transformer layers of the nanoGPT shapes, M=8, a few steps.  Variants:
-    "ternary" sends int8 ternary signs (the sign8 and ternary vote kernels);
-    "unpacked" adds a 48-column matrix, so that no sign can be packed inside
-    the GEMM and the pack kernel runs."""
+    "ternary" sends int8 ternary signs (written by the last GEMM, then the
+    ternary vote kernels); "ragged" adds a 48-column matrix, so that the last
+    GEMM's 32-column chunks straddle words of the bit stream (OR-ed in);
+    "fp32" and "ternary-fp32" run the fp32 Newton-Schulz path, whose signs
+    come from the pack and ternary sign kernels."""
     import torch
     import sign_muon_optimizer_b200 as smo
     shapes = SHAPES[: 4 * args.capture_layers]
     flags = smo.SIGNMUON_POST_POLAR if WL["post_polar"] else 0
-    if args.capture_variant == "ternary":
+    if args.capture_variant in ("ternary", "ternary-fp32"):
         flags |= smo.SIGNMUON_TERNARY
-    elif args.capture_variant == "unpacked":
+    if args.capture_variant in ("fp32", "ternary-fp32"):
+        flags |= smo.SIGNMUON_NS_FP32
+    if args.capture_variant == "ragged":
         shapes = shapes + [(768, 48)]
     opt = smo.SignMuon(shapes, M, beta=HP["beta"], lam=HP["lam"], K=K_NS, eps=HP["eps"], scale=WL["scale"],
                        P=WL["P"], flags=flags)
@@ -854,7 +858,7 @@ def main():
                     help="skip the short passes of the ResNet-50, LLaMA-layer vote and NS sweep configurations")
     ap.add_argument("--capture-layers", type=int, default=0,
                     help="profiler capture mode on the first L layers; prints no bench line")
-    ap.add_argument("--capture-variant", default="nanogpt", choices=["nanogpt", "ternary", "unpacked"])
+    ap.add_argument("--capture-variant", default="nanogpt", choices=["nanogpt", "ternary", "ragged", "fp32", "ternary-fp32"])
     ap.add_argument("--workload", default="nanogpt",
                     choices=["nanogpt", "llama_vote", "vote_100m", "ns_sweep", "ns_sweep_full", "resnet50",
                              "ternary_vote", "variants", "collectives", "cublas", "all"],
