@@ -370,3 +370,70 @@ def test_ternary_signs_in_gemm_match_kept_polar(post_polar):
         assert np.array_equal(out[True]["t"][m], np.sign(out[True]["U"][m]).astype(np.int8))
     assert np.array_equal(out[True]["D"].view(np.uint32), out[False]["D"].view(np.uint32))
     assert np.array_equal(out[True]["W"].view(np.uint32), out[False]["W"].view(np.uint32))
+
+
+@pytest.mark.parametrize("case", ["quintic-ternary", "quintic-ragged", "gram-ternary", "tieplus-ternary-post"])
+def test_epilogue_signs_across_flag_combinations(case):
+    """The signs written by the last GEMM's epilogue under flag combinations:
+    quintic with the ternary wire, quintic with one-bit signs of ragged
+    column counts, the Gram-space iteration with the ternary wire, and tie to
+    +1 with the ternary wire and the post-vote polar step.  A handle that
+    keeps U and one that does not run the same step: their signs, directions
+    and W must be identical, and the signs must be those of the kept U (the
+    one-bit bit = U >= 0, the ternary sign(U)); the kept U must be the
+    oracle's polar factor within the bf16 tolerance."""
+    flags = {"quintic-ternary": smo.SIGNMUON_NS_QUINTIC | smo.SIGNMUON_TERNARY,
+             "quintic-ragged": smo.SIGNMUON_NS_QUINTIC,
+             "gram-ternary": smo.SIGNMUON_NS_GRAM | smo.SIGNMUON_TERNARY,
+             "tieplus-ternary-post": smo.SIGNMUON_TIE_PLUS | smo.SIGNMUON_TERNARY | smo.SIGNMUON_POST_POLAR}[case]
+    shapes = ([(300, 1000), (3072, 768), (520, 1600)] if case.startswith("gram")
+              else [(3, 5), (130, 70), (64, 147), (96, 300), (256, 512)])
+    order = "quintic" if case.startswith("quintic") else "cubic"
+    ternary = bool(flags & smo.SIGNMUON_TERNARY)
+    M, seed = 4, 97
+    if case.startswith("gram"):
+        assert smo.signmuon_plan_tables(shapes, M, 5, "spectral", 2, flags)["gram_ns"] == 1
+    d = synth.numel(shapes)
+    w0 = synth.weights0(shapes, seed)
+    mom0 = synth.momentum0(shapes, M, seed, scale=0.5)
+    G = synth.gradients(shapes, M, 1.0, step=1, config_id=seed)
+    out = {}
+    for keep in (True, False):
+        h = smo.SignMuon(shapes, M, beta=HP["beta"], lam=HP["lam"], K=5, eps=HP["eps"], scale="spectral", P=2,
+                         flags=flags | (smo.SIGNMUON_KEEP_POLAR if keep else 0))
+        for m in range(M):
+            h.set_momentum(m, dev(mom0[m]))
+        W = dev(w0)
+        h.step(W, [dev(g) for g in G], HP["eta"])
+        sg, U, mom = [], [], []
+        for m in range(M):
+            if ternary:
+                s = torch.full((d,), 7, dtype=torch.int8, device="cuda")
+                h.get_ternary_signs(m, s)
+            else:
+                s = torch.zeros(ref.packed_nbytes(d), dtype=torch.uint8, device="cuda")
+                h.get_signs(m, s)
+            sg.append(host(s))
+            if keep:
+                x = torch.zeros(d, device="cuda")
+                h.get_polar(m, x)
+                U.append(host(x))
+                y = torch.zeros(d, device="cuda")
+                h.get_momentum(m, y)
+                mom.append(host(y))
+        D = torch.zeros(d, device="cuda")
+        h.get_direction(D)
+        out[keep] = dict(s=sg, U=U, mom=mom, D=host(D), W=host(W))
+    for m in range(M):
+        assert np.array_equal(out[True]["s"][m], out[False]["s"][m])
+        u = out[True]["U"][m]
+        if ternary:
+            assert np.array_equal(out[True]["s"][m], np.sign(u).astype(np.int8))
+        else:
+            want = np.packbits(u >= 0, bitorder="little")
+            assert np.array_equal(out[True]["s"][m][: want.size], want)
+        teacher = oracle_polar_flat(out[True]["mom"][m].astype(np.float64), shapes, 5, HP["eps"], "spectral", 2,
+                                    order)
+        assert_polar_close(u, teacher, "bf16", f"{case} worker {m}")
+    assert np.array_equal(out[True]["D"].view(np.uint32), out[False]["D"].view(np.uint32))
+    assert np.array_equal(out[True]["W"].view(np.uint32), out[False]["W"].view(np.uint32))
