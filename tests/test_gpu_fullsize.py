@@ -444,3 +444,36 @@ def test_ns_sweep_8192_known_polar_factor(order, K, precision):
     # a sharper bound than the absolute tolerance at this entry scale (|U| ~ 1e-2)
     rel = {"fp32": 0.02, "bf16": 0.1}[precision]
     assert err <= rel * np.max(np.abs(want)), f"relative error {err / np.max(np.abs(want)):.3e}"
+
+
+@pytest.mark.parametrize("name,steps,flags", [("resnet50", 12, 0), ("nanogpt", 4, "post")])
+def test_full_size_steps_are_deterministic(name, steps, flags):
+    """Two handles run the same sequence of full-size steps (fresh gradients
+    every step, the asynchronous mode the bench times): W and every worker's
+    momentum must come out bit-identical.  Nothing in a step depends on
+    scheduling -- the GEMM tiles, the power iteration's slot sums in a fixed
+    order, the vote's integer counts, and the one-bit signs OR-ed into words
+    for ResNet-50's ragged 147-column stem -- so any race would show here."""
+    wl = synth.WORKLOADS[name]
+    shapes, M = wl["shapes"], wl["M"]
+    f = smo.SIGNMUON_ASYNC | (smo.SIGNMUON_POST_POLAR if flags == "post" else 0)
+    outs = []
+    for _ in range(2):
+        opt = smo.SignMuon(shapes, M, beta=HP["beta"], lam=HP["lam"], K=wl["K"], eps=HP["eps"], scale=wl["scale"],
+                           P=wl["P"], flags=f)
+        W = synth.device_weights0(shapes, config_id=61)
+        for t in range(steps):
+            G = synth.device_gradients(shapes, M, wl["sigma"], step=t, config_id=61)
+            opt.step(W, [G[m] for m in range(M)], HP["eta"])
+            del G
+        opt.sync()
+        moms = []
+        for m in range(M):
+            x = torch.empty(opt.d, device="cuda")
+            opt.get_momentum(m, x)
+            moms.append(x)
+        outs.append((W, moms))
+        opt.close()
+    assert torch.equal(outs[0][0].view(torch.int32), outs[1][0].view(torch.int32))
+    for m in range(M):
+        assert torch.equal(outs[0][1][m].view(torch.int32), outs[1][1][m].view(torch.int32))
