@@ -931,6 +931,162 @@ k_vote_stream(WorkerPtrs signs, int M, int64_t ntiles,
   }
 }
 
+// Vote staging for M <= 15 (the post-vote input without D, as k_vote_stream
+// MODE 3 computes it): bit-sliced counters.  Lane t of a warp takes entries
+// 128 t .. 128 t + 127 of its chunk, four 32-bit words of every worker's
+// stream, loaded as in k_vote_stream (8 workers per batch, double-buffered).
+// Each word keeps four bit planes of the count c of set bits, one ripple add
+// per worker (7 logic operations for 32 entries); the majority sgn(2c - M)
+// is +1 where c >= TP and -1 where c < TN (bit masks P and N, from a borrow
+// chain against each constant), 0 on a tie; and a 16-entry table in shared
+// memory turns each pair of entries' four mask bits into their two bf16
+// values (+1 = 0x3F80, -1 = 0xBF80, 0), which go out through shared memory so
+// that every store writes whole 128-byte rows of the chunk's X.
+constexpr int kVoteSlicedMaxM = 15;
+
+// c >= T for the count in bit planes c[0..3] (c <= 15): no borrow out of c - T
+__device__ __forceinline__ uint32_t planes_ge(const uint32_t (&c)[4], int T) {
+  if (T <= 0) return 0xFFFFFFFFu;
+  if (T > 15) return 0u;
+  uint32_t b = 0u;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) b = ((T >> j) & 1) ? (~c[j] | b) : (~c[j] & b);
+  return ~b;
+}
+
+__global__ void __launch_bounds__(kVoteWarps * 32, 6)
+k_vote_stage_sliced(WorkerPtrs signs, int M, int64_t nchunks, int tie_plus, VoteStage st) {
+  griddep_wait();
+  griddep_launch();
+  __shared__ uint32_t lut[16];
+  extern __shared__ __align__(16) uint8_t vsm[];   // [warp][2][kVoteBatch][512]
+  if (threadIdx.x < 16) {
+    // index bits 0, 1: entries 2k, 2k + 1 are +1; bits 2, 3: they are -1
+    const uint32_t i = threadIdx.x;
+    const uint32_t lo = (i & 1u) ? 0x3F80u : ((i & 4u) ? 0xBF80u : 0u);
+    const uint32_t hi = (i & 2u) ? 0x3F80u : ((i & 8u) ? 0xBF80u : 0u);
+    lut[i] = lo | (hi << 16);
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int64_t gw = (int64_t)blockIdx.x * kVoteWarps + wid;
+  const int64_t nw = (int64_t)gridDim.x * kVoteWarps;
+  const uint32_t buf0 = (uint32_t)__cvta_generic_to_shared(vsm) + (uint32_t)wid * (2 * kVoteBatch * kVoteTileB);
+  const int nbatch = (M + kVoteBatch - 1) / kVoteBatch;
+  const int TP = tie_plus ? (M + 1) / 2 : M / 2 + 1;   // c >= TP: the majority is +1
+  const int TN = (M + 1) / 2;                           // c < TN: it is -1
+  auto issue = [&](int64_t t, int bt, int buf) {
+    const uint32_t dst = buf0 + (uint32_t)buf * (kVoteBatch * kVoteTileB) + (uint32_t)lane * 16;
+    const int64_t boff = st.off[t].x >> 3;
+    // a lane's 16 bytes hold entries 128 lane .. 128 lane + 127 of the chunk;
+    // pieces wholly past a short chunk's end are not read
+    const bool live = lane * 128 < st.chunks[t].len;
+#pragma unroll
+    for (int i = 0; i < kVoteBatch; ++i) {
+      const int m = bt * kVoteBatch + i;
+      if (m < M && live)
+        cp_async16(dst + (uint32_t)i * kVoteTileB, reinterpret_cast<const uint8_t*>(signs.p[m]) + boff + lane * 16);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  int64_t tile = gw;
+  int batch = 0;
+  if (tile >= nchunks) return;
+  issue(tile, 0, 0);
+  int cur = 0;
+  uint32_t c[4][4];   // [word][plane]
+#pragma unroll
+  for (int w = 0; w < 4; ++w)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) c[w][j] = 0u;
+  while (true) {
+    int64_t ntile = tile;
+    int nbt = batch + 1;
+    if (nbt == nbatch) { nbt = 0; ntile += nw; }
+    if (ntile < nchunks) {
+      issue(ntile, nbt, cur ^ 1);
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+    } else {
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+    }
+    __syncwarp();
+    const uint32_t src = buf0 + (uint32_t)cur * (kVoteBatch * kVoteTileB);
+    const int nm = min(kVoteBatch, M - batch * kVoteBatch);
+    for (int i = 0; i < nm; ++i) {
+      uint32_t v[4];
+      asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                   : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3])
+                   : "r"(src + (uint32_t)i * kVoteTileB + (uint32_t)lane * 16));
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        // count += bit, in bit planes (counts stay below 16)
+        const uint32_t t0 = c[w][0] & v[w];
+        c[w][0] ^= v[w];
+        const uint32_t t1 = c[w][1] & t0;
+        c[w][1] ^= t0;
+        const uint32_t t2 = c[w][2] & t1;
+        c[w][2] ^= t1;
+        c[w][3] ^= t2;
+      }
+    }
+    __syncwarp();
+    if (batch == nbatch - 1) {
+      const longlong2 o = st.off[tile];
+      const int len = st.chunks[tile].len;
+      __nv_bfloat16* xo = st.X + o.y;
+      uint32_t P[4], N[4];
+      int nz = 0;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const int e0 = lane * 128 + w * 32;
+        const uint32_t valid = e0 >= len ? 0u : (e0 + 32 <= len ? 0xFFFFFFFFu : ((1u << (len - e0)) - 1u));
+        P[w] = planes_ge(c[w], TP) & valid;
+        N[w] = ~planes_ge(c[w], TN) & valid;
+        nz += __popc(P[w] | N[w]);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) c[w][j] = 0u;
+      }
+      nz = __reduce_add_sync(0xffffffffu, nz);
+      if (lane == 0) st.partials[tile] = (float)nz;
+      // The bf16 values through the batch buffer just counted (32 rows of
+      // 128 bytes, 16-byte units XOR-swizzled by row), in two halves of 64
+      // entries per lane: lane t writes row t, then each store instruction
+      // sends four whole rows (128 contiguous bytes each) to the chunk's X.
+#pragma unroll
+      for (int hlf = 0; hlf < 2; ++hlf) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {   // 8 entries = 16 bytes each
+          const uint32_t p8 = (P[2 * hlf + u / 4] >> (8 * (u & 3))) & 0xFFu;
+          const uint32_t n8 = (N[2 * hlf + u / 4] >> (8 * (u & 3))) & 0xFFu;
+          uint32_t q[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) q[k] = lut[((p8 >> (2 * k)) & 3u) | (((n8 >> (2 * k)) & 3u) << 2)];
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(src + (uint32_t)(lane * 128 + ((u ^ (lane & 7)) * 16))),
+                       "r"(q[0]), "r"(q[1]), "r"(q[2]), "r"(q[3])
+                       : "memory");
+        }
+        __syncwarp();
+#pragma unroll
+        for (int jr = 0; jr < 8; ++jr) {
+          const int row = 4 * jr + lane / 8, u = lane & 7;
+          const int e = row * 128 + 64 * hlf + 8 * u;   // the unit's first entry in the chunk
+          uint4 q;
+          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(q.x), "=r"(q.y), "=r"(q.z), "=r"(q.w)
+                       : "r"(src + (uint32_t)(row * 128 + ((u ^ (row & 7)) * 16)))
+                       : "memory");
+          if (e < len) *reinterpret_cast<uint4*>(xo + e) = q;   // len is a multiple of 8
+        }
+        __syncwarp();
+      }
+    }
+    tile = ntile;
+    batch = nbt;
+    cur ^= 1;
+    if (tile >= nchunks) break;
+  }
+}
+
 // Majority of the packed signs staged straight into the Newton-Schulz input of
 // the post-vote polar step ([paper] §4, orthogonalising the aggregated
 // direction): per 4096-entry chunk of one matrix, the majority sgn(2c - M) of
@@ -1330,7 +1486,11 @@ void launch_vote_stage(cudaStream_t s, const WorkerPtrs& signs, int M, void* X, 
     const VoteStage st{reinterpret_cast<__nv_bfloat16*>(X), chunks, reinterpret_cast<const longlong2*>(stage_off),
                        partials};
     const int64_t warps = ((int64_t)n_chunks + kVoteWarps - 1) / kVoteWarps;
-    if (D == nullptr) {
+    if (D == nullptr && M <= kVoteSlicedMaxM) {
+      const int blocks = stream_grid((const void*)k_vote_stage_sliced, kVoteWarps * 32, smem, warps, 8);
+      launch_pdl(k_vote_stage_sliced, dim3(blocks), dim3(kVoteWarps * 32), smem, s, signs, M, (int64_t)n_chunks,
+                 tie_plus, st);
+    } else if (D == nullptr) {
       const int blocks = stream_grid((const void*)k_vote_stream<3, false>, kVoteWarps * 32, smem, warps, 8);
       launch_pdl(k_vote_stream<3, false>, dim3(blocks), dim3(kVoteWarps * 32), smem, s, signs, M, (int64_t)n_chunks,
                  nullptr, nullptr, nullptr, 0.f, nullptr, nullptr, tie_plus, st);
