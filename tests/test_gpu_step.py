@@ -134,13 +134,14 @@ def test_step_ragged_post_polar(precision, scale, P):
     _compare_step(shapes, M, gpu, want, precision, True)
 
 
-@pytest.mark.parametrize("M", [3, 4, 9])
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 9, 15, 16])
 def test_step_post_polar_streamed_stage(M):
     """Shapes whose matrices start at multiples of 128 entries and have a
     multiple of 8 columns: the majority is staged into the post-vote input by
-    the streaming vote kernel, one warp per chunk.  Ragged chunks (512 and 64
-    entries, the last below one lane's 128), odd and even M, and a second
-    batch of workers (M = 9)."""
+    the streaming vote kernels, one warp per chunk -- bit-sliced counters up
+    to 15 workers (M = 15 the largest), byte counters from 16.  Ragged chunks
+    (512 and 64 entries, the last below one lane's 128), odd and even M, and
+    a second batch of workers (M >= 9)."""
     shapes = [(136, 64), (64, 200), (128, 128), (96, 136), (8, 8)]
     h, gpu, want = _run_one_step(shapes, M, 1.0, 5, "spectral", 2, "bf16", True, seed=37)
     _compare_step(shapes, M, gpu, want, "bf16", True)
@@ -158,6 +159,16 @@ def test_step_one_and_two_workers(M, post_polar):
     shapes = [(130, 70), (64, 147), (96, 300), (8, 8)]
     h, gpu, want = _run_one_step(shapes, M, 1.0, 5, "spectral", 2, "fp32", post_polar, seed=61 + M)
     _compare_step(shapes, M, gpu, want, "fp32", post_polar)
+
+
+@pytest.mark.parametrize("M", [4, 7])
+def test_step_post_polar_streamed_stage_tie_plus(M):
+    """The bit-sliced staging with ties to +1 (its threshold moves from
+    floor(M/2) + 1 to ceil(M/2)): even M, where ties occur, and odd M."""
+    shapes = [(136, 64), (64, 200), (128, 128), (8, 8)]
+    h, gpu, want = _run_one_step(shapes, M, 1.0, 5, "spectral", 2, "bf16", True, seed=43,
+                                 extra_flags=smo.SIGNMUON_TIE_PLUS, tie=1)
+    _compare_step(shapes, M, gpu, want, "bf16", True, tie=1)
 
 
 def test_step_quintic_fp32():
